@@ -1,0 +1,389 @@
+"""Throughput of the LatentMoE layer forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole layer forward (router, top-K, down-projection,
+permutation, expert GEMMs, combine, up-projection and shared experts) over
+one batch of T synthetic tokens, through the library's C ABI.
+
+* value:   tokens/s of all ranks with inputs already resident in HBM, timed
+           with CUDA events over exactly K steps (max over ranks).
+* e2e:     the same metric with the input copied from pinned host memory and
+           the output copied back to pinned host memory inside every step.
+* roofline: the grouped expert GEMM launches (the dominant kernel), timed
+           with CUDA events recorded by the library at its stage boundaries
+           on the launch stream, against the measured B200 peak.
+* cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload
+           (rank 0, N = 1 only).
+
+--impl reference times the oracle itself (the reference arm of this path) on
+the host cores, on bounded samples of the same workload.
+
+With N > 1 (torchrun) every rank runs an independent replica on its own batch
+(no data-path collective; weak scaling); the process group only carries the
+barrier and the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import lmoe_inputs as LI  # noqa: E402
+
+METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % of HBM (decode) or tensor (prefill) peak"
+DEFAULT_WORKLOAD = "std_moe_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+REASON_FIELDS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,"
+             + ",".join(f"clocks_event_reasons.{r}" for r in REASON_FIELDS))
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "20",
+                 "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4 + len(REASON_FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, v in zip(REASON_FIELDS, parts[4:]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# algorithmic work of the dominant kernel (the two grouped expert GEMMs)
+# --------------------------------------------------------------------------
+def expert_gemm_work(wl, counts: np.ndarray):
+    """Algorithmic bytes and flops of expert GEMM 1 + GEMM 2 for one forward.
+
+    bytes = weights of every expert that received at least one row (W1_e and
+    W2_e once each) + the activation rows read and written (z rows in, a out,
+    a in, y out), in the storage format of the workload.
+    flops = 2 * (T*K) * l * m * 2.
+    """
+    rows = int(counts.sum())
+    used = int(np.count_nonzero(counts))
+    if wl.dtype == "nvfp4":
+        wbytes = used * 2 * wl.m * wl.l * (0.5 + 1.0 / 16)
+        abytes = rows * (wl.l + wl.m) * (0.5 + 1.0 / 16) + rows * (wl.m * (0.5 + 1.0 / 16) + wl.l * 2)
+    else:
+        eb = 4 if wl.dtype == "f32" else 2
+        wbytes = used * 2 * wl.m * wl.l * eb
+        abytes = rows * (wl.l + wl.m) * eb * 2
+    flops = 2.0 * rows * wl.l * wl.m * 2
+    return wbytes + abytes, flops, used
+
+
+def traffic_record(workload: str):
+    """DRAM traffic per expert-GEMM launch pair from a committed ncu capture,
+    valid only while the GEMM source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, "latentmoe_fwd_b200", "csrc", "gemm_tc.cuh")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    entry = rec.get(workload)
+    if not entry or entry.get("gemm_source_sha") != h:
+        return None
+    return entry.get("traffic_bytes_per_forward")
+
+
+# --------------------------------------------------------------------------
+# the CPU oracle, timed (bounded sample)
+# --------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def oracle_tokens_per_s(wl, inp, n_tokens: int, seed: int = 0):
+    from oracle import lmoe_oracle as O
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(wl.T, size=min(n_tokens, wl.T), replace=False))
+    t0 = time.perf_counter()
+    O.forward(wl, inp, tokens=toks)
+    dt = time.perf_counter() - t0
+    return len(toks) / dt, dt, len(toks)
+
+
+def run_reference(args, wl):
+    """Reference arm: the oracle on the host cores, K timed steps of a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = LI.make_inputs(wl)
+    per_step = max(1, 64 // max(1, args.steps))
+    for i in range(args.warmup):
+        oracle_tokens_per_s(wl, inp, per_step, seed=1000 + i)
+    total_t, total_tok = 0.0, 0
+    for i in range(args.steps):
+        _, dt, n = oracle_tokens_per_s(wl, inp, per_step, seed=i)
+        total_t += dt
+        total_tok += n
+    v = total_tok / total_t
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl),
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} random token(s) of the {wl.name} batch per step, "
+                                   f"fp64 NumPy oracle with full weights"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl):
+    c = {"workload": wl.name, "T": wl.T, "d": wl.d, "l": wl.l, "N": wl.N, "K": wl.K, "m": wl.m,
+         "n_shared": wl.n_shared, "m_shared": wl.m_shared, "identity_projections": wl.identity,
+         "zipf_bias": wl.zipf_bias, "outliers": wl.outliers, "parallelism": "replicas (one layer per GPU)"}
+    return c
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(LI.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample", type=int, default=None, help="oracle tokens for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = LI.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+
+    import latentmoe_fwd_b200 as L
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    t_gen = time.perf_counter()
+    inp = LI.make_inputs(wl)
+    log(f"[bench] inputs for {wl.name} generated in {time.perf_counter() - t_gen:.1f}s")
+    st = "f32" if wl.dtype == "f32" else "bf16"
+
+    def dev(a):
+        if a is None:
+            return None
+        if st == "f32":
+            return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    t = {k: dev(inp[k]) for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
+    bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).cuda()
+    tdtype = torch.float32 if st == "f32" else torch.bfloat16
+    x_host = torch.from_numpy(np.ascontiguousarray(inp["x"]).view(np.int16 if st != "f32" else np.float32))
+    x_host = (x_host.view(torch.bfloat16) if st != "f32" else x_host).pin_memory()
+    x = x_host.cuda()
+    out = torch.empty((wl.T, wl.d), dtype=tdtype, device="cuda")
+    out_host = torch.empty((wl.T, wl.d), dtype=tdtype).pin_memory()
+    cfg = L.config(T=wl.T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m, n_shared=wl.n_shared, m_shared=wl.m_shared,
+                   act=L.F32 if st == "f32" else L.BF16,
+                   expert={"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype], identity=wl.identity)
+    w = L.weights(w_router=t["w_router"], router_bias=bias, w_down=t["w_down"], w_up=t["w_up"], w1=t["w1"],
+                  w2=t["w2"], ws1=t["ws1"], ws2=t["ws2"])
+    ws = L.workspace(cfg, L.OP_FORWARD)
+    stream = torch.cuda.current_stream()
+
+    # routing statistics of this batch (outside any timed region)
+    idx = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    gw = torch.empty((wl.T, wl.K), dtype=torch.float32, device="cuda")
+    rws = L.workspace(cfg, L.OP_ROUTE)
+    L.route(cfg, x, t["w_router"], bias, None, idx, gw, None, rws)
+    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=wl.N)
+    alg_bytes, alg_flops, used = expert_gemm_work(wl, counts)
+
+    for _ in range(args.warmup):
+        L.forward(cfg, w, x, out, ws)
+    stv, info = L.read_device_error(ws)
+    if stv != L.OK:
+        raise RuntimeError(f"device error during warm-up: {L.status_string(stv)} info={info:#x}")
+
+    # ---- device-resident timed region ----
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(L.TRACE_EVENTS)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    time.sleep(0.05)
+    launches0 = L.kernel_launch_count()
+    start.record(stream)
+    for i in range(K):
+        L.forward_traced(cfg, w, x, out, ws, ev[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = L.kernel_launch_count() - launches0
+    clocks = sampler.stop()
+    barrier()
+    stv, info = L.read_device_error(ws)
+    if stv != L.OK:
+        raise RuntimeError(f"device error in the timed region: {L.status_string(stv)} info={info:#x}")
+    ms = start.elapsed_time(end)
+    stage_ms = np.zeros(L.TRACE_EVENTS - 1)
+    for i in range(K):
+        for j in range(L.TRACE_EVENTS - 1):
+            stage_ms[j] += ev[i][j].elapsed_time(ev[i][j + 1])
+    stage_ms /= K
+
+    # ---- end-to-end through host buffers ----
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(K):
+        x.copy_(x_host, non_blocking=True)
+        L.forward(cfg, w, x, out, ws)
+        out_host.copy_(out, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+
+    tokens = wl.T * K * world
+    value = tokens / (ms / 1000.0)
+    e2e_value = tokens / (e2e_ms / 1000.0)
+
+    peaks, peak_src = load_peaks()
+    gemm_ms = stage_ms[3] + stage_ms[4]          # expert GEMM 1 + 2 (two launches)
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    if wl.dtype == "nvfp4":
+        tensor_peak = tensor_peak * 4.0          # nominal FP4 : BF16 dense ratio (9 : 2.25)
+    t_tc = alg_flops / (tensor_peak * 1e12)
+    if wl.dtype == "f32":
+        roof = {"bound": "launch", "achieved": None, "peak": None, "unit": None, "frac": None, "traffic": None}
+    elif t_hbm >= t_tc:
+        ach = alg_bytes / (gemm_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    else:
+        ach = alg_flops / (gemm_ms / 1000.0) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": ach / tensor_peak}
+    if "traffic" not in roof:
+        tr = traffic_record(wl.name)
+        roof["traffic"] = tr
+    roof.update({
+        "kernel": "tc_gemm_kernel (grouped expert GEMM 1 + GEMM 2, 2 launches per step)",
+        "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops, "experts_used": used,
+        "kernel_ms_per_step": gemm_ms, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
+        else "fallback", "peak_kind": "hbm_gbs" if roof.get("bound") == "hbm" else "bf16_tflops_sustained"})
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = args.cpu_sample or {"tiny_f32": 64, "std_moe_bf16": 128, "ultra_decode": 32, "ultra_zipf": 32,
+                                "ultra_nvfp4": 16}.get(wl.name, 32)
+        v, dt, ntok = oracle_tokens_per_s(wl, inp, n)
+        cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{ntok} random tokens of the {wl.name} batch, full weights, fp64 NumPy "
+                         f"({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp32" if wl.dtype == "f32" else ("nvfp4+bf16" if wl.dtype == "nvfp4"
+                                                                             else "bf16"),
+            "data": "synthetic", "config": {**workload_config(wl),
+                                            "l2": "no flush: weights alone exceed the 126 MB L2"
+                                            if wl.dtype != "f32" else "tiny (fits L2)"},
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() *
+                                                                                     x_host.element_size()),
+                    "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+            "stage_ms": {n: float(v) for n, v in zip(L.TRACE_STAGES, stage_ms)},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

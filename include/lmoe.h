@@ -1,0 +1,245 @@
+/*
+ * lmoe.h -- C ABI of a B200 (sm_100a) LatentMoE layer forward.
+ *
+ * The layer (Nemotron 3 whitepaper, as summarised on the greeksharifa page,
+ * section 2.2 "LatentMoE"; notes.yuuk.io page, section 2 "LatentMoE"):
+ *
+ *   logits = x W_r^T (+ b)                      router on the d-dim hidden state
+ *   (idx, g) = top-K(logits), softmax renormalised over the K chosen
+ *   z = x W_dn^T                                 d -> l latent down-projection
+ *   a = relu(z W1_e^T)^2, y = g * (a W2_e^T)     routed experts in l, per expert e
+ *   c_t = sum_k y(t, k)                          gate-weighted combine
+ *   out = c W_up^T + sum_s Ws2_s relu(Ws1_s x)^2 l -> d up-projection + shared experts
+ *
+ * NVFP4 (same page, section 2.4 "NVFP4 Training"): E2M1 elements, 16-element
+ * micro-blocks with an E4M3 scale, and an FP32 per-tensor global scale.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named x, w*, out, ... are DEVICE pointers unless the comment says
+ *    host. The caller owns and allocates every buffer; the library never
+ *    allocates or frees memory. Scratch memory is the caller's workspace,
+ *    sized by lmoe_workspace_size().
+ *  - Matrices are row-major. Weights use the [out][in] layout, so every
+ *    contraction is "row-major activations x K-major weights".
+ *  - BF16 tensors are 2-byte bfloat16; F32 tensors are 4-byte IEEE floats.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). No call synchronises the host except
+ *    lmoe_read_device_error().
+ *  - Errors a host can see (NULL pointer, unsupported shape, misalignment,
+ *    workspace too small) are returned before anything is launched. Errors
+ *    found on the device (a pipeline wait that timed out, an index out of
+ *    range) are written to an error word in the first 8 bytes of the
+ *    workspace and read with lmoe_read_device_error(). A new workspace must
+ *    have its first 256 bytes zeroed once before its first use; the library
+ *    only ever writes the word on an error, and reading it clears it.
+ *    Kernels never trap.
+ *  - Inputs are assumed finite. Results are deterministic run to run (no
+ *    floating-point atomics).
+ *  - Device pointers must be 16-byte aligned; row pitches must be multiples
+ *    of 16 bytes (for BF16: dimensions that are multiples of 8).
+ */
+#ifndef LMOE_H_
+#define LMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LMOE_OK = 0,
+  LMOE_ERR_INVALID_ARG = 1,    /* NULL pointer, bad size, K > N, misalignment */
+  LMOE_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. a dtype mix) */
+  LMOE_ERR_WORKSPACE = 3,      /* workspace NULL or smaller than required */
+  LMOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+  LMOE_ERR_DEVICE_TIMEOUT = 5, /* a device pipeline wait exceeded its limit */
+  LMOE_ERR_DEVICE_BOUNDS = 6   /* a device index check failed */
+} lmoe_status;
+
+typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1, LMOE_NVFP4 = 2 } lmoe_dtype;
+
+/* Scale-factor layouts of an NVFP4 tensor [rows][cols]:
+ * ROWMAJOR: byte (r, j) at r * (cols/16) + j, j = block index along the row.
+ * MMA_TILED: the layout the block-scaled tensor-core MMA reads. Rows are
+ *   grouped in blocks of 128 and columns in groups of 64 (4 scales); each
+ *   (row block rb, column group cg) is a 512-byte atom at
+ *   (rb * ceil(cols/64) + cg) * 512, and inside it scale (r, j) sits at
+ *   (r % 32) * 16 + ((r % 128) / 32) * 4 + (j % 4). rows are padded to a
+ *   multiple of 128 and cols to a multiple of 64 (padding bytes are written 0). */
+typedef enum { LMOE_SF_ROWMAJOR = 0, LMOE_SF_MMA_TILED = 1 } lmoe_sf_layout;
+
+/* Flag: l == d and there is no down/up projection (the standard-MoE limit). */
+#define LMOE_FLAG_IDENTITY_PROJ 1u
+
+typedef struct {
+  int64_t T;        /* tokens */
+  int32_t d;        /* hidden size */
+  int32_t l;        /* latent size (== d with LMOE_FLAG_IDENTITY_PROJ) */
+  int32_t N;        /* routed experts */
+  int32_t K;        /* experts per token, 1 <= K <= N */
+  int32_t m;        /* routed expert hidden size */
+  int32_t n_shared; /* always-on shared experts (0 = none) */
+  int32_t m_shared; /* shared expert hidden size */
+  int32_t act;      /* lmoe_dtype of x, router, projections and the stored
+                       intermediates z, a, y, c, out: LMOE_F32 or LMOE_BF16 */
+  int32_t expert;   /* lmoe_dtype of the routed expert weights and the latent
+                       activations fed to them: LMOE_F32 (with act F32),
+                       LMOE_BF16 or LMOE_NVFP4 (with act BF16) */
+  uint32_t flags;   /* LMOE_FLAG_* */
+} lmoe_config;
+
+/* Layer weights (device pointers, `act` dtype unless stated).
+ *  w_router [N][d]; router_bias [N] F32 or NULL;
+ *  w_down [l][d], w_up [d][l] (NULL with LMOE_FLAG_IDENTITY_PROJ);
+ *  w1 [N][m][l], w2 [N][l][m]: routed experts. For expert == LMOE_NVFP4 these
+ *    are packed E2M1 codes ([N][m][l/2], [N][l][m/2] bytes; element 2j in the
+ *    low nibble), w1_sf / w2_sf their E4M3 block scales in LMOE_SF_MMA_TILED
+ *    layout per expert matrix (as written by lmoe_nvfp4_quantize), and
+ *    w1_gs / w2_gs [N] F32 the per-matrix global scales;
+ *  a_global_scale: NVFP4 only, device pointer to one F32: the static scale of
+ *    the expert hidden activation a, as a checkpoint carries it;
+ *  ws1 [S][m_s][d], ws2 [S][d][m_s]: shared experts (NULL when n_shared == 0). */
+typedef struct {
+  const void* w_router;
+  const float* router_bias;
+  const void* w_down;
+  const void* w_up;
+  const void* w1;
+  const void* w2;
+  const uint8_t* w1_sf;
+  const uint8_t* w2_sf;
+  const float* w1_gs;
+  const float* w2_gs;
+  const float* a_global_scale;
+  const void* ws1;
+  const void* ws2;
+} lmoe_weights;
+
+/* Workspace size queries, one per entry point. */
+typedef enum {
+  LMOE_OP_ROUTE = 0,
+  LMOE_OP_PERMUTE = 1,
+  LMOE_OP_EXPERT_FFN = 2,
+  LMOE_OP_COMBINE = 3,
+  LMOE_OP_FORWARD = 4,
+  LMOE_OP_NVFP4_QUANTIZE = 5
+} lmoe_op;
+
+/* Bytes of workspace `op` needs for `cfg` (for LMOE_OP_NVFP4_QUANTIZE the
+ * tensor is taken as [cfg->T][cfg->l]). Returns 0 for an invalid config. */
+size_t lmoe_workspace_size(const lmoe_config* cfg, int op);
+
+/* Rows of the expert-grouped (padded) buffers: each expert's rows start at a
+ * multiple of 128, so the buffers hold at most T*K + N*127 rows, rounded up
+ * to a multiple of 128. */
+int64_t lmoe_padded_rows(const lmoe_config* cfg);
+
+/* Router: logits = x W_r^T + b, then per token the K experts with the largest
+ * logits (ties to the lower index), in that order, and their gates
+ * g_k = exp(l_k - l_max) / sum_j exp(l_j - l_max) over the chosen K (the
+ * softmax over all N restricted to the K and renormalised).
+ *  x [T][d] (act), w_router [N][d] (act), bias [N] F32 or NULL.
+ *  logits_in: NULL to compute the logits; else [T][N] F32 logits to route
+ *    (x, w_router, bias are then ignored and may be NULL).
+ *  topk_idx [T][K] int32, topk_w [T][K] F32: outputs.
+ *  logits_out [T][N] F32 or NULL: the computed logits (bias included). */
+lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_router,
+                       const float* bias, const float* logits_in, int32_t* topk_idx,
+                       float* topk_w, float* logits_out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Dispatch grouped by expert: a stable counting sort of the slots
+ * f = t*K + k by expert (expert ascending, then f ascending).
+ *  topk_idx [T][K] int32 (each in [0, N); out-of-range -> device bounds error).
+ *  offsets [N+1] int32: expert e owns sorted positions [offsets[e], offsets[e+1]).
+ *  perm_src [T*K] int32: sorted position r holds slot perm_src[r].
+ *  inv_perm [T*K] int32: slot f sits at sorted position inv_perm[f].
+ *  padded_offsets [N+1] int32: expert e's rows in the padded buffers start at
+ *    padded_offsets[e] (a multiple of 128); sorted position r of expert e is
+ *    padded row r - offsets[e] + padded_offsets[e].
+ *  rows / row_bytes / permuted_rows (all optional, NULL/0 to skip): gather the
+ *    token rows rows[t] (row_bytes each, a multiple of 16) to padded rows.
+ *  rows_sf / permuted_sf (optional): NVFP4 row-major scales [T][row_cols/16]
+ *    of `rows`, re-laid to LMOE_SF_MMA_TILED at the padded rows; row_cols is
+ *    2*row_bytes (the rows then hold packed E2M1 codes).
+ *  topk_w / perm_gate (optional): the gate of each padded row ([padded] F32). */
+lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets,
+                         int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
+                         const void* rows, int64_t row_bytes, void* permuted_rows,
+                         const uint8_t* rows_sf, uint8_t* permuted_sf, const float* topk_w,
+                         float* perm_gate, void* ws, size_t ws_bytes, void* stream);
+
+/* Routed expert FFNs on the padded expert-grouped rows:
+ *  y = g * (relu(z_e W1_e^T)^2 W2_e^T) for the rows of each expert e.
+ *  permuted_in [padded][l]: `act` rows, or for expert == NVFP4 packed E2M1
+ *    codes [padded][l/2] with permuted_sf (MMA_TILED) and in_global_scale
+ *    (device pointer to one F32).
+ *  offsets, padded_offsets [N+1]: from lmoe_permute.
+ *  perm_gate [padded] F32 or NULL (gates of 1).
+ *  y_perm [padded][l] (act): output; padding rows are left unspecified. */
+lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w,
+                            const void* permuted_in, const uint8_t* permuted_sf,
+                            const float* in_global_scale, const int32_t* offsets,
+                            const int32_t* padded_offsets, const float* perm_gate,
+                            void* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Combine: c_t = sum_{k=0..K-1} w[t][k] * y_perm[row(t*K+k)], summed in fp32
+ * in k order, stored as `act`; row(f) = inv_perm[f] - offsets[e] +
+ * padded_offsets[e] with e = topk_idx[f]. topk_w NULL means the gates were
+ * already applied (w = 1). c [T][l]. No workspace. */
+lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32_t* topk_idx,
+                         const int32_t* inv_perm, const int32_t* offsets,
+                         const int32_t* padded_offsets, const float* topk_w, void* c,
+                         void* stream);
+
+/* The whole layer: route, down-project (NVFP4: quantise z with its current
+ * amax), permute, expert FFNs, combine, up-project and add the shared
+ * experts. x [T][d] (act) -> out [T][d] (act). */
+lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x,
+                         void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* lmoe_forward with stage tracing: when `events` is not NULL it holds
+ * LMOE_TRACE_EVENTS cudaEvent_t handles (created by the caller) that are
+ * recorded on `stream` at the stage boundaries, in order:
+ *   0 start, 1 after routing, 2 after the down-projection (and NVFP4
+ *   quantisation of z), 3 after the permutation and gather, 4 after expert
+ *   GEMM 1, 5 after expert GEMM 2, 6 after the combine, 7 after the shared
+ *   experts and up-projection (end).
+ * Stages that do not run for a configuration record their event at the same
+ * point as the previous one. Costs one event record per stage. */
+#define LMOE_TRACE_EVENTS 8
+lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, const void* x,
+                                void* out, void* ws, size_t ws_bytes, void* stream,
+                                void* const* events);
+
+/* NVFP4 two-level quantisation of in [rows][cols] (F32 or BF16, cols a
+ * multiple of 16) along its rows:
+ *  s_g = global_in ? *global_in : fp32(amax / 2688) (1 when amax == 0);
+ *  per 16-block: s_b = E4M3_satfinite_rn(amax_b / (s_g * 6));
+ *  q_i = E2M1_satfinite_rn(x_i / (dec(s_b) * s_g)) (all codes +0 if dec(s_b) == 0).
+ *  codes [rows][cols/2] (low nibble first), sf per sf_layout, global_out
+ *  (device F32, may be NULL) receives s_g. global_in: device pointer or NULL. */
+lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
+                                const float* global_in, uint8_t* codes, uint8_t* sf,
+                                float* global_out, int sf_layout, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* Synchronises `stream`, returns the device error status recorded in the
+ * workspace `ws` (LMOE_OK if none) and clears it. `info` (host, may be NULL)
+ * receives a kernel-specific detail word. */
+lmoe_status lmoe_read_device_error(void* ws, void* stream, uint32_t* info);
+
+/* Static description of a status code. */
+const char* lmoe_status_string(lmoe_status s);
+
+/* Number of kernels launched by this library since load (host counter; used
+ * by harnesses to report how many of the library's kernels a region ran). */
+uint64_t lmoe_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMOE_H_ */

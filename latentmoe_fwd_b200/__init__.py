@@ -1,0 +1,199 @@
+"""Python binding of liblmoe.so, the B200 LatentMoE layer-forward library.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. PyTorch provides device memory and streams. Importing this package
+loads the shared library and fails loudly if it has not been built
+(``python latentmoe_fwd_b200/build.py``).
+
+Entry points mirror include/lmoe.h: ``route``, ``permute``, ``expert_ffn``,
+``combine``, ``forward``, ``nvfp4_quantize``, plus ``workspace_size``,
+``padded_rows``, ``read_device_error`` and ``kernel_launch_count``.
+Tensor arguments are torch tensors (or None); their ``data_ptr()`` is passed.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblmoe.so")
+
+# status codes
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_DEVICE_BOUNDS = range(7)
+F32, BF16, NVFP4 = 0, 1, 2
+SF_ROWMAJOR, SF_MMA_TILED = 0, 1
+FLAG_IDENTITY_PROJ = 1
+OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE = range(6)
+
+EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permute",
+           "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
+           "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
+           "lmoe_forward_traced")
+TRACE_EVENTS = 8
+TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("l", ctypes.c_int32),
+                ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("m", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32), ("m_shared", ctypes.c_int32),
+                ("act", ctypes.c_int32), ("expert", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "w_router", "router_bias", "w_down", "w_up", "w1", "w2", "w1_sf", "w2_sf",
+        "w1_gs", "w2_gs", "a_global_scale", "ws1", "ws2")]
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python latentmoe_fwd_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    C = ctypes.POINTER(Config)
+    W = ctypes.POINTER(Weights)
+    sig = {
+        "lmoe_workspace_size": (ctypes.c_size_t, [C, ctypes.c_int]),
+        "lmoe_padded_rows": (I64, [C]),
+        "lmoe_route": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "lmoe_permute": (ctypes.c_int, [C, P, P, P, P, P, P, I64, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "lmoe_expert_ffn": (ctypes.c_int, [C, W, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "lmoe_combine": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
+        "lmoe_forward": (ctypes.c_int, [C, W, P, P, P, ctypes.c_size_t, P]),
+        "lmoe_forward_traced": (ctypes.c_int, [C, W, P, P, P, ctypes.c_size_t, P, ctypes.POINTER(P)]),
+        "lmoe_nvfp4_quantize": (ctypes.c_int, [P, ctypes.c_int, I64, I64, P, P, P, P, ctypes.c_int, P,
+                                               ctypes.c_size_t, P]),
+        "lmoe_read_device_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
+        "lmoe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "lmoe_kernel_launch_count": (ctypes.c_uint64, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(s: int) -> str:
+    return lib.lmoe_status_string(int(s)).decode()
+
+
+def _p(t):
+    """Device (or host) pointer of a tensor, or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != OK:
+        raise LmoeError(st, where)
+
+
+def config(T, d, l, N, K, m, n_shared=0, m_shared=0, act=BF16, expert=BF16, identity=False) -> Config:
+    return Config(T=T, d=d, l=l, N=N, K=K, m=m, n_shared=n_shared, m_shared=m_shared, act=act,
+                  expert=expert, flags=FLAG_IDENTITY_PROJ if identity else 0)
+
+
+def weights(**tensors) -> Weights:
+    w = Weights()
+    for k, v in tensors.items():
+        setattr(w, k, _p(v))
+    w._keep = tensors   # keep the tensors alive as long as the struct
+    return w
+
+
+def workspace_size(cfg: Config, op: int) -> int:
+    return int(lib.lmoe_workspace_size(ctypes.byref(cfg), op))
+
+
+def padded_rows(cfg: Config) -> int:
+    return int(lib.lmoe_padded_rows(ctypes.byref(cfg)))
+
+
+def kernel_launch_count() -> int:
+    return int(lib.lmoe_kernel_launch_count())
+
+
+def workspace(cfg: Config, op: int, device="cuda"):
+    """A workspace tensor for `op`; its error word starts cleared."""
+    import torch
+    n = workspace_size(cfg, op)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def route(cfg, x, w_router, bias, logits_in, topk_idx, topk_w, logits_out, ws, stream=None):
+    _check(lib.lmoe_route(ctypes.byref(cfg), _p(x), _p(w_router), _p(bias), _p(logits_in), _p(topk_idx),
+                          _p(topk_w), _p(logits_out), _p(ws), ws.numel(), _stream(stream)), "lmoe_route")
+
+
+def permute(cfg, topk_idx, offsets, perm_src, inv_perm, padded_offsets, rows=None, row_bytes=0,
+            permuted_rows=None, rows_sf=None, permuted_sf=None, topk_w=None, perm_gate=None, ws=None,
+            stream=None):
+    _check(lib.lmoe_permute(ctypes.byref(cfg), _p(topk_idx), _p(offsets), _p(perm_src), _p(inv_perm),
+                            _p(padded_offsets), _p(rows), int(row_bytes), _p(permuted_rows), _p(rows_sf),
+                            _p(permuted_sf), _p(topk_w), _p(perm_gate), _p(ws), ws.numel(),
+                            _stream(stream)), "lmoe_permute")
+
+
+def expert_ffn(cfg, w: Weights, permuted_in, permuted_sf, in_global_scale, offsets, padded_offsets,
+               perm_gate, y_perm, ws, stream=None):
+    _check(lib.lmoe_expert_ffn(ctypes.byref(cfg), ctypes.byref(w), _p(permuted_in), _p(permuted_sf),
+                               _p(in_global_scale), _p(offsets), _p(padded_offsets), _p(perm_gate),
+                               _p(y_perm), _p(ws), ws.numel(), _stream(stream)), "lmoe_expert_ffn")
+
+
+def combine(cfg, y_perm, topk_idx, inv_perm, offsets, padded_offsets, topk_w, c, stream=None):
+    _check(lib.lmoe_combine(ctypes.byref(cfg), _p(y_perm), _p(topk_idx), _p(inv_perm), _p(offsets),
+                            _p(padded_offsets), _p(topk_w), _p(c), _stream(stream)), "lmoe_combine")
+
+
+def forward(cfg, w: Weights, x, out, ws, stream=None):
+    _check(lib.lmoe_forward(ctypes.byref(cfg), ctypes.byref(w), _p(x), _p(out), _p(ws), ws.numel(),
+                            _stream(stream)), "lmoe_forward")
+
+
+def forward_traced(cfg, w: Weights, x, out, ws, events, stream=None):
+    """lmoe_forward recording ``TRACE_EVENTS`` torch.cuda.Event objects (timing
+    enabled) at the stage boundaries on the launch stream."""
+    assert len(events) == TRACE_EVENTS
+    arr = (ctypes.c_void_p * TRACE_EVENTS)(*[e.cuda_event for e in events])
+    _check(lib.lmoe_forward_traced(ctypes.byref(cfg), ctypes.byref(w), _p(x), _p(out), _p(ws), ws.numel(),
+                                   _stream(stream), arr), "lmoe_forward_traced")
+
+
+def nvfp4_quantize(x, in_dtype, rows, cols, global_in, codes, sf, global_out, sf_layout, ws, stream=None):
+    _check(lib.lmoe_nvfp4_quantize(_p(x), int(in_dtype), int(rows), int(cols), _p(global_in), _p(codes),
+                                   _p(sf), _p(global_out), int(sf_layout), _p(ws), ws.numel(),
+                                   _stream(stream)), "lmoe_nvfp4_quantize")
+
+
+def read_device_error(ws, stream=None):
+    """Synchronise, return (status, info) of the workspace's error word and clear it."""
+    info = ctypes.c_uint32(0)
+    st = lib.lmoe_read_device_error(_p(ws), _stream(stream), ctypes.byref(info))
+    return int(st), int(info.value)

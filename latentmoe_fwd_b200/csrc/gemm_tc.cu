@@ -1,0 +1,124 @@
+// Host side of the tcgen05 GEMM: TMA tensor maps, tile-size and epilogue
+// dispatch, persistent-grid sizing.
+#include <mutex>
+
+#include "gemm_tc.cuh"
+#include "lmoe_internal.h"
+
+namespace lmoe {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a BF16 tensor [groups][rows][k] (k contiguous); box = 64 x box_rows x 1,
+// 128-byte swizzle, zero fill out of bounds.
+static bool make_map_bf16(CUtensorMap* map, const TcOperand& op, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || !op.ptr) return false;
+  if ((reinterpret_cast<uintptr_t>(op.ptr) & 15) != 0 || (op.k * 2) % 16 != 0) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(op.k), static_cast<cuuint64_t>(op.rows),
+                        static_cast<cuuint64_t>(op.groups)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(op.k * 2), static_cast<cuuint64_t>(op.rows * op.k * 2)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(op.ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int EPI>
+static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
+                             const CUtensorMap& b1, const TcParams& p, int grid, cudaStream_t s) {
+  using Sm = TcSmem<BN, STAGES>;
+  auto kern = tc_gemm_kernel<BN, STAGES, EPI>;
+  static int configured_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    configured_dev = dev;
+  }
+  kern<<<grid, 192, Sm::kBytes, s>>>(a0, b0, a1, b1, p);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+template <int BN, int STAGES>
+static lmoe_status dispatch_epi(int epi, const CUtensorMap& a0, const CUtensorMap& b0,
+                                const CUtensorMap& a1, const CUtensorMap& b1, const TcParams& p,
+                                int grid, cudaStream_t s) {
+  switch (epi) {
+    case EPI_F32_BIAS: return launch_tc<BN, STAGES, EPI_F32_BIAS>(a0, b0, a1, b1, p, grid, s);
+    case EPI_BF16: return launch_tc<BN, STAGES, EPI_BF16>(a0, b0, a1, b1, p, grid, s);
+    case EPI_SQRELU: return launch_tc<BN, STAGES, EPI_SQRELU>(a0, b0, a1, b1, p, grid, s);
+    case EPI_GATE: return launch_tc<BN, STAGES, EPI_GATE>(a0, b0, a1, b1, p, grid, s);
+    case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(a0, b0, a1, b1, p, grid, s);
+  }
+  return LMOE_ERR_INVALID_ARG;
+}
+
+lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) {
+  const int bn = L.bn;
+  if (bn != 32 && bn != 64 && bn != 128 && bn != 256) return LMOE_ERR_INVALID_ARG;
+  // A always has 128-row boxes (activation rows normal, weight rows swap); B has BN-row boxes.
+  CUtensorMap maps[4];
+  for (int sg = 0; sg < L.nseg; ++sg) {
+    if (!make_map_bf16(&maps[2 * sg], L.a[sg], 128)) return LMOE_ERR_INVALID_ARG;
+    if (!make_map_bf16(&maps[2 * sg + 1], L.b[sg], bn)) return LMOE_ERR_INVALID_ARG;
+  }
+  if (L.nseg == 1) {
+    maps[2] = maps[0];
+    maps[3] = maps[1];
+  }
+  TcParams p;
+  p.swap = L.swap;
+  p.grouped = L.grouped;
+  p.rows = L.rows;
+  p.cols = L.cols;
+  p.nseg = L.nseg;
+  for (int sg = 0; sg < 2; ++sg) {
+    p.seg[sg].kblocks = L.kblocks[sg];
+    p.seg[sg].a_kgroup = L.a_kgroup[sg];
+    p.seg[sg].b_kgroup = L.b_kgroup[sg];
+  }
+  p.offsets = L.offsets;
+  p.padded_offsets = L.padded_offsets;
+  p.groups = L.groups;
+  p.out = L.out;
+  p.ld_out = L.ld_out;
+  p.bias = L.bias;
+  p.row_scale = L.row_scale;
+  p.residual = static_cast<const __nv_bfloat16*>(L.residual);
+  p.ld_res = L.ld_res;
+  p.err = DevErr{err_word};
+  const int sms = device_sm_count();
+  int64_t grid = L.max_tiles < sms ? L.max_tiles : sms;
+  if (grid <= 0) return LMOE_OK;
+  const int g = static_cast<int>(grid);
+  switch (bn) {
+    case 256: return dispatch_epi<256, 4>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
+    case 128: return dispatch_epi<128, 6>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
+    case 64: return dispatch_epi<64, 8>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
+    case 32: return dispatch_epi<32, 10>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
+  }
+  return LMOE_ERR_INVALID_ARG;
+}
+
+}  // namespace lmoe

@@ -1,0 +1,383 @@
+// Persistent BF16 tensor-core GEMM for sm_100a (tcgen05 + TMEM + TMA).
+//
+//   D[rows, cols] = A[rows, K] . B[cols, K]^T   (both operands K-major)
+//
+// One CTA per SM loops over output tiles. Warp roles:
+//   warp 0      TMA producer: streams 64-wide K slices of A and B into a ring
+//               of shared-memory stages (128-byte swizzle).
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
+//               K=16 each) into one of two TMEM accumulators, and commits
+//               stage releases / accumulator-ready signals to mbarriers.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (one TMEM lane = one row
+//               per thread), apply the fused epilogue, store to global.
+// The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
+//
+// Tile kinds:
+//   normal: A = activation rows (128 per tile), B = weight rows (BN per tile).
+//   swap:   A = weight rows (128 per tile), B = activation rows (<= BN tokens);
+//           used when the token count is tiny and the GEMM streams weights.
+//   grouped: activation rows are the expert-grouped padded buffer (each
+//           expert's rows start at a multiple of 128); the weight operand is a
+//           3-D map [experts][rows][K] indexed by the tile's expert.
+// Up to two K segments are summed into one accumulator (used for
+// out = c W_up^T + sum_s as_s Ws2_s^T).
+#pragma once
+
+#include "lmoe_device.cuh"
+
+namespace lmoe {
+
+enum EpiKind : int {
+  EPI_F32_BIAS = 0,   // out f32 = acc (+ bias[col])
+  EPI_BF16 = 1,       // out bf16 = acc
+  EPI_SQRELU = 2,     // out bf16 = relu(acc)^2
+  EPI_GATE = 3,       // out bf16 = acc * row_scale[row]
+  EPI_ADD_RES = 4     // out bf16 = acc + residual[row][col]
+};
+
+struct TcSeg {
+  int kblocks;     // 64-wide K blocks in this segment
+  int a_kgroup;    // >0: the K axis of A is split into groups of a_kgroup along its 3rd dim
+  int b_kgroup;    // same for B
+};
+
+struct TcParams {
+  int swap;        // 0 normal, 1 swap (A = weights)
+  int grouped;     // 1: expert-grouped activations
+  int rows;        // dense: activation rows (tokens)
+  int cols;        // output features (weight rows per expert)
+  int nseg;        // 1 or 2
+  TcSeg seg[2];
+  const int* offsets;         // grouped: [G+1] valid-row offsets
+  const int* padded_offsets;  // grouped: [G+1] padded-row offsets (multiples of 128)
+  int groups;                 // grouped: number of experts
+  void* out;
+  long long ld_out;           // elements
+  const float* bias;          // EPI_F32_BIAS: [cols] or nullptr
+  const float* row_scale;     // EPI_GATE: per activation row, or nullptr (= 1)
+  const __nv_bfloat16* residual;
+  long long ld_res;
+  DevErr err;
+};
+
+template <int BN, int STAGES>
+struct TcSmem {
+  static constexpr int kABytes = 128 * 128;           // 128 rows x 64 bf16
+  static constexpr int kBBytes = BN * 128;            // BN rows x 64 bf16
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, tmem ptr, abort
+  static constexpr int kBytes = kBarOffset + (2 * STAGES + 5) * 8 + 16 + 1024;  // +1024 alignment slack
+};
+
+struct TileInfo {
+  int valid;      // 0: skip (empty expert)
+  int expert;     // grouped: expert; else 0
+  int act0;       // first activation row of the tile
+  int act_n;      // valid activation rows (<= 128 normal, <= BN swap)
+  int w0;         // first weight row (output feature) of the tile
+};
+
+__device__ __forceinline__ int find_expert(const int* poff, int groups, int row) {
+  // largest e with poff[e] <= row (poff is non-decreasing); the expert owning
+  // padded row `row` is the one whose range is non-empty and contains it.
+  int lo = 0, hi = groups;  // answer in [0, groups-1]
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(poff + mid) <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int BN>
+__device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
+  const int ntw_normal = (p.cols + BN - 1) / BN;
+  const int ntw_swap = (p.cols + 127) / 128;
+  if (!p.swap) {
+    int mt = p.grouped ? (__ldg(p.padded_offsets + p.groups) >> 7) : (p.rows + 127) / 128;
+    return mt * ntw_normal;
+  }
+  return p.grouped ? p.groups * ntw_swap : ntw_swap;
+}
+
+template <int BN>
+__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t) {
+  TileInfo ti;
+  ti.valid = 1;
+  ti.expert = 0;
+  if (!p.swap) {
+    const int ntw = (p.cols + BN - 1) / BN;
+    const int nt = t % ntw, mt = t / ntw;
+    ti.w0 = nt * BN;
+    ti.act0 = mt * 128;
+    if (p.grouped) {
+      const int e = find_expert(p.padded_offsets, p.groups, ti.act0);
+      const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+      const int end = __ldg(p.padded_offsets + e) + n_e;
+      ti.expert = e;
+      ti.act_n = min(128, end - ti.act0);
+      if (ti.act_n <= 0) ti.valid = 0;
+    } else {
+      ti.act_n = min(128, p.rows - ti.act0);
+    }
+  } else {
+    const int ntw = (p.cols + 127) / 128;
+    ti.w0 = (t % ntw) * 128;
+    if (p.grouped) {
+      const int e = t / ntw;
+      const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+      ti.expert = e;
+      ti.act0 = __ldg(p.padded_offsets + e);
+      ti.act_n = min(n_e, BN);
+      if (n_e <= 0) ti.valid = 0;
+    } else {
+      ti.act0 = 0;
+      ti.act_n = min(p.rows, BN);
+    }
+  }
+  return ti;
+}
+
+template <int EPI>
+__device__ __forceinline__ float epi_value(float acc, const TcParams& p, long long row, int col) {
+  if (EPI == EPI_SQRELU) {
+    float r = fmaxf(acc, 0.0f);
+    return r * r;
+  } else if (EPI == EPI_GATE) {
+    return p.row_scale ? acc * __ldg(p.row_scale + row) : acc;
+  } else if (EPI == EPI_F32_BIAS) {
+    return p.bias ? acc + __ldg(p.bias + col) : acc;
+  } else if (EPI == EPI_ADD_RES) {
+    return acc + __bfloat162float(p.residual[row * p.ld_res + col]);
+  }
+  return acc;
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                   const TcParams p) {
+  using S = TcSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    if (p.nseg > 1) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
+  }
+  if (warp == 1) tmem_alloc(tmem_ptr, S::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_ptr;
+
+  const int ntiles = tc_num_tiles<BN>(p);
+  const int kb_total = p.seg[0].kblocks + (p.nseg > 1 ? p.seg[1].kblocks : 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      const uint64_t pol_w = policy_evict_first();   // weights: streamed
+      const uint64_t pol_a = policy_evict_last();    // activations: reused across tiles
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;
+      uint32_t last_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileInfo ti = tc_tile<BN>(p, t);
+        if (!ti.valid) continue;
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x100 + stage)) { ok = false; break; }
+          uint8_t* sa = smem + stage * S::kStageBytes;
+          uint8_t* sb = sa + S::kABytes;
+          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+          const int sg = (p.nseg > 1 && kb >= p.seg[0].kblocks) ? 1 : 0;
+          const int k = (sg ? kb - p.seg[0].kblocks : kb) * 64;
+          const CUtensorMap* ma = sg ? &tmA1 : &tmA0;
+          const CUtensorMap* mb = sg ? &tmB1 : &tmB0;
+          const int akg = p.seg[sg].a_kgroup, bkg = p.seg[sg].b_kgroup;
+          int a_row, a_grp, b_row, b_grp;
+          if (!p.swap) {
+            a_row = ti.act0; a_grp = 0; b_row = ti.w0; b_grp = ti.expert;
+          } else {
+            a_row = ti.w0; a_grp = ti.expert; b_row = ti.act0; b_grp = 0;
+          }
+          const uint64_t pa = p.swap ? pol_w : pol_a;
+          const uint64_t pb = p.swap ? pol_a : pol_w;
+          if (akg > 0) tma_load_3d(sa, ma, &full[stage], k % akg, a_row, k / akg, pa);
+          else tma_load_3d(sa, ma, &full[stage], k, a_row, a_grp, pa);
+          if (bkg > 0) tma_load_3d(sb, mb, &full[stage], k % bkg, b_row, k / bkg, pb);
+          else tma_load_3d(sb, mb, &full[stage], k, b_row, b_grp, pb);
+          issued_mask |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        // let every load already issued land before the CTA's memory goes away
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) {
+            long long t0 = clock64();
+            while (!mbar_try_wait(&full[s], (last_par >> s) & 1) && clock64() - t0 < kWaitLimitCycles / 4) {}
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      bool any = false;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const TileInfo ti = tc_tile<BN>(p, t);
+        if (!ti.valid) continue;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, 0x200 + acc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x300 + stage)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
+          const uint32_t sb = sa + S::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32), sdesc_kmajor_sw128(sb + kk * 32), idesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+          }
+          any = true;
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        ++local;
+      }
+      if (any) {
+        mma_commit(drain);
+        long long t0 = clock64();
+        while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles / 4) {}
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;          // TMEM lane quadrant this warp may access
+    const int r = q * 32 + lane;     // accumulator row of this thread
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const TileInfo ti = tc_tile<BN>(p, t);
+      if (!ti.valid) continue;
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, 0x400 + acc)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, v);
+        tmem_ld_wait();
+        if (!p.swap) {
+          const long long row = ti.act0 + r;
+          if (r < ti.act_n) {
+            const int col0 = ti.w0 + c * 32;
+            if (EPI == EPI_F32_BIAS) {
+              float* o = reinterpret_cast<float*>(p.out) + row * p.ld_out + col0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                if (col0 + j < p.cols) {
+                  float4 f;
+                  f.x = epi_value<EPI>(__uint_as_float(v[j + 0]), p, row, col0 + j + 0);
+                  f.y = epi_value<EPI>(__uint_as_float(v[j + 1]), p, row, col0 + j + 1);
+                  f.z = epi_value<EPI>(__uint_as_float(v[j + 2]), p, row, col0 + j + 2);
+                  f.w = epi_value<EPI>(__uint_as_float(v[j + 3]), p, row, col0 + j + 3);
+                  *reinterpret_cast<float4*>(o + j) = f;
+                }
+              }
+            } else {
+              __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                if (col0 + j < p.cols) {
+                  uint4 u;
+                  u.x = pack_bf16x2(epi_value<EPI>(__uint_as_float(v[j + 0]), p, row, col0 + j + 0),
+                                    epi_value<EPI>(__uint_as_float(v[j + 1]), p, row, col0 + j + 1));
+                  u.y = pack_bf16x2(epi_value<EPI>(__uint_as_float(v[j + 2]), p, row, col0 + j + 2),
+                                    epi_value<EPI>(__uint_as_float(v[j + 3]), p, row, col0 + j + 3));
+                  u.z = pack_bf16x2(epi_value<EPI>(__uint_as_float(v[j + 4]), p, row, col0 + j + 4),
+                                    epi_value<EPI>(__uint_as_float(v[j + 5]), p, row, col0 + j + 5));
+                  u.w = pack_bf16x2(epi_value<EPI>(__uint_as_float(v[j + 6]), p, row, col0 + j + 6),
+                                    epi_value<EPI>(__uint_as_float(v[j + 7]), p, row, col0 + j + 7));
+                  *reinterpret_cast<uint4*>(o + j) = u;
+                }
+              }
+            }
+          }
+        } else {
+          // swap: this thread owns output feature `col`; columns of the
+          // accumulator are activation rows (tokens)
+          const int col = ti.w0 + r;
+          if (col < p.cols) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = c * 32 + j;
+              if (tok < ti.act_n) {
+                const long long row = ti.act0 + tok;
+                const float val = epi_value<EPI>(__uint_as_float(v[j]), p, row, col);
+                if (EPI == EPI_F32_BIAS)
+                  reinterpret_cast<float*>(p.out)[row * p.ld_out + col] = val;
+                else
+                  reinterpret_cast<__nv_bfloat16*>(p.out)[row * p.ld_out + col] = __float2bfloat16_rn(val);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      ++local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+}  // namespace lmoe

@@ -1,0 +1,640 @@
+// C ABI of the LatentMoE layer forward: argument checks, workspace carving and
+// the launch sequence of each entry point. Every launch is asynchronous on the
+// caller's stream; nothing here allocates device memory.
+#include <atomic>
+#include <cstring>
+#include <functional>
+
+#include "gemm_tc.cuh"
+#include "lmoe_internal.h"
+
+namespace lmoe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+size_t act_bytes(const lmoe_config* c) { return c->act == LMOE_F32 ? 4 : 2; }
+
+bool identity(const lmoe_config* c) { return (c->flags & LMOE_FLAG_IDENTITY_PROJ) != 0; }
+
+int64_t padded_rows(const lmoe_config* c) {
+  const int64_t slots = c->T * c->K;
+  const int64_t nonempty = slots < c->N ? slots : c->N;
+  return (slots + 127 * nonempty + 127) / 128 * 128;
+}
+
+lmoe_status check_config(const lmoe_config* c) {
+  if (!c) return LMOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->T > (int64_t(1) << 31) / 64) return LMOE_ERR_INVALID_ARG;
+  if (c->d <= 0 || c->l <= 0 || c->N <= 0 || c->K <= 0 || c->m <= 0) return LMOE_ERR_INVALID_ARG;
+  if (c->K > c->N) return LMOE_ERR_INVALID_ARG;
+  if (c->K > 32 || c->N > 1024) return LMOE_ERR_UNSUPPORTED;
+  if (c->n_shared < 0 || (c->n_shared > 0 && c->m_shared <= 0)) return LMOE_ERR_INVALID_ARG;
+  if (c->d % 8 || c->l % 8 || c->m % 8 || (c->n_shared && c->m_shared % 8)) return LMOE_ERR_INVALID_ARG;
+  if (identity(c) && c->l != c->d) return LMOE_ERR_INVALID_ARG;
+  if (c->act != LMOE_F32 && c->act != LMOE_BF16) return LMOE_ERR_UNSUPPORTED;
+  if (c->act == LMOE_F32 && c->expert != LMOE_F32) return LMOE_ERR_UNSUPPORTED;
+  if (c->act == LMOE_BF16 && c->expert != LMOE_BF16 && c->expert != LMOE_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  if (c->act == LMOE_BF16 && c->n_shared > 0 && c->m_shared % 64) return LMOE_ERR_UNSUPPORTED;
+  if (c->expert == LMOE_NVFP4 && (c->l % 256 || c->m % 256)) return LMOE_ERR_UNSUPPORTED;
+  return LMOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Workspace layout (byte offsets; region sizes 0 when unused).
+struct Layout {
+  size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0,
+         offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, scratch = 0, gate = 0, zp = 0,
+         zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, total = 0;
+};
+
+Layout layout(const lmoe_config* c, int op) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += up(bytes);
+    return o;
+  };
+  const int64_t T = c->T, K = c->K, N = c->N;
+  const int64_t P = padded_rows(c);
+  const size_t ab = act_bytes(c);
+  const bool fp4 = c->expert == LMOE_NVFP4;
+  L.err = take(256);
+  if (op == LMOE_OP_ROUTE) {
+    L.logits = take(T * N * 4);
+  } else if (op == LMOE_OP_PERMUTE) {
+    L.scratch = take(static_cast<size_t>(permute_chunks(T * K) + 1) * N * 4);
+  } else if (op == LMOE_OP_EXPERT_FFN) {
+    L.a = take(P * c->m * (fp4 ? 1 : ab) / (fp4 ? 2 : 1));
+    if (fp4) L.a_sf = take(P * c->m / 16);
+  } else if (op == LMOE_OP_NVFP4_QUANTIZE) {
+    L.partials = take(nvfp4_partials(T * c->l) * 4);
+  } else if (op == LMOE_OP_FORWARD) {
+    L.logits = take(T * N * 4);
+    L.idx = take(T * K * 4);
+    L.w = take(T * K * 4);
+    if (!identity(c)) L.z = take(T * c->l * ab);
+    if (fp4) {
+      L.zq = take(T * c->l / 2);
+      L.zq_sf = take(T * c->l / 16);
+      L.z_gs = take(16);
+      L.partials = take(nvfp4_partials(T * c->l) * 4);
+    }
+    L.offsets = take((N + 1) * 4);
+    L.poff = take((N + 1) * 4);
+    L.perm_src = take(T * K * 4);
+    L.inv_perm = take(T * K * 4);
+    L.scratch = take(static_cast<size_t>(permute_chunks(T * K) + 1) * N * 4);
+    L.gate = take(P * 4);
+    if (fp4) {
+      L.zp = take(P * c->l / 2);
+      L.zp_sf = take(P * c->l / 16);
+      L.a = take(P * c->m / 2);
+      L.a_sf = take(P * c->m / 16);
+    } else {
+      L.zp = take(P * c->l * ab);
+      L.a = take(P * c->m * ab);
+    }
+    L.y = take(P * c->l * ab);
+    L.c = take(T * c->l * ab);
+    if (c->n_shared) L.hs = take(T * static_cast<int64_t>(c->n_shared) * c->m_shared * ab);
+  }
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+uint32_t* err_word(void* ws) { return static_cast<uint32_t*>(ws); }
+
+// Token-count threshold below which GEMMs put the weights on the MMA's M side.
+int swap_bn(int64_t T) { return T <= 32 ? 32 : (T <= 64 ? 64 : 0); }
+
+int normal_bn(int cols) { return cols >= 256 ? 256 : cols > 64 ? 128 : cols > 32 ? 64 : 32; }
+
+int kblocks(int64_t k) { return static_cast<int>((k + 63) / 64); }
+
+// out[rows, cols] = epi(x[rows, k] . W[cols, k]^T) with BF16 operands.
+lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int64_t k, void* out,
+                       int64_t ld_out, int epi, const float* bias, const void* residual, int64_t ld_res,
+                       uint32_t* err, cudaStream_t s) {
+  if (rows == 0) return LMOE_OK;
+  TcLaunch L;
+  const int sbn = swap_bn(rows);
+  const TcOperand act{x, k, rows, 1};
+  const TcOperand wt{w, k, cols, 1};
+  L.rows = static_cast<int>(rows);
+  L.cols = cols;
+  L.kblocks[0] = kblocks(k);
+  if (sbn) {
+    L.swap = 1;
+    L.bn = sbn;
+    L.a[0] = wt;
+    L.b[0] = act;
+    L.max_tiles = (cols + 127) / 128;
+  } else {
+    L.bn = normal_bn(cols);
+    L.a[0] = act;
+    L.b[0] = wt;
+    L.max_tiles = ((rows + 127) / 128) * ((cols + L.bn - 1) / L.bn);
+  }
+  L.out = out;
+  L.ld_out = ld_out;
+  L.epi = epi;
+  L.bias = bias;
+  L.residual = residual;
+  L.ld_res = ld_res;
+  return tc_gemm(L, err, s);
+}
+
+}  // namespace
+}  // namespace lmoe
+
+using namespace lmoe;
+
+extern "C" {
+
+const char* lmoe_status_string(lmoe_status s) {
+  switch (s) {
+    case LMOE_OK: return "ok";
+    case LMOE_ERR_INVALID_ARG: return "invalid argument";
+    case LMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LMOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case LMOE_ERR_CUDA: return "CUDA error";
+    case LMOE_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case LMOE_ERR_DEVICE_BOUNDS: return "device index out of range";
+  }
+  return "unknown status";
+}
+
+uint64_t lmoe_kernel_launch_count(void) { return g_launches.load(); }
+
+size_t lmoe_workspace_size(const lmoe_config* cfg, int op) {
+  if (op == LMOE_OP_NVFP4_QUANTIZE) {
+    if (!cfg || cfg->T < 0 || cfg->l <= 0) return 0;
+    return layout(cfg, op).total;
+  }
+  if (check_config(cfg) != LMOE_OK) return 0;
+  if (op == LMOE_OP_COMBINE) return 0;
+  if (op < LMOE_OP_ROUTE || op > LMOE_OP_NVFP4_QUANTIZE) return 0;
+  return layout(cfg, op).total;
+}
+
+int64_t lmoe_padded_rows(const lmoe_config* cfg) {
+  if (check_config(cfg) != LMOE_OK) return 0;
+  return padded_rows(cfg);
+}
+
+lmoe_status lmoe_read_device_error(void* ws, void* stream, uint32_t* info) {
+  if (!ws) return LMOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LMOE_ERR_CUDA;
+  uint32_t w[2] = {0, 0};
+  if (cudaMemcpy(w, ws, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(w)) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (info) *info = w[1];
+  return static_cast<lmoe_status>(w[0]);
+}
+
+lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_router, const float* bias,
+                       const float* logits_in, int32_t* topk_idx, float* topk_w, float* logits_out,
+                       void* ws, size_t ws_bytes, void* stream) {
+  lmoe_status st = check_config(cfg);
+  if (st != LMOE_OK) return st;
+  if (!topk_idx || !topk_w) return LMOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < layout(cfg, LMOE_OP_ROUTE).total) return LMOE_ERR_WORKSPACE;
+  if (!logits_in && (!x || !w_router)) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router)) return LMOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(cfg, LMOE_OP_ROUTE);
+  uint32_t* err = err_word(ws);
+  const float* logits = logits_in;
+  if (!logits) {
+    float* lg = logits_out ? logits_out : at<float>(ws, L.logits);
+    if (cfg->act == LMOE_F32) {
+      SimtLaunch S;
+      S.rows = static_cast<int>(cfg->T);
+      S.cols = cfg->N;
+      S.k = cfg->d;
+      S.a = static_cast<const float*>(x);
+      S.b = static_cast<const float*>(w_router);
+      S.out = lg;
+      S.ld_out = cfg->N;
+      S.bias = bias;
+      S.epi = EPI_F32_BIAS;
+      st = simt_gemm(S, err, s);
+    } else {
+      st = dense_bf16(x, cfg->T, w_router, cfg->N, cfg->d, lg, cfg->N, EPI_F32_BIAS, bias, nullptr, 0, err, s);
+    }
+    if (st != LMOE_OK) return st;
+    logits = lg;
+  }
+  return launch_topk(logits, cfg->T, cfg->N, cfg->K, topk_idx, topk_w, err, s);
+}
+
+lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets, int32_t* perm_src,
+                         int32_t* inv_perm, int32_t* padded_offsets, const void* rows, int64_t row_bytes,
+                         void* permuted_rows, const uint8_t* rows_sf, uint8_t* permuted_sf,
+                         const float* topk_w, float* perm_gate, void* ws, size_t ws_bytes, void* stream) {
+  lmoe_status st = check_config(cfg);
+  if (st != LMOE_OK) return st;
+  if (!topk_idx || !offsets || !perm_src || !inv_perm || !padded_offsets) return LMOE_ERR_INVALID_ARG;
+  if ((rows == nullptr) != (permuted_rows == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if (rows && (row_bytes <= 0 || row_bytes % 16 || !aligned16(rows) || !aligned16(permuted_rows)))
+    return LMOE_ERR_INVALID_ARG;
+  if ((rows_sf == nullptr) != (permuted_sf == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if (rows_sf && (!rows || (row_bytes * 2) % 64)) return LMOE_ERR_INVALID_ARG;
+  if ((topk_w == nullptr) != (perm_gate == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < layout(cfg, LMOE_OP_PERMUTE).total) return LMOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(cfg, LMOE_OP_PERMUTE);
+  uint32_t* err = err_word(ws);
+  st = launch_permute(topk_idx, cfg->T, cfg->K, cfg->N, offsets, perm_src, inv_perm, padded_offsets,
+                      at<int32_t>(ws, L.scratch), topk_w, perm_gate, err, s);
+  if (st != LMOE_OK) return st;
+  if (rows || rows_sf)
+    st = launch_gather(topk_idx, perm_src, offsets, padded_offsets, cfg->T * cfg->K, cfg->K, rows, row_bytes,
+                       permuted_rows, rows_sf, permuted_sf, padded_rows(cfg), s);
+  return st;
+}
+
+}  // extern "C"
+
+namespace lmoe {
+namespace {
+
+// Routed experts on padded expert-grouped rows (BF16 or fp32 experts).
+lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const void* zin,
+                            const int32_t* offsets, const int32_t* poff, const float* gate, void* a,
+                            void* y, uint32_t* err, cudaStream_t s,
+                            const std::function<void()>& between = std::function<void()>()) {
+  const int64_t P = padded_rows(cfg);
+  lmoe_status st;
+  if (cfg->act == LMOE_F32) {
+    SimtLaunch g1;
+    g1.grouped = 1;
+    g1.rows = static_cast<int>(P);
+    g1.cols = cfg->m;
+    g1.k = cfg->l;
+    g1.a = static_cast<const float*>(zin);
+    g1.b = static_cast<const float*>(w->w1);
+    g1.offsets = offsets;
+    g1.padded_offsets = poff;
+    g1.groups = cfg->N;
+    g1.out = static_cast<float*>(a);
+    g1.ld_out = cfg->m;
+    g1.epi = EPI_SQRELU;
+    if ((st = simt_gemm(g1, err, s)) != LMOE_OK) return st;
+    if (between) between();
+    SimtLaunch g2 = g1;
+    g2.cols = cfg->l;
+    g2.k = cfg->m;
+    g2.a = static_cast<const float*>(a);
+    g2.b = static_cast<const float*>(w->w2);
+    g2.out = static_cast<float*>(y);
+    g2.ld_out = cfg->l;
+    g2.epi = EPI_GATE;
+    g2.row_scale = gate;
+    return simt_gemm(g2, err, s);
+  }
+  const int sbn = swap_bn(cfg->T);
+  TcLaunch g1;
+  g1.grouped = 1;
+  g1.cols = cfg->m;
+  g1.kblocks[0] = kblocks(cfg->l);
+  g1.offsets = offsets;
+  g1.padded_offsets = poff;
+  g1.groups = cfg->N;
+  const TcOperand zop{zin, cfg->l, P, 1};
+  const TcOperand w1op{w->w1, cfg->l, cfg->m, cfg->N};
+  if (sbn) {
+    g1.swap = 1;
+    g1.bn = sbn;
+    g1.a[0] = w1op;
+    g1.b[0] = zop;
+    g1.max_tiles = static_cast<int64_t>(cfg->N) * ((cfg->m + 127) / 128);
+  } else {
+    g1.bn = normal_bn(cfg->m);
+    g1.a[0] = zop;
+    g1.b[0] = w1op;
+    g1.max_tiles = (P / 128) * ((cfg->m + g1.bn - 1) / g1.bn);
+  }
+  g1.out = a;
+  g1.ld_out = cfg->m;
+  g1.epi = EPI_SQRELU;
+  if ((st = tc_gemm(g1, err, s)) != LMOE_OK) return st;
+  if (between) between();
+  TcLaunch g2 = g1;
+  g2.cols = cfg->l;
+  g2.kblocks[0] = kblocks(cfg->m);
+  const TcOperand aop{a, cfg->m, P, 1};
+  const TcOperand w2op{w->w2, cfg->m, cfg->l, cfg->N};
+  if (sbn) {
+    g2.a[0] = w2op;
+    g2.b[0] = aop;
+    g2.max_tiles = static_cast<int64_t>(cfg->N) * ((cfg->l + 127) / 128);
+  } else {
+    g2.bn = normal_bn(cfg->l);
+    g2.a[0] = aop;
+    g2.b[0] = w2op;
+    g2.max_tiles = (P / 128) * ((cfg->l + g2.bn - 1) / g2.bn);
+  }
+  g2.out = y;
+  g2.ld_out = cfg->l;
+  g2.epi = EPI_GATE;
+  g2.row_scale = gate;
+  return tc_gemm(g2, err, s);
+}
+
+}  // namespace
+}  // namespace lmoe
+
+extern "C" {
+
+lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w, const void* permuted_in,
+                            const uint8_t* permuted_sf, const float* in_global_scale, const int32_t* offsets,
+                            const int32_t* padded_offsets, const float* perm_gate, void* y_perm, void* ws,
+                            size_t ws_bytes, void* stream) {
+  lmoe_status st = check_config(cfg);
+  if (st != LMOE_OK) return st;
+  if (!w || !w->w1 || !w->w2 || !permuted_in || !offsets || !padded_offsets || !y_perm)
+    return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(permuted_in) || !aligned16(y_perm) || !aligned16(w->w1) || !aligned16(w->w2))
+    return LMOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < layout(cfg, LMOE_OP_EXPERT_FFN).total) return LMOE_ERR_WORKSPACE;
+  if (cfg->expert == LMOE_NVFP4) {
+    (void)permuted_sf;
+    (void)in_global_scale;
+    return LMOE_ERR_UNSUPPORTED;
+  }
+  const Layout L = layout(cfg, LMOE_OP_EXPERT_FFN);
+  return expert_ffn_impl(cfg, w, permuted_in, offsets, padded_offsets, perm_gate, at<void>(ws, L.a), y_perm,
+                         err_word(ws), static_cast<cudaStream_t>(stream));
+}
+
+lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32_t* topk_idx,
+                         const int32_t* inv_perm, const int32_t* offsets, const int32_t* padded_offsets,
+                         const float* topk_w, void* c, void* stream) {
+  lmoe_status st = check_config(cfg);
+  if (st != LMOE_OK) return st;
+  if (!y_perm || !topk_idx || !inv_perm || !offsets || !padded_offsets || !c) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(c)) return LMOE_ERR_INVALID_ARG;
+  return launch_combine(y_perm, cfg->act, topk_idx, inv_perm, offsets, padded_offsets, topk_w, c, cfg->T,
+                        cfg->K, cfg->l, static_cast<cudaStream_t>(stream));
+}
+
+lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* global_in,
+                                uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!in || !codes || !sf) return LMOE_ERR_INVALID_ARG;
+  if (rows < 0 || cols <= 0 || cols % 16) return LMOE_ERR_INVALID_ARG;
+  if (in_dtype != LMOE_F32 && in_dtype != LMOE_BF16) return LMOE_ERR_INVALID_ARG;
+  if (sf_layout != LMOE_SF_ROWMAJOR && sf_layout != LMOE_SF_MMA_TILED) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(in) || (reinterpret_cast<uintptr_t>(codes) & 7)) return LMOE_ERR_INVALID_ARG;
+  lmoe_config q{};
+  q.T = rows;
+  q.l = static_cast<int32_t>(cols);
+  if (!ws || ws_bytes < layout(&q, LMOE_OP_NVFP4_QUANTIZE).total) return LMOE_ERR_WORKSPACE;
+  const Layout L = layout(&q, LMOE_OP_NVFP4_QUANTIZE);
+  if (rows == 0) return LMOE_OK;
+  return launch_nvfp4_quantize(in, in_dtype, rows, cols, global_in, codes, sf, global_out, sf_layout,
+                               at<float>(ws, L.partials), nvfp4_partials(rows * cols), err_word(ws),
+                               static_cast<cudaStream_t>(stream));
+}
+
+lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x, void* out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  return lmoe_forward_traced(cfg, w, x, out, ws, ws_bytes, stream, nullptr);
+}
+
+lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, const void* x, void* out,
+                                void* ws, size_t ws_bytes, void* stream, void* const* events) {
+  lmoe_status st = check_config(cfg);
+  if (st != LMOE_OK) return st;
+  if (!w || !w->w_router || !w->w1 || !w->w2) return LMOE_ERR_INVALID_ARG;
+  const bool ident = identity(cfg);
+  if (ident != (w->w_down == nullptr) || ident != (w->w_up == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if (cfg->n_shared && (!w->ws1 || !w->ws2)) return LMOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < layout(cfg, LMOE_OP_FORWARD).total) return LMOE_ERR_WORKSPACE;
+  if (cfg->expert == LMOE_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return LMOE_OK;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return LMOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Layout L = layout(cfg, LMOE_OP_FORWARD);
+  uint32_t* err = err_word(ws);
+  const int64_t T = cfg->T;
+  int next_event = 0;
+  auto mark = [&](int upto) {
+    // record every event up to and including stage `upto` (skipped stages share a time)
+    while (events && next_event <= upto) cudaEventRecord(static_cast<cudaEvent_t>(events[next_event++]), s);
+  };
+  mark(0);
+  const int d = cfg->d, l = cfg->l, N = cfg->N, K = cfg->K;
+  const size_t ab = act_bytes(cfg);
+  const bool f32 = cfg->act == LMOE_F32;
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* gw = at<float>(ws, L.w);
+  float* logits = at<float>(ws, L.logits);
+
+  // 1. router logits (+ bias) and top-K gates
+  if (f32) {
+    SimtLaunch S;
+    S.rows = static_cast<int>(T);
+    S.cols = N;
+    S.k = d;
+    S.a = static_cast<const float*>(x);
+    S.b = static_cast<const float*>(w->w_router);
+    S.out = logits;
+    S.ld_out = N;
+    S.bias = w->router_bias;
+    S.epi = EPI_F32_BIAS;
+    st = simt_gemm(S, err, s);
+  } else {
+    st = dense_bf16(x, T, w->w_router, N, d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0, err, s);
+  }
+  if (st != LMOE_OK) return st;
+  if ((st = launch_topk(logits, T, N, K, idx, gw, err, s)) != LMOE_OK) return st;
+  mark(1);
+
+  // 2. latent down-projection d -> l
+  const void* z = x;
+  if (!ident) {
+    void* zb = at<void>(ws, L.z);
+    if (f32) {
+      SimtLaunch S;
+      S.rows = static_cast<int>(T);
+      S.cols = l;
+      S.k = d;
+      S.a = static_cast<const float*>(x);
+      S.b = static_cast<const float*>(w->w_down);
+      S.out = static_cast<float*>(zb);
+      S.ld_out = l;
+      S.epi = EPI_BF16;
+      st = simt_gemm(S, err, s);
+    } else {
+      st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, err, s);
+    }
+    if (st != LMOE_OK) return st;
+    z = zb;
+  }
+  mark(2);
+
+  // 3. dispatch grouped by expert (padded rows), gates per padded row
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* poff = at<int32_t>(ws, L.poff);
+  int32_t* perm_src = at<int32_t>(ws, L.perm_src);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  float* gate = at<float>(ws, L.gate);
+  void* zp = at<void>(ws, L.zp);
+  if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
+                           err, s)) != LMOE_OK)
+    return st;
+  if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, static_cast<int64_t>(l) * ab, zp, nullptr,
+                          nullptr, padded_rows(cfg), s)) != LMOE_OK)
+    return st;
+  mark(3);
+
+  // 4. routed expert FFNs in l, gate applied in the second GEMM's epilogue
+  void* y = at<void>(ws, L.y);
+  if ((st = expert_ffn_impl(cfg, w, zp, offsets, poff, gate, at<void>(ws, L.a), y, err, s,
+                            events ? [&]() { mark(4); } : std::function<void()>())) != LMOE_OK)
+    return st;
+  mark(5);
+
+  // 5. combine; with identity projections and no shared experts it is the output
+  const bool combine_is_out = ident && cfg->n_shared == 0;
+  void* c = combine_is_out ? out : at<void>(ws, L.c);
+  if ((st = launch_combine(y, cfg->act, idx, inv_perm, offsets, poff, nullptr, c, T, K, l, s)) != LMOE_OK)
+    return st;
+  mark(6);
+  if (combine_is_out) {
+    mark(7);
+    return LMOE_OK;
+  }
+
+  // 6. shared experts' hidden layer on the d-dim x: hs = relu(x Ws1^T)^2, all S at once
+  const int S = cfg->n_shared, ms = cfg->m_shared;
+  void* hs = S ? at<void>(ws, L.hs) : nullptr;
+  if (S) {
+    if (f32) {
+      SimtLaunch G;
+      G.rows = static_cast<int>(T);
+      G.cols = S * ms;
+      G.k = d;
+      G.a = static_cast<const float*>(x);
+      G.b = static_cast<const float*>(w->ws1);
+      G.out = static_cast<float*>(hs);
+      G.ld_out = static_cast<int64_t>(S) * ms;
+      G.epi = EPI_SQRELU;
+      st = simt_gemm(G, err, s);
+    } else {
+      st = dense_bf16(x, T, w->ws1, S * ms, d, hs, static_cast<int64_t>(S) * ms, EPI_SQRELU, nullptr, nullptr, 0,
+                      err, s);
+    }
+    if (st != LMOE_OK) return st;
+  }
+
+  // 7. up-projection l -> d plus the shared experts' output layer
+  if (f32) {
+    if (!ident) {
+      SimtLaunch U;
+      U.rows = static_cast<int>(T);
+      U.cols = d;
+      U.k = l;
+      U.a = static_cast<const float*>(c);
+      U.b = static_cast<const float*>(w->w_up);
+      U.out = static_cast<float*>(out);
+      U.ld_out = d;
+      U.epi = EPI_BF16;
+      if ((st = simt_gemm(U, err, s)) != LMOE_OK) return st;
+    }
+    for (int sh = 0; sh < S; ++sh) {
+      // out (+)= hs_s Ws2_s^T, hs_s = columns [sh*ms, (sh+1)*ms) of hs
+      SimtLaunch U;
+      U.rows = static_cast<int>(T);
+      U.cols = d;
+      U.k = ms;
+      U.b = static_cast<const float*>(w->ws2) + static_cast<int64_t>(sh) * d * ms;
+      U.out = static_cast<float*>(out);
+      U.ld_out = d;
+      U.a = static_cast<const float*>(hs) + static_cast<int64_t>(sh) * ms;
+      U.lda = static_cast<int64_t>(S) * ms;
+      if (ident && sh == 0) {
+        U.epi = EPI_ADD_RES;
+        U.residual = static_cast<const float*>(c);
+        U.ld_res = l;
+      } else {
+        U.epi = EPI_BF16;
+        U.accumulate = 1;
+      }
+      if ((st = simt_gemm(U, err, s)) != LMOE_OK) return st;
+    }
+    return LMOE_OK;
+  }
+
+  TcLaunch U;
+  U.rows = static_cast<int>(T);
+  U.cols = d;
+  U.out = out;
+  U.ld_out = d;
+  U.epi = EPI_BF16;
+  const int sbn = swap_bn(T);
+  int sg = 0;
+  // segment: (activation operand, weight operand, K, weight K-group)
+  auto add_seg = [&](TcOperand act, TcOperand wt, int64_t k, int wgroup) {
+    if (sbn) {
+      U.a[sg] = wt;
+      U.b[sg] = act;
+      U.a_kgroup[sg] = wgroup;
+    } else {
+      U.a[sg] = act;
+      U.b[sg] = wt;
+      U.b_kgroup[sg] = wgroup;
+    }
+    U.kblocks[sg] = kblocks(k);
+    ++sg;
+  };
+  if (!ident) add_seg(TcOperand{c, l, T, 1}, TcOperand{w->w_up, l, d, 1}, l, 0);
+  if (S) add_seg(TcOperand{hs, static_cast<int64_t>(S) * ms, T, 1}, TcOperand{w->ws2, ms, d, S},
+                 static_cast<int64_t>(S) * ms, ms);
+  U.nseg = sg;
+  if (ident) {
+    U.epi = EPI_ADD_RES;
+    U.residual = c;
+    U.ld_res = l;
+  }
+  if (sbn) {
+    U.swap = 1;
+    U.bn = sbn;
+    U.max_tiles = (d + 127) / 128;
+  } else {
+    U.bn = normal_bn(d);
+    U.max_tiles = ((T + 127) / 128) * ((d + U.bn - 1) / U.bn);
+  }
+  return tc_gemm(U, err, s);
+}
+
+}  // extern "C"

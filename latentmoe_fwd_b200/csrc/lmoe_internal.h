@@ -1,0 +1,95 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lmoe.h"
+
+namespace lmoe {
+
+void count_launch();                 // bump the library's kernel-launch counter
+int device_sm_count();               // SMs of the current device (cached per device)
+
+// ----- tensor-core GEMM (gemm_tc.cu) -----
+struct TcOperand {
+  const void* ptr;     // BF16 [groups][rows][k], k contiguous
+  int64_t k;
+  int64_t rows;
+  int64_t groups;
+};
+
+struct TcLaunch {
+  int swap = 0;
+  int grouped = 0;
+  int rows = 0;                  // dense: activation rows
+  int cols = 0;                  // output features
+  int nseg = 1;
+  TcOperand a[2] = {};
+  TcOperand b[2] = {};
+  int kblocks[2] = {0, 0};
+  int a_kgroup[2] = {0, 0};
+  int b_kgroup[2] = {0, 0};
+  const int* offsets = nullptr;
+  const int* padded_offsets = nullptr;
+  int groups = 0;
+  int64_t max_tiles = 0;         // host upper bound of the tile count (grid sizing)
+  void* out = nullptr;
+  int64_t ld_out = 0;
+  const float* bias = nullptr;
+  const float* row_scale = nullptr;
+  const void* residual = nullptr;
+  int64_t ld_res = 0;
+  int epi = 0;
+  int bn = 256;
+};
+
+lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream);
+
+// ----- fp32 SIMT GEMM (gemm_simt.cu) -----
+struct SimtLaunch {
+  int grouped = 0;
+  int rows = 0;            // dense: activation rows; grouped: padded rows bound
+  int cols = 0;
+  int k = 0;
+  const float* a = nullptr;       // [rows][lda]
+  int64_t lda = 0;                // 0: k
+  const float* b = nullptr;       // [groups][cols][k]
+  const int* offsets = nullptr;
+  const int* padded_offsets = nullptr;
+  int groups = 1;
+  float* out = nullptr;
+  int64_t ld_out = 0;
+  const float* bias = nullptr;
+  const float* row_scale = nullptr;
+  const float* residual = nullptr;
+  int64_t ld_res = 0;
+  int epi = 0;
+  int accumulate = 0;      // 1: out += result (before the epilogue's rounding; fp32 so exact order)
+};
+
+lmoe_status simt_gemm(const SimtLaunch& L, uint32_t* err_word, cudaStream_t stream);
+
+// ----- small kernels (lmoe_kernels.cu) -----
+lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w,
+                        uint32_t* err, cudaStream_t s);
+int permute_chunks(int64_t slots);
+lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
+                           int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
+                           int32_t* scratch, const float* topk_w, float* perm_gate,
+                           uint32_t* err, cudaStream_t s);
+lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int32_t* offsets,
+                          const int32_t* padded_offsets, int64_t slots, int K, const void* rows,
+                          int64_t row_bytes, void* out_rows, const uint8_t* rows_sf,
+                          uint8_t* out_sf, int64_t padded_rows, cudaStream_t s);
+lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
+                           const int32_t* offsets, const int32_t* padded_offsets, const float* w,
+                           void* c, int64_t T, int K, int l, cudaStream_t s);
+lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
+                                  const float* global_in, uint8_t* codes, uint8_t* sf,
+                                  float* global_out, int sf_layout, float* partials,
+                                  int npartials, uint32_t* err, cudaStream_t s);
+int nvfp4_partials(int64_t elems);
+
+}  // namespace lmoe

@@ -1,0 +1,616 @@
+// Router top-K, expert-grouped permutation, gather, combine and the NVFP4
+// quantiser. These steps are bound by memory latency or bandwidth, not by
+// arithmetic: they use coalesced 16-byte accesses, warp intrinsics and
+// shared memory, and no global atomics in the data path.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "lmoe_device.cuh"
+#include "lmoe_internal.h"
+
+namespace lmoe {
+
+// ===========================================================================
+// Top-K + renormalised softmax gates: one warp per token.
+// Selection order: logit descending, expert index ascending (ties to the
+// lower index). Gates: exp(l_k - l_max) / sum over the K chosen.
+// ===========================================================================
+template <int NPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T,
+                                                   int N, int K, int32_t* __restrict__ idx,
+                                                   float* __restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const float* row = logits + t * N;
+  float v[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int col = lane + 32 * i;
+    v[i] = col < N ? __ldg(row + col) : -INFINITY;
+  }
+  uint32_t taken = 0;
+  float my_sel = -INFINITY;  // lane k keeps the k-th selected logit
+  int my_idx = 0;
+  for (int k = 0; k < K; ++k) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int col = lane + 32 * i;
+      const bool live = col < N && !((taken >> i) & 1u);
+      if (live && (v[i] > bv || (v[i] == bv && col < bi))) {
+        bv = v[i];
+        bi = col;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == k) {
+      my_sel = bv;
+      my_idx = bi;
+    }
+  }
+  const float lmax = __shfl_sync(0xffffffffu, my_sel, 0);
+  const float e = lane < K ? expf(my_sel - lmax) : 0.0f;
+  float sum = e;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < K) {
+    idx[t * K + lane] = my_idx;
+    w[t * K + lane] = __fdiv_rn(e, sum);
+  }
+}
+
+lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w,
+                        uint32_t* err, cudaStream_t s) {
+  (void)err;
+  if (T == 0) return LMOE_OK;
+  const int blocks = static_cast<int>((T * 32 + 255) / 256);
+  const int npl = (N + 31) / 32;
+#define LMOE_TOPK(NPLV) \
+  topk_kernel<NPLV><<<blocks, 256, 0, s>>>(logits, T, N, K, idx, w)
+  if (npl <= 1) LMOE_TOPK(1);
+  else if (npl <= 2) LMOE_TOPK(2);
+  else if (npl <= 4) LMOE_TOPK(4);
+  else if (npl <= 8) LMOE_TOPK(8);
+  else if (npl <= 16) LMOE_TOPK(16);
+  else if (npl <= 32) LMOE_TOPK(32);
+  else return LMOE_ERR_UNSUPPORTED;
+#undef LMOE_TOPK
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+// ===========================================================================
+// Permutation: stable counting sort of slots f = t*K + k by expert.
+//   pass 1 (count):  per chunk of kChunk slots, a shared-memory histogram.
+//   pass 2 (scan):   one CTA: per-expert prefix over chunks, then the
+//                    exclusive scan over experts -> offsets and padded offsets
+//                    (each expert's padded range is a multiple of 128 rows).
+//   pass 3 (scatter): every warp walks 32-slot steps of its part of the chunk
+//                    in order; __match_any_sync gives the rank among equal
+//                    experts inside a step, running per-warp counters keep
+//                    the order across steps, so the sort is stable.
+// ===========================================================================
+constexpr int kPermWarps = 8;
+constexpr int kPermSlotsPerWarp = 1024;
+constexpr int kChunk = kPermWarps * kPermSlotsPerWarp;   // 8192 slots per CTA
+constexpr int kPad = 128;
+
+int permute_chunks(int64_t slots) { return static_cast<int>((slots + kChunk - 1) / kChunk); }
+
+__global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx,
+                                                         int64_t slots, int N,
+                                                         int32_t* __restrict__ cnt, DevErr err) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t f0 = static_cast<int64_t>(blockIdx.x) * kChunk;
+  const int64_t f1 = min(slots, f0 + kChunk);
+  for (int64_t f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
+    const int e = __ldg(idx + f);
+    if (e < 0 || e >= N) {
+      dev_report(err, kErrBounds, static_cast<uint32_t>(f));
+      continue;
+    }
+    atomicAdd(&hist[e], 1);   // shared-memory counter; global buffers are written once below
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[static_cast<int64_t>(blockIdx.x) * N + e] = hist[e];
+}
+
+// Block-wide exclusive scan of one value per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) smem_warp[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int s = smem_warp[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += y;
+    }
+    smem_warp[lane] = s;   // inclusive over warps
+  }
+  __syncthreads();
+  const int base = wid > 0 ? smem_warp[wid - 1] : 0;
+  if (total) *total = smem_warp[31];
+  const int r = base + x - v;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ cnt, int nchunks, int N,
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ poff) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < N) {
+    int c = 0;
+    for (; c + 4 <= nchunks; c += 4) {
+      const int v0 = cnt[static_cast<int64_t>(c) * N + e];
+      const int v1 = cnt[static_cast<int64_t>(c + 1) * N + e];
+      const int v2 = cnt[static_cast<int64_t>(c + 2) * N + e];
+      const int v3 = cnt[static_cast<int64_t>(c + 3) * N + e];
+      cnt[static_cast<int64_t>(c) * N + e] = run;
+      cnt[static_cast<int64_t>(c + 1) * N + e] = run + v0;
+      cnt[static_cast<int64_t>(c + 2) * N + e] = run + v0 + v1;
+      cnt[static_cast<int64_t>(c + 3) * N + e] = run + v0 + v1 + v2;
+      run += v0 + v1 + v2 + v3;
+    }
+    for (; c < nchunks; ++c) {
+      const int v0 = cnt[static_cast<int64_t>(c) * N + e];
+      cnt[static_cast<int64_t>(c) * N + e] = run;
+      run += v0;
+    }
+  }
+  int total = 0;
+  const int off = block_exclusive_scan(e < N ? run : 0, warp_sums, &total);
+  const int padded = e < N ? ((run + kPad - 1) / kPad) * kPad : 0;
+  int ptotal = 0;
+  const int poffv = block_exclusive_scan(padded, warp_sums, &ptotal);
+  if (e < N) {
+    offsets[e] = off;
+    poff[e] = poffv;
+  }
+  if (e == 0) {
+    offsets[N] = total;
+    poff[N] = ptotal;
+  }
+}
+
+__global__ void __launch_bounds__(256) perm_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t slots, int N, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff,
+    int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm,
+    const float* __restrict__ topk_w, float* __restrict__ perm_gate) {
+  extern __shared__ int32_t wcnt[];   // [kPermWarps][N]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kPermWarps * N; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  const int64_t f0 = static_cast<int64_t>(blockIdx.x) * kChunk + static_cast<int64_t>(wid) * kPermSlotsPerWarp;
+  const int64_t f1 = min(slots, f0 + kPermSlotsPerWarp);
+  int32_t* my = wcnt + wid * N;
+  const unsigned lt = (1u << lane) - 1u;
+  // per-warp counts
+  for (int64_t s = f0; s < f1; s += 32) {
+    const int64_t f = s + lane;
+    const bool live = f < f1;
+    int e = live ? __ldg(idx + f) : -1;
+    if (e >= N) e = -1;   // out of range: reported by the count pass, skipped here
+    const unsigned act = __ballot_sync(0xffffffffu, live && e >= 0);
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (live && e >= 0 && (peers & act & lt) == 0) my[e] += __popc(peers & act);
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive prefix over the warps of this chunk, per expert
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int run = 0;
+    for (int w2 = 0; w2 < kPermWarps; ++w2) {
+      const int c = wcnt[w2 * N + e];
+      wcnt[w2 * N + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int32_t* cbase = base + static_cast<int64_t>(blockIdx.x) * N;
+  for (int64_t s = f0; s < f1; s += 32) {
+    const int64_t f = s + lane;
+    const bool live = f < f1;
+    int e = live ? __ldg(idx + f) : -1;
+    if (e >= N) e = -1;
+    const unsigned act = __ballot_sync(0xffffffffu, live && e >= 0);
+    const unsigned peers = __match_any_sync(0xffffffffu, e) & act;
+    int r = 0;
+    if (live && e >= 0) {
+      r = __ldg(offsets + e) + __ldg(cbase + e) + my[e] + __popc(peers & lt);
+    }
+    __syncwarp();
+    if (live && e >= 0) {
+      if ((peers & lt) == 0) my[e] += __popc(peers);
+      perm_src[r] = static_cast<int32_t>(f);
+      inv_perm[f] = r;
+      if (perm_gate) {
+        const int p = r - __ldg(offsets + e) + __ldg(poff + e);
+        perm_gate[p] = __ldg(topk_w + f);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
+                           int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
+                           int32_t* scratch, const float* topk_w, float* perm_gate,
+                           uint32_t* err, cudaStream_t s) {
+  if (N > 1024) return LMOE_ERR_UNSUPPORTED;
+  const int64_t slots = T * K;
+  const int nch = permute_chunks(slots);
+  DevErr de{err};
+  if (nch > 0) {
+    perm_count_kernel<<<nch, 256, N * sizeof(int32_t), s>>>(idx, slots, N, scratch, de);
+    count_launch();
+  }
+  perm_scan_kernel<<<1, 1024, 0, s>>>(scratch, nch, N, offsets, padded_offsets);
+  count_launch();
+  if (nch > 0) {
+    const size_t sm = static_cast<size_t>(kPermWarps) * N * sizeof(int32_t);
+    perm_scatter_kernel<<<nch, 256, sm, s>>>(idx, slots, N, scratch, offsets, padded_offsets, perm_src,
+                                            inv_perm, topk_w, perm_gate);
+    count_launch();
+  }
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+// ===========================================================================
+// Gather token rows into the padded expert-grouped buffer: one warp per
+// sorted position, 16-byte loads and stores. NVFP4 block scales move from the
+// row-major [T][cols/16] layout to the MMA-tiled layout at the padded row.
+// ===========================================================================
+__device__ __forceinline__ int64_t sf_tiled_offset(int64_t row, int j, int groups64) {
+  const int64_t atom = (row >> 7) * groups64 + (j >> 2);
+  return atom * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ perm_src,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int64_t slots, int K,
+    const uint8_t* __restrict__ rows, int64_t row_bytes, uint8_t* __restrict__ out,
+    const uint8_t* __restrict__ rows_sf, uint8_t* __restrict__ out_sf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (r >= slots) return;
+  const int f = __ldg(perm_src + r);
+  const int t = f / K;
+  const int e = __ldg(idx + f);
+  const int64_t p = r - __ldg(offsets + e) + __ldg(poff + e);
+  if (out) {
+    const uint4* src = reinterpret_cast<const uint4*>(rows + static_cast<int64_t>(t) * row_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(out + p * row_bytes);
+    const int64_t n16 = row_bytes >> 4;
+    for (int64_t i = lane; i < n16; i += 32) dst[i] = __ldg(src + i);
+  }
+  if (out_sf) {
+    const int cols = static_cast<int>(row_bytes * 2);
+    const int nsf = cols / 16;
+    const int groups64 = (cols + 63) / 64;
+    const uint8_t* src = rows_sf + static_cast<int64_t>(t) * nsf;
+    for (int j = lane * 4; j < nsf; j += 128) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (j + b < nsf) word |= static_cast<uint32_t>(__ldg(src + j + b)) << (8 * b);
+      *reinterpret_cast<uint32_t*>(out_sf + sf_tiled_offset(p, j, groups64)) = word;
+    }
+  }
+}
+
+lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int32_t* offsets,
+                          const int32_t* padded_offsets, int64_t slots, int K, const void* rows,
+                          int64_t row_bytes, void* out_rows, const uint8_t* rows_sf,
+                          uint8_t* out_sf, int64_t padded_rows, cudaStream_t s) {
+  (void)padded_rows;
+  if (slots == 0) return LMOE_OK;
+  const int64_t blocks = (slots * 32 + 255) / 256;
+  gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      idx, perm_src, offsets, padded_offsets, slots, K, static_cast<const uint8_t*>(rows), row_bytes,
+      static_cast<uint8_t*>(out_rows), rows_sf, out_sf);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+// ===========================================================================
+// Combine: c_t = sum_k w_tk * y[row(t,k)], fp32 in k order, one CTA per token.
+// ===========================================================================
+template <typename TA>
+__global__ void __launch_bounds__(256) combine_kernel(
+    const TA* __restrict__ y, const int32_t* __restrict__ idx, const int32_t* __restrict__ inv_perm,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, const float* __restrict__ w,
+    TA* __restrict__ c, int K, int l) {
+  extern __shared__ int64_t rowk[];   // [K] padded rows of this token
+  __shared__ float wk[64];
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < K) {
+    const int64_t f = t * K + threadIdx.x;
+    const int e = __ldg(idx + f);
+    rowk[threadIdx.x] = static_cast<int64_t>(__ldg(inv_perm + f)) - __ldg(offsets + e) + __ldg(poff + e);
+    wk[threadIdx.x] = w ? __ldg(w + f) : 1.0f;
+  }
+  __syncthreads();
+  constexpr int V = 16 / sizeof(TA);   // elements per 16-byte vector
+  for (int col = threadIdx.x * V; col < l; col += blockDim.x * V) {
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(y + rowk[k] * l + col));
+      const float g = wk[k];
+      if constexpr (sizeof(TA) == 2) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f2 = __bfloat1622float2(h[i]);
+          acc[2 * i] += g * f2.x;
+          acc[2 * i + 1] += g * f2.y;
+        }
+      } else {
+        const float* f4 = reinterpret_cast<const float*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += g * f4[i];
+      }
+    }
+    uint4 o;
+    if constexpr (sizeof(TA) == 2) {
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+    } else {
+      o.x = __float_as_uint(acc[0]);
+      o.y = __float_as_uint(acc[1]);
+      o.z = __float_as_uint(acc[2]);
+      o.w = __float_as_uint(acc[3]);
+    }
+    *reinterpret_cast<uint4*>(c + t * l + col) = o;
+  }
+}
+
+lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
+                           const int32_t* offsets, const int32_t* padded_offsets, const float* w,
+                           void* c, int64_t T, int K, int l, cudaStream_t s) {
+  if (T == 0) return LMOE_OK;
+  if (K > 64) return LMOE_ERR_UNSUPPORTED;
+  const size_t sm = static_cast<size_t>(K) * sizeof(int64_t);
+  if (act == LMOE_BF16)
+    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, sm, s>>>(
+        static_cast<const __nv_bfloat16*>(y), idx, inv_perm, offsets, padded_offsets, w,
+        static_cast<__nv_bfloat16*>(c), K, l);
+  else
+    combine_kernel<float><<<static_cast<unsigned>(T), 256, sm, s>>>(
+        static_cast<const float*>(y), idx, inv_perm, offsets, padded_offsets, w,
+        static_cast<float*>(c), K, l);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+// ===========================================================================
+// NVFP4 quantiser.
+//   pass 1: |x| max with one partial per CTA (no float atomics).
+//   pass 2: every CTA reduces the partials (same order -> same s_g), then one
+//           thread per 16-element block: E4M3 block scale and E2M1 codes with
+//           the hardware round-to-nearest-even, satfinite conversions.
+// ===========================================================================
+constexpr int kQThreads = 256;
+
+int nvfp4_partials(int64_t elems) {
+  const int64_t want = (elems + 8 * 1024 - 1) / (8 * 1024);
+  return static_cast<int>(want < 1 ? 1 : (want > 1184 ? 1184 : want));
+}
+
+template <typename TI>
+__device__ __forceinline__ float load_abs_max(const TI* p, int64_t i) {
+  return fabsf(static_cast<float>(p[i]));
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(kQThreads) nvfp4_amax_kernel(const TI* __restrict__ in, int64_t n,
+                                                               float* __restrict__ partials) {
+  __shared__ float red[kQThreads / 32];
+  float m = 0.0f;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    m = fmaxf(m, fabsf(static_cast<float>(in[i])));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = 0.0f;
+    for (int i = 0; i < kQThreads / 32; ++i) r = fmaxf(r, red[i]);
+    partials[blockIdx.x] = r;
+  }
+}
+
+// E4M3 code -> value (exact): subnormal f * 2^-9, normal (8 + f) * 2^(e - 10).
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const int e = (c >> 3) & 15, f = c & 7;
+  return e == 0 ? ldexpf(static_cast<float>(f), -9) : ldexpf(static_cast<float>(8 + f), e - 10);
+}
+
+// fp32 -> E4M3 (round to nearest even, saturating to 448): PTX cvt.
+__device__ __forceinline__ uint32_t cvt_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
+// eight fp32 -> eight E2M1 codes in one 32-bit word, element 2i in the low
+// nibble of byte i (PTX cvt, round to nearest even, saturating).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float x0, float x1, float x2, float x3, float x4,
+                                               float x5, float x6, float x7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
+  return r;
+}
+
+// Every CTA reduces the per-CTA maxima the same way (max is exact, so the
+// order does not matter) and derives s_g = fp32(amax / 2688), 1 when amax = 0.
+__device__ __forceinline__ float cta_global_scale(const float* partials, int np, const float* global_in) {
+  __shared__ float red[kQThreads / 32];
+  __shared__ float result;
+  if (global_in) return __ldg(global_in);
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) m = fmaxf(m, __ldg(partials + i));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = 0.0f;
+    for (int i = 0; i < kQThreads / 32; ++i) r = fmaxf(r, red[i]);
+    result = r == 0.0f ? 1.0f : __fdiv_rn(r, 2688.0f);
+  }
+  __syncthreads();
+  return result;
+}
+
+template <typename TI>
+__device__ __forceinline__ void load16(const TI* src, float (&x)[16]) {
+  if constexpr (sizeof(TI) == 2) {
+    const uint4* p = reinterpret_cast<const uint4*>(src);
+    const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+    const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
+    const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 a = __bfloat1622float2(h0[i]);
+      const float2 b = __bfloat1622float2(h1[i]);
+      x[2 * i] = a.x;
+      x[2 * i + 1] = a.y;
+      x[8 + 2 * i] = b.x;
+      x[8 + 2 * i + 1] = b.y;
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldg(p + i);
+      x[4 * i] = v.x;
+      x[4 * i + 1] = v.y;
+      x[4 * i + 2] = v.z;
+      x[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// Quantise one 16-element block: returns the E4M3 scale code, writes 8 code bytes.
+__device__ __forceinline__ uint32_t nvfp4_block(const float (&x)[16], float s_g, uint2& codes) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const float t = __fmul_rn(s_g, 6.0f);
+  const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, t));
+  const float dec = e4m3_value(sb);
+  uint32_t lo = 0, hi = 0;
+  if (dec != 0.0f) {
+    const float sc = __fmul_rn(dec, s_g);
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(x[i], sc);
+    lo = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+    hi = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+  }
+  codes.x = lo;
+  codes.y = hi;
+  return sb;
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(kQThreads) nvfp4_encode_kernel(
+    const TI* __restrict__ in, int64_t rows, int64_t cols, const float* __restrict__ partials, int np,
+    const float* __restrict__ global_in, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+    float* __restrict__ global_out, int tiled) {
+  const float s_g = cta_global_scale(partials, np, global_in);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && global_out) *global_out = s_g;
+  const int64_t nb = cols / 16;
+  // tiled layout: cover the padded grid so that padding scale bytes are zero
+  const int64_t rows_cov = tiled ? ((rows + 127) / 128) * 128 : rows;
+  const int64_t nb_cov = tiled ? ((cols + 63) / 64) * 4 : nb;
+  const int groups64 = static_cast<int>((cols + 63) / 64);
+  const int64_t total = rows_cov * nb_cov;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = b / nb_cov, j = b % nb_cov;
+    uint32_t scode = 0;
+    if (r < rows && j < nb) {
+      float x[16];
+      load16<TI>(in + r * cols + j * 16, x);
+      uint2 c;
+      scode = nvfp4_block(x, s_g, c);
+      *reinterpret_cast<uint2*>(codes + r * (cols / 2) + j * 8) = c;
+    }
+    if (tiled) sf[sf_tiled_offset(r, static_cast<int>(j), groups64)] = static_cast<uint8_t>(scode);
+    else sf[r * nb + j] = static_cast<uint8_t>(scode);
+  }
+}
+
+lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
+                                  const float* global_in, uint8_t* codes, uint8_t* sf,
+                                  float* global_out, int sf_layout, float* partials, int npartials,
+                                  uint32_t* err, cudaStream_t s) {
+  (void)err;
+  const int64_t n = rows * cols;
+  if (!global_in) {
+    if (in_dtype == LMOE_BF16)
+      nvfp4_amax_kernel<__nv_bfloat16><<<npartials, kQThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(in), n, partials);
+    else
+      nvfp4_amax_kernel<float><<<npartials, kQThreads, 0, s>>>(static_cast<const float*>(in), n, partials);
+    count_launch();
+  }
+  const int tiled = sf_layout == LMOE_SF_MMA_TILED;
+  const int64_t rows_cov = tiled ? ((rows + 127) / 128) * 128 : rows;
+  const int64_t nb_cov = tiled ? ((cols + 63) / 64) * 4 : cols / 16;
+  const int64_t total = rows_cov * nb_cov;
+  const int sms = device_sm_count();
+  int64_t blocks = (total + kQThreads - 1) / kQThreads;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  if (blocks < 1) blocks = 1;
+  if (in_dtype == LMOE_BF16)
+    nvfp4_encode_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kQThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(in), rows, cols, partials, global_in ? 0 : npartials, global_in,
+        codes, sf, global_out, tiled);
+  else
+    nvfp4_encode_kernel<float><<<static_cast<unsigned>(blocks), kQThreads, 0, s>>>(
+        static_cast<const float*>(in), rows, cols, partials, global_in ? 0 : npartials, global_in, codes,
+        sf, global_out, tiled);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+}  // namespace lmoe

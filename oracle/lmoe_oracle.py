@@ -406,10 +406,11 @@ def forward(wl, inp, tokens=None, idx_override=None, precision: str | None = Non
             ws2 = to_f64(inp["ws2"][s], st)
             hs = rho(sq_relu(x @ ws1.T), prec)
             out = out + hs @ ws2.T
+    out_unrounded = out
     out = rho(out, prec)
     return dict(logits=logits, idx=idx, gates=gates, z=z, z_global_scale=zq_scale,
                 counts=counts, offsets=offsets, perm_src=perm_src, inv_perm=inv_perm,
-                a=a, y=y, c=c, out=out, tokens=tok)
+                a=a, y=y, c=c, out=out, out_unrounded=out_unrounded, tokens=tok)
 
 
 def brute_force_topk(logits_row, K: int):

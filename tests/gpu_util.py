@@ -1,0 +1,89 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device,
+build the C-ABI config/weights, compare against the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import latentmoe_fwd_b200 as L
+
+
+def to_dev(a, dtype_tag):
+    """numpy (BF16 bits as uint16, or float32) -> cuda tensor."""
+    if a is None:
+        return None
+    if dtype_tag == "f32":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def cfg_of(wl, T=None):
+    act = L.F32 if wl.dtype == "f32" else L.BF16
+    expert = {"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype]
+    return L.config(T=wl.T if T is None else T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m,
+                    n_shared=wl.n_shared, m_shared=wl.m_shared, act=act, expert=expert,
+                    identity=wl.identity)
+
+
+class DevLayer:
+    """Device copies of one workload's inputs and the C-ABI weight struct."""
+
+    def __init__(self, wl, inp):
+        self.wl = wl
+        st = "f32" if wl.dtype == "f32" else "bf16"
+        self.st = st
+        self.x = to_dev(inp["x"], st)
+        self.t = {k: to_dev(inp[k], st) for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
+        self.bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).cuda()
+        self.cfg = cfg_of(wl)
+        self.w = L.weights(w_router=self.t["w_router"], router_bias=self.bias, w_down=self.t["w_down"],
+                           w_up=self.t["w_up"], w1=self.t["w1"], w2=self.t["w2"], ws1=self.t["ws1"],
+                           ws2=self.t["ws2"])
+
+    def forward(self):
+        out = torch.empty((self.wl.T, self.wl.d), dtype=self.x.dtype, device="cuda")
+        ws = L.workspace(self.cfg, L.OP_FORWARD)
+        L.forward(self.cfg, self.w, self.x, out, ws)
+        st, info = L.read_device_error(ws)
+        assert st == L.OK, (L.status_string(st), hex(info))
+        return out
+
+    def route(self):
+        T, N, K = self.wl.T, self.wl.N, self.wl.K
+        idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+        logits = torch.empty((T, N), dtype=torch.float32, device="cuda")
+        ws = L.workspace(self.cfg, L.OP_ROUTE)
+        L.route(self.cfg, self.x, self.t["w_router"], self.bias, None, idx, w, logits, ws)
+        torch.cuda.synchronize()
+        return idx.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy()
+
+
+def as_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel_max_err(got: np.ndarray, ref: np.ndarray) -> float:
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    return float(np.max(np.abs(got - ref))) / rms
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    _, e = np.frexp(np.abs(v))
+    e = np.maximum(e - 1, -126)
+    return np.ldexp(1.0, e - 7)
+
+
+def bf16_parity(got: np.ndarray, ref_unrounded: np.ndarray, ref_rounded: np.ndarray):
+    """(excess, raw) errors of a BF16 output, both relative to RMS(ref).
+
+    excess: max over elements of |got - exact| beyond half a BF16 step of the
+      oracle's value -- the error a BF16 output adds on top of its own
+      unavoidable representation error. This is what the 2e-2 * RMS and
+      8e-2 * RMS bars are applied to.
+    raw: max |got - RN_bf16(oracle)|, reported alongside.
+    """
+    rms = float(np.sqrt(np.mean(ref_rounded ** 2)))
+    excess = np.maximum(0.0, np.abs(got - ref_unrounded) - bf16_ulp(ref_rounded) / 2).max() / rms
+    raw = np.abs(got - ref_rounded).max() / rms
+    return float(excess), float(raw)

@@ -1,0 +1,105 @@
+"""The C-ABI library loads on a host without a GPU, exports every function
+include/lmoe.h declares, and rejects invalid arguments on the host before
+launching anything (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _ensure_built():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("lmoe_build", os.path.join(ROOT, "latentmoe_fwd_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_ensure_built()
+import latentmoe_fwd_b200 as L  # noqa: E402
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lmoe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for want in ("lmoe_route", "lmoe_permute", "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward",
+                 "lmoe_nvfp4_quantize", "lmoe_workspace_size", "lmoe_read_device_error",
+                 "lmoe_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(L.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_wraps_every_export():
+    assert set(L.EXPORTS) <= set(_declared())
+
+
+def test_status_strings():
+    assert L.status_string(L.OK) == "ok"
+    assert "workspace" in L.status_string(L.ERR_WORKSPACE)
+
+
+def test_workspace_sizes_and_padded_rows():
+    cfg = L.config(T=16384, d=8192, l=2048, N=512, K=22, m=1024)
+    assert L.padded_rows(cfg) == ((16384 * 22 + 127 * 512 + 127) // 128) * 128
+    fwd = L.workspace_size(cfg, L.OP_FORWARD)
+    assert fwd > 3 * 16384 * 22 * 2048 * 2          # z_perm, y and a at least
+    assert L.workspace_size(cfg, L.OP_COMBINE) == 0
+    assert 0 < L.workspace_size(cfg, L.OP_ROUTE) < fwd
+    bad = L.config(T=4, d=64, l=64, N=4, K=5, m=64)    # K > N
+    assert L.workspace_size(bad, L.OP_FORWARD) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=5), L.ERR_INVALID_ARG),               # K > N
+    (dict(K=33, N=64), L.ERR_UNSUPPORTED),        # K above the warp-per-token limit
+    (dict(d=60), L.ERR_INVALID_ARG),              # rows not a multiple of 16 bytes
+    (dict(act=L.F32, expert=L.BF16), L.ERR_UNSUPPORTED),
+    (dict(expert=L.NVFP4, l=128), L.ERR_UNSUPPORTED),
+])
+def test_invalid_configs_rejected_on_host(kw, status):
+    base = dict(T=4, d=64, l=64, N=4, K=2, m=64)
+    base.update(kw)
+    cfg = L.config(**base)
+    w = L.weights(w_router=16, w1=16, w2=16, w_down=16, w_up=16)
+    st = L.lib.lmoe_forward(ctypes.byref(cfg), ctypes.byref(w), 16, 16, 16, 1 << 40, None)
+    assert st == status
+
+
+def test_null_and_workspace_errors_rejected_on_host():
+    cfg = L.config(T=4, d=64, l=32, N=4, K=2, m=64)
+    w = L.weights(w_router=16, w1=16, w2=16, w_down=16, w_up=16)
+    # workspace too small
+    assert L.lib.lmoe_forward(ctypes.byref(cfg), ctypes.byref(w), 16, 16, 16, 8, None) == L.ERR_WORKSPACE
+    # missing w_up while not identity
+    w2 = L.weights(w_router=16, w1=16, w2=16, w_down=16)
+    assert L.lib.lmoe_forward(ctypes.byref(cfg), ctypes.byref(w2), 16, 16, 16, 1 << 40, None) == L.ERR_INVALID_ARG
+    # misaligned x
+    assert L.lib.lmoe_forward(ctypes.byref(cfg), ctypes.byref(w), 18, 16, 16, 1 << 40, None) == L.ERR_INVALID_ARG
+    # route needs outputs
+    assert L.lib.lmoe_route(ctypes.byref(cfg), 16, 16, None, None, None, None, None, 16, 1 << 20,
+                            None) == L.ERR_INVALID_ARG
+    # nvfp4: cols must be a multiple of 16
+    assert L.lib.lmoe_nvfp4_quantize(16, L.BF16, 4, 24, None, 16, 16, None, 0, 16, 1 << 20,
+                                     None) == L.ERR_INVALID_ARG
+    # permute: rows without a destination
+    assert L.lib.lmoe_permute(ctypes.byref(cfg), 16, 16, 16, 16, 16, 16, 64, None, None, None, None, None,
+                              16, 1 << 20, None) == L.ERR_INVALID_ARG
+
+
+def test_launch_counter_starts_and_is_monotone():
+    a = L.kernel_launch_count()
+    b = L.kernel_launch_count()
+    assert b >= a >= 0

@@ -1,0 +1,64 @@
+"""Parity at the workloads' full sizes, in the launch configuration the
+benchmark times (lmoe_forward on the whole batch).
+
+* routing over every token: bit-exact against the oracle's selection from its
+  own fp64 logits, except documented near-ties (gap < 1e-5);
+* the permutation of the GPU's routing: bit-exact over every slot;
+* outputs: a seeded sample of tokens the oracle computes one by one, with the
+  same error measure as the reduced-size tests (BF16: max|err| beyond half a
+  BF16 step <= 2e-2 * RMS).
+"""
+import numpy as np
+import pytest
+import torch
+
+import lmoe_inputs as LI
+from oracle import lmoe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+L = pytest.importorskip("latentmoe_fwd_b200")
+from gpu_util import DevLayer, as_f64, bf16_parity  # noqa: E402
+
+SAMPLE = 24
+
+
+@pytest.mark.parametrize("name", ["std_moe_bf16", "ultra_decode", "ultra_zipf"])
+def test_full_size_bf16(name):
+    wl = LI.WORKLOADS[name]
+    inp = LI.make_inputs(wl)
+    dev = DevLayer(wl, inp)
+    out = as_f64(dev.forward())
+    gidx, gw, glogits = dev.route()
+
+    # routing over every token
+    x = O.from_bf16_bits(inp["x"])
+    logits = O.router_logits(x, O.from_bf16_bits(inp["w_router"]), inp["router_bias"])
+    ridx, rgates = O.route_topk(logits, wl.K)
+    near = O.near_tie_tokens(logits, wl.K)
+    same = np.all(gidx == ridx, axis=1)
+    assert np.all(same | near), f"{np.sum(~(same | near))} tokens routed differently without a near-tie"
+    ok = same
+    assert np.max(np.abs(gw[ok] - rgates[ok])) <= 1e-5
+    print(f"{name}: {np.sum(near)} near-tie tokens, {np.sum(~same)} routed differently")
+
+    # permutation of the GPU's routing, every slot
+    T, K, N = wl.T, wl.K, wl.N
+    cfg = dev.cfg
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device="cuda")
+    offsets, poff, perm_src, inv_perm = i32(N + 1), i32(N + 1), i32(T * K), i32(T * K)
+    ws = L.workspace(cfg, L.OP_PERMUTE)
+    L.permute(cfg, torch.from_numpy(gidx).cuda(), offsets, perm_src, inv_perm, poff, ws=ws)
+    assert L.read_device_error(ws)[0] == L.OK
+    _, r_off, r_src, r_inv = O.permute(gidx, N)
+    assert np.array_equal(offsets.cpu().numpy(), r_off)
+    assert np.array_equal(perm_src.cpu().numpy(), r_src)
+    assert np.array_equal(inv_perm.cpu().numpy(), r_inv)
+
+    # sampled outputs
+    rng = np.random.default_rng(123)
+    toks = np.sort(rng.choice(T, size=min(SAMPLE, T), replace=False))
+    ref = O.forward(wl, inp, tokens=toks, idx_override=gidx[toks])
+    excess, raw = bf16_parity(out[toks], ref["out_unrounded"], ref["out"])
+    print(f"{name}: sampled {len(toks)} tokens: excess {excess:.3e} * RMS, raw {raw:.3e} * RMS")
+    assert excess <= 2e-2
