@@ -181,6 +181,9 @@ def forward_traced(cfg, w: Weights, x, out, ws, events, stream=None):
     """lmoe_forward recording ``TRACE_EVENTS`` torch.cuda.Event objects (timing
     enabled) at the stage boundaries on the launch stream."""
     assert len(events) == TRACE_EVENTS
+    for e in events:
+        if e.cuda_event == 0:      # torch creates the CUDA event on its first record
+            e.record()
     arr = (ctypes.c_void_p * TRACE_EVENTS)(*[e.cuda_event for e in events])
     _check(lib.lmoe_forward_traced(ctypes.byref(cfg), ctypes.byref(w), _p(x), _p(out), _p(ws), ws.numel(),
                                    _stream(stream), arr), "lmoe_forward_traced")

@@ -1,0 +1,372 @@
+// Grouped block-scaled NVFP4 GEMM for sm_100a (tcgen05.mma kind::mxf4nvf4,
+// 16-element blocks with E4M3 scales), used for the routed experts when the
+// expert weights and the latent activations are NVFP4:
+//
+//   acc[r, c] = sum_k (q_a[r,k] * sa[r,k/16]) * (q_w[c,k] * sw[c,k/16])
+//   GEMM 1: a = relu(acc * s_z * s_w1[e])^2, quantised to NVFP4 with the
+//           static scale s_a (codes + MMA-tiled scales written directly)
+//   GEMM 2: y = acc * s_a * s_w2[e] * gate[row], stored as BF16
+//
+// Structure as the BF16 kernel (TMA producer warp, single-thread MMA issuer,
+// four epilogue warps, persistent tiles of 128 activation rows x 256 output
+// features), plus:
+//  * each stage carries the tile's scale atoms (512 B = 128 rows x 4 scales),
+//    fetched with bulk copies and moved shared -> tensor memory with
+//    tcgen05.cp (32 lanes x 128 bit, replicated over the four lane quarters)
+//    just before the MMAs that read them; copies and MMAs issued by one
+//    thread execute in order, so one scale buffer in TMEM suffices;
+//  * the two 256-column accumulators overlap in TMEM columns [192, 256) to
+//    leave room for the scales ([0,256) and [192,448); scales at 448+); the
+//    epilogue drains that shared slice first and then releases the MMA.
+#pragma once
+
+#include "lmoe_device.cuh"
+
+namespace lmoe {
+
+enum Fp4Epi : int { FP4_EPI_SQRELU_QUANT = 0, FP4_EPI_GATE_BF16 = 1 };
+
+struct Fp4Params {
+  int cols;                   // output features per expert
+  int kblocks;                // 256-element K blocks
+  int sf_groups_a;            // K / 64: scale atoms per 128-row block of A
+  int sf_groups_b;            // K / 64 for B
+  const uint8_t* sfa;         // activation scales, MMA-tiled over the padded rows
+  const uint8_t* sfb;         // weight scales, MMA-tiled, expert-major
+  long long sfb_expert_bytes; // bytes of one expert's weight scales
+  const int* offsets;
+  const int* padded_offsets;
+  int groups;
+  const float* in_scale;      // global scale of A (device scalar)
+  const float* w_scale;       // [groups] global scales of B
+  const float* out_scale;     // GEMM1: static global scale of a (device scalar)
+  const float* row_scale;     // GEMM2: gate per padded row (nullable)
+  void* out;                  // GEMM1: codes [rows][cols/2]; GEMM2: bf16 [rows][cols]
+  uint8_t* out_sf;            // GEMM1: MMA-tiled scales of a
+  long long ld_out;           // GEMM2: elements per row
+  DevErr err;
+};
+
+struct Fp4Smem {
+  static constexpr int kA = 128 * 128;       // 128 rows x 256 fp4
+  static constexpr int kB = 256 * 128;       // 256 rows x 256 fp4
+  static constexpr int kSFA = 4 * 512;       // 4 atoms (4 K-blocks of 64) x 128 rows
+  static constexpr int kSFB = 8 * 512;       // 4 K-blocks x 2 row blocks
+  static constexpr int kStage = kA + kB + kSFA + kSFB;   // 55296
+  static constexpr int kStages = 4;
+  static constexpr int kBarOffset = kStages * kStage;
+  static constexpr int kBytes = kBarOffset + (2 * kStages + 6) * 8 + 16 + 1024;
+  static constexpr int kAccCols = 256;
+  static constexpr int kAcc1 = 192;          // second accumulator starts here
+  static constexpr int kSfaCol = 448;
+  static constexpr int kSfbCol = 464;
+};
+
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
+  return (1u << 7)                                   // A format E2M1
+         | (1u << 10)                                // B format E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (0u << 23)                                // scale format UE4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory descriptor of one 512-byte scale atom (32 rows x 16 B, no
+// swizzle; 8-row core matrices 128 B apart) as the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;     // leading byte offset
+  d |= static_cast<uint64_t>(128 >> 4) << 32;     // stride byte offset (next 8 rows)
+  d |= static_cast<uint64_t>(1) << 46;            // version
+  return d;                                       // swizzle none
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// E4M3 scale of a block and its exact value (see the quantiser).
+__device__ __forceinline__ uint32_t fp4_cvt_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
+__device__ __forceinline__ float fp4_e4m3_value(uint32_t c) {
+  const int e = (c >> 3) & 15, f = c & 7;
+  return e == 0 ? ldexpf(static_cast<float>(f), -9) : ldexpf(static_cast<float>(8 + f), e - 10);
+}
+
+__device__ __forceinline__ uint32_t fp4_cvt_x8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// Quantise 16 values with global scale s_g: returns the E4M3 code and 8 code bytes.
+__device__ __forceinline__ uint32_t fp4_quant16(const float* x, float s_g, uint2& codes) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const uint32_t sb = fp4_cvt_e4m3(__fdiv_rn(amax, __fmul_rn(s_g, 6.0f)));
+  const float dec = fp4_e4m3_value(sb);
+  codes.x = 0;
+  codes.y = 0;
+  if (dec != 0.0f) {
+    const float sc = __fmul_rn(dec, s_g);
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(x[i], sc);
+    codes.x = fp4_cvt_x8(v);
+    codes.y = fp4_cvt_x8(v + 8);
+  }
+  return sb;
+}
+
+__device__ __forceinline__ long long fp4_sf_offset(long long row, int j, int groups64) {
+  return ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(192, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Fp4Params p) {
+  using S = Fp4Smem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
+  uint64_t* empty = full + S::kStages;
+  uint64_t* tfull = empty + S::kStages;   // [2]
+  uint64_t* overlap_free = tfull + 2;     // [1]: previous tile drained the shared slice
+  uint64_t* drain = overlap_free + 1;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&tfull[0], 1);
+    mbar_init(&tfull[1], 1);
+    mbar_init(overlap_free, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_ptr, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_ptr;
+
+  const int ntw = (p.cols + 255) / 256;
+  const int ntiles = (__ldg(p.padded_offsets + p.groups) >> 7) * ntw;
+
+  auto tile_of = [&](int t, int& e, int& act0, int& act_n, int& w0) {
+    w0 = (t % ntw) * 256;
+    act0 = (t / ntw) * 128;
+    e = find_expert(p.padded_offsets, p.groups, act0);
+    const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+    act_n = min(128, __ldg(p.padded_offsets + e) + n_e - act0);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int e, act0, act_n, w0;
+        tile_of(t, e, act0, act_n, w0);
+        if (act_n <= 0) continue;
+        const uint8_t* sfa_blk = p.sfa + static_cast<long long>(act0 >> 7) * p.sf_groups_a * 512;
+        const uint8_t* sfb_e = p.sfb + static_cast<long long>(e) * p.sfb_expert_bytes;
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x1100 + stage)) { ok = false; break; }
+          uint8_t* sa = smem + stage * S::kStage;
+          uint8_t* sb = sa + S::kA;
+          uint8_t* ssfa = sb + S::kB;
+          uint8_t* ssfb = ssfa + S::kSFA;
+          mbar_arrive_expect_tx(&full[stage], S::kStage);
+          tma_load_3d(sa, &tmA, &full[stage], kb * 128, act0, 0, pol_a);
+          tma_load_3d(sb, &tmB, &full[stage], kb * 128, w0, e, pol_w);
+          bulk_load(ssfa, sfa_blk + kb * 4 * 512, S::kSFA, &full[stage]);
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb)
+            bulk_load(ssfb + nb * 2048,
+                      sfb_e + (static_cast<long long>((w0 >> 7) + nb) * p.sf_groups_b + kb * 4) * 512, 2048,
+                      &full[stage]);
+          issued_mask |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < S::kStages; ++s)
+          if (issued_mask & (1u << s)) {
+            long long t0 = clock64();
+            while (!mbar_try_wait(&full[s], (last_par >> s) & 1) && clock64() - t0 < kWaitLimitCycles / 4) {}
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_nvfp4(128, 256);
+      const uint32_t sfa_t = tmem_base + S::kSfaCol;
+      const uint32_t sfb_t = tmem_base + S::kSfbCol;
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true, any = false;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int e, act0, act_n, w0;
+        tile_of(t, e, act0, act_n, w0);
+        if (act_n <= 0) continue;
+        if (local > 0) {
+          if (!mbar_wait(overlap_free, (local - 1) & 1, abort_flag, p.err, 0x1200)) { ok = false; break; }
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ((local & 1) ? S::kAcc1 : 0);
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x1300 + stage)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* sa = smem + stage * S::kStage;
+          const uint32_t a_s = smem_u32(sa);
+          const uint32_t b_s = a_s + S::kA;
+          const uint32_t sfa_s = b_s + S::kB;
+          const uint32_t sfb_s = sfa_s + S::kSFA;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            tmem_cp_sf(sfa_t + kk * 4, sdesc_sf_atom(sfa_s + kk * 512));
+            tmem_cp_sf(sfb_t + kk * 8, sdesc_sf_atom(sfb_s + kk * 512));
+            tmem_cp_sf(sfb_t + kk * 8 + 4, sdesc_sf_atom(sfb_s + 2048 + kk * 512));
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_nvfp4(d_tmem, sdesc_kmajor_sw128(a_s + kk * 32), sdesc_kmajor_sw128(b_s + kk * 32), idesc,
+                      sfa_t + kk * 4, sfb_t + kk * 8, (kb | kk) != 0 ? 1u : 0u);
+          }
+          any = true;
+          mma_commit(&empty[stage]);
+          if (++stage == S::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[local & 1]);
+        ++local;
+      }
+      if (any) {
+        mma_commit(drain);
+        long long t0 = clock64();
+        while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles / 4) {}
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int local = 0;
+    const float in_s = __ldg(p.in_scale);
+    const float out_s = (EPI == FP4_EPI_SQRELU_QUANT) ? __ldg(p.out_scale) : 0.0f;
+    const int groups64_out = (p.cols + 63) / 64;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int e, act0, act_n, w0;
+      tile_of(t, e, act0, act_n, w0);
+      if (act_n <= 0) continue;
+      const int buf = local & 1;
+      if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1400 + buf)) break;
+      tc_fence_after();
+      const float scale = __fmul_rn(in_s, __ldg(p.w_scale + e)) * (EPI == FP4_EPI_GATE_BF16 ? 1.0f : 1.0f);
+      const uint32_t acc_col = buf ? S::kAcc1 : 0;
+      const long long row = act0 + r;
+      const bool row_ok = r < act_n;
+      const float gate = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && row_ok) ? __ldg(p.row_scale + row) : 1.0f;
+#pragma unroll 1
+      for (int i = 0; i < 8; ++i) {
+        // drain the TMEM slice shared with the other accumulator first
+        const int c = buf ? i : (i + 6) & 7;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc_col + c * 32, v);
+        tmem_ld_wait();
+        if (i == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(overlap_free);
+        }
+        const int col0 = w0 + c * 32;
+        if (!row_ok || col0 >= p.cols) continue;
+        if (EPI == FP4_EPI_SQRELU_QUANT) {
+          float a[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float h = fmaxf(__uint_as_float(v[j]) * scale, 0.0f);
+            a[j] = h * h;
+          }
+          uint2 c0, c1;
+          const uint32_t s0 = fp4_quant16(a, out_s, c0);
+          const uint32_t s1 = fp4_quant16(a + 16, out_s, c1);
+          uint8_t* codes = reinterpret_cast<uint8_t*>(p.out) + row * (p.cols / 2) + col0 / 2;
+          *reinterpret_cast<uint4*>(codes) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+          const int j0 = col0 / 16;
+          p.out_sf[fp4_sf_offset(row, j0, groups64_out)] = static_cast<uint8_t>(s0);
+          p.out_sf[fp4_sf_offset(row, j0 + 1, groups64_out)] = static_cast<uint8_t>(s1);
+        } else {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
+          const float sg = scale * gate;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(v[j + 0]) * sg, __uint_as_float(v[j + 1]) * sg);
+            u.y = pack_bf16x2(__uint_as_float(v[j + 2]) * sg, __uint_as_float(v[j + 3]) * sg);
+            u.z = pack_bf16x2(__uint_as_float(v[j + 4]) * sg, __uint_as_float(v[j + 5]) * sg);
+            u.w = pack_bf16x2(__uint_as_float(v[j + 6]) * sg, __uint_as_float(v[j + 7]) * sg);
+            *reinterpret_cast<uint4*>(o + j) = u;
+          }
+        }
+      }
+      ++local;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace lmoe

@@ -79,17 +79,6 @@ struct TileInfo {
   int w0;         // first weight row (output feature) of the tile
 };
 
-__device__ __forceinline__ int find_expert(const int* poff, int groups, int row) {
-  // largest e with poff[e] <= row (poff is non-decreasing); the expert owning
-  // padded row `row` is the one whose range is non-empty and contains it.
-  int lo = 0, hi = groups;  // answer in [0, groups-1]
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (__ldg(poff + mid) <= row) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 template <int BN>
 __device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
   const int ntw_normal = (p.cols + BN - 1) / BN;
@@ -375,6 +364,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, S::kTmemCols);
   }

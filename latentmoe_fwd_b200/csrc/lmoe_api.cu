@@ -369,6 +369,56 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   return tc_gemm(g2, err, s);
 }
 
+// Routed experts with NVFP4 weights and latent activations: two block-scaled
+// GEMMs; the first quantises a = relu(h)^2 to NVFP4 (static scale) in its epilogue.
+lmoe_status expert_ffn_fp4(const lmoe_config* cfg, const lmoe_weights* w, const void* zcodes, const uint8_t* zsf,
+                           const float* z_gs, const int32_t* offsets, const int32_t* poff, const float* gate,
+                           void* a_codes, uint8_t* a_sf, void* y, uint32_t* err, cudaStream_t s,
+                           const std::function<void()>& between = std::function<void()>()) {
+  const int64_t P = padded_rows(cfg);
+  Fp4Launch g1;
+  g1.a_codes = zcodes;
+  g1.a_sf = zsf;
+  g1.a_rows = P;
+  g1.b_codes = w->w1;
+  g1.b_sf = w->w1_sf;
+  g1.k = cfg->l;
+  g1.cols = cfg->m;
+  g1.groups = cfg->N;
+  g1.offsets = offsets;
+  g1.padded_offsets = poff;
+  g1.in_scale = z_gs;
+  g1.w_scale = w->w1_gs;
+  g1.out_scale = w->a_global_scale;
+  g1.quant_out = 1;
+  g1.out = a_codes;
+  g1.out_sf = a_sf;
+  lmoe_status st = fp4_gemm(g1, err, s);
+  if (st != LMOE_OK) return st;
+  if (between) between();
+  Fp4Launch g2 = g1;
+  g2.a_codes = a_codes;
+  g2.a_sf = a_sf;
+  g2.b_codes = w->w2;
+  g2.b_sf = w->w2_sf;
+  g2.k = cfg->m;
+  g2.cols = cfg->l;
+  g2.in_scale = w->a_global_scale;
+  g2.w_scale = w->w2_gs;
+  g2.out_scale = nullptr;
+  g2.row_scale = gate;
+  g2.quant_out = 0;
+  g2.out = y;
+  g2.out_sf = nullptr;
+  g2.ld_out = cfg->l;
+  return fp4_gemm(g2, err, s);
+}
+
+bool fp4_weights_ok(const lmoe_weights* w) {
+  return w->w1_sf && w->w2_sf && w->w1_gs && w->w2_gs && w->a_global_scale && aligned16(w->w1_sf) &&
+         aligned16(w->w2_sf);
+}
+
 }  // namespace
 }  // namespace lmoe
 
@@ -385,12 +435,13 @@ lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w, const
   if (!aligned16(permuted_in) || !aligned16(y_perm) || !aligned16(w->w1) || !aligned16(w->w2))
     return LMOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < layout(cfg, LMOE_OP_EXPERT_FFN).total) return LMOE_ERR_WORKSPACE;
-  if (cfg->expert == LMOE_NVFP4) {
-    (void)permuted_sf;
-    (void)in_global_scale;
-    return LMOE_ERR_UNSUPPORTED;
-  }
   const Layout L = layout(cfg, LMOE_OP_EXPERT_FFN);
+  if (cfg->expert == LMOE_NVFP4) {
+    if (!permuted_sf || !in_global_scale || !fp4_weights_ok(w) || !aligned16(permuted_sf)) return LMOE_ERR_INVALID_ARG;
+    return expert_ffn_fp4(cfg, w, permuted_in, permuted_sf, in_global_scale, offsets, padded_offsets, perm_gate,
+                          at<void>(ws, L.a), at<uint8_t>(ws, L.a_sf), y_perm, err_word(ws),
+                          static_cast<cudaStream_t>(stream));
+  }
   return expert_ffn_impl(cfg, w, permuted_in, offsets, padded_offsets, perm_gate, at<void>(ws, L.a), y_perm,
                          err_word(ws), static_cast<cudaStream_t>(stream));
 }
@@ -439,7 +490,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   if (ident != (w->w_down == nullptr) || ident != (w->w_up == nullptr)) return LMOE_ERR_INVALID_ARG;
   if (cfg->n_shared && (!w->ws1 || !w->ws2)) return LMOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < layout(cfg, LMOE_OP_FORWARD).total) return LMOE_ERR_WORKSPACE;
-  if (cfg->expert == LMOE_NVFP4) return LMOE_ERR_UNSUPPORTED;
+  const bool fp4 = cfg->expert == LMOE_NVFP4;
+  if (fp4 && !fp4_weights_ok(w)) return LMOE_ERR_INVALID_ARG;
   if (cfg->T == 0) return LMOE_OK;
   if (!x || !out || !aligned16(x) || !aligned16(out)) return LMOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -500,6 +552,18 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     if (st != LMOE_OK) return st;
     z = zb;
   }
+  uint8_t* zq_sf = nullptr;
+  float* z_gs = nullptr;
+  if (fp4) {
+    // NVFP4 latent activations: current per-tensor amax, row-major block scales
+    zq_sf = at<uint8_t>(ws, L.zq_sf);
+    z_gs = at<float>(ws, L.z_gs);
+    if ((st = launch_nvfp4_quantize(z, LMOE_BF16, T, l, nullptr, at<uint8_t>(ws, L.zq), zq_sf, z_gs,
+                                    LMOE_SF_ROWMAJOR, at<float>(ws, L.partials), nvfp4_partials(T * l), err, s)) !=
+        LMOE_OK)
+      return st;
+    z = at<void>(ws, L.zq);
+  }
   mark(2);
 
   // 3. dispatch grouped by expert (padded rows), gates per padded row
@@ -512,16 +576,22 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
                            err, s)) != LMOE_OK)
     return st;
-  if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, static_cast<int64_t>(l) * ab, zp, nullptr,
-                          nullptr, padded_rows(cfg), s)) != LMOE_OK)
+  const int64_t row_bytes = fp4 ? l / 2 : static_cast<int64_t>(l) * ab;
+  uint8_t* zp_sf = fp4 ? at<uint8_t>(ws, L.zp_sf) : nullptr;
+  if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, zq_sf, zp_sf,
+                          padded_rows(cfg), s)) != LMOE_OK)
     return st;
   mark(3);
 
   // 4. routed expert FFNs in l, gate applied in the second GEMM's epilogue
   void* y = at<void>(ws, L.y);
-  if ((st = expert_ffn_impl(cfg, w, zp, offsets, poff, gate, at<void>(ws, L.a), y, err, s,
-                            events ? [&]() { mark(4); } : std::function<void()>())) != LMOE_OK)
-    return st;
+  const std::function<void()> between = events ? std::function<void()>([&]() { mark(4); }) : std::function<void()>();
+  if (fp4)
+    st = expert_ffn_fp4(cfg, w, zp, zp_sf, z_gs, offsets, poff, gate, at<void>(ws, L.a), at<uint8_t>(ws, L.a_sf), y,
+                        err, s, between);
+  else
+    st = expert_ffn_impl(cfg, w, zp, offsets, poff, gate, at<void>(ws, L.a), y, err, s, between);
+  if (st != LMOE_OK) return st;
   mark(5);
 
   // 5. combine; with identity projections and no shared experts it is the output
@@ -592,6 +662,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
       }
       if ((st = simt_gemm(U, err, s)) != LMOE_OK) return st;
     }
+    mark(7);
     return LMOE_OK;
   }
 
@@ -634,7 +705,9 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     U.bn = normal_bn(d);
     U.max_tiles = ((T + 127) / 128) * ((d + U.bn - 1) / U.bn);
   }
-  return tc_gemm(U, err, s);
+  st = tc_gemm(U, err, s);
+  mark(7);
+  return st;
 }
 
 }  // extern "C"

@@ -47,6 +47,30 @@ struct TcLaunch {
 
 lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream);
 
+// ----- grouped NVFP4 expert GEMM (gemm_fp4.cu) -----
+struct Fp4Launch {
+  const void* a_codes = nullptr;     // [a_rows][k/2] packed E2M1 (padded expert-grouped rows)
+  const uint8_t* a_sf = nullptr;     // MMA-tiled scales of A
+  int64_t a_rows = 0;                // padded rows (multiple of 128)
+  const void* b_codes = nullptr;     // [groups][cols][k/2]
+  const uint8_t* b_sf = nullptr;     // per expert, MMA-tiled
+  int64_t k = 0;
+  int cols = 0;
+  int groups = 0;
+  const int* offsets = nullptr;
+  const int* padded_offsets = nullptr;
+  const float* in_scale = nullptr;   // device scalar
+  const float* w_scale = nullptr;    // [groups]
+  const float* out_scale = nullptr;  // device scalar (quant_out)
+  const float* row_scale = nullptr;  // gates (GEMM 2)
+  int quant_out = 0;                 // 1: relu^2 + NVFP4 codes/scales out; 0: BF16 out * gate
+  void* out = nullptr;
+  uint8_t* out_sf = nullptr;
+  int64_t ld_out = 0;
+};
+
+lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream);
+
 // ----- fp32 SIMT GEMM (gemm_simt.cu) -----
 struct SimtLaunch {
   int grouped = 0;

@@ -250,12 +250,16 @@ def route_topk(logits, K: int):
 
 
 def near_tie_tokens(logits, K: int, gap: float = 1e-5) -> np.ndarray:
-    """Tokens whose K-th and (K+1)-th largest logits differ by less than ``gap``."""
+    """Tokens whose routing output is decided by a logit gap below ``gap``:
+    two consecutive values among the K+1 largest logits (the K-th against the
+    (K+1)-th decides the chosen set; consecutive chosen ones decide their
+    order in the output) differ by less than ``gap``."""
     logits = np.asarray(logits, dtype=np.float64)
-    if K >= logits.shape[1]:
-        return np.zeros(logits.shape[0], dtype=bool)
     s = -np.sort(-logits, axis=1)
-    return (s[:, K - 1] - s[:, K]) < gap
+    top = s[:, :min(K + 1, logits.shape[1])]
+    if top.shape[1] < 2:
+        return np.zeros(logits.shape[0], dtype=bool)
+    return np.min(top[:, :-1] - top[:, 1:], axis=1) < gap
 
 
 # ----------------------------------------------------------------------------

@@ -25,6 +25,36 @@ def cfg_of(wl, T=None):
                     identity=wl.identity)
 
 
+def quantize_dev(x: torch.Tensor, rows: int, cols: int, layout=L.SF_ROWMAJOR, global_in=None):
+    """lmoe_nvfp4_quantize on a device tensor: (codes, sf, global scale)."""
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    if layout == L.SF_MMA_TILED:
+        sf = torch.empty((((rows + 127) // 128) * 128 * ((cols + 63) // 64) * 4,), dtype=torch.uint8, device="cuda")
+    else:
+        sf = torch.empty((rows, cols // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = L.workspace(L.config(T=rows, d=cols, l=cols, N=1, K=1, m=cols), L.OP_NVFP4_QUANTIZE)
+    dt = L.BF16 if x.dtype == torch.bfloat16 else L.F32
+    L.nvfp4_quantize(x, dt, rows, cols, global_in, codes, sf, g, layout, ws)
+    st, info = L.read_device_error(ws)
+    assert st == L.OK, (st, info)
+    return codes, sf, g
+
+
+def quantize_experts_dev(w: torch.Tensor):
+    """Per-expert NVFP4 weights [N][rows][cols] with MMA-tiled scales."""
+    N, rows, cols = w.shape
+    codes = torch.empty((N, rows, cols // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((N, rows * cols // 16), dtype=torch.uint8, device="cuda")
+    gs = torch.empty(N, dtype=torch.float32, device="cuda")
+    for e in range(N):
+        c, f, g = quantize_dev(w[e], rows, cols, L.SF_MMA_TILED)
+        codes[e].copy_(c)
+        sf[e].copy_(f)
+        gs[e:e + 1].copy_(g)
+    return codes, sf, gs
+
+
 class DevLayer:
     """Device copies of one workload's inputs and the C-ABI weight struct."""
 
@@ -36,9 +66,16 @@ class DevLayer:
         self.t = {k: to_dev(inp[k], st) for k in ("w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
         self.bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).cuda()
         self.cfg = cfg_of(wl)
+        extra = {}
+        if wl.dtype == "nvfp4":
+            c1, f1, g1 = quantize_experts_dev(self.t["w1"])
+            c2, f2, g2 = quantize_experts_dev(self.t["w2"])
+            a_gs = torch.tensor([inp["a_global_scale"]], dtype=torch.float32, device="cuda")
+            self.t.update(w1=c1, w2=c2)
+            extra = dict(w1_sf=f1, w2_sf=f2, w1_gs=g1, w2_gs=g2, a_global_scale=a_gs)
         self.w = L.weights(w_router=self.t["w_router"], router_bias=self.bias, w_down=self.t["w_down"],
                            w_up=self.t["w_up"], w1=self.t["w1"], w2=self.t["w2"], ws1=self.t["ws1"],
-                           ws2=self.t["ws2"])
+                           ws2=self.t["ws2"], **extra)
 
     def forward(self):
         out = torch.empty((self.wl.T, self.wl.d), dtype=self.x.dtype, device="cuda")

@@ -37,6 +37,12 @@ def test_full_size_bf16(name):
     ridx, rgates = O.route_topk(logits, wl.K)
     near = O.near_tie_tokens(logits, wl.K)
     same = np.all(gidx == ridx, axis=1)
+    dl = np.abs(glogits.astype(np.float64) - logits)
+    srt = -np.sort(-logits, axis=1)
+    gaps = srt[:, :wl.K] - srt[:, 1:wl.K + 1]
+    bad = np.where(~same)[0]
+    print(f"{name}: logit error max {dl.max():.3e} mean {dl.mean():.3e}; misrouted {bad.size}; "
+          f"their min adjacent gap {[float(gaps[t].min()) for t in bad[:16]]}")
     assert np.all(same | near), f"{np.sum(~(same | near))} tokens routed differently without a near-tie"
     ok = same
     assert np.max(np.abs(gw[ok] - rgates[ok])) <= 1e-5

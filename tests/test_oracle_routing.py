@@ -80,9 +80,14 @@ def test_router_bias_shifts_selection():
 
 
 def test_near_tie_detection():
-    logits = np.array([[3.0, 2.0, 2.0 - 1e-6, 0.0], [3.0, 2.0, 1.0, 0.0]])
+    logits = np.array([[3.0, 2.0, 2.0 - 1e-6, 0.0],      # K-th vs (K+1)-th: set ambiguous
+                       [3.0, 2.0, 1.0, 0.0],             # clear
+                       [3.0, 3.0 - 1e-6, 1.0, 0.0],      # order of the two chosen ambiguous
+                       [3.0, 2.0, 1.0, 1.0 - 1e-7]])     # tie below the (K+1)-th: irrelevant
     flags = O.near_tie_tokens(logits, 2)
-    assert list(flags) == [True, False]
+    assert list(flags) == [True, False, True, False]
+    assert O.near_tie_tokens(np.array([[1.0, 1.0]]), 2)[0]    # K = N: only the order can tie
+    assert O.near_tie_tokens(np.array([[1.0, 1.0 - 1e-9]]), 1)[0]
 
 
 def _naive_permute(idx, N):
