@@ -252,7 +252,9 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
     if (st != LMOE_OK) return st;
     logits = lg;
   }
-  return launch_topk(logits, cfg->T, cfg->N, cfg->K, topk_idx, topk_w, err, s);
+  const bool computed = logits_in == nullptr;
+  return launch_topk(logits, cfg->T, cfg->N, cfg->K, topk_idx, topk_w, computed ? x : nullptr,
+                     computed ? w_router : nullptr, computed ? bias : nullptr, cfg->d, cfg->act, err, s);
 }
 
 lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets, int32_t* perm_src,
@@ -528,7 +530,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     st = dense_bf16(x, T, w->w_router, N, d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0, err, s);
   }
   if (st != LMOE_OK) return st;
-  if ((st = launch_topk(logits, T, N, K, idx, gw, err, s)) != LMOE_OK) return st;
+  if ((st = launch_topk(logits, T, N, K, idx, gw, x, w->w_router, w->router_bias, d, cfg->act, err, s)) != LMOE_OK)
+    return st;
   mark(1);
 
   // 2. latent down-projection d -> l

@@ -96,8 +96,9 @@ struct SimtLaunch {
 lmoe_status simt_gemm(const SimtLaunch& L, uint32_t* err_word, cudaStream_t stream);
 
 // ----- small kernels (lmoe_kernels.cu) -----
-lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w,
-                        uint32_t* err, cudaStream_t s);
+// x / w_router non-null: refine near-tied decisions with exact logits (see the kernel).
+lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w, const void* x,
+                        const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s);
 int permute_chunks(int64_t slots);
 lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,

@@ -14,32 +14,101 @@ namespace lmoe {
 // Top-K + renormalised softmax gates: one warp per token.
 // Selection order: logit descending, expert index ascending (ties to the
 // lower index). Gates: exp(l_k - l_max) / sum over the K chosen.
+//
+// Exact decisions from approximate logits: tensor-core logits carry fp32
+// accumulation error. When the kernel is given x and W_r, every adjacent pair
+// among the K+1 largest logits (and any further expert near the K-th) whose
+// gap is within 2*tau gets its logits recomputed exactly (products of the
+// stored operands summed in fp64), and the candidates are re-ranked. Experts
+// left approximate are more than 2*tau from every neighbour, so their order
+// is exact as long as the logit error is below tau. tau scales with the
+// token's bias-free logit RMS (the size of the GEMM's partial sums):
+// tau = 2^-10 * RMS + 2^-20 * max|logit|.
 // ===========================================================================
-template <int NPL>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T,
-                                                   int N, int K, int32_t* __restrict__ idx,
-                                                   float* __restrict__ w) {
+template <typename TA>
+__device__ __forceinline__ double exact_dot(const TA* __restrict__ x, const TA* __restrict__ w, int d, int lane) {
+  double acc = 0.0;
+  if constexpr (sizeof(TA) == 2) {
+    for (int j = lane * 8; j < d; j += 256) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + j));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(w + j));
+      const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa = __bfloat1622float2(ha[i]);
+        const float2 fb = __bfloat1622float2(hb[i]);
+        acc = fma(static_cast<double>(fa.x), static_cast<double>(fb.x), acc);
+        acc = fma(static_cast<double>(fa.y), static_cast<double>(fb.y), acc);
+      }
+    }
+  } else {
+    for (int j = lane * 4; j < d; j += 128) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(x + j));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(w + j));
+      acc = fma(static_cast<double>(a.x), static_cast<double>(b.x), acc);
+      acc = fma(static_cast<double>(a.y), static_cast<double>(b.y), acc);
+      acc = fma(static_cast<double>(a.z), static_cast<double>(b.z), acc);
+      acc = fma(static_cast<double>(a.w), static_cast<double>(b.w), acc);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  return acc;
+}
+
+// (value desc, index asc) ordering
+__device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+template <int NPL, typename TA>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T, int N, int K,
+                                                   int32_t* __restrict__ idx, float* __restrict__ w,
+                                                   const TA* __restrict__ x, const TA* __restrict__ wr,
+                                                   const float* __restrict__ bias, int d) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
+  const bool refine = x != nullptr;
   const float* row = logits + t * N;
   float v[NPL];
+  float sq = 0.0f, vmax_abs = 0.0f;
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
     const int col = lane + 32 * i;
     v[i] = col < N ? __ldg(row + col) : -INFINITY;
+    if (col < N) {
+      const float nb = v[i] - (bias ? __ldg(bias + col) : 0.0f);
+      sq = fmaf(nb, nb, sq);
+      vmax_abs = fmaxf(vmax_abs, fabsf(v[i]));
+    }
   }
+  float tau = 0.0f;
+  if (refine) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      vmax_abs = fmaxf(vmax_abs, __shfl_xor_sync(0xffffffffu, vmax_abs, off));
+    }
+    tau = ldexpf(sqrtf(sq / static_cast<float>(N)), -10) + ldexpf(vmax_abs, -20);
+  }
+  // extract candidates in (approximate) order: the K best, the (K+1)-th, and
+  // while refining, further experts within 2 tau of the K-th (at most 32)
   uint32_t taken = 0;
-  float my_sel = -INFINITY;  // lane k keeps the k-th selected logit
-  int my_idx = 0;
-  for (int k = 0; k < K; ++k) {
+  float my_v = -INFINITY;   // lane c holds candidate c
+  int my_i = 0x7fffffff;
+  int C = 0;
+  float kth = -INFINITY;
+  const int cmax = min(N, 32);
+  while (C < cmax) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int col = lane + 32 * i;
       const bool live = col < N && !((taken >> i) & 1u);
-      if (live && (v[i] > bv || (v[i] == bv && col < bi))) {
+      if (live && before(v[i], col, bv, bi)) {
         bv = v[i];
         bi = col;
       }
@@ -48,36 +117,74 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     for (int off = 16; off > 0; off >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (ov > bv || (ov == bv && oi < bi)) {
+      if (before(ov, oi, bv, bi)) {
         bv = ov;
         bi = oi;
       }
     }
+    if (C >= K && !(refine && bv >= kth - 2.0f * tau)) break;   // not a boundary candidate
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == k) {
-      my_sel = bv;
-      my_idx = bi;
+    if (lane == C) {
+      my_v = bv;
+      my_i = bi;
+    }
+    if (C == K - 1) kth = bv;
+    ++C;
+    if (!refine && C >= K) break;
+  }
+  if (refine) {
+    // mark candidates that have a neighbour within 2 tau; recompute them exactly
+    const float up = __shfl_up_sync(0xffffffffu, my_v, 1);
+    const float dn = __shfl_down_sync(0xffffffffu, my_v, 1);
+    const bool mark = lane < C && ((lane > 0 && up - my_v <= 2.0f * tau) || (lane + 1 < C && my_v - dn <= 2.0f * tau));
+    unsigned todo = __ballot_sync(0xffffffffu, mark);
+    const TA* xt = x + t * d;
+    while (todo) {
+      const int c = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int e = __shfl_sync(0xffffffffu, my_i, c);
+      double ex = exact_dot<TA>(xt, wr + static_cast<int64_t>(e) * d, d, lane);
+      if (bias) ex += static_cast<double>(__ldg(bias + e));
+      if (lane == c) my_v = static_cast<float>(ex);
     }
   }
-  const float lmax = __shfl_sync(0xffffffffu, my_sel, 0);
-  const float e = lane < K ? expf(my_sel - lmax) : 0.0f;
+  // rank of each candidate among the C
+  int rank = 0;
+  for (int c = 0; c < C; ++c) {
+    const float ov = __shfl_sync(0xffffffffu, my_v, c);
+    const int oi = __shfl_sync(0xffffffffu, my_i, c);
+    if (lane < C && c != lane && before(ov, oi, my_v, my_i)) ++rank;
+  }
+  const bool chosen = lane < C && rank < K;
+  // the largest logit is rank 0
+  const unsigned top_mask = __ballot_sync(0xffffffffu, lane < C && rank == 0);
+  const float lmax = __shfl_sync(0xffffffffu, my_v, __ffs(top_mask) - 1);
+  const float e = chosen ? expf(my_v - lmax) : 0.0f;
   float sum = e;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-  if (lane < K) {
-    idx[t * K + lane] = my_idx;
-    w[t * K + lane] = __fdiv_rn(e, sum);
+  if (chosen) {
+    idx[t * K + rank] = my_i;
+    w[t * K + rank] = __fdiv_rn(e, sum);
   }
 }
 
-lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w,
-                        uint32_t* err, cudaStream_t s) {
+lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w, const void* x,
+                        const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s) {
   (void)err;
   if (T == 0) return LMOE_OK;
   const int blocks = static_cast<int>((T * 32 + 255) / 256);
   const int npl = (N + 31) / 32;
-#define LMOE_TOPK(NPLV) \
-  topk_kernel<NPLV><<<blocks, 256, 0, s>>>(logits, T, N, K, idx, w)
+#define LMOE_TOPK(NPLV)                                                                                    \
+  do {                                                                                                    \
+    if (act == LMOE_F32)                                                                                  \
+      topk_kernel<NPLV, float><<<blocks, 256, 0, s>>>(logits, T, N, K, idx, w, static_cast<const float*>(x), \
+                                                      static_cast<const float*>(w_router), bias, d);      \
+    else                                                                                                  \
+      topk_kernel<NPLV, __nv_bfloat16><<<blocks, 256, 0, s>>>(                                            \
+          logits, T, N, K, idx, w, static_cast<const __nv_bfloat16*>(x),                                  \
+          static_cast<const __nv_bfloat16*>(w_router), bias, d);                                          \
+  } while (0)
   if (npl <= 1) LMOE_TOPK(1);
   else if (npl <= 2) LMOE_TOPK(2);
   else if (npl <= 4) LMOE_TOPK(4);

@@ -1,0 +1,86 @@
+"""GPU parity of lmoe_expert_ffn alone: the oracle's latent rows z, routing and
+gates go in (z quantised by the bit-exact NVFP4 quantiser for NVFP4 experts,
+rows permuted by the bit-exact permutation), and the gate-weighted expert
+outputs y are compared row by row with the oracle's y.
+
+Tolerance: max|err| beyond half a BF16 step <= 2e-2 * RMS(y) for BF16
+experts, 8e-2 * RMS(y) for NVFP4 experts.
+"""
+import numpy as np
+import pytest
+import torch
+
+import lmoe_inputs as LI
+from oracle import lmoe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+L = pytest.importorskip("latentmoe_fwd_b200")
+from gpu_util import DevLayer, bf16_parity, quantize_dev  # noqa: E402
+
+
+def _run_expert_ffn(wl, inp):
+    ref = O.forward(wl, inp)
+    dev = DevLayer(wl, inp)
+    cfg = dev.cfg
+    T, K, N, l = wl.T, wl.K, wl.N, wl.l
+    P = L.padded_rows(cfg)
+    z_bits = LI.bf16_bits(ref["z"] if wl.dtype != "nvfp4" else O.round_bf16(
+        O.from_bf16_bits(inp["x"]) @ O.from_bf16_bits(inp["w_down"]).T))
+    z = torch.from_numpy(z_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    idx = torch.from_numpy(ref["idx"]).cuda()
+    gates = torch.from_numpy(ref["gates"].astype(np.float32)).cuda()
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device="cuda")
+    offsets, poff, perm_src, inv_perm = i32(N + 1), i32(N + 1), i32(T * K), i32(T * K)
+    pgate = torch.zeros(P, dtype=torch.float32, device="cuda")
+    ws = L.workspace(cfg, L.OP_PERMUTE)
+    extra = {}
+    if wl.dtype == "nvfp4":
+        codes, sf, zgs = quantize_dev(z, T, l)
+        zp = torch.zeros((P, l // 2), dtype=torch.uint8, device="cuda")
+        zp_sf = torch.zeros(P * l // 16, dtype=torch.uint8, device="cuda")
+        L.permute(cfg, idx, offsets, perm_src, inv_perm, poff, codes, l // 2, zp, sf, zp_sf, gates, pgate, ws=ws)
+        extra = dict(permuted_sf=zp_sf, in_global_scale=zgs)
+    else:
+        zp = torch.zeros((P, l), dtype=torch.bfloat16, device="cuda")
+        L.permute(cfg, idx, offsets, perm_src, inv_perm, poff, z, l * 2, zp, topk_w=gates, perm_gate=pgate, ws=ws)
+    assert L.read_device_error(ws)[0] == L.OK
+    y = torch.zeros((P, l), dtype=torch.bfloat16, device="cuda")
+    ews = L.workspace(cfg, L.OP_EXPERT_FFN)
+    L.expert_ffn(cfg, dev.w, zp, extra.get("permuted_sf"), extra.get("in_global_scale"), offsets, poff, pgate, y,
+                 ews)
+    st, info = L.read_device_error(ews)
+    assert st == L.OK, (L.status_string(st), hex(info))
+    # padded row of every sorted position
+    off = offsets.cpu().numpy()
+    pof = poff.cpu().numpy()
+    flat = ref["idx"].reshape(-1)
+    src = ref["perm_src"]
+    prow = np.arange(T * K) - off[flat[src]] + pof[flat[src]]
+    got = y.float().cpu().numpy().astype(np.float64)[prow]
+    return got, ref, flat[src]
+
+
+def _check(wl, tol):
+    inp = LI.make_inputs(wl)
+    got, ref, expert_of_row = _run_expert_ffn(wl, inp)
+    want = ref["y"]
+    exact = want  # y is a rounding point of the oracle: compare against it with the half-step allowance
+    excess, raw = bf16_parity(got, exact, want)
+    rms = np.sqrt(np.mean(want ** 2))
+    row_err = np.max(np.abs(got - want), axis=1) / rms
+    bad = np.where(row_err > tol)[0]
+    print(f"{wl.name} T={wl.T}: y excess {excess:.3e} raw {raw:.3e} * RMS; rows over tol {bad.size}; "
+          f"experts of bad rows {sorted(set(expert_of_row[bad].tolist()))[:20]}; "
+          f"first bad rows {bad[:10].tolist()}")
+    assert excess <= tol
+
+
+@pytest.mark.parametrize("T", [130, 700])
+def test_expert_ffn_nvfp4(T):
+    _check(LI.reduced("ultra_nvfp4", T=T, d=512, l=256, N=16, K=4, m=512), 8e-2)
+
+
+@pytest.mark.parametrize("T", [20, 300])
+def test_expert_ffn_bf16(T):
+    _check(LI.reduced("ultra_decode", T=T, d=512, l=256, N=16, K=4, m=384), 2e-2)
