@@ -171,6 +171,29 @@ lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_
                          const uint8_t* rows_sf, uint8_t* permuted_sf, const float* topk_w,
                          float* perm_gate, void* ws, size_t ws_bytes, void* stream);
 
+/* lmoe_permute without a workspace: the same permutation, offsets, padded
+ * offsets and optional row/scale/gate gathers, bit for bit, for callers that
+ * cannot allocate device memory -- e.g. a plugin that an inference runtime
+ * hands only its input and output buffers, or a latency-critical loop that
+ * must not call cudaMalloc (an allocation can synchronise the device).
+ * The pages have no counterpart to this entry point; it is a deployment aid.
+ *  - Scratch: a fixed 512 KiB array in device memory defined by the library
+ *    (every GPU that loads the library holds it until the process exits).
+ *    It holds (ceil(T*K / 8192) + 1) * N counters at most 131072, e.g.
+ *    T*K up to about 2 million slots with N = 512; larger problems return
+ *    LMOE_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array: calls that overlap on the GPU (two
+ *    streams, or two host threads) race and must be serialised by the caller.
+ *  - There is no error word: an out-of-range expert index is skipped without
+ *    a report (lmoe_permute reports it). Allocates nothing. */
+lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets,
+                                 int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
+                                 const void* rows, int64_t row_bytes, void* permuted_rows,
+                                 const uint8_t* rows_sf, uint8_t* permuted_sf, const float* topk_w,
+                                 float* perm_gate, void* stream);
+
 /* Routed expert FFNs on the padded expert-grouped rows:
  *  y = g * (relu(z_e W1_e^T)^2 W2_e^T) for the rows of each expert e.
  *  permuted_in [padded][l]: `act` rows, or for expert == NVFP4 packed E2M1

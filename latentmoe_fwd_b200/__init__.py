@@ -28,7 +28,7 @@ OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE =
 EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permute",
            "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
-           "lmoe_forward_traced")
+           "lmoe_forward_traced", "lmoe_permute_noalloc")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -65,6 +65,7 @@ def _load():
         "lmoe_padded_rows": (I64, [C]),
         "lmoe_route": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
         "lmoe_permute": (ctypes.c_int, [C, P, P, P, P, P, P, I64, P, P, P, P, P, P, ctypes.c_size_t, P]),
+        "lmoe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, I64, P, P, P, P, P, P]),
         "lmoe_expert_ffn": (ctypes.c_int, [C, W, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
         "lmoe_combine": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "lmoe_forward": (ctypes.c_int, [C, W, P, P, P, ctypes.c_size_t, P]),
@@ -158,6 +159,17 @@ def permute(cfg, topk_idx, offsets, perm_src, inv_perm, padded_offsets, rows=Non
                             _p(padded_offsets), _p(rows), int(row_bytes), _p(permuted_rows), _p(rows_sf),
                             _p(permuted_sf), _p(topk_w), _p(perm_gate), _p(ws), ws.numel(),
                             _stream(stream)), "lmoe_permute")
+
+
+def permute_noalloc(cfg, topk_idx, offsets, perm_src, inv_perm, padded_offsets, rows=None, row_bytes=0,
+                    permuted_rows=None, rows_sf=None, permuted_sf=None, topk_w=None, perm_gate=None,
+                    stream=None):
+    """lmoe_permute without a workspace (the library's fixed scratch array is
+    used instead), for callers that may not allocate device memory."""
+    _check(lib.lmoe_permute_noalloc(ctypes.byref(cfg), _p(topk_idx), _p(offsets), _p(perm_src), _p(inv_perm),
+                                    _p(padded_offsets), _p(rows), int(row_bytes), _p(permuted_rows),
+                                    _p(rows_sf), _p(permuted_sf), _p(topk_w), _p(perm_gate), _stream(stream)),
+           "lmoe_permute_noalloc")
 
 
 def expert_ffn(cfg, w: Weights, permuted_in, permuted_sf, in_global_scale, offsets, padded_offsets,

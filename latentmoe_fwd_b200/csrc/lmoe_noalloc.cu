@@ -1,0 +1,75 @@
+// lmoe_permute_noalloc: the expert-grouped permutation without a caller
+// workspace. Its scratch (the per-chunk expert count table of the counting
+// sort) lives in a fixed array in device memory that the library defines, so
+// the call needs no allocation at all -- for callers that are handed their
+// input and output buffers but may not allocate device memory themselves.
+#include <mutex>
+
+#include "lmoe_internal.h"
+
+namespace lmoe {
+namespace {
+
+// Scratch of the counting sort: (chunks + 1) * N int32 counters, chunks =
+// ceil(T*K / 8192). 128 Ki entries = 512 KiB, held by every GPU that loads
+// the library until the process exits.
+constexpr int64_t kStaticScratchEntries = 128 * 1024;
+static __device__ __align__(256) int32_t g_permute_scratch[kStaticScratchEntries];
+
+// Device address of the array, looked up once per device (host code cannot
+// use the symbol itself as a device pointer).
+constexpr int kMaxDevices = 64;
+int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+std::mutex g_scratch_mutex;
+
+lmoe_status static_scratch(int32_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LMOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return LMOE_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return LMOE_OK;
+}
+
+}  // namespace
+}  // namespace lmoe
+
+extern "C" lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets,
+                                            int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
+                                            const void* rows, int64_t row_bytes, void* permuted_rows,
+                                            const uint8_t* rows_sf, uint8_t* permuted_sf, const float* topk_w,
+                                            float* perm_gate, void* stream) {
+  using namespace lmoe;
+  if (!cfg || !topk_idx || !offsets || !perm_src || !inv_perm || !padded_offsets) return LMOE_ERR_INVALID_ARG;
+  if (cfg->T < 0 || cfg->N <= 0 || cfg->K <= 0 || cfg->K > cfg->N) return LMOE_ERR_INVALID_ARG;
+  if (cfg->N > 1024 || cfg->K > 32) return LMOE_ERR_UNSUPPORTED;
+  if ((rows == nullptr) != (permuted_rows == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if (rows && (row_bytes <= 0 || row_bytes % 16 || (reinterpret_cast<uintptr_t>(rows) & 15) ||
+               (reinterpret_cast<uintptr_t>(permuted_rows) & 15)))
+    return LMOE_ERR_INVALID_ARG;
+  if ((rows_sf == nullptr) != (permuted_sf == nullptr)) return LMOE_ERR_INVALID_ARG;
+  if (rows_sf && (!rows || (row_bytes * 2) % 64)) return LMOE_ERR_INVALID_ARG;
+  if ((topk_w == nullptr) != (perm_gate == nullptr)) return LMOE_ERR_INVALID_ARG;
+  const int64_t slots = cfg->T * cfg->K;
+  const int64_t need = static_cast<int64_t>(permute_chunks(slots) + 1) * cfg->N;
+  if (need > kStaticScratchEntries) return LMOE_ERR_WORKSPACE;   // beyond the fixed scratch
+  int32_t* scratch = nullptr;
+  lmoe_status st = static_scratch(&scratch);
+  if (st != LMOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // No error word: an out-of-range expert index is skipped without a report.
+  st = launch_permute(topk_idx, cfg->T, cfg->K, cfg->N, offsets, perm_src, inv_perm, padded_offsets, scratch,
+                      topk_w, perm_gate, nullptr, s);
+  if (st != LMOE_OK) return st;
+  if (rows || rows_sf) {
+    const int64_t nonempty = slots < cfg->N ? slots : cfg->N;
+    const int64_t padded = (slots + 127 * nonempty + 127) / 128 * 128;
+    st = launch_gather(topk_idx, perm_src, offsets, padded_offsets, slots, cfg->K, rows, row_bytes, permuted_rows,
+                       rows_sf, permuted_sf, padded, s);
+  }
+  return st;
+}
