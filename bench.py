@@ -142,6 +142,23 @@ def traffic_record(workload: str):
     return entry.get("traffic_bytes_per_forward")
 
 
+def quantize_experts(L, w):
+    """NVFP4 copies of expert weights [N][rows][cols] through lmoe_nvfp4_quantize:
+    packed codes, MMA-tiled block scales and one global scale per expert matrix."""
+    import torch
+    N, rows, cols = w.shape
+    codes = torch.empty((N, rows, cols // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((N, rows * cols // 16), dtype=torch.uint8, device="cuda")
+    gs = torch.empty(N, dtype=torch.float32, device="cuda")
+    ws = L.workspace(L.config(T=rows, d=cols, l=cols, N=1, K=1, m=cols), L.OP_NVFP4_QUANTIZE)
+    for e in range(N):
+        L.nvfp4_quantize(w[e], L.BF16, rows, cols, None, codes[e], sf[e], gs[e:e + 1], L.SF_MMA_TILED, ws)
+    st, info = L.read_device_error(ws)
+    if st != L.OK:
+        raise RuntimeError(f"weight quantisation failed: {L.status_string(st)}")
+    return codes, sf, gs
+
+
 # --------------------------------------------------------------------------
 # the CPU oracle, timed (bounded sample)
 # --------------------------------------------------------------------------
@@ -213,8 +230,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample", type=int, default=None, help="oracle tokens for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (smaller captures for ncu)")
     args = ap.parse_args()
     wl = LI.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        wl = LI.replace(wl, T=args.tokens)
     if args.impl == "reference":
         return run_reference(args, wl)
 
@@ -258,8 +279,17 @@ def main():
     cfg = L.config(T=wl.T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m, n_shared=wl.n_shared, m_shared=wl.m_shared,
                    act=L.F32 if st == "f32" else L.BF16,
                    expert={"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype], identity=wl.identity)
+    extra = {}
+    if wl.dtype == "nvfp4":
+        # setup, not timed: NVFP4 expert weights (per-matrix global scale, MMA-tiled block scales)
+        for key in ("w1", "w2"):
+            codes, sf, gs = quantize_experts(L, t[key])
+            t[key] = codes
+            extra[key + "_sf"], extra[key + "_gs"] = sf, gs
+        extra["a_global_scale"] = torch.tensor([inp["a_global_scale"]], dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
     w = L.weights(w_router=t["w_router"], router_bias=bias, w_down=t["w_down"], w_up=t["w_up"], w1=t["w1"],
-                  w2=t["w2"], ws1=t["ws1"], ws2=t["ws2"])
+                  w2=t["w2"], ws1=t["ws1"], ws2=t["ws2"], **extra)
     ws = L.workspace(cfg, L.OP_FORWARD)
     stream = torch.cuda.current_stream()
 

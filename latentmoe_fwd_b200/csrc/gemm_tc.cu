@@ -70,6 +70,7 @@ static lmoe_status dispatch_epi(int epi, const CUtensorMap& a0, const CUtensorMa
     case EPI_SQRELU: return launch_tc<BN, STAGES, EPI_SQRELU>(a0, b0, a1, b1, p, grid, s);
     case EPI_GATE: return launch_tc<BN, STAGES, EPI_GATE>(a0, b0, a1, b1, p, grid, s);
     case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(a0, b0, a1, b1, p, grid, s);
+    case EPI_PARTIAL: return launch_tc<BN, STAGES, EPI_PARTIAL>(a0, b0, a1, b1, p, grid, s);
   }
   return LMOE_ERR_INVALID_ARG;
 }
@@ -107,18 +108,37 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   p.row_scale = L.row_scale;
   p.residual = static_cast<const __nv_bfloat16*>(L.residual);
   p.ld_res = L.ld_res;
+  p.ksplit = L.ksplit > 1 ? L.ksplit : 1;
+  p.partial = L.partial;
   p.err = DevErr{err_word};
+  if (p.ksplit > 1 && (L.grouped || !L.partial)) return LMOE_ERR_INVALID_ARG;
   const int sms = device_sm_count();
-  int64_t grid = L.max_tiles < sms ? L.max_tiles : sms;
+  const int64_t tiles = L.max_tiles * p.ksplit;
+  int64_t grid = tiles < sms ? tiles : sms;
   if (grid <= 0) return LMOE_OK;
   const int g = static_cast<int>(grid);
+  const int epi = p.ksplit > 1 ? static_cast<int>(EPI_PARTIAL) : L.epi;
+  lmoe_status st = LMOE_ERR_INVALID_ARG;
   switch (bn) {
-    case 256: return dispatch_epi<256, 4>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
-    case 128: return dispatch_epi<128, 6>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
-    case 64: return dispatch_epi<64, 8>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
-    case 32: return dispatch_epi<32, 10>(L.epi, maps[0], maps[1], maps[2], maps[3], p, g, stream);
+    case 256: st = dispatch_epi<256, 4>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
+    case 128: st = dispatch_epi<128, 6>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
+    case 64: st = dispatch_epi<64, 8>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
+    case 32: st = dispatch_epi<32, 10>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
   }
-  return LMOE_ERR_INVALID_ARG;
+  if (st != LMOE_OK || p.ksplit == 1) return st;
+  // deterministic reduction of the partial sums (fixed split order) + the real epilogue
+  const int64_t n = static_cast<int64_t>(L.rows) * L.cols;
+  int rblocks = static_cast<int>((n + 255) / 256);
+  if (rblocks > sms * 8) rblocks = sms * 8;
+  switch (L.epi) {
+    case EPI_F32_BIAS: splitk_reduce_kernel<EPI_F32_BIAS><<<rblocks, 256, 0, stream>>>(p); break;
+    case EPI_BF16: splitk_reduce_kernel<EPI_BF16><<<rblocks, 256, 0, stream>>>(p); break;
+    case EPI_SQRELU: splitk_reduce_kernel<EPI_SQRELU><<<rblocks, 256, 0, stream>>>(p); break;
+    case EPI_ADD_RES: splitk_reduce_kernel<EPI_ADD_RES><<<rblocks, 256, 0, stream>>>(p); break;
+    default: return LMOE_ERR_INVALID_ARG;
+  }
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
 }  // namespace lmoe

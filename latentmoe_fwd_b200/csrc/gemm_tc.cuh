@@ -32,7 +32,8 @@ enum EpiKind : int {
   EPI_BF16 = 1,       // out bf16 = acc
   EPI_SQRELU = 2,     // out bf16 = relu(acc)^2
   EPI_GATE = 3,       // out bf16 = acc * row_scale[row]
-  EPI_ADD_RES = 4     // out bf16 = acc + residual[row][col]
+  EPI_ADD_RES = 4,    // out bf16 = acc + residual[row][col]
+  EPI_PARTIAL = 5     // split-K: fp32 partial sums, the epilogue runs in the reduction
 };
 
 struct TcSeg {
@@ -57,6 +58,8 @@ struct TcParams {
   const float* row_scale;     // EPI_GATE: per activation row, or nullptr (= 1)
   const __nv_bfloat16* residual;
   long long ld_res;
+  int ksplit;                 // >1: split the K blocks of every tile; partial sums go to `partial`
+  float* partial;             // [ksplit][rows][cols] fp32 (split-K only)
   DevErr err;
 };
 
@@ -77,24 +80,37 @@ struct TileInfo {
   int act0;       // first activation row of the tile
   int act_n;      // valid activation rows (<= 128 normal, <= BN swap)
   int w0;         // first weight row (output feature) of the tile
+  int split;      // split-K index
+  int kb0, kb1;   // K blocks [kb0, kb1) of this tile
 };
 
 template <int BN>
 __device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
   const int ntw_normal = (p.cols + BN - 1) / BN;
   const int ntw_swap = (p.cols + 127) / 128;
+  int n;
   if (!p.swap) {
     int mt = p.grouped ? (__ldg(p.padded_offsets + p.groups) >> 7) : (p.rows + 127) / 128;
-    return mt * ntw_normal;
+    n = mt * ntw_normal;
+  } else {
+    n = p.grouped ? p.groups * ntw_swap : ntw_swap;
   }
-  return p.grouped ? p.groups * ntw_swap : ntw_swap;
+  return n * p.ksplit;
 }
 
 template <int BN>
-__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t) {
+__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t, int kb_total) {
   TileInfo ti;
   ti.valid = 1;
   ti.expert = 0;
+  ti.split = t % p.ksplit;
+  t /= p.ksplit;
+  {
+    const int per = (kb_total + p.ksplit - 1) / p.ksplit;
+    ti.kb0 = ti.split * per;
+    ti.kb1 = min(kb_total, ti.kb0 + per);
+    if (ti.kb0 >= ti.kb1) ti.valid = 0;
+  }
   if (!p.swap) {
     const int ntw = (p.cols + BN - 1) / BN;
     const int nt = t % ntw, mt = t / ntw;
@@ -201,9 +217,9 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t last_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tc_tile<BN>(p, t);
+        const TileInfo ti = tc_tile<BN>(p, t, kb_total);
         if (!ti.valid) continue;
-        for (int kb = 0; kb < kb_total; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x100 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStageBytes;
           uint8_t* sb = sa + S::kABytes;
@@ -249,14 +265,14 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       bool any = false;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tc_tile<BN>(p, t);
+        const TileInfo ti = tc_tile<BN>(p, t, kb_total);
         if (!ti.valid) continue;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, 0x200 + acc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kb_total; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x300 + stage)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
@@ -264,7 +280,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32), sdesc_kmajor_sw128(sb + kk * 32), idesc,
-                     (kb | kk) != 0 ? 1u : 0u);
+                     (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           }
           any = true;
           mma_commit(&empty[stage]);
@@ -286,7 +302,7 @@ __global__ void __launch_bounds__(192, 1)
     const int r = q * 32 + lane;     // accumulator row of this thread
     int local = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const TileInfo ti = tc_tile<BN>(p, t);
+      const TileInfo ti = tc_tile<BN>(p, t, kb_total);
       if (!ti.valid) continue;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -302,7 +318,14 @@ __global__ void __launch_bounds__(192, 1)
           const long long row = ti.act0 + r;
           if (r < ti.act_n) {
             const int col0 = ti.w0 + c * 32;
-            if (EPI == EPI_F32_BIAS) {
+            if (EPI == EPI_PARTIAL) {
+              float* o = p.partial + (static_cast<long long>(ti.split) * p.rows + row) * p.cols + col0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                if (col0 + j < p.cols)
+                  *reinterpret_cast<float4*>(o + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                                                   __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            } else if (EPI == EPI_F32_BIAS) {
               float* o = reinterpret_cast<float*>(p.out) + row * p.ld_out + col0;
 #pragma unroll
               for (int j = 0; j < 32; j += 4) {
@@ -344,6 +367,10 @@ __global__ void __launch_bounds__(192, 1)
               const int tok = c * 32 + j;
               if (tok < ti.act_n) {
                 const long long row = ti.act0 + tok;
+                if (EPI == EPI_PARTIAL) {
+                  p.partial[(static_cast<long long>(ti.split) * p.rows + row) * p.cols + col] = __uint_as_float(v[j]);
+                  continue;
+                }
                 const float val = epi_value<EPI>(__uint_as_float(v[j]), p, row, col);
                 if (EPI == EPI_F32_BIAS)
                   reinterpret_cast<float*>(p.out)[row * p.ld_out + col] = val;
@@ -367,6 +394,24 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+// Split-K reduction: out[row, col] = epi(sum over splits in order of partial[s][row][col]).
+template <int EPI>
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const TcParams p) {
+  const long long n = static_cast<long long>(p.rows) * p.cols;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float acc = 0.0f;
+    for (int sp = 0; sp < p.ksplit; ++sp) acc += p.partial[sp * n + i];
+    const long long row = i / p.cols;
+    const int col = static_cast<int>(i % p.cols);
+    const float val = epi_value<EPI>(acc, p, row, col);
+    if (EPI == EPI_F32_BIAS)
+      reinterpret_cast<float*>(p.out)[row * p.ld_out + col] = val;
+    else
+      reinterpret_cast<__nv_bfloat16*>(p.out)[row * p.ld_out + col] = __float2bfloat16_rn(val);
   }
 }
 

@@ -60,8 +60,27 @@ lmoe_status check_config(const lmoe_config* c) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// Weight-major (swap) tiles are used up to this many tokens.
+constexpr int64_t kSwapMaxTokens = 64;
+// Split-K of the weight-major dense GEMMs: at most this many splits.
+constexpr int kMaxSplits = 32;
+
+int64_t max_dense_cols(const lmoe_config* c, int op) {
+  int64_t m = c->N;
+  if (op == LMOE_OP_FORWARD) {
+    m = m > c->l ? m : c->l;
+    m = m > c->d ? m : c->d;
+    const int64_t sh = static_cast<int64_t>(c->n_shared) * c->m_shared;
+    m = m > sh ? m : sh;
+  }
+  return m;
+}
+
+int64_t splitk_floats(const lmoe_config* c, int op) { return c->T * max_dense_cols(c, op) * kMaxSplits; }
+
 // Workspace layout (byte offsets; region sizes 0 when unused).
 struct Layout {
+  size_t splitk = 0;        // fp32 split-K partial sums of the weight-major dense GEMMs (T <= 64)
   size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0,
          offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, scratch = 0, gate = 0, zp = 0,
          zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, total = 0;
@@ -80,6 +99,8 @@ Layout layout(const lmoe_config* c, int op) {
   const size_t ab = act_bytes(c);
   const bool fp4 = c->expert == LMOE_NVFP4;
   L.err = take(256);
+  if ((op == LMOE_OP_ROUTE || op == LMOE_OP_FORWARD) && T <= kSwapMaxTokens)
+    L.splitk = take(splitk_floats(c, op) * 4);
   if (op == LMOE_OP_ROUTE) {
     L.logits = take(T * N * 4);
   } else if (op == LMOE_OP_PERMUTE) {
@@ -138,9 +159,20 @@ int normal_bn(int cols) { return cols >= 256 ? 256 : cols > 64 ? 128 : cols > 32
 int kblocks(int64_t k) { return static_cast<int>((k + 63) / 64); }
 
 // out[rows, cols] = epi(x[rows, k] . W[cols, k]^T) with BF16 operands.
+// Splits for a weight-major GEMM with `tiles` output tiles and `kb` K blocks:
+// enough to fill the GPU, at least two K blocks per split, within the buffer.
+int choose_splits(int64_t tiles, int kb, int64_t rows, int64_t cols, float* partial) {
+  if (!partial) return 1;
+  const int sms = device_sm_count();
+  int sp = static_cast<int>((sms + tiles - 1) / tiles);
+  if (sp > kb / 2) sp = kb / 2;
+  if (sp > kMaxSplits) sp = kMaxSplits;
+  return sp > 1 ? sp : 1;
+}
+
 lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int64_t k, void* out,
                        int64_t ld_out, int epi, const float* bias, const void* residual, int64_t ld_res,
-                       uint32_t* err, cudaStream_t s) {
+                       float* partial, uint32_t* err, cudaStream_t s) {
   if (rows == 0) return LMOE_OK;
   TcLaunch L;
   const int sbn = swap_bn(rows);
@@ -155,6 +187,8 @@ lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int
     L.a[0] = wt;
     L.b[0] = act;
     L.max_tiles = (cols + 127) / 128;
+    L.ksplit = choose_splits(L.max_tiles, L.kblocks[0], rows, cols, partial);
+    L.partial = partial;
   } else {
     L.bn = normal_bn(cols);
     L.a[0] = act;
@@ -247,7 +281,8 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
       S.epi = EPI_F32_BIAS;
       st = simt_gemm(S, err, s);
     } else {
-      st = dense_bf16(x, cfg->T, w_router, cfg->N, cfg->d, lg, cfg->N, EPI_F32_BIAS, bias, nullptr, 0, err, s);
+      st = dense_bf16(x, cfg->T, w_router, cfg->N, cfg->d, lg, cfg->N, EPI_F32_BIAS, bias, nullptr, 0,
+                      L.splitk ? at<float>(ws, L.splitk) : nullptr, err, s);
     }
     if (st != LMOE_OK) return st;
     logits = lg;
@@ -509,6 +544,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   const int d = cfg->d, l = cfg->l, N = cfg->N, K = cfg->K;
   const size_t ab = act_bytes(cfg);
   const bool f32 = cfg->act == LMOE_F32;
+  float* splitk = L.splitk ? at<float>(ws, L.splitk) : nullptr;
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* gw = at<float>(ws, L.w);
   float* logits = at<float>(ws, L.logits);
@@ -527,7 +563,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     S.epi = EPI_F32_BIAS;
     st = simt_gemm(S, err, s);
   } else {
-    st = dense_bf16(x, T, w->w_router, N, d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0, err, s);
+    st = dense_bf16(x, T, w->w_router, N, d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0, splitk, err, s);
   }
   if (st != LMOE_OK) return st;
   if ((st = launch_topk(logits, T, N, K, idx, gw, x, w->w_router, w->router_bias, d, cfg->act, err, s)) != LMOE_OK)
@@ -550,7 +586,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
       S.epi = EPI_BF16;
       st = simt_gemm(S, err, s);
     } else {
-      st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, err, s);
+      st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s);
     }
     if (st != LMOE_OK) return st;
     z = zb;
@@ -625,7 +661,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
       st = simt_gemm(G, err, s);
     } else {
       st = dense_bf16(x, T, w->ws1, S * ms, d, hs, static_cast<int64_t>(S) * ms, EPI_SQRELU, nullptr, nullptr, 0,
-                      err, s);
+                      splitk, err, s);
     }
     if (st != LMOE_OK) return st;
   }
@@ -704,6 +740,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     U.swap = 1;
     U.bn = sbn;
     U.max_tiles = (d + 127) / 128;
+    U.ksplit = choose_splits(U.max_tiles, U.kblocks[0] + (U.nseg > 1 ? U.kblocks[1] : 0), T, d, splitk);
+    U.partial = splitk;
   } else {
     U.bn = normal_bn(d);
     U.max_tiles = ((T + 127) / 128) * ((d + U.bn - 1) / U.bn);

@@ -43,6 +43,8 @@ struct TcLaunch {
   int64_t ld_res = 0;
   int epi = 0;
   int bn = 256;
+  int ksplit = 1;                // >1: split-K with fp32 partials in `partial`, then a reduction
+  float* partial = nullptr;      // [ksplit][rows][cols]
 };
 
 lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream);
@@ -99,11 +101,15 @@ lmoe_status simt_gemm(const SimtLaunch& L, uint32_t* err_word, cudaStream_t stre
 // x / w_router non-null: refine near-tied decisions with exact logits (see the kernel).
 lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w, const void* x,
                         const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s);
-int permute_chunks(int64_t slots);
+// Slots per warp of the counting sort: the workspace path uses short chunks
+// (more CTAs in flight); the fixed-scratch path keeps 1024 (fewer counters).
+constexpr int kPermSlotsPerWarp = 128;
+constexpr int kPermSlotsPerWarpStatic = 1024;
+int permute_chunks(int64_t slots, int slots_per_warp = kPermSlotsPerWarp);
 lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
                            int32_t* scratch, const float* topk_w, float* perm_gate,
-                           uint32_t* err, cudaStream_t s);
+                           uint32_t* err, cudaStream_t s, int slots_per_warp = kPermSlotsPerWarp);
 lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int32_t* offsets,
                           const int32_t* padded_offsets, int64_t slots, int K, const void* rows,
                           int64_t row_bytes, void* out_rows, const uint8_t* rows_sf,

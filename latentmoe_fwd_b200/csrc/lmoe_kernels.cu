@@ -209,20 +209,23 @@ lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* i
 //                    the order across steps, so the sort is stable.
 // ===========================================================================
 constexpr int kPermWarps = 8;
-constexpr int kPermSlotsPerWarp = 1024;
-constexpr int kChunk = kPermWarps * kPermSlotsPerWarp;   // 8192 slots per CTA
 constexpr int kPad = 128;
 
-int permute_chunks(int64_t slots) { return static_cast<int>((slots + kChunk - 1) / kChunk); }
+// A chunk is kPermWarps * slots_per_warp consecutive slots, one CTA each.
+int permute_chunks(int64_t slots, int slots_per_warp) {
+  const int64_t chunk = static_cast<int64_t>(kPermWarps) * slots_per_warp;
+  return static_cast<int>((slots + chunk - 1) / chunk);
+}
 
 __global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx,
-                                                         int64_t slots, int N,
+                                                         int64_t slots, int N, int spw,
                                                          int32_t* __restrict__ cnt, DevErr err) {
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int64_t f0 = static_cast<int64_t>(blockIdx.x) * kChunk;
-  const int64_t f1 = min(slots, f0 + kChunk);
+  const int64_t chunk = static_cast<int64_t>(kPermWarps) * spw;
+  const int64_t f0 = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int64_t f1 = min(slots, f0 + chunk);
   for (int64_t f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
     const int e = __ldg(idx + f);
     if (e < 0 || e >= N) {
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
 }
 
 __global__ void __launch_bounds__(256) perm_scatter_kernel(
-    const int32_t* __restrict__ idx, int64_t slots, int N, const int32_t* __restrict__ base,
+    const int32_t* __restrict__ idx, int64_t slots, int N, int spw, const int32_t* __restrict__ base,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff,
     int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm,
     const float* __restrict__ topk_w, float* __restrict__ perm_gate) {
@@ -312,8 +315,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kPermWarps * N; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
-  const int64_t f0 = static_cast<int64_t>(blockIdx.x) * kChunk + static_cast<int64_t>(wid) * kPermSlotsPerWarp;
-  const int64_t f1 = min(slots, f0 + kPermSlotsPerWarp);
+  const int64_t f0 = (static_cast<int64_t>(blockIdx.x) * kPermWarps + wid) * spw;
+  const int64_t f1 = min(slots, f0 + spw);
   int32_t* my = wcnt + wid * N;
   const unsigned lt = (1u << lane) - 1u;
   // per-warp counts
@@ -367,21 +370,22 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
 lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
                            int32_t* scratch, const float* topk_w, float* perm_gate,
-                           uint32_t* err, cudaStream_t s) {
+                           uint32_t* err, cudaStream_t s, int slots_per_warp) {
   if (N > 1024) return LMOE_ERR_UNSUPPORTED;
+  if (slots_per_warp <= 0 || slots_per_warp % 32) return LMOE_ERR_INVALID_ARG;
   const int64_t slots = T * K;
-  const int nch = permute_chunks(slots);
+  const int nch = permute_chunks(slots, slots_per_warp);
   DevErr de{err};
   if (nch > 0) {
-    perm_count_kernel<<<nch, 256, N * sizeof(int32_t), s>>>(idx, slots, N, scratch, de);
+    perm_count_kernel<<<nch, 256, N * sizeof(int32_t), s>>>(idx, slots, N, slots_per_warp, scratch, de);
     count_launch();
   }
   perm_scan_kernel<<<1, 1024, 0, s>>>(scratch, nch, N, offsets, padded_offsets);
   count_launch();
   if (nch > 0) {
     const size_t sm = static_cast<size_t>(kPermWarps) * N * sizeof(int32_t);
-    perm_scatter_kernel<<<nch, 256, sm, s>>>(idx, slots, N, scratch, offsets, padded_offsets, perm_src,
-                                            inv_perm, topk_w, perm_gate);
+    perm_scatter_kernel<<<nch, 256, sm, s>>>(idx, slots, N, slots_per_warp, scratch, offsets, padded_offsets,
+                                            perm_src, inv_perm, topk_w, perm_gate);
     count_launch();
   }
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;

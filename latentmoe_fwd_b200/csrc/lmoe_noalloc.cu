@@ -55,7 +55,7 @@ extern "C" lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_
   if (rows_sf && (!rows || (row_bytes * 2) % 64)) return LMOE_ERR_INVALID_ARG;
   if ((topk_w == nullptr) != (perm_gate == nullptr)) return LMOE_ERR_INVALID_ARG;
   const int64_t slots = cfg->T * cfg->K;
-  const int64_t need = static_cast<int64_t>(permute_chunks(slots) + 1) * cfg->N;
+  const int64_t need = static_cast<int64_t>(permute_chunks(slots, kPermSlotsPerWarpStatic) + 1) * cfg->N;
   if (need > kStaticScratchEntries) return LMOE_ERR_WORKSPACE;   // beyond the fixed scratch
   int32_t* scratch = nullptr;
   lmoe_status st = static_scratch(&scratch);
@@ -63,7 +63,7 @@ extern "C" lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // No error word: an out-of-range expert index is skipped without a report.
   st = launch_permute(topk_idx, cfg->T, cfg->K, cfg->N, offsets, perm_src, inv_perm, padded_offsets, scratch,
-                      topk_w, perm_gate, nullptr, s);
+                      topk_w, perm_gate, nullptr, s, kPermSlotsPerWarpStatic);
   if (st != LMOE_OK) return st;
   if (rows || rows_sf) {
     const int64_t nonempty = slots < cfg->N ? slots : cfg->N;

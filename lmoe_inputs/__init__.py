@@ -39,7 +39,7 @@ from dataclasses import dataclass, replace, asdict
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "bf16_bits", "reduced"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "bf16_bits", "reduced", "replace"]
 
 
 @dataclass(frozen=True)

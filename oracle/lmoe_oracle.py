@@ -292,6 +292,12 @@ def sq_relu(h):
     return np.square(np.maximum(h, 0.0))
 
 
+def weights_view(wl, inp, cache: bool = False) -> _Weights:
+    """The weights object ``forward`` uses; pass one with cache=True to several
+    calls on the same inputs to quantise each NVFP4 expert matrix once."""
+    return _Weights(wl, inp, cache)
+
+
 def quantize_expert_weights(w_bf16_f64: np.ndarray):
     """NVFP4 codes, scales and per-matrix global scale of each expert matrix
     [N, rows, cols] (blocks along the contraction dim, i.e. along cols)."""
@@ -302,26 +308,32 @@ def quantize_expert_weights(w_bf16_f64: np.ndarray):
 
 
 class _Weights:
-    """fp64 views of the stored weights, converted expert by expert on demand."""
+    """fp64 views of the stored weights, converted expert by expert on demand.
+    With cache=True the NVFP4 quantisation of each expert matrix (codes,
+    scales, global scale) is kept, so repeated calls only dequantise."""
 
-    def __init__(self, wl, inp):
+    def __init__(self, wl, inp, cache: bool = False):
         self.wl = wl
         self.inp = inp
         self.st = "f32" if wl.dtype == "f32" else "bf16"
+        self._q = {} if cache else None
 
     def dense(self, key):
         return to_f64(self.inp[key], self.st)
 
     def expert(self, key, e):
         """fp64 values of expert e's matrix as the GEMM sees them."""
-        w = to_f64(self.inp[key][e], self.st)
         if self.wl.dtype == "nvfp4":
-            return nvfp4_fake_quant(w)[0]
-        return w
+            if self._q is not None:
+                if (key, e) not in self._q:
+                    self._q[(key, e)] = nvfp4_quantize(to_f64(self.inp[key][e], self.st))
+                return nvfp4_dequantize(*self._q[(key, e)])
+            return nvfp4_fake_quant(to_f64(self.inp[key][e], self.st))[0]
+        return to_f64(self.inp[key][e], self.st)
 
 
 def forward(wl, inp, tokens=None, idx_override=None, precision: str | None = None,
-            weights: _Weights | None = None) -> dict:
+            weights: _Weights | None = None, z_rows=None) -> dict:
     """One LatentMoE layer forward.
 
     wl: a ``lmoe_inputs.Workload``; inp: ``lmoe_inputs.make_inputs(wl)``.
@@ -330,6 +342,10 @@ def forward(wl, inp, tokens=None, idx_override=None, precision: str | None = Non
       global scale of z is still taken over all T tokens.
     idx_override: optional [len(tokens), K] expert choice (e.g. the GPU's
       choice on documented near-ties); the gates follow the override.
+    z_rows: NVFP4 only, optional [len(tokens), l] BF16-valued latent rows to
+      quantise instead of the rounded down-projection (an alternative rounding
+      of a documented rounding near-tie); the global scale stays the one of
+      the full z.
     precision: "f64" (no rounding points), else the workload's own
       ("f32" | "bf16" | "nvfp4").
 
@@ -366,7 +382,8 @@ def forward(wl, inp, tokens=None, idx_override=None, precision: str | None = Non
         if prec == "nvfp4":
             z_full = round_bf16(x_all @ w_down.T)
             zq_scale = nvfp4_global_scale(z_full)
-            z = nvfp4_fake_quant(z_full[tok], zq_scale)[0]
+            zsel = z_full[tok] if z_rows is None else np.asarray(z_rows, dtype=np.float64)
+            z = nvfp4_fake_quant(zsel, zq_scale)[0]
         else:
             z = rho(x @ w_down.T, prec)
             zq_scale = None

@@ -75,3 +75,34 @@ def test_full_size_bf16(name):
     excess, raw = bf16_parity(out[toks], ref["out_unrounded"], ref["out"])
     print(f"{name}: sampled {len(toks)} tokens: excess {excess:.3e} * RMS, raw {raw:.3e} * RMS")
     assert excess <= 2e-2
+
+
+def test_full_size_nvfp4():
+    """NVFP4 workload at full size: weights quantised on the GPU (bit-exact per
+    expert against the oracle for a sample of experts), routing checked over
+    every token, outputs of sampled tokens within 8e-2 * RMS beyond half a BF16
+    step, allowing the documented z-rounding near-ties."""
+    from test_gpu_nvfp4 import _tiled_to_rowmajor, nvfp4_token_errors
+    wl = LI.WORKLOADS["ultra_nvfp4"]
+    inp = LI.make_inputs(wl)
+    dev = DevLayer(wl, inp)
+    for e in (0, 257, 511):
+        rc, rsf, rg = O.nvfp4_quantize(O.from_bf16_bits(inp["w1"][e]))
+        assert np.array_equal(dev.t["w1"][e].cpu().numpy(), rc)
+        assert np.array_equal(_tiled_to_rowmajor(dev.w._keep["w1_sf"][e].cpu().numpy(), wl.m, wl.l), rsf)
+        assert dev.w._keep["w1_gs"][e].item() == np.float32(rg)
+    out = as_f64(dev.forward())
+    gidx, _, glogits = dev.route()
+    x = O.from_bf16_bits(inp["x"])
+    logits = O.router_logits(x, O.from_bf16_bits(inp["w_router"]), None)
+    ridx, _ = O.route_topk(logits, wl.K)
+    near = O.near_tie_tokens(logits, wl.K)
+    same = np.all(gidx == ridx, axis=1)
+    print(f"ultra_nvfp4: {np.sum(near)} near-tie tokens, {np.sum(~same)} routed differently")
+    assert np.all(same | near)
+    rng = np.random.default_rng(321)
+    toks = np.sort(rng.choice(wl.T, size=12, replace=False))
+    err, n_tied, n_var = nvfp4_token_errors(wl, inp, out, gidx, toks, 8e-2)
+    print(f"ultra_nvfp4: sampled {len(toks)} tokens: max|err| beyond BF16 half-step {err.max():.3e} * RMS; "
+          f"{n_tied} re-checked against {n_var} variants")
+    assert err.max() <= 8e-2

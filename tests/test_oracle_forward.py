@@ -255,3 +255,21 @@ def test_correctly_rounded_bf16_output_can_exceed_two_percent_of_rms():
     _, e = np.frexp(np.abs(r["out"]))
     half_step = np.ldexp(1.0, np.maximum(e - 1, -126) - 7) / 2
     assert np.all(np.abs(O.round_bf16(r["out_unrounded"]) - r["out_unrounded"]) <= half_step)
+
+
+def test_nvfp4_z_rows_override_and_weight_cache_are_transparent():
+    wl = _tiny(dtype="nvfp4", T=6, d=64, l=32, m=48, outliers=True)
+    inp = LI.make_inputs(wl)
+    base = O.forward(wl, inp)
+    x = O.from_bf16_bits(inp["x"])
+    z_full = O.round_bf16(x @ O.from_bf16_bits(inp["w_down"]).T)
+    W = O.weights_view(wl, inp, cache=True)
+    same = O.forward(wl, inp, tokens=[1, 4], z_rows=z_full[[1, 4]], weights=W)
+    assert np.array_equal(same["out"], base["out"][[1, 4]])
+    again = O.forward(wl, inp, tokens=[1, 4], weights=W)      # cached quantised experts
+    assert np.array_equal(again["out"], base["out"][[1, 4]])
+    # a different z row changes that token only through its own quantised latent
+    alt = z_full[[1]].copy()
+    alt[0, 0] = -alt[0, 0] + 1.0
+    moved = O.forward(wl, inp, tokens=[1], z_rows=alt, weights=W)
+    assert not np.array_equal(moved["out"], base["out"][[1]])
