@@ -53,7 +53,7 @@ static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const 
       return LMOE_ERR_CUDA;
     configured_dev = dev;
   }
-  kern<<<grid, 192, Fp4Smem::kBytes, s>>>(a, b, p);
+  kern<<<grid, Fp4Smem::kThreads, Fp4Smem::kBytes, s>>>(a, b, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

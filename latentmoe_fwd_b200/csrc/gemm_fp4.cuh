@@ -8,8 +8,9 @@
 //   GEMM 2: y = acc * s_a * s_w2[e] * gate[row], stored as BF16
 //
 // Structure as the BF16 kernel (TMA producer warp, single-thread MMA issuer,
-// four epilogue warps, persistent tiles of 128 activation rows x 256 output
-// features), plus:
+// persistent tiles of 128 activation rows x 256 output features), but with
+// eight epilogue warps -- two per TMEM lane quarter, each draining half of the
+// columns -- because quantising a in GEMM 1 costs more than the MMAs; plus:
 //  * each stage carries the tile's scale atoms (512 B = 128 rows x 4 scales),
 //    fetched with bulk copies and moved shared -> tensor memory with
 //    tcgen05.cp (32 lanes x 128 bit, replicated over the four lane quarters)
@@ -56,6 +57,7 @@ struct Fp4Smem {
   static constexpr int kStages = 4;
   static constexpr int kBarOffset = kStages * kStage;
   static constexpr int kBytes = kBarOffset + (2 * kStages + 6) * 8 + 16 + 1024;
+  static constexpr int kThreads = 64 + 256;   // producer, MMA, eight epilogue warps
   static constexpr int kAccCols = 256;
   static constexpr int kAcc1 = 192;          // second accumulator starts here
   static constexpr int kSfaCol = 448;
@@ -140,9 +142,10 @@ __device__ __forceinline__ uint32_t fp4_quant16(const float* x, float s_g, uint2
   codes.y = 0;
   if (dec != 0.0f) {
     const float sc = __fmul_rn(dec, s_g);
+    const float rc = __frcp_rn(sc);
     float v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(x[i], sc);
+    for (int i = 0; i < 16; ++i) v[i] = e2m1_operand(x[i], sc, rc);
     codes.x = fp4_cvt_x8(v);
     codes.y = fp4_cvt_x8(v + 8);
   }
@@ -154,7 +157,7 @@ __device__ __forceinline__ long long fp4_sf_offset(long long row, int j, int gro
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Fp4Params p) {
   using S = Fp4Smem;
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&tfull[0], 1);
     mbar_init(&tfull[1], 1);
-    mbar_init(overlap_free, 4);
+    mbar_init(overlap_free, 8);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -295,7 +298,8 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    const int q = warp & 3;
+    const int q = warp & 3;             // TMEM lane quarter
+    const int half = (warp - 2) >> 2;   // which four of the eight 32-column chunks
     const int r = q * 32 + lane;
     int local = 0;
     const float in_s = __ldg(p.in_scale);
@@ -313,14 +317,16 @@ __global__ void __launch_bounds__(192, 1)
       const long long row = act0 + r;
       const bool row_ok = r < act_n;
       const float gate = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && row_ok) ? __ldg(p.row_scale + row) : 1.0f;
+      // chunks of this warp; the TMEM slice shared with the other accumulator
+      // (chunks 6,7 of buffer 0, chunks 0,1 of buffer 1) is drained first
+      const bool owns_shared = buf ? half == 0 : half == 1;
 #pragma unroll 1
-      for (int i = 0; i < 8; ++i) {
-        // drain the TMEM slice shared with the other accumulator first
-        const int c = buf ? i : (i + 6) & 7;
+      for (int i = 0; i < 4; ++i) {
+        const int c = half * 4 + (owns_shared && !buf ? (i + 2) & 3 : i);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc_col + c * 32, v);
         tmem_ld_wait();
-        if (i == 1) {
+        if (i == (owns_shared ? 1 : 0)) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(overlap_free);

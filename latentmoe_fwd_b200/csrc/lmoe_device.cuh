@@ -228,6 +228,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// The E2M1 code of RN(x / sc) from the cheaper x * RN(1 / sc): the two differ
+// by a few ulp at most, so they give the same code unless the value lies
+// within a hair of an E2M1 rounding boundary (0.25, 0.75, 1.25, 1.75, 2.5,
+// 3.5, 5); there the exact quotient is used. Codes equal the division's.
+__device__ __forceinline__ float e2m1_operand(float x, float sc, float rc) {
+  const float v = x * rc;
+  const float a = fabsf(v);
+  float d = fabsf(a - 0.25f);
+  d = fminf(d, fabsf(a - 0.75f));
+  d = fminf(d, fabsf(a - 1.25f));
+  d = fminf(d, fabsf(a - 1.75f));
+  d = fminf(d, fabsf(a - 2.5f));
+  d = fminf(d, fabsf(a - 3.5f));
+  d = fminf(d, fabsf(a - 5.0f));
+  return d <= a * 0x1p-19f ? __fdiv_rn(x, sc) : v;
+}
+
 // Expert owning padded row `row`: the largest e with poff[e] <= row among
 // the non-decreasing padded offsets (empty experts have equal neighbours).
 __device__ __forceinline__ int find_expert(const int* poff, int groups, int row) {

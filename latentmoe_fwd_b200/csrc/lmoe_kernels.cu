@@ -25,31 +25,55 @@ namespace lmoe {
 // token's bias-free logit RMS (the size of the GEMM's partial sums):
 // tau = 2^-10 * RMS + 2^-20 * max|logit|.
 // ===========================================================================
+// Exact logit of one expert: the stored operands' products (exact in fp64)
+// summed in fp64, the warp's lanes striding over d with eight 16-byte loads of
+// x and of the weight row in flight per lane (latency-bound otherwise).
 template <typename TA>
 __device__ __forceinline__ double exact_dot(const TA* __restrict__ x, const TA* __restrict__ w, int d, int lane) {
+  constexpr int V = 16 / sizeof(TA);   // elements per 16-byte vector
   double acc = 0.0;
-  if constexpr (sizeof(TA) == 2) {
-    for (int j = lane * 8; j < d; j += 256) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + j));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(w + j));
-      const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&b);
+  int j = lane * V;
+  for (; j + 7 * 32 * V < d; j += 8 * 32 * V) {
+    uint4 a[8], b[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      a[u] = __ldg(reinterpret_cast<const uint4*>(x + j + u * 32 * V));
+      b[u] = __ldg(reinterpret_cast<const uint4*>(w + j + u * 32 * V));
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if constexpr (sizeof(TA) == 2) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 fa = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&a[u])[i]);
+          const float2 fb = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&b[u])[i]);
+          acc = fma(static_cast<double>(fa.x), static_cast<double>(fb.x), acc);
+          acc = fma(static_cast<double>(fa.y), static_cast<double>(fb.y), acc);
+        }
+      } else {
+        const float* fa = reinterpret_cast<const float*>(&a[u]);
+        const float* fb = reinterpret_cast<const float*>(&b[u]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc = fma(static_cast<double>(fa[i]), static_cast<double>(fb[i]), acc);
+      }
+    }
+  }
+  for (; j < d; j += 32 * V) {   // remainder, one vector at a time
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + j));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(w + j));
+    if constexpr (sizeof(TA) == 2) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float2 fa = __bfloat1622float2(ha[i]);
-        const float2 fb = __bfloat1622float2(hb[i]);
+        const float2 fa = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&a)[i]);
+        const float2 fb = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&b)[i]);
         acc = fma(static_cast<double>(fa.x), static_cast<double>(fb.x), acc);
         acc = fma(static_cast<double>(fa.y), static_cast<double>(fb.y), acc);
       }
-    }
-  } else {
-    for (int j = lane * 4; j < d; j += 128) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(x + j));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(w + j));
-      acc = fma(static_cast<double>(a.x), static_cast<double>(b.x), acc);
-      acc = fma(static_cast<double>(a.y), static_cast<double>(b.y), acc);
-      acc = fma(static_cast<double>(a.z), static_cast<double>(b.z), acc);
-      acc = fma(static_cast<double>(a.w), static_cast<double>(b.w), acc);
+    } else {
+      const float* fa = reinterpret_cast<const float*>(&a);
+      const float* fb = reinterpret_cast<const float*>(&b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc = fma(static_cast<double>(fa[i]), static_cast<double>(fb[i]), acc);
     }
   }
 #pragma unroll
@@ -143,9 +167,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       const int c = __ffs(todo) - 1;
       todo &= todo - 1;
       const int e = __shfl_sync(0xffffffffu, my_i, c);
-      double ex = exact_dot<TA>(xt, wr + static_cast<int64_t>(e) * d, d, lane);
-      if (bias) ex += static_cast<double>(__ldg(bias + e));
-      if (lane == c) my_v = static_cast<float>(ex);
+      double v = exact_dot<TA>(xt, wr + static_cast<int64_t>(e) * d, d, lane);
+      if (bias) v += static_cast<double>(__ldg(bias + e));
+      if (lane == c) my_v = static_cast<float>(v);
     }
   }
   // rank of each candidate among the C
@@ -651,9 +675,10 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float (&x)[16], float s_g,
   uint32_t lo = 0, hi = 0;
   if (dec != 0.0f) {
     const float sc = __fmul_rn(dec, s_g);
+    const float rc = __frcp_rn(sc);
     float v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(x[i], sc);
+    for (int i = 0; i < 16; ++i) v[i] = e2m1_operand(x[i], sc, rc);   // = RN(x / sc) for the code
     lo = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
     hi = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
   }

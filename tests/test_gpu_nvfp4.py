@@ -208,3 +208,42 @@ def test_nvfp4_weights_quantised_bit_exact_per_expert():
 def test_nvfp4_forward_reduced(T):
     wl = LI.reduced("ultra_nvfp4", T=T, d=512, l=256, N=16, K=4, m=512)
     _nvfp4_layer(wl)
+
+
+def test_quantize_codes_at_e2m1_boundaries_with_irregular_scales():
+    """Elements at k * sc and a few fp32 ulp around it, for every E2M1 rounding
+    boundary k and irregular block scales sc = dec(s_b) * s_g: the device must
+    reproduce the codes of RN(x / sc) exactly (it multiplies by RN(1/sc) and
+    falls back to the quotient only near a boundary)."""
+    rng = np.random.default_rng(29)
+    f32 = np.float32
+    bounds = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float32)
+    s_g = f32(0.0137)
+    t = f32(s_g * f32(6.0))
+    blocks = []
+    for D in rng.choice(O.E4M3_MAG[8:120], 40):          # normal E4M3 block scales
+        D = f32(D)
+        amax = f32(D * t)                                   # block max -> scale code D
+        sc = f32(f32(O.e4m3_decode(O.e4m3_encode(f32(amax / t)))) * s_g)
+        vals = []
+        for k in bounds:
+            base = f32(k * sc)
+            for step in (-3, -2, -1, 0, 1, 2, 3):
+                v = base
+                for _ in range(abs(step)):
+                    v = np.nextafter(v, f32(np.inf) if step > 0 else f32(0))
+                vals.append(v)
+        vals = np.array(vals, dtype=np.float32)
+        for i in range(0, len(vals), 15):
+            blk = np.zeros(16, dtype=np.float32)
+            blk[0] = amax
+            chunk = vals[i:i + 15] * rng.choice([-1, 1], len(vals[i:i + 15])).astype(np.float32)
+            blk[1:1 + len(chunk)] = chunk
+            blocks.append(blk)
+    v = np.stack(blocks)
+    x = torch.from_numpy(v).cuda()
+    gin = torch.tensor([float(s_g)], dtype=torch.float32, device="cuda")
+    codes, sf, _ = quantize_dev(x, v.shape[0], 16, global_in=gin)
+    rc, rsf, _ = O.nvfp4_quantize(v.astype(np.float64), float(s_g))
+    assert np.array_equal(sf.cpu().numpy(), rsf)
+    assert np.array_equal(codes.cpu().numpy(), rc)
