@@ -211,6 +211,16 @@ def run_reference(args, wl):
     return 0
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings across the process group
+    (every rank takes part; all ranks get the result)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def workload_config(wl):
     c = {"workload": wl.name, "T": wl.T, "d": wl.d, "l": wl.l, "N": wl.N, "K": wl.K, "m": wl.m,
          "n_shared": wl.n_shared, "m_shared": wl.m_shared, "identity_projections": wl.identity,
@@ -349,9 +359,7 @@ def main():
     e2e_ms = e_start.elapsed_time(e_end)
 
     if world > 1:
-        tt = torch.tensor([ms, e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), float(tt[1])
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], "cuda")
 
     tokens = wl.T * K * world
     value = tokens / (ms / 1000.0)

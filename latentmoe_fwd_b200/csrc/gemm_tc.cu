@@ -44,7 +44,8 @@ static bool make_map_bf16(CUtensorMap* map, const TcOperand& op, int box_rows) {
 
 template <int BN, int STAGES, int EPI>
 static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& a1,
-                             const CUtensorMap& b1, const TcParams& p, int grid, cudaStream_t s) {
+                             const CUtensorMap& b1, const CUtensorMap& bs, const TcParams& p, int grid,
+                             cudaStream_t s) {
   using Sm = TcSmem<BN, STAGES>;
   auto kern = tc_gemm_kernel<BN, STAGES, EPI>;
   static int configured_dev = -1;
@@ -55,22 +56,20 @@ static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const
       return LMOE_ERR_CUDA;
     configured_dev = dev;
   }
-  kern<<<grid, 192, Sm::kBytes, s>>>(a0, b0, a1, b1, p);
+  kern<<<grid, 192, Sm::kBytes, s>>>(a0, b0, a1, b1, bs, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
 template <int BN, int STAGES>
-static lmoe_status dispatch_epi(int epi, const CUtensorMap& a0, const CUtensorMap& b0,
-                                const CUtensorMap& a1, const CUtensorMap& b1, const TcParams& p,
-                                int grid, cudaStream_t s) {
+static lmoe_status dispatch_epi(int epi, const CUtensorMap* m, const TcParams& p, int grid, cudaStream_t s) {
   switch (epi) {
-    case EPI_F32_BIAS: return launch_tc<BN, STAGES, EPI_F32_BIAS>(a0, b0, a1, b1, p, grid, s);
-    case EPI_BF16: return launch_tc<BN, STAGES, EPI_BF16>(a0, b0, a1, b1, p, grid, s);
-    case EPI_SQRELU: return launch_tc<BN, STAGES, EPI_SQRELU>(a0, b0, a1, b1, p, grid, s);
-    case EPI_GATE: return launch_tc<BN, STAGES, EPI_GATE>(a0, b0, a1, b1, p, grid, s);
-    case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(a0, b0, a1, b1, p, grid, s);
-    case EPI_PARTIAL: return launch_tc<BN, STAGES, EPI_PARTIAL>(a0, b0, a1, b1, p, grid, s);
+    case EPI_F32_BIAS: return launch_tc<BN, STAGES, EPI_F32_BIAS>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_BF16: return launch_tc<BN, STAGES, EPI_BF16>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_SQRELU: return launch_tc<BN, STAGES, EPI_SQRELU>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_GATE: return launch_tc<BN, STAGES, EPI_GATE>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_PARTIAL: return launch_tc<BN, STAGES, EPI_PARTIAL>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
   }
   return LMOE_ERR_INVALID_ARG;
 }
@@ -79,7 +78,8 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   const int bn = L.bn;
   if (bn != 32 && bn != 64 && bn != 128 && bn != 256) return LMOE_ERR_INVALID_ARG;
   // A always has 128-row boxes (activation rows normal, weight rows swap); B has BN-row boxes.
-  CUtensorMap maps[4];
+  // maps: A0, B0, A1, B1, and a 32-row token box of B0 for small weight-major tiles
+  CUtensorMap maps[5];
   for (int sg = 0; sg < L.nseg; ++sg) {
     if (!make_map_bf16(&maps[2 * sg], L.a[sg], 128)) return LMOE_ERR_INVALID_ARG;
     if (!make_map_bf16(&maps[2 * sg + 1], L.b[sg], bn)) return LMOE_ERR_INVALID_ARG;
@@ -88,6 +88,12 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
     maps[2] = maps[0];
     maps[3] = maps[1];
   }
+  if (L.swap && L.grouped && bn > 32) {
+    if (!make_map_bf16(&maps[4], L.b[0], 32)) return LMOE_ERR_INVALID_ARG;
+  } else {
+    maps[4] = maps[1];
+  }
+  if (L.grouped && L.groups > 1024) return LMOE_ERR_UNSUPPORTED;
   TcParams p;
   p.swap = L.swap;
   p.grouped = L.grouped;
@@ -120,10 +126,10 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   const int epi = p.ksplit > 1 ? static_cast<int>(EPI_PARTIAL) : L.epi;
   lmoe_status st = LMOE_ERR_INVALID_ARG;
   switch (bn) {
-    case 256: st = dispatch_epi<256, 4>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
-    case 128: st = dispatch_epi<128, 6>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
-    case 64: st = dispatch_epi<64, 8>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
-    case 32: st = dispatch_epi<32, 10>(epi, maps[0], maps[1], maps[2], maps[3], p, g, stream); break;
+    case 256: st = dispatch_epi<256, 4>(epi, maps, p, g, stream); break;
+    case 128: st = dispatch_epi<128, 6>(epi, maps, p, g, stream); break;
+    case 64: st = dispatch_epi<64, 8>(epi, maps, p, g, stream); break;
+    case 32: st = dispatch_epi<32, 10>(epi, maps, p, g, stream); break;
   }
   if (st != LMOE_OK || p.ksplit == 1) return st;
   // deterministic reduction of the partial sums (fixed split order) + the real epilogue

@@ -71,7 +71,12 @@ struct TcSmem {
   static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
   static constexpr int kBarOffset = STAGES * kStageBytes;
   // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, tmem ptr, abort
-  static constexpr int kBytes = kBarOffset + (2 * STAGES + 5) * 8 + 16 + 1024;  // +1024 alignment slack
+  static constexpr int kPrefixOffset = kBarOffset + (2 * STAGES + 5) * 8 + 16;
+  // weight-major grouped tiles: prefix over experts of their tile counts
+  static constexpr int kMaxGroups = 1024;
+  // weight-major epilogue: one 32 x 32 BF16 transpose tile per epilogue warp
+  static constexpr int kEpiOffset = (kPrefixOffset + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kBytes = kEpiOffset + 4 * 32 * 32 * 2 + 1024;  // +1024 alignment slack
 };
 
 struct TileInfo {
@@ -82,10 +87,40 @@ struct TileInfo {
   int w0;         // first weight row (output feature) of the tile
   int split;      // split-K index
   int kb0, kb1;   // K blocks [kb0, kb1) of this tile
+  int wshared;    // weight-major: other tiles of this expert read the same weight rows
 };
 
+// Weight-major grouped tiles: expert e owns ceil(n_e / BN) token tiles times
+// ceil(cols / 128) weight tiles. prefix[e] = tiles of experts before e, built
+// by every CTA in shared memory at start.
 template <int BN>
-__device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
+__device__ __forceinline__ void build_tile_prefix(const TcParams& p, int* prefix) {
+  const int ntw = (p.cols + 127) / 128;
+  for (int e = threadIdx.x; e < p.groups; e += blockDim.x) {
+    const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+    prefix[e + 1] = ((n_e + BN - 1) / BN) * ntw;
+  }
+  if (threadIdx.x == 0) prefix[0] = 0;
+  __syncthreads();
+  if (threadIdx.x < 32) {   // inclusive scan of prefix[1..groups] by one warp
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int base = 1; base <= p.groups; base += 32) {
+      const int i = base + lane;
+      int v = i <= p.groups ? prefix[i] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
+      }
+      if (i <= p.groups) prefix[i] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ int tc_num_tiles(const TcParams& p, const int* prefix) {
   const int ntw_normal = (p.cols + BN - 1) / BN;
   const int ntw_swap = (p.cols + 127) / 128;
   int n;
@@ -93,16 +128,17 @@ __device__ __forceinline__ int tc_num_tiles(const TcParams& p) {
     int mt = p.grouped ? (__ldg(p.padded_offsets + p.groups) >> 7) : (p.rows + 127) / 128;
     n = mt * ntw_normal;
   } else {
-    n = p.grouped ? p.groups * ntw_swap : ntw_swap;
+    n = p.grouped ? prefix[p.groups] : ntw_swap;
   }
   return n * p.ksplit;
 }
 
 template <int BN>
-__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t, int kb_total) {
+__device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t, int kb_total, const int* prefix) {
   TileInfo ti;
   ti.valid = 1;
   ti.expert = 0;
+  ti.wshared = 0;
   ti.split = t % p.ksplit;
   t /= p.ksplit;
   {
@@ -128,20 +164,42 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t, int kb_tot
     }
   } else {
     const int ntw = (p.cols + 127) / 128;
-    ti.w0 = (t % ntw) * 128;
     if (p.grouped) {
-      const int e = t / ntw;
+      // largest e with prefix[e] <= t (it owns at least one tile)
+      int lo = 0, hi = p.groups - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      const int e = lo;
       const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+      const int ntt = (n_e + BN - 1) / BN;
+      const int local = t - prefix[e];
+      // the weight tiles of one token tile are consecutive: CTAs running at the
+      // same time share the token rows, and the expert's weights (reused by
+      // every token tile) stay in L2
+      const int tt = local / ntw, mw = local % ntw;
       ti.expert = e;
-      ti.act0 = __ldg(p.padded_offsets + e);
-      ti.act_n = min(n_e, BN);
-      if (n_e <= 0) ti.valid = 0;
+      ti.wshared = ntt > 1;
+      ti.w0 = mw * 128;
+      ti.act0 = __ldg(p.padded_offsets + e) + tt * BN;
+      ti.act_n = min(BN, n_e - tt * BN);
+      if (ti.act_n <= 0) ti.valid = 0;
     } else {
+      ti.w0 = (t % ntw) * 128;
       ti.act0 = 0;
       ti.act_n = min(p.rows, BN);
     }
   }
   return ti;
+}
+
+// MMA N of a tile: its rows (normal) or its tokens rounded up to 16 (weight-major).
+template <int BN>
+__device__ __forceinline__ int tile_mma_n(const TcParams& p, const TileInfo& ti) {
+  if (!p.swap) return BN;
+  const int n = (ti.act_n + 15) & ~15;
+  return n < 16 ? 16 : n;
 }
 
 template <int EPI>
@@ -163,7 +221,7 @@ template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmBs, const TcParams p) {
   using S = TcSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -174,9 +232,12 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
+  int* tile_prefix = reinterpret_cast<int*>(smem + S::kPrefixOffset);
+  __nv_bfloat16* epi_tile = reinterpret_cast<__nv_bfloat16*>(smem + S::kEpiOffset);
 
   const int warp = warp_id();
   const int lane = lane_id();
+  if (p.swap && p.grouped) build_tile_prefix<BN>(p, tile_prefix);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -203,7 +264,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
 
-  const int ntiles = tc_num_tiles<BN>(p);
+  const int ntiles = tc_num_tiles<BN>(p, tile_prefix);
   const int kb_total = p.seg[0].kblocks + (p.nseg > 1 ? p.seg[1].kblocks : 0);
 
   if (warp == 0) {
@@ -211,19 +272,22 @@ __global__ void __launch_bounds__(192, 1)
       // ---------------- TMA producer ----------------
       const uint64_t pol_w = policy_evict_first();   // weights: streamed
       const uint64_t pol_a = policy_evict_last();    // activations: reused across tiles
+      const uint64_t pol_n = policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0;
       uint32_t last_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tc_tile<BN>(p, t, kb_total);
+        const TileInfo ti = tc_tile<BN>(p, t, kb_total, tile_prefix);
         if (!ti.valid) continue;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x100 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStageBytes;
           uint8_t* sb = sa + S::kABytes;
-          mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+          // weight-major tiles of at most 32 tokens fetch a 32-row token box
+          const bool small_b = BN > 32 && p.swap && p.grouped && ti.act_n <= 32;
+          mbar_arrive_expect_tx(&full[stage], small_b ? S::kABytes + 32 * 128 : S::kStageBytes);
           const int sg = (p.nseg > 1 && kb >= p.seg[0].kblocks) ? 1 : 0;
           const int k = (sg ? kb - p.seg[0].kblocks : kb) * 64;
           const CUtensorMap* ma = sg ? &tmA1 : &tmA0;
@@ -235,11 +299,17 @@ __global__ void __launch_bounds__(192, 1)
           } else {
             a_row = ti.w0; a_grp = ti.expert; b_row = ti.act0; b_grp = 0;
           }
-          const uint64_t pa = p.swap ? pol_w : pol_a;
-          const uint64_t pb = p.swap ? pol_a : pol_w;
+          // weights are streamed (evict first) unless several tiles of this
+          // expert share them (weight-major tiles of an expert with more tokens
+          // than one tile holds); activation rows are kept (evict last)
+          // weight-major tiles: the weights are kept when other token tiles of
+          // the expert will read them again, streamed otherwise
+          const uint64_t pa = p.swap ? (ti.wshared ? pol_a : pol_w) : pol_a;
+          const uint64_t pb = p.swap ? (ti.wshared ? pol_n : pol_a) : pol_w;
           if (akg > 0) tma_load_3d(sa, ma, &full[stage], k % akg, a_row, k / akg, pa);
           else tma_load_3d(sa, ma, &full[stage], k, a_row, a_grp, pa);
           if (bkg > 0) tma_load_3d(sb, mb, &full[stage], k % bkg, b_row, k / bkg, pb);
+          else if (small_b) tma_load_3d(sb, &tmBs, &full[stage], k, b_row, b_grp, pb);
           else tma_load_3d(sb, mb, &full[stage], k, b_row, b_grp, pb);
           issued_mask |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -258,20 +328,21 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
       bool any = false;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const TileInfo ti = tc_tile<BN>(p, t, kb_total);
+        const TileInfo ti = tc_tile<BN>(p, t, kb_total, tile_prefix);
         if (!ti.valid) continue;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, 0x200 + acc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t idesc = idesc_bf16_f32(128, tile_mma_n<BN>(p, ti));
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x300 + stage)) { ok = false; break; }
           tc_fence_after();
@@ -302,15 +373,16 @@ __global__ void __launch_bounds__(192, 1)
     const int r = q * 32 + lane;     // accumulator row of this thread
     int local = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const TileInfo ti = tc_tile<BN>(p, t, kb_total);
+      const TileInfo ti = tc_tile<BN>(p, t, kb_total, tile_prefix);
       if (!ti.valid) continue;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, 0x400 + acc)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+      const int nchunks = p.swap ? (ti.act_n + 31) / 32 : BN / 32;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < nchunks; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + c * 32, v);
         tmem_ld_wait();
@@ -357,9 +429,35 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
           }
+        } else if (EPI != EPI_PARTIAL && EPI != EPI_F32_BIAS) {
+          // weight-major, BF16 out: this lane owns output feature w0 + r and 32
+          // tokens; transpose the warp's 32 x 32 block through shared memory so
+          // each token's 32 features go out as 16-byte stores
+          __nv_bfloat16* tb = epi_tile + (warp & 3) * 32 * 32;
+          const int col = ti.w0 + r;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const long long row = ti.act0 + c * 32 + j;
+            const bool live = c * 32 + j < ti.act_n && col < p.cols;
+            const float val = live ? epi_value<EPI>(__uint_as_float(v[j]), p, row, col) : 0.0f;
+            tb[j * 32 + lane] = __float2bfloat16_rn(val);
+          }
+          __syncwarp();
+          const int seg = lane & 3;              // 8 features of the warp's 32
+          const int col0 = ti.w0 + q * 32 + seg * 8;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = (lane >> 2) + 8 * i;   // token within the chunk
+            const int tok = c * 32 + j;
+            if (tok < ti.act_n && col0 < p.cols) {
+              const uint4 u = *reinterpret_cast<const uint4*>(tb + j * 32 + seg * 8);
+              __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (ti.act0 + tok) * p.ld_out + col0;
+              *reinterpret_cast<uint4*>(o) = u;
+            }
+          }
+          __syncwarp();
         } else {
-          // swap: this thread owns output feature `col`; columns of the
-          // accumulator are activation rows (tokens)
+          // weight-major, fp32 or split-K partial out: scalar stores
           const int col = ti.w0 + r;
           if (col < p.cols) {
 #pragma unroll

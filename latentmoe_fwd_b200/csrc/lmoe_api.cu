@@ -287,9 +287,11 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
     if (st != LMOE_OK) return st;
     logits = lg;
   }
-  const bool computed = logits_in == nullptr;
-  return launch_topk(logits, cfg->T, cfg->N, cfg->K, topk_idx, topk_w, computed ? x : nullptr,
-                     computed ? w_router : nullptr, computed ? bias : nullptr, cfg->d, cfg->act, err, s);
+  // computed logits get their near-tied decisions refined exactly; caller
+  // logits are taken as they are
+  const bool refine = logits_in == nullptr;
+  return launch_topk(logits, cfg->T, cfg->N, cfg->K, topk_idx, topk_w, refine ? x : nullptr,
+                     refine ? w_router : nullptr, refine ? bias : nullptr, cfg->d, cfg->act, err, s);
 }
 
 lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets, int32_t* perm_src,
@@ -357,7 +359,10 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
     g2.row_scale = gate;
     return simt_gemm(g2, err, s);
   }
-  const int sbn = swap_bn(cfg->T);
+  // Weight-major tiles for every grouped GEMM: 128 weight rows x up to BN
+  // tokens of one expert, the MMA's N set per tile, so no token padding is
+  // multiplied; small token counts use narrow tiles.
+  const int sbn = swap_bn(cfg->T) ? swap_bn(cfg->T) : 256;
   TcLaunch g1;
   g1.grouped = 1;
   g1.cols = cfg->m;
@@ -372,7 +377,7 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
     g1.bn = sbn;
     g1.a[0] = w1op;
     g1.b[0] = zop;
-    g1.max_tiles = static_cast<int64_t>(cfg->N) * ((cfg->m + 127) / 128);
+    g1.max_tiles = (static_cast<int64_t>(cfg->T) * cfg->K / sbn + cfg->N) * ((cfg->m + 127) / 128);
   } else {
     g1.bn = normal_bn(cfg->m);
     g1.a[0] = zop;
@@ -392,7 +397,7 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   if (sbn) {
     g2.a[0] = w2op;
     g2.b[0] = aop;
-    g2.max_tiles = static_cast<int64_t>(cfg->N) * ((cfg->l + 127) / 128);
+    g2.max_tiles = (static_cast<int64_t>(cfg->T) * cfg->K / sbn + cfg->N) * ((cfg->l + 127) / 128);
   } else {
     g2.bn = normal_bn(cfg->l);
     g2.a[0] = aop;

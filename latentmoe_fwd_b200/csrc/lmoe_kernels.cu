@@ -25,13 +25,46 @@ namespace lmoe {
 // token's bias-free logit RMS (the size of the GEMM's partial sums):
 // tau = 2^-10 * RMS + 2^-20 * max|logit|.
 // ===========================================================================
-// Exact logit of one expert: the stored operands' products (exact in fp64)
-// summed in fp64, the warp's lanes striding over d with eight 16-byte loads of
-// x and of the weight row in flight per lane (latency-bound otherwise).
+// Exact logit of one expert. Products of two BF16 (or the fp32 layer's
+// fp32) values are formed exactly where the format allows and summed as an
+// unevaluated fp32 pair (hi, lo) with error-free TwoSum steps, so the result
+// carries ~48 significant bits -- without fp64 arithmetic, which is slow on
+// this part. The warp's lanes stride over d with eight 16-byte loads of x and
+// of the weight row in flight per lane.
+__device__ __forceinline__ void two_sum_acc(float& hi, float& lo, float p) {
+  const float s = __fadd_rn(hi, p);
+  const float bb = __fsub_rn(s, hi);
+  const float err = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bb)), __fsub_rn(p, bb));
+  hi = s;
+  lo = __fadd_rn(lo, err);
+}
+
+template <typename TA>
+__device__ __forceinline__ void dot_vec(const uint4& a, const uint4& b, float& hi, float& lo) {
+  if constexpr (sizeof(TA) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fa = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&a)[i]);
+      const float2 fb = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&b)[i]);
+      two_sum_acc(hi, lo, __fmul_rn(fa.x, fb.x));   // exact: 8 x 8 significant bits
+      two_sum_acc(hi, lo, __fmul_rn(fa.y, fb.y));
+    }
+  } else {
+    const float* fa = reinterpret_cast<const float*>(&a);
+    const float* fb = reinterpret_cast<const float*>(&b);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float p = __fmul_rn(fa[i], fb[i]);
+      two_sum_acc(hi, lo, p);
+      lo = __fadd_rn(lo, fmaf(fa[i], fb[i], -p));   // the product's own rounding error
+    }
+  }
+}
+
 template <typename TA>
 __device__ __forceinline__ double exact_dot(const TA* __restrict__ x, const TA* __restrict__ w, int d, int lane) {
   constexpr int V = 16 / sizeof(TA);   // elements per 16-byte vector
-  double acc = 0.0;
+  float hi = 0.0f, lo = 0.0f;
   int j = lane * V;
   for (; j + 7 * 32 * V < d; j += 8 * 32 * V) {
     uint4 a[8], b[8];
@@ -41,44 +74,18 @@ __device__ __forceinline__ double exact_dot(const TA* __restrict__ x, const TA* 
       b[u] = __ldg(reinterpret_cast<const uint4*>(w + j + u * 32 * V));
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if constexpr (sizeof(TA) == 2) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 fa = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&a[u])[i]);
-          const float2 fb = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&b[u])[i]);
-          acc = fma(static_cast<double>(fa.x), static_cast<double>(fb.x), acc);
-          acc = fma(static_cast<double>(fa.y), static_cast<double>(fb.y), acc);
-        }
-      } else {
-        const float* fa = reinterpret_cast<const float*>(&a[u]);
-        const float* fb = reinterpret_cast<const float*>(&b[u]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc = fma(static_cast<double>(fa[i]), static_cast<double>(fb[i]), acc);
-      }
-    }
+    for (int u = 0; u < 8; ++u) dot_vec<TA>(a[u], b[u], hi, lo);
   }
-  for (; j < d; j += 32 * V) {   // remainder, one vector at a time
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + j));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(w + j));
-    if constexpr (sizeof(TA) == 2) {
+  for (; j < d; j += 32 * V)   // remainder, one vector at a time
+    dot_vec<TA>(__ldg(reinterpret_cast<const uint4*>(x + j)), __ldg(reinterpret_cast<const uint4*>(w + j)), hi, lo);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 fa = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&a)[i]);
-        const float2 fb = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&b)[i]);
-        acc = fma(static_cast<double>(fa.x), static_cast<double>(fb.x), acc);
-        acc = fma(static_cast<double>(fa.y), static_cast<double>(fb.y), acc);
-      }
-    } else {
-      const float* fa = reinterpret_cast<const float*>(&a);
-      const float* fb = reinterpret_cast<const float*>(&b);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc = fma(static_cast<double>(fa[i]), static_cast<double>(fb[i]), acc);
-    }
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ohi = __shfl_xor_sync(0xffffffffu, hi, off);
+    const float olo = __shfl_xor_sync(0xffffffffu, lo, off);
+    two_sum_acc(hi, lo, ohi);
+    lo = __fadd_rn(lo, olo);
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  return acc;
+  return static_cast<double>(hi) + static_cast<double>(lo);
 }
 
 // (value desc, index asc) ordering
