@@ -435,11 +435,33 @@ __global__ void __launch_bounds__(192, 1)
           // each token's 32 features go out as 16-byte stores
           __nv_bfloat16* tb = epi_tile + (warp & 3) * 32 * 32;
           const int col = ti.w0 + r;
+          // per-token operands of the chunk are fetched before any store: the
+          // gate of token c*32+lane by this lane (one coalesced load, then
+          // shuffles), the residual row values into registers
+          float gate = 1.0f;
+          if (EPI == EPI_GATE && p.row_scale) {
+            const int tk = c * 32 + lane;
+            gate = tk < ti.act_n ? __ldg(p.row_scale + ti.act0 + tk) : 0.0f;
+          }
+          float res[32];
+          if (EPI == EPI_ADD_RES) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const bool live = c * 32 + j < ti.act_n && col < p.cols;
+              res[j] = live ? __bfloat162float(p.residual[(ti.act0 + c * 32 + j) * p.ld_res + col]) : 0.0f;
+            }
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const long long row = ti.act0 + c * 32 + j;
-            const bool live = c * 32 + j < ti.act_n && col < p.cols;
-            const float val = live ? epi_value<EPI>(__uint_as_float(v[j]), p, row, col) : 0.0f;
+            float val = __uint_as_float(v[j]);
+            if (EPI == EPI_SQRELU) {
+              val = fmaxf(val, 0.0f);
+              val = val * val;
+            } else if (EPI == EPI_GATE) {
+              val = val * __shfl_sync(0xffffffffu, gate, j);
+            } else if (EPI == EPI_ADD_RES) {
+              val = val + res[j];
+            }
             tb[j * 32 + lane] = __float2bfloat16_rn(val);
           }
           __syncwarp();
