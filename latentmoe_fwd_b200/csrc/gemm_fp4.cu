@@ -59,7 +59,7 @@ static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const 
 }
 
 lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream) {
-  if (L.k % 256 || L.cols % 256) return LMOE_ERR_UNSUPPORTED;
+  if (L.k % 256 || L.cols % 256 || L.groups > Fp4Smem::kMaxGroups) return LMOE_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
   if (!make_map_fp4(&ma, L.a_codes, L.k, L.a_rows, 1, 128)) return LMOE_ERR_INVALID_ARG;
   if (!make_map_fp4(&mb, L.b_codes, L.k, L.cols, L.groups, 256)) return LMOE_ERR_INVALID_ARG;
@@ -81,6 +81,7 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   p.out = L.out;
   p.out_sf = L.out_sf;
   p.ld_out = L.ld_out;
+  p.out_vec32 = (reinterpret_cast<uintptr_t>(L.out) % 32 == 0) && (L.ld_out * 2) % 32 == 0;
   p.err = DevErr{err_word};
   const int sms = device_sm_count();
   const int64_t tiles = (L.a_rows / 128) * (L.cols / 256);

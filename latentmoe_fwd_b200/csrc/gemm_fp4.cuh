@@ -45,6 +45,7 @@ struct Fp4Params {
   void* out;                  // GEMM1: codes [rows][cols/2]; GEMM2: bf16 [rows][cols]
   uint8_t* out_sf;            // GEMM1: MMA-tiled scales of a
   long long ld_out;           // GEMM2: elements per row
+  int out_vec32;              // GEMM2: rows start on 32-byte boundaries (32-byte stores)
   DevErr err;
 };
 
@@ -56,7 +57,11 @@ struct Fp4Smem {
   static constexpr int kStage = kA + kB + kSFA + kSFB;   // 55296
   static constexpr int kStages = 4;
   static constexpr int kBarOffset = kStages * kStage;
-  static constexpr int kBytes = kBarOffset + (2 * kStages + 6) * 8 + 16 + 1024;
+  static constexpr int kMaxGroups = 1024;
+  // per-expert padded start and real end rows, copied once per CTA so that
+  // the tile -> expert lookup is a short walk in shared memory
+  static constexpr int kRowsOffset = kBarOffset + 256;
+  static constexpr int kBytes = kRowsOffset + 2 * (kMaxGroups + 1) * 4 + 1024;
   static constexpr int kThreads = 64 + 256;   // producer, MMA, eight epilogue warps
   static constexpr int kAccCols = 256;
   static constexpr int kAcc1 = 192;          // second accumulator starts here
@@ -118,19 +123,6 @@ __device__ __forceinline__ float fp4_e4m3_value(uint32_t c) {
   return e == 0 ? ldexpf(static_cast<float>(f), -9) : ldexpf(static_cast<float>(8 + f), e - 10);
 }
 
-__device__ __forceinline__ uint32_t fp4_cvt_x8(const float* v) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(r)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  return r;
-}
-
 // Quantise 16 values with global scale s_g: returns the E4M3 code and 8 code bytes.
 __device__ __forceinline__ uint32_t fp4_quant16(const float* x, float s_g, uint2& codes) {
   float amax = 0.0f;
@@ -142,12 +134,7 @@ __device__ __forceinline__ uint32_t fp4_quant16(const float* x, float s_g, uint2
   codes.y = 0;
   if (dec != 0.0f) {
     const float sc = __fmul_rn(dec, s_g);
-    const float rc = __frcp_rn(sc);
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = e2m1_operand(x[i], sc, rc);
-    codes.x = fp4_cvt_x8(v);
-    codes.y = fp4_cvt_x8(v + 8);
+    codes = e2m1_codes16(x, sc, __frcp_rn(sc));
   }
   return sb;
 }
@@ -187,6 +174,13 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
+  int* s_pstart = reinterpret_cast<int*>(smem + S::kRowsOffset);   // [groups + 1] padded starts
+  int* s_rend = s_pstart + S::kMaxGroups + 1;                          // [groups] real ends
+  for (int g = threadIdx.x; g <= p.groups; g += blockDim.x) {
+    const int ps = __ldg(p.padded_offsets + g);
+    s_pstart[g] = ps;
+    if (g < p.groups) s_rend[g] = ps + __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+  }
   if (warp == 1) tmem_alloc(tmem_ptr, 512);
   tc_fence_before();
   __syncthreads();
@@ -194,20 +188,23 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
   const uint32_t tmem_base = *tmem_ptr;
 
   const int ntw = (p.cols + 255) / 256;
-  const int ntiles = (__ldg(p.padded_offsets + p.groups) >> 7) * ntw;
+  const int ntiles = (s_pstart[p.groups] >> 7) * ntw;
 
+  // a CTA visits its tiles in increasing order, so the owning expert (the
+  // largest e with padded start <= act0) only moves forward
+  int cur_e = 0;
   auto tile_of = [&](int t, int& e, int& act0, int& act_n, int& w0) {
     w0 = (t % ntw) * 256;
     act0 = (t / ntw) * 128;
-    e = find_expert(p.padded_offsets, p.groups, act0);
-    const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
-    act_n = min(128, __ldg(p.padded_offsets + e) + n_e - act0);
+    while (cur_e + 1 < p.groups && s_pstart[cur_e + 1] <= act0) ++cur_e;
+    e = cur_e;
+    act_n = min(128, s_rend[e] - act0);
   };
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_w = policy_evict_normal();   // read again by the expert's other row tiles
+      const uint64_t pol_a = policy_evict_last();     // read by every column tile
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_par = 0;
@@ -305,34 +302,28 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     const float in_s = __ldg(p.in_scale);
     const float out_s = (EPI == FP4_EPI_SQRELU_QUANT) ? __ldg(p.out_scale) : 0.0f;
     const int groups64_out = (p.cols + 63) / 64;
+    const uint64_t pol_out = policy_evict_first();
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int e, act0, act_n, w0;
       tile_of(t, e, act0, act_n, w0);
       if (act_n <= 0) continue;
       const int buf = local & 1;
-      if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1400 + buf)) break;
-      tc_fence_after();
-      const float scale = __fmul_rn(in_s, __ldg(p.w_scale + e)) * (EPI == FP4_EPI_GATE_BF16 ? 1.0f : 1.0f);
-      const uint32_t acc_col = buf ? S::kAcc1 : 0;
       const long long row = act0 + r;
       const bool row_ok = r < act_n;
+      // per-tile scalars fetched before the accumulator is ready
       const float gate = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && row_ok) ? __ldg(p.row_scale + row) : 1.0f;
-      // chunks of this warp; the TMEM slice shared with the other accumulator
-      // (chunks 6,7 of buffer 0, chunks 0,1 of buffer 1) is drained first
-      const bool owns_shared = buf ? half == 0 : half == 1;
-#pragma unroll 1
-      for (int i = 0; i < 4; ++i) {
-        const int c = half * 4 + (owns_shared && !buf ? (i + 2) & 3 : i);
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc_col + c * 32, v);
-        tmem_ld_wait();
-        if (i == (owns_shared ? 1 : 0)) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(overlap_free);
-        }
+      const float scale = __fmul_rn(in_s, __ldg(p.w_scale + e));
+      if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1400 + buf)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (buf ? S::kAcc1 : 0);
+      auto release = [&]() {   // this warp no longer reads the TMEM slice the next tile overwrites
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(overlap_free);
+      };
+      auto emit = [&](int c, const uint32_t (&v)[32]) {
         const int col0 = w0 + c * 32;
-        if (!row_ok || col0 >= p.cols) continue;
+        if (!row_ok || col0 >= p.cols) return;
         if (EPI == FP4_EPI_SQRELU_QUANT) {
           float a[32];
 #pragma unroll
@@ -344,13 +335,24 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
           const uint32_t s0 = fp4_quant16(a, out_s, c0);
           const uint32_t s1 = fp4_quant16(a + 16, out_s, c1);
           uint8_t* codes = reinterpret_cast<uint8_t*>(p.out) + row * (p.cols / 2) + col0 / 2;
-          *reinterpret_cast<uint4*>(codes) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+          st_global_v4_hint(codes, make_uint4(c0.x, c0.y, c1.x, c1.y), pol_out);
           const int j0 = col0 / 16;
           p.out_sf[fp4_sf_offset(row, j0, groups64_out)] = static_cast<uint8_t>(s0);
           p.out_sf[fp4_sf_offset(row, j0 + 1, groups64_out)] = static_cast<uint8_t>(s1);
         } else {
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
           const float sg = scale * gate;
+          if (p.out_vec32) {   // whole 32-byte sectors per store
+#pragma unroll
+            for (int j = 0; j < 32; j += 16) {
+              uint32_t u[8];
+#pragma unroll
+              for (int h = 0; h < 8; ++h)
+                u[h] = pack_bf16x2(__uint_as_float(v[j + 2 * h]) * sg, __uint_as_float(v[j + 2 * h + 1]) * sg);
+              st_global_v8_hint(o + j, u, pol_out);
+            }
+            return;
+          }
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             uint4 u;
@@ -358,8 +360,40 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
             u.y = pack_bf16x2(__uint_as_float(v[j + 2]) * sg, __uint_as_float(v[j + 3]) * sg);
             u.z = pack_bf16x2(__uint_as_float(v[j + 4]) * sg, __uint_as_float(v[j + 5]) * sg);
             u.w = pack_bf16x2(__uint_as_float(v[j + 6]) * sg, __uint_as_float(v[j + 7]) * sg);
-            *reinterpret_cast<uint4*>(o + j) = u;
+            st_global_v4_hint(o + j, u, pol_out);
           }
+        }
+      };
+      // The slice shared with the other accumulator (chunks 6,7 of buffer 0,
+      // chunks 0,1 of buffer 1) is read first, both chunks at once, and the
+      // MMA released before any arithmetic; the other warps release at once.
+      const bool owns_shared = buf ? half == 0 : half == 1;
+      if (owns_shared) {
+        const int c0 = buf ? 0 : 6;
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(acc + c0 * 32, v0);
+        tmem_ld_32x32b_x32(acc + (c0 + 1) * 32, v1);
+        tmem_ld_wait();
+        release();
+        emit(c0, v0);
+        emit(c0 + 1, v1);
+        const int c2 = buf ? 2 : 4;
+#pragma unroll 1
+        for (int i = 0; i < 2; ++i) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(acc + (c2 + i) * 32, v);
+          tmem_ld_wait();
+          emit(c2 + i, v);
+        }
+      } else {
+        release();
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+          const int c = half * 4 + i;
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(acc + c * 32, v);
+          tmem_ld_wait();
+          emit(c, v);
         }
       }
       ++local;

@@ -228,21 +228,60 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The E2M1 code of RN(x / sc) from the cheaper x * RN(1 / sc): the two differ
-// by a few ulp at most, so they give the same code unless the value lies
-// within a hair of an E2M1 rounding boundary (0.25, 0.75, 1.25, 1.75, 2.5,
-// 3.5, 5); there the exact quotient is used. Codes equal the division's.
-__device__ __forceinline__ float e2m1_operand(float x, float sc, float rc) {
-  const float v = x * rc;
-  const float a = fabsf(v);
-  float d = fabsf(a - 0.25f);
-  d = fminf(d, fabsf(a - 0.75f));
-  d = fminf(d, fabsf(a - 1.25f));
-  d = fminf(d, fabsf(a - 1.75f));
-  d = fminf(d, fabsf(a - 2.5f));
-  d = fminf(d, fabsf(a - 3.5f));
-  d = fminf(d, fabsf(a - 5.0f));
-  return d <= a * 0x1p-19f ? __fdiv_rn(x, sc) : v;
+// 16-byte global store with an L2 eviction-priority hint (createpolicy word).
+__device__ __forceinline__ void st_global_v4_hint(void* ptr, const uint4& v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
+}
+
+// 32-byte global store (one full sector) with an L2 eviction-priority hint;
+// the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8_hint(void* ptr, const uint32_t (&u)[8], uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;" ::"l"(ptr), "r"(u[0]),
+               "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "l"(pol)
+               : "memory");
+}
+
+// Eight E2M1 codes (two per byte, the first value in the low nibble) with
+// round-to-nearest-even and saturation to +-6.
+__device__ __forceinline__ uint32_t cvt_e2m1_x8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// E2M1 codes of q_i = RN(x_i / sc) for 16 values, without 16 divisions.
+// With rc = RN(1/sc), the products x * RN(rc * (1 - 2^-20)) and
+// x * RN(rc * (1 + 2^-20)) bracket q (their relative distance to x/sc is
+// 2^-20 minus a few 2^-24 roundings, q's is at most 2^-24). Rounding to E2M1
+// is monotone, so where both ends give the same code q gives it too; only
+// when a value sits within ~2^-20 of an E2M1 rounding boundary (the codes of
+// the two ends differ) are the exact quotients taken. Codes equal the
+// division's in every case.
+__device__ __forceinline__ uint2 e2m1_codes16(const float* x, float sc, float rc) {
+  const float rlo = __fmul_rn(rc, 1.0f - 0x1p-20f);
+  const float rhi = __fmul_rn(rc, 1.0f + 0x1p-20f);
+  float lo[16], hi[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    lo[i] = __fmul_rn(x[i], rlo);
+    hi[i] = __fmul_rn(x[i], rhi);
+  }
+  uint2 c = make_uint2(cvt_e2m1_x8(lo), cvt_e2m1_x8(lo + 8));
+  if (c.x != cvt_e2m1_x8(hi) || c.y != cvt_e2m1_x8(hi + 8)) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) lo[i] = __fdiv_rn(x[i], sc);
+    c = make_uint2(cvt_e2m1_x8(lo), cvt_e2m1_x8(lo + 8));
+  }
+  return c;
 }
 
 // Expert owning padded row `row`: the largest e with poff[e] <= row among

@@ -11,26 +11,33 @@
 namespace lmoe {
 
 // ===========================================================================
-// Top-K + renormalised softmax gates: one warp per token.
+// Top-K + renormalised softmax gates.
 // Selection order: logit descending, expert index ascending (ties to the
 // lower index). Gates: exp(l_k - l_max) / sum over the K chosen.
 //
 // Exact decisions from approximate logits: tensor-core logits carry fp32
 // accumulation error. When the kernel is given x and W_r, every adjacent pair
 // among the K+1 largest logits (and any further expert near the K-th) whose
-// gap is within 2*tau gets its logits recomputed exactly (products of the
-// stored operands summed in fp64), and the candidates are re-ranked. Experts
-// left approximate are more than 2*tau from every neighbour, so their order
-// is exact as long as the logit error is below tau. tau scales with the
-// token's bias-free logit RMS (the size of the GEMM's partial sums):
-// tau = 2^-10 * RMS + 2^-20 * max|logit|.
+// gap is within 2*tau gets its logits recomputed exactly, and the candidates
+// are re-ranked. Experts left approximate are more than 2*tau from every
+// neighbour, so their order is exact as long as the logit error is below
+// tau. tau scales with the token's bias-free logit RMS (the size of the
+// GEMM's partial sums): tau = 2^-10 * RMS + 2^-20 * max|logit|.
+//
+// Work split: a block of eight warps owns `tpb` tokens (eight, or one when
+// there are few tokens). A token's warp extracts its candidates; the exact
+// dot products of all of the block's marked candidates then form one pool
+// that every warp of the block draws from, each dot split over up to eight
+// warps when the pool is small, so a decode batch of a few tokens does not
+// run its dots one after another on one warp.
 // ===========================================================================
-// Exact logit of one expert. Products of two BF16 (or the fp32 layer's
-// fp32) values are formed exactly where the format allows and summed as an
-// unevaluated fp32 pair (hi, lo) with error-free TwoSum steps, so the result
-// carries ~48 significant bits -- without fp64 arithmetic, which is slow on
-// this part. The warp's lanes stride over d with eight 16-byte loads of x and
-// of the weight row in flight per lane.
+constexpr int kTopkWarps = 8;
+constexpr int kTopkPieces = kTopkWarps * 32;
+
+// Exact logit pieces. Products of two BF16 (or the fp32 layer's fp32) values
+// are formed exactly where the format allows and summed as an unevaluated
+// fp32 pair (hi, lo) with error-free TwoSum steps, so the result carries ~48
+// significant bits -- without fp64 arithmetic, which is slow on this part.
 __device__ __forceinline__ void two_sum_acc(float& hi, float& lo, float p) {
   const float s = __fadd_rn(hi, p);
   const float bb = __fsub_rn(s, hi);
@@ -61,12 +68,16 @@ __device__ __forceinline__ void dot_vec(const uint4& a, const uint4& b, float& h
   }
 }
 
+// Double-word sum of x[j] * w[j] over j in [j0, j1) (multiples of the 16-byte
+// vector), reduced over the warp. Eight 16-byte loads of each operand are in
+// flight per lane; two accumulator pairs shorten the dependency chain.
 template <typename TA>
-__device__ __forceinline__ double exact_dot(const TA* __restrict__ x, const TA* __restrict__ w, int d, int lane) {
+__device__ __forceinline__ float2 exact_dot_range(const TA* __restrict__ x, const TA* __restrict__ w, int j0, int j1,
+                                                  int lane) {
   constexpr int V = 16 / sizeof(TA);   // elements per 16-byte vector
-  float hi = 0.0f, lo = 0.0f;
-  int j = lane * V;
-  for (; j + 7 * 32 * V < d; j += 8 * 32 * V) {
+  float hi0 = 0.0f, lo0 = 0.0f, hi1 = 0.0f, lo1 = 0.0f;
+  int j = j0 + lane * V;
+  for (; j + 7 * 32 * V < j1; j += 8 * 32 * V) {
     uint4 a[8], b[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -74,18 +85,23 @@ __device__ __forceinline__ double exact_dot(const TA* __restrict__ x, const TA* 
       b[u] = __ldg(reinterpret_cast<const uint4*>(w + j + u * 32 * V));
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) dot_vec<TA>(a[u], b[u], hi, lo);
+    for (int u = 0; u < 8; u += 2) {
+      dot_vec<TA>(a[u], b[u], hi0, lo0);
+      dot_vec<TA>(a[u + 1], b[u + 1], hi1, lo1);
+    }
   }
-  for (; j < d; j += 32 * V)   // remainder, one vector at a time
-    dot_vec<TA>(__ldg(reinterpret_cast<const uint4*>(x + j)), __ldg(reinterpret_cast<const uint4*>(w + j)), hi, lo);
+  for (; j < j1; j += 32 * V)   // remainder, one vector at a time
+    dot_vec<TA>(__ldg(reinterpret_cast<const uint4*>(x + j)), __ldg(reinterpret_cast<const uint4*>(w + j)), hi0, lo0);
+  two_sum_acc(hi0, lo0, hi1);
+  lo0 = __fadd_rn(lo0, lo1);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    const float ohi = __shfl_xor_sync(0xffffffffu, hi, off);
-    const float olo = __shfl_xor_sync(0xffffffffu, lo, off);
-    two_sum_acc(hi, lo, ohi);
-    lo = __fadd_rn(lo, olo);
+    const float ohi = __shfl_xor_sync(0xffffffffu, hi0, off);
+    const float olo = __shfl_xor_sync(0xffffffffu, lo0, off);
+    two_sum_acc(hi0, lo0, ohi);
+    lo0 = __fadd_rn(lo0, olo);
   }
-  return static_cast<double>(hi) + static_cast<double>(lo);
+  return make_float2(hi0, lo0);
 }
 
 // (value desc, index asc) ordering
@@ -93,107 +109,176 @@ __device__ __forceinline__ bool before(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
+// Unsigned key with the order of the float (-0 and +0 equal); 0 marks
+// "nothing", NaN sorts below every number.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 1u;
+  if (f == 0.0f) return 0x80000000u;
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 template <int NPL, typename TA>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T, int N, int K,
-                                                   int32_t* __restrict__ idx, float* __restrict__ w,
-                                                   const TA* __restrict__ x, const TA* __restrict__ wr,
-                                                   const float* __restrict__ bias, int d) {
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits, int64_t T, int N,
+                                                               int K, int tpb, int32_t* __restrict__ idx,
+                                                               float* __restrict__ w, const TA* __restrict__ x,
+                                                               const TA* __restrict__ wr,
+                                                               const float* __restrict__ bias, int d) {
+  __shared__ int s_njobs[kTopkWarps];
+  __shared__ int s_expert[kTopkWarps * 32];
+  __shared__ float2 s_part[kTopkPieces];
+  constexpr unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
+  const int warp = threadIdx.x >> 5;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * tpb + warp;
+  const bool has_token = warp < tpb && t < T;
   const bool refine = x != nullptr;
-  const float* row = logits + t * N;
-  float v[NPL];
-  float sq = 0.0f, vmax_abs = 0.0f;
-#pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    const int col = lane + 32 * i;
-    v[i] = col < N ? __ldg(row + col) : -INFINITY;
-    if (col < N) {
-      const float nb = v[i] - (bias ? __ldg(bias + col) : 0.0f);
-      sq = fmaf(nb, nb, sq);
-      vmax_abs = fmaxf(vmax_abs, fabsf(v[i]));
-    }
-  }
-  float tau = 0.0f;
-  if (refine) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      vmax_abs = fmaxf(vmax_abs, __shfl_xor_sync(0xffffffffu, vmax_abs, off));
-    }
-    tau = ldexpf(sqrtf(sq / static_cast<float>(N)), -10) + ldexpf(vmax_abs, -20);
-  }
-  // extract candidates in (approximate) order: the K best, the (K+1)-th, and
-  // while refining, further experts within 2 tau of the K-th (at most 32)
-  uint32_t taken = 0;
+
   float my_v = -INFINITY;   // lane c holds candidate c
   int my_i = 0x7fffffff;
   int C = 0;
-  float kth = -INFINITY;
-  const int cmax = min(N, 32);
-  while (C < cmax) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+  unsigned todo = 0;
+  if (has_token) {
+    const float* row = logits + t * N;
+    float v[NPL];
+    uint32_t key[NPL];
+    float sq = 0.0f, vmax_abs = 0.0f;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int col = lane + 32 * i;
-      const bool live = col < N && !((taken >> i) & 1u);
-      if (live && before(v[i], col, bv, bi)) {
-        bv = v[i];
-        bi = col;
+      v[i] = col < N ? __ldg(row + col) : -INFINITY;
+      key[i] = col < N ? order_key(v[i]) : 0u;
+      if (col < N) {
+        const float nb = v[i] - (bias ? __ldg(bias + col) : 0.0f);
+        sq = fmaf(nb, nb, sq);
+        vmax_abs = fmaxf(vmax_abs, fabsf(v[i]));
       }
     }
+    float tau = 0.0f;
+    if (refine) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (before(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
+      for (int off = 16; off > 0; off >>= 1) {
+        sq += __shfl_xor_sync(FULL, sq, off);
+        vmax_abs = fmaxf(vmax_abs, __shfl_xor_sync(FULL, vmax_abs, off));
+      }
+      tau = ldexpf(sqrtf(sq / static_cast<float>(N)), -10) + ldexpf(vmax_abs, -20);
+    }
+    // this lane's best remaining entry (largest key, lowest column on ties)
+    uint32_t taken = 0;
+    uint32_t hk = 0;
+    int hi_i = 0;
+    float hv = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (key[i] > hk) {
+        hk = key[i];
+        hi_i = i;
+        hv = v[i];
+      }
+    // extract candidates in (approximate) order: the K best, the (K+1)-th, and
+    // while refining, further experts within 2 tau of the K-th (at most 32)
+    float kth = -INFINITY;
+    const int cmax = min(N, 32);
+    while (C < cmax) {
+      const uint32_t mk = __reduce_max_sync(FULL, hk);
+      if (mk == 0u) break;
+      const unsigned bal = __ballot_sync(FULL, hk == mk);
+      int wl = __ffs(bal) - 1;
+      if (bal & (bal - 1u))   // equal values in several lanes: the lowest column wins
+        wl = static_cast<int>(__reduce_min_sync(FULL, hk == mk ? static_cast<uint32_t>(hi_i * 32 + lane) : ~0u) & 31u);
+      const float bv = __shfl_sync(FULL, hv, wl);
+      const int bi = __shfl_sync(FULL, hi_i * 32 + lane, wl);
+      if (C >= K && !(refine && bv >= kth - 2.0f * tau)) break;   // not a boundary candidate
+      if (lane == C) {
+        my_v = bv;
+        my_i = bi;
+      }
+      if (C == K - 1) kth = bv;
+      ++C;
+      if (!refine && C >= K) break;
+      if (lane == wl) {   // the winning lane moves on to its next entry
+        taken |= 1u << hi_i;
+        hk = 0;
+        hv = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          if (!((taken >> i) & 1u) && key[i] > hk) {
+            hk = key[i];
+            hi_i = i;
+            hv = v[i];
+          }
       }
     }
-    if (C >= K && !(refine && bv >= kth - 2.0f * tau)) break;   // not a boundary candidate
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == C) {
-      my_v = bv;
-      my_i = bi;
+    if (refine) {
+      // mark candidates that have a neighbour within 2 tau
+      const float up = __shfl_up_sync(FULL, my_v, 1);
+      const float dn = __shfl_down_sync(FULL, my_v, 1);
+      const bool mark =
+          lane < C && ((lane > 0 && up - my_v <= 2.0f * tau) || (lane + 1 < C && my_v - dn <= 2.0f * tau));
+      todo = __ballot_sync(FULL, mark);
+      if (mark) s_expert[warp * 32 + __popc(todo & ((1u << lane) - 1u))] = my_i;
     }
-    if (C == K - 1) kth = bv;
-    ++C;
-    if (!refine && C >= K) break;
   }
   if (refine) {
-    // mark candidates that have a neighbour within 2 tau; recompute them exactly
-    const float up = __shfl_up_sync(0xffffffffu, my_v, 1);
-    const float dn = __shfl_down_sync(0xffffffffu, my_v, 1);
-    const bool mark = lane < C && ((lane > 0 && up - my_v <= 2.0f * tau) || (lane + 1 < C && my_v - dn <= 2.0f * tau));
-    unsigned todo = __ballot_sync(0xffffffffu, mark);
-    const TA* xt = x + t * d;
-    while (todo) {
-      const int c = __ffs(todo) - 1;
-      todo &= todo - 1;
-      const int e = __shfl_sync(0xffffffffu, my_i, c);
-      double v = exact_dot<TA>(xt, wr + static_cast<int64_t>(e) * d, d, lane);
-      if (bias) v += static_cast<double>(__ldg(bias + e));
-      if (lane == c) my_v = static_cast<float>(v);
+    // pooled exact dots: jobs numbered in warp order, each split into nseg pieces
+    if (lane == 0) s_njobs[warp] = has_token ? __popc(todo) : 0;
+    __syncthreads();
+    const int nj = lane < kTopkWarps ? s_njobs[lane] : 0;
+    int incl = nj;
+#pragma unroll
+    for (int off = 1; off < kTopkWarps; off <<= 1) {
+      const int o = __shfl_up_sync(FULL, incl, off);
+      if (lane >= off) incl += o;
+    }
+    const int total = __shfl_sync(FULL, incl, kTopkWarps - 1);
+    if (total > 0) {
+      const int nseg = total >= kTopkWarps ? 1 : kTopkWarps / total;
+      constexpr int V = 16 / sizeof(TA);
+      const int chunk = ((d / V + nseg - 1) / nseg) * V;
+      for (int pc = warp; pc < total * nseg; pc += kTopkWarps) {
+        const int job = pc / nseg;
+        const int seg = pc - job * nseg;
+        const int ow = __popc(__ballot_sync(FULL, lane < kTopkWarps && incl <= job));   // owning warp
+        const int excl = __shfl_sync(FULL, incl - nj, ow);
+        const int e = s_expert[ow * 32 + (job - excl)];
+        const int64_t tok = static_cast<int64_t>(blockIdx.x) * tpb + ow;
+        const int j0 = min(d, seg * chunk);
+        const int j1 = min(d, j0 + chunk);
+        const float2 r = exact_dot_range<TA>(x + tok * d, wr + static_cast<int64_t>(e) * d, j0, j1, lane);
+        if (lane == 0) s_part[pc] = r;
+      }
+      __syncthreads();
+      const int my_excl = __shfl_sync(FULL, incl - nj, warp);
+      if ((todo >> lane) & 1u) {
+        const int job = my_excl + __popc(todo & ((1u << lane) - 1u));
+        float hi = 0.0f, lo = 0.0f;
+        for (int sg = 0; sg < nseg; ++sg) {
+          const float2 r = s_part[job * nseg + sg];
+          two_sum_acc(hi, lo, r.x);
+          lo = __fadd_rn(lo, r.y);
+        }
+        double val = static_cast<double>(hi) + static_cast<double>(lo);
+        if (bias) val += static_cast<double>(__ldg(bias + my_i));
+        my_v = static_cast<float>(val);
+      }
     }
   }
+  if (!has_token) return;
   // rank of each candidate among the C
   int rank = 0;
   for (int c = 0; c < C; ++c) {
-    const float ov = __shfl_sync(0xffffffffu, my_v, c);
-    const int oi = __shfl_sync(0xffffffffu, my_i, c);
+    const float ov = __shfl_sync(FULL, my_v, c);
+    const int oi = __shfl_sync(FULL, my_i, c);
     if (lane < C && c != lane && before(ov, oi, my_v, my_i)) ++rank;
   }
   const bool chosen = lane < C && rank < K;
   // the largest logit is rank 0
-  const unsigned top_mask = __ballot_sync(0xffffffffu, lane < C && rank == 0);
-  const float lmax = __shfl_sync(0xffffffffu, my_v, __ffs(top_mask) - 1);
+  const unsigned top_mask = __ballot_sync(FULL, lane < C && rank == 0);
+  const float lmax = __shfl_sync(FULL, my_v, __ffs(top_mask) - 1);
   const float e = chosen ? expf(my_v - lmax) : 0.0f;
   float sum = e;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(FULL, sum, off);
   if (chosen) {
     idx[t * K + rank] = my_i;
     w[t * K + rank] = __fdiv_rn(e, sum);
@@ -204,17 +289,22 @@ lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* i
                         const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s) {
   (void)err;
   if (T == 0) return LMOE_OK;
-  const int blocks = static_cast<int>((T * 32 + 255) / 256);
+  // few tokens: one token per block, so the block's eight warps share its dots
+  const int tpb = (x != nullptr && T <= 1024) ? 1 : kTopkWarps;
+  const int64_t blocks64 = (T + tpb - 1) / tpb;
+  if (blocks64 > 0x7fffffff) return LMOE_ERR_UNSUPPORTED;
+  const int blocks = static_cast<int>(blocks64);
   const int npl = (N + 31) / 32;
-#define LMOE_TOPK(NPLV)                                                                                    \
-  do {                                                                                                    \
-    if (act == LMOE_F32)                                                                                  \
-      topk_kernel<NPLV, float><<<blocks, 256, 0, s>>>(logits, T, N, K, idx, w, static_cast<const float*>(x), \
-                                                      static_cast<const float*>(w_router), bias, d);      \
-    else                                                                                                  \
-      topk_kernel<NPLV, __nv_bfloat16><<<blocks, 256, 0, s>>>(                                            \
-          logits, T, N, K, idx, w, static_cast<const __nv_bfloat16*>(x),                                  \
-          static_cast<const __nv_bfloat16*>(w_router), bias, d);                                          \
+#define LMOE_TOPK(NPLV)                                                                                       \
+  do {                                                                                                       \
+    if (act == LMOE_F32)                                                                                     \
+      topk_kernel<NPLV, float><<<blocks, kTopkWarps * 32, 0, s>>>(                                           \
+          logits, T, N, K, tpb, idx, w, static_cast<const float*>(x), static_cast<const float*>(w_router),   \
+          bias, d);                                                                                          \
+    else                                                                                                     \
+      topk_kernel<NPLV, __nv_bfloat16><<<blocks, kTopkWarps * 32, 0, s>>>(                                   \
+          logits, T, N, K, tpb, idx, w, static_cast<const __nv_bfloat16*>(x),                                \
+          static_cast<const __nv_bfloat16*>(w_router), bias, d);                                             \
   } while (0)
   if (npl <= 1) LMOE_TOPK(1);
   else if (npl <= 2) LMOE_TOPK(2);
@@ -605,22 +695,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   return r & 0xFFu;
 }
 
-// eight fp32 -> eight E2M1 codes in one 32-bit word, element 2i in the low
-// nibble of byte i (PTX cvt, round to nearest even, saturating).
-__device__ __forceinline__ uint32_t cvt_e2m1x8(float x0, float x1, float x2, float x3, float x4,
-                                               float x5, float x6, float x7) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(r)
-      : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
-  return r;
-}
-
 // Every CTA reduces the per-CTA maxima the same way (max is exact, so the
 // order does not matter) and derives s_g = fp32(amax / 2688), 1 when amax = 0.
 __device__ __forceinline__ float cta_global_scale(const float* partials, int np, const float* global_in) {
@@ -682,12 +756,9 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float (&x)[16], float s_g,
   uint32_t lo = 0, hi = 0;
   if (dec != 0.0f) {
     const float sc = __fmul_rn(dec, s_g);
-    const float rc = __frcp_rn(sc);
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = e2m1_operand(x[i], sc, rc);   // = RN(x / sc) for the code
-    lo = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
-    hi = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+    const uint2 c = e2m1_codes16(x, sc, __frcp_rn(sc));   // codes of RN(x / sc)
+    lo = c.x;
+    hi = c.y;
   }
   codes.x = lo;
   codes.y = hi;

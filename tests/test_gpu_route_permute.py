@@ -49,6 +49,61 @@ def test_topk_exact_ties_go_to_lower_index():
     assert np.max(np.abs(w - rw)) <= 1e-6
 
 
+def test_topk_signed_zeros_tie_to_lower_index():
+    logits = np.full((3, 40), -1.0, dtype=np.float32)
+    logits[0, 5], logits[0, 9] = np.float32(-0.0), np.float32(0.0)    # equal values: expert 5 first
+    logits[1, 9], logits[1, 5] = np.float32(-0.0), np.float32(0.0)
+    logits[2, 30], logits[2, 2] = np.float32(0.0), np.float32(-0.0)
+    idx, w = _route_from_logits(logits, 40, 2)
+    assert idx.tolist() == [[5, 9], [5, 9], [2, 30]]
+    assert np.allclose(w, 0.5)
+
+
+@pytest.mark.parametrize("T", [3, 1100])
+def test_route_computed_all_logits_equal(T):
+    # zero router weights: every logit is exactly 0, so every candidate is in
+    # a tie and gets an exact recompute; the lower index wins each tie
+    N, K, d = 512, 22, 256
+    cfg = L.config(T=T, d=d, l=d, N=N, K=K, m=64)
+    x = torch.randn((T, d), device="cuda").to(torch.bfloat16)
+    wr = torch.zeros((N, d), device="cuda", dtype=torch.bfloat16)
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    ws = L.workspace(cfg, L.OP_ROUTE)
+    L.route(cfg, x, wr, None, None, idx, w, None, ws)
+    st, _ = L.read_device_error(ws)
+    assert st == L.OK
+    assert np.array_equal(idx.cpu().numpy(), np.tile(np.arange(K, dtype=np.int32), (T, 1)))
+    assert np.allclose(w.cpu().numpy(), 1.0 / K, rtol=0, atol=1e-7)
+
+
+@pytest.mark.parametrize("T", [5, 1500])
+def test_route_computed_bit_exact_outside_near_ties(T):
+    # logits computed on the device (tensor-core GEMM + exact refinement)
+    # against the oracle's fp64 decisions; both refinement layouts (one
+    # token per block for small T, eight per block above)
+    wl = LI.reduced("ultra_zipf", T=T, d=512, l=64, m=64)
+    inp = LI.make_inputs(wl)
+    cfg = L.config(T=T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m)
+    bits = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    x, wr = bits(inp["x"]), bits(inp["w_router"])
+    bias = torch.from_numpy(inp["router_bias"]).cuda()
+    idx = torch.empty((T, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, wl.K), dtype=torch.float32, device="cuda")
+    ws = L.workspace(cfg, L.OP_ROUTE)
+    L.route(cfg, x, wr, bias, None, idx, w, None, ws)
+    st, _ = L.read_device_error(ws)
+    assert st == L.OK
+    logits = O.router_logits(O.from_bf16_bits(inp["x"]), O.from_bf16_bits(inp["w_router"]), inp["router_bias"])
+    ridx, rw = O.route_topk(logits, wl.K)
+    srt = -np.sort(-logits, axis=1)[:, :wl.K + 1]
+    clear = np.min(srt[:, :-1] - srt[:, 1:], axis=1) >= 1e-5       # rows without a near-tie
+    assert clear.mean() > 0.9
+    got = idx.cpu().numpy()
+    assert np.array_equal(got[clear], ridx[clear])
+    assert np.max(np.abs(w.cpu().numpy()[clear] - rw[clear])) <= 1e-6
+
+
 def test_topk_zipf_biased_logits():
     wl = LI.reduced("ultra_zipf", T=257, d=64, l=32, m=32)
     inp = LI.make_inputs(wl)
