@@ -126,6 +126,30 @@ def expert_gemm_work(wl, counts: np.ndarray):
     return wbytes + abytes, flops, used
 
 
+GEMM_SOURCES = ("gemm_tc.cuh", "gemm_tc2.cuh", "gemm_fp4.cuh", "lmoe_device.cuh")
+
+
+def gemm_source_sha() -> str:
+    """sha256 prefix over the expert-GEMM kernel sources (traffic figures
+    taken with ncu stay valid only while these are unchanged)."""
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "latentmoe_fwd_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def expert_gemm_kernel(wl) -> str:
+    """The kernel that runs the grouped expert GEMMs of this workload."""
+    if wl.dtype == "nvfp4":
+        return "fp4_gemm_kernel (grouped NVFP4 expert GEMM 1 + GEMM 2, 2 launches per step)"
+    if wl.dtype == "f32":
+        return "simt_gemm_kernel (fp32 layer)"
+    if wl.T > 64 and wl.T * wl.K >= 64 * wl.N:
+        return "tc2_gemm_kernel (CTA-pair grouped expert GEMM 1 + GEMM 2, 2 launches per step)"
+    return "tc_gemm_kernel (grouped expert GEMM 1 + GEMM 2, 2 launches per step)"
+
+
 def traffic_record(workload: str):
     """DRAM traffic per expert-GEMM launch pair from a committed ncu capture,
     valid only while the GEMM source is unchanged."""
@@ -134,8 +158,7 @@ def traffic_record(workload: str):
         return None
     with open(p) as f:
         rec = json.load(f)
-    src = os.path.join(ROOT, "latentmoe_fwd_b200", "csrc", "gemm_tc.cuh")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    h = gemm_source_sha()
     entry = rec.get(workload)
     if not entry or entry.get("gemm_source_sha") != h:
         return None
@@ -386,10 +409,12 @@ def main():
         tr = traffic_record(wl.name)
         roof["traffic"] = tr
     roof.update({
-        "kernel": "tc_gemm_kernel (grouped expert GEMM 1 + GEMM 2, 2 launches per step)",
+        "kernel": expert_gemm_kernel(wl),
         "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops, "experts_used": used,
         "kernel_ms_per_step": gemm_ms, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
-        else "fallback", "peak_kind": "hbm_gbs" if roof.get("bound") == "hbm" else "bf16_tflops_sustained"})
+        else "fallback", "peak_kind": "hbm_gbs" if roof.get("bound") == "hbm" else
+        ("bf16_tflops_sustained x 4 (nominal FP4 : BF16 dense ratio)" if wl.dtype == "nvfp4"
+         else "bf16_tflops_sustained")})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -3,6 +3,7 @@
 #include <mutex>
 
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "lmoe_internal.h"
 
 namespace lmoe {
@@ -145,6 +146,73 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   }
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+// ----- CTA-pair grouped GEMM (weight-major expert tiles) -----
+template <int EPI>
+static lmoe_status launch_tc2(const CUtensorMap* m, const TcParams& p, int64_t max_tiles, cudaStream_t s) {
+  auto kern = tc2_gemm_kernel<EPI>;
+  static int configured_dev = -1;
+  static int max_clusters = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Tc2Smem::kBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (configured_dev != dev) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Smem::kBytes) != cudaSuccess)
+      return LMOE_ERR_CUDA;
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return LMOE_ERR_CUDA;
+    max_clusters = n;
+    configured_dev = dev;
+  }
+  const int64_t clusters = max_tiles < max_clusters ? max_tiles : max_clusters;
+  if (clusters <= 0) return LMOE_OK;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], p) != cudaSuccess) return LMOE_ERR_CUDA;
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+lmoe_status tc2_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) {
+  if (!L.swap || !L.grouped || L.nseg != 1 || L.ksplit > 1) return LMOE_ERR_INVALID_ARG;
+  if (L.groups > Tc2Smem::kMaxGroups) return LMOE_ERR_UNSUPPORTED;
+  // maps: weights (A, 128-row boxes), tokens (B) with 128/64/32/16-row boxes
+  CUtensorMap maps[5];
+  if (!make_map_bf16(&maps[0], L.a[0], 128)) return LMOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (!make_map_bf16(&maps[1 + i], L.b[0], 128 >> i)) return LMOE_ERR_INVALID_ARG;
+  TcParams p = {};
+  p.swap = 1;
+  p.grouped = 1;
+  p.rows = L.rows;
+  p.cols = L.cols;
+  p.nseg = 1;
+  p.seg[0].kblocks = L.kblocks[0];
+  p.offsets = L.offsets;
+  p.padded_offsets = L.padded_offsets;
+  p.groups = L.groups;
+  p.out = L.out;
+  p.ld_out = L.ld_out;
+  p.row_scale = L.row_scale;
+  p.ksplit = 1;
+  p.err = DevErr{err_word};
+  switch (L.epi) {
+    case EPI_BF16: return launch_tc2<EPI_BF16>(maps, p, L.max_tiles, stream);
+    case EPI_SQRELU: return launch_tc2<EPI_SQRELU>(maps, p, L.max_tiles, stream);
+    case EPI_GATE: return launch_tc2<EPI_GATE>(maps, p, L.max_tiles, stream);
+  }
+  return LMOE_ERR_INVALID_ARG;
 }
 
 }  // namespace lmoe

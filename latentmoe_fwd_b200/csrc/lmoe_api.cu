@@ -387,7 +387,16 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   g1.out = a;
   g1.ld_out = cfg->m;
   g1.epi = EPI_SQRELU;
-  if ((st = tc_gemm(g1, err, s)) != LMOE_OK) return st;
+  // enough tokens per expert on average: CTA pairs, 256 features x 256 tokens per tile
+  const bool pairs = sbn == 256 && static_cast<int64_t>(cfg->T) * cfg->K >= 64LL * cfg->N;
+  const int64_t pair_token_tiles = static_cast<int64_t>(cfg->T) * cfg->K / 256 + cfg->N;
+  if (pairs) {
+    g1.max_tiles = pair_token_tiles * ((cfg->m + 255) / 256);
+    st = tc2_gemm(g1, err, s);
+  } else {
+    st = tc_gemm(g1, err, s);
+  }
+  if (st != LMOE_OK) return st;
   if (between) between();
   TcLaunch g2 = g1;
   g2.cols = cfg->l;
@@ -408,6 +417,10 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   g2.ld_out = cfg->l;
   g2.epi = EPI_GATE;
   g2.row_scale = gate;
+  if (pairs) {
+    g2.max_tiles = pair_token_tiles * ((cfg->l + 255) / 256);
+    return tc2_gemm(g2, err, s);
+  }
   return tc_gemm(g2, err, s);
 }
 

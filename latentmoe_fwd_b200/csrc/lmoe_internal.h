@@ -48,6 +48,9 @@ struct TcLaunch {
 };
 
 lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream);
+// Weight-major grouped GEMM on CTA pairs (M = 256 features per pair, up to 256
+// tokens per tile); max_tiles bounds the pair-tile count.
+lmoe_status tc2_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream);
 
 // ----- grouped NVFP4 expert GEMM (gemm_fp4.cu) -----
 struct Fp4Launch {

@@ -84,3 +84,12 @@ def test_expert_ffn_nvfp4(T):
 @pytest.mark.parametrize("T", [20, 300])
 def test_expert_ffn_bf16(T):
     _check(LI.reduced("ultra_decode", T=T, d=512, l=256, N=16, K=4, m=384), 2e-2)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=300, d=512, l=256, N=16, K=4, m=384),      # 64+ tokens per expert: CTA-pair tiles
+    dict(T=1500, d=512, l=200, N=16, K=4, m=320),     # several token tiles per expert, ragged K and features
+])
+def test_expert_ffn_bf16_pair_tiles_skewed(shape):
+    # Zipf-biased routing: some experts take several 256-token tiles, others a few rows
+    _check(LI.reduced("ultra_zipf", **shape), 2e-2)
