@@ -123,7 +123,23 @@ def expert_gemm_work(wl, counts: np.ndarray):
         wbytes = used * 2 * wl.m * wl.l * eb
         abytes = rows * (wl.l + wl.m) * eb * 2
     flops = 2.0 * rows * wl.l * wl.m * 2
+    if wl.n_shared and shared_fused(wl):
+        # the shared experts' two layers run in the same two launches
+        sm = wl.n_shared * wl.m_shared
+        wbytes += 2 * sm * wl.d * 2
+        abytes += wl.T * wl.d * 2 * 2 + wl.T * sm * 2 * 2
+        flops += 2.0 * wl.T * wl.d * sm * 2
     return wbytes + abytes, flops, used
+
+
+def pair_tiles(wl) -> bool:
+    """Grouped BF16 expert GEMMs run on CTA pairs (T > 64, >= 64 rows per expert)."""
+    return wl.dtype == "bf16" and wl.T > 64 and wl.T * wl.K >= 64 * wl.N
+
+
+def shared_fused(wl) -> bool:
+    """The shared experts' layers ride along in the CTA-pair expert-GEMM launches."""
+    return bool(wl.n_shared) and pair_tiles(wl)
 
 
 GEMM_SOURCES = ("gemm_tc.cuh", "gemm_tc2.cuh", "gemm_fp4.cuh", "lmoe_device.cuh")
@@ -145,8 +161,9 @@ def expert_gemm_kernel(wl) -> str:
         return "fp4_gemm_kernel (grouped NVFP4 expert GEMM 1 + GEMM 2, 2 launches per step)"
     if wl.dtype == "f32":
         return "simt_gemm_kernel (fp32 layer)"
-    if wl.T > 64 and wl.T * wl.K >= 64 * wl.N:
-        return "tc2_gemm_kernel (CTA-pair grouped expert GEMM 1 + GEMM 2, 2 launches per step)"
+    if pair_tiles(wl):
+        extra = " with the shared experts' hidden and output layers" if shared_fused(wl) else ""
+        return f"tc2_gemm_kernel (CTA-pair grouped expert GEMM 1 + GEMM 2{extra}, 2 launches per step)"
     return "tc_gemm_kernel (grouped expert GEMM 1 + GEMM 2, 2 launches per step)"
 
 

@@ -95,7 +95,7 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
     maps[4] = maps[1];
   }
   if (L.grouped && L.groups > 1024) return LMOE_ERR_UNSUPPORTED;
-  TcParams p;
+  TcParams p = {};
   p.swap = L.swap;
   p.grouped = L.grouped;
   p.rows = L.rows;
@@ -150,7 +150,7 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
 
 // ----- CTA-pair grouped GEMM (weight-major expert tiles) -----
 template <int EPI>
-static lmoe_status launch_tc2(const CUtensorMap* m, const TcParams& p, int64_t max_tiles, cudaStream_t s) {
+static lmoe_status launch_tc2(const Tc2Maps& m, const TcParams& p, int64_t max_tiles, cudaStream_t s) {
   auto kern = tc2_gemm_kernel<EPI>;
   static int configured_dev = -1;
   static int max_clusters = 0;
@@ -179,7 +179,7 @@ static lmoe_status launch_tc2(const CUtensorMap* m, const TcParams& p, int64_t m
   const int64_t clusters = max_tiles < max_clusters ? max_tiles : max_clusters;
   if (clusters <= 0) return LMOE_OK;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], p) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, m, p) != cudaSuccess) return LMOE_ERR_CUDA;
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -187,11 +187,24 @@ static lmoe_status launch_tc2(const CUtensorMap* m, const TcParams& p, int64_t m
 lmoe_status tc2_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) {
   if (!L.swap || !L.grouped || L.nseg != 1 || L.ksplit > 1) return LMOE_ERR_INVALID_ARG;
   if (L.groups > Tc2Smem::kMaxGroups) return LMOE_ERR_UNSUPPORTED;
-  // maps: weights (A, 128-row boxes), tokens (B) with 128/64/32/16-row boxes
-  CUtensorMap maps[5];
-  if (!make_map_bf16(&maps[0], L.a[0], 128)) return LMOE_ERR_INVALID_ARG;
+  // maps: weights (A, 128-row boxes), tokens (B) with 128/64/32/16-row boxes;
+  // the same for the dense extra problem (copies of the first five without one)
+  Tc2Maps maps;
+  if (!make_map_bf16(&maps.m[0], L.a[0], 128)) return LMOE_ERR_INVALID_ARG;
   for (int i = 0; i < 4; ++i)
-    if (!make_map_bf16(&maps[1 + i], L.b[0], 128 >> i)) return LMOE_ERR_INVALID_ARG;
+    if (!make_map_bf16(&maps.m[1 + i], L.b[0], 128 >> i)) return LMOE_ERR_INVALID_ARG;
+  const bool extra = L.rows_x > 0;
+  if (extra) {
+    if (L.cols_x <= 0) return LMOE_ERR_INVALID_ARG;
+    if (L.x_kgroup > 0 ? (L.x_wt.k != L.x_kgroup || L.x_kgroup % 64 || L.x_act.k != L.x_kgroup * L.x_wt.groups)
+                       : L.x_act.k != L.x_wt.k)
+      return LMOE_ERR_INVALID_ARG;
+    if (!make_map_bf16(&maps.m[5], L.x_wt, 128)) return LMOE_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i)
+      if (!make_map_bf16(&maps.m[6 + i], L.x_act, 128 >> i)) return LMOE_ERR_INVALID_ARG;
+  } else {
+    for (int i = 0; i < 5; ++i) maps.m[5 + i] = maps.m[i];
+  }
   TcParams p = {};
   p.swap = 1;
   p.grouped = 1;
@@ -206,11 +219,18 @@ lmoe_status tc2_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream)
   p.ld_out = L.ld_out;
   p.row_scale = L.row_scale;
   p.ksplit = 1;
+  p.rows_x = extra ? L.rows_x : 0;
+  p.cols_x = extra ? L.cols_x : 0;
+  p.kblocks_x = extra ? static_cast<int>((L.x_act.k + 63) / 64) : 0;
+  p.kgroup_x = extra ? L.x_kgroup : 0;
+  p.out_x = extra ? L.out_x : nullptr;
+  p.ld_out_x = extra ? L.ld_out_x : 0;
   p.err = DevErr{err_word};
+  const int64_t tiles = L.max_tiles + (extra ? ((L.rows_x + 255) / 256) * ((L.cols_x + 255) / 256) : 0);
   switch (L.epi) {
-    case EPI_BF16: return launch_tc2<EPI_BF16>(maps, p, L.max_tiles, stream);
-    case EPI_SQRELU: return launch_tc2<EPI_SQRELU>(maps, p, L.max_tiles, stream);
-    case EPI_GATE: return launch_tc2<EPI_GATE>(maps, p, L.max_tiles, stream);
+    case EPI_BF16: return launch_tc2<EPI_BF16>(maps, p, tiles, stream);
+    case EPI_SQRELU: return launch_tc2<EPI_SQRELU>(maps, p, tiles, stream);
+    case EPI_GATE: return launch_tc2<EPI_GATE>(maps, p, tiles, stream);
   }
   return LMOE_ERR_INVALID_ARG;
 }

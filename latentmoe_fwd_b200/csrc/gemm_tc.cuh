@@ -60,6 +60,14 @@ struct TcParams {
   long long ld_res;
   int ksplit;                 // >1: split the K blocks of every tile; partial sums go to `partial`
   float* partial;             // [ksplit][rows][cols] fp32 (split-K only)
+  // CTA-pair grouped launches only: one dense problem computed in the same
+  // launch, out_x[rows_x, cols_x] = epi(X[rows_x, K_x] . Wx[cols_x, K_x]^T)
+  int rows_x;                 // 0: none
+  int cols_x;
+  int kblocks_x;
+  int kgroup_x;               // >0: the extra weights are [K / kgroup_x][cols_x][kgroup_x] (K split in groups)
+  void* out_x;
+  long long ld_out_x;
   DevErr err;
 };
 

@@ -107,18 +107,44 @@ struct Tc2Smem {
 };
 
 // Pair tile t: expert e, token tile tt (256 tokens), weight tile of 256
-// features; the weight tiles of one token tile are consecutive.
+// features; the weight tiles of one token tile are consecutive. With a dense
+// extra problem its tiles are spread evenly among the grouped ones (tile i is
+// an extra tile when floor((i+1) Tx / n) > floor(i Tx / n)), so that its
+// tensor work overlaps the weight streaming of the grouped tiles.
 struct Tile2 {
   int valid;
+  int extra;   // 1: a tile of the dense extra problem
   int expert;
-  int act0;    // first padded token row of the tile
+  int act0;    // first token row of the tile (padded grouped row, or row of X)
   int act_n;   // tokens in the tile
   int w0;      // first feature of the pair's 256
   int n;       // MMA N: act_n rounded up to 32
+  int kblocks;
 };
 
-__device__ __forceinline__ Tile2 tc2_tile(const TcParams& p, int t, const int* prefix) {
+__device__ __forceinline__ int tc2_extra_tiles(const TcParams& p) {
+  return p.rows_x > 0 ? ((p.rows_x + 255) / 256) * ((p.cols_x + 255) / 256) : 0;
+}
+
+__device__ __forceinline__ Tile2 tc2_tile(const TcParams& p, int i, int ntiles, int nextra, const int* prefix) {
   Tile2 ti;
+  const long long before = static_cast<long long>(i) * nextra / ntiles;
+  if (nextra > 0 && static_cast<long long>(i + 1) * nextra / ntiles > before) {
+    const int j = static_cast<int>(before);
+    const int ntw = (p.cols_x + 255) / 256;
+    ti.extra = 1;
+    ti.expert = 0;
+    ti.w0 = (j % ntw) * 256;
+    ti.act0 = (j / ntw) * Tc2Smem::kTokens;
+    ti.act_n = min(Tc2Smem::kTokens, p.rows_x - ti.act0);
+    ti.valid = ti.act_n > 0;
+    ti.n = (ti.act_n + 31) & ~31;
+    ti.kblocks = p.kblocks_x;
+    return ti;
+  }
+  const int t = i - static_cast<int>(before);
+  ti.extra = 0;
+  ti.kblocks = p.seg[0].kblocks;
   const int ntw = (p.cols + 255) / 256;
   int lo = 0, hi = p.groups - 1;   // largest e with prefix[e] <= t
   while (lo < hi) {
@@ -138,12 +164,15 @@ __device__ __forceinline__ Tile2 tc2_tile(const TcParams& p, int t, const int* p
   return ti;
 }
 
-// tmB[i]: token maps with boxes of 128 >> i rows (i = 0..3).
+// Tensor maps: [0] grouped weights (128-row boxes), [1..4] grouped token rows
+// with boxes of 128, 64, 32, 16 rows; [5..9] the same for the extra problem.
+struct Tc2Maps {
+  CUtensorMap m[10];
+};
+
 template <int EPI>
 __global__ void __launch_bounds__(192, 1)
-    tc2_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB128,
-                    const __grid_constant__ CUtensorMap tmB64, const __grid_constant__ CUtensorMap tmB32,
-                    const __grid_constant__ CUtensorMap tmB16, const TcParams p) {
+    tc2_gemm_kernel(const __grid_constant__ Tc2Maps maps, const TcParams p) {
   using S = Tc2Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -200,8 +229,12 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB128);
+    tma_prefetch_desc(&maps.m[0]);
+    tma_prefetch_desc(&maps.m[1]);
+    if (p.rows_x > 0) {
+      tma_prefetch_desc(&maps.m[5]);
+      tma_prefetch_desc(&maps.m[6]);
+    }
   }
   if (warp == 1) tmem_alloc_pair(tmem_ptr, S::kTmemCols);
   tc_fence_before();
@@ -209,8 +242,8 @@ __global__ void __launch_bounds__(192, 1)
   cluster_barrier();   // both CTAs' barriers and TMEM exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_ptr;
-  const int ntiles = prefix[p.groups];
-  const int kblocks = p.seg[0].kblocks;
+  const int nextra = tc2_extra_tiles(p);
+  const int ntiles = prefix[p.groups] + nextra;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -218,33 +251,39 @@ __global__ void __launch_bounds__(192, 1)
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
       const uint64_t pol_norm = policy_evict_normal();
-      const CUtensorMap* bmaps[4] = {&tmB128, &tmB64, &tmB32, &tmB16};
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, issued = false;
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
-        const Tile2 ti = tc2_tile(p, t, prefix);
+        const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix);
         if (!ti.valid) continue;
         const int half = ti.n >> 1;
         const int b_row0 = ti.act0 + static_cast<int>(rank) * half;
-        // weights are kept in L2 when the expert's other token tiles read them again
-        const bool wshared = ti.act0 + S::kTokens < __ldg(p.padded_offsets + ti.expert) +
-                                                         (__ldg(p.offsets + ti.expert + 1) - __ldg(p.offsets + ti.expert));
+        const CUtensorMap* amap = &maps.m[ti.extra ? 5 : 0];
+        const CUtensorMap* bmap0 = &maps.m[ti.extra ? 6 : 1];
+        // weights are kept in L2 when other token tiles read them again (the
+        // expert's next token tile; every token tile of the extra problem)
+        const bool wshared =
+            ti.extra ? p.rows_x > S::kTokens
+                     : ti.act0 + S::kTokens < __ldg(p.padded_offsets + ti.expert) +
+                                                  (__ldg(p.offsets + ti.expert + 1) - __ldg(p.offsets + ti.expert));
         const uint64_t pa = wshared ? pol_keep : pol_stream;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = 0; kb < ti.kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x2100 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStageBytes;
           uint8_t* sb = sa + S::kABytes;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::kABytes + ti.n * 128);
           const uint32_t bar = cluster_map(smem_u32(&full[stage]), 0);
           const int k = kb * 64;
-          tma_load_3d_pair(sa, &tmA, bar, k, ti.w0 + static_cast<int>(rank) * 128, ti.expert, pa);
+          const int kg = ti.extra ? p.kgroup_x : 0;   // K split over the weight tensor's groups
+          tma_load_3d_pair(sa, amap, bar, kg ? k % kg : k, ti.w0 + static_cast<int>(rank) * 128,
+                           kg ? k / kg : ti.expert, pa);
           int done = 0;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int box = 128 >> i;
             if (half - done >= box) {
-              tma_load_3d_pair(sb + done * 128, bmaps[i], bar, k, b_row0 + done, 0, pol_norm);
+              tma_load_3d_pair(sb + done * 128, bmap0 + i, bar, k, b_row0 + done, 0, pol_norm);
               done += box;
             }
           }
@@ -267,14 +306,14 @@ __global__ void __launch_bounds__(192, 1)
       int local = 0;
       bool ok = true, any = false;
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
-        const Tile2 ti = tc2_tile(p, t, prefix);
+        const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix);
         if (!ti.valid) continue;
         const int acc = local & 1;
         if (!mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.err, 0x2200 + acc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
         const uint32_t idesc = idesc_bf16_f32(256, ti.n);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = 0; kb < ti.kblocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x2300 + stage)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
@@ -303,13 +342,17 @@ __global__ void __launch_bounds__(192, 1)
     const int r = q * 32 + lane;   // feature row of this thread within the CTA's 128
     int local = 0;
     for (int t = cluster; t < ntiles; t += nclusters) {
-      const Tile2 ti = tc2_tile(p, t, prefix);
+      const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix);
       if (!ti.valid) continue;
       const int acc = local & 1;
       if (!mbar_wait(&tfull[acc], (local >> 1) & 1, abort_flag, p.err, 0x2400 + acc)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
       const int wbase = ti.w0 + static_cast<int>(rank) * 128;
+      const int cols = ti.extra ? p.cols_x : p.cols;
+      __nv_bfloat16* const out = reinterpret_cast<__nv_bfloat16*>(ti.extra ? p.out_x : p.out);
+      const long long ld_out = ti.extra ? p.ld_out_x : p.ld_out;
+      const float* const row_scale = ti.extra ? nullptr : p.row_scale;
       const int nchunks = (ti.act_n + 31) / 32;
       __nv_bfloat16* tb = epi_tile + q * 32 * 32;
 #pragma unroll 1
@@ -321,9 +364,9 @@ __global__ void __launch_bounds__(192, 1)
         // 32 x 32 block through shared memory so each token's 32 features go
         // out as 16-byte stores
         float gate = 1.0f;
-        if (EPI == EPI_GATE && p.row_scale) {
+        if (EPI == EPI_GATE && row_scale) {
           const int tk = c * 32 + lane;
-          gate = tk < ti.act_n ? __ldg(p.row_scale + ti.act0 + tk) : 0.0f;
+          gate = tk < ti.act_n ? __ldg(row_scale + ti.act0 + tk) : 0.0f;
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -343,10 +386,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = 0; i < 4; ++i) {
           const int j = (lane >> 2) + 8 * i;
           const int tok = c * 32 + j;
-          if (tok < ti.act_n && col0 < p.cols) {
+          if (tok < ti.act_n && col0 < cols) {
             const uint4 u = *reinterpret_cast<const uint4*>(tb + j * 32 + seg * 8);
-            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (ti.act0 + tok) * p.ld_out + col0;
-            *reinterpret_cast<uint4*>(o) = u;
+            *reinterpret_cast<uint4*>(out + (ti.act0 + tok) * ld_out + col0) = u;
           }
         }
         __syncwarp();

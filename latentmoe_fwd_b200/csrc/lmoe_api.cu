@@ -83,7 +83,7 @@ struct Layout {
   size_t splitk = 0;        // fp32 split-K partial sums of the weight-major dense GEMMs (T <= 64)
   size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0,
          offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, scratch = 0, gate = 0, zp = 0,
-         zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, total = 0;
+         zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, ys = 0, total = 0;
 };
 
 Layout layout(const lmoe_config* c, int op) {
@@ -138,7 +138,10 @@ Layout layout(const lmoe_config* c, int op) {
     }
     L.y = take(P * c->l * ab);
     L.c = take(T * c->l * ab);
-    if (c->n_shared) L.hs = take(T * static_cast<int64_t>(c->n_shared) * c->m_shared * ab);
+    if (c->n_shared) {
+      L.hs = take(T * static_cast<int64_t>(c->n_shared) * c->m_shared * ab);
+      L.ys = take(T * c->d * ab);
+    }
   }
   L.total = off;
   return L;
@@ -326,10 +329,27 @@ namespace lmoe {
 namespace {
 
 // Routed experts on padded expert-grouped rows (BF16 or fp32 experts).
+// A dense problem that may ride along in the first expert GEMM's launch:
+// out = relu(act . wt^T)^2 (the shared experts' hidden layer).
+struct SharedHidden {
+  const void* x = nullptr;    // [T][d]
+  const void* ws1 = nullptr;  // [S*m_s][d]
+  int64_t d = 0;
+  int cols = 0;               // S * m_s
+  void* out = nullptr;        // [T][S*m_s]
+  bool done = false;          // set when it was computed in that launch
+  // and their output layer in the second launch: ys = hs . [Ws2_1 .. Ws2_S]^T
+  const void* ws2 = nullptr;  // [S][d][m_s]
+  int S = 0, ms = 0;
+  void* ys = nullptr;         // [T][d]
+  bool ys_done = false;
+};
+
 lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const void* zin,
                             const int32_t* offsets, const int32_t* poff, const float* gate, void* a,
                             void* y, uint32_t* err, cudaStream_t s,
-                            const std::function<void()>& between = std::function<void()>()) {
+                            const std::function<void()>& between = std::function<void()>(),
+                            SharedHidden* shared = nullptr) {
   const int64_t P = padded_rows(cfg);
   lmoe_status st;
   if (cfg->act == LMOE_F32) {
@@ -392,13 +412,25 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   const int64_t pair_token_tiles = static_cast<int64_t>(cfg->T) * cfg->K / 256 + cfg->N;
   if (pairs) {
     g1.max_tiles = pair_token_tiles * ((cfg->m + 255) / 256);
+    if (shared && shared->cols > 0) {
+      g1.x_act = TcOperand{shared->x, shared->d, cfg->T, 1};
+      g1.x_wt = TcOperand{shared->ws1, shared->d, shared->cols, 1};
+      g1.rows_x = static_cast<int>(cfg->T);
+      g1.cols_x = shared->cols;
+      g1.out_x = shared->out;
+      g1.ld_out_x = shared->cols;
+    }
     st = tc2_gemm(g1, err, s);
+    if (st == LMOE_OK && shared && shared->cols > 0) shared->done = true;
   } else {
     st = tc_gemm(g1, err, s);
   }
   if (st != LMOE_OK) return st;
   if (between) between();
   TcLaunch g2 = g1;
+  g2.rows_x = 0;   // the extra problem belongs to the first launch only
+  g2.cols_x = 0;
+  g2.out_x = nullptr;
   g2.cols = cfg->l;
   g2.kblocks[0] = kblocks(cfg->m);
   const TcOperand aop{a, cfg->m, P, 1};
@@ -419,7 +451,19 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   g2.row_scale = gate;
   if (pairs) {
     g2.max_tiles = pair_token_tiles * ((cfg->l + 255) / 256);
-    return tc2_gemm(g2, err, s);
+    const bool with_ys = shared && shared->done && shared->ys;
+    if (with_ys) {
+      g2.x_act = TcOperand{shared->out, static_cast<int64_t>(shared->S) * shared->ms, cfg->T, 1};
+      g2.x_wt = TcOperand{shared->ws2, shared->ms, shared->d, shared->S};
+      g2.x_kgroup = shared->ms;
+      g2.rows_x = static_cast<int>(cfg->T);
+      g2.cols_x = static_cast<int>(shared->d);
+      g2.out_x = shared->ys;
+      g2.ld_out_x = shared->d;
+    }
+    st = tc2_gemm(g2, err, s);
+    if (st == LMOE_OK && with_ys) shared->ys_done = true;
+    return st;
   }
   return tc_gemm(g2, err, s);
 }
@@ -508,7 +552,7 @@ lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32
   if (st != LMOE_OK) return st;
   if (!y_perm || !topk_idx || !inv_perm || !offsets || !padded_offsets || !c) return LMOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(c)) return LMOE_ERR_INVALID_ARG;
-  return launch_combine(y_perm, cfg->act, topk_idx, inv_perm, offsets, padded_offsets, topk_w, c, cfg->T,
+  return launch_combine(y_perm, cfg->act, topk_idx, inv_perm, offsets, padded_offsets, topk_w, nullptr, c, cfg->T,
                         cfg->K, cfg->l, static_cast<cudaStream_t>(stream));
 }
 
@@ -640,21 +684,40 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     return st;
   mark(3);
 
-  // 4. routed expert FFNs in l, gate applied in the second GEMM's epilogue
+  // 4. routed expert FFNs in l, gate applied in the second GEMM's epilogue; the
+  // shared experts' hidden layer (BF16) is offered to the first GEMM's launch
+  const int S = cfg->n_shared, ms = cfg->m_shared;
+  void* hs = S ? at<void>(ws, L.hs) : nullptr;
+  SharedHidden shared_hidden;
+  if (S && !f32 && !fp4) {
+    shared_hidden.x = x;
+    shared_hidden.ws1 = w->ws1;
+    shared_hidden.d = d;
+    shared_hidden.cols = S * ms;
+    shared_hidden.out = hs;
+    shared_hidden.ws2 = w->ws2;
+    shared_hidden.S = S;
+    shared_hidden.ms = ms;
+    shared_hidden.ys = at<void>(ws, L.ys);
+  }
   void* y = at<void>(ws, L.y);
   const std::function<void()> between = events ? std::function<void()>([&]() { mark(4); }) : std::function<void()>();
   if (fp4)
     st = expert_ffn_fp4(cfg, w, zp, zp_sf, z_gs, offsets, poff, gate, at<void>(ws, L.a), at<uint8_t>(ws, L.a_sf), y,
                         err, s, between);
   else
-    st = expert_ffn_impl(cfg, w, zp, offsets, poff, gate, at<void>(ws, L.a), y, err, s, between);
+    st = expert_ffn_impl(cfg, w, zp, offsets, poff, gate, at<void>(ws, L.a), y, err, s, between,
+                         shared_hidden.cols > 0 ? &shared_hidden : nullptr);
   if (st != LMOE_OK) return st;
   mark(5);
 
-  // 5. combine; with identity projections and no shared experts it is the output
-  const bool combine_is_out = ident && cfg->n_shared == 0;
+  // 5. combine; with identity projections it is the output when there are no
+  // shared experts or their output ys is already there (then combine adds it)
+  const bool ys_ready = shared_hidden.ys_done;
+  const bool combine_is_out = ident && (cfg->n_shared == 0 || ys_ready);
   void* c = combine_is_out ? out : at<void>(ws, L.c);
-  if ((st = launch_combine(y, cfg->act, idx, inv_perm, offsets, poff, nullptr, c, T, K, l, s)) != LMOE_OK)
+  if ((st = launch_combine(y, cfg->act, idx, inv_perm, offsets, poff, nullptr, ident && ys_ready ? at<void>(ws, L.ys)
+                           : nullptr, c, T, K, l, s)) != LMOE_OK)
     return st;
   mark(6);
   if (combine_is_out) {
@@ -662,10 +725,9 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     return LMOE_OK;
   }
 
-  // 6. shared experts' hidden layer on the d-dim x: hs = relu(x Ws1^T)^2, all S at once
-  const int S = cfg->n_shared, ms = cfg->m_shared;
-  void* hs = S ? at<void>(ws, L.hs) : nullptr;
-  if (S) {
+  // 6. shared experts' hidden layer on the d-dim x: hs = relu(x Ws1^T)^2, all S at
+  // once (already done when it rode along in the first expert GEMM's launch)
+  if (S && !shared_hidden.done) {
     if (f32) {
       SimtLaunch G;
       G.rows = static_cast<int>(T);
@@ -746,13 +808,18 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     ++sg;
   };
   if (!ident) add_seg(TcOperand{c, l, T, 1}, TcOperand{w->w_up, l, d, 1}, l, 0);
-  if (S) add_seg(TcOperand{hs, static_cast<int64_t>(S) * ms, T, 1}, TcOperand{w->ws2, ms, d, S},
-                 static_cast<int64_t>(S) * ms, ms);
+  if (S && !ys_ready)
+    add_seg(TcOperand{hs, static_cast<int64_t>(S) * ms, T, 1}, TcOperand{w->ws2, ms, d, S},
+            static_cast<int64_t>(S) * ms, ms);
   U.nseg = sg;
   if (ident) {
     U.epi = EPI_ADD_RES;
     U.residual = c;
     U.ld_res = l;
+  } else if (ys_ready) {   // out = c W_up^T + ys
+    U.epi = EPI_ADD_RES;
+    U.residual = at<void>(ws, L.ys);
+    U.ld_res = d;
   }
   if (sbn) {
     U.swap = 1;

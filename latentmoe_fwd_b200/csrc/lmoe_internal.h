@@ -45,6 +45,14 @@ struct TcLaunch {
   int bn = 256;
   int ksplit = 1;                // >1: split-K with fp32 partials in `partial`, then a reduction
   float* partial = nullptr;      // [ksplit][rows][cols]
+  // tc2_gemm only: a dense problem in the same launch, out_x = epi(x_act . x_wt^T)
+  TcOperand x_act = {};          // [rows_x][k] activations
+  TcOperand x_wt = {};           // [cols_x][k] weights, or [groups][cols_x][x_kgroup] with K split in groups
+  int x_kgroup = 0;
+  int rows_x = 0;
+  int cols_x = 0;
+  void* out_x = nullptr;
+  int64_t ld_out_x = 0;
 };
 
 lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream);
@@ -119,7 +127,7 @@ lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int
                           uint8_t* out_sf, int64_t padded_rows, cudaStream_t s);
 lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
                            const int32_t* offsets, const int32_t* padded_offsets, const float* w,
-                           void* c, int64_t T, int K, int l, cudaStream_t s);
+                           const void* resid, void* c, int64_t T, int K, int l, cudaStream_t s);
 lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                   const float* global_in, uint8_t* codes, uint8_t* sf,
                                   float* global_out, int sf_layout, float* partials,

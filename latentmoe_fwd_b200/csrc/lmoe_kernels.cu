@@ -576,7 +576,7 @@ template <typename TA>
 __global__ void __launch_bounds__(256) combine_kernel(
     const TA* __restrict__ y, const int32_t* __restrict__ idx, const int32_t* __restrict__ inv_perm,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, const float* __restrict__ w,
-    TA* __restrict__ c, int K, int l) {
+    const TA* __restrict__ resid, TA* __restrict__ c, int K, int l) {
   extern __shared__ int64_t rowk[];   // [K] padded rows of this token
   __shared__ float wk[64];
   const int64_t t = blockIdx.x;
@@ -609,6 +609,22 @@ __global__ void __launch_bounds__(256) combine_kernel(
         for (int i = 0; i < 4; ++i) acc[i] += g * f4[i];
       }
     }
+    if (resid) {   // + a [T, l] term (the shared experts' output) after the K routed rows
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(resid + t * l + col));
+      if constexpr (sizeof(TA) == 2) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f2 = __bfloat1622float2(h[i]);
+          acc[2 * i] += f2.x;
+          acc[2 * i + 1] += f2.y;
+        }
+      } else {
+        const float* f4 = reinterpret_cast<const float*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += f4[i];
+      }
+    }
     uint4 o;
     if constexpr (sizeof(TA) == 2) {
       o.x = pack_bf16x2(acc[0], acc[1]);
@@ -627,18 +643,18 @@ __global__ void __launch_bounds__(256) combine_kernel(
 
 lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
                            const int32_t* offsets, const int32_t* padded_offsets, const float* w,
-                           void* c, int64_t T, int K, int l, cudaStream_t s) {
+                           const void* resid, void* c, int64_t T, int K, int l, cudaStream_t s) {
   if (T == 0) return LMOE_OK;
   if (K > 64) return LMOE_ERR_UNSUPPORTED;
   const size_t sm = static_cast<size_t>(K) * sizeof(int64_t);
   if (act == LMOE_BF16)
     combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, sm, s>>>(
         static_cast<const __nv_bfloat16*>(y), idx, inv_perm, offsets, padded_offsets, w,
-        static_cast<__nv_bfloat16*>(c), K, l);
+        static_cast<const __nv_bfloat16*>(resid), static_cast<__nv_bfloat16*>(c), K, l);
   else
     combine_kernel<float><<<static_cast<unsigned>(T), 256, sm, s>>>(
         static_cast<const float*>(y), idx, inv_perm, offsets, padded_offsets, w,
-        static_cast<float*>(c), K, l);
+        static_cast<const float*>(resid), static_cast<float*>(c), K, l);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

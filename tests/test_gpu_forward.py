@@ -79,8 +79,10 @@ def test_ultra_zipf_reduced():
     _check_layer(wl, BF16_TOL)
 
 
-@pytest.mark.parametrize("T", [16, 200])
+@pytest.mark.parametrize("T", [16, 200, 700])
 def test_latent_with_shared_two_segment_up_projection(T):
+    # T = 700: CTA-pair expert GEMMs; the shared hidden layer (K = d != l) rides
+    # along in the first expert GEMM's launch
     wl = LI.Workload("latent_shared", T=T, d=384, l=128, N=8, K=2, m=256, n_shared=1, m_shared=128)
     _check_layer(wl, BF16_TOL)
 
