@@ -163,11 +163,13 @@ int kblocks(int64_t k) { return static_cast<int>((k + 63) / 64); }
 
 // out[rows, cols] = epi(x[rows, k] . W[cols, k]^T) with BF16 operands.
 // Splits for a weight-major GEMM with `tiles` output tiles and `kb` K blocks:
-// enough to fill the GPU, at least two K blocks per split, within the buffer.
+// as many as fit in one wave of the GPU (a second, partial wave would double
+// the time of a weight-streaming GEMM), at least two K blocks per split,
+// within the buffer.
 int choose_splits(int64_t tiles, int kb, int64_t rows, int64_t cols, float* partial) {
   if (!partial) return 1;
   const int sms = device_sm_count();
-  int sp = static_cast<int>((sms + tiles - 1) / tiles);
+  int sp = static_cast<int>(sms / tiles);
   if (sp > kb / 2) sp = kb / 2;
   if (sp > kMaxSplits) sp = kMaxSplits;
   return sp > 1 ? sp : 1;
