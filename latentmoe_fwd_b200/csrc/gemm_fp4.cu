@@ -53,7 +53,7 @@ static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const 
       return LMOE_ERR_CUDA;
     configured_dev = dev;
   }
-  kern<<<grid, Fp4Smem::kThreads, Fp4Smem::kBytes, s>>>(a, b, p);
+  launch_k(kern, dim3(grid), dim3(Fp4Smem::kThreads), Fp4Smem::kBytes, s, a, b, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

@@ -147,6 +147,7 @@ template <int EPI>
 __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Fp4Params p) {
+  pdl_begin();
   using S = Fp4Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

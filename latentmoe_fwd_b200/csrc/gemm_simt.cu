@@ -25,6 +25,7 @@ __device__ __forceinline__ float simt_epi(int epi, float acc, const SimtLaunch& 
 }
 
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtLaunch p) {
+  pdl_begin();
   __shared__ float sa[kSK][kST + 1];
   __shared__ float sb[kSK][kST + 1];
   const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kST;
@@ -90,7 +91,7 @@ lmoe_status simt_gemm(const SimtLaunch& L, uint32_t* err_word, cudaStream_t stre
   (void)err_word;
   if (L.rows <= 0 || L.cols <= 0) return LMOE_OK;
   dim3 grid((L.cols + kST - 1) / kST, (L.rows + kST - 1) / kST);
-  simt_gemm_kernel<<<grid, 256, 0, stream>>>(L);
+  launch_k(simt_gemm_kernel, dim3(grid), dim3(256), 0, stream, L);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

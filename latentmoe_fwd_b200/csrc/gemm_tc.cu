@@ -57,7 +57,7 @@ static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const
       return LMOE_ERR_CUDA;
     configured_dev = dev;
   }
-  kern<<<grid, 192, Sm::kBytes, s>>>(a0, b0, a1, b1, bs, p);
+  launch_k(kern, dim3(grid), dim3(192), Sm::kBytes, s, a0, b0, a1, b1, bs, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -138,10 +138,10 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   int rblocks = static_cast<int>((n + 255) / 256);
   if (rblocks > sms * 8) rblocks = sms * 8;
   switch (L.epi) {
-    case EPI_F32_BIAS: splitk_reduce_kernel<EPI_F32_BIAS><<<rblocks, 256, 0, stream>>>(p); break;
-    case EPI_BF16: splitk_reduce_kernel<EPI_BF16><<<rblocks, 256, 0, stream>>>(p); break;
-    case EPI_SQRELU: splitk_reduce_kernel<EPI_SQRELU><<<rblocks, 256, 0, stream>>>(p); break;
-    case EPI_ADD_RES: splitk_reduce_kernel<EPI_ADD_RES><<<rblocks, 256, 0, stream>>>(p); break;
+    case EPI_F32_BIAS: launch_k(splitk_reduce_kernel<EPI_F32_BIAS>, dim3(rblocks), dim3(256), 0, stream, p); break;
+    case EPI_BF16: launch_k(splitk_reduce_kernel<EPI_BF16>, dim3(rblocks), dim3(256), 0, stream, p); break;
+    case EPI_SQRELU: launch_k(splitk_reduce_kernel<EPI_SQRELU>, dim3(rblocks), dim3(256), 0, stream, p); break;
+    case EPI_ADD_RES: launch_k(splitk_reduce_kernel<EPI_ADD_RES>, dim3(rblocks), dim3(256), 0, stream, p); break;
     default: return LMOE_ERR_INVALID_ARG;
   }
   count_launch();
@@ -157,11 +157,13 @@ static lmoe_status launch_tc2(const Tc2Maps& m, const TcParams& p, int64_t max_t
   int dev = 0;
   cudaGetDevice(&dev);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Tc2Smem::kBytes;
   cfg.stream = s;
@@ -179,6 +181,7 @@ static lmoe_status launch_tc2(const Tc2Maps& m, const TcParams& p, int64_t max_t
   const int64_t clusters = max_tiles < max_clusters ? max_tiles : max_clusters;
   if (clusters <= 0) return LMOE_OK;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.numAttrs = 2;   // cluster shape + programmatic serialisation (occupancy was queried with the shape only)
   if (cudaLaunchKernelEx(&cfg, kern, m, p) != cudaSuccess) return LMOE_ERR_CUDA;
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;

@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmBs, const TcParams p) {
+  pdl_begin();
   using S = TcSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -528,6 +529,7 @@ __global__ void __launch_bounds__(192, 1)
 // Split-K reduction: out[row, col] = epi(sum over splits in order of partial[s][row][col]).
 template <int EPI>
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const TcParams p) {
+  pdl_begin();
   const long long n = static_cast<long long>(p.rows) * p.cols;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {

@@ -173,6 +173,7 @@ struct Tc2Maps {
 template <int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc2_gemm_kernel(const __grid_constant__ Tc2Maps maps, const TcParams p) {
+  pdl_begin();
   using S = Tc2Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

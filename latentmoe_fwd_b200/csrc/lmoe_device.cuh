@@ -34,6 +34,16 @@ constexpr uint32_t kErrBounds = 6;
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: wait until the preceding kernel of the
+// stream has completed and its writes are visible, then let the next kernel
+// be scheduled. Called first by every kernel, before any global access.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Shared memory addresses and mbarriers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

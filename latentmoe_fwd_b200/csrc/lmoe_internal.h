@@ -9,6 +9,27 @@
 
 namespace lmoe {
 
+// Every kernel of the library is launched with programmatic stream
+// serialisation: the next kernel's blocks may be scheduled while this one
+// finishes, and each kernel starts with griddepcontrol.wait (all of the
+// preceding grid's work and memory visible) before any global access, so
+// only the launch latency between kernels is hidden.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 void count_launch();                 // bump the library's kernel-launch counter
 int device_sm_count();               // SMs of the current device (cached per device)
 

@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
                                                                float* __restrict__ w, const TA* __restrict__ x,
                                                                const TA* __restrict__ wr,
                                                                const float* __restrict__ bias, int d) {
+  pdl_begin();
   __shared__ int s_njobs[kTopkWarps];
   __shared__ int s_expert[kTopkWarps * 32];
   __shared__ float2 s_part[kTopkPieces];
@@ -298,13 +299,12 @@ lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* i
 #define LMOE_TOPK(NPLV)                                                                                       \
   do {                                                                                                       \
     if (act == LMOE_F32)                                                                                     \
-      topk_kernel<NPLV, float><<<blocks, kTopkWarps * 32, 0, s>>>(                                           \
-          logits, T, N, K, tpb, idx, w, static_cast<const float*>(x), static_cast<const float*>(w_router),   \
-          bias, d);                                                                                          \
+      launch_k(topk_kernel<NPLV, float>, dim3(blocks), dim3(kTopkWarps * 32), 0, s, logits, T, N, K, tpb, idx, \
+               w, static_cast<const float*>(x), static_cast<const float*>(w_router), bias, d);               \
     else                                                                                                     \
-      topk_kernel<NPLV, __nv_bfloat16><<<blocks, kTopkWarps * 32, 0, s>>>(                                   \
-          logits, T, N, K, tpb, idx, w, static_cast<const __nv_bfloat16*>(x),                                \
-          static_cast<const __nv_bfloat16*>(w_router), bias, d);                                             \
+      launch_k(topk_kernel<NPLV, __nv_bfloat16>, dim3(blocks), dim3(kTopkWarps * 32), 0, s, logits, T, N, K,   \
+               tpb, idx, w, static_cast<const __nv_bfloat16*>(x),                                            \
+               static_cast<const __nv_bfloat16*>(w_router), bias, d);                                        \
   } while (0)
   if (npl <= 1) LMOE_TOPK(1);
   else if (npl <= 2) LMOE_TOPK(2);
@@ -341,6 +341,7 @@ int permute_chunks(int64_t slots, int slots_per_warp) {
 __global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx,
                                                          int64_t slots, int N, int spw,
                                                          int32_t* __restrict__ cnt, DevErr err) {
+  pdl_begin();
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -390,6 +391,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* 
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ cnt, int nchunks, int N,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ poff) {
+  pdl_begin();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   int run = 0;
@@ -432,6 +434,7 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff,
     int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm,
     const float* __restrict__ topk_w, float* __restrict__ perm_gate) {
+  pdl_begin();
   extern __shared__ int32_t wcnt[];   // [kPermWarps][N]
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kPermWarps * N; i += blockDim.x) wcnt[i] = 0;
@@ -498,15 +501,17 @@ lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t*
   const int nch = permute_chunks(slots, slots_per_warp);
   DevErr de{err};
   if (nch > 0) {
-    perm_count_kernel<<<nch, 256, N * sizeof(int32_t), s>>>(idx, slots, N, slots_per_warp, scratch, de);
+    launch_k(perm_count_kernel, dim3(nch), dim3(256), N * sizeof(int32_t), s, idx, slots, N, slots_per_warp, scratch,
+             de);
     count_launch();
   }
-  perm_scan_kernel<<<1, 1024, 0, s>>>(scratch, nch, N, offsets, padded_offsets);
+  launch_k(perm_scan_kernel, dim3(1), dim3(1024), 0, s, scratch, nch, N, offsets, padded_offsets);
   count_launch();
   if (nch > 0) {
     const size_t sm = static_cast<size_t>(kPermWarps) * N * sizeof(int32_t);
-    perm_scatter_kernel<<<nch, 256, sm, s>>>(idx, slots, N, slots_per_warp, scratch, offsets, padded_offsets,
-                                            perm_src, inv_perm, topk_w, perm_gate);
+    launch_k(perm_scatter_kernel, dim3(nch), dim3(256), sm, s, idx, slots, N, slots_per_warp,
+             static_cast<const int32_t*>(scratch), static_cast<const int32_t*>(offsets),
+             static_cast<const int32_t*>(padded_offsets), perm_src, inv_perm, topk_w, perm_gate);
     count_launch();
   }
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
@@ -527,6 +532,7 @@ __global__ void __launch_bounds__(256) gather_kernel(
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int64_t slots, int K,
     const uint8_t* __restrict__ rows, int64_t row_bytes, uint8_t* __restrict__ out,
     const uint8_t* __restrict__ rows_sf, uint8_t* __restrict__ out_sf) {
+  pdl_begin();
   const int lane = threadIdx.x & 31;
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (r >= slots) return;
@@ -570,9 +576,9 @@ lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int
   (void)padded_rows;
   if (slots == 0) return LMOE_OK;
   const int64_t blocks = (slots * 32 + 255) / 256;
-  gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-      idx, perm_src, offsets, padded_offsets, slots, K, static_cast<const uint8_t*>(rows), row_bytes,
-      static_cast<uint8_t*>(out_rows), rows_sf, out_sf);
+  launch_k(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, idx, perm_src, offsets,
+           padded_offsets, slots, K, static_cast<const uint8_t*>(rows), row_bytes, static_cast<uint8_t*>(out_rows),
+           rows_sf, out_sf);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -585,6 +591,7 @@ __global__ void __launch_bounds__(256) combine_kernel(
     const TA* __restrict__ y, const int32_t* __restrict__ idx, const int32_t* __restrict__ inv_perm,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, const float* __restrict__ w,
     const TA* __restrict__ resid, TA* __restrict__ c, int K, int l) {
+  pdl_begin();
   extern __shared__ int64_t rowk[];   // [K] padded rows of this token
   __shared__ float wk[64];
   const int64_t t = blockIdx.x;
@@ -656,13 +663,13 @@ lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int
   if (K > 64) return LMOE_ERR_UNSUPPORTED;
   const size_t sm = static_cast<size_t>(K) * sizeof(int64_t);
   if (act == LMOE_BF16)
-    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(T), 256, sm, s>>>(
-        static_cast<const __nv_bfloat16*>(y), idx, inv_perm, offsets, padded_offsets, w,
-        static_cast<const __nv_bfloat16*>(resid), static_cast<__nv_bfloat16*>(c), K, l);
+    launch_k(combine_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(T)), dim3(256), sm, s,
+             static_cast<const __nv_bfloat16*>(y), idx, inv_perm, offsets, padded_offsets, w,
+             static_cast<const __nv_bfloat16*>(resid), static_cast<__nv_bfloat16*>(c), K, l);
   else
-    combine_kernel<float><<<static_cast<unsigned>(T), 256, sm, s>>>(
-        static_cast<const float*>(y), idx, inv_perm, offsets, padded_offsets, w,
-        static_cast<const float*>(resid), static_cast<float*>(c), K, l);
+    launch_k(combine_kernel<float>, dim3(static_cast<unsigned>(T)), dim3(256), sm, s, static_cast<const float*>(y),
+             idx, inv_perm, offsets, padded_offsets, w, static_cast<const float*>(resid), static_cast<float*>(c), K,
+             l);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -689,6 +696,7 @@ __device__ __forceinline__ float load_abs_max(const TI* p, int64_t i) {
 template <typename TI>
 __global__ void __launch_bounds__(kQThreads) nvfp4_amax_kernel(const TI* __restrict__ in, int64_t n,
                                                                float* __restrict__ partials) {
+  pdl_begin();
   __shared__ float red[kQThreads / 32];
   float m = 0.0f;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -794,6 +802,7 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_encode_kernel(
     const TI* __restrict__ in, int64_t rows, int64_t cols, const float* __restrict__ partials, int np,
     const float* __restrict__ global_in, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
     float* __restrict__ global_out, int tiled) {
+  pdl_begin();
   const float s_g = cta_global_scale(partials, np, global_in);
   if (blockIdx.x == 0 && threadIdx.x == 0 && global_out) *global_out = s_g;
   const int64_t nb = cols / 16;
@@ -826,9 +835,11 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
   const int64_t n = rows * cols;
   if (!global_in) {
     if (in_dtype == LMOE_BF16)
-      nvfp4_amax_kernel<__nv_bfloat16><<<npartials, kQThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(in), n, partials);
+      launch_k(nvfp4_amax_kernel<__nv_bfloat16>, dim3(npartials), dim3(kQThreads), 0, s,
+               static_cast<const __nv_bfloat16*>(in), n, partials);
     else
-      nvfp4_amax_kernel<float><<<npartials, kQThreads, 0, s>>>(static_cast<const float*>(in), n, partials);
+      launch_k(nvfp4_amax_kernel<float>, dim3(npartials), dim3(kQThreads), 0, s, static_cast<const float*>(in), n,
+               partials);
     count_launch();
   }
   const int tiled = sf_layout == LMOE_SF_MMA_TILED;
@@ -840,13 +851,13 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
   if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
   if (blocks < 1) blocks = 1;
   if (in_dtype == LMOE_BF16)
-    nvfp4_encode_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kQThreads, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(in), rows, cols, partials, global_in ? 0 : npartials, global_in,
-        codes, sf, global_out, tiled);
+    launch_k(nvfp4_encode_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
+             static_cast<const __nv_bfloat16*>(in), rows, cols, static_cast<const float*>(partials),
+             global_in ? 0 : npartials, global_in, codes, sf, global_out, tiled);
   else
-    nvfp4_encode_kernel<float><<<static_cast<unsigned>(blocks), kQThreads, 0, s>>>(
-        static_cast<const float*>(in), rows, cols, partials, global_in ? 0 : npartials, global_in, codes,
-        sf, global_out, tiled);
+    launch_k(nvfp4_encode_kernel<float>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
+             static_cast<const float*>(in), rows, cols, static_cast<const float*>(partials), global_in ? 0 : npartials,
+             global_in, codes, sf, global_out, tiled);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
