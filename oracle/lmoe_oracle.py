@@ -198,6 +198,41 @@ def nvfp4_quantize(X, s_g: float | None = None):
     return codes, sb_code, s_g
 
 
+def nvfp4_quantize_2d(X, s_g: float | None = None):
+    """NVFP4 with two-dimensional weight blocks: one E4M3 scale per 16 rows x
+    16 columns (greeksharifa page, section 2.4 "NVFP4 Training": the recipe
+    scales weights in two-dimensional blocks; the block size is read as the
+    16-element micro-block squared, so that W and W^T quantise alike).
+
+    The block amax runs over the block's 256 elements (rows past the end of
+    X count as 0); every other step is nvfp4_quantize's. The scale is written
+    to each of the block's rows, so the result has nvfp4_quantize's layout
+    (codes [rows, cols/2], scales [rows, cols/16]) and decodes the same way.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    rows, cols = X.shape
+    assert cols % NVFP4_BLOCK == 0
+    if s_g is None:
+        s_g = nvfp4_global_scale(X)
+    s_g = float(round_f32(s_g))
+    nrb = -(-rows // NVFP4_BLOCK)
+    Xp = np.zeros((nrb * NVFP4_BLOCK, cols))
+    Xp[:rows] = X
+    amax_2d = np.max(np.abs(Xp.reshape(nrb, NVFP4_BLOCK, cols // NVFP4_BLOCK, NVFP4_BLOCK)), axis=(1, 3))
+    t = round_f32(s_g * E2M1_MAX)
+    sb_code_2d = e4m3_encode(round_f32(amax_2d / t))
+    sb_code = np.repeat(sb_code_2d, NVFP4_BLOCK, axis=0)[:rows]      # [rows, cols/16]
+    sb = e4m3_decode(sb_code)
+    sc = round_f32(sb * s_g)
+    blocks = X.reshape(rows, cols // NVFP4_BLOCK, NVFP4_BLOCK)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = round_f32(blocks / sc[..., None])
+    q = e2m1_encode(v)
+    q = np.where((sb == 0.0)[..., None], np.uint8(0), q).astype(np.uint8).reshape(rows, cols)
+    codes = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
+    return codes, sb_code.astype(np.uint8), s_g
+
+
 def nvfp4_unpack(codes) -> np.ndarray:
     codes = np.asarray(codes, dtype=np.uint8)
     out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), dtype=np.uint8)

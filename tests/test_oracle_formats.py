@@ -201,3 +201,70 @@ def test_nvfp4_zero_scale_block_is_all_zero_codes():
     codes, sf, s_g = O.nvfp4_quantize(X)
     assert sf[0, 0] == 0
     assert np.all(O.nvfp4_unpack(codes)[0, :16] == 0)
+
+
+# ---- two-dimensional (16 x 16) weight blocks ----
+
+def test_nvfp4_2d_transpose_symmetry():
+    """16 x 16 blocks quantise W and W^T alike: codes and scales transpose."""
+    rng = np.random.default_rng(11)
+    W = O.round_bf16(rng.standard_normal((48, 64)) * np.exp(rng.uniform(-3, 3, (48, 1))))
+    c, sf, g = O.nvfp4_quantize_2d(W)
+    ct, sft, gt = O.nvfp4_quantize_2d(W.T.copy())
+    assert g == gt
+    assert np.array_equal(O.nvfp4_unpack(ct), O.nvfp4_unpack(c).T)
+    i, j = np.meshgrid(np.arange(48), np.arange(64), indexing="ij")
+    assert np.array_equal(sft[j, i // 16], sf[i, j // 16])
+    # a row-wise (1 x 16) quantiser does not have this property on the same data
+    c1, sf1, _ = O.nvfp4_quantize(W)
+    c1t, _, _ = O.nvfp4_quantize(W.T.copy())
+    assert not np.array_equal(O.nvfp4_unpack(c1t), O.nvfp4_unpack(c1).T)
+
+
+def test_nvfp4_2d_equals_1d_when_block_rows_repeat():
+    rng = np.random.default_rng(12)
+    base = O.round_bf16(rng.standard_normal((3, 80)))
+    W = np.repeat(base, 16, axis=0)               # every 16-row block: one row repeated
+    c2, s2, g2 = O.nvfp4_quantize_2d(W)
+    c1, s1, g1 = O.nvfp4_quantize(W)
+    assert g1 == g2 and np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+@pytest.mark.parametrize("s_g", [1.0, 2.0 ** -4])
+def test_nvfp4_2d_round_trip_exact(s_g):
+    """Blocks of grid points times a power-of-two block scale, one entry +-6 per
+    16 x 16 block: every fp32 step is exact and the round trip is the identity."""
+    rng = np.random.default_rng(13)
+    rows, cols = 32, 48
+    X = np.zeros((rows, cols))
+    for rb in range(rows // 16):
+        for cb in range(cols // 16):
+            sb = 2.0 ** rng.integers(-5, 8)
+            q = rng.choice(O.E2M1_MAG, (16, 16)) * rng.choice([-1.0, 1.0], (16, 16))
+            q[rng.integers(16), rng.integers(16)] = 6.0
+            X[rb * 16:(rb + 1) * 16, cb * 16:(cb + 1) * 16] = q * sb * s_g
+    codes, sf, g = O.nvfp4_quantize_2d(X, s_g)
+    assert np.array_equal(O.nvfp4_dequantize(codes, sf, g), X)
+
+
+def test_nvfp4_2d_brute_force_ragged_rows():
+    """Rows not a multiple of 16: the last block's scale comes from its rows
+    only; every scale and code checked element by element."""
+    rng = np.random.default_rng(14)
+    W = O.round_bf16(rng.standard_normal((21, 32)) * np.exp(rng.uniform(-2, 2, (21, 2)).repeat(16, axis=1)))
+    codes, sf, s_g = O.nvfp4_quantize_2d(W)
+    q = O.nvfp4_unpack(codes)
+    for rb in range(2):
+        r0, r1 = rb * 16, min(21, rb * 16 + 16)
+        for cb in range(2):
+            blk = W[r0:r1, cb * 16:(cb + 1) * 16]
+            amax = np.float32(np.max(np.abs(blk)))
+            r_f32 = np.float32(amax / np.float32(np.float32(s_g) * np.float32(6.0)))
+            code = torch.tensor([float(r_f32)]).to(torch.float8_e4m3fn).view(torch.uint8).item()
+            assert np.all(sf[r0:r1, cb] == code)
+            sb = O.e4m3_decode(code)
+            sc = np.float32(np.float32(sb) * np.float32(s_g))
+            for r in range(r0, r1):
+                for i in range(16):
+                    v = float(np.float32(np.float32(W[r, cb * 16 + i]) / sc)) if sb != 0 else 0.0
+                    assert q[r, cb * 16 + i] == (_brute_e2m1(v) if sb != 0 else 0)
