@@ -201,6 +201,41 @@ def quantize_experts(L, w):
     return codes, sf, gs
 
 
+def quantizer_rates(L, w, hbm_gbs):
+    """lmoe_nvfp4_quantize over all experts' W1 as one [N*rows, cols] matrix
+    (current amax, MMA-tiled scales), with 1 x 16 and with 16 x 16 scale
+    blocks: ms per call and the rate on its algorithmic bytes (the amax pass
+    reads the input, the encode pass reads it again and writes codes and
+    scales: 2 + 2 + 0.5625 bytes per element)."""
+    import torch
+    N, rows, cols = w.shape
+    R = N * rows
+    flat = w.reshape(R, cols)
+    codes = torch.empty((R, cols // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((((R + 127) // 128) * 128 * (cols // 16),), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = L.workspace(L.config(T=R, d=cols, l=cols, N=1, K=1, m=cols), L.OP_NVFP4_QUANTIZE)
+    alg = R * cols * (2 + 2 + 0.5625)
+    out = {"rows": R, "cols": cols, "algorithmic_bytes": alg}
+    for name, layout in (("1x16", L.SF_MMA_TILED), ("16x16", L.SF_MMA_TILED | L.SF_BLOCK_16X16)):
+        L.nvfp4_quantize(flat, L.BF16, R, cols, None, codes, sf, g, layout, ws)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        a.record()
+        for _ in range(reps):
+            L.nvfp4_quantize(flat, L.BF16, R, cols, None, codes, sf, g, layout, ws)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        gbs = alg / (ms / 1000.0) / 1e9
+        out[name] = {"ms": ms, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs}
+    st, info = L.read_device_error(ws)
+    if st != L.OK:
+        raise RuntimeError(f"quantiser measurement failed: {L.status_string(st)}")
+    return out
+
+
 # --------------------------------------------------------------------------
 # the CPU oracle, timed (bounded sample)
 # --------------------------------------------------------------------------
@@ -332,8 +367,11 @@ def main():
                    act=L.F32 if st == "f32" else L.BF16,
                    expert={"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype], identity=wl.identity)
     extra = {}
+    quant = None
     if wl.dtype == "nvfp4":
         # setup, not timed: NVFP4 expert weights (per-matrix global scale, MMA-tiled block scales)
+        # the quantiser's own rate, on the BF16 W1 before it is replaced (outside the timed region)
+        quant = quantizer_rates(L, t["w1"], load_peaks()[0]["hbm_gbs"]) if rank == 0 and world == 1 else None
         for key in ("w1", "w2"):
             codes, sf, gs = quantize_experts(L, t[key])
             t[key] = codes
@@ -497,6 +535,8 @@ def main():
             "clocks": clocks,
             "stage_ms": {n: float(v) for n, v in zip(L.TRACE_STAGES, stage_ms)},
         }
+        if quant is not None:
+            line["nvfp4_quantize"] = quant
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -70,6 +70,14 @@ typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1, LMOE_NVFP4 = 2 } lmoe_dtype;
  *   multiple of 128 and cols to a multiple of 64 (padding bytes are written 0). */
 typedef enum { LMOE_SF_ROWMAJOR = 0, LMOE_SF_MMA_TILED = 1 } lmoe_sf_layout;
 
+/* OR-ed into lmoe_nvfp4_quantize's sf_layout: two-dimensional scale blocks of
+ * 16 rows x 16 columns (the greeksharifa page on the Nemotron 3 whitepaper,
+ * section 2.4 "NVFP4 Training": the recipe scales weights in 2-D blocks, so a
+ * matrix and its transpose quantise alike). Each block's scale is the E4M3
+ * rounding of its 256-element amax / (6 s_g) and is stored in every one of its
+ * rows' 1 x 16 entries, so GEMMs and decoders read the result unchanged. */
+#define LMOE_SF_BLOCK_16X16 0x10
+
 /* Flag: l == d and there is no down/up projection (the standard-MoE limit). */
 #define LMOE_FLAG_IDENTITY_PROJ 1u
 
@@ -243,7 +251,11 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
  *  per 16-block: s_b = E4M3_satfinite_rn(amax_b / (s_g * 6));
  *  q_i = E2M1_satfinite_rn(x_i / (dec(s_b) * s_g)) (all codes +0 if dec(s_b) == 0).
  *  codes [rows][cols/2] (low nibble first), sf per sf_layout, global_out
- *  (device F32, may be NULL) receives s_g. global_in: device pointer or NULL. */
+ *  (device F32, may be NULL) receives s_g. global_in: device pointer or NULL.
+ *  sf_layout | LMOE_SF_BLOCK_16X16: amax_b over 16 x 16 blocks instead (rows
+ *  need not be a multiple of 16: the last block has the remaining rows).
+ *  Errors: LMOE_ERR_INVALID_ARG for null pointers, cols % 16, an unknown
+ *  layout, an unaligned input (16 B) or code buffer (8 B). */
 lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                 const float* global_in, uint8_t* codes, uint8_t* sf,
                                 float* global_out, int sf_layout, void* ws, size_t ws_bytes,

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(HERE, "liblmoe.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_DEVICE_BOUNDS = range(7)
 F32, BF16, NVFP4 = 0, 1, 2
 SF_ROWMAJOR, SF_MMA_TILED = 0, 1
+SF_BLOCK_16X16 = 0x10          # OR into the layout: 16 x 16 scale blocks
 FLAG_IDENTITY_PROJ = 1
 OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE = range(6)
 

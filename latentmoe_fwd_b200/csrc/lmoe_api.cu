@@ -564,7 +564,8 @@ lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int6
   if (!in || !codes || !sf) return LMOE_ERR_INVALID_ARG;
   if (rows < 0 || cols <= 0 || cols % 16) return LMOE_ERR_INVALID_ARG;
   if (in_dtype != LMOE_F32 && in_dtype != LMOE_BF16) return LMOE_ERR_INVALID_ARG;
-  if (sf_layout != LMOE_SF_ROWMAJOR && sf_layout != LMOE_SF_MMA_TILED) return LMOE_ERR_INVALID_ARG;
+  const int base_layout = sf_layout & ~LMOE_SF_BLOCK_16X16;
+  if (base_layout != LMOE_SF_ROWMAJOR && base_layout != LMOE_SF_MMA_TILED) return LMOE_ERR_INVALID_ARG;
   if (!aligned16(in) || (reinterpret_cast<uintptr_t>(codes) & 7)) return LMOE_ERR_INVALID_ARG;
   lmoe_config q{};
   q.T = rows;

@@ -827,6 +827,58 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_encode_kernel(
   }
 }
 
+// Two-dimensional blocks: one thread per 16-row group x 16-column block. The
+// scale comes from the amax over the block's (up to) 256 elements; each of its
+// rows is then quantised with it and carries it in its own scale entry, so
+// the output has the 1 x 16 layout and every consumer reads it unchanged.
+template <typename TI>
+__global__ void __launch_bounds__(kQThreads) nvfp4_encode2d_kernel(
+    const TI* __restrict__ in, int64_t rows, int64_t cols, const float* __restrict__ partials, int np,
+    const float* __restrict__ global_in, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+    float* __restrict__ global_out, int tiled) {
+  pdl_begin();
+  const float s_g = cta_global_scale(partials, np, global_in);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && global_out) *global_out = s_g;
+  const int64_t nb = cols / 16;
+  const int64_t rows_cov = tiled ? ((rows + 127) / 128) * 128 : rows;
+  const int64_t nb_cov = tiled ? ((cols + 63) / 64) * 4 : nb;
+  const int groups64 = static_cast<int>((cols + 63) / 64);
+  const int64_t total = ((rows_cov + 15) / 16) * nb_cov;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r0 = (b / nb_cov) * 16, j = b % nb_cov;
+    const int64_t r1 = r0 + 16 < rows_cov ? r0 + 16 : rows_cov;
+    const int nr = (j < nb && r0 < rows) ? static_cast<int>(rows - r0 < 16 ? rows - r0 : 16) : 0;
+    uint32_t scode = 0;
+    if (nr > 0) {
+      float x[16];
+      float amax = 0.0f;
+      for (int i = 0; i < nr; ++i) {
+        load16<TI>(in + (r0 + i) * cols + j * 16, x);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      }
+      scode = cvt_e4m3(__fdiv_rn(amax, __fmul_rn(s_g, 6.0f)));
+      const float dec = e4m3_value(scode);
+      const float sc = __fmul_rn(dec, s_g);
+      const float rc = dec != 0.0f ? __frcp_rn(sc) : 0.0f;
+      for (int i = 0; i < nr; ++i) {
+        uint2 c = make_uint2(0u, 0u);
+        if (dec != 0.0f) {
+          load16<TI>(in + (r0 + i) * cols + j * 16, x);
+          c = e2m1_codes16(x, sc, rc);   // codes of RN(x / sc)
+        }
+        *reinterpret_cast<uint2*>(codes + (r0 + i) * (cols / 2) + j * 8) = c;
+      }
+    }
+    for (int64_t r = r0; r < r1; ++r) {
+      const uint8_t v = (r < rows && j < nb) ? static_cast<uint8_t>(scode) : 0;
+      if (tiled) sf[sf_tiled_offset(r, static_cast<int>(j), groups64)] = v;
+      else sf[r * nb + j] = v;
+    }
+  }
+}
+
 lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                   const float* global_in, uint8_t* codes, uint8_t* sf,
                                   float* global_out, int sf_layout, float* partials, int npartials,
@@ -842,15 +894,25 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
                partials);
     count_launch();
   }
-  const int tiled = sf_layout == LMOE_SF_MMA_TILED;
+  const bool blk2d = (sf_layout & LMOE_SF_BLOCK_16X16) != 0;
+  const int tiled = (sf_layout & ~LMOE_SF_BLOCK_16X16) == LMOE_SF_MMA_TILED;
   const int64_t rows_cov = tiled ? ((rows + 127) / 128) * 128 : rows;
   const int64_t nb_cov = tiled ? ((cols + 63) / 64) * 4 : cols / 16;
-  const int64_t total = rows_cov * nb_cov;
+  const int64_t total = (blk2d ? (rows_cov + 15) / 16 : rows_cov) * nb_cov;
   const int sms = device_sm_count();
   int64_t blocks = (total + kQThreads - 1) / kQThreads;
   if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
   if (blocks < 1) blocks = 1;
-  if (in_dtype == LMOE_BF16)
+  if (blk2d) {
+    if (in_dtype == LMOE_BF16)
+      launch_k(nvfp4_encode2d_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
+               static_cast<const __nv_bfloat16*>(in), rows, cols, static_cast<const float*>(partials),
+               global_in ? 0 : npartials, global_in, codes, sf, global_out, tiled);
+    else
+      launch_k(nvfp4_encode2d_kernel<float>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
+               static_cast<const float*>(in), rows, cols, static_cast<const float*>(partials),
+               global_in ? 0 : npartials, global_in, codes, sf, global_out, tiled);
+  } else if (in_dtype == LMOE_BF16)
     launch_k(nvfp4_encode_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
              static_cast<const __nv_bfloat16*>(in), rows, cols, static_cast<const float*>(partials),
              global_in ? 0 : npartials, global_in, codes, sf, global_out, tiled);

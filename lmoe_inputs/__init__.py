@@ -57,6 +57,7 @@ class Workload:
     identity: bool = False       # l == d, no down/up projection
     zipf_bias: bool = False
     outliers: bool = False
+    w_block2d: bool = False      # nvfp4: expert weights scaled in 16 x 16 blocks
     seed: int = 0
 
     def as_dict(self):

@@ -359,11 +359,12 @@ class _Weights:
     def expert(self, key, e):
         """fp64 values of expert e's matrix as the GEMM sees them."""
         if self.wl.dtype == "nvfp4":
+            quant = nvfp4_quantize_2d if getattr(self.wl, "w_block2d", False) else nvfp4_quantize
             if self._q is not None:
                 if (key, e) not in self._q:
-                    self._q[(key, e)] = nvfp4_quantize(to_f64(self.inp[key][e], self.st))
+                    self._q[(key, e)] = quant(to_f64(self.inp[key][e], self.st))
                 return nvfp4_dequantize(*self._q[(key, e)])
-            return nvfp4_fake_quant(to_f64(self.inp[key][e], self.st))[0]
+            return nvfp4_dequantize(*quant(to_f64(self.inp[key][e], self.st)))
         return to_f64(self.inp[key][e], self.st)
 
 

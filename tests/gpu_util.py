@@ -28,7 +28,7 @@ def cfg_of(wl, T=None):
 def quantize_dev(x: torch.Tensor, rows: int, cols: int, layout=L.SF_ROWMAJOR, global_in=None):
     """lmoe_nvfp4_quantize on a device tensor: (codes, sf, global scale)."""
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
-    if layout == L.SF_MMA_TILED:
+    if (layout & ~L.SF_BLOCK_16X16) == L.SF_MMA_TILED:
         sf = torch.empty((((rows + 127) // 128) * 128 * ((cols + 63) // 64) * 4,), dtype=torch.uint8, device="cuda")
     else:
         sf = torch.empty((rows, cols // 16), dtype=torch.uint8, device="cuda")
@@ -41,14 +41,16 @@ def quantize_dev(x: torch.Tensor, rows: int, cols: int, layout=L.SF_ROWMAJOR, gl
     return codes, sf, g
 
 
-def quantize_experts_dev(w: torch.Tensor):
-    """Per-expert NVFP4 weights [N][rows][cols] with MMA-tiled scales."""
+def quantize_experts_dev(w: torch.Tensor, block2d: bool = False):
+    """Per-expert NVFP4 weights [N][rows][cols] with MMA-tiled scales (16 x 16
+    scale blocks with block2d)."""
     N, rows, cols = w.shape
     codes = torch.empty((N, rows, cols // 2), dtype=torch.uint8, device="cuda")
     sf = torch.empty((N, rows * cols // 16), dtype=torch.uint8, device="cuda")
     gs = torch.empty(N, dtype=torch.float32, device="cuda")
+    layout = L.SF_MMA_TILED | (L.SF_BLOCK_16X16 if block2d else 0)
     for e in range(N):
-        c, f, g = quantize_dev(w[e], rows, cols, L.SF_MMA_TILED)
+        c, f, g = quantize_dev(w[e], rows, cols, layout)
         codes[e].copy_(c)
         sf[e].copy_(f)
         gs[e:e + 1].copy_(g)
@@ -68,8 +70,8 @@ class DevLayer:
         self.cfg = cfg_of(wl)
         extra = {}
         if wl.dtype == "nvfp4":
-            c1, f1, g1 = quantize_experts_dev(self.t["w1"])
-            c2, f2, g2 = quantize_experts_dev(self.t["w2"])
+            c1, f1, g1 = quantize_experts_dev(self.t["w1"], wl.w_block2d)
+            c2, f2, g2 = quantize_experts_dev(self.t["w2"], wl.w_block2d)
             a_gs = torch.tensor([inp["a_global_scale"]], dtype=torch.float32, device="cuda")
             self.t.update(w1=c1, w2=c2)
             extra = dict(w1_sf=f1, w2_sf=f2, w1_gs=g1, w2_gs=g2, a_global_scale=a_gs)

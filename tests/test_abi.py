@@ -103,3 +103,14 @@ def test_launch_counter_starts_and_is_monotone():
     a = L.kernel_launch_count()
     b = L.kernel_launch_count()
     assert b >= a >= 0
+
+
+def test_nvfp4_quantize_layout_flags():
+    src = open(os.path.join(ROOT, "include", "lmoe.h")).read()
+    assert "#define LMOE_SF_BLOCK_16X16 0x10" in src
+    assert L.SF_BLOCK_16X16 == 0x10
+    ws = ctypes.create_string_buffer(4096)
+    fake = ctypes.c_void_p(4096)   # never dereferenced: the layout is rejected first
+    for bad in (2, 3, 0x20, 0x12):
+        st = L.lib.lmoe_nvfp4_quantize(fake, 1, 16, 16, None, fake, fake, None, bad, ws, 4096, None)
+        assert st == L.ERR_INVALID_ARG

@@ -247,3 +247,60 @@ def test_quantize_codes_at_e2m1_boundaries_with_irregular_scales():
     rc, rsf, _ = O.nvfp4_quantize(v.astype(np.float64), float(s_g))
     assert np.array_equal(sf.cpu().numpy(), rsf)
     assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+# ---- two-dimensional (16 x 16) weight scale blocks ----
+
+@pytest.mark.parametrize("rows,cols", [(48, 64), (21, 96), (300, 2048), (1, 16)])
+def test_quantize_2d_bit_exact(rows, cols):
+    rng = np.random.default_rng(rows * 17 + cols)
+    v = rng.standard_normal((rows, cols)) * np.exp(rng.uniform(-3, 3, (rows, 1)))
+    x, xv = _bf16_dev(v)
+    codes, sf, g = quantize_dev(x, rows, cols, L.SF_ROWMAJOR | L.SF_BLOCK_16X16)
+    rc, rsf, rg = O.nvfp4_quantize_2d(xv)
+    assert g.item() == np.float32(rg)
+    assert np.array_equal(sf.cpu().numpy(), rsf)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+def test_quantize_2d_f32_input_given_global_and_tiled_layout():
+    rng = np.random.default_rng(21)
+    rows, cols = 200, 320                       # ragged last 16-row block and 128-row tile
+    v = (rng.standard_normal((rows, cols)) * 3).astype(np.float32)
+    x = torch.from_numpy(v).cuda()
+    gin = torch.tensor([0.0071], dtype=torch.float32, device="cuda")
+    codes, sf, g = quantize_dev(x, rows, cols, L.SF_MMA_TILED | L.SF_BLOCK_16X16, global_in=gin)
+    rc, rsf, rg = O.nvfp4_quantize_2d(v.astype(np.float64), float(np.float32(0.0071)))
+    assert g.item() == np.float32(rg)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    sfn = sf.cpu().numpy()
+    assert np.array_equal(_tiled_to_rowmajor(sfn, rows, cols), rsf)
+    # padding rows of the last 128-row tile carry zero scales
+    pad = np.ones(sfn.shape, dtype=bool)
+    r = np.arange(rows)[:, None]
+    j = np.arange(cols // 16)[None, :]
+    g64 = (cols + 63) // 64
+    pad[((r >> 7) * g64 + (j >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3)] = False
+    assert np.all(sfn[pad] == 0)
+
+
+def test_quantize_2d_transpose_property_on_device():
+    rng = np.random.default_rng(22)
+    v = rng.standard_normal((64, 96)) * np.exp(rng.uniform(-2, 2, (64, 1)))
+    x, xv = _bf16_dev(v)
+    xt = x.t().contiguous()
+    c, sf, g = quantize_dev(x, 64, 96, L.SF_ROWMAJOR | L.SF_BLOCK_16X16)
+    ct, sft, gt = quantize_dev(xt, 96, 64, L.SF_ROWMAJOR | L.SF_BLOCK_16X16)
+    assert g.item() == gt.item()
+    assert np.array_equal(O.nvfp4_unpack(ct.cpu().numpy()), O.nvfp4_unpack(c.cpu().numpy()).T)
+    i, jj = np.meshgrid(np.arange(64), np.arange(96), indexing="ij")
+    assert np.array_equal(sft.cpu().numpy()[jj, i // 16], sf.cpu().numpy()[i, jj // 16])
+
+
+@pytest.mark.parametrize("T", [130, 700])
+def test_nvfp4_forward_with_16x16_weight_blocks(T):
+    # the block-scaled GEMMs read 2-D-scaled weights unchanged (their scales
+    # repeated over each block's 16 rows); parity against the oracle with the
+    # same 2-D quantisation of W1 and W2
+    wl = LI.reduced("ultra_nvfp4", T=T, d=512, l=256, N=16, K=4, m=512, w_block2d=True)
+    _nvfp4_layer(wl)
