@@ -512,7 +512,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n = args.cpu_sample or {"tiny_f32": 64, "std_moe_bf16": 128, "ultra_decode": 32, "ultra_zipf": 32,
-                                "ultra_nvfp4": 16}.get(wl.name, 32)
+                                "ultra_nvfp4": 16, "ultra_decode_nvfp4": 16}.get(wl.name, 32)
         v, dt, ntok = oracle_tokens_per_s(wl, inp, n)
         cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{ntok} random tokens of the {wl.name} batch, full weights, fp64 NumPy "

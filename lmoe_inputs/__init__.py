@@ -16,6 +16,7 @@ limit uses l=d with 128 experts, 6 active and two always-on shared experts):
 * ``ultra_zipf``      T=16384, same shapes, additive Zipf(1.1) router bias
 * ``ultra_nvfp4``     T=8192,  same shapes, NVFP4 experts and latent
                       activations, 0.1% of x scaled by 50
+* ``ultra_decode_nvfp4`` T=32, the same NVFP4 layer in decode
 
 Recipe (every tensor from its own ``SeedSequence`` child, so generation order
 and thread count do not change any value):
@@ -74,6 +75,8 @@ WORKLOADS = {
                            dtype="bf16", zipf_bias=True),
     "ultra_nvfp4": Workload("ultra_nvfp4", T=8192, d=8192, l=2048, N=512, K=22, m=1024,
                             dtype="nvfp4", outliers=True),
+    "ultra_decode_nvfp4": Workload("ultra_decode_nvfp4", T=32, d=8192, l=2048, N=512, K=22, m=1024,
+                                   dtype="nvfp4", outliers=True),
 }
 
 
