@@ -374,8 +374,9 @@ def main():
         quant = quantizer_rates(L, t["w1"], load_peaks()[0]["hbm_gbs"]) if rank == 0 and world == 1 else None
         for key in ("w1", "w2"):
             codes, sf, gs = quantize_experts(L, t[key])
-            t[key] = codes
+            t[key] = codes                         # the BF16 copy is released
             extra[key + "_sf"], extra[key + "_gs"] = sf, gs
+        torch.cuda.empty_cache()
         extra["a_global_scale"] = torch.tensor([inp["a_global_scale"]], dtype=torch.float32, device="cuda")
         torch.cuda.synchronize()
     w = L.weights(w_router=t["w_router"], router_bias=bias, w_down=t["w_down"], w_up=t["w_up"], w1=t["w1"],

@@ -95,6 +95,7 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
     maps[4] = maps[1];
   }
   if (L.grouped && L.groups > 1024) return LMOE_ERR_UNSUPPORTED;
+  if (L.grouped && !L.swap) return LMOE_ERR_INVALID_ARG;   // grouped tiles are weight-major
   TcParams p = {};
   p.swap = L.swap;
   p.grouped = L.grouped;

@@ -13,12 +13,13 @@
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
 //
 // Tile kinds:
-//   normal: A = activation rows (128 per tile), B = weight rows (BN per tile).
+//   normal: A = activation rows (128 per tile), B = weight rows (BN per tile);
+//           dense GEMMs only.
 //   swap:   A = weight rows (128 per tile), B = activation rows (<= BN tokens);
 //           used when the token count is tiny and the GEMM streams weights.
-//   grouped: activation rows are the expert-grouped padded buffer (each
-//           expert's rows start at a multiple of 128); the weight operand is a
-//           3-D map [experts][rows][K] indexed by the tile's expert.
+//   grouped (swap only): activation rows are the expert-grouped padded buffer;
+//           the weight operand is a 3-D map [experts][rows][K] indexed by the
+//           tile's expert.
 // Up to two K segments are summed into one accumulator (used for
 // out = c W_up^T + sum_s as_s Ws2_s^T).
 #pragma once
@@ -133,8 +134,7 @@ __device__ __forceinline__ int tc_num_tiles(const TcParams& p, const int* prefix
   const int ntw_swap = (p.cols + 127) / 128;
   int n;
   if (!p.swap) {
-    int mt = p.grouped ? (__ldg(p.padded_offsets + p.groups) >> 7) : (p.rows + 127) / 128;
-    n = mt * ntw_normal;
+    n = ((p.rows + 127) / 128) * ntw_normal;
   } else {
     n = p.grouped ? prefix[p.groups] : ntw_swap;
   }
@@ -160,16 +160,7 @@ __device__ __forceinline__ TileInfo tc_tile(const TcParams& p, int t, int kb_tot
     const int nt = t % ntw, mt = t / ntw;
     ti.w0 = nt * BN;
     ti.act0 = mt * 128;
-    if (p.grouped) {
-      const int e = find_expert(p.padded_offsets, p.groups, ti.act0);
-      const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
-      const int end = __ldg(p.padded_offsets + e) + n_e;
-      ti.expert = e;
-      ti.act_n = min(128, end - ti.act0);
-      if (ti.act_n <= 0) ti.valid = 0;
-    } else {
-      ti.act_n = min(128, p.rows - ti.act0);
-    }
+    ti.act_n = min(128, p.rows - ti.act0);
   } else {
     const int ntw = (p.cols + 127) / 128;
     if (p.grouped) {

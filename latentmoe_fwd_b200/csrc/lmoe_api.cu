@@ -385,6 +385,7 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   // tokens of one expert, the MMA's N set per tile, so no token padding is
   // multiplied; small token counts use narrow tiles.
   const int sbn = swap_bn(cfg->T) ? swap_bn(cfg->T) : 256;
+  const int64_t single_tiles = static_cast<int64_t>(cfg->T) * cfg->K / sbn + cfg->N;
   TcLaunch g1;
   g1.grouped = 1;
   g1.cols = cfg->m;
@@ -394,18 +395,11 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   g1.groups = cfg->N;
   const TcOperand zop{zin, cfg->l, P, 1};
   const TcOperand w1op{w->w1, cfg->l, cfg->m, cfg->N};
-  if (sbn) {
-    g1.swap = 1;
-    g1.bn = sbn;
-    g1.a[0] = w1op;
-    g1.b[0] = zop;
-    g1.max_tiles = (static_cast<int64_t>(cfg->T) * cfg->K / sbn + cfg->N) * ((cfg->m + 127) / 128);
-  } else {
-    g1.bn = normal_bn(cfg->m);
-    g1.a[0] = zop;
-    g1.b[0] = w1op;
-    g1.max_tiles = (P / 128) * ((cfg->m + g1.bn - 1) / g1.bn);
-  }
+  g1.swap = 1;
+  g1.bn = sbn;
+  g1.a[0] = w1op;
+  g1.b[0] = zop;
+  g1.max_tiles = single_tiles * ((cfg->m + 127) / 128);
   g1.out = a;
   g1.ld_out = cfg->m;
   g1.epi = EPI_SQRELU;
@@ -437,16 +431,9 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   g2.kblocks[0] = kblocks(cfg->m);
   const TcOperand aop{a, cfg->m, P, 1};
   const TcOperand w2op{w->w2, cfg->m, cfg->l, cfg->N};
-  if (sbn) {
-    g2.a[0] = w2op;
-    g2.b[0] = aop;
-    g2.max_tiles = (static_cast<int64_t>(cfg->T) * cfg->K / sbn + cfg->N) * ((cfg->l + 127) / 128);
-  } else {
-    g2.bn = normal_bn(cfg->l);
-    g2.a[0] = aop;
-    g2.b[0] = w2op;
-    g2.max_tiles = (P / 128) * ((cfg->l + g2.bn - 1) / g2.bn);
-  }
+  g2.a[0] = w2op;
+  g2.b[0] = aop;
+  g2.max_tiles = single_tiles * ((cfg->l + 127) / 128);
   g2.out = y;
   g2.ld_out = cfg->l;
   g2.epi = EPI_GATE;

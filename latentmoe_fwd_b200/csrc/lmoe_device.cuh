@@ -294,19 +294,6 @@ __device__ __forceinline__ uint2 e2m1_codes16(const float* x, float sc, float rc
   return c;
 }
 
-// Expert owning padded row `row`: the largest e with poff[e] <= row among
-// the non-decreasing padded offsets (empty experts have equal neighbours).
-__device__ __forceinline__ int find_expert(const int* poff, int groups, int row) {
-  // largest e with poff[e] <= row (poff is non-decreasing); the expert owning
-  // padded row `row` is the one whose range is non-empty and contains it.
-  int lo = 0, hi = groups;  // answer in [0, groups-1]
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (__ldg(poff + mid) <= row) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
