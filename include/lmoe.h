@@ -269,6 +269,17 @@ lmoe_status lmoe_read_device_error(void* ws, void* stream, uint32_t* info);
 /* Static description of a status code. */
 const char* lmoe_status_string(lmoe_status s);
 
+/* Self test of the device failure path (no counterpart on the pages): one
+ * thread waits on an mbarrier that nothing arrives on, through the same
+ * bounded wait every pipeline uses, shortened to limit_cycles (1 ..
+ * 4e9 SM clock cycles). The wait gives up, records LMOE_ERR_DEVICE_TIMEOUT
+ * with info 0x7001 in the workspace error word (first 256 bytes of `ws`,
+ * zeroed before first use) and the kernel returns; lmoe_read_device_error
+ * reports it and the context stays usable. Asynchronous on `stream`.
+ * Errors: LMOE_ERR_WORKSPACE (ws NULL or < 256 bytes), LMOE_ERR_INVALID_ARG
+ * (limit out of range). */
+lmoe_status lmoe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_cycles, void* stream);
+
 /* Number of kernels launched by this library since load (host counter; used
  * by harnesses to report how many of the library's kernels a region ran). */
 uint64_t lmoe_kernel_launch_count(void);

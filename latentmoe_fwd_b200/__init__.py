@@ -29,7 +29,7 @@ OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE =
 EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permute",
            "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
-           "lmoe_forward_traced", "lmoe_permute_noalloc")
+           "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -76,6 +76,7 @@ def _load():
         "lmoe_read_device_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "lmoe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "lmoe_kernel_launch_count": (ctypes.c_uint64, []),
+        "lmoe_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_size_t, ctypes.c_uint64, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -206,6 +207,12 @@ def nvfp4_quantize(x, in_dtype, rows, cols, global_in, codes, sf, global_out, sf
     _check(lib.lmoe_nvfp4_quantize(_p(x), int(in_dtype), int(rows), int(cols), _p(global_in), _p(codes),
                                    _p(sf), _p(global_out), int(sf_layout), _p(ws), ws.numel(),
                                    _stream(stream)), "lmoe_nvfp4_quantize")
+
+
+def selftest_wait_timeout(ws, limit_cycles: int, stream=None):
+    """lmoe_selftest_wait_timeout: a bounded device wait that runs out."""
+    _check(lib.lmoe_selftest_wait_timeout(_p(ws), ws.numel(), int(limit_cycles), _stream(stream)),
+           "lmoe_selftest_wait_timeout")
 
 
 def read_device_error(ws, stream=None):

@@ -231,6 +231,12 @@ const char* lmoe_status_string(lmoe_status s) {
 
 uint64_t lmoe_kernel_launch_count(void) { return g_launches.load(); }
 
+lmoe_status lmoe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_cycles, void* stream) {
+  if (!ws || ws_bytes < 256) return LMOE_ERR_WORKSPACE;
+  if (limit_cycles == 0 || limit_cycles > static_cast<uint64_t>(kWaitLimitCycles)) return LMOE_ERR_INVALID_ARG;
+  return launch_selftest_wait(err_word(ws), static_cast<long long>(limit_cycles), static_cast<cudaStream_t>(stream));
+}
+
 size_t lmoe_workspace_size(const lmoe_config* cfg, int op) {
   if (op == LMOE_OP_NVFP4_QUANTIZE) {
     if (!cfg || cfg->T < 0 || cfg->l <= 0) return 0;

@@ -81,16 +81,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: returns false (and records a timeout) if the phase with the
-// given parity has not completed within the limit, or if another warp of the
-// CTA already gave up (*abort set).
+// given parity has not completed within `limit` cycles, or if another warp of
+// the CTA already gave up (*abort set).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          DevErr err, uint32_t where) {
+                                          DevErr err, uint32_t where, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       dev_report(err, kErrTimeout, where);
       return false;

@@ -924,4 +924,29 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
+// ===========================================================================
+// Failure-path self test: one thread waits on an mbarrier nothing arrives
+// on, through the pipelines' bounded wait with a short limit; the wait gives
+// up, records a timeout (info 0x7001) in the error word and the kernel
+// returns, leaving the context usable.
+// ===========================================================================
+__global__ void __launch_bounds__(32) selftest_wait_kernel(DevErr err, long long limit) {
+  pdl_begin();
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, err, 0x7001, limit);
+}
+
+lmoe_status launch_selftest_wait(uint32_t* err, long long limit, cudaStream_t s) {
+  launch_k(selftest_wait_kernel, dim3(1), dim3(32), 0, s, DevErr{err}, limit);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
 }  // namespace lmoe

@@ -114,3 +114,11 @@ def test_nvfp4_quantize_layout_flags():
     for bad in (2, 3, 0x20, 0x12):
         st = L.lib.lmoe_nvfp4_quantize(fake, 1, 16, 16, None, fake, fake, None, bad, ws, 4096, None)
         assert st == L.ERR_INVALID_ARG
+
+
+def test_selftest_wait_rejects_bad_arguments_on_host():
+    small = ctypes.create_string_buffer(128)
+    assert L.lib.lmoe_selftest_wait_timeout(small, 128, 1000, None) == L.ERR_WORKSPACE
+    ws = ctypes.create_string_buffer(256)
+    assert L.lib.lmoe_selftest_wait_timeout(ws, 256, 0, None) == L.ERR_INVALID_ARG
+    assert L.lib.lmoe_selftest_wait_timeout(ws, 256, 5_000_000_000, None) == L.ERR_INVALID_ARG
