@@ -81,10 +81,13 @@ int64_t splitk_floats(const lmoe_config* c, int op) { return c->T * max_dense_co
 // Workspace layout (byte offsets; region sizes 0 when unused).
 struct Layout {
   size_t splitk = 0;        // fp32 split-K partial sums of the weight-major dense GEMMs (T <= 64)
+  size_t rsplit = 0;        // fp32 split-K partial sums of the token-major router GEMM (few tiles)
   size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0,
          offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, scratch = 0, gate = 0, zp = 0,
          zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, ys = 0, total = 0;
 };
+
+int tokmajor_splits(int64_t rows, int cols, int64_t k);
 
 Layout layout(const lmoe_config* c, int op) {
   Layout L;
@@ -101,6 +104,10 @@ Layout layout(const lmoe_config* c, int op) {
   L.err = take(256);
   if ((op == LMOE_OP_ROUTE || op == LMOE_OP_FORWARD) && T <= kSwapMaxTokens)
     L.splitk = take(splitk_floats(c, op) * 4);
+  if ((op == LMOE_OP_ROUTE || op == LMOE_OP_FORWARD) && T > kSwapMaxTokens && c->act != LMOE_F32) {
+    const int sp = tokmajor_splits(T, static_cast<int>(N), c->d);
+    if (sp > 1) L.rsplit = take(static_cast<size_t>(T) * N * sp * 4);
+  }
   if (op == LMOE_OP_ROUTE) {
     L.logits = take(T * N * 4);
   } else if (op == LMOE_OP_PERMUTE) {
@@ -175,6 +182,21 @@ int choose_splits(int64_t tiles, int kb, int64_t rows, int64_t cols, float* part
   return sp > 1 ? sp : 1;
 }
 
+// Split-K of a token-major dense GEMM whose 128 x BN tiles fill less than half
+// the GPU (the router at a few thousand tokens): splits to fill one wave, at
+// least two K blocks each, at most 8.
+int tokmajor_splits(int64_t rows, int cols, int64_t k) {
+  const int bn = normal_bn(cols);
+  const int64_t tiles = ((rows + 127) / 128) * ((cols + bn - 1) / bn);
+  const int sms = device_sm_count();
+  if (tiles * 2 > sms) return 1;
+  int sp = static_cast<int>(sms / tiles);
+  const int kb = kblocks(k);
+  if (sp > kb / 2) sp = kb / 2;
+  if (sp > 8) sp = 8;
+  return sp > 1 ? sp : 1;
+}
+
 lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int64_t k, void* out,
                        int64_t ld_out, int epi, const float* bias, const void* residual, int64_t ld_res,
                        float* partial, uint32_t* err, cudaStream_t s) {
@@ -199,6 +221,10 @@ lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int
     L.a[0] = act;
     L.b[0] = wt;
     L.max_tiles = ((rows + 127) / 128) * ((cols + L.bn - 1) / L.bn);
+    if (partial) {   // a buffer of rows * cols * tokmajor_splits() floats
+      L.ksplit = tokmajor_splits(rows, cols, k);
+      L.partial = partial;
+    }
   }
   L.out = out;
   L.ld_out = ld_out;
@@ -293,7 +319,7 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
       st = simt_gemm(S, err, s);
     } else {
       st = dense_bf16(x, cfg->T, w_router, cfg->N, cfg->d, lg, cfg->N, EPI_F32_BIAS, bias, nullptr, 0,
-                      L.splitk ? at<float>(ws, L.splitk) : nullptr, err, s);
+                      L.splitk ? at<float>(ws, L.splitk) : (L.rsplit ? at<float>(ws, L.rsplit) : nullptr), err, s);
     }
     if (st != LMOE_OK) return st;
     logits = lg;
@@ -621,7 +647,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     S.epi = EPI_F32_BIAS;
     st = simt_gemm(S, err, s);
   } else {
-    st = dense_bf16(x, T, w->w_router, N, d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0, splitk, err, s);
+    st = dense_bf16(x, T, w->w_router, N, d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0,
+                    L.rsplit ? at<float>(ws, L.rsplit) : splitk, err, s);
   }
   if (st != LMOE_OK) return st;
   if ((st = launch_topk(logits, T, N, K, idx, gw, x, w->w_router, w->router_bias, d, cfg->act, err, s)) != LMOE_OK)

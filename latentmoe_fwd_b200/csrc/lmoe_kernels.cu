@@ -607,9 +607,7 @@ __global__ void __launch_bounds__(256) combine_kernel(
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.0f;
-    for (int k = 0; k < K; ++k) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(y + rowk[k] * l + col));
-      const float g = wk[k];
+    auto add = [&](const uint4& u, float g) {
       if constexpr (sizeof(TA) == 2) {
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -623,7 +621,17 @@ __global__ void __launch_bounds__(256) combine_kernel(
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[i] += g * f4[i];
       }
+    };
+    // four of the token's rows in flight at a time; the sums stay in k order
+    int k = 0;
+    for (; k + 4 <= K; k += 4) {
+      uint4 u[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) u[q] = __ldg(reinterpret_cast<const uint4*>(y + rowk[k + q] * l + col));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) add(u[q], wk[k + q]);
     }
+    for (; k < K; ++k) add(__ldg(reinterpret_cast<const uint4*>(y + rowk[k] * l + col)), wk[k]);
     if (resid) {   // + a [T, l] term (the shared experts' output) after the K routed rows
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(resid + t * l + col));
       if constexpr (sizeof(TA) == 2) {
