@@ -227,7 +227,9 @@ lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32
 
 /* The whole layer: route, down-project (NVFP4: quantise z with its current
  * amax), permute, expert FFNs, combine, up-project and add the shared
- * experts. x [T][d] (act) -> out [T][d] (act). */
+ * experts. x [T][d] (act) -> out [T][d] (act). N must be a multiple of 8
+ * (the router GEMM stores logit rows in 16-byte vectors; LMOE_ERR_UNSUPPORTED
+ * otherwise, also from lmoe_route when it computes the logits). */
 lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x,
                          void* out, void* ws, size_t ws_bytes, void* stream);
 

@@ -298,6 +298,7 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
   if (!topk_idx || !topk_w) return LMOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < layout(cfg, LMOE_OP_ROUTE).total) return LMOE_ERR_WORKSPACE;
   if (!logits_in && (!x || !w_router)) return LMOE_ERR_INVALID_ARG;
+  if (!logits_in && cfg->N % 8) return LMOE_ERR_UNSUPPORTED;   // router GEMM: 16-byte logit stores
   if (!aligned16(x) || !aligned16(w_router)) return LMOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Layout L = layout(cfg, LMOE_OP_ROUTE);
@@ -615,6 +616,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   if (fp4 && !fp4_weights_ok(w)) return LMOE_ERR_INVALID_ARG;
   if (cfg->T == 0) return LMOE_OK;
   if (!x || !out || !aligned16(x) || !aligned16(out)) return LMOE_ERR_INVALID_ARG;
+  if (cfg->N % 8) return LMOE_ERR_UNSUPPORTED;   // the router GEMM stores logit rows in 16-byte vectors
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Layout L = layout(cfg, LMOE_OP_FORWARD);
   uint32_t* err = err_word(ws);

@@ -164,18 +164,37 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
       }
       tau = ldexpf(sqrtf(sq / static_cast<float>(N)), -10) + ldexpf(vmax_abs, -20);
     }
-    // this lane's best remaining entry (largest key, lowest column on ties)
+    // this lane's best and second-best remaining entries (largest key, lowest
+    // column on ties); a lane that wins moves its second up, and scans its
+    // entries again only when it wins without a known second
     uint32_t taken = 0;
-    uint32_t hk = 0;
-    int hi_i = 0;
-    float hv = -INFINITY;
+    uint32_t hk = 0, hk2 = 0;
+    int hi_i = 0, hi2 = 0;
+    float hv = -INFINITY, hv2 = -INFINITY;
+    auto top2 = [&]() {
+      hk = 0;
+      hk2 = 0;
+      hv = -INFINITY;
+      hv2 = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i)
-      if (key[i] > hk) {
-        hk = key[i];
-        hi_i = i;
-        hv = v[i];
+      for (int i = 0; i < NPL; ++i) {
+        const uint32_t ki = ((taken >> i) & 1u) ? 0u : key[i];
+        if (ki > hk) {
+          hk2 = hk;
+          hi2 = hi_i;
+          hv2 = hv;
+          hk = ki;
+          hi_i = i;
+          hv = v[i];
+        } else if (ki > hk2) {
+          hk2 = ki;
+          hi2 = i;
+          hv2 = v[i];
+        }
       }
+    };
+    top2();
+    bool second = true;   // hk2 is the best entry after hk (0: none left)
     // extract candidates in (approximate) order: the K best, the (K+1)-th, and
     // while refining, further experts within 2 tau of the K-th (at most 32)
     float kth = -INFINITY;
@@ -199,15 +218,15 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
       if (!refine && C >= K) break;
       if (lane == wl) {   // the winning lane moves on to its next entry
         taken |= 1u << hi_i;
-        hk = 0;
-        hv = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i)
-          if (!((taken >> i) & 1u) && key[i] > hk) {
-            hk = key[i];
-            hi_i = i;
-            hv = v[i];
-          }
+        if (second) {
+          hk = hk2;
+          hi_i = hi2;
+          hv = hv2;
+          second = false;
+        } else {
+          top2();
+          second = true;
+        }
       }
     }
     if (refine) {

@@ -122,3 +122,12 @@ def test_selftest_wait_rejects_bad_arguments_on_host():
     ws = ctypes.create_string_buffer(256)
     assert L.lib.lmoe_selftest_wait_timeout(ws, 256, 0, None) == L.ERR_INVALID_ARG
     assert L.lib.lmoe_selftest_wait_timeout(ws, 256, 5_000_000_000, None) == L.ERR_INVALID_ARG
+
+
+def test_router_gemm_needs_n_multiple_of_8():
+    cfg = L.config(T=4, d=64, l=64, N=4, K=2, m=64)
+    w = L.weights(w_router=16, w1=16, w2=16, w_down=16, w_up=16)
+    assert L.lib.lmoe_forward(ctypes.byref(cfg), ctypes.byref(w), 16, 16, 16, 1 << 40, None) == L.ERR_UNSUPPORTED
+    idx = 16
+    assert L.lib.lmoe_route(ctypes.byref(cfg), 16, 16, None, None, idx, idx, None, 16, 1 << 30,
+                            None) == L.ERR_UNSUPPORTED

@@ -112,3 +112,18 @@ def test_zero_tokens_is_a_no_op():
     L.forward(cfg, w, x, out, ws)
     assert L.read_device_error(ws)[0] == L.OK
     assert wl.T == 0
+
+
+@pytest.mark.parametrize("T", [300, 2100])
+def test_largest_expert_count_and_top_k(T):
+    # N = 1024 experts and K = 32 (the library's limits); T = 2100 gives
+    # T*K >= 64*N, so the expert GEMMs run on CTA pairs over 1024 groups
+    wl = LI.Workload("max_experts", T=T, d=256, l=128, N=1024, K=32, m=128, dtype="bf16")
+    _check_layer(wl, BF16_TOL)
+
+
+def test_top_1_of_8_experts():
+    # K = 1 with the smallest expert count the router GEMM takes (N a multiple
+    # of 8); T*K >= 64*N puts the expert GEMMs on CTA pairs
+    wl = LI.Workload("top1_of_8", T=700, d=256, l=128, N=8, K=1, m=192, dtype="bf16")
+    _check_layer(wl, BF16_TOL)
