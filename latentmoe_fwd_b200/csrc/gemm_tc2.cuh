@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
       const int wbase = ti.w0 + static_cast<int>(rank) * 128;
+      const uint64_t pol_out = policy_evict_first();   // outputs stream out; the next kernel reads them from HBM
       const int cols = ti.extra ? p.cols_x : p.cols;
       __nv_bfloat16* const out = reinterpret_cast<__nv_bfloat16*>(ti.extra ? p.out_x : p.out);
       const long long ld_out = ti.extra ? p.ld_out_x : p.ld_out;
@@ -389,7 +390,7 @@ __global__ void __launch_bounds__(192, 1)
           const int tok = c * 32 + j;
           if (tok < ti.act_n && col0 < cols) {
             const uint4 u = *reinterpret_cast<const uint4*>(tb + j * 32 + seg * 8);
-            *reinterpret_cast<uint4*>(out + (ti.act0 + tok) * ld_out + col0) = u;
+            st_global_v4_hint(out + (ti.act0 + tok) * ld_out + col0, u, pol_out);
           }
         }
         __syncwarp();

@@ -563,15 +563,18 @@ __global__ void __launch_bounds__(256) gather_kernel(
     const uint4* src = reinterpret_cast<const uint4*>(rows + static_cast<int64_t>(t) * row_bytes);
     uint4* dst = reinterpret_cast<uint4*>(out + p * row_bytes);
     const int64_t n16 = row_bytes >> 4;
+    // the permuted copy streams through L2 (evict first) so the source rows,
+    // read K times, stay
+    const uint64_t pol = policy_evict_first();
     int64_t i = lane;
     for (; i + 96 < n16; i += 128) {   // four 16-byte loads in flight per lane
       const uint4 v0 = __ldg(src + i), v1 = __ldg(src + i + 32), v2 = __ldg(src + i + 64), v3 = __ldg(src + i + 96);
-      dst[i] = v0;
-      dst[i + 32] = v1;
-      dst[i + 64] = v2;
-      dst[i + 96] = v3;
+      st_global_v4_hint(dst + i, v0, pol);
+      st_global_v4_hint(dst + i + 32, v1, pol);
+      st_global_v4_hint(dst + i + 64, v2, pol);
+      st_global_v4_hint(dst + i + 96, v3, pol);
     }
-    for (; i < n16; i += 32) dst[i] = __ldg(src + i);
+    for (; i < n16; i += 32) st_global_v4_hint(dst + i, __ldg(src + i), pol);
   }
   if (out_sf) {
     const int cols = static_cast<int>(row_bytes * 2);
