@@ -81,6 +81,17 @@ typedef enum { LMOE_SF_ROWMAJOR = 0, LMOE_SF_MMA_TILED = 1 } lmoe_sf_layout;
 /* Flag: l == d and there is no down/up projection (the standard-MoE limit). */
 #define LMOE_FLAG_IDENTITY_PROJ 1u
 
+/* Supported configurations (every entry point that takes a config checks
+ * them before launching anything):
+ *  LMOE_ERR_INVALID_ARG: T < 0 or T > 2^25; d, l, N, K or m not positive;
+ *    K > N; n_shared < 0, or n_shared > 0 with m_shared <= 0; d, l, m or
+ *    m_shared not a multiple of 8; LMOE_FLAG_IDENTITY_PROJ with l != d.
+ *  LMOE_ERR_UNSUPPORTED: K > 32 or N > 1024; act F32 with expert other than
+ *    F32; act BF16 with expert F32; act BF16 with shared experts and m_shared
+ *    not a multiple of 64; expert NVFP4 with l or m not a multiple of 256;
+ *    N not a multiple of 8 where the logits are computed (lmoe_forward,
+ *    lmoe_route without logits_in). */
+
 typedef struct {
   int64_t T;        /* tokens */
   int32_t d;        /* hidden size */

@@ -283,9 +283,13 @@ lmoe_status lmoe_read_device_error(void* ws, void* stream, uint32_t* info) {
   if (!ws) return LMOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return LMOE_ERR_CUDA;
+  // read and clear on the caller's stream, so the clear is ordered before any
+  // kernel the caller launches on it afterwards (a plain cudaMemset runs on the
+  // legacy stream, which a non-blocking stream does not wait for)
   uint32_t w[2] = {0, 0};
-  if (cudaMemcpy(w, ws, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
-  if (cudaMemset(ws, 0, sizeof(w)) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (cudaMemcpyAsync(w, ws, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(w), s) != cudaSuccess) return LMOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LMOE_ERR_CUDA;
   if (info) *info = w[1];
   return static_cast<lmoe_status>(w[0]);
 }

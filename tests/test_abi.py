@@ -60,6 +60,9 @@ def test_workspace_sizes_and_padded_rows():
     assert 0 < L.workspace_size(cfg, L.OP_ROUTE) < fwd
     bad = L.config(T=4, d=64, l=64, N=4, K=5, m=64)    # K > N
     assert L.workspace_size(bad, L.OP_FORWARD) == 0
+    # the token limit: 2^25 tokens are accepted, one more is not
+    assert L.workspace_size(L.config(T=2**25, d=64, l=64, N=8, K=2, m=64), L.OP_FORWARD) > 0
+    assert L.workspace_size(L.config(T=2**25 + 1, d=64, l=64, N=8, K=2, m=64), L.OP_FORWARD) == 0
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -68,6 +71,19 @@ def test_workspace_sizes_and_padded_rows():
     (dict(d=60), L.ERR_INVALID_ARG),              # rows not a multiple of 16 bytes
     (dict(act=L.F32, expert=L.BF16), L.ERR_UNSUPPORTED),
     (dict(expert=L.NVFP4, l=128), L.ERR_UNSUPPORTED),
+    (dict(expert=L.NVFP4, l=256, m=128), L.ERR_UNSUPPORTED),
+    (dict(T=-1), L.ERR_INVALID_ARG),
+    (dict(T=2**25 + 1), L.ERR_INVALID_ARG),
+    (dict(m=0), L.ERR_INVALID_ARG),
+    (dict(l=60), L.ERR_INVALID_ARG),
+    (dict(identity=True, l=32), L.ERR_INVALID_ARG),
+    (dict(n_shared=-1), L.ERR_INVALID_ARG),
+    (dict(n_shared=1, m_shared=0), L.ERR_INVALID_ARG),
+    (dict(n_shared=1, m_shared=36), L.ERR_INVALID_ARG),
+    (dict(n_shared=1, m_shared=40), L.ERR_UNSUPPORTED),   # BF16 shared experts: m_shared % 64
+    (dict(N=1032, K=2), L.ERR_UNSUPPORTED),
+    (dict(expert=L.F32), L.ERR_UNSUPPORTED),              # BF16 activations, fp32 experts
+    (dict(act=L.NVFP4, expert=L.NVFP4), L.ERR_UNSUPPORTED),
 ])
 def test_invalid_configs_rejected_on_host(kw, status):
     base = dict(T=4, d=64, l=64, N=4, K=2, m=64)
