@@ -65,3 +65,18 @@ def test_reference_arm_other_ranks_exit_quietly():
                    {"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_cpu_baseline_sample_is_time_bounded():
+    sys.path.insert(0, ROOT)
+    import bench
+    import lmoe_inputs as LI
+    wl = LI.WORKLOADS["tiny_f32"]
+    inp = LI.make_inputs(wl)
+    v, dt, ntok, calls = bench.oracle_sample(wl, inp, 16, min_seconds=0.2, max_calls=1000)
+    assert calls >= 2 and ntok == 16 * calls       # repeated until the time bound
+    assert dt >= 0.2 or calls == 1000
+    assert v == pytest.approx(ntok / dt)
+    _, _, ntok1, calls1 = bench.oracle_sample(wl, inp, 16, min_seconds=1e9, max_calls=3)
+    assert calls1 == 3 and ntok1 == 48              # and by the call cap
+    assert set(bench.CPU_SAMPLE_TOKENS) == set(LI.WORKLOADS)
