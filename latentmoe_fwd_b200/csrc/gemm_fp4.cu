@@ -45,13 +45,13 @@ template <int EPI>
 static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const Fp4Params& p, int grid,
                               cudaStream_t s) {
   auto kern = fp4_gemm_kernel<EPI>;
-  static int configured_dev = -1;
+  static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_dev != dev) {
+  if (!device_configured(configured, dev)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp4Smem::kBytes) != cudaSuccess)
       return LMOE_ERR_CUDA;
-    configured_dev = dev;
+    mark_configured(configured, dev);
   }
   launch_k(kern, dim3(grid), dim3(Fp4Smem::kThreads), Fp4Smem::kBytes, s, a, b, p);
   count_launch();

@@ -49,13 +49,13 @@ static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const
                              cudaStream_t s) {
   using Sm = TcSmem<BN, STAGES>;
   auto kern = tc_gemm_kernel<BN, STAGES, EPI>;
-  static int configured_dev = -1;
+  static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_dev != dev) {
+  if (!device_configured(configured, dev)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes) != cudaSuccess)
       return LMOE_ERR_CUDA;
-    configured_dev = dev;
+    mark_configured(configured, dev);
   }
   launch_k(kern, dim3(grid), dim3(192), Sm::kBytes, s, a0, b0, a1, b1, bs, p);
   count_launch();
@@ -153,8 +153,8 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
 template <int EPI>
 static lmoe_status launch_tc2(const Tc2Maps& m, const TcParams& p, int64_t max_tiles, cudaStream_t s) {
   auto kern = tc2_gemm_kernel<EPI>;
-  static int configured_dev = -1;
-  static int max_clusters = 0;
+  static std::atomic<uint64_t> configured{0};
+  static std::atomic<int> max_clusters_dev[64];
   int dev = 0;
   cudaGetDevice(&dev);
   cudaLaunchConfig_t cfg = {};
@@ -170,14 +170,17 @@ static lmoe_status launch_tc2(const Tc2Maps& m, const TcParams& p, int64_t max_t
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (configured_dev != dev) {
+  int max_clusters = 0;
+  if (device_configured(configured, dev)) {
+    max_clusters = max_clusters_dev[dev].load(std::memory_order_relaxed);
+  } else {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tc2Smem::kBytes) != cudaSuccess)
       return LMOE_ERR_CUDA;
     cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return LMOE_ERR_CUDA;
-    max_clusters = n;
-    configured_dev = dev;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters <= 0)
+      return LMOE_ERR_CUDA;
+    if (dev >= 0 && dev < 64) max_clusters_dev[dev].store(max_clusters, std::memory_order_relaxed);
+    mark_configured(configured, dev);
   }
   const int64_t clusters = max_tiles < max_clusters ? max_tiles : max_clusters;
   if (clusters <= 0) return LMOE_OK;

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/lmoe.h"
 
 namespace lmoe {
@@ -32,6 +34,16 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
 
 void count_launch();                 // bump the library's kernel-launch counter
 int device_sm_count();               // SMs of the current device (cached per device)
+
+// One-time per-device setup of a kernel (function attributes persist per
+// device): a bit per device ordinal below 64; devices from 64 on are set up
+// on every call. Concurrent first calls may both run the (idempotent) setup.
+inline bool device_configured(const std::atomic<uint64_t>& mask, int dev) {
+  return dev >= 0 && dev < 64 && ((mask.load(std::memory_order_acquire) >> dev) & 1u);
+}
+inline void mark_configured(std::atomic<uint64_t>& mask, int dev) {
+  if (dev >= 0 && dev < 64) mask.fetch_or(uint64_t(1) << dev, std::memory_order_release);
+}
 
 // ----- tensor-core GEMM (gemm_tc.cu) -----
 struct TcOperand {
