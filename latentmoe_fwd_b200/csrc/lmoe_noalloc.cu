@@ -45,7 +45,8 @@ extern "C" lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_
                                             float* perm_gate, void* stream) {
   using namespace lmoe;
   if (!cfg || !topk_idx || !offsets || !perm_src || !inv_perm || !padded_offsets) return LMOE_ERR_INVALID_ARG;
-  if (cfg->T < 0 || cfg->N <= 0 || cfg->K <= 0 || cfg->K > cfg->N) return LMOE_ERR_INVALID_ARG;
+  if (cfg->T < 0 || cfg->T > (int64_t(1) << 31) / 64) return LMOE_ERR_INVALID_ARG;   // as every entry point
+  if (cfg->N <= 0 || cfg->K <= 0 || cfg->K > cfg->N) return LMOE_ERR_INVALID_ARG;
   if (cfg->N > 1024 || cfg->K > 32) return LMOE_ERR_UNSUPPORTED;
   if ((rows == nullptr) != (permuted_rows == nullptr)) return LMOE_ERR_INVALID_ARG;
   if (rows && (row_bytes <= 0 || row_bytes % 16 || (reinterpret_cast<uintptr_t>(rows) & 15) ||

@@ -147,3 +147,14 @@ def test_router_gemm_needs_n_multiple_of_8():
     idx = 16
     assert L.lib.lmoe_route(ctypes.byref(cfg), 16, 16, None, None, idx, idx, None, 16, 1 << 30,
                             None) == L.ERR_UNSUPPORTED
+
+
+def test_noalloc_permute_host_checks():
+    def call(cfg):
+        return L.lib.lmoe_permute_noalloc(ctypes.byref(cfg), 16, 16, 16, 16, 16, None, 0, None, None, None,
+                                          None, None, None)
+    assert call(L.config(T=2**25 + 1, d=8, l=8, N=8, K=2, m=8)) == L.ERR_INVALID_ARG
+    assert call(L.config(T=4, d=8, l=8, N=4, K=5, m=8)) == L.ERR_INVALID_ARG          # K > N
+    assert call(L.config(T=4, d=8, l=8, N=2048, K=2, m=8)) == L.ERR_UNSUPPORTED
+    # beyond the fixed 131072-counter scratch: (ceil(T*K / 8192) + 1) * N counters
+    assert call(L.config(T=300000, d=8, l=8, N=1024, K=8, m=8)) == L.ERR_WORKSPACE
