@@ -172,6 +172,9 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
 /* Dispatch grouped by expert: a stable counting sort of the slots
  * f = t*K + k by expert (expert ascending, then f ascending).
  *  topk_idx [T][K] int32 (each in [0, N); out-of-range -> device bounds error).
+ *    A slot with an out-of-range expert is left out: offsets[N] counts only
+ *    the in-range slots, its inv_perm entry is not written, and it is neither
+ *    gathered nor given a gate.
  *  offsets [N+1] int32: expert e owns sorted positions [offsets[e], offsets[e+1]).
  *  perm_src [T*K] int32: sorted position r holds slot perm_src[r].
  *  inv_perm [T*K] int32: slot f sits at sorted position inv_perm[f].
@@ -230,7 +233,8 @@ lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w,
 /* Combine: c_t = sum_{k=0..K-1} w[t][k] * y_perm[row(t*K+k)], summed in fp32
  * in k order, stored as `act`; row(f) = inv_perm[f] - offsets[e] +
  * padded_offsets[e] with e = topk_idx[f]. topk_w NULL means the gates were
- * already applied (w = 1). c [T][l]. No workspace. */
+ * already applied (w = 1). c [T][l]. No workspace. A slot whose expert index
+ * is out of range (left out by lmoe_permute) contributes nothing. */
 lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32_t* topk_idx,
                          const int32_t* inv_perm, const int32_t* offsets,
                          const int32_t* padded_offsets, const float* topk_w, void* c,

@@ -358,7 +358,7 @@ lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_
   if (st != LMOE_OK) return st;
   if (rows || rows_sf)
     st = launch_gather(topk_idx, perm_src, offsets, padded_offsets, cfg->T * cfg->K, cfg->K, rows, row_bytes,
-                       permuted_rows, rows_sf, permuted_sf, padded_rows(cfg), s);
+                       permuted_rows, rows_sf, permuted_sf, cfg->N, s);
   return st;
 }
 
@@ -579,7 +579,7 @@ lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32
   if (!y_perm || !topk_idx || !inv_perm || !offsets || !padded_offsets || !c) return LMOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(c)) return LMOE_ERR_INVALID_ARG;
   return launch_combine(y_perm, cfg->act, topk_idx, inv_perm, offsets, padded_offsets, topk_w, nullptr, c, cfg->T,
-                        cfg->K, cfg->l, static_cast<cudaStream_t>(stream));
+                        cfg->K, cfg->N, cfg->l, static_cast<cudaStream_t>(stream));
 }
 
 lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* global_in,
@@ -708,8 +708,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     return st;
   const int64_t row_bytes = fp4 ? l / 2 : static_cast<int64_t>(l) * ab;
   uint8_t* zp_sf = fp4 ? at<uint8_t>(ws, L.zp_sf) : nullptr;
-  if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, zq_sf, zp_sf,
-                          padded_rows(cfg), s)) != LMOE_OK)
+  if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, zq_sf, zp_sf, N, s)) !=
+      LMOE_OK)
     return st;
   mark(3);
 
@@ -746,7 +746,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   const bool combine_is_out = ident && (cfg->n_shared == 0 || ys_ready);
   void* c = combine_is_out ? out : at<void>(ws, L.c);
   if ((st = launch_combine(y, cfg->act, idx, inv_perm, offsets, poff, nullptr, ident && ys_ready ? at<void>(ws, L.ys)
-                           : nullptr, c, T, K, l, s)) != LMOE_OK)
+                           : nullptr, c, T, K, N, l, s)) != LMOE_OK)
     return st;
   mark(6);
   if (combine_is_out) {

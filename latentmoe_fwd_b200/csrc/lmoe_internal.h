@@ -157,11 +157,11 @@ lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t*
 lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int32_t* offsets,
                           const int32_t* padded_offsets, int64_t slots, int K, const void* rows,
                           int64_t row_bytes, void* out_rows, const uint8_t* rows_sf,
-                          uint8_t* out_sf, int64_t padded_rows, cudaStream_t s);
+                          uint8_t* out_sf, int N, cudaStream_t s);
 lmoe_status launch_selftest_wait(uint32_t* err, long long limit_cycles, cudaStream_t s);
 lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
                            const int32_t* offsets, const int32_t* padded_offsets, const float* w,
-                           const void* resid, void* c, int64_t T, int K, int l, cudaStream_t s);
+                           const void* resid, void* c, int64_t T, int K, int N, int l, cudaStream_t s);
 lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                   const float* global_in, uint8_t* codes, uint8_t* sf,
                                   float* global_out, int sf_layout, float* partials,

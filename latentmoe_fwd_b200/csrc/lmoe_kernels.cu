@@ -548,13 +548,15 @@ __device__ __forceinline__ int64_t sf_tiled_offset(int64_t row, int j, int group
 
 __global__ void __launch_bounds__(256) gather_kernel(
     const int32_t* __restrict__ idx, const int32_t* __restrict__ perm_src,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int64_t slots, int K,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int64_t slots, int K, int N,
     const uint8_t* __restrict__ rows, int64_t row_bytes, uint8_t* __restrict__ out,
     const uint8_t* __restrict__ rows_sf, uint8_t* __restrict__ out_sf) {
   pdl_begin();
   const int lane = threadIdx.x & 31;
   const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (r >= slots) return;
+  // sorted positions past offsets[N] exist only when some expert index was out
+  // of range (the permutation leaves those slots out): nothing to copy there
+  if (r >= slots || r >= __ldg(offsets + N)) return;
   const int f = __ldg(perm_src + r);
   const int t = f / K;
   const int e = __ldg(idx + f);
@@ -594,12 +596,11 @@ __global__ void __launch_bounds__(256) gather_kernel(
 lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int32_t* offsets,
                           const int32_t* padded_offsets, int64_t slots, int K, const void* rows,
                           int64_t row_bytes, void* out_rows, const uint8_t* rows_sf,
-                          uint8_t* out_sf, int64_t padded_rows, cudaStream_t s) {
-  (void)padded_rows;
+                          uint8_t* out_sf, int N, cudaStream_t s) {
   if (slots == 0) return LMOE_OK;
   const int64_t blocks = (slots * 32 + 255) / 256;
   launch_k(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, idx, perm_src, offsets,
-           padded_offsets, slots, K, static_cast<const uint8_t*>(rows), row_bytes, static_cast<uint8_t*>(out_rows),
+           padded_offsets, slots, K, N, static_cast<const uint8_t*>(rows), row_bytes, static_cast<uint8_t*>(out_rows),
            rows_sf, out_sf);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
@@ -612,18 +613,38 @@ template <typename TA>
 __global__ void __launch_bounds__(256) combine_kernel(
     const TA* __restrict__ y, const int32_t* __restrict__ idx, const int32_t* __restrict__ inv_perm,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, const float* __restrict__ w,
-    const TA* __restrict__ resid, TA* __restrict__ c, int K, int l) {
+    const TA* __restrict__ resid, TA* __restrict__ c, int K, int N, int l) {
   pdl_begin();
-  extern __shared__ int64_t rowk[];   // [K] padded rows of this token
-  __shared__ float wk[64];
+  extern __shared__ int64_t rowk[];   // [K] padded rows of the token's in-range slots, in k order
+  __shared__ float wk[32];
+  __shared__ int s_nk;
   const int64_t t = blockIdx.x;
-  if (threadIdx.x < K) {
-    const int64_t f = t * K + threadIdx.x;
-    const int e = __ldg(idx + f);
-    rowk[threadIdx.x] = static_cast<int64_t>(__ldg(inv_perm + f)) - __ldg(offsets + e) + __ldg(poff + e);
-    wk[threadIdx.x] = w ? __ldg(w + f) : 1.0f;
+  if (threadIdx.x < 32) {
+    // an out-of-range expert index contributes nothing (the permutation left
+    // its slot out and reported it); the others keep their k order
+    const int k = threadIdx.x;
+    bool ok = false;
+    int64_t row = 0;
+    float g = 0.0f;
+    if (k < K) {
+      const int64_t f = t * K + k;
+      const int e = __ldg(idx + f);
+      ok = e >= 0 && e < N;
+      if (ok) {
+        row = static_cast<int64_t>(__ldg(inv_perm + f)) - __ldg(offsets + e) + __ldg(poff + e);
+        g = w ? __ldg(w + f) : 1.0f;
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    if (ok) {
+      const int pos = __popc(m & ((1u << k) - 1u));
+      rowk[pos] = row;
+      wk[pos] = g;
+    }
+    if (k == 0) s_nk = __popc(m);
   }
   __syncthreads();
+  const int nk = s_nk;
   constexpr int V = 16 / sizeof(TA);   // elements per 16-byte vector
   for (int col = threadIdx.x * V; col < l; col += blockDim.x * V) {
     float acc[V];
@@ -646,14 +667,14 @@ __global__ void __launch_bounds__(256) combine_kernel(
     };
     // four of the token's rows in flight at a time; the sums stay in k order
     int k = 0;
-    for (; k + 4 <= K; k += 4) {
+    for (; k + 4 <= nk; k += 4) {
       uint4 u[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) u[q] = __ldg(reinterpret_cast<const uint4*>(y + rowk[k + q] * l + col));
 #pragma unroll
       for (int q = 0; q < 4; ++q) add(u[q], wk[k + q]);
     }
-    for (; k < K; ++k) add(__ldg(reinterpret_cast<const uint4*>(y + rowk[k] * l + col)), wk[k]);
+    for (; k < nk; ++k) add(__ldg(reinterpret_cast<const uint4*>(y + rowk[k] * l + col)), wk[k]);
     if (resid) {   // + a [T, l] term (the shared experts' output) after the K routed rows
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(resid + t * l + col));
       if constexpr (sizeof(TA) == 2) {
@@ -688,18 +709,18 @@ __global__ void __launch_bounds__(256) combine_kernel(
 
 lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
                            const int32_t* offsets, const int32_t* padded_offsets, const float* w,
-                           const void* resid, void* c, int64_t T, int K, int l, cudaStream_t s) {
+                           const void* resid, void* c, int64_t T, int K, int N, int l, cudaStream_t s) {
   if (T == 0) return LMOE_OK;
-  if (K > 64) return LMOE_ERR_UNSUPPORTED;
+  if (K > 32) return LMOE_ERR_UNSUPPORTED;
   const size_t sm = static_cast<size_t>(K) * sizeof(int64_t);
   if (act == LMOE_BF16)
     launch_k(combine_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(T)), dim3(256), sm, s,
              static_cast<const __nv_bfloat16*>(y), idx, inv_perm, offsets, padded_offsets, w,
-             static_cast<const __nv_bfloat16*>(resid), static_cast<__nv_bfloat16*>(c), K, l);
+             static_cast<const __nv_bfloat16*>(resid), static_cast<__nv_bfloat16*>(c), K, N, l);
   else
     launch_k(combine_kernel<float>, dim3(static_cast<unsigned>(T)), dim3(256), sm, s, static_cast<const float*>(y),
              idx, inv_perm, offsets, padded_offsets, w, static_cast<const float*>(resid), static_cast<float*>(c), K,
-             l);
+             N, l);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

@@ -67,10 +67,8 @@ extern "C" lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_
                       topk_w, perm_gate, nullptr, s, kPermSlotsPerWarpStatic);
   if (st != LMOE_OK) return st;
   if (rows || rows_sf) {
-    const int64_t nonempty = slots < cfg->N ? slots : cfg->N;
-    const int64_t padded = (slots + 127 * nonempty + 127) / 128 * 128;
     st = launch_gather(topk_idx, perm_src, offsets, padded_offsets, slots, cfg->K, rows, row_bytes, permuted_rows,
-                       rows_sf, permuted_sf, padded, s);
+                       rows_sf, permuted_sf, cfg->N, s);
   }
   return st;
 }

@@ -200,3 +200,62 @@ def test_permute_out_of_range_expert_reports_bounds_error():
     assert info == 3 * K + 0
     st2, _ = L.read_device_error(ws)
     assert st2 == L.OK          # reading clears the word
+
+
+def test_out_of_range_expert_is_left_out_of_gather_and_combine():
+    """A slot whose expert index is >= N is reported, left out of the sorted
+    positions (offsets[N] counts only in-range slots), not gathered, and
+    contributes nothing to the combine. Buffers start zeroed, so every index
+    the kernels could take stays inside them."""
+    T, N, K, l = 10, 8, 2, 64
+    idx = np.zeros((T, K), dtype=np.int32)
+    idx[:, 1] = 1
+    idx[3, 0] = 9
+    idx[6, 1] = 8        # == N: out of range as well
+    bad = {(3, 0), (6, 1)}
+    rng = np.random.default_rng(21)
+    rows32 = rng.standard_normal((T, l)).astype(np.float32)
+    # powers of two: every gate * row product is exact, so fused and separate
+    # multiply-adds round alike and the comparison can be bit-exact
+    w = rng.choice([0.25, 0.5, 1.0, 2.0], size=(T, K)).astype(np.float32)
+    cfg = L.config(T=T, d=l, l=l, N=N, K=K, m=64)
+    P = L.padded_rows(cfg)
+    z32 = lambda n: torch.zeros(n, dtype=torch.int32, device="cuda")
+    rows = torch.from_numpy(rows32).cuda().to(torch.bfloat16)
+    prow = torch.zeros((P, l), dtype=torch.bfloat16, device="cuda")
+    pgate = torch.zeros(P, dtype=torch.float32, device="cuda")
+    offsets, perm_src, inv_perm, poff = z32(N + 1), z32(T * K), z32(T * K), z32(N + 1)
+    idx_d = torch.from_numpy(idx).cuda()
+    w_d = torch.from_numpy(w).cuda()
+    ws = L.workspace(cfg, L.OP_PERMUTE)
+    L.permute(cfg, idx_d, offsets, perm_src, inv_perm, poff, rows, l * 2, prow, None, None, w_d, pgate, ws=ws)
+    st, info = L.read_device_error(ws)
+    assert st == L.ERR_DEVICE_BOUNDS and info in (3 * K + 0, 6 * K + 1)
+    off, pf = offsets.cpu().numpy(), poff.cpu().numpy()
+    assert off[N] == T * K - len(bad)
+    assert off[1] - off[0] == T - 1 and off[2] - off[1] == T - 1 and off[N] == off[2]
+    # exactly the in-range slots are gathered, with their gates; padding stays zero
+    expect = torch.zeros((P, l), dtype=torch.bfloat16)
+    gexp = torch.zeros(P, dtype=torch.float32)
+    ip = inv_perm.cpu().numpy()
+    for t in range(T):
+        for k in range(K):
+            if (t, k) in bad:
+                continue
+            e = idx[t, k]
+            p = ip[t * K + k] - off[e] + pf[e]
+            expect[p] = rows[t].cpu()
+            gexp[p] = float(w[t, k])
+    assert torch.equal(prow.cpu(), expect)
+    assert torch.equal(pgate.cpu(), gexp)
+    # combine over the gathered rows: c_t = sum over in-range k, fp32 in k order
+    c = torch.zeros((T, l), dtype=torch.bfloat16, device="cuda")
+    L.combine(cfg, prow, idx_d, inv_perm, offsets, poff, w_d, c)
+    torch.cuda.synchronize()
+    rb = rows.float().cpu().numpy()
+    acc = np.zeros((T, l), dtype=np.float32)
+    for t in range(T):
+        for k in range(K):
+            if (t, k) not in bad:
+                acc[t] += np.float32(w[t, k]) * rb[t]
+    assert torch.equal(c.cpu(), torch.from_numpy(acc).to(torch.bfloat16))
