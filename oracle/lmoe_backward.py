@@ -1,0 +1,249 @@
+"""Plain, slow, fp64 CPU oracle of the LatentMoE layer's backward pass and of
+the NVFP4 training recipe's pieces.
+
+TEST INFRASTRUCTURE. Only the test suite may import this module. The CUDA
+library never calls it and shares no code with it.
+
+What it computes.
+
+* ``backward``: the gradients of the layer forward of ``lmoe_oracle`` (its
+  fp64 form, no rounding points) with respect to x and every weight, for an
+  upstream gradient dout [T, d]. The layer is the one of the Nemotron 3
+  whitepaper as summarised on the greeksharifa page, section 2.2 "LatentMoE"
+  (router and shared experts on the d-dim x, routed experts in the latent l).
+  The choice of the K experts is piecewise constant in the logits, so away
+  from ties the router receives gradient only through the K renormalised
+  gates g_k = exp(l_k) / sum_j exp(l_j) (j over the chosen K), whose
+  derivative is dg_k / dl_j = g_k (delta_kj - g_j) for chosen j and 0 for the
+  others.
+* The NVFP4 training recipe named on the same page, section 2.4 "NVFP4
+  Training", and on the Japanese summary page, section 4 "NVFP4 pre-training":
+  weights, activations and gradients are quantised so that fprop, dgrad and
+  wgrad run as NVFP4 GEMMs; weights use two-dimensional scale blocks; the
+  inputs of wgrad get a random Hadamard transform; gradients are rounded
+  stochastically. The pages give no more detail; the readings taken:
+  - RHT: 16-point blocks along the contraction dimension, each block v mapped
+    to H16 diag(s) v / 4 with H16 the Sylvester Hadamard matrix and s a
+    random +-1 vector of 16 signs shared by all blocks (an input). It is
+    orthonormal, so it leaves an unquantised wgrad product unchanged.
+  - Stochastic rounding of an element to E2M1: between its two grid
+    neighbours lo <= |v| < hi it takes hi when u * (hi - lo) < |v| - lo for a
+    uniform u in [0, 1) (an input, one per element), else lo; |v| >= 6
+    saturates to 6; the sign is kept. The block scales still round to
+    nearest even.
+  - Which operand gets what, for one linear layer Y = X W^T: dgrad
+    dX = dY W quantises dY along its rows (the contraction dim) with
+    stochastic rounding and W with 16 x 16 blocks (the fprop codes, as 2-D
+    blocks quantise W and W^T alike); wgrad dW = dY^T X transforms dY and X
+    along the tokens (the contraction dim), then quantises both along the
+    tokens, dY with stochastic rounding and X to nearest.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import lmoe_oracle as O
+
+# ----------------------------------------------------------------------------
+# The layer's gradients (fp64)
+# ----------------------------------------------------------------------------
+
+
+class ParamWeights:
+    """fp64 weights in the interface ``lmoe_oracle.forward`` reads
+    (``dense(key)``, ``expert(key, e)``, storage tag ``st``)."""
+
+    def __init__(self, params: dict):
+        self.p = params
+        self.st = "f64"
+
+    def dense(self, key):
+        return self.p[key]
+
+    def expert(self, key, e):
+        return self.p[key][e]
+
+
+def params_from_inputs(wl, inp) -> dict:
+    """fp64 values of a workload's stored inputs, as the layer reads them
+    (NVFP4 expert matrices dequantised)."""
+    W = O._Weights(wl, inp)
+    p = {"x": W.dense("x"), "w_router": W.dense("w_router"), "router_bias": inp.get("router_bias")}
+    p["w_down"] = None if wl.identity else W.dense("w_down")
+    p["w_up"] = None if wl.identity else W.dense("w_up")
+    p["w1"] = np.stack([W.expert("w1", e) for e in range(wl.N)])
+    p["w2"] = np.stack([W.expert("w2", e) for e in range(wl.N)])
+    p["ws1"] = W.dense("ws1") if wl.n_shared else None
+    p["ws2"] = W.dense("ws2") if wl.n_shared else None
+    return p
+
+
+def backward(params: dict, K: int, dout) -> dict:
+    """Gradients of out = layer(params) contracted with dout [T, d].
+
+    params: fp64 arrays x [T, d], w_router [N, d], router_bias [N] or None,
+    w_down [l, d] / w_up [d, l] (both None for identity projections),
+    w1 [N, m, l], w2 [N, l, m], ws1 [S, m_s, d] / ws2 [S, d, m_s] or None.
+
+    Returns dx, dw_router, drouter_bias (None without a bias), dw_down,
+    dw_up (None for identity), dw1, dw2, dws1, dws2 (None without shared
+    experts), and the forward's idx and gates.
+    """
+    x = np.asarray(params["x"], dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    T = x.shape[0]
+    wr, bias = params["w_router"], params.get("router_bias")
+    w_down, w_up = params.get("w_down"), params.get("w_up")
+    w1, w2 = params["w1"], params["w2"]
+    N = w1.shape[0]
+
+    # forward quantities the gradients need
+    logits = O.router_logits(x, wr, bias)
+    idx, gates = O.route_topk(logits, K)
+    z = x if w_down is None else x @ w_down.T
+
+    # up-projection: out = c W_up^T (+ shared); c = sum_k g_k o_k
+    dc = dout if w_up is None else dout @ w_up
+    c = np.zeros((T, z.shape[1]))
+    dz = np.zeros_like(z)
+    dgate = np.zeros((T, K))
+    dw1 = np.zeros_like(w1)
+    dw2 = np.zeros_like(w2)
+    for e in range(N):
+        t, k = np.nonzero(idx == e)          # the slots routed to expert e
+        if t.size == 0:
+            continue
+        ze = z[t]
+        h = ze @ w1[e].T                     # [n_e, m]
+        a = O.sq_relu(h)
+        o = a @ w2[e].T                      # ungated expert output [n_e, l]
+        g = gates[t, k]
+        np.add.at(c, t, g[:, None] * o)
+        dy = dc[t]                           # gradient reaching each slot's gated output
+        dgate[t, k] = np.sum(dy * o, axis=1)
+        do = g[:, None] * dy
+        dw2[e] = do.T @ a
+        dh = (do @ w2[e]) * 2.0 * np.maximum(h, 0.0)
+        dw1[e] = dh.T @ ze
+        np.add.at(dz, t, dh @ w1[e])
+    dw_up = None if w_up is None else dout.T @ c
+
+    # gates -> logits (renormalised softmax over the chosen K)
+    dsel = gates * (dgate - np.sum(gates * dgate, axis=1, keepdims=True))
+    dlogits = np.zeros((T, N))
+    np.put_along_axis(dlogits, idx.astype(np.int64), dsel, axis=1)
+    dw_router = dlogits.T @ x
+    dbias = None if bias is None else np.sum(dlogits, axis=0)
+    dx = dlogits @ wr
+
+    # down-projection
+    if w_down is None:
+        dw_down = None
+        dx = dx + dz
+    else:
+        dw_down = dz.T @ x
+        dx = dx + dz @ w_down
+
+    # shared experts on x: out += relu(x Ws1_s^T)^2 Ws2_s^T
+    dws1 = dws2 = None
+    if params.get("ws1") is not None:
+        ws1, ws2 = params["ws1"], params["ws2"]
+        dws1, dws2 = np.zeros_like(ws1), np.zeros_like(ws2)
+        for s in range(ws1.shape[0]):
+            pre = x @ ws1[s].T
+            hs = O.sq_relu(pre)
+            dws2[s] = dout.T @ hs
+            dpre = (dout @ ws2[s]) * 2.0 * np.maximum(pre, 0.0)
+            dws1[s] = dpre.T @ x
+            dx = dx + dpre @ ws1[s]
+
+    return dict(dx=dx, dw_router=dw_router, drouter_bias=dbias, dw_down=dw_down, dw_up=dw_up,
+                dw1=dw1, dw2=dw2, dws1=dws1, dws2=dws2, idx=idx, gates=gates)
+
+
+# ----------------------------------------------------------------------------
+# NVFP4 training pieces
+# ----------------------------------------------------------------------------
+
+
+def hadamard16() -> np.ndarray:
+    """The 16 x 16 Sylvester Hadamard matrix (entries +-1): H_1 = [1],
+    H_2n = [[H_n, H_n], [H_n, -H_n]]."""
+    H = np.ones((1, 1))
+    while H.shape[0] < 16:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def rht(X, signs, axis: int = 0) -> np.ndarray:
+    """Random Hadamard transform of X along ``axis`` (its length a multiple of
+    16): every block of 16 consecutive entries v becomes H16 diag(signs) v / 4."""
+    X = np.asarray(X, dtype=np.float64)
+    signs = np.asarray(signs, dtype=np.float64)
+    assert signs.shape == (16,) and np.all(np.abs(signs) == 1.0)
+    Xm = np.moveaxis(X, axis, 0)
+    n = Xm.shape[0]
+    assert n % 16 == 0
+    M = hadamard16() * signs[None, :] / 4.0
+    blocks = Xm.reshape((n // 16, 16) + Xm.shape[1:])
+    out = np.einsum("ij,bj...->bi...", M, blocks).reshape(Xm.shape)
+    return np.moveaxis(out, 0, axis)
+
+
+def e2m1_sr_encode(v, u) -> np.ndarray:
+    """Stochastic rounding to E2M1 codes: |v| >= 6 -> 6; otherwise, with
+    lo <= |v| < hi the neighbouring grid points, hi if u * (hi - lo) < |v| - lo
+    else lo (exact comparison; u in [0, 1)). The sign bit is the sign of v."""
+    v = np.asarray(v, dtype=np.float64)
+    u = np.broadcast_to(np.asarray(u, dtype=np.float64), v.shape)
+    a = np.abs(v)
+    grid = O.E2M1_MAG
+    lo_i = np.clip(np.searchsorted(grid, a, side="right") - 1, 0, len(grid) - 1)
+    hi_i = np.minimum(lo_i + 1, len(grid) - 1)
+    lo, hi = grid[lo_i], grid[hi_i]
+    up = (hi_i > lo_i) & (u * (hi - lo) < a - lo)
+    code = np.where(a >= O.E2M1_MAX, len(grid) - 1, np.where(up, hi_i, lo_i))
+    return (code | np.where(np.signbit(v), 8, 0)).astype(np.uint8)
+
+
+def nvfp4_quantize_sr(X, u, s_g: float | None = None):
+    """``lmoe_oracle.nvfp4_quantize`` with the element step rounded
+    stochastically (u [rows, cols] uniforms in [0, 1)); the global and block
+    scales are the round-to-nearest ones of that function."""
+    X = np.asarray(X, dtype=np.float64)
+    rows, cols = X.shape
+    _, sb_code, s_g = O.nvfp4_quantize(X, s_g)
+    sb = O.e4m3_decode(sb_code)
+    sc = O.round_f32(sb * s_g)
+    blocks = X.reshape(rows, cols // O.NVFP4_BLOCK, O.NVFP4_BLOCK)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = O.round_f32(blocks / sc[..., None])
+    q = e2m1_sr_encode(v, np.asarray(u, dtype=np.float64).reshape(blocks.shape))
+    q = np.where((sb == 0.0)[..., None], np.uint8(0), q).astype(np.uint8).reshape(rows, cols)
+    codes = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
+    return codes, sb_code, s_g
+
+
+def _deq(q):
+    return O.nvfp4_dequantize(*q)
+
+
+def nvfp4_linear_backward(X, W, dY, signs, u_dgrad, u_wgrad) -> dict:
+    """dgrad and wgrad of one linear layer Y = X W^T under the NVFP4 training
+    recipe (readings in the module docstring); products summed in fp64.
+
+    X [T, n_in], W [n_out, n_in], dY [T, n_out] (T, n_in, n_out multiples of
+    16); signs [16]; u_dgrad [T, n_out] and u_wgrad [n_out, T] uniforms.
+    Returns dX [T, n_in] and dW [n_out, n_in].
+    """
+    X, W, dY = (np.asarray(a, dtype=np.float64) for a in (X, W, dY))
+    # dgrad: contraction over n_out; dY along its rows, W with 2-D blocks
+    dY_q = _deq(nvfp4_quantize_sr(dY, u_dgrad))
+    W_q = _deq(O.nvfp4_quantize_2d(W))
+    dX = dY_q @ W_q
+    # wgrad: contraction over the tokens; both operands transformed and
+    # quantised along the tokens
+    dYt = rht(dY, signs, axis=0).T          # [n_out, T]
+    Xt = rht(X, signs, axis=0).T            # [n_in, T]
+    dW = _deq(nvfp4_quantize_sr(dYt, u_wgrad)) @ _deq(O.nvfp4_quantize(Xt)).T
+    return dict(dX=dX, dW=dW)

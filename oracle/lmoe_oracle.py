@@ -52,9 +52,12 @@ def from_bf16_bits(u: np.ndarray) -> np.ndarray:
 
 
 def to_f64(a, dtype: str) -> np.ndarray:
-    """Stored tensor (uint16 BF16 bits or float32) -> exact float64 values."""
+    """Stored tensor (uint16 BF16 bits, float32, or float64 values passed
+    through with dtype "f64") -> exact float64 values."""
     if a is None:
         return None
+    if dtype == "f64":
+        return np.asarray(a, dtype=np.float64)
     if dtype == "f32":
         return np.asarray(a, dtype=np.float32).astype(np.float64)
     return from_bf16_bits(a)
