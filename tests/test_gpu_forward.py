@@ -26,8 +26,8 @@ L = pytest.importorskip("latentmoe_fwd_b200")
 from gpu_util import DevLayer, as_f64, bf16_parity, rel_max_err  # noqa: E402
 
 
-def _check_layer(wl, tol):
-    inp = LI.make_inputs(wl)
+def _check_layer(wl, tol, inp=None):
+    inp = LI.make_inputs(wl) if inp is None else inp
     dev = DevLayer(wl, inp)
     out = as_f64(dev.forward())
     ref = O.forward(wl, inp)
@@ -127,3 +127,22 @@ def test_top_1_of_8_experts():
     # of 8); T*K >= 64*N puts the expert GEMMs on CTA pairs
     wl = LI.Workload("top1_of_8", T=700, d=256, l=128, N=8, K=1, m=192, dtype="bf16")
     _check_layer(wl, BF16_TOL)
+
+
+@pytest.mark.parametrize("T,N,K", [(700, 16, 2), (2100, 32, 4), (48, 16, 2)])
+def test_every_token_routed_to_the_same_experts(T, N, K):
+    # a router bias of +100 on K experts sends every token to those K: each
+    # takes all T rows (several tiles, CTA pairs for T > 64, weight-major
+    # 48-token tiles below), every other expert is empty; one shared expert
+    # rides along
+    wl = LI.Workload("same_experts", T=T, d=256, l=128, N=N, K=K, m=192, n_shared=1, m_shared=128,
+                     dtype="bf16")
+    inp = LI.make_inputs(wl)
+    hot = np.arange(K) * 3 + 1
+    bias = np.zeros(N, dtype=np.float32)
+    bias[hot] = 100.0
+    inp["router_bias"] = bias
+    ref_idx = O.route_topk(O.router_logits(O.to_f64(inp["x"], "bf16"), O.to_f64(inp["w_router"], "bf16"),
+                                           bias), K)[0]
+    assert np.all(np.sort(ref_idx, axis=1) == np.sort(hot))
+    _check_layer(wl, BF16_TOL, inp)
