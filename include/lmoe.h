@@ -147,12 +147,13 @@ typedef enum {
 } lmoe_op;
 
 /* Bytes of workspace `op` needs for `cfg` (for LMOE_OP_NVFP4_QUANTIZE the
- * tensor is taken as [cfg->T][cfg->l]). Returns 0 for an invalid config. */
+ * tensor is taken as [cfg->T][cfg->l]). Returns 0 for an invalid config or
+ * an unknown op, and for LMOE_OP_COMBINE (which needs none). */
 size_t lmoe_workspace_size(const lmoe_config* cfg, int op);
 
 /* Rows of the expert-grouped (padded) buffers: each expert's rows start at a
  * multiple of 128, so the buffers hold at most T*K + N*127 rows, rounded up
- * to a multiple of 128. */
+ * to a multiple of 128. Returns 0 for an invalid config. */
 int64_t lmoe_padded_rows(const lmoe_config* cfg);
 
 /* Router: logits = x W_r^T + b, then per token the K experts with the largest
@@ -163,7 +164,11 @@ int64_t lmoe_padded_rows(const lmoe_config* cfg);
  *  logits_in: NULL to compute the logits; else [T][N] F32 logits to route
  *    (x, w_router, bias are then ignored and may be NULL).
  *  topk_idx [T][K] int32, topk_w [T][K] F32: outputs.
- *  logits_out [T][N] F32 or NULL: the computed logits (bias included). */
+ *  logits_out [T][N] F32 or NULL: the computed logits (bias included).
+ *  Errors: the config checks above; LMOE_ERR_INVALID_ARG for NULL outputs,
+ *  NULL x or w_router when logits are computed, or x / w_router not 16-byte
+ *  aligned; LMOE_ERR_UNSUPPORTED for N % 8 when logits are computed;
+ *  LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT. */
 lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_router,
                        const float* bias, const float* logits_in, int32_t* topk_idx,
                        float* topk_w, float* logits_out, void* ws, size_t ws_bytes,
@@ -186,7 +191,13 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
  *  rows_sf / permuted_sf (optional): NVFP4 row-major scales [T][row_cols/16]
  *    of `rows`, re-laid to LMOE_SF_MMA_TILED at the padded rows; row_cols is
  *    2*row_bytes (the rows then hold packed E2M1 codes).
- *  topk_w / perm_gate (optional): the gate of each padded row ([padded] F32). */
+ *  topk_w / perm_gate (optional): the gate of each padded row ([padded] F32).
+ *  Errors: the config checks above; LMOE_ERR_INVALID_ARG for a NULL index
+ *  buffer, rows without permuted_rows (or scales, gates without their
+ *  destination), row_bytes not a positive multiple of 16, unaligned rows,
+ *  scales whose row width 2*row_bytes is not a multiple of 64;
+ *  LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_BOUNDS (info = the
+ *  first out-of-range slot f seen). */
 lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_t* offsets,
                          int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
                          const void* rows, int64_t row_bytes, void* permuted_rows,
@@ -223,7 +234,10 @@ lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_t* topk_idx
  *    (device pointer to one F32).
  *  offsets, padded_offsets [N+1]: from lmoe_permute.
  *  perm_gate [padded] F32 or NULL (gates of 1).
- *  y_perm [padded][l] (act): output; padding rows are left unspecified. */
+ *  y_perm [padded][l] (act): output; padding rows are left unspecified.
+ *  Errors: the config checks above; LMOE_ERR_INVALID_ARG for NULL or
+ *  unaligned buffers or weights (NVFP4: also missing scales or global
+ *  scales); LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT. */
 lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w,
                             const void* permuted_in, const uint8_t* permuted_sf,
                             const float* in_global_scale, const int32_t* offsets,
@@ -234,7 +248,9 @@ lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w,
  * in k order, stored as `act`; row(f) = inv_perm[f] - offsets[e] +
  * padded_offsets[e] with e = topk_idx[f]. topk_w NULL means the gates were
  * already applied (w = 1). c [T][l]. No workspace. A slot whose expert index
- * is out of range (left out by lmoe_permute) contributes nothing. */
+ * is out of range (left out by lmoe_permute) contributes nothing.
+ * Errors: the config checks above; LMOE_ERR_INVALID_ARG for NULL buffers or
+ * unaligned y_perm / c. There is no error word (no device errors). */
 lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32_t* topk_idx,
                          const int32_t* inv_perm, const int32_t* offsets,
                          const int32_t* padded_offsets, const float* topk_w, void* c,
@@ -244,7 +260,13 @@ lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32
  * amax), permute, expert FFNs, combine, up-project and add the shared
  * experts. x [T][d] (act) -> out [T][d] (act). N must be a multiple of 8
  * (the router GEMM stores logit rows in 16-byte vectors; LMOE_ERR_UNSUPPORTED
- * otherwise, also from lmoe_route when it computes the logits). */
+ * otherwise, also from lmoe_route when it computes the logits).
+ * Errors: the config checks above; LMOE_ERR_INVALID_ARG for NULL w,
+ * w_router, w1 or w2, w_down / w_up given with LMOE_FLAG_IDENTITY_PROJ or
+ * missing without it, missing shared-expert weights, missing NVFP4 scales,
+ * NULL or unaligned x / out (not checked when T == 0, which launches
+ * nothing), or a weight a TMA descriptor cannot address (not 16-byte
+ * aligned); LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT. */
 lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x,
                          void* out, void* ws, size_t ws_bytes, void* stream);
 
@@ -279,8 +301,10 @@ lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int6
                                 void* stream);
 
 /* Synchronises `stream`, returns the device error status recorded in the
- * workspace `ws` (LMOE_OK if none) and clears it. `info` (host, may be NULL)
- * receives a kernel-specific detail word. */
+ * workspace `ws` (LMOE_OK if none) and clears it (the read and the clear run
+ * on `stream`). `info` (host, may be NULL) receives a kernel-specific detail
+ * word. Errors: LMOE_ERR_INVALID_ARG for a NULL ws; LMOE_ERR_CUDA when the
+ * synchronisation, the read or the clear fails. */
 lmoe_status lmoe_read_device_error(void* ws, void* stream, uint32_t* info);
 
 /* Static description of a status code. */
