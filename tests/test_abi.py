@@ -158,3 +158,28 @@ def test_noalloc_permute_host_checks():
     assert call(L.config(T=4, d=8, l=8, N=2048, K=2, m=8)) == L.ERR_UNSUPPORTED
     # beyond the fixed 131072-counter scratch: (ceil(T*K / 8192) + 1) * N counters
     assert call(L.config(T=300000, d=8, l=8, N=1024, K=8, m=8)) == L.ERR_WORKSPACE
+
+
+def test_documented_host_errors_of_each_entry_point():
+    P = ctypes.byref
+    cfg = L.config(T=4, d=64, l=32, N=8, K=2, m=64)
+    w = L.weights(w_router=16, w1=16, w2=16, w_down=16, w_up=16)
+    big = 1 << 40
+    # expert FFN: missing weights, unaligned output, NVFP4 without scales
+    assert L.lib.lmoe_expert_ffn(P(cfg), P(L.weights(w1=16)), 16, None, None, 16, 16, None, 16, 16, big,
+                                 None) == L.ERR_INVALID_ARG
+    assert L.lib.lmoe_expert_ffn(P(cfg), P(w), 16, None, None, 16, 16, None, 24, 16, big, None) == L.ERR_INVALID_ARG
+    assert L.lib.lmoe_expert_ffn(P(cfg), P(w), 16, None, None, 16, 16, None, 16, 16, 8, None) == L.ERR_WORKSPACE
+    cfg4 = L.config(T=4, d=256, l=256, N=8, K=2, m=256, expert=L.NVFP4)
+    assert L.lib.lmoe_expert_ffn(P(cfg4), P(w), 16, 16, 16, 16, 16, None, 16, 16, big, None) == L.ERR_INVALID_ARG
+    # combine: NULL or unaligned buffers
+    assert L.lib.lmoe_combine(P(cfg), None, 16, 16, 16, 16, None, 16, None) == L.ERR_INVALID_ARG
+    assert L.lib.lmoe_combine(P(cfg), 16, 16, 16, 16, 16, None, 40, None) == L.ERR_INVALID_ARG
+    # forward: projections given with the identity flag; missing shared weights
+    ident = L.config(T=4, d=64, l=64, N=8, K=2, m=64, identity=True)
+    assert L.lib.lmoe_forward(P(ident), P(w), 16, 16, 16, big, None) == L.ERR_INVALID_ARG
+    shared = L.config(T=4, d=64, l=32, N=8, K=2, m=64, n_shared=1, m_shared=64)
+    assert L.lib.lmoe_forward(P(shared), P(w), 16, 16, 16, big, None) == L.ERR_INVALID_ARG
+    # reading the error word needs a workspace
+    info = ctypes.c_uint32(0)
+    assert L.lib.lmoe_read_device_error(None, None, ctypes.byref(info)) == L.ERR_INVALID_ARG
