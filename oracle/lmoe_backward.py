@@ -37,6 +37,9 @@ What it computes.
     blocks quantise W and W^T alike); wgrad dW = dY^T X transforms dY and X
     along the tokens (the contraction dim), then quantises both along the
     tokens, dY with stochastic rounding and X to nearest.
+  - The uniforms: passed in, or drawn by ``sr_uniforms`` from Philox-4x32-10
+    (the counter-based generator of Salmon et al., SC11), which a kernel can
+    evaluate element by element from the same published definition.
 """
 from __future__ import annotations
 
@@ -222,6 +225,45 @@ def nvfp4_quantize_sr(X, u, s_g: float | None = None):
     q = np.where((sb == 0.0)[..., None], np.uint8(0), q).astype(np.uint8).reshape(rows, cols)
     codes = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
     return codes, sb_code, s_g
+
+
+# Philox-4x32-10 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
+# SC11, section 5): the counter-based generator both sides of a stochastic
+# rounding kernel can evaluate independently, element by element.
+_PHILOX_M = (0xD2511F53, 0xCD9E8D57)
+_PHILOX_W = (0x9E3779B9, 0xBB67AE85)
+
+
+def philox4x32_10(counter, key) -> np.ndarray:
+    """Philox-4x32-10 of counters [..., 4] (uint32 words) under key [2]:
+    ten rounds; each round takes the 64-bit products of words 0 and 2 with the
+    two multipliers and sets (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0); the key
+    grows by the two Weyl constants between rounds. Returns [..., 4] uint32."""
+    c = np.asarray(counter, dtype=np.uint64) & np.uint64(0xFFFFFFFF)
+    k0, k1 = (int(v) & 0xFFFFFFFF for v in key)
+    c0, c1, c2, c3 = (c[..., i] for i in range(4))
+    m32 = np.uint64(0xFFFFFFFF)
+    for r in range(10):
+        if r:
+            k0 = (k0 + _PHILOX_W[0]) & 0xFFFFFFFF
+            k1 = (k1 + _PHILOX_W[1]) & 0xFFFFFFFF
+        p0 = c0 * np.uint64(_PHILOX_M[0])
+        p1 = c2 * np.uint64(_PHILOX_M[1])
+        c0, c1, c2, c3 = ((p1 >> np.uint64(32)) ^ c1 ^ np.uint64(k0), p1 & m32,
+                          (p0 >> np.uint64(32)) ^ c3 ^ np.uint64(k1), p0 & m32)
+    return np.stack([c0, c1, c2, c3], axis=-1).astype(np.uint32)
+
+
+def sr_uniforms(n: int, seed: int, stream: int = 0) -> np.ndarray:
+    """n uniforms in [0, 1) for stochastic rounding, element i from word i % 4
+    of Philox-4x32-10 at counter (i // 4 low word, i // 4 high word, stream, 0)
+    under key (seed low word, seed high word): u = (word >> 8) * 2^-24, a
+    24-bit value every fp32 holds exactly."""
+    i = np.arange((n + 3) // 4, dtype=np.uint64)
+    ctr = np.stack([i & np.uint64(0xFFFFFFFF), i >> np.uint64(32),
+                    np.full_like(i, stream & 0xFFFFFFFF), np.zeros_like(i)], axis=-1)
+    words = philox4x32_10(ctr, (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)).reshape(-1)[:n]
+    return (words >> np.uint32(8)).astype(np.float64) * 2.0 ** -24
 
 
 def _deq(q):

@@ -295,3 +295,29 @@ def test_nvfp4_wgrad_exact_when_the_transformed_operands_are_representable():
     r = B.nvfp4_linear_backward(X, W, dY, s, rng.random((T, n_out)), rng.random((n_out, T)))
     assert np.array_equal(r["dW"], Rd @ Rx.T)
     assert np.allclose(r["dW"], dY.T @ X, rtol=1e-12, atol=1e-9)
+
+
+def test_philox_known_answer_vectors():
+    rows = []
+    with open(__file__.replace("test_oracle_backward.py", "golden/philox4x32_10_kat.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([int(w, 16) for w in line.split()])
+    assert len(rows) == 3
+    for r in rows:
+        got = B.philox4x32_10(np.array(r[:4], dtype=np.uint64), r[4:6])
+        assert got.tolist() == r[6:10]
+    # vectorised over counters: the same words as one call per counter
+    ctrs = np.array([r[:4] for r in rows], dtype=np.uint64)
+    assert B.philox4x32_10(ctrs, rows[0][4:6])[0].tolist() == rows[0][6:10]
+
+
+def test_sr_uniforms_layout_and_range():
+    u = B.sr_uniforms(10, seed=5, stream=2)
+    w = B.philox4x32_10(np.array([[0, 0, 2, 0], [1, 0, 2, 0], [2, 0, 2, 0]], dtype=np.uint64), (5, 0)).reshape(-1)
+    assert np.array_equal(u, (w[:10] >> 8).astype(np.float64) / 2.0 ** 24)
+    big = B.sr_uniforms(1 << 20, seed=1)
+    assert big.min() >= 0.0 and big.max() < 1.0
+    assert np.all(big * 2.0 ** 24 == np.floor(big * 2.0 ** 24))         # 24-bit values
+    assert abs(big.mean() - 0.5) < 5 * np.sqrt(1 / 12 / big.size)
+    assert not np.array_equal(B.sr_uniforms(64, seed=1), B.sr_uniforms(64, seed=1, stream=1))
