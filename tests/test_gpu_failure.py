@@ -2,7 +2,6 @@
 out (an mbarrier nothing arrives on) records LMOE_ERR_DEVICE_TIMEOUT in the
 workspace error word and returns; the host reads the status and the context
 stays usable for the next layer forward."""
-import numpy as np
 import pytest
 import torch
 

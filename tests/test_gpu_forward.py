@@ -12,7 +12,6 @@ oracle's exactly except on near-ties (gap between the K-th and (K+1)-th logit
 Sizes span several 128-row tiles per expert, ragged last tiles, ragged
 output-feature tiles and both GEMM tile kinds (token-major and weight-major).
 """
-from dataclasses import replace
 
 import numpy as np
 import pytest

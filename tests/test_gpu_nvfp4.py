@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 
 L = pytest.importorskip("latentmoe_fwd_b200")
 import nvfp4_ties  # noqa: E402
-from gpu_util import DevLayer, as_f64, bf16_parity, quantize_dev  # noqa: E402
+from gpu_util import DevLayer, as_f64, quantize_dev  # noqa: E402
 
 
 def _bf16_dev(v: np.ndarray):
