@@ -168,12 +168,11 @@ int normal_bn(int cols) { return cols >= 256 ? 256 : cols > 64 ? 128 : cols > 32
 
 int kblocks(int64_t k) { return static_cast<int>((k + 63) / 64); }
 
-// out[rows, cols] = epi(x[rows, k] . W[cols, k]^T) with BF16 operands.
 // Splits for a weight-major GEMM with `tiles` output tiles and `kb` K blocks:
 // as many as fit in one wave of the GPU (a second, partial wave would double
 // the time of a weight-streaming GEMM), at least two K blocks per split,
 // within the buffer.
-int choose_splits(int64_t tiles, int kb, int64_t rows, int64_t cols, float* partial) {
+int choose_splits(int64_t tiles, int kb, float* partial) {
   if (!partial) return 1;
   const int sms = device_sm_count();
   int sp = static_cast<int>(sms / tiles);
@@ -197,6 +196,7 @@ int tokmajor_splits(int64_t rows, int cols, int64_t k) {
   return sp > 1 ? sp : 1;
 }
 
+// out[rows, cols] = epi(x[rows, k] . W[cols, k]^T) with BF16 operands.
 lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int64_t k, void* out,
                        int64_t ld_out, int epi, const float* bias, const void* residual, int64_t ld_res,
                        float* partial, uint32_t* err, cudaStream_t s) {
@@ -214,7 +214,7 @@ lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int
     L.a[0] = wt;
     L.b[0] = act;
     L.max_tiles = (cols + 127) / 128;
-    L.ksplit = choose_splits(L.max_tiles, L.kblocks[0], rows, cols, partial);
+    L.ksplit = choose_splits(L.max_tiles, L.kblocks[0], partial);
     L.partial = partial;
   } else {
     L.bn = normal_bn(cols);
@@ -854,7 +854,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     U.swap = 1;
     U.bn = sbn;
     U.max_tiles = (d + 127) / 128;
-    U.ksplit = choose_splits(U.max_tiles, U.kblocks[0] + (U.nseg > 1 ? U.kblocks[1] : 0), T, d, splitk);
+    U.ksplit = choose_splits(U.max_tiles, U.kblocks[0] + (U.nseg > 1 ? U.kblocks[1] : 0), splitk);
     U.partial = splitk;
   } else {
     U.bn = normal_bn(d);
