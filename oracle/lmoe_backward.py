@@ -270,22 +270,124 @@ def _deq(q):
     return O.nvfp4_dequantize(*q)
 
 
-def nvfp4_linear_backward(X, W, dY, signs, u_dgrad, u_wgrad) -> dict:
+def nvfp4_linear_backward(X, W, dY, signs, u_dgrad, u_wgrad, quantize: bool = True) -> dict:
     """dgrad and wgrad of one linear layer Y = X W^T under the NVFP4 training
     recipe (readings in the module docstring); products summed in fp64.
 
     X [T, n_in], W [n_out, n_in], dY [T, n_out] (T, n_in, n_out multiples of
     16); signs [16]; u_dgrad [T, n_out] and u_wgrad [n_out, T] uniforms.
+    quantize=False makes every quantiser the identity (the transform stays),
+    which leaves the plain products dY W and dY^T X.
     Returns dX [T, n_in] and dW [n_out, n_in].
     """
     X, W, dY = (np.asarray(a, dtype=np.float64) for a in (X, W, dY))
+    q_sr = (lambda A, u: _deq(nvfp4_quantize_sr(A, u))) if quantize else (lambda A, u: A)
+    q_2d = (lambda A: _deq(O.nvfp4_quantize_2d(A))) if quantize else (lambda A: A)
+    q_rn = (lambda A: _deq(O.nvfp4_quantize(A))) if quantize else (lambda A: A)
     # dgrad: contraction over n_out; dY along its rows, W with 2-D blocks
-    dY_q = _deq(nvfp4_quantize_sr(dY, u_dgrad))
-    W_q = _deq(O.nvfp4_quantize_2d(W))
-    dX = dY_q @ W_q
+    dX = q_sr(dY, u_dgrad) @ q_2d(W)
     # wgrad: contraction over the tokens; both operands transformed and
     # quantised along the tokens
     dYt = rht(dY, signs, axis=0).T          # [n_out, T]
     Xt = rht(X, signs, axis=0).T            # [n_in, T]
-    dW = _deq(nvfp4_quantize_sr(dYt, u_wgrad)) @ _deq(O.nvfp4_quantize(Xt)).T
+    dW = q_sr(dYt, u_wgrad) @ q_rn(Xt).T
     return dict(dX=dX, dW=dW)
+
+
+def _fake_quant(A, s_g=None):
+    return O.nvfp4_fake_quant(A, s_g)[0]
+
+
+def backward_nvfp4(params: dict, K: int, dout, signs, seed: int, a_global_scale=None,
+                   quantize: bool = True) -> dict:
+    """The layer's gradients with its routed experts trained under the NVFP4
+    recipe: the expert GEMMs' forward reads NVFP4 z (current amax), NVFP4 a
+    (``a_global_scale``, else its current amax) and 2-D-block NVFP4 weights;
+    their dgrad and wgrad are ``nvfp4_linear_backward``, with each expert's
+    rows padded by zero rows to a multiple of 16 for the token transform. The
+    router, the latent projections and the shared experts stay unquantised
+    (the recipe keeps such layers in higher precision; the latent projections
+    stay BF16 on the pages), and every quantiser passes its gradient straight
+    through. Uniforms come from ``sr_uniforms(seed, stream)`` with stream
+    4 e + 2 g + j for expert e, GEMM g (0: first, 1: second) and j (0: dgrad,
+    1: wgrad). quantize=False turns every quantiser into the identity.
+    Returns the same keys as ``backward``.
+    """
+    x = np.asarray(params["x"], dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    T = x.shape[0]
+    wr, bias = params["w_router"], params.get("router_bias")
+    w_down, w_up = params.get("w_down"), params.get("w_up")
+    w1, w2 = params["w1"], params["w2"]
+    N, m, l = w1.shape
+    fq = _fake_quant if quantize else (lambda A, s_g=None: A)
+    fq2 = (lambda A: _deq(O.nvfp4_quantize_2d(A))) if quantize else (lambda A: A)
+
+    logits = O.router_logits(x, wr, bias)
+    idx, gates = O.route_topk(logits, K)
+    z = x if w_down is None else x @ w_down.T
+    zq = fq(z)
+    dc = dout if w_up is None else dout @ w_up
+    c = np.zeros((T, l))
+    dz = np.zeros_like(z)
+    dgate = np.zeros((T, K))
+    dw1, dw2 = np.zeros_like(w1), np.zeros_like(w2)
+
+    def pad16(A):
+        R = -(-A.shape[0] // 16) * 16
+        out = np.zeros((R,) + A.shape[1:])
+        out[:A.shape[0]] = A
+        return out
+
+    def uni(rows, cols, stream):
+        return sr_uniforms(rows * cols, seed, stream).reshape(rows, cols)
+
+    for e in range(N):
+        t, k = np.nonzero(idx == e)
+        n = t.size
+        if n == 0:
+            continue
+        ze = zq[t]
+        h = ze @ fq2(w1[e]).T
+        aq = fq(O.sq_relu(h), a_global_scale)
+        o = aq @ fq2(w2[e]).T
+        g = gates[t, k]
+        np.add.at(c, t, g[:, None] * o)
+        dy = dc[t]
+        dgate[t, k] = np.sum(dy * o, axis=1)
+        do = g[:, None] * dy
+        R = -(-n // 16) * 16
+        r2 = nvfp4_linear_backward(pad16(aq), w2[e], pad16(do), signs, uni(R, l, 4 * e + 2),
+                                   uni(l, R, 4 * e + 3), quantize)
+        dw2[e] = r2["dW"]
+        dh = r2["dX"][:n] * 2.0 * np.maximum(h, 0.0)
+        r1 = nvfp4_linear_backward(pad16(ze), w1[e], pad16(dh), signs, uni(R, m, 4 * e + 0),
+                                   uni(m, R, 4 * e + 1), quantize)
+        dw1[e] = r1["dW"]
+        np.add.at(dz, t, r1["dX"][:n])
+    dw_up = None if w_up is None else dout.T @ c
+
+    dsel = gates * (dgate - np.sum(gates * dgate, axis=1, keepdims=True))
+    dlogits = np.zeros((T, N))
+    np.put_along_axis(dlogits, idx.astype(np.int64), dsel, axis=1)
+    dw_router = dlogits.T @ x
+    dbias = None if bias is None else np.sum(dlogits, axis=0)
+    dx = dlogits @ wr
+    if w_down is None:
+        dw_down = None
+        dx = dx + dz
+    else:
+        dw_down = dz.T @ x
+        dx = dx + dz @ w_down
+    dws1 = dws2 = None
+    if params.get("ws1") is not None:
+        ws1, ws2 = params["ws1"], params["ws2"]
+        dws1, dws2 = np.zeros_like(ws1), np.zeros_like(ws2)
+        for s in range(ws1.shape[0]):
+            pre = x @ ws1[s].T
+            dws2[s] = dout.T @ O.sq_relu(pre)
+            dpre = (dout @ ws2[s]) * 2.0 * np.maximum(pre, 0.0)
+            dws1[s] = dpre.T @ x
+            dx = dx + dpre @ ws1[s]
+    return dict(dx=dx, dw_router=dw_router, drouter_bias=dbias, dw_down=dw_down, dw_up=dw_up,
+                dw1=dw1, dw2=dw2, dws1=dws1, dws2=dws2, idx=idx, gates=gates)

@@ -321,3 +321,37 @@ def test_sr_uniforms_layout_and_range():
     assert np.all(big * 2.0 ** 24 == np.floor(big * 2.0 ** 24))         # 24-bit values
     assert abs(big.mean() - 0.5) < 5 * np.sqrt(1 / 12 / big.size)
     assert not np.array_equal(B.sr_uniforms(64, seed=1), B.sr_uniforms(64, seed=1, stream=1))
+
+
+@pytest.mark.parametrize("identity,S", [(False, 1), (True, 0)])
+def test_nvfp4_layer_backward_without_quantisation_is_the_exact_backward(identity, S):
+    """With every quantiser the identity, the NVFP4 composition (per-expert
+    padding, operand wiring, token transform) must reproduce the exact
+    gradients: the transform is orthonormal and the padding rows are zero."""
+    p = _params(41, T=21, d=32, l=32, N=5, m=48, S=S, ms=16, identity=identity)
+    dout = np.random.default_rng(6).standard_normal((21, 32))
+    s = np.random.default_rng(7).choice([-1.0, 1.0], 16)
+    exact = B.backward(p, 2, dout)
+    comp = B.backward_nvfp4(p, 2, dout, s, seed=3, quantize=False)
+    for k in GRADS:
+        if exact[k] is None:
+            assert comp[k] is None
+            continue
+        assert np.allclose(comp[k], exact[k], rtol=1e-10, atol=1e-12), k
+
+
+def test_nvfp4_layer_backward_seeds_and_quantisation():
+    p = _params(43, T=40, d=32, l=32, N=4, m=32, S=0)
+    dout = np.random.default_rng(8).standard_normal((40, 32))
+    s = np.random.default_rng(9).choice([-1.0, 1.0], 16)
+    a = B.backward_nvfp4(p, 2, dout, s, seed=1)
+    b = B.backward_nvfp4(p, 2, dout, s, seed=1)
+    c = B.backward_nvfp4(p, 2, dout, s, seed=2)
+    for k in ("dx", "dw1", "dw2", "dw_router"):
+        assert np.array_equal(a[k], b[k]), k                    # the uniforms are a function of the seed
+    assert not np.array_equal(a["dw1"], c["dw1"])              # stochastic rounding depends on them
+    exact = B.backward(p, 2, dout)
+    for k in ("dx", "dw1", "dw2"):
+        assert not np.allclose(a[k], exact[k], rtol=1e-6)      # the quantisers act
+        cos = np.sum(a[k] * exact[k]) / (np.linalg.norm(a[k]) * np.linalg.norm(exact[k]))
+        assert cos > 0.9, (k, cos)                              # and stay a gradient of the same layer
