@@ -40,6 +40,12 @@ What it computes.
   - The uniforms: passed in, or drawn by ``sr_uniforms`` from Philox-4x32-10
     (the counter-based generator of Salmon et al., SC11), which a kernel can
     evaluate element by element from the same published definition.
+* ``backward_nvfp4``: the layer's gradients with only its routed experts'
+  GEMMs under that recipe (NVFP4 z, a and 2-D-block weights in their
+  forward; ``nvfp4_linear_backward`` for their dgrad and wgrad, each
+  expert's rows padded with zero rows to a multiple of 16); the router, the
+  latent projections and the shared experts stay unquantised, and every
+  quantiser passes its gradient straight through.
 """
 from __future__ import annotations
 
