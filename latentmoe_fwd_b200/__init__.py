@@ -5,9 +5,11 @@ kernels. PyTorch provides device memory and streams. Importing this package
 loads the shared library and fails loudly if it has not been built
 (``python latentmoe_fwd_b200/build.py``).
 
-Entry points mirror include/lmoe.h: ``route``, ``permute``, ``expert_ffn``,
-``combine``, ``forward``, ``nvfp4_quantize``, plus ``workspace_size``,
-``padded_rows``, ``read_device_error`` and ``kernel_launch_count``.
+Entry points mirror include/lmoe.h: ``route``, ``permute`` (and
+``permute_noalloc``), ``expert_ffn``, ``combine``, ``forward`` (and
+``forward_traced``), ``nvfp4_quantize``, plus ``workspace_size``,
+``padded_rows``, ``workspace``, ``read_device_error``,
+``selftest_wait_timeout`` and ``kernel_launch_count``.
 Tensor arguments are torch tensors (or None); their ``data_ptr()`` is passed.
 """
 from __future__ import annotations
