@@ -14,7 +14,9 @@ one batch of T synthetic tokens, through the library's C ABI.
 * roofline: the grouped expert GEMM launches (the dominant kernel), timed
            with CUDA events recorded by the library at its stage boundaries
            on the launch stream (a pass of K forwards right after the timed
-           region), against the measured B200 peak.
+           region). Their algorithmic work is the layer's own: the used
+           experts' weights once (bytes) and 2*T*K*l*m*2 (flops); the binding
+           roof is the slower of the two at the measured burst peaks.
 * cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload
            (rank 0, N = 1 only).
 
@@ -44,7 +46,7 @@ sys.path.insert(0, ROOT)
 import lmoe_inputs as LI  # noqa: E402
 
 METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % of HBM (decode) or tensor (prefill) peak"
-DEFAULT_WORKLOAD = "std_moe_bf16"
+DEFAULT_WORKLOAD = "ultra_zipf"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -108,30 +110,39 @@ class ClockSampler:
 # algorithmic work of the dominant kernel (the two grouped expert GEMMs)
 # --------------------------------------------------------------------------
 def expert_gemm_work(wl, counts: np.ndarray):
-    """Algorithmic bytes and flops of expert GEMM 1 + GEMM 2 for one forward.
+    """Algorithmic work of expert GEMM 1 + GEMM 2 (the two grouped launches)
+    for one forward, by the layer's definition rather than this design's
+    data movement.
 
-    bytes = weights of every expert that received at least one row (W1_e and
-    W2_e once each) + the activation rows read and written (z rows in, a out,
-    a in, y out), in the storage format of the workload.
-    flops = 2 * (T*K) * l * m * 2.
+    bytes: W1_e and W2_e of every expert that received at least one row, each
+      read once, in the workload's weight format (NVFP4: 0.5 byte per element
+      plus one E4M3 scale per 16), plus the shared experts' Ws1 and Ws2 where
+      their two layers run in the same launches.
+    flops: 2 * (T*K) * l * m * 2 (+ 2 * T * d * S * m_s * 2 with the shared
+      layers).
+    traffic_model: the activation rows the two launches read and write in this
+      design (gathered z rows in, a out and back in, y out; with the shared
+      layers x in, hs out and back in, ys out). They are intermediates the
+      design materialises, reported beside the algorithmic bytes, not in them.
+    Returns (bytes, flops, experts used, traffic_model bytes).
     """
     rows = int(counts.sum())
     used = int(np.count_nonzero(counts))
     if wl.dtype == "nvfp4":
-        wbytes = used * 2 * wl.m * wl.l * (0.5 + 1.0 / 16)
-        abytes = rows * (wl.l + wl.m) * (0.5 + 1.0 / 16) + rows * (wl.m * (0.5 + 1.0 / 16) + wl.l * 2)
+        q = 0.5 + 1.0 / 16
+        wbytes = used * 2 * wl.m * wl.l * q
+        abytes = rows * (wl.l + wl.m) * q + rows * (wl.m * q + wl.l * 2)
     else:
         eb = 4 if wl.dtype == "f32" else 2
         wbytes = used * 2 * wl.m * wl.l * eb
         abytes = rows * (wl.l + wl.m) * eb * 2
     flops = 2.0 * rows * wl.l * wl.m * 2
     if wl.n_shared and shared_fused(wl):
-        # the shared experts' two layers run in the same two launches
         sm = wl.n_shared * wl.m_shared
         wbytes += 2 * sm * wl.d * 2
         abytes += wl.T * wl.d * 2 * 2 + wl.T * sm * 2 * 2
         flops += 2.0 * wl.T * wl.d * sm * 2
-    return wbytes + abytes, flops, used
+    return wbytes, flops, used, abytes
 
 
 def pair_tiles(wl) -> bool:
@@ -236,6 +247,37 @@ def quantizer_rates(L, w, hbm_gbs):
     return out
 
 
+def roofline(wl, alg_bytes, alg_flops, gemm_ms, peaks, peak_src):
+    """Roofline of the expert-GEMM launches against the burst peaks (the
+    launches are timed inside millisecond steps, not seconds-long loops).
+
+    The binding roof is the slower of bytes / HBM copy bandwidth and flops /
+    dense tensor peak (BF16 burst; NVFP4: 4 x the BF16 burst, the nominal
+    9 : 2.25 dense ratio). achieved = algorithmic work / measured launch time,
+    frac = achieved / peak. The sustained tensor peak is given beside it."""
+    if wl.dtype == "f32":
+        return {"bound": "launch", "achieved": None, "peak": None, "unit": None, "frac": None, "traffic": None,
+                "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops, "kernel_ms_per_step": gemm_ms}
+    ratio = 4.0 if wl.dtype == "nvfp4" else 1.0
+    tc_peak = peaks["bf16_tflops"] * ratio
+    tc_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * ratio
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = alg_flops / (tc_peak * 1e12)
+    src = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    tc_kind = "bf16_tflops x 4 (nominal FP4 : BF16 dense ratio)" if ratio > 1 else "bf16_tflops"
+    if t_hbm >= t_tc:
+        ach = alg_bytes / (gemm_ms / 1000.0) / 1e9
+        r = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": ach / peaks["hbm_gbs"], "peak_kind": "hbm_gbs"}
+    else:
+        ach = alg_flops / (gemm_ms / 1000.0) / 1e12
+        r = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak,
+             "peak_kind": tc_kind, "peak_sustained": tc_sust, "frac_of_sustained": ach / tc_sust}
+    r.update({"algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops, "kernel_ms_per_step": gemm_ms,
+              "time_at_hbm_peak_ms": t_hbm * 1e3, "time_at_tensor_peak_ms": t_tc * 1e3, "peak_source": src})
+    return r
+
+
 # --------------------------------------------------------------------------
 # the CPU oracle, timed (bounded sample)
 # --------------------------------------------------------------------------
@@ -278,12 +320,15 @@ def oracle_sample(wl, inp, n_tokens: int, min_seconds: float = 10.0, max_calls: 
 
 
 def run_reference(args, wl):
-    """Reference arm: the oracle on the host cores, K timed steps of a bounded sample."""
+    """Reference arm: the oracle on the host cores. Each step is one oracle
+    call on a fresh seeded sample of the workload's tokens, of the same size
+    as the CPU baseline's calls (CPU_SAMPLE_TOKENS), so the two measure the
+    same thing."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     inp = LI.make_inputs(wl)
-    per_step = max(1, 64 // max(1, args.steps))
+    per_step = min(args.cpu_sample or CPU_SAMPLE_TOKENS.get(wl.name, 32), wl.T)
     for i in range(args.warmup):
         oracle_tokens_per_s(wl, inp, per_step, seed=1000 + i)
     total_t, total_tok = 0.0, 0
@@ -299,8 +344,8 @@ def run_reference(args, wl):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(wl),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{per_step} random token(s) of the {wl.name} batch per step, "
-                                   f"fp64 NumPy oracle with full weights"},
+                         "sample": f"{args.steps} call(s) on {per_step} random tokens of the {wl.name} batch "
+                                   f"each ({total_tok} tokens), full weights, fp64 NumPy ({total_t:.1f} s)"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -318,9 +363,11 @@ def max_over_ranks(values, device):
 
 
 def workload_config(wl):
+    """The workload's description, identical in both arms."""
     c = {"workload": wl.name, "T": wl.T, "d": wl.d, "l": wl.l, "N": wl.N, "K": wl.K, "m": wl.m,
          "n_shared": wl.n_shared, "m_shared": wl.m_shared, "identity_projections": wl.identity,
-         "zipf_bias": wl.zipf_bias, "outliers": wl.outliers, "parallelism": "replicas (one layer per GPU)"}
+         "zipf_bias": wl.zipf_bias, "outliers": wl.outliers, "parallelism": "replicas (one layer per GPU)",
+         "l2": "no flush: weights alone exceed the 126 MB L2" if wl.dtype != "f32" else "tiny (fits L2)"}
     return c
 
 
@@ -409,7 +456,7 @@ def main():
     rws = L.workspace(cfg, L.OP_ROUTE)
     L.route(cfg, x, t["w_router"], bias, None, idx, gw, None, rws)
     counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=wl.N)
-    alg_bytes, alg_flops, used = expert_gemm_work(wl, counts)
+    alg_bytes, alg_flops, used, model_bytes = expert_gemm_work(wl, counts)
 
     for _ in range(args.warmup):
         L.forward(cfg, w, x, out, ws)
@@ -503,31 +550,10 @@ def main():
 
     peaks, peak_src = load_peaks()
     gemm_ms = stage_ms[3] + stage_ms[4]          # expert GEMM 1 + 2 (two launches)
-    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    if wl.dtype == "nvfp4":
-        tensor_peak = tensor_peak * 4.0          # nominal FP4 : BF16 dense ratio (9 : 2.25)
-    t_tc = alg_flops / (tensor_peak * 1e12)
-    if wl.dtype == "f32":
-        roof = {"bound": "launch", "achieved": None, "peak": None, "unit": None, "frac": None, "traffic": None}
-    elif t_hbm >= t_tc:
-        ach = alg_bytes / (gemm_ms / 1000.0) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"]}
-    else:
-        ach = alg_flops / (gemm_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": ach / tensor_peak}
-    if "traffic" not in roof:
-        tr = traffic_record(wl.name)
-        roof["traffic"] = tr
-    roof.update({
-        "kernel": expert_gemm_kernel(wl),
-        "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops, "experts_used": used,
-        "kernel_ms_per_step": gemm_ms, "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
-        else "fallback", "peak_kind": "hbm_gbs" if roof.get("bound") == "hbm" else
-        ("bf16_tflops_sustained x 4 (nominal FP4 : BF16 dense ratio)" if wl.dtype == "nvfp4"
-         else "bf16_tflops_sustained")})
+    roof = roofline(wl, alg_bytes, alg_flops, gemm_ms, peaks, peak_src)
+    roof.update({"kernel": expert_gemm_kernel(wl), "experts_used": used,
+                 "traffic_model": model_bytes, "step_ms": ms / K})
+    roof["traffic"] = traffic_record(wl.name)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -543,9 +569,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp32" if wl.dtype == "f32" else ("nvfp4+bf16" if wl.dtype == "nvfp4"
                                                                              else "bf16"),
-            "data": "synthetic", "config": {**workload_config(wl),
-                                            "l2": "no flush: weights alone exceed the 126 MB L2"
-                                            if wl.dtype != "f32" else "tiny (fits L2)"},
+            "data": "synthetic", "config": workload_config(wl),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() *
                                                                                      x_host.element_size()),

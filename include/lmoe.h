@@ -156,7 +156,11 @@ size_t lmoe_workspace_size(const lmoe_config* cfg, int op);
  * to a multiple of 128. Returns 0 for an invalid config. */
 int64_t lmoe_padded_rows(const lmoe_config* cfg);
 
-/* Router: logits = x W_r^T + b, then per token the K experts with the largest
+/* Router (greeksharifa page, section 2.2 "LatentMoE": the routing gate reads
+ * the d-dim hidden state, outside the latent compression; the Nemotron 3 Nano
+ * blog's architecture section: a learned router over the routed experts).
+ * The score function, tie rule and renormalisation are not on the pages; the
+ * reading taken: logits = x W_r^T + b, then per token the K experts with the largest
  * logits (ties to the lower index), in that order, and their gates
  * g_k = exp(l_k - l_max) / sum_j exp(l_j - l_max) over the chosen K (the
  * softmax over all N restricted to the K and renormalised).
@@ -174,7 +178,9 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
                        float* topk_w, float* logits_out, void* ws, size_t ws_bytes,
                        void* stream);
 
-/* Dispatch grouped by expert: a stable counting sort of the slots
+/* Dispatch grouped by expert (greeksharifa page, section 2.2 "LatentMoE": the
+ * routed experts run on the latent z, so the rows sent to each expert are
+ * l-dim; the pages give no dispatch layout). A stable counting sort of the slots
  * f = t*K + k by expert (expert ascending, then f ascending).
  *  topk_idx [T][K] int32 (each in [0, N); out-of-range -> device bounds error).
  *    A slot with an out-of-range expert is left out: offsets[N] counts only
@@ -217,6 +223,10 @@ lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_
  *    LMOE_ERR_WORKSPACE before anything is launched.
  *  - The first call on each device looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
+ *    The address is cached per device together with the id of the context it
+ *    was looked up in; a call in a new context (after cudaDeviceReset, for
+ *    instance) looks it up again, so make the first call after such a reset
+ *    before any stream capture too.
  *  - All calls share the one array: calls that overlap on the GPU (two
  *    streams, or two host threads) race and must be serialised by the caller.
  *  - There is no error word: an out-of-range expert index is skipped without
@@ -227,7 +237,10 @@ lmoe_status lmoe_permute_noalloc(const lmoe_config* cfg, const int32_t* topk_idx
                                  const uint8_t* rows_sf, uint8_t* permuted_sf, const float* topk_w,
                                  float* perm_gate, void* stream);
 
-/* Routed expert FFNs on the padded expert-grouped rows:
+/* Routed expert FFNs in the latent dimension (greeksharifa page, section 2.2
+ * "LatentMoE": every routed expert maps l -> m -> l; section 2.4 "NVFP4
+ * Training" for the NVFP4 operands; the activation is not on the pages and is
+ * read as squared ReLU), on the padded expert-grouped rows:
  *  y = g * (relu(z_e W1_e^T)^2 W2_e^T) for the rows of each expert e.
  *  permuted_in [padded][l]: `act` rows, or for expert == NVFP4 packed E2M1
  *    codes [padded][l/2] with permuted_sf (MMA_TILED) and in_global_scale
@@ -244,7 +257,9 @@ lmoe_status lmoe_expert_ffn(const lmoe_config* cfg, const lmoe_weights* w,
                             const int32_t* padded_offsets, const float* perm_gate,
                             void* y_perm, void* ws, size_t ws_bytes, void* stream);
 
-/* Combine: c_t = sum_{k=0..K-1} w[t][k] * y_perm[row(t*K+k)], summed in fp32
+/* Combine (greeksharifa page, section 2.2 "LatentMoE": the experts' outputs
+ * are summed in l and then projected back to d):
+ * c_t = sum_{k=0..K-1} w[t][k] * y_perm[row(t*K+k)], summed in fp32
  * in k order, stored as `act`; row(f) = inv_perm[f] - offsets[e] +
  * padded_offsets[e] with e = topk_idx[f]. topk_w NULL means the gates were
  * already applied (w = 1). c [T][l]. No workspace. A slot whose expert index
@@ -256,7 +271,9 @@ lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32
                          const int32_t* padded_offsets, const float* topk_w, void* c,
                          void* stream);
 
-/* The whole layer: route, down-project (NVFP4: quantise z with its current
+/* The whole layer (greeksharifa page, section 2.2 "LatentMoE"; notes.yuuk.io
+ * page, section 2 "LatentMoE"; the two always-on shared experts of the
+ * Nemotron 3 Nano blog's architecture section): route, down-project (NVFP4: quantise z with its current
  * amax), permute, expert FFNs, combine, up-project and add the shared
  * experts. x [T][d] (act) -> out [T][d] (act). N must be a multiple of 8
  * (the router GEMM stores logit rows in 16-byte vectors; LMOE_ERR_UNSUPPORTED
@@ -284,7 +301,10 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
                                 void* out, void* ws, size_t ws_bytes, void* stream,
                                 void* const* events);
 
-/* NVFP4 two-level quantisation of in [rows][cols] (F32 or BF16, cols a
+/* NVFP4 quantiser (greeksharifa page, section 2.4 "NVFP4 Training": E2M1
+ * elements, 16-element micro-blocks with an E4M3 scale and an FP32 per-tensor
+ * global scale; the scale formulas are not on the pages and are read as the
+ * standard two-level recipe below). Two-level quantisation of in [rows][cols] (F32 or BF16, cols a
  * multiple of 16) along its rows:
  *  s_g = global_in ? *global_in : fp32(amax / 2688) (1 when amax == 0);
  *  per 16-block: s_b = E4M3_satfinite_rn(amax_b / (s_g * 6));

@@ -16,22 +16,63 @@ namespace {
 constexpr int64_t kStaticScratchEntries = 128 * 1024;
 static __device__ __align__(256) int32_t g_permute_scratch[kStaticScratchEntries];
 
-// Device address of the array, looked up once per device (host code cannot
-// use the symbol itself as a device pointer).
+// Device address of the array. Host code cannot use the symbol itself as a
+// device pointer, so the address is looked up with cudaGetSymbolAddress, with
+// the device current, at the first call on that device. The cached address
+// belongs to the context it was looked up in: it is keyed on that context's
+// process-unique id (cuCtxGetId), so after cudaDeviceReset, or any teardown
+// and re-creation of the device's context, the next call looks it up again
+// instead of handing the kernel an address the library no longer owns.
 constexpr int kMaxDevices = 64;
-int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  int32_t* ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context (0 when none is current or the
+// driver entry points are missing).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 lmoe_status static_scratch(int32_t** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LMOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  ScratchEntry& e = g_scratch[dev];
+  unsigned long long ctx = current_context_id();
+  if (e.ptr == nullptr || ctx == 0 || e.ctx_id != ctx) {
+    // the lookup also makes the device's primary context current if no
+    // context was yet, so the id is read again after it
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return LMOE_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    e.ptr = static_cast<int32_t*>(p);
+    e.ctx_id = ctx ? ctx : current_context_id();   // 0 (no id available) never matches: look up every call
   }
-  *out = g_scratch_ptr[dev];
+  *out = e.ptr;
   return LMOE_OK;
 }
 

@@ -126,3 +126,15 @@ def bf16_parity(got: np.ndarray, ref_unrounded: np.ndarray, ref_rounded: np.ndar
     excess = np.maximum(0.0, np.abs(got - ref_unrounded) - bf16_ulp(ref_rounded) / 2).max() / rms
     raw = np.abs(got - ref_rounded).max() / rms
     return float(excess), float(raw)
+
+
+def bf16_raw_within(got: np.ndarray, ref_rounded: np.ndarray, tol: float):
+    """Raw bound, element by element: |got - RN_bf16(oracle)| <= tol * RMS + one
+    BF16 step of the element. A correct BF16 output can sit one step away
+    from the oracle's rounding (its own accumulation rounds on the other side
+    of a midpoint), so the step is allowed on top of the output tolerance.
+    Returns (all within, max over elements of |err| / bound)."""
+    rms = float(np.sqrt(np.mean(ref_rounded ** 2)))
+    bound = tol * rms + bf16_ulp(ref_rounded)
+    r = np.abs(got - ref_rounded) / bound
+    return bool(np.all(r <= 1.0)), float(r.max())

@@ -80,3 +80,48 @@ def test_cpu_baseline_sample_is_time_bounded():
     _, _, ntok1, calls1 = bench.oracle_sample(wl, inp, 16, min_seconds=1e9, max_calls=3)
     assert calls1 == 3 and ntok1 == 48              # and by the call cap
     assert set(bench.CPU_SAMPLE_TOKENS) == set(LI.WORKLOADS)
+
+
+def test_reference_arm_config_matches_our_arm():
+    """Both arms describe the workload with the same dict (the driver compares them)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import lmoe_inputs as LI
+    for name in LI.WORKLOADS:
+        c = bench.workload_config(LI.WORKLOADS[name])
+        assert c["workload"] == name and "l2" in c
+
+
+def test_expert_gemm_work_counts_weights_once_and_flops_by_definition():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import lmoe_inputs as LI
+    wl = LI.WORKLOADS["ultra_zipf"]
+    counts = np.zeros(wl.N, dtype=np.int64)
+    counts[:3] = [1000, 10, 1]                      # three experts used, 1011 rows
+    b, f, used, model = bench.expert_gemm_work(wl, counts)
+    assert used == 3
+    assert b == 3 * 2 * wl.m * wl.l * 2             # W1_e and W2_e of the used experts, BF16
+    assert f == 2.0 * 1011 * wl.l * wl.m * 2
+    assert model == 1011 * (wl.l + wl.m) * 2 * 2    # z in, a out, a in, y out: not algorithmic
+    wq = LI.WORKLOADS["ultra_nvfp4"]
+    bq, _, _, _ = bench.expert_gemm_work(wq, counts)
+    assert bq == 3 * 2 * wq.m * wq.l * (0.5 + 1 / 16)
+
+
+def test_roofline_uses_burst_peaks_and_the_binding_roof():
+    sys.path.insert(0, ROOT)
+    import bench
+    import lmoe_inputs as LI
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    wl = LI.WORKLOADS["ultra_zipf"]
+    r = bench.roofline(wl, 4e9, 3.2e12, 2.0, peaks, "measured")
+    assert r["bound"] == "tensor" and r["peak"] == 1600.0
+    assert r["achieved"] == pytest.approx(3.2e12 / 2e-3 / 1e12)
+    assert r["frac"] == pytest.approx(1600.0 / 1600.0)
+    assert r["frac_of_sustained"] == pytest.approx(1600.0 / 1400.0)
+    rq = bench.roofline(LI.WORKLOADS["ultra_nvfp4"], 1.2e9, 1.5e12, 0.5, peaks, "measured")
+    assert rq["bound"] == "tensor" and rq["peak"] == 6400.0          # 4 x BF16 burst
+    rd = bench.roofline(LI.WORKLOADS["ultra_decode"], 3e9, 6e9, 0.5, peaks, "fallback")
+    assert rd["bound"] == "hbm" and rd["frac"] == pytest.approx(3e9 / 0.5e-3 / 1e9 / 6000.0)
