@@ -18,7 +18,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "liblmoe.so")
+# LMOE_LIBRARY selects another build of the same library (for instance the
+# bounds-checking debug build, liblmoe_checks.so); the default is the release build.
+LIB_PATH = os.environ.get("LMOE_LIBRARY") or os.path.join(HERE, "liblmoe.so")
 
 # status codes
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_DEVICE_BOUNDS = range(7)

@@ -1,6 +1,12 @@
 """Build liblmoe.so (the C-ABI library) for sm_100a with nvcc, in-tree.
 
-Usage: python latentmoe_fwd_b200/build.py [--jobs N] [--verbose] [--force]
+Usage: python latentmoe_fwd_b200/build.py [--jobs N] [--verbose] [--force] [--checks]
+
+--checks builds the debug variant liblmoe_checks.so (compiled with
+-DLMOE_CHECKS: device bounds checks on the expert-grouped row ranges that
+come from caller-supplied offsets; a failed check records
+LMOE_ERR_DEVICE_BOUNDS and skips the rows). Load it by setting
+LMOE_LIBRARY to its path before importing the package.
 
 Run as a script (not ``-m``) so that the package, which loads the
 library on import, is not imported before the library exists.
@@ -18,6 +24,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "liblmoe.so")
+BUILD_CHECKS = os.path.join(HERE, "_build_checks")
+LIB_CHECKS = os.path.join(HERE, "liblmoe_checks.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -35,20 +43,24 @@ def _newest_input():
     return max(os.path.getmtime(f) for f in files)
 
 
-def up_to_date() -> bool:
-    return os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input()
+def up_to_date(lib: str = LIB) -> bool:
+    return os.path.exists(lib) and os.path.getmtime(lib) >= _newest_input()
 
 
-def build(jobs: int | None = None, verbose: bool = False, force: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(jobs: int | None = None, verbose: bool = False, force: bool = False, extra=(),
+          checks: bool = False) -> str:
+    lib_path, build_dir = (LIB_CHECKS, BUILD_CHECKS) if checks else (LIB, BUILD)
+    if checks:
+        extra = (*extra, "-DLMOE_CHECKS")
+    if not force and up_to_date(lib_path):
+        return lib_path
+    os.makedirs(build_dir, exist_ok=True)
     newest_hdr = max(os.path.getmtime(os.path.join(CSRC, f)) for f in os.listdir(CSRC)
                      if not f.endswith(".cu"))
     newest_hdr = max(newest_hdr, os.path.getmtime(os.path.join(ROOT, "include", "lmoe.h")))
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         if (not force and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(src)
                 and os.path.getmtime(obj) >= newest_hdr):
             return obj, ""
@@ -68,13 +80,13 @@ def build(jobs: int | None = None, verbose: bool = False, force: bool = False, e
             if log:
                 sys.stderr.write(log)
     objs = [o for o, _ in results]
-    tmp = LIB + ".tmp"
+    tmp = lib_path + ".tmp"
     cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
@@ -82,5 +94,6 @@ if __name__ == "__main__":
     ap.add_argument("--jobs", type=int, default=None)
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--checks", action="store_true", help="build the bounds-checking debug variant")
     a = ap.parse_args()
-    print(build(a.jobs, a.verbose, a.force))
+    print(build(a.jobs, a.verbose, a.force, checks=a.checks))

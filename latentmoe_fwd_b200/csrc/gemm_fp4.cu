@@ -64,6 +64,7 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   if (!make_map_fp4(&ma, L.a_codes, L.k, L.a_rows, 1, 128)) return LMOE_ERR_INVALID_ARG;
   if (!make_map_fp4(&mb, L.b_codes, L.k, L.cols, L.groups, 256)) return LMOE_ERR_INVALID_ARG;
   Fp4Params p;
+  p.rows = static_cast<int>(L.a_rows);
   p.cols = L.cols;
   p.kblocks = static_cast<int>(L.k / 256);
   p.sf_groups_a = static_cast<int>(L.k / 64);

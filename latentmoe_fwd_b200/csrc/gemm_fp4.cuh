@@ -28,6 +28,7 @@ namespace lmoe {
 enum Fp4Epi : int { FP4_EPI_SQRELU_QUANT = 0, FP4_EPI_GATE_BF16 = 1 };
 
 struct Fp4Params {
+  int rows;                   // padded rows of A (a multiple of 128)
   int cols;                   // output features per expert
   int kblocks;                // 256-element K blocks
   int sf_groups_a;            // K / 64: scale atoms per 128-row block of A
@@ -178,9 +179,23 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
   int* s_pstart = reinterpret_cast<int*>(smem + S::kRowsOffset);   // [groups + 1] padded starts
   int* s_rend = s_pstart + S::kMaxGroups + 1;                          // [groups] real ends
   for (int g = threadIdx.x; g <= p.groups; g += blockDim.x) {
-    const int ps = __ldg(p.padded_offsets + g);
+    int ps = __ldg(p.padded_offsets + g);
+    if (kChecks && (ps < 0 || ps > p.rows || (ps & 127))) {
+      dev_report(p.err, kErrBounds, 0x5300);
+      ps = p.rows;
+    }
     s_pstart[g] = ps;
-    if (g < p.groups) s_rend[g] = ps + __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+    if (g < p.groups) {
+      int n_e = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+      if (kChecks) {   // the expert's rows must fit its padded range
+        const int pe = __ldg(p.padded_offsets + g + 1);
+        if (n_e < 0 || pe < ps || pe > p.rows || ps + n_e > pe) {
+          dev_report(p.err, kErrBounds, 0x5301);
+          n_e = 0;
+        }
+      }
+      s_rend[g] = ps + n_e;
+    }
   }
   if (warp == 1) tmem_alloc(tmem_ptr, 512);
   tc_fence_before();

@@ -71,6 +71,7 @@ static lmoe_status dispatch_epi(int epi, const CUtensorMap* m, const TcParams& p
     case EPI_GATE: return launch_tc<BN, STAGES, EPI_GATE>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_PARTIAL: return launch_tc<BN, STAGES, EPI_PARTIAL>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_SCATTER: return launch_tc<BN, STAGES, EPI_SCATTER>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
   }
   return LMOE_ERR_INVALID_ARG;
 }
@@ -118,8 +119,12 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   p.ld_res = L.ld_res;
   p.ksplit = L.ksplit > 1 ? L.ksplit : 1;
   p.partial = L.partial;
+  p.scatter_rows = L.scatter_rows;
+  p.scatter_k = L.scatter_k;
   p.err = DevErr{err_word};
   if (p.ksplit > 1 && (L.grouped || !L.partial)) return LMOE_ERR_INVALID_ARG;
+  if (L.epi == EPI_SCATTER && (L.swap || L.ksplit > 1 || !L.scatter_rows || L.scatter_k <= 0))
+    return LMOE_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   const int64_t tiles = L.max_tiles * p.ksplit;
   int64_t grid = tiles < sms ? tiles : sms;

@@ -34,7 +34,9 @@ enum EpiKind : int {
   EPI_SQRELU = 2,     // out bf16 = relu(acc)^2
   EPI_GATE = 3,       // out bf16 = acc * row_scale[row]
   EPI_ADD_RES = 4,    // out bf16 = acc + residual[row][col]
-  EPI_PARTIAL = 5     // split-K: fp32 partial sums, the epilogue runs in the reduction
+  EPI_PARTIAL = 5,    // split-K: fp32 partial sums, the epilogue runs in the reduction
+  EPI_SCATTER = 6     // out bf16 = acc, row t stored at each padded row scatter_rows[t*K + k]
+                      // (k < scatter_k; negative entries skipped): token-major tiles only
 };
 
 struct TcSeg {
@@ -61,6 +63,8 @@ struct TcParams {
   long long ld_res;
   int ksplit;                 // >1: split the K blocks of every tile; partial sums go to `partial`
   float* partial;             // [ksplit][rows][cols] fp32 (split-K only)
+  const int* scatter_rows;    // EPI_SCATTER: [rows][scatter_k] destination rows of each row
+  int scatter_k;
   // CTA-pair grouped launches only: one dense problem computed in the same
   // launch, out_x[rows_x, cols_x] = epi(X[rows_x, K_x] . Wx[cols_x, K_x]^T)
   int rows_x;                 // 0: none
@@ -106,7 +110,14 @@ template <int BN>
 __device__ __forceinline__ void build_tile_prefix(const TcParams& p, int* prefix) {
   const int ntw = (p.cols + 127) / 128;
   for (int e = threadIdx.x; e < p.groups; e += blockDim.x) {
-    const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+    int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+    if (kChecks) {   // the expert's rows must fit its padded range inside the buffer
+      const int ps = __ldg(p.padded_offsets + e), pe = __ldg(p.padded_offsets + e + 1);
+      if (n_e < 0 || ps < 0 || pe > p.rows || ps + n_e > pe) {
+        dev_report(p.err, kErrBounds, 0x5100);
+        n_e = 0;
+      }
+    }
     prefix[e + 1] = ((n_e + BN - 1) / BN) * ntw;
   }
   if (threadIdx.x == 0) prefix[0] = 0;
@@ -397,6 +408,27 @@ __global__ void __launch_bounds__(192, 1)
                 if (col0 + j < p.cols)
                   *reinterpret_cast<float4*>(o + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
                                                                    __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            } else if (EPI == EPI_SCATTER) {
+              // the token's row goes to each of its K slots' padded rows (the
+              // expert-grouped GEMM input), streamed past L2
+              uint4 u[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                u[j].x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                u[j].y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                u[j].z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                u[j].w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+              }
+              const uint64_t pol = policy_evict_first();
+              const int* dst = p.scatter_rows + row * p.scatter_k;
+              for (int kk = 0; kk < p.scatter_k; ++kk) {
+                const int pr = __ldg(dst + kk);
+                if (pr < 0) continue;
+                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(pr) * p.ld_out + col0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  if (col0 + 8 * j < p.cols) st_global_v4_hint(o + 8 * j, u[j], pol);
+              }
             } else if (EPI == EPI_F32_BIAS) {
               float* o = reinterpret_cast<float*>(p.out) + row * p.ld_out + col0;
 #pragma unroll

@@ -198,7 +198,14 @@ __global__ void __launch_bounds__(192, 1)
   {
     const int ntw = (p.cols + 255) / 256;
     for (int e = threadIdx.x; e < p.groups; e += blockDim.x) {
-      const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+      int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+      if (kChecks) {   // the expert's rows must fit its padded range inside the buffer
+        const int ps = __ldg(p.padded_offsets + e), pe = __ldg(p.padded_offsets + e + 1);
+        if (n_e < 0 || ps < 0 || pe > p.rows || ps + n_e > pe) {
+          dev_report(p.err, kErrBounds, 0x5200);
+          n_e = 0;
+        }
+      }
       prefix[e + 1] = ((n_e + S::kTokens - 1) / S::kTokens) * ntw;
     }
     if (threadIdx.x == 0) prefix[0] = 0;

@@ -83,7 +83,7 @@ struct Layout {
   size_t splitk = 0;        // fp32 split-K partial sums of the weight-major dense GEMMs (T <= 64)
   size_t rsplit = 0;        // fp32 split-K partial sums of the token-major router GEMM (few tiles)
   size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0,
-         offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, scratch = 0, gate = 0, zp = 0,
+         offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, slot_row = 0, scratch = 0, gate = 0, zp = 0,
          zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, ys = 0, total = 0;
 };
 
@@ -132,6 +132,7 @@ Layout layout(const lmoe_config* c, int op) {
     L.poff = take((N + 1) * 4);
     L.perm_src = take(T * K * 4);
     L.inv_perm = take(T * K * 4);
+    L.slot_row = take(T * K * 4);
     L.scratch = take(static_cast<size_t>(permute_chunks(T * K) + 1) * N * 4);
     L.gate = take(P * 4);
     if (fp4) {
@@ -425,6 +426,7 @@ lmoe_status expert_ffn_impl(const lmoe_config* cfg, const lmoe_weights* w, const
   const int64_t single_tiles = static_cast<int64_t>(cfg->T) * cfg->K / sbn + cfg->N;
   TcLaunch g1;
   g1.grouped = 1;
+  g1.rows = static_cast<int>(P);   // padded rows (bounds of the debug build's checks)
   g1.cols = cfg->m;
   g1.kblocks[0] = kblocks(cfg->l);
   g1.offsets = offsets;
@@ -661,57 +663,83 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     return st;
   mark(1);
 
-  // 2. latent down-projection d -> l
-  const void* z = x;
-  if (!ident) {
-    void* zb = at<void>(ws, L.z);
-    if (f32) {
-      SimtLaunch S;
-      S.rows = static_cast<int>(T);
-      S.cols = l;
-      S.k = d;
-      S.a = static_cast<const float*>(x);
-      S.b = static_cast<const float*>(w->w_down);
-      S.out = static_cast<float*>(zb);
-      S.ld_out = l;
-      S.epi = EPI_BF16;
-      st = simt_gemm(S, err, s);
-    } else {
-      st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s);
-    }
-    if (st != LMOE_OK) return st;
-    z = zb;
-  }
-  uint8_t* zq_sf = nullptr;
-  float* z_gs = nullptr;
-  if (fp4) {
-    // NVFP4 latent activations: current per-tensor amax, row-major block scales
-    zq_sf = at<uint8_t>(ws, L.zq_sf);
-    z_gs = at<float>(ws, L.z_gs);
-    if ((st = launch_nvfp4_quantize(z, LMOE_BF16, T, l, nullptr, at<uint8_t>(ws, L.zq), zq_sf, z_gs,
-                                    LMOE_SF_ROWMAJOR, at<float>(ws, L.partials), nvfp4_partials(T * l), err, s)) !=
-        LMOE_OK)
-      return st;
-    z = at<void>(ws, L.zq);
-  }
-  mark(2);
-
-  // 3. dispatch grouped by expert (padded rows), gates per padded row
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* poff = at<int32_t>(ws, L.poff);
   int32_t* perm_src = at<int32_t>(ws, L.perm_src);
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   float* gate = at<float>(ws, L.gate);
   void* zp = at<void>(ws, L.zp);
-  if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
-                           err, s)) != LMOE_OK)
-    return st;
-  const int64_t row_bytes = fp4 ? l / 2 : static_cast<int64_t>(l) * ab;
-  uint8_t* zp_sf = fp4 ? at<uint8_t>(ws, L.zp_sf) : nullptr;
-  if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, zq_sf, zp_sf, N, s)) !=
-      LMOE_OK)
-    return st;
-  mark(3);
+  uint8_t* zq_sf = nullptr;
+  float* z_gs = nullptr;
+  // BF16 latent layer with token-major tiles: the permutation runs first and
+  // the down-projection's epilogue writes each token's z row straight to the
+  // padded rows of its K slots, so z is never stored and gathered
+  const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens;
+  if (scatter_z) {
+    int32_t* slot_row = at<int32_t>(ws, L.slot_row);
+    if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
+                             err, s, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
+      return st;
+    TcLaunch D;
+    D.rows = static_cast<int>(T);
+    D.cols = l;
+    D.kblocks[0] = kblocks(d);
+    D.bn = normal_bn(l);
+    D.a[0] = TcOperand{x, d, T, 1};
+    D.b[0] = TcOperand{w->w_down, d, l, 1};
+    D.max_tiles = ((T + 127) / 128) * ((l + D.bn - 1) / D.bn);
+    D.out = zp;
+    D.ld_out = l;
+    D.epi = EPI_SCATTER;
+    D.scatter_rows = slot_row;
+    D.scatter_k = K;
+    if ((st = tc_gemm(D, err, s)) != LMOE_OK) return st;
+    mark(3);
+  } else {
+    // 2. latent down-projection d -> l
+    const void* z = x;
+    if (!ident) {
+      void* zb = at<void>(ws, L.z);
+      if (f32) {
+        SimtLaunch S;
+        S.rows = static_cast<int>(T);
+        S.cols = l;
+        S.k = d;
+        S.a = static_cast<const float*>(x);
+        S.b = static_cast<const float*>(w->w_down);
+        S.out = static_cast<float*>(zb);
+        S.ld_out = l;
+        S.epi = EPI_BF16;
+        st = simt_gemm(S, err, s);
+      } else {
+        st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s);
+      }
+      if (st != LMOE_OK) return st;
+      z = zb;
+    }
+    if (fp4) {
+      // NVFP4 latent activations: current per-tensor amax, row-major block scales
+      zq_sf = at<uint8_t>(ws, L.zq_sf);
+      z_gs = at<float>(ws, L.z_gs);
+      if ((st = launch_nvfp4_quantize(z, LMOE_BF16, T, l, nullptr, at<uint8_t>(ws, L.zq), zq_sf, z_gs,
+                                      LMOE_SF_ROWMAJOR, at<float>(ws, L.partials), nvfp4_partials(T * l), err, s)) !=
+          LMOE_OK)
+        return st;
+      z = at<void>(ws, L.zq);
+    }
+    mark(2);
+
+    // 3. dispatch grouped by expert (padded rows), gates per padded row
+    if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
+                             err, s)) != LMOE_OK)
+      return st;
+    const int64_t row_bytes = fp4 ? l / 2 : static_cast<int64_t>(l) * ab;
+    uint8_t* zp_sf = fp4 ? at<uint8_t>(ws, L.zp_sf) : nullptr;
+    if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, zq_sf, zp_sf, N, s)) !=
+        LMOE_OK)
+      return st;
+    mark(3);
+  }
 
   // 4. routed expert FFNs in l, gate applied in the second GEMM's epilogue; the
   // shared experts' hidden layer (BF16) is offered to the first GEMM's launch
@@ -732,8 +760,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   void* y = at<void>(ws, L.y);
   const std::function<void()> between = events ? std::function<void()>([&]() { mark(4); }) : std::function<void()>();
   if (fp4)
-    st = expert_ffn_fp4(cfg, w, zp, zp_sf, z_gs, offsets, poff, gate, at<void>(ws, L.a), at<uint8_t>(ws, L.a_sf), y,
-                        err, s, between);
+    st = expert_ffn_fp4(cfg, w, zp, at<uint8_t>(ws, L.zp_sf), z_gs, offsets, poff, gate, at<void>(ws, L.a),
+                        at<uint8_t>(ws, L.a_sf), y, err, s, between);
   else
     st = expert_ffn_impl(cfg, w, zp, offsets, poff, gate, at<void>(ws, L.a), y, err, s, between,
                          shared_hidden.cols > 0 ? &shared_hidden : nullptr);

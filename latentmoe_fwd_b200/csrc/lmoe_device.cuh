@@ -30,6 +30,18 @@ __device__ __forceinline__ void dev_report(DevErr e, uint32_t status, uint32_t i
 constexpr uint32_t kErrTimeout = 5;
 constexpr uint32_t kErrBounds = 6;
 
+// Debug build with device bounds checks (compiled with -DLMOE_CHECKS): the
+// expert-grouped row ranges the GEMMs and the combine derive from offsets a
+// caller may pass in are range-checked before use; a failed check records
+// LMOE_ERR_DEVICE_BOUNDS (info = the place) where the kernel has an error
+// word, and the rows it names are skipped. The release build trusts those
+// offsets, as the header documents.
+#ifdef LMOE_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+
 // Wall-clock bound of every pipeline wait (about 2 s at 1.9 GHz).
 constexpr long long kWaitLimitCycles = 4000000000LL;
 

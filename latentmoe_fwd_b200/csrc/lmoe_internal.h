@@ -78,6 +78,8 @@ struct TcLaunch {
   int bn = 256;
   int ksplit = 1;                // >1: split-K with fp32 partials in `partial`, then a reduction
   float* partial = nullptr;      // [ksplit][rows][cols]
+  const int* scatter_rows = nullptr;   // EPI_SCATTER (token-major only): [rows][scatter_k] destination rows
+  int scatter_k = 0;
   // tc2_gemm only: a dense problem in the same launch, out_x = epi(x_act . x_wt^T)
   TcOperand x_act = {};          // [rows_x][k] activations
   TcOperand x_wt = {};           // [cols_x][k] weights, or [groups][cols_x][x_kgroup] with K split in groups
@@ -150,10 +152,13 @@ lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* i
 constexpr int kPermSlotsPerWarp = 128;
 constexpr int kPermSlotsPerWarpStatic = 1024;
 int permute_chunks(int64_t slots, int slots_per_warp = kPermSlotsPerWarp);
+// scratch: (permute_chunks() + 1) * N int32. slot_row (optional, [T*K]): the
+// padded row of each slot (-1 for a slot left out).
 lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
                            int32_t* scratch, const float* topk_w, float* perm_gate,
-                           uint32_t* err, cudaStream_t s, int slots_per_warp = kPermSlotsPerWarp);
+                           uint32_t* err, cudaStream_t s, int slots_per_warp = kPermSlotsPerWarp,
+                           int32_t* slot_row = nullptr);
 lmoe_status launch_gather(const int32_t* idx, const int32_t* perm_src, const int32_t* offsets,
                           const int32_t* padded_offsets, int64_t slots, int K, const void* rows,
                           int64_t row_bytes, void* out_rows, const uint8_t* rows_sf,

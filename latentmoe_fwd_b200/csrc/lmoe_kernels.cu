@@ -339,17 +339,22 @@ lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* i
 
 // ===========================================================================
 // Permutation: stable counting sort of slots f = t*K + k by expert.
-//   pass 1 (count):  per chunk of kChunk slots, a shared-memory histogram.
-//   pass 2 (scan):   one CTA: per-expert prefix over chunks, then the
-//                    exclusive scan over experts -> offsets and padded offsets
-//                    (each expert's padded range is a multiple of 128 rows).
-//   pass 3 (scatter): every warp walks 32-slot steps of its part of the chunk
-//                    in order; __match_any_sync gives the rank among equal
-//                    experts inside a step, running per-warp counters keep
-//                    the order across steps, so the sort is stable.
+//   pass 1 (count):  per chunk of slots, a shared-memory histogram, stored
+//                    expert-major: cnt[e * nchunks + chunk].
+//   pass 2 (scan):   a warp per expert turns its row of chunk counts into
+//                    exclusive prefixes (coalesced, 32 chunks per step) and
+//                    stores the expert's total at cnt[N * nchunks + e].
+//   pass 3 (scatter): every CTA first scans the N totals in shared memory
+//                    (offsets, and padded offsets with each expert's range a
+//                    multiple of 128 rows; CTA 0 stores both), then its warps
+//                    walk 32-slot steps of their part of the chunk in order;
+//                    __match_any_sync gives the rank among equal experts
+//                    inside a step, running per-warp counters keep the order
+//                    across steps, so the sort is stable.
 // ===========================================================================
 constexpr int kPermWarps = 8;
 constexpr int kPad = 128;
+constexpr int kScanWarps = 32;
 
 // A chunk is kPermWarps * slots_per_warp consecutive slots, one CTA each.
 int permute_chunks(int64_t slots, int slots_per_warp) {
@@ -358,7 +363,7 @@ int permute_chunks(int64_t slots, int slots_per_warp) {
 }
 
 __global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restrict__ idx,
-                                                         int64_t slots, int N, int spw,
+                                                         int64_t slots, int N, int spw, int nch,
                                                          int32_t* __restrict__ cnt, DevErr err) {
   pdl_begin();
   extern __shared__ int32_t hist[];
@@ -376,11 +381,34 @@ __global__ void __launch_bounds__(256) perm_count_kernel(const int32_t* __restri
     atomicAdd(&hist[e], 1);   // shared-memory counter; global buffers are written once below
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[static_cast<int64_t>(blockIdx.x) * N + e] = hist[e];
+  for (int e = threadIdx.x; e < N; e += blockDim.x) cnt[static_cast<int64_t>(e) * nch + blockIdx.x] = hist[e];
 }
 
-// Block-wide exclusive scan of one value per thread (blockDim.x == 1024).
-__device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* total) {
+// Warp per expert: exclusive prefix of its chunk counts, total at the end.
+__global__ void __launch_bounds__(kScanWarps * 32) perm_scan_kernel(int32_t* __restrict__ cnt, int nch, int N) {
+  pdl_begin();
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * kScanWarps + (threadIdx.x >> 5);
+  if (e >= N) return;
+  int32_t* row = cnt + static_cast<int64_t>(e) * nch;
+  int carry = 0;
+  for (int c0 = 0; c0 < nch; c0 += 32) {
+    const int c = c0 + lane;
+    const int v = c < nch ? row[c] : 0;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (c < nch) row[c] = carry + x - v;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) cnt[static_cast<int64_t>(N) * nch + e] = carry;
+}
+
+// Exclusive scan of v over a 256-thread block; *total gets the block's sum.
+__device__ __forceinline__ int block256_exclusive_scan(int v, int* smem_warp, int* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -390,72 +418,65 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* 
   }
   if (lane == 31) smem_warp[wid] = x;
   __syncthreads();
-  if (wid == 0) {
-    int s = smem_warp[lane];
+  int base = 0, all = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, off);
-      if (lane >= off) s += y;
-    }
-    smem_warp[lane] = s;   // inclusive over warps
+  for (int w2 = 0; w2 < 8; ++w2) {
+    const int sw = smem_warp[w2];
+    if (w2 < wid) base += sw;
+    all += sw;
   }
   __syncthreads();
-  const int base = wid > 0 ? smem_warp[wid - 1] : 0;
-  if (total) *total = smem_warp[31];
-  const int r = base + x - v;
-  __syncthreads();
-  return r;
-}
-
-__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ cnt, int nchunks, int N,
-                                                         int32_t* __restrict__ offsets,
-                                                         int32_t* __restrict__ poff) {
-  pdl_begin();
-  __shared__ int warp_sums[32];
-  const int e = threadIdx.x;
-  int run = 0;
-  if (e < N) {
-    int c = 0;
-    for (; c + 4 <= nchunks; c += 4) {
-      const int v0 = cnt[static_cast<int64_t>(c) * N + e];
-      const int v1 = cnt[static_cast<int64_t>(c + 1) * N + e];
-      const int v2 = cnt[static_cast<int64_t>(c + 2) * N + e];
-      const int v3 = cnt[static_cast<int64_t>(c + 3) * N + e];
-      cnt[static_cast<int64_t>(c) * N + e] = run;
-      cnt[static_cast<int64_t>(c + 1) * N + e] = run + v0;
-      cnt[static_cast<int64_t>(c + 2) * N + e] = run + v0 + v1;
-      cnt[static_cast<int64_t>(c + 3) * N + e] = run + v0 + v1 + v2;
-      run += v0 + v1 + v2 + v3;
-    }
-    for (; c < nchunks; ++c) {
-      const int v0 = cnt[static_cast<int64_t>(c) * N + e];
-      cnt[static_cast<int64_t>(c) * N + e] = run;
-      run += v0;
-    }
-  }
-  int total = 0;
-  const int off = block_exclusive_scan(e < N ? run : 0, warp_sums, &total);
-  const int padded = e < N ? ((run + kPad - 1) / kPad) * kPad : 0;
-  int ptotal = 0;
-  const int poffv = block_exclusive_scan(padded, warp_sums, &ptotal);
-  if (e < N) {
-    offsets[e] = off;
-    poff[e] = poffv;
-  }
-  if (e == 0) {
-    offsets[N] = total;
-    poff[N] = ptotal;
-  }
+  *total = all;
+  return base + x - v;
 }
 
 __global__ void __launch_bounds__(256) perm_scatter_kernel(
-    const int32_t* __restrict__ idx, int64_t slots, int N, int spw, const int32_t* __restrict__ base,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff,
+    const int32_t* __restrict__ idx, int64_t slots, int N, int spw, int nch, const int32_t* __restrict__ cnt,
+    int32_t* __restrict__ offsets_out, int32_t* __restrict__ poff_out,
     int32_t* __restrict__ perm_src, int32_t* __restrict__ inv_perm,
-    const float* __restrict__ topk_w, float* __restrict__ perm_gate) {
+    const float* __restrict__ topk_w, float* __restrict__ perm_gate, int32_t* __restrict__ slot_row) {
   pdl_begin();
-  extern __shared__ int32_t wcnt[];   // [kPermWarps][N]
+  extern __shared__ int32_t sm[];
+  int32_t* wcnt = sm;                          // [kPermWarps][N]
+  int32_t* s_off = sm + kPermWarps * N;        // [N]
+  int32_t* s_poff = s_off + N;                 // [N]
+  __shared__ int warp_sums[8];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  // offsets and padded offsets of all experts from their totals: each thread
+  // owns four consecutive experts (N <= 1024)
+  {
+    const int32_t* tot = cnt + static_cast<int64_t>(N) * nch;
+    int v[4], pv[4], sum = 0, psum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = threadIdx.x * 4 + i;
+      v[i] = e < N ? __ldg(tot + e) : 0;
+      pv[i] = ((v[i] + kPad - 1) / kPad) * kPad;
+      sum += v[i];
+      psum += pv[i];
+    }
+    int total = 0, ptotal = 0;
+    int run = block256_exclusive_scan(sum, warp_sums, &total);
+    int prun = block256_exclusive_scan(psum, warp_sums, &ptotal);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = threadIdx.x * 4 + i;
+      if (e < N) {
+        s_off[e] = run;
+        s_poff[e] = prun;
+        if (blockIdx.x == 0) {
+          offsets_out[e] = run;
+          poff_out[e] = prun;
+        }
+      }
+      run += v[i];
+      prun += pv[i];
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      offsets_out[N] = total;
+      poff_out[N] = ptotal;
+    }
+  }
   for (int i = threadIdx.x; i < kPermWarps * N; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
   const int64_t f0 = (static_cast<int64_t>(blockIdx.x) * kPermWarps + wid) * spw;
@@ -484,7 +505,6 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     }
   }
   __syncthreads();
-  const int32_t* cbase = base + static_cast<int64_t>(blockIdx.x) * N;
   for (int64_t s = f0; s < f1; s += 32) {
     const int64_t f = s + lane;
     const bool live = f < f1;
@@ -494,17 +514,18 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     const unsigned peers = __match_any_sync(0xffffffffu, e) & act;
     int r = 0;
     if (live && e >= 0) {
-      r = __ldg(offsets + e) + __ldg(cbase + e) + my[e] + __popc(peers & lt);
+      r = s_off[e] + __ldg(cnt + static_cast<int64_t>(e) * nch + blockIdx.x) + my[e] + __popc(peers & lt);
     }
     __syncwarp();
     if (live && e >= 0) {
       if ((peers & lt) == 0) my[e] += __popc(peers);
       perm_src[r] = static_cast<int32_t>(f);
       inv_perm[f] = r;
-      if (perm_gate) {
-        const int p = r - __ldg(offsets + e) + __ldg(poff + e);
-        perm_gate[p] = __ldg(topk_w + f);
-      }
+      const int p = r - s_off[e] + s_poff[e];
+      if (perm_gate) perm_gate[p] = __ldg(topk_w + f);
+      if (slot_row) slot_row[f] = p;
+    } else if (live && slot_row) {
+      slot_row[f] = -1;   // a slot left out (expert index out of range)
     }
     __syncwarp();
   }
@@ -513,26 +534,25 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
 lmoe_status launch_permute(const int32_t* idx, int64_t T, int K, int N, int32_t* offsets,
                            int32_t* perm_src, int32_t* inv_perm, int32_t* padded_offsets,
                            int32_t* scratch, const float* topk_w, float* perm_gate,
-                           uint32_t* err, cudaStream_t s, int slots_per_warp) {
+                           uint32_t* err, cudaStream_t s, int slots_per_warp, int32_t* slot_row) {
   if (N > 1024) return LMOE_ERR_UNSUPPORTED;
   if (slots_per_warp <= 0 || slots_per_warp % 32) return LMOE_ERR_INVALID_ARG;
   const int64_t slots = T * K;
   const int nch = permute_chunks(slots, slots_per_warp);
   DevErr de{err};
   if (nch > 0) {
-    launch_k(perm_count_kernel, dim3(nch), dim3(256), N * sizeof(int32_t), s, idx, slots, N, slots_per_warp, scratch,
-             de);
+    launch_k(perm_count_kernel, dim3(nch), dim3(256), N * sizeof(int32_t), s, idx, slots, N, slots_per_warp, nch,
+             scratch, de);
     count_launch();
   }
-  launch_k(perm_scan_kernel, dim3(1), dim3(1024), 0, s, scratch, nch, N, offsets, padded_offsets);
+  launch_k(perm_scan_kernel, dim3((N + kScanWarps - 1) / kScanWarps), dim3(kScanWarps * 32), 0, s, scratch, nch, N);
   count_launch();
-  if (nch > 0) {
-    const size_t sm = static_cast<size_t>(kPermWarps) * N * sizeof(int32_t);
-    launch_k(perm_scatter_kernel, dim3(nch), dim3(256), sm, s, idx, slots, N, slots_per_warp,
-             static_cast<const int32_t*>(scratch), static_cast<const int32_t*>(offsets),
-             static_cast<const int32_t*>(padded_offsets), perm_src, inv_perm, topk_w, perm_gate);
-    count_launch();
-  }
+  // at least one CTA: it also stores the offsets (all zero without slots)
+  const size_t sm = (static_cast<size_t>(kPermWarps) + 2) * N * sizeof(int32_t);
+  launch_k(perm_scatter_kernel, dim3(nch > 0 ? nch : 1), dim3(256), sm, s, idx, slots, N, slots_per_warp, nch,
+           static_cast<const int32_t*>(scratch), offsets, padded_offsets, perm_src, inv_perm, topk_w, perm_gate,
+           slot_row);
+  count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
@@ -633,6 +653,8 @@ __global__ void __launch_bounds__(256) combine_kernel(
       if (ok) {
         row = static_cast<int64_t>(__ldg(inv_perm + f)) - __ldg(offsets + e) + __ldg(poff + e);
         g = w ? __ldg(w + f) : 1.0f;
+        // debug build: a row outside the padded rows (caller-supplied offsets) is skipped
+        if (kChecks && (row < 0 || row >= __ldg(poff + N))) ok = false;
       }
     }
     const unsigned m = __ballot_sync(0xffffffffu, ok);
