@@ -31,6 +31,13 @@ and thread count do not change any value):
 * NVFP4 workloads also carry ``a_global_scale``: the static per-layer FP32
   scale of the FFN hidden activation a = relu(h)^2, as an inference checkpoint
   carries it. Its synthetic value covers |h| <= 16 (a <= 256): 256 / (6 * 448).
+* Workloads with FP8 shared experts carry two static per-layer FP32 scales
+  the same way: ``shared_x_scale`` = 256 / 448 for the shared experts' input x
+  (covers |x| <= 256, the outliers included) and ``shared_h_scale`` = 512 / 448
+  for their hidden layer (covers values up to 512).
+* ``ultra_nvfp4_fp8shared`` T=8192, the NVFP4 layer with two always-on shared
+  experts of width 1024 in FP8 (the Ultra checkpoint recipe: NVFP4 routed,
+  FP8 shared experts)
 """
 from __future__ import annotations
 
@@ -59,6 +66,7 @@ class Workload:
     zipf_bias: bool = False
     outliers: bool = False
     w_block2d: bool = False      # nvfp4: expert weights scaled in 16 x 16 blocks
+    shared_fp8: bool = False     # shared experts in FP8 (E4M3, per-tensor scales)
     seed: int = 0
 
     def as_dict(self):
@@ -77,6 +85,9 @@ WORKLOADS = {
                             dtype="nvfp4", outliers=True),
     "ultra_decode_nvfp4": Workload("ultra_decode_nvfp4", T=32, d=8192, l=2048, N=512, K=22, m=1024,
                                    dtype="nvfp4", outliers=True),
+    "ultra_nvfp4_fp8shared": Workload("ultra_nvfp4_fp8shared", T=8192, d=8192, l=2048, N=512, K=22, m=1024,
+                                      n_shared=2, m_shared=1024, dtype="nvfp4", outliers=True,
+                                      shared_fp8=True),
 }
 
 
@@ -172,4 +183,10 @@ def make_inputs(wl: Workload, threads: int | None = None) -> dict:
     inp["a_global_scale"] = (256.0 / (6.0 * 448.0)) if wl.dtype == "nvfp4" else None
     if inp["a_global_scale"] is not None:
         inp["a_global_scale"] = float(np.float32(inp["a_global_scale"]))
+    if wl.shared_fp8:
+        inp["shared_x_scale"] = float(np.float32(256.0 / 448.0))
+        inp["shared_h_scale"] = float(np.float32(512.0 / 448.0))
+    else:
+        inp["shared_x_scale"] = None
+        inp["shared_h_scale"] = None
     return inp

@@ -262,6 +262,63 @@ def nvfp4_fake_quant(X, s_g: float | None = None):
 # ----------------------------------------------------------------------------
 
 
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) with per-tensor FP32 scales: the shared experts of the Ultra
+# checkpoint recipe (chathome page on Nemotron 3 Ultra, quantisation
+# paragraph: NVFP4 routed experts next to FP8 shared experts; jiwasawa blog on
+# Nemotron 3 Nano, FP8 section: post-training quantisation of weights and
+# activations to FP8). The pages give the format only; the reading taken:
+# one FP32 scale per weight tensor, amax / 448, and static per-layer FP32
+# scales for the two activations (the shared experts' input x and their
+# hidden layer), as an inference checkpoint carries them.
+# ----------------------------------------------------------------------------
+
+def fp8_scale(X) -> float:
+    """Per-tensor FP32 scale of a weight tensor: fp32(amax / 448); 1 when amax is 0."""
+    amax = float(np.max(np.abs(X))) if np.size(X) else 0.0
+    if amax == 0.0:
+        return 1.0
+    return float(round_f32(amax / E4M3_MAX))
+
+
+def fp8_quantize(X, s: float) -> np.ndarray:
+    """E4M3 codes of X / s: E4M3_rn_satfinite(fp32(x / s)), s an fp32 value.
+    The division is an fp32 operation, emulated exactly (fp64 then fp32)."""
+    return e4m3_encode(round_f32(np.asarray(X, dtype=np.float64) / s))
+
+
+def fp8_dequantize(codes, s: float) -> np.ndarray:
+    """x_hat = e4m3(q) * s, exact in fp64."""
+    return e4m3_decode(codes) * s
+
+
+def fp8_fake_quant(X, s: float) -> np.ndarray:
+    return fp8_dequantize(fp8_quantize(X, s), s)
+
+
+def shared_experts_fp8(x, ws1, ws2, s_x: float, s_h: float):
+    """Sum over the S shared experts of hs_s Ws2_s^T with FP8 operands.
+
+    x [T, d]; ws1 [S, m_s, d] and ws2 [S, d, m_s] (fp64 values of the stored
+    BF16 weights). Each weight tensor (all S experts' Ws1 as one tensor, all
+    their Ws2 as another) is quantised with its own amax scale; x with the
+    static scale s_x; the hidden layer hs = relu(x_hat Ws1_hat^T)^2 is stored
+    as FP8 with the static scale s_h (its rounding point). Returns (sum
+    [T, d], hs codes [T, S*m_s], (s_w1, s_w2))."""
+    S, ms, d = ws1.shape
+    w1 = ws1.reshape(S * ms, d)
+    s_w1, s_w2 = fp8_scale(w1), fp8_scale(ws2)
+    xq = fp8_fake_quant(x, s_x)
+    w1q = fp8_fake_quant(w1, s_w1)
+    w2q = fp8_fake_quant(ws2, s_w2)
+    h_codes = fp8_quantize(sq_relu(xq @ w1q.T), s_h)
+    hs = fp8_dequantize(h_codes, s_h)
+    out = np.zeros((x.shape[0], d))
+    for s in range(S):
+        out += hs[:, s * ms:(s + 1) * ms] @ w2q[s].T
+    return out, h_codes, (s_w1, s_w2)
+
+
 def router_logits(x, w_router, bias=None) -> np.ndarray:
     """logits[t, e] = x_t . W_r[e] (+ b[e]); the gate reads the d-dim x."""
     logits = np.asarray(x, dtype=np.float64) @ np.asarray(w_router, dtype=np.float64).T
@@ -460,7 +517,11 @@ def forward(wl, inp, tokens=None, idx_override=None, precision: str | None = Non
         out = c.copy()
     else:
         out = c @ W.dense("w_up").T
-    if wl.n_shared:
+    if wl.n_shared and getattr(wl, "shared_fp8", False) and prec != "f64":
+        ys, _, _ = shared_experts_fp8(x, to_f64(inp["ws1"], st), to_f64(inp["ws2"], st),
+                                      inp["shared_x_scale"], inp["shared_h_scale"])
+        out = out + ys
+    elif wl.n_shared:
         for s in range(wl.n_shared):
             ws1 = to_f64(inp["ws1"][s], st)
             ws2 = to_f64(inp["ws2"][s], st)
