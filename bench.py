@@ -303,7 +303,7 @@ def oracle_tokens_per_s(wl, inp, n_tokens: int, seed: int = 0):
 # tokens per oracle call of the CPU baseline (the NVFP4 oracle quantises every
 # expert matrix the sample touches, so its calls stay small)
 CPU_SAMPLE_TOKENS = {"tiny_f32": 64, "std_moe_bf16": 128, "ultra_decode": 32, "ultra_zipf": 32,
-                     "ultra_nvfp4": 4, "ultra_decode_nvfp4": 4}
+                     "ultra_nvfp4": 4, "ultra_decode_nvfp4": 4, "ultra_nvfp4_fp8shared": 4}
 
 
 def oracle_sample(wl, inp, n_tokens: int, min_seconds: float = 10.0, max_calls: int = 10000):
