@@ -431,7 +431,8 @@ def main():
     out_host = torch.empty((wl.T, wl.d), dtype=tdtype).pin_memory()
     cfg = L.config(T=wl.T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m, n_shared=wl.n_shared, m_shared=wl.m_shared,
                    act=L.F32 if st == "f32" else L.BF16,
-                   expert={"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype], identity=wl.identity)
+                   expert={"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype], identity=wl.identity,
+                   shared_fp8=wl.shared_fp8)
     extra = {}
     quant = None
     if wl.dtype == "nvfp4":
@@ -444,6 +445,20 @@ def main():
             extra[key + "_sf"], extra[key + "_gs"] = sf, gs
         torch.cuda.empty_cache()
         extra["a_global_scale"] = torch.tensor([inp["a_global_scale"]], dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+    if wl.shared_fp8:
+        # setup, not timed: FP8 shared-expert weights, one scale per stacked tensor
+        S, ms, d = wl.n_shared, wl.m_shared, wl.d
+        q = {}
+        for key, rows, cols in (("ws1", S * ms, d), ("ws2", S * d, ms)):
+            codes = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+            scale = torch.empty(1, dtype=torch.float32, device="cuda")
+            qws = L.workspace(L.config(T=rows, d=cols, l=cols, N=1, K=1, m=cols), L.OP_FP8_QUANTIZE)
+            L.fp8_quantize(t[key].reshape(rows, cols), L.BF16, rows, cols, None, codes, scale, qws)
+            q[key], extra[key + "_scale"] = codes, scale
+        t["ws1"], t["ws2"] = q["ws1"], q["ws2"]
+        extra["shared_x_scale"] = torch.tensor([inp["shared_x_scale"]], dtype=torch.float32, device="cuda")
+        extra["shared_h_scale"] = torch.tensor([inp["shared_h_scale"]], dtype=torch.float32, device="cuda")
         torch.cuda.synchronize()
     w = L.weights(w_router=t["w_router"], router_bias=bias, w_down=t["w_down"], w_up=t["w_up"], w1=t["w1"],
                   w2=t["w2"], ws1=t["ws1"], ws2=t["ws2"], **extra)
@@ -567,8 +582,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp32" if wl.dtype == "f32" else ("nvfp4+bf16" if wl.dtype == "nvfp4"
-                                                                             else "bf16"),
+            "vs_baseline": None, "dtype": "fp32" if wl.dtype == "f32" else (
+                ("nvfp4+fp8+bf16" if wl.shared_fp8 else "nvfp4+bf16") if wl.dtype == "nvfp4" else "bf16"),
             "data": "synthetic", "config": workload_config(wl),
             "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(x_host.numel() *

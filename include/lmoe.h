@@ -81,6 +81,17 @@ typedef enum { LMOE_SF_ROWMAJOR = 0, LMOE_SF_MMA_TILED = 1 } lmoe_sf_layout;
 /* Flag: l == d and there is no down/up projection (the standard-MoE limit). */
 #define LMOE_FLAG_IDENTITY_PROJ 1u
 
+/* Flag: the shared experts run in FP8 (E4M3), as in the Ultra checkpoint
+ * recipe (chathome page on Nemotron 3 Ultra, quantisation paragraph: NVFP4
+ * routed experts with FP8 shared experts). ws1 / ws2 then hold E4M3 codes
+ * (lmoe_fp8_quantize of each weight tensor, one scale per tensor: all S
+ * experts' Ws1 as one [S*m_s][d] tensor, all their Ws2 as one [S*d][m_s]
+ * tensor) with their scales in ws1_scale / ws2_scale; x is quantised with the
+ * static scale shared_x_scale, the hidden layer relu(x Ws1^T)^2 is stored as
+ * E4M3 with the static scale shared_h_scale, and the output layer's sum (in
+ * BF16) is added to the layer output. Needs act BF16 and n_shared > 0. */
+#define LMOE_FLAG_SHARED_FP8 2u
+
 /* Supported configurations (every entry point that takes a config checks
  * them before launching anything):
  *  LMOE_ERR_INVALID_ARG: T < 0 or T > 2^25; d, l, N, K or m not positive;
@@ -89,6 +100,8 @@ typedef enum { LMOE_SF_ROWMAJOR = 0, LMOE_SF_MMA_TILED = 1 } lmoe_sf_layout;
  *  LMOE_ERR_UNSUPPORTED: K > 32 or N > 1024; act F32 with expert other than
  *    F32; act BF16 with expert F32; act BF16 with shared experts and m_shared
  *    not a multiple of 64; expert NVFP4 with l or m not a multiple of 256;
+ *    LMOE_FLAG_SHARED_FP8 with act F32, d not a multiple of 16 or m_shared
+ *    not a multiple of 128 (LMOE_ERR_INVALID_ARG without shared experts);
  *    N not a multiple of 8 where the logits are computed (lmoe_forward,
  *    lmoe_route without logits_in). */
 
@@ -119,7 +132,11 @@ typedef struct {
  *    w1_gs / w2_gs [N] F32 the per-matrix global scales;
  *  a_global_scale: NVFP4 only, device pointer to one F32: the static scale of
  *    the expert hidden activation a, as a checkpoint carries it;
- *  ws1 [S][m_s][d], ws2 [S][d][m_s]: shared experts (NULL when n_shared == 0). */
+ *  ws1 [S][m_s][d], ws2 [S][d][m_s]: shared experts (NULL when n_shared == 0);
+ *    E4M3 codes (1 byte each) with LMOE_FLAG_SHARED_FP8;
+ *  ws1_scale, ws2_scale, shared_x_scale, shared_h_scale: LMOE_FLAG_SHARED_FP8
+ *    only, device pointers to one F32 each (the two weight tensors' scales and
+ *    the static scales of the shared experts' input and hidden layer). */
 typedef struct {
   const void* w_router;
   const float* router_bias;
@@ -134,6 +151,10 @@ typedef struct {
   const float* a_global_scale;
   const void* ws1;
   const void* ws2;
+  const float* ws1_scale;
+  const float* ws2_scale;
+  const float* shared_x_scale;
+  const float* shared_h_scale;
 } lmoe_weights;
 
 /* Workspace size queries, one per entry point. */
@@ -143,11 +164,12 @@ typedef enum {
   LMOE_OP_EXPERT_FFN = 2,
   LMOE_OP_COMBINE = 3,
   LMOE_OP_FORWARD = 4,
-  LMOE_OP_NVFP4_QUANTIZE = 5
+  LMOE_OP_NVFP4_QUANTIZE = 5,
+  LMOE_OP_FP8_QUANTIZE = 6
 } lmoe_op;
 
-/* Bytes of workspace `op` needs for `cfg` (for LMOE_OP_NVFP4_QUANTIZE the
- * tensor is taken as [cfg->T][cfg->l]). Returns 0 for an invalid config or
+/* Bytes of workspace `op` needs for `cfg` (for LMOE_OP_NVFP4_QUANTIZE and
+ * LMOE_OP_FP8_QUANTIZE the tensor is taken as [cfg->T][cfg->l]). Returns 0 for an invalid config or
  * an unknown op, and for LMOE_OP_COMBINE (which needs none). */
 size_t lmoe_workspace_size(const lmoe_config* cfg, int op);
 
@@ -319,6 +341,21 @@ lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int6
                                 const float* global_in, uint8_t* codes, uint8_t* sf,
                                 float* global_out, int sf_layout, void* ws, size_t ws_bytes,
                                 void* stream);
+
+/* FP8 quantiser (the format of the shared experts in the Ultra checkpoint
+ * recipe: chathome page on Nemotron 3 Ultra, quantisation paragraph; one FP32
+ * scale per tensor is the reading taken, the pages give only the format):
+ *  s = scale_in ? *scale_in : fp32(amax / 448) (1 when amax == 0);
+ *  q = E4M3_satfinite_rn(fp32(x / s)) for every element of in [rows][cols]
+ *  (F32 or BF16, cols a multiple of 16), codes [rows][cols] (1 byte each);
+ *  scale_out (device F32, may be NULL) receives s. scale_in: device pointer
+ *  or NULL (a static scale, as for activations).
+ *  Errors: LMOE_ERR_INVALID_ARG for null pointers, cols % 16, an unaligned
+ *  input or code buffer (16 B); LMOE_ERR_WORKSPACE (scale_in NULL and the
+ *  workspace smaller than lmoe_workspace_size(LMOE_OP_FP8_QUANTIZE)). */
+lmoe_status lmoe_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
+                              const float* scale_in, uint8_t* codes, float* scale_out, void* ws,
+                              size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, returns the device error status recorded in the
  * workspace `ws` (LMOE_OK if none) and clears it (the read and the clear run

@@ -7,7 +7,7 @@ loads the shared library and fails loudly if it has not been built
 
 Entry points mirror include/lmoe.h: ``route``, ``permute`` (and
 ``permute_noalloc``), ``expert_ffn``, ``combine``, ``forward`` (and
-``forward_traced``), ``nvfp4_quantize``, plus ``workspace_size``,
+``forward_traced``), ``nvfp4_quantize``, ``fp8_quantize``, plus ``workspace_size``,
 ``padded_rows``, ``workspace``, ``read_device_error``,
 ``selftest_wait_timeout`` and ``kernel_launch_count``.
 Tensor arguments are torch tensors (or None); their ``data_ptr()`` is passed.
@@ -28,12 +28,13 @@ F32, BF16, NVFP4 = 0, 1, 2
 SF_ROWMAJOR, SF_MMA_TILED = 0, 1
 SF_BLOCK_16X16 = 0x10          # OR into the layout: 16 x 16 scale blocks
 FLAG_IDENTITY_PROJ = 1
-OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE = range(6)
+FLAG_SHARED_FP8 = 2            # shared experts in FP8 (E4M3, per-tensor scales)
+OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE, OP_FP8_QUANTIZE = range(7)
 
 EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permute",
            "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
-           "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout")
+           "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -48,7 +49,8 @@ class Config(ctypes.Structure):
 class Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "w_router", "router_bias", "w_down", "w_up", "w1", "w2", "w1_sf", "w2_sf",
-        "w1_gs", "w2_gs", "a_global_scale", "ws1", "ws2")]
+        "w1_gs", "w2_gs", "a_global_scale", "ws1", "ws2", "ws1_scale", "ws2_scale", "shared_x_scale",
+        "shared_h_scale")]
 
 
 class LmoeError(RuntimeError):
@@ -81,6 +83,7 @@ def _load():
         "lmoe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "lmoe_kernel_launch_count": (ctypes.c_uint64, []),
         "lmoe_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_size_t, ctypes.c_uint64, P]),
+        "lmoe_fp8_quantize": (ctypes.c_int, [P, ctypes.c_int, I64, I64, P, P, P, P, ctypes.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -119,9 +122,11 @@ def _check(st: int, where: str):
         raise LmoeError(st, where)
 
 
-def config(T, d, l, N, K, m, n_shared=0, m_shared=0, act=BF16, expert=BF16, identity=False) -> Config:
+def config(T, d, l, N, K, m, n_shared=0, m_shared=0, act=BF16, expert=BF16, identity=False,
+           shared_fp8=False) -> Config:
+    flags = (FLAG_IDENTITY_PROJ if identity else 0) | (FLAG_SHARED_FP8 if shared_fp8 else 0)
     return Config(T=T, d=d, l=l, N=N, K=K, m=m, n_shared=n_shared, m_shared=m_shared, act=act,
-                  expert=expert, flags=FLAG_IDENTITY_PROJ if identity else 0)
+                  expert=expert, flags=flags)
 
 
 def weights(**tensors) -> Weights:
@@ -211,6 +216,14 @@ def nvfp4_quantize(x, in_dtype, rows, cols, global_in, codes, sf, global_out, sf
     _check(lib.lmoe_nvfp4_quantize(_p(x), int(in_dtype), int(rows), int(cols), _p(global_in), _p(codes),
                                    _p(sf), _p(global_out), int(sf_layout), _p(ws), ws.numel(),
                                    _stream(stream)), "lmoe_nvfp4_quantize")
+
+
+def fp8_quantize(x, in_dtype, rows, cols, scale_in, codes, scale_out, ws=None, stream=None):
+    """lmoe_fp8_quantize: E4M3 codes of x / s with one FP32 scale per tensor
+    (scale_in, or amax / 448 when scale_in is None; scale_out receives it)."""
+    _check(lib.lmoe_fp8_quantize(_p(x), int(in_dtype), int(rows), int(cols), _p(scale_in), _p(codes),
+                                 _p(scale_out), _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "lmoe_fp8_quantize")
 
 
 def selftest_wait_timeout(ws, limit_cycles: int, stream=None):

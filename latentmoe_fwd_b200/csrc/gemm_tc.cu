@@ -26,20 +26,22 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over a BF16 tensor [groups][rows][k] (k contiguous); box = 64 x box_rows x 1,
-// 128-byte swizzle, zero fill out of bounds.
+// 3-D map over a tensor [groups][rows][k] (k contiguous) of BF16 (box = 64 x
+// box_rows x 1) or E4M3 bytes (box = 128 x box_rows x 1): 128 bytes of K per
+// row either way, 128-byte swizzle, zero fill out of bounds.
 static bool make_map_bf16(CUtensorMap* map, const TcOperand& op, int box_rows) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc || !op.ptr) return false;
-  if ((reinterpret_cast<uintptr_t>(op.ptr) & 15) != 0 || (op.k * 2) % 16 != 0) return false;
+  if (!enc || !op.ptr || (op.elem != 1 && op.elem != 2)) return false;
+  const int64_t eb = op.elem;
+  if ((reinterpret_cast<uintptr_t>(op.ptr) & 15) != 0 || (op.k * eb) % 16 != 0) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(op.k), static_cast<cuuint64_t>(op.rows),
                         static_cast<cuuint64_t>(op.groups)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(op.k * 2), static_cast<cuuint64_t>(op.rows * op.k * 2)};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(op.k * eb), static_cast<cuuint64_t>(op.rows * op.k * eb)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(op.ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                   const_cast<void*>(op.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -72,6 +74,8 @@ static lmoe_status dispatch_epi(int epi, const CUtensorMap* m, const TcParams& p
     case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_PARTIAL: return launch_tc<BN, STAGES, EPI_PARTIAL>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_SCATTER: return launch_tc<BN, STAGES, EPI_SCATTER>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_SQRELU_Q8: return launch_tc<BN, STAGES, EPI_SQRELU_Q8>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
+    case EPI_SCALE: return launch_tc<BN, STAGES, EPI_SCALE>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
   }
   return LMOE_ERR_INVALID_ARG;
 }
@@ -121,7 +125,16 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   p.partial = L.partial;
   p.scatter_rows = L.scatter_rows;
   p.scatter_k = L.scatter_k;
+  p.fp8 = L.fp8;
+  p.scale_a = L.scale_a;
+  p.scale_w = L.scale_w;
+  p.out_scale = L.out_scale;
   p.err = DevErr{err_word};
+  for (int sg = 0; sg < L.nseg; ++sg)   // one operand kind per launch
+    if (L.a[sg].elem != (L.fp8 ? 1 : 2) || L.b[sg].elem != (L.fp8 ? 1 : 2)) return LMOE_ERR_INVALID_ARG;
+  if ((L.epi == EPI_SQRELU_Q8 && !L.out_scale) || ((L.epi == EPI_SQRELU_Q8 || L.epi == EPI_SCALE) && !L.fp8))
+    return LMOE_ERR_INVALID_ARG;
+  if (L.fp8 && L.grouped) return LMOE_ERR_UNSUPPORTED;
   if (p.ksplit > 1 && (L.grouped || !L.partial)) return LMOE_ERR_INVALID_ARG;
   if (L.epi == EPI_SCATTER && (L.swap || L.ksplit > 1 || !L.scatter_rows || L.scatter_k <= 0))
     return LMOE_ERR_INVALID_ARG;
@@ -148,6 +161,8 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
     case EPI_BF16: launch_k(splitk_reduce_kernel<EPI_BF16>, dim3(rblocks), dim3(256), 0, stream, p); break;
     case EPI_SQRELU: launch_k(splitk_reduce_kernel<EPI_SQRELU>, dim3(rblocks), dim3(256), 0, stream, p); break;
     case EPI_ADD_RES: launch_k(splitk_reduce_kernel<EPI_ADD_RES>, dim3(rblocks), dim3(256), 0, stream, p); break;
+    case EPI_SQRELU_Q8: launch_k(splitk_reduce_kernel<EPI_SQRELU_Q8>, dim3(rblocks), dim3(256), 0, stream, p); break;
+    case EPI_SCALE: launch_k(splitk_reduce_kernel<EPI_SCALE>, dim3(rblocks), dim3(256), 0, stream, p); break;
     default: return LMOE_ERR_INVALID_ARG;
   }
   count_launch();

@@ -35,8 +35,10 @@ enum EpiKind : int {
   EPI_GATE = 3,       // out bf16 = acc * row_scale[row]
   EPI_ADD_RES = 4,    // out bf16 = acc + residual[row][col]
   EPI_PARTIAL = 5,    // split-K: fp32 partial sums, the epilogue runs in the reduction
-  EPI_SCATTER = 6     // out bf16 = acc, row t stored at each padded row scatter_rows[t*K + k]
+  EPI_SCATTER = 6,    // out bf16 = acc, row t stored at each padded row scatter_rows[t*K + k]
                       // (k < scatter_k; negative entries skipped): token-major tiles only
+  EPI_SQRELU_Q8 = 7,  // out E4M3 byte = E4M3(relu(acc * s_a * s_w)^2 / out_scale)
+  EPI_SCALE = 8       // out bf16 = acc * s_a * s_w
 };
 
 struct TcSeg {
@@ -65,6 +67,12 @@ struct TcParams {
   float* partial;             // [ksplit][rows][cols] fp32 (split-K only)
   const int* scatter_rows;    // EPI_SCATTER: [rows][scatter_k] destination rows of each row
   int scatter_k;
+  // FP8 operands (E4M3 codes, 1 byte each; K blocks of 128 elements, the same
+  // 128 bytes per row per stage as BF16): tcgen05.mma kind::f8f6f4
+  int fp8;
+  const float* scale_a;       // EPI_SQRELU_Q8 / EPI_SCALE: per-tensor scales of the two operands
+  const float* scale_w;       //   (device scalars; the product multiplies the accumulator)
+  const float* out_scale;     // EPI_SQRELU_Q8: static scale of the E4M3 output
   // CTA-pair grouped launches only: one dense problem computed in the same
   // launch, out_x[rows_x, cols_x] = epi(X[rows_x, K_x] . Wx[cols_x, K_x]^T)
   int rows_x;                 // 0: none
@@ -212,9 +220,22 @@ __device__ __forceinline__ int tile_mma_n(const TcParams& p, const TileInfo& ti)
   return n < 16 ? 16 : n;
 }
 
+// Product of the two operands' FP8 scales (1 for BF16 operands).
+__device__ __forceinline__ float fp8_acc_scale(const TcParams& p) {
+  return (p.scale_a && p.scale_w) ? __fmul_rn(__ldg(p.scale_a), __ldg(p.scale_w)) : 1.0f;
+}
+
+// E4M3 code of relu(acc * sc)^2 / out_scale (round to nearest even, saturating).
+__device__ __forceinline__ uint32_t sqrelu_e4m3(float acc, float sc, float out_scale) {
+  const float h = fmaxf(__fmul_rn(acc, sc), 0.0f);
+  return cvt_to_e4m3(__fdiv_rn(__fmul_rn(h, h), out_scale));
+}
+
 template <int EPI>
 __device__ __forceinline__ float epi_value(float acc, const TcParams& p, long long row, int col) {
-  if (EPI == EPI_SQRELU) {
+  if (EPI == EPI_SCALE) {
+    return __fmul_rn(acc, fp8_acc_scale(p));
+  } else if (EPI == EPI_SQRELU) {
     float r = fmaxf(acc, 0.0f);
     return r * r;
   } else if (EPI == EPI_GATE) {
@@ -300,7 +321,7 @@ __global__ void __launch_bounds__(192, 1)
           const bool small_b = BN > 32 && p.swap && p.grouped && ti.act_n <= 32;
           mbar_arrive_expect_tx(&full[stage], small_b ? S::kABytes + 32 * 128 : S::kStageBytes);
           const int sg = (p.nseg > 1 && kb >= p.seg[0].kblocks) ? 1 : 0;
-          const int k = (sg ? kb - p.seg[0].kblocks : kb) * 64;
+          const int k = (sg ? kb - p.seg[0].kblocks : kb) * (p.fp8 ? 128 : 64);
           const CUtensorMap* ma = sg ? &tmA1 : &tmA0;
           const CUtensorMap* mb = sg ? &tmB1 : &tmB0;
           const int akg = p.seg[sg].a_kgroup, bkg = p.seg[sg].b_kgroup;
@@ -353,16 +374,23 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, 0x200 + acc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const uint32_t idesc = idesc_bf16_f32(128, tile_mma_n<BN>(p, ti));
+        const uint32_t idesc = p.fp8 ? idesc_e4m3_f32(128, tile_mma_n<BN>(p, ti))
+                                     : idesc_bf16_f32(128, tile_mma_n<BN>(p, ti));
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x300 + stage)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
           const uint32_t sb = sa + S::kABytes;
+          if (p.fp8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32), sdesc_kmajor_sw128(sb + kk * 32), idesc,
-                     (kb != ti.kb0 || kk != 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_e4m3(d_tmem, sdesc_kmajor_sw128(sa + kk * 32), sdesc_kmajor_sw128(sb + kk * 32), idesc,
+                       (kb != ti.kb0 || kk != 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(d_tmem, sdesc_kmajor_sw128(sa + kk * 32), sdesc_kmajor_sw128(sb + kk * 32), idesc,
+                       (kb != ti.kb0 || kk != 0) ? 1u : 0u);
           }
           any = true;
           mma_commit(&empty[stage]);
@@ -408,6 +436,19 @@ __global__ void __launch_bounds__(192, 1)
                 if (col0 + j < p.cols)
                   *reinterpret_cast<float4*>(o + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
                                                                    __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            } else if (EPI == EPI_SQRELU_Q8) {
+              const float sc = fp8_acc_scale(p);
+              const float os = __ldg(p.out_scale);
+              uint32_t w[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                w[j] = sqrelu_e4m3(__uint_as_float(v[4 * j]), sc, os) |
+                       (sqrelu_e4m3(__uint_as_float(v[4 * j + 1]), sc, os) << 8) |
+                       (sqrelu_e4m3(__uint_as_float(v[4 * j + 2]), sc, os) << 16) |
+                       (sqrelu_e4m3(__uint_as_float(v[4 * j + 3]), sc, os) << 24);
+              uint8_t* o = reinterpret_cast<uint8_t*>(p.out) + row * p.ld_out + col0;
+              if (col0 + 16 <= p.cols) *reinterpret_cast<uint4*>(o) = make_uint4(w[0], w[1], w[2], w[3]);
+              if (col0 + 32 <= p.cols) *reinterpret_cast<uint4*>(o + 16) = make_uint4(w[4], w[5], w[6], w[7]);
             } else if (EPI == EPI_SCATTER) {
               // the token's row goes to each of its K slots' padded rows (the
               // expert-grouped GEMM input), streamed past L2
@@ -461,7 +502,7 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
           }
-        } else if (EPI != EPI_PARTIAL && EPI != EPI_F32_BIAS) {
+        } else if (EPI != EPI_PARTIAL && EPI != EPI_F32_BIAS && EPI != EPI_SQRELU_Q8) {
           // weight-major, BF16 out: this lane owns output feature w0 + r and 32
           // tokens; transpose the warp's 32 x 32 block through shared memory so
           // each token's 32 features go out as 16-byte stores
@@ -523,6 +564,11 @@ __global__ void __launch_bounds__(192, 1)
                   p.partial[(static_cast<long long>(ti.split) * p.rows + row) * p.cols + col] = __uint_as_float(v[j]);
                   continue;
                 }
+                if (EPI == EPI_SQRELU_Q8) {
+                  reinterpret_cast<uint8_t*>(p.out)[row * p.ld_out + col] = static_cast<uint8_t>(
+                      sqrelu_e4m3(__uint_as_float(v[j]), fp8_acc_scale(p), __ldg(p.out_scale)));
+                  continue;
+                }
                 const float val = epi_value<EPI>(__uint_as_float(v[j]), p, row, col);
                 if (EPI == EPI_F32_BIAS)
                   reinterpret_cast<float*>(p.out)[row * p.ld_out + col] = val;
@@ -560,6 +606,11 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const TcParams p) {
     for (int sp = 0; sp < p.ksplit; ++sp) acc += p.partial[sp * n + i];
     const long long row = i / p.cols;
     const int col = static_cast<int>(i % p.cols);
+    if (EPI == EPI_SQRELU_Q8) {
+      reinterpret_cast<uint8_t*>(p.out)[row * p.ld_out + col] =
+          static_cast<uint8_t>(sqrelu_e4m3(acc, fp8_acc_scale(p), __ldg(p.out_scale)));
+      continue;
+    }
     const float val = epi_value<EPI>(acc, p, row, col);
     if (EPI == EPI_F32_BIAS)
       reinterpret_cast<float*>(p.out)[row * p.ld_out + col] = val;

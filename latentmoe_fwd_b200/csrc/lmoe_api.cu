@@ -55,8 +55,14 @@ lmoe_status check_config(const lmoe_config* c) {
   if (c->act == LMOE_BF16 && c->expert != LMOE_BF16 && c->expert != LMOE_NVFP4) return LMOE_ERR_UNSUPPORTED;
   if (c->act == LMOE_BF16 && c->n_shared > 0 && c->m_shared % 64) return LMOE_ERR_UNSUPPORTED;
   if (c->expert == LMOE_NVFP4 && (c->l % 256 || c->m % 256)) return LMOE_ERR_UNSUPPORTED;
+  if (c->flags & LMOE_FLAG_SHARED_FP8) {
+    if (c->n_shared <= 0) return LMOE_ERR_INVALID_ARG;
+    if (c->act != LMOE_BF16 || c->d % 16 || c->m_shared % 128) return LMOE_ERR_UNSUPPORTED;
+  }
   return LMOE_OK;
 }
+
+bool shared_fp8(const lmoe_config* c) { return (c->flags & LMOE_FLAG_SHARED_FP8) != 0 && c->n_shared > 0; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -82,7 +88,7 @@ int64_t splitk_floats(const lmoe_config* c, int op) { return c->T * max_dense_co
 struct Layout {
   size_t splitk = 0;        // fp32 split-K partial sums of the weight-major dense GEMMs (T <= 64)
   size_t rsplit = 0;        // fp32 split-K partial sums of the token-major router GEMM (few tiles)
-  size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0,
+  size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0, xq = 0,
          offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, slot_row = 0, scratch = 0, gate = 0, zp = 0,
          zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, ys = 0, total = 0;
 };
@@ -115,7 +121,7 @@ Layout layout(const lmoe_config* c, int op) {
   } else if (op == LMOE_OP_EXPERT_FFN) {
     L.a = take(P * c->m * (fp4 ? 1 : ab) / (fp4 ? 2 : 1));
     if (fp4) L.a_sf = take(P * c->m / 16);
-  } else if (op == LMOE_OP_NVFP4_QUANTIZE) {
+  } else if (op == LMOE_OP_NVFP4_QUANTIZE || op == LMOE_OP_FP8_QUANTIZE) {
     L.partials = take(nvfp4_partials(T * c->l) * 4);
   } else if (op == LMOE_OP_FORWARD) {
     L.logits = take(T * N * 4);
@@ -147,8 +153,9 @@ Layout layout(const lmoe_config* c, int op) {
     L.y = take(P * c->l * ab);
     L.c = take(T * c->l * ab);
     if (c->n_shared) {
-      L.hs = take(T * static_cast<int64_t>(c->n_shared) * c->m_shared * ab);
+      L.hs = take(T * static_cast<int64_t>(c->n_shared) * c->m_shared * ab);   // E4M3 codes with FP8 shared experts
       L.ys = take(T * c->d * ab);
+      if (shared_fp8(c)) L.xq = take(T * c->d);
     }
   }
   L.total = off;
@@ -236,6 +243,64 @@ lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int
   return tc_gemm(L, err, s);
 }
 
+// out[rows, cols] = epi(x[rows, k] . W^T) with E4M3 operands; W is [cols][k],
+// or [k / wgroup][cols][wgroup] (the K axis split over a stack of matrices)
+// when wgroup > 0. epi: EPI_SQRELU_Q8 (E4M3 out) or EPI_SCALE (BF16 out).
+lmoe_status dense_fp8(const void* x, int64_t rows, const void* w, int cols, int64_t k, int wgroup, void* out,
+                      int64_t ld_out, int epi, const float* scale_a, const float* scale_w, const float* out_scale,
+                      float* partial, uint32_t* err, cudaStream_t s) {
+  if (rows == 0) return LMOE_OK;
+  TcLaunch L;
+  const int sbn = swap_bn(rows);
+  TcOperand act{x, k, rows, 1};
+  act.elem = 1;
+  TcOperand wt{w, wgroup ? wgroup : k, cols, wgroup ? k / wgroup : 1};
+  wt.elem = 1;
+  L.fp8 = 1;
+  L.rows = static_cast<int>(rows);
+  L.cols = cols;
+  L.kblocks[0] = static_cast<int>((k + 127) / 128);
+  if (sbn) {
+    L.swap = 1;
+    L.bn = sbn;
+    L.a[0] = wt;
+    L.b[0] = act;
+    L.a_kgroup[0] = wgroup;
+    L.max_tiles = (cols + 127) / 128;
+    L.ksplit = choose_splits(L.max_tiles, L.kblocks[0], partial);
+    L.partial = partial;
+  } else {
+    L.bn = normal_bn(cols);
+    L.a[0] = act;
+    L.b[0] = wt;
+    L.b_kgroup[0] = wgroup;
+    L.max_tiles = ((rows + 127) / 128) * ((cols + L.bn - 1) / L.bn);
+  }
+  L.out = out;
+  L.ld_out = ld_out;
+  L.epi = epi;
+  L.scale_a = scale_a;
+  L.scale_w = scale_w;
+  L.out_scale = out_scale;
+  return tc_gemm(L, err, s);
+}
+
+// The shared experts in FP8: xq = E4M3(x / s_x); hs = E4M3(relu(xq Ws1^T * s_x
+// s_w1)^2 / s_h) over all S experts at once; ys = hs [Ws2_1 .. Ws2_S]^T * s_h
+// s_w2 in BF16 (added to the layer output by the combine or the up-projection).
+lmoe_status shared_experts_fp8(const lmoe_config* cfg, const lmoe_weights* w, const void* x, uint8_t* xq,
+                               uint8_t* hq, void* ys, float* partial, uint32_t* err, cudaStream_t s) {
+  const int64_t T = cfg->T;
+  const int S = cfg->n_shared, ms = cfg->m_shared, d = cfg->d;
+  lmoe_status st = launch_fp8_quantize(x, LMOE_BF16, T, d, w->shared_x_scale, xq, nullptr, nullptr, 0, s);
+  if (st != LMOE_OK) return st;
+  st = dense_fp8(xq, T, w->ws1, S * ms, d, 0, hq, static_cast<int64_t>(S) * ms, EPI_SQRELU_Q8, w->shared_x_scale,
+                 w->ws1_scale, w->shared_h_scale, partial, err, s);
+  if (st != LMOE_OK) return st;
+  return dense_fp8(hq, T, w->ws2, d, static_cast<int64_t>(S) * ms, ms, ys, d, EPI_SCALE, w->shared_h_scale,
+                   w->ws2_scale, nullptr, partial, err, s);
+}
+
 }  // namespace
 }  // namespace lmoe
 
@@ -265,7 +330,7 @@ lmoe_status lmoe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit
 }
 
 size_t lmoe_workspace_size(const lmoe_config* cfg, int op) {
-  if (op == LMOE_OP_NVFP4_QUANTIZE) {
+  if (op == LMOE_OP_NVFP4_QUANTIZE || op == LMOE_OP_FP8_QUANTIZE) {
     if (!cfg || cfg->T < 0 || cfg->l <= 0) return 0;
     return layout(cfg, op).total;
   }
@@ -604,6 +669,26 @@ lmoe_status lmoe_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int6
                                static_cast<cudaStream_t>(stream));
 }
 
+lmoe_status lmoe_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,
+                              uint8_t* codes, float* scale_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!in || !codes || rows < 0 || cols <= 0 || cols % 16) return LMOE_ERR_INVALID_ARG;
+  if (in_dtype != LMOE_BF16 && in_dtype != LMOE_F32) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(codes)) return LMOE_ERR_INVALID_ARG;
+  float* partials = nullptr;
+  int np = 0;
+  if (!scale_in) {
+    lmoe_config c = {};
+    c.T = rows;
+    c.l = static_cast<int32_t>(cols);
+    const Layout L = layout(&c, LMOE_OP_FP8_QUANTIZE);
+    if (!ws || ws_bytes < L.total) return LMOE_ERR_WORKSPACE;
+    partials = at<float>(ws, L.partials);
+    np = nvfp4_partials(rows * cols);
+  }
+  return launch_fp8_quantize(in, in_dtype, rows, cols, scale_in, codes, scale_out, partials, np,
+                             static_cast<cudaStream_t>(stream));
+}
+
 lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x, void* out, void* ws,
                          size_t ws_bytes, void* stream) {
   return lmoe_forward_traced(cfg, w, x, out, ws, ws_bytes, stream, nullptr);
@@ -617,6 +702,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   const bool ident = identity(cfg);
   if (ident != (w->w_down == nullptr) || ident != (w->w_up == nullptr)) return LMOE_ERR_INVALID_ARG;
   if (cfg->n_shared && (!w->ws1 || !w->ws2)) return LMOE_ERR_INVALID_ARG;
+  if (shared_fp8(cfg) && (!w->ws1_scale || !w->ws2_scale || !w->shared_x_scale || !w->shared_h_scale))
+    return LMOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < layout(cfg, LMOE_OP_FORWARD).total) return LMOE_ERR_WORKSPACE;
   const bool fp4 = cfg->expert == LMOE_NVFP4;
   if (fp4 && !fp4_weights_ok(w)) return LMOE_ERR_INVALID_ARG;
@@ -746,7 +833,8 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   const int S = cfg->n_shared, ms = cfg->m_shared;
   void* hs = S ? at<void>(ws, L.hs) : nullptr;
   SharedHidden shared_hidden;
-  if (S && !f32 && !fp4) {
+  const bool fp8sh = shared_fp8(cfg);
+  if (S && !f32 && !fp4 && !fp8sh) {
     shared_hidden.x = x;
     shared_hidden.ws1 = w->ws1;
     shared_hidden.d = d;
@@ -770,7 +858,17 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
 
   // 5. combine; with identity projections it is the output when there are no
   // shared experts or their output ys is already there (then combine adds it)
-  const bool ys_ready = shared_hidden.ys_done;
+  bool ys_ready = shared_hidden.ys_done;
+  // FP8 shared experts: with identity projections their output is added by the
+  // combine, so it is computed first; otherwise with the up-projection (stage 7)
+  auto run_shared_fp8 = [&]() {
+    return shared_experts_fp8(cfg, w, x, at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.hs), at<void>(ws, L.ys), splitk,
+                              err, s);
+  };
+  if (fp8sh && ident) {
+    if ((st = run_shared_fp8()) != LMOE_OK) return st;
+    ys_ready = true;
+  }
   const bool combine_is_out = ident && (cfg->n_shared == 0 || ys_ready);
   void* c = combine_is_out ? out : at<void>(ws, L.c);
   if ((st = launch_combine(y, cfg->act, idx, inv_perm, offsets, poff, nullptr, ident && ys_ready ? at<void>(ws, L.ys)
@@ -784,7 +882,10 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
 
   // 6. shared experts' hidden layer on the d-dim x: hs = relu(x Ws1^T)^2, all S at
   // once (already done when it rode along in the first expert GEMM's launch)
-  if (S && !shared_hidden.done) {
+  if (fp8sh && !ys_ready) {
+    if ((st = run_shared_fp8()) != LMOE_OK) return st;
+    ys_ready = true;
+  } else if (S && !shared_hidden.done) {
     if (f32) {
       SimtLaunch G;
       G.rows = static_cast<int>(T);

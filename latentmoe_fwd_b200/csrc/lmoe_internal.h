@@ -47,10 +47,11 @@ inline void mark_configured(std::atomic<uint64_t>& mask, int dev) {
 
 // ----- tensor-core GEMM (gemm_tc.cu) -----
 struct TcOperand {
-  const void* ptr;     // BF16 [groups][rows][k], k contiguous
+  const void* ptr;     // [groups][rows][k], k contiguous: BF16, or E4M3 bytes with elem == 1
   int64_t k;
   int64_t rows;
   int64_t groups;
+  int elem = 2;        // bytes per element: 2 (BF16) or 1 (E4M3)
 };
 
 struct TcLaunch {
@@ -80,6 +81,10 @@ struct TcLaunch {
   float* partial = nullptr;      // [ksplit][rows][cols]
   const int* scatter_rows = nullptr;   // EPI_SCATTER (token-major only): [rows][scatter_k] destination rows
   int scatter_k = 0;
+  int fp8 = 0;                   // 1: E4M3 operands (every segment), K blocks of 128
+  const float* scale_a = nullptr;     // EPI_SQRELU_Q8 / EPI_SCALE: operand scales (device scalars)
+  const float* scale_w = nullptr;
+  const float* out_scale = nullptr;   // EPI_SQRELU_Q8: static scale of the E4M3 output
   // tc2_gemm only: a dense problem in the same launch, out_x = epi(x_act . x_wt^T)
   TcOperand x_act = {};          // [rows_x][k] activations
   TcOperand x_wt = {};           // [cols_x][k] weights, or [groups][cols_x][x_kgroup] with K split in groups
@@ -172,5 +177,9 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
                                   float* global_out, int sf_layout, float* partials,
                                   int npartials, uint32_t* err, cudaStream_t s);
 int nvfp4_partials(int64_t elems);
+// FP8 E4M3 codes of in / s with one FP32 scale per tensor (scale_in, or the
+// tensor's amax / 448 when scale_in is null; scale_out receives it).
+lmoe_status launch_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,
+                                uint8_t* codes, float* scale_out, float* partials, int npartials, cudaStream_t s);
 
 }  // namespace lmoe

@@ -801,8 +801,10 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
 }
 
 // Every CTA reduces the per-CTA maxima the same way (max is exact, so the
-// order does not matter) and derives s_g = fp32(amax / 2688), 1 when amax = 0.
-__device__ __forceinline__ float cta_global_scale(const float* partials, int np, const float* global_in) {
+// order does not matter) and derives s_g = fp32(amax / divisor), 1 when amax
+// = 0 (divisor 2688 = 6 * 448 for NVFP4, 448 for FP8).
+__device__ __forceinline__ float cta_global_scale(const float* partials, int np, const float* global_in,
+                                                  float divisor = 2688.0f) {
   __shared__ float red[kQThreads / 32];
   __shared__ float result;
   if (global_in) return __ldg(global_in);
@@ -815,7 +817,7 @@ __device__ __forceinline__ float cta_global_scale(const float* partials, int np,
   if (threadIdx.x == 0) {
     float r = 0.0f;
     for (int i = 0; i < kQThreads / 32; ++i) r = fmaxf(r, red[i]);
-    result = r == 0.0f ? 1.0f : __fdiv_rn(r, 2688.0f);
+    result = r == 0.0f ? 1.0f : __fdiv_rn(r, divisor);
   }
   __syncthreads();
   return result;
@@ -993,6 +995,64 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
     launch_k(nvfp4_encode_kernel<float>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
              static_cast<const float*>(in), rows, cols, static_cast<const float*>(partials), global_in ? 0 : npartials,
              global_in, codes, sf, global_out, tiled);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+// ===========================================================================
+// FP8 (E4M3) with one FP32 scale per tensor (the shared experts' weights and
+// activations): s = scale_in ? *scale_in : fp32(amax / 448) (1 when amax = 0);
+// q = E4M3_rn_satfinite(fp32(x / s)), the division an IEEE fp32 division as
+// the definition states. A thread per 16 elements, 16 code bytes per store.
+// ===========================================================================
+template <typename TI>
+__global__ void __launch_bounds__(kQThreads) fp8_encode_kernel(const TI* __restrict__ in, int64_t n,
+                                                               const float* __restrict__ partials, int np,
+                                                               const float* __restrict__ scale_in,
+                                                               uint8_t* __restrict__ codes,
+                                                               float* __restrict__ scale_out) {
+  pdl_begin();
+  const float s = cta_global_scale(partials, np, scale_in, 448.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = s;
+  const int64_t nv = n / 16;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float x[16];
+    load16<TI>(in + v * 16, x);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = cvt_e4m3(__fdiv_rn(x[4 * j], s)) | (cvt_e4m3(__fdiv_rn(x[4 * j + 1], s)) << 8) |
+             (cvt_e4m3(__fdiv_rn(x[4 * j + 2], s)) << 16) | (cvt_e4m3(__fdiv_rn(x[4 * j + 3], s)) << 24);
+    *reinterpret_cast<uint4*>(codes + v * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+lmoe_status launch_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,
+                                uint8_t* codes, float* scale_out, float* partials, int npartials, cudaStream_t s) {
+  const int64_t n = rows * cols;
+  if (n == 0) return LMOE_OK;
+  if (!scale_in) {
+    if (in_dtype == LMOE_BF16)
+      launch_k(nvfp4_amax_kernel<__nv_bfloat16>, dim3(npartials), dim3(kQThreads), 0, s,
+               static_cast<const __nv_bfloat16*>(in), n, partials);
+    else
+      launch_k(nvfp4_amax_kernel<float>, dim3(npartials), dim3(kQThreads), 0, s, static_cast<const float*>(in), n,
+               partials);
+    count_launch();
+  }
+  const int sms = device_sm_count();
+  int64_t blocks = (n / 16 + kQThreads - 1) / kQThreads;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  if (blocks < 1) blocks = 1;
+  const int np = scale_in ? 0 : npartials;
+  if (in_dtype == LMOE_BF16)
+    launch_k(fp8_encode_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
+             static_cast<const __nv_bfloat16*>(in), n, static_cast<const float*>(partials), np, scale_in, codes,
+             scale_out);
+  else
+    launch_k(fp8_encode_kernel<float>, dim3(static_cast<unsigned>(blocks)), dim3(kQThreads), 0, s,
+             static_cast<const float*>(in), n, static_cast<const float*>(partials), np, scale_in, codes, scale_out);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

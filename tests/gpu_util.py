@@ -22,7 +22,18 @@ def cfg_of(wl, T=None):
     expert = {"f32": L.F32, "bf16": L.BF16, "nvfp4": L.NVFP4}[wl.dtype]
     return L.config(T=wl.T if T is None else T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m,
                     n_shared=wl.n_shared, m_shared=wl.m_shared, act=act, expert=expert,
-                    identity=wl.identity)
+                    identity=wl.identity, shared_fp8=getattr(wl, "shared_fp8", False))
+
+
+def fp8_quantize_dev(x: torch.Tensor, rows: int, cols: int, scale_in=None):
+    """lmoe_fp8_quantize on a device tensor: (codes [rows][cols] uint8, scale [1])."""
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+    scale = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = L.workspace(L.config(T=rows, d=cols, l=cols, N=1, K=1, m=cols), L.OP_FP8_QUANTIZE)
+    dt = L.BF16 if x.dtype == torch.bfloat16 else L.F32
+    L.fp8_quantize(x, dt, rows, cols, scale_in, codes, scale, ws)
+    torch.cuda.synchronize()
+    return codes, scale
 
 
 def quantize_dev(x: torch.Tensor, rows: int, cols: int, layout=L.SF_ROWMAJOR, global_in=None):
@@ -75,6 +86,15 @@ class DevLayer:
             a_gs = torch.tensor([inp["a_global_scale"]], dtype=torch.float32, device="cuda")
             self.t.update(w1=c1, w2=c2)
             extra = dict(w1_sf=f1, w2_sf=f2, w1_gs=g1, w2_gs=g2, a_global_scale=a_gs)
+        if getattr(wl, "shared_fp8", False):
+            # each shared weight tensor (all S experts stacked) quantised with its own amax scale
+            S, ms, d = wl.n_shared, wl.m_shared, wl.d
+            q1, s1 = fp8_quantize_dev(self.t["ws1"].reshape(S * ms, d), S * ms, d)
+            q2, s2 = fp8_quantize_dev(self.t["ws2"].reshape(S * d, ms), S * d, ms)
+            self.t.update(ws1=q1.reshape(S, ms, d), ws2=q2.reshape(S, d, ms))
+            extra.update(ws1_scale=s1, ws2_scale=s2,
+                         shared_x_scale=torch.tensor([inp["shared_x_scale"]], dtype=torch.float32, device="cuda"),
+                         shared_h_scale=torch.tensor([inp["shared_h_scale"]], dtype=torch.float32, device="cuda"))
         self.w = L.weights(w_router=self.t["w_router"], router_bias=self.bias, w_down=self.t["w_down"],
                            w_up=self.t["w_up"], w1=self.t["w1"], w2=self.t["w2"], ws1=self.t["ws1"],
                            ws2=self.t["ws2"], **extra)

@@ -183,3 +183,23 @@ def test_documented_host_errors_of_each_entry_point():
     # reading the error word needs a workspace
     info = ctypes.c_uint32(0)
     assert L.lib.lmoe_read_device_error(None, None, ctypes.byref(info)) == L.ERR_INVALID_ARG
+
+
+def test_fp8_shared_config_checks():
+    """LMOE_FLAG_SHARED_FP8: m_shared must be a multiple of 128 and there must
+    be shared experts (host-side checks; no GPU needed)."""
+    base = dict(T=64, d=512, l=256, N=8, K=2, m=256, shared_fp8=True)
+    assert L.workspace_size(L.config(**base, n_shared=2, m_shared=64), L.OP_FORWARD) == 0
+    assert L.workspace_size(L.config(**base, n_shared=0, m_shared=0), L.OP_FORWARD) == 0
+    assert L.workspace_size(L.config(**base, n_shared=2, m_shared=128), L.OP_FORWARD) > 0
+    assert L.workspace_size(L.config(T=100, d=64, l=64, N=1, K=1, m=64), L.OP_FP8_QUANTIZE) > 0
+
+
+def test_fp8_quantize_host_errors():
+    dummy = 256   # a fake aligned address; nothing is launched on these errors
+    with pytest.raises(L.LmoeError) as e:
+        L.fp8_quantize(dummy, L.BF16, 4, 24, None, dummy, None, stream=0)   # cols % 16
+    assert e.value.status == L.ERR_INVALID_ARG
+    with pytest.raises(L.LmoeError) as e:
+        L.fp8_quantize(dummy, L.BF16, 4, 32, None, dummy, None, stream=0)   # amax scale needs a workspace
+    assert e.value.status == L.ERR_WORKSPACE

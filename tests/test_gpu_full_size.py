@@ -203,10 +203,10 @@ def test_full_size_expert_ffn_every_tile(name):
     assert raw_ok
 
 
-@pytest.mark.parametrize("name", ["ultra_nvfp4", "ultra_decode_nvfp4"])
+@pytest.mark.parametrize("name", ["ultra_nvfp4", "ultra_decode_nvfp4", "ultra_nvfp4_fp8shared"])
 def test_full_size_nvfp4(name):
-    """NVFP4 workloads at full size (the T=8192 layer and the same layer in
-    decode): weights quantised on the GPU (bit-exact per expert against the
+    """NVFP4 workloads at full size (the T=8192 layer, the same layer in
+    decode, and the T=8192 layer with FP8 shared experts): weights quantised on the GPU (bit-exact per expert against the
     oracle for a sample of experts), routing checked over every token, outputs
     of a stratified token sample within 8e-2 * RMS beyond half a BF16 step,
     allowing the documented z-rounding near-ties."""

@@ -136,11 +136,28 @@ def test_hardware_e2m1_conversion_sweep():
     assert np.array_equal(got, O.e2m1_encode(v.astype(np.float64)))
 
 
+def prequantize_experts(W, experts, threads=16):
+    """Fill the oracle weights view's NVFP4 cache for W1 and W2 of the given
+    experts on a thread pool (the quantiser is array code, so threads overlap)."""
+    import concurrent.futures as cf
+    quant = O.nvfp4_quantize_2d if getattr(W.wl, "w_block2d", False) else O.nvfp4_quantize
+    todo = [(k, int(e)) for e in experts for k in ("w1", "w2") if (k, int(e)) not in W._q]
+
+    def one(ke):
+        k, e = ke
+        return ke, quant(O.to_f64(W.inp[k][e], W.st))
+
+    with cf.ThreadPoolExecutor(threads) as ex:
+        for ke, q in ex.map(one, todo):
+            W._q[ke] = q
+
+
 def nvfp4_token_errors(wl, inp, out, gidx, toks, tol):
     """Per-token max|err| beyond half a BF16 step, relative to RMS(oracle out),
     for the given tokens; tokens over `tol` whose latent z has code-changing
     rounding near-ties are re-compared against every alternative rounding."""
     W = O.weights_view(wl, inp, cache=True)
+    prequantize_experts(W, np.unique(gidx[toks]))
     ref = O.forward(wl, inp, tokens=toks, idx_override=gidx[toks], weights=W)
     rms = np.sqrt(np.mean(ref["out"] ** 2))
 
