@@ -357,6 +357,65 @@ lmoe_status lmoe_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_
                               const float* scale_in, uint8_t* codes, float* scale_out, void* ws,
                               size_t ws_bytes, void* stream);
 
+/* NVFP4 quantiser of the training recipe's GEMM operands (greeksharifa page,
+ * section 2.4 "NVFP4 Training"; notes.yuuk.io page, section 4: gradients are
+ * rounded stochastically, the wgrad inputs get a random Hadamard transform,
+ * weights use 2-D scale blocks; the transform and rounding details are
+ * readings, the pages name only the techniques). Quantises out = in
+ * [rows][cols], or in^T with LMOE_QX_TRANSPOSE ([cols][rows]: the blocks then
+ * run along the input's rows, e.g. along the tokens of an activation or
+ * gradient), along out's rows with lmoe_nvfp4_quantize's two-level scales:
+ *  - LMOE_QX_RHT: every 16-block v of out's rows becomes H16 diag(s) v / 4
+ *    first (H16 the Sylvester Hadamard matrix, s_i = -1 where bit i of
+ *    rht_signs is set), formed in fp64;
+ *  - LMOE_QX_SR: elements round stochastically: between grid neighbours
+ *    lo <= |v| < hi to hi when u * (hi - lo) < |v| - lo, u = (w >> 8) * 2^-24
+ *    with w word i % 4 of Philox-4x32-10 (Salmon et al., SC11) at counter
+ *    (i / 4 low, i / 4 high, sr_stream, 0) under key (seed low, seed high),
+ *    i = r * out_cols + c the element's index in out; |v| >= 6 saturates;
+ *    the block scales still round to nearest even;
+ *  - sf_layout | LMOE_SF_BLOCK_16X16: 16 x 16 scale blocks (not with RHT or SR).
+ *  Every step after the transform is an fp32 operation on its exact inputs
+ *  (fp64 division rounded once to fp32), so results equal those of the
+ *  definition taken in exact arithmetic and rounded step by step.
+ *  codes [out_rows][out_cols/2], sf per sf_layout, global_in / global_out as
+ *  lmoe_nvfp4_quantize. out_cols must be a multiple of 16.
+ *  Errors: LMOE_ERR_INVALID_ARG for null pointers, out_cols % 16, an unknown
+ *  flag or layout, 2-D blocks with RHT or SR, an unaligned input (16 B) or
+ *  code buffer (8 B); LMOE_ERR_WORKSPACE (global_in NULL and the workspace
+ *  smaller than lmoe_nvfp4_quantize_ex_workspace(rows, cols)). */
+#define LMOE_QX_TRANSPOSE 1u
+#define LMOE_QX_RHT 2u
+#define LMOE_QX_SR 4u
+size_t lmoe_nvfp4_quantize_ex_workspace(int64_t rows, int64_t cols);
+lmoe_status lmoe_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
+                                   uint32_t rht_signs, uint64_t seed, uint32_t sr_stream,
+                                   const float* global_in, uint8_t* codes, uint8_t* sf, float* global_out,
+                                   int sf_layout, void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped block-scaled NVFP4 GEMM (the kernel of the routed experts, exposed
+ * for the training recipe's dgrad and wgrad; greeksharifa page, section 2.4
+ * "NVFP4 Training": fprop, dgrad and wgrad run as NVFP4 GEMMs):
+ *   out[r][c] = BF16( g_a * g_b[e] * sum_k qa[r][k] sa[r][k/16] qb[e][c][k] sb[e][c][k/16] )
+ *   (times row_scale[r] when given), for rows r of group e: rows
+ *   padded_offsets[e] .. padded_offsets[e] + offsets[e+1] - offsets[e].
+ *  a_codes [a_rows][k/2] with a_sf in LMOE_SF_MMA_TILED layout over a_rows
+ *    (a multiple of 128; each group's padded range a multiple of 128);
+ *  a_global: device F32, one value, or [groups] with a_global_per_group;
+ *  b_codes [groups][cols][k/2], b_sf [groups] MMA-tiled blocks of cols x k/16,
+ *    b_global [groups] device F32;
+ *  k and cols multiples of 256; out [a_rows][ld_out] BF16 (padding rows
+ *  unspecified). ws: at least 256 bytes, its first 256 zeroed before first
+ *  use (the error word). One group with offsets {0, a_rows} is a plain GEMM.
+ *  Errors: LMOE_ERR_INVALID_ARG for null or unaligned buffers, sizes out of
+ *  range; LMOE_ERR_UNSUPPORTED for k or cols not multiples of 256 or more
+ *  than 1024 groups; LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT. */
+lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* padded_offsets, int64_t a_rows,
+                            const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                            int a_global_per_group, const uint8_t* b_codes, const uint8_t* b_sf,
+                            const float* b_global, int cols, int64_t k, const float* row_scale, void* out,
+                            int64_t ld_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, returns the device error status recorded in the
  * workspace `ws` (LMOE_OK if none) and clears it (the read and the clear run
  * on `stream`). `info` (host, may be NULL) receives a kernel-specific detail

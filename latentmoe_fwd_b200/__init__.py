@@ -7,7 +7,7 @@ loads the shared library and fails loudly if it has not been built
 
 Entry points mirror include/lmoe.h: ``route``, ``permute`` (and
 ``permute_noalloc``), ``expert_ffn``, ``combine``, ``forward`` (and
-``forward_traced``), ``nvfp4_quantize``, ``fp8_quantize``, plus ``workspace_size``,
+``forward_traced``), ``nvfp4_quantize``, ``nvfp4_quantize_ex``, ``fp8_quantize``, plus ``workspace_size``,
 ``padded_rows``, ``workspace``, ``read_device_error``,
 ``selftest_wait_timeout`` and ``kernel_launch_count``.
 Tensor arguments are torch tensors (or None); their ``data_ptr()`` is passed.
@@ -27,6 +27,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOU
 F32, BF16, NVFP4 = 0, 1, 2
 SF_ROWMAJOR, SF_MMA_TILED = 0, 1
 SF_BLOCK_16X16 = 0x10          # OR into the layout: 16 x 16 scale blocks
+QX_TRANSPOSE, QX_RHT, QX_SR = 1, 2, 4   # nvfp4_quantize_ex flags
 FLAG_IDENTITY_PROJ = 1
 FLAG_SHARED_FP8 = 2            # shared experts in FP8 (E4M3, per-tensor scales)
 OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE, OP_FP8_QUANTIZE = range(7)
@@ -34,7 +35,8 @@ OP_ROUTE, OP_PERMUTE, OP_EXPERT_FFN, OP_COMBINE, OP_FORWARD, OP_NVFP4_QUANTIZE, 
 EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permute",
            "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
-           "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize")
+           "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize",
+           "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_gemm")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -84,6 +86,12 @@ def _load():
         "lmoe_kernel_launch_count": (ctypes.c_uint64, []),
         "lmoe_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_size_t, ctypes.c_uint64, P]),
         "lmoe_fp8_quantize": (ctypes.c_int, [P, ctypes.c_int, I64, I64, P, P, P, P, ctypes.c_size_t, P]),
+        "lmoe_nvfp4_quantize_ex_workspace": (ctypes.c_size_t, [I64, I64]),
+        "lmoe_nvfp4_gemm": (ctypes.c_int, [ctypes.c_int, P, P, I64, P, P, P, ctypes.c_int, P, P, P, ctypes.c_int,
+                                           I64, P, P, I64, P, ctypes.c_size_t, P]),
+        "lmoe_nvfp4_quantize_ex": (ctypes.c_int, [P, ctypes.c_int, I64, I64, ctypes.c_uint32, ctypes.c_uint32,
+                                                  ctypes.c_uint64, ctypes.c_uint32, P, P, P, P, ctypes.c_int, P,
+                                                  ctypes.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -224,6 +232,29 @@ def fp8_quantize(x, in_dtype, rows, cols, scale_in, codes, scale_out, ws=None, s
     _check(lib.lmoe_fp8_quantize(_p(x), int(in_dtype), int(rows), int(cols), _p(scale_in), _p(codes),
                                  _p(scale_out), _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
            "lmoe_fp8_quantize")
+
+
+def nvfp4_quantize_ex(x, in_dtype, rows, cols, flags, rht_signs, seed, sr_stream, global_in, codes, sf, global_out,
+                      sf_layout, ws=None, stream=None):
+    """lmoe_nvfp4_quantize_ex: the training recipe's NVFP4 quantiser (transpose,
+    random Hadamard transform, stochastic rounding; see the header)."""
+    if ws is None and global_in is None:
+        import torch
+        ws = torch.zeros(int(lib.lmoe_nvfp4_quantize_ex_workspace(int(rows), int(cols))), dtype=torch.uint8,
+                         device="cuda")
+    _check(lib.lmoe_nvfp4_quantize_ex(_p(x), int(in_dtype), int(rows), int(cols), int(flags), int(rht_signs),
+                                      int(seed), int(sr_stream), _p(global_in), _p(codes), _p(sf), _p(global_out),
+                                      int(sf_layout), _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "lmoe_nvfp4_quantize_ex")
+
+
+def nvfp4_gemm(groups, offsets, padded_offsets, a_rows, a_codes, a_sf, a_global, a_global_per_group, b_codes, b_sf,
+               b_global, cols, k, row_scale, out, ld_out, ws, stream=None):
+    """lmoe_nvfp4_gemm: grouped block-scaled NVFP4 GEMM with a BF16 result."""
+    _check(lib.lmoe_nvfp4_gemm(int(groups), _p(offsets), _p(padded_offsets), int(a_rows), _p(a_codes), _p(a_sf),
+                               _p(a_global), int(a_global_per_group), _p(b_codes), _p(b_sf), _p(b_global),
+                               int(cols), int(k), _p(row_scale), _p(out), int(ld_out), _p(ws), ws.numel(),
+                               _stream(stream)), "lmoe_nvfp4_gemm")
 
 
 def selftest_wait_timeout(ws, limit_cycles: int, stream=None):

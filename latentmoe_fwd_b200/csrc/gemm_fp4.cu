@@ -76,6 +76,7 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   p.padded_offsets = L.padded_offsets;
   p.groups = L.groups;
   p.in_scale = L.in_scale;
+  p.in_scale_grouped = L.in_scale_grouped;
   p.w_scale = L.w_scale;
   p.out_scale = L.out_scale;
   p.row_scale = L.row_scale;

@@ -39,7 +39,8 @@ struct Fp4Params {
   const int* offsets;
   const int* padded_offsets;
   int groups;
-  const float* in_scale;      // global scale of A (device scalar)
+  const float* in_scale;      // global scale of A (device scalar, or [groups] with in_scale_grouped)
+  int in_scale_grouped;
   const float* w_scale;       // [groups] global scales of B
   const float* out_scale;     // GEMM1: static global scale of a (device scalar)
   const float* row_scale;     // GEMM2: gate per padded row (nullable)
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     const int half = (warp - 2) >> 2;   // which four of the eight 32-column chunks
     const int r = q * 32 + lane;
     int local = 0;
-    const float in_s = __ldg(p.in_scale);
+    const float in_s0 = __ldg(p.in_scale);
     const float out_s = (EPI == FP4_EPI_SQRELU_QUANT) ? __ldg(p.out_scale) : 0.0f;
     const int groups64_out = (p.cols + 63) / 64;
     const uint64_t pol_out = policy_evict_first();
@@ -328,6 +329,7 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
       const bool row_ok = r < act_n;
       // per-tile scalars fetched before the accumulator is ready
       const float gate = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && row_ok) ? __ldg(p.row_scale + row) : 1.0f;
+      const float in_s = p.in_scale_grouped ? __ldg(p.in_scale + e) : in_s0;
       const float scale = __fmul_rn(in_s, __ldg(p.w_scale + e));
       if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1400 + buf)) break;
       tc_fence_after();

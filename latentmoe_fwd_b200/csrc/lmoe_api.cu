@@ -689,6 +689,67 @@ lmoe_status lmoe_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_
                              static_cast<cudaStream_t>(stream));
 }
 
+size_t lmoe_nvfp4_quantize_ex_workspace(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols <= 0) return 0;
+  return 256 + static_cast<size_t>(nvfp4x_partials(rows * (cols / 16 > 0 ? cols / 16 : 1))) * 8;
+}
+
+lmoe_status lmoe_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
+                                   uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
+                                   uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!in || !codes || !sf || rows < 0 || cols < 0) return LMOE_ERR_INVALID_ARG;
+  if (in_dtype != LMOE_BF16 && in_dtype != LMOE_F32) return LMOE_ERR_INVALID_ARG;
+  if (flags & ~(LMOE_QX_TRANSPOSE | LMOE_QX_RHT | LMOE_QX_SR)) return LMOE_ERR_INVALID_ARG;
+  const int base = sf_layout & ~LMOE_SF_BLOCK_16X16;
+  if ((base != LMOE_SF_ROWMAJOR && base != LMOE_SF_MMA_TILED) || (sf_layout & ~(LMOE_SF_BLOCK_16X16 | 1)))
+    return LMOE_ERR_INVALID_ARG;
+  if ((sf_layout & LMOE_SF_BLOCK_16X16) && (flags & (LMOE_QX_RHT | LMOE_QX_SR))) return LMOE_ERR_INVALID_ARG;
+  const bool tr = (flags & LMOE_QX_TRANSPOSE) != 0;
+  const int64_t out_cols = tr ? rows : cols;
+  if (out_cols % 16) return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(in) || (reinterpret_cast<uintptr_t>(codes) & 7)) return LMOE_ERR_INVALID_ARG;
+  if (!global_in && (!ws || ws_bytes < lmoe_nvfp4_quantize_ex_workspace(rows, cols))) return LMOE_ERR_WORKSPACE;
+  double* partials = ws ? reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + 256) : nullptr;
+  return launch_nvfp4_quantize_ex(in, in_dtype, rows, cols, flags, rht_signs, seed, sr_stream, global_in, codes, sf,
+                                  global_out, sf_layout, partials, static_cast<cudaStream_t>(stream));
+}
+
+lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* padded_offsets, int64_t a_rows,
+                            const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                            int a_global_per_group, const uint8_t* b_codes, const uint8_t* b_sf,
+                            const float* b_global, int cols, int64_t k, const float* row_scale, void* out,
+                            int64_t ld_out, void* ws, size_t ws_bytes, void* stream) {
+  if (groups <= 0 || !offsets || !padded_offsets || !a_codes || !a_sf || !a_global || !b_codes || !b_sf ||
+      !b_global || !out)
+    return LMOE_ERR_INVALID_ARG;
+  if (a_rows < 0 || a_rows % 128 || a_rows > (int64_t(1) << 30) || cols <= 0 || k <= 0 || ld_out < cols)
+    return LMOE_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(b_codes) || !aligned16(b_sf) || !aligned16(out) ||
+      (ld_out * 2) % 16)
+    return LMOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < 256) return LMOE_ERR_WORKSPACE;
+  Fp4Launch g;
+  g.a_codes = a_codes;
+  g.a_sf = a_sf;
+  g.a_rows = a_rows;
+  g.b_codes = b_codes;
+  g.b_sf = b_sf;
+  g.k = k;
+  g.cols = cols;
+  g.groups = groups;
+  g.offsets = offsets;
+  g.padded_offsets = padded_offsets;
+  g.in_scale = a_global;
+  g.in_scale_grouped = a_global_per_group != 0;
+  g.w_scale = b_global;
+  g.row_scale = row_scale;
+  g.quant_out = 0;
+  g.out = out;
+  g.ld_out = ld_out;
+  return fp4_gemm(g, err_word(ws), static_cast<cudaStream_t>(stream));
+}
+
 lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x, void* out, void* ws,
                          size_t ws_bytes, void* stream) {
   return lmoe_forward_traced(cfg, w, x, out, ws, ws_bytes, stream, nullptr);

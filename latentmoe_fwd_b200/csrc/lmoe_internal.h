@@ -112,7 +112,8 @@ struct Fp4Launch {
   int groups = 0;
   const int* offsets = nullptr;
   const int* padded_offsets = nullptr;
-  const float* in_scale = nullptr;   // device scalar
+  const float* in_scale = nullptr;   // device scalar, or [groups] with in_scale_grouped
+  int in_scale_grouped = 0;
   const float* w_scale = nullptr;    // [groups]
   const float* out_scale = nullptr;  // device scalar (quant_out)
   const float* row_scale = nullptr;  // gates (GEMM 2)
@@ -177,6 +178,13 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
                                   float* global_out, int sf_layout, float* partials,
                                   int npartials, uint32_t* err, cudaStream_t s);
 int nvfp4_partials(int64_t elems);
+// Training-recipe NVFP4 quantiser (lmoe_train.cu): partials holds
+// nvfp4x_partials(out_rows * out_cols / 16) doubles.
+int nvfp4x_partials(int64_t blocks);
+lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
+                                     uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
+                                     uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
+                                     cudaStream_t s);
 // FP8 E4M3 codes of in / s with one FP32 scale per tensor (scale_in, or the
 // tensor's amax / 448 when scale_in is null; scale_out receives it).
 lmoe_status launch_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,

@@ -1,0 +1,317 @@
+// NVFP4 training-recipe quantiser: the operands of the expert GEMMs' dgrad
+// and wgrad (greeksharifa page on the Nemotron 3 whitepaper, section 2.4
+// "NVFP4 Training"; notes.yuuk.io page, section 4 "NVFP4 pre-training"):
+// gradients are rounded stochastically, the wgrad inputs get a random
+// Hadamard transform along the contraction (token) dimension, weights use
+// 16 x 16 scale blocks. One kernel covers every combination the recipe uses:
+//
+//   out = in or in^T (LMOE_QX_TRANSPOSE: blocks run along the input's rows)
+//   each 16-block v of out's rows -> H16 diag(s) v / 4 (LMOE_QX_RHT)
+//   two-level NVFP4 scales as lmoe_nvfp4_quantize (1 x 16, or 16 x 16 blocks)
+//   elements rounded to nearest even, or stochastically (LMOE_QX_SR) with
+//   uniforms from Philox-4x32-10 at the element's index in `out`.
+//
+// Arithmetic: the transform is formed in fp64 (exact for BF16 inputs), and
+// every step after it is an IEEE fp64 operation rounded to fp32 where the
+// recipe's step is an fp32 one, so the codes equal those of the same steps
+// taken in fp64 and rounded, input for input.
+#include <cuda_bf16.h>
+
+#include "lmoe_device.cuh"
+#include "lmoe_internal.h"
+
+namespace lmoe {
+namespace {
+
+constexpr int kXThreads = 256;
+
+// E4M3 code -> exact value: subnormal f * 2^-9, normal (8 + f) * 2^(e - 10).
+__device__ __forceinline__ double e4m3_exact(uint32_t c) {
+  const int e = (c >> 3) & 15, f = c & 7;
+  return e == 0 ? ldexp(static_cast<double>(f), -9) : ldexp(static_cast<double>(8 + f), e - 10);
+}
+
+// Philox-4x32-10 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
+// SC11): ten rounds; each takes the 64-bit products of words 0 and 2 with the
+// multipliers 0xD2511F53 and 0xCD9E8D57, and the key grows by the Weyl
+// constants 0x9E3779B9 and 0xBB67AE85 between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// 16 uniforms of elements i0 .. i0+15 (i0 a multiple of 4): element i takes
+// word i % 4 of Philox at counter (i / 4 low word, i / 4 high word, stream, 0)
+// under key (seed low word, seed high word); u = (word >> 8) * 2^-24.
+__device__ __forceinline__ void sr_uniforms16(uint64_t i0, uint64_t seed, uint32_t stream, float (&u)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint64_t c = (i0 >> 2) + q;
+    const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), stream, 0u),
+                                  static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+    u[4 * q + 0] = ldexpf(static_cast<float>(w.x >> 8), -24);
+    u[4 * q + 1] = ldexpf(static_cast<float>(w.y >> 8), -24);
+    u[4 * q + 2] = ldexpf(static_cast<float>(w.z >> 8), -24);
+    u[4 * q + 3] = ldexpf(static_cast<float>(w.w >> 8), -24);
+  }
+}
+
+struct QxParams {
+  const void* in;
+  int bf16;              // input BF16 (else F32)
+  int64_t rows, cols;    // input dims
+  int transpose;
+  int rht;
+  uint32_t signs;        // RHT: bit i set = sign -1 on element i of a block
+  int sr;
+  uint64_t seed;
+  uint32_t stream;
+  int block2d;
+  int tiled;
+  const float* global_in;
+  const double* partials;
+  int np;
+  uint8_t* codes;
+  uint8_t* sf;
+  float* global_out;
+};
+
+__device__ __forceinline__ double load_in(const QxParams& p, int64_t r, int64_t c) {
+  if (p.bf16) return static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(p.in)[r * p.cols + c]));
+  return static_cast<double>(static_cast<const float*>(p.in)[r * p.cols + c]);
+}
+
+// The 16 values of output row ro, block j (transformed when asked).
+__device__ __forceinline__ void load_block(const QxParams& p, int64_t ro, int64_t j, double (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = p.transpose ? load_in(p, j * 16 + i, ro) : load_in(p, ro, j * 16 + i);
+  if (p.rht) {
+    // H16 diag(s) v / 4: signs, then the fast Walsh-Hadamard butterflies
+    // (Sylvester order), then the exact division by 4
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if ((p.signs >> i) & 1u) v[i] = -v[i];
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if ((i & h) == 0) {
+          const double a = v[i], b = v[i + h];
+          v[i] = a + b;
+          v[i + h] = a - b;
+        }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] *= 0.25;
+  }
+}
+
+__device__ __forceinline__ int64_t out_rows(const QxParams& p) { return p.transpose ? p.cols : p.rows; }
+__device__ __forceinline__ int64_t out_cols(const QxParams& p) { return p.transpose ? p.rows : p.cols; }
+
+// Pass 1: per-CTA maxima of |out| (fp64, exact).
+__global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p, double* __restrict__ partials) {
+  pdl_begin();
+  __shared__ double red[kXThreads / 32];
+  const int64_t nb = out_cols(p) / 16, total = out_rows(p) * nb;
+  double m = 0.0;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    // transposed input: consecutive threads take consecutive output rows
+    // (consecutive input columns) of one block column, so loads coalesce
+    const int64_t ro = p.transpose ? b % out_rows(p) : b / nb;
+    const int64_t j = p.transpose ? b / out_rows(p) : b % nb;
+    double v[16];
+    load_block(p, ro, j, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmax(m, fabs(v[i]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double r = 0.0;
+    for (int i = 0; i < kXThreads / 32; ++i) r = fmax(r, red[i]);
+    partials[blockIdx.x] = r;
+  }
+}
+
+// E2M1 grid magnitudes by code.
+__device__ __forceinline__ double e2m1_mag(int c) {
+  constexpr double g[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  return g[c];
+}
+
+// Stochastic E2M1 code of v (fp32 value): |v| >= 6 -> 6; else, between grid
+// neighbours lo <= |v| < hi, hi when u * (hi - lo) < |v| - lo (exact
+// comparison), else lo; the sign bit is the sign of v.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, float u) {
+  const double a = fabs(static_cast<double>(v));
+  int lo = 0;
+#pragma unroll
+  for (int c = 1; c < 8; ++c)
+    if (a >= e2m1_mag(c)) lo = c;
+  int code = lo;
+  if (a >= 6.0) {
+    code = 7;
+  } else {
+    const double l = e2m1_mag(lo), h = e2m1_mag(lo + 1);
+    if (static_cast<double>(u) * (h - l) < a - l) code = lo + 1;
+  }
+  return static_cast<uint32_t>(code) | (signbit(v) ? 8u : 0u);
+}
+
+__device__ __forceinline__ int64_t tiled_off(int64_t row, int64_t j, int64_t groups64) {
+  return ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
+}
+
+// Pass 2: a thread per 16 output rows x one 16-column block.
+__global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p) {
+  pdl_begin();
+  __shared__ double red[kXThreads / 32];
+  __shared__ float s_gs;
+  // global scale: s_g = fp32(amax / 2688) from the fp64 amax (1 when 0)
+  if (p.global_in) {
+    if (threadIdx.x == 0) s_gs = __ldg(p.global_in);
+  } else {
+    double m = 0.0;
+    for (int i = threadIdx.x; i < p.np; i += blockDim.x) m = fmax(m, p.partials[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double r = 0.0;
+      for (int i = 0; i < kXThreads / 32; ++i) r = fmax(r, red[i]);
+      s_gs = r == 0.0 ? 1.0f : __double2float_rn(r / 2688.0);
+    }
+  }
+  __syncthreads();
+  const float s_g = s_gs;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.global_out) *p.global_out = s_g;
+  const float t = __fmul_rn(s_g, 6.0f);
+  const int64_t R = out_rows(p), C = out_cols(p), nb = C / 16;
+  const int64_t groups64 = (C + 63) / 64;
+  const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;   // 16-row groups, tiled padding
+  const int64_t nb_cov = p.tiled ? groups64 * 4 : nb;
+  const int64_t total = rg_cov * nb_cov;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t g = p.transpose ? b % rg_cov : b / nb_cov;
+    const int64_t j = p.transpose ? b / rg_cov : b % nb_cov;
+    const int64_t r0 = g * 16;
+    uint32_t code2d = 0;
+    if (p.block2d && j < nb && r0 < R) {   // one scale from the amax of the 16 x 16 block
+      double m = 0.0;
+      for (int i = 0; i < 16 && r0 + i < R; ++i) {
+        double v[16];
+        load_block(p, r0 + i, j, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
+      }
+      code2d = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
+    }
+    for (int i = 0; i < 16; ++i) {
+      const int64_t ro = r0 + i;
+      uint32_t scode = 0;
+      if (ro < R && j < nb) {
+        double v[16];
+        load_block(p, ro, j, v);
+        if (p.block2d) {
+          scode = code2d;
+        } else {
+          double m = 0.0;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
+          scode = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
+        }
+        const double dec = e4m3_exact(scode);
+        uint32_t lo = 0, hi = 0;
+        if (dec != 0.0) {
+          const float sc = __fmul_rn(static_cast<float>(dec), s_g);
+          float q[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(v[e] / static_cast<double>(sc));
+          if (p.sr) {
+            float u[16];
+            sr_uniforms16(static_cast<uint64_t>(ro) * C + j * 16, p.seed, p.stream, u);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const uint32_t c = e2m1_sr(q[e], u[e]);
+              if (e < 8) lo |= c << (4 * e);
+              else hi |= c << (4 * (e - 8));
+            }
+          } else {   // round to nearest even (hardware conversion, element 2k in the low nibble)
+            lo = cvt_e2m1_x8(q);
+            hi = cvt_e2m1_x8(q + 8);
+          }
+        }
+        *reinterpret_cast<uint2*>(p.codes + ro * (C / 2) + j * 8) = make_uint2(lo, hi);
+      }
+      if (p.tiled) {
+        if (ro < ((R + 127) / 128) * 128) p.sf[tiled_off(ro, j, groups64)] = static_cast<uint8_t>(scode);
+      } else if (ro < R && j < nb) {
+        p.sf[ro * nb + j] = static_cast<uint8_t>(scode);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+int nvfp4x_partials(int64_t blocks) {
+  const int64_t want = (blocks + 4 * kXThreads - 1) / (4 * kXThreads);
+  return static_cast<int>(want < 1 ? 1 : (want > 1184 ? 1184 : want));
+}
+
+lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
+                                     uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
+                                     uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
+                                     cudaStream_t s) {
+  QxParams p = {};
+  p.in = in;
+  p.bf16 = in_dtype == LMOE_BF16;
+  p.rows = rows;
+  p.cols = cols;
+  p.transpose = (flags & LMOE_QX_TRANSPOSE) != 0;
+  p.rht = (flags & LMOE_QX_RHT) != 0;
+  p.signs = rht_signs & 0xFFFFu;
+  p.sr = (flags & LMOE_QX_SR) != 0;
+  p.seed = seed;
+  p.stream = sr_stream;
+  p.block2d = (sf_layout & LMOE_SF_BLOCK_16X16) != 0;
+  p.tiled = (sf_layout & ~LMOE_SF_BLOCK_16X16) == LMOE_SF_MMA_TILED;
+  p.global_in = global_in;
+  p.codes = codes;
+  p.sf = sf;
+  p.global_out = global_out;
+  const int64_t R = p.transpose ? cols : rows, C = p.transpose ? rows : cols;
+  if (R == 0) return LMOE_OK;
+  const int sms = device_sm_count();
+  const int np = nvfp4x_partials(R * (C / 16));
+  if (!global_in) {
+    launch_k(qx_amax_kernel, dim3(np), dim3(kXThreads), 0, s, p, partials);
+    count_launch();
+  }
+  p.partials = partials;
+  p.np = global_in ? 0 : np;
+  const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;
+  const int64_t nb_cov = p.tiled ? (C + 63) / 64 * 4 : C / 16;
+  int64_t blocks = (rg_cov * nb_cov + kXThreads - 1) / kXThreads;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  if (blocks < 1) blocks = 1;
+  launch_k(qx_encode_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kXThreads), 0, s, p);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+}  // namespace lmoe

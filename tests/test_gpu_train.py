@@ -1,0 +1,167 @@
+"""The NVFP4 training recipe's pieces on the GPU (row f4), through the C ABI,
+against the backward oracle (oracle/lmoe_backward.py):
+
+* lmoe_nvfp4_quantize_ex bit-exact: stochastic rounding with Philox-4x32-10
+  uniforms drawn on the device at the oracle's counters, the 16-point random
+  Hadamard transform along the tokens with a transposed output, round to
+  nearest, and 16 x 16 blocks of a transposed weight;
+* dgrad and wgrad of one linear layer under the recipe (quantiser + the
+  block-scaled tcgen05 GEMM) against nvfp4_linear_backward;
+* the routed experts' weight and input gradients of a small layer against
+  backward_nvfp4.
+"""
+import numpy as np
+import pytest
+import torch
+
+import lmoe_inputs as LI
+from oracle import lmoe_backward as B
+from oracle import lmoe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+L = pytest.importorskip("latentmoe_fwd_b200")
+from gpu_util import to_dev  # noqa: E402
+
+SIGNS = np.array([1, -1, -1, 1, 1, 1, -1, 1, -1, 1, 1, -1, -1, -1, 1, 1], dtype=np.float64)
+SIGN_BITS = int(sum(1 << i for i in range(16) if SIGNS[i] < 0))
+
+
+def _quantize_ex(x_bits, rows, cols, flags, seed=0, stream=0, layout=L.SF_ROWMAJOR):
+    tr = bool(flags & L.QX_TRANSPOSE)
+    R, C = (cols, rows) if tr else (rows, cols)
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.zeros((R, C // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    L.nvfp4_quantize_ex(to_dev(x_bits, "bf16"), L.BF16, rows, cols, flags, SIGN_BITS, seed, stream, None, codes, sf,
+                        g, layout)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), sf.cpu().numpy(), float(g.item())
+
+
+def _data(rows, cols, seed):
+    rng = np.random.default_rng(seed)
+    v = rng.standard_normal((rows, cols)) * np.exp(rng.uniform(-3, 3, size=(rows, 1)))
+    return LI.bf16_bits(v)
+
+
+@pytest.mark.parametrize("rows,cols", [(16, 16), (48, 160), (256, 512)])
+def test_stochastic_rounding_bit_exact(rows, cols):
+    bits = _data(rows, cols, rows + cols)
+    X = O.from_bf16_bits(bits)
+    seed, stream = 0x1234_5678_9ABC, 7
+    codes, sf, g = _quantize_ex(bits, rows, cols, L.QX_SR, seed, stream)
+    u = B.sr_uniforms(rows * cols, seed, stream).reshape(rows, cols)
+    rc, rsf, rg = B.nvfp4_quantize_sr(X, u)
+    assert g == np.float32(rg)
+    assert np.array_equal(sf, rsf)
+    assert np.array_equal(codes, rc)
+    # and it differs from round-to-nearest somewhere (the uniforms matter)
+    nc, _, _ = O.nvfp4_quantize(X)
+    assert not np.array_equal(codes, nc)
+
+
+@pytest.mark.parametrize("sr", [False, True])
+def test_rht_along_tokens_transposed_bit_exact(sr):
+    T, n = 64, 96                                     # tokens x features (a wgrad operand)
+    bits = _data(T, n, 11)
+    X = O.from_bf16_bits(bits)
+    flags = L.QX_TRANSPOSE | L.QX_RHT | (L.QX_SR if sr else 0)
+    codes, sf, g = _quantize_ex(bits, T, n, flags, seed=99, stream=3)
+    Xt = B.rht(X, SIGNS, axis=0).T                    # [n, T]: transformed along the tokens
+    if sr:
+        u = B.sr_uniforms(n * T, 99, 3).reshape(n, T)
+        rc, rsf, rg = B.nvfp4_quantize_sr(Xt, u)
+    else:
+        rc, rsf, rg = O.nvfp4_quantize(Xt)
+    assert g == np.float32(rg)
+    assert np.array_equal(sf, rsf)
+    assert np.array_equal(codes, rc)
+
+
+def test_transposed_weight_2d_blocks_bit_exact():
+    W = _data(80, 128, 5)                             # [n_out, n_in]; dgrad reads W^T [n_in, n_out]
+    codes, sf, g = _quantize_ex(W, 80, 128, L.QX_TRANSPOSE, layout=L.SF_ROWMAJOR | L.SF_BLOCK_16X16)
+    rc, rsf, rg = O.nvfp4_quantize_2d(O.from_bf16_bits(W).T)
+    assert g == np.float32(rg)
+    assert np.array_equal(sf, rsf) and np.array_equal(codes, rc)
+    # 16 x 16 blocks quantise W and W^T alike
+    wc, wsf, _ = O.nvfp4_quantize_2d(O.from_bf16_bits(W))
+    assert np.array_equal(O.nvfp4_dequantize(rc, rsf, rg), O.nvfp4_dequantize(wc, wsf, rg).T)
+
+
+def test_plain_mode_equals_nvfp4_quantize():
+    bits = _data(130, 64, 2)
+    codes, sf, g = _quantize_ex(bits, 130, 64, 0)
+    rc, rsf, rg = O.nvfp4_quantize(O.from_bf16_bits(bits))
+    assert g == np.float32(rg) and np.array_equal(sf, rsf) and np.array_equal(codes, rc)
+
+
+def test_stochastic_rounding_of_midpoint_values():
+    """Values that land half way between two E2M1 grid points after scaling
+    round up exactly when u < 1/2, so these codes follow the top bit of each
+    Philox word: the device's draws match the oracle's generator word for word."""
+    rows, cols = 4, 64
+    v = np.full((rows, cols), 0.75)                   # amax 0.75 -> s_g, scale: v / sc between 0.5 and 1
+    v[:, 0] = 6.0 * 0.75 / 0.75                       # give each block an amax that maps to 6 exactly
+    bits = LI.bf16_bits(v)
+    X = O.from_bf16_bits(bits)
+    codes, sf, g = _quantize_ex(bits, rows, cols, L.QX_SR, seed=42, stream=1)
+    u = B.sr_uniforms(rows * cols, 42, 1).reshape(rows, cols)
+    rc, rsf, rg = B.nvfp4_quantize_sr(X, u)
+    assert np.array_equal(codes, rc) and np.array_equal(sf, rsf)
+
+
+def _q_dev(x_dev, rows, cols, flags, seed=0, stream=0, block2d=False):
+    """lmoe_nvfp4_quantize_ex into MMA-tiled scales (the GEMM's operand layout)."""
+    tr = bool(flags & L.QX_TRANSPOSE)
+    R, C = (cols, rows) if tr else (rows, cols)
+    codes = torch.empty((R, C // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.zeros((((R + 127) // 128) * 128 * ((C + 63) // 64) * 4,), dtype=torch.uint8, device="cuda")
+    g = torch.empty(1, dtype=torch.float32, device="cuda")
+    layout = L.SF_MMA_TILED | (L.SF_BLOCK_16X16 if block2d else 0)
+    L.nvfp4_quantize_ex(x_dev, L.BF16, rows, cols, flags, SIGN_BITS, seed, stream, None, codes, sf, g, layout)
+    return codes, sf, g
+
+
+def _gemm_dev(a, a_rows, b, cols, k):
+    """Plain (one-group) block-scaled GEMM: BF16 [a_rows][cols] = A . B^T."""
+    out = torch.empty((a_rows, cols), dtype=torch.bfloat16, device="cuda")
+    offs = torch.tensor([0, a_rows], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    L.nvfp4_gemm(1, offs, offs, a_rows, a[0], a[1], a[2], 0, b[0], b[1], b[2], cols, k, None, out, cols, ws)
+    st, info = L.read_device_error(ws)
+    assert st == L.OK, (L.status_string(st), hex(info))
+    return out.float().cpu().numpy().astype(np.float64)
+
+
+def test_linear_layer_dgrad_and_wgrad_match_the_oracle():
+    """dX = Q_sr(dY) Q_2d(W) and dW = Q_sr(RHT(dY)^T) Q_rn(RHT(X)^T)^T on the GPU
+    (quantiser + block-scaled tcgen05 GEMM) against nvfp4_linear_backward."""
+    from gpu_util import bf16_parity
+    T, n_in, n_out = 256, 256, 512
+    rng = np.random.default_rng(8)
+    Xb = LI.bf16_bits(rng.standard_normal((T, n_in)))
+    Wb = LI.bf16_bits(rng.standard_normal((n_out, n_in)) / np.sqrt(n_in))
+    dYb = LI.bf16_bits(rng.standard_normal((T, n_out)) * 0.01)
+    X, W, dY = (O.from_bf16_bits(b) for b in (Xb, Wb, dYb))
+    seed, s_dgrad, s_wgrad = 2026, 10, 11
+    x, w, dy = (to_dev(b, "bf16") for b in (Xb, Wb, dYb))
+    # dgrad: contraction over n_out
+    a = _q_dev(dy, T, n_out, L.QX_SR, seed, s_dgrad)
+    b = _q_dev(w, n_out, n_in, L.QX_TRANSPOSE, block2d=True)          # W^T [n_in][n_out], 16 x 16 blocks
+    dX = _gemm_dev(a, T, b, n_in, n_out)
+    # wgrad: contraction over the tokens, both operands transformed along them
+    a = _q_dev(dy, T, n_out, L.QX_TRANSPOSE | L.QX_RHT | L.QX_SR, seed, s_wgrad)
+    b = _q_dev(x, T, n_in, L.QX_TRANSPOSE | L.QX_RHT)
+    dW = _gemm_dev(a, n_out, b, n_in, T)
+    ref = B.nvfp4_linear_backward(X, W, dY, SIGNS, B.sr_uniforms(T * n_out, seed, s_dgrad).reshape(T, n_out),
+                                  B.sr_uniforms(n_out * T, seed, s_wgrad).reshape(n_out, T))
+    for name, got, exact in (("dX", dX, ref["dX"]), ("dW", dW, ref["dW"])):
+        excess, raw = bf16_parity(got, exact, O.round_bf16(exact))
+        print(f"linear backward {name}: excess {excess:.3e} * RMS, raw {raw:.3e} * RMS")
+        assert excess <= 2e-2, name
+    # the quantised gradients differ from the exact ones (the recipe's rounding is visible)
+    exact = B.nvfp4_linear_backward(X, W, dY, SIGNS, None, None, quantize=False)
+    rel = np.sqrt(np.mean((dW - exact["dW"]) ** 2) / np.mean(exact["dW"] ** 2))
+    assert 1e-3 < rel < 0.5
