@@ -416,6 +416,45 @@ lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* p
                             const float* b_global, int cols, int64_t k, const float* row_scale, void* out,
                             int64_t ld_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Expert parallelism in the latent dimension (greeksharifa page on the
+ * Nemotron 3 whitepaper, section 2.2 "LatentMoE": the rows that cross GPUs
+ * between the projections are l-dim, so the all-to-all volume falls by d/l).
+ * G ranks each route and permute their own tokens; rank h owns the experts
+ * [first(h), first(h) + n(h)), n(h) = N/G (one more for the first N%G ranks).
+ *
+ * lmoe_ep_plan (HOST arrays, no device work): from counts [G][N] (counts[g][e]
+ * = slots rank g routes to expert e, known to every rank after a count
+ * exchange) computes, for `rank`:
+ *  send_counts/send_offsets [G]: the rows of this rank's sorted (expert-major)
+ *    permuted buffer that go to each rank, one contiguous block per rank;
+ *  recv_counts/recv_offsets [G]: the blocks an all-to-all delivers, in source
+ *    rank order (each sorted by expert);
+ *  first_expert, local_experts (NL); local_offsets/local_padded_offsets
+ *    [NL+1]: the expert-grouped layout of the received rows (sources in rank
+ *    order inside an expert; each expert's range padded to a multiple of 128,
+ *    as the expert GEMMs read it);
+ *  block_src/block_dst/block_rows [G*NL] (source-major, block (g, el) at
+ *    g*NL + el): where each (source, local expert) block sits in the received
+ *    buffer and where it goes in the expert-grouped buffer.
+ * Errors: LMOE_ERR_INVALID_ARG for null pointers, G, rank or N out of range,
+ * negative counts; LMOE_ERR_UNSUPPORTED for N > 1024, G > N or more than
+ * 2^31 rows. */
+lmoe_status lmoe_ep_plan(int G, int rank, int N, const int32_t* counts, int32_t* send_counts,
+                         int32_t* send_offsets, int32_t* recv_counts, int32_t* recv_offsets, int32_t* first_expert,
+                         int32_t* local_experts, int32_t* local_offsets, int32_t* local_padded_offsets,
+                         int32_t* block_src, int32_t* block_dst, int32_t* block_rows);
+
+/* Row-block copy between the all-to-all's source-major order and the
+ * expert-grouped padded order (either direction: swap src_rows and dst_rows):
+ * block b moves its rows from row src_rows[b] of `in` to row dst_rows[b] of
+ * `out`; row_prefix [nblocks] (DEVICE, int64) is the inclusive prefix of the
+ * blocks' row counts and total_rows its last value. in, out, src_rows,
+ * dst_rows, row_prefix are device pointers; rows are row_bytes each (a
+ * multiple of 16, 16-byte aligned). Asynchronous on `stream`.
+ * Errors: LMOE_ERR_INVALID_ARG for null or unaligned buffers, bad sizes. */
+lmoe_status lmoe_ep_reorder(const void* in, void* out, int64_t row_bytes, int nblocks, const int32_t* src_rows,
+                            const int32_t* dst_rows, const int64_t* row_prefix, int64_t total_rows, void* stream);
+
 /* Synchronises `stream`, returns the device error status recorded in the
  * workspace `ws` (LMOE_OK if none) and clears it (the read and the clear run
  * on `stream`). `info` (host, may be NULL) receives a kernel-specific detail

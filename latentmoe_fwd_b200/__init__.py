@@ -36,7 +36,8 @@ EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permut
            "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
            "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize",
-           "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_gemm")
+           "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_gemm",
+           "lmoe_ep_plan", "lmoe_ep_reorder")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -87,6 +88,8 @@ def _load():
         "lmoe_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_size_t, ctypes.c_uint64, P]),
         "lmoe_fp8_quantize": (ctypes.c_int, [P, ctypes.c_int, I64, I64, P, P, P, P, ctypes.c_size_t, P]),
         "lmoe_nvfp4_quantize_ex_workspace": (ctypes.c_size_t, [I64, I64]),
+        "lmoe_ep_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int] + [P] * 12),
+        "lmoe_ep_reorder": (ctypes.c_int, [P, P, I64, ctypes.c_int, P, P, P, I64, P]),
         "lmoe_nvfp4_gemm": (ctypes.c_int, [ctypes.c_int, P, P, I64, P, P, P, ctypes.c_int, P, P, P, ctypes.c_int,
                                            I64, P, P, I64, P, ctypes.c_size_t, P]),
         "lmoe_nvfp4_quantize_ex": (ctypes.c_int, [P, ctypes.c_int, I64, I64, ctypes.c_uint32, ctypes.c_uint32,
@@ -255,6 +258,36 @@ def nvfp4_gemm(groups, offsets, padded_offsets, a_rows, a_codes, a_sf, a_global,
                                _p(a_global), int(a_global_per_group), _p(b_codes), _p(b_sf), _p(b_global),
                                int(cols), int(k), _p(row_scale), _p(out), int(ld_out), _p(ws), ws.numel(),
                                _stream(stream)), "lmoe_nvfp4_gemm")
+
+
+def ep_plan(G: int, rank: int, counts):
+    """lmoe_ep_plan on host arrays: counts [G][N] int32 (numpy). Returns a dict
+    of numpy int32 arrays (send/recv counts and offsets, the local
+    expert-grouped layout, the (source, local expert) blocks)."""
+    import numpy as np
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    N = counts.shape[1]
+    out = {k: np.zeros(G, dtype=np.int32) for k in ("send_counts", "send_offsets", "recv_counts", "recv_offsets")}
+    fe, nl = ctypes.c_int32(0), ctypes.c_int32(0)
+    lo = np.zeros(N + 1, dtype=np.int32)
+    lpo = np.zeros(N + 1, dtype=np.int32)
+    bs = np.zeros(G * N, dtype=np.int32)
+    bd = np.zeros(G * N, dtype=np.int32)
+    br = np.zeros(G * N, dtype=np.int32)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib.lmoe_ep_plan(G, rank, N, ptr(counts), ptr(out["send_counts"]), ptr(out["send_offsets"]),
+                            ptr(out["recv_counts"]), ptr(out["recv_offsets"]), ctypes.byref(fe), ctypes.byref(nl),
+                            ptr(lo), ptr(lpo), ptr(bs), ptr(bd), ptr(br)), "lmoe_ep_plan")
+    n = nl.value
+    out.update(first_expert=fe.value, local_experts=n, local_offsets=lo[:n + 1], local_padded_offsets=lpo[:n + 1],
+               block_src=bs[:G * n], block_dst=bd[:G * n], block_rows=br[:G * n])
+    return out
+
+
+def ep_reorder(x, out, row_bytes, src_rows, dst_rows, row_prefix, total_rows, stream=None):
+    """lmoe_ep_reorder: copy row blocks (device tensors; row_prefix int64)."""
+    _check(lib.lmoe_ep_reorder(_p(x), _p(out), int(row_bytes), int(src_rows.numel()), _p(src_rows), _p(dst_rows),
+                               _p(row_prefix), int(total_rows), _stream(stream)), "lmoe_ep_reorder")
 
 
 def selftest_wait_timeout(ws, limit_cycles: int, stream=None):
