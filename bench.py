@@ -385,10 +385,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the workload's token count (smaller captures for ncu)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override the workload's expert count (smaller captures for ncu)")
     args = ap.parse_args()
     wl = LI.WORKLOADS[args.workload]
     if args.tokens is not None:
         wl = LI.replace(wl, T=args.tokens)
+    if args.experts is not None:
+        wl = LI.replace(wl, N=args.experts)
     if args.impl == "reference":
         return run_reference(args, wl)
 

@@ -203,6 +203,68 @@ def test_full_size_expert_ffn_every_tile(name):
     assert raw_ok
 
 
+def test_full_size_nvfp4_expert_ffn_every_tile():
+    """lmoe_expert_ffn on the NVFP4 path at full size (ultra_nvfp4): the
+    oracle's routing and its BF16 z quantised on the GPU (the quantiser is
+    bit-exact, so both sides start from the same codes), rows of every
+    128-row tile of every expert against the oracle's expert FFN with its
+    NVFP4 rounding points (z and a fake-quantised, 16-element blocks)."""
+    from test_gpu_nvfp4 import prequantize_experts
+    from gpu_util import quantize_dev
+    name = "ultra_nvfp4"
+    wl, inp, _, ridx, rgates = _oracle_routing(name)
+    T, K, N, l, m = wl.T, wl.K, wl.N, wl.l, wl.m
+    x = O.from_bf16_bits(inp["x"])
+    z = O.round_bf16(x @ O.from_bf16_bits(inp["w_down"]).T)          # the oracle's stored z
+    dev = DevLayer(wl, inp)
+    cfg = dev.cfg
+    P = L.padded_rows(cfg)
+    zq, zsf, zgs = quantize_dev(to_dev(LI.bf16_bits(z), "bf16"), T, l)
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device="cuda")
+    offsets, poff, perm_src, inv_perm = i32(N + 1), i32(N + 1), i32(T * K), i32(T * K)
+    zp = torch.zeros((P, l // 2), dtype=torch.uint8, device="cuda")
+    zpsf = torch.zeros((P * l // 16,), dtype=torch.uint8, device="cuda")
+    pg = torch.zeros(P, dtype=torch.float32, device="cuda")
+    ws = L.workspace(cfg, L.OP_PERMUTE)
+    L.permute(cfg, torch.from_numpy(ridx.astype(np.int32)).cuda(), offsets, perm_src, inv_perm, poff, zq, l // 2,
+              zp, rows_sf=zsf, permuted_sf=zpsf, topk_w=torch.from_numpy(rgates.astype(np.float32)).cuda(),
+              perm_gate=pg, ws=ws)
+    assert L.read_device_error(ws)[0] == L.OK
+    y = torch.empty((P, l), dtype=torch.bfloat16, device="cuda")
+    ws2 = L.workspace(cfg, L.OP_EXPERT_FFN)
+    L.expert_ffn(cfg, dev.w, zp, zpsf, zgs, offsets, poff, pg, y, ws2)
+    assert L.read_device_error(ws2)[0] == L.OK
+    poff_h = poff.cpu().numpy()
+
+    counts, r_off, r_src, _ = O.permute(ridx, N)
+    pos = _expert_rows(counts, tile=128)
+    W = O.weights_view(wl, inp, cache=True)
+    prequantize_experts(W, np.nonzero(counts)[0])
+    s_z = float(zgs.item())
+    assert s_z == np.float32(O.nvfp4_global_scale(z))
+    a_gs = inp["a_global_scale"]
+    g32 = rgates.astype(np.float32).astype(np.float64)
+    by_e = {}
+    for e, p in pos:
+        by_e.setdefault(e, []).append(p)
+    got_rows, ref_rows, ref_exact = [], [], []
+    for e, ps in by_e.items():
+        ps = np.array(ps)
+        slots = r_src[r_off[e] + ps]
+        t, k = slots // K, slots % K
+        zq_rows = O.nvfp4_fake_quant(z[t], s_z)[0]
+        aq = O.nvfp4_fake_quant(O.sq_relu(zq_rows @ W.expert("w1", e).T), a_gs)[0]
+        yx = g32[t, k][:, None] * (aq @ W.expert("w2", e).T)
+        ref_exact.append(yx)
+        ref_rows.append(O.round_bf16(yx))
+        got_rows.append(poff_h[e] + ps)
+    got = as_f64(y[torch.from_numpy(np.concatenate(got_rows)).cuda()])
+    excess, raw = bf16_parity(got, np.concatenate(ref_exact), np.concatenate(ref_rows))
+    print(f"{name}: {len(pos)} expert-FFN rows from every 128-row tile: excess {excess:.3e} * RMS, "
+          f"raw {raw:.3e} * RMS")
+    assert excess <= 8e-2
+
+
 @pytest.mark.parametrize("name", ["ultra_nvfp4", "ultra_decode_nvfp4", "ultra_nvfp4_fp8shared"])
 def test_full_size_nvfp4(name):
     """NVFP4 workloads at full size (the T=8192 layer, the same layer in

@@ -170,10 +170,10 @@ def nvfp4_token_errors(wl, inp, out, gidx, toks, tol):
     bad = np.where(err > tol)[0]
     n_var = 0
     if bad.size:
-        zx = nvfp4_ties.z_exact(inp, toks[bad])
+        zx, tnorm = nvfp4_ties.z_exact(inp, toks[bad])
         pairs, rows = [], []
         for i, b in enumerate(bad):
-            zr, ties = nvfp4_ties.code_changing_ties(zx[i], ref["z_global_scale"])
+            zr, ties = nvfp4_ties.code_changing_ties(zx[i], ref["z_global_scale"], tnorm[i])
             for row in nvfp4_ties.variant_rows(zr, ties):
                 pairs.append(b)
                 rows.append(row)
@@ -184,6 +184,10 @@ def nvfp4_token_errors(wl, inp, out, gidx, toks, tol):
             for b, e in zip(pairs, e_alt):
                 err[b] = min(err[b], e)
             n_var = len(rows)
+        still = [int(b) for b in bad if err[b] > tol]
+        if still:
+            print(f"{wl.name}: tokens over {tol} after the z-rounding variants: "
+                  f"{[(int(toks[b]), round(float(err[b]), 4)) for b in still[:8]]}")
     return err, bad.size, n_var
 
 
