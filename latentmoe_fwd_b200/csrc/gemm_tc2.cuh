@@ -92,10 +92,11 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
 }
 
 struct Tc2Smem {
-  static constexpr int kABytes = 128 * 128;   // 128 weight rows x 64 bf16
+  static constexpr int kABytes = 128 * 128;   // 128 weight rows x 64 bf16 (one K atom)
   static constexpr int kBBytes = 128 * 128;   // up to 128 token rows x 64 bf16
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = 6;
+  static constexpr int kAtoms = 1;            // 64-wide K atoms per stage
+  static constexpr int kStageBytes = kAtoms * (kABytes + kBBytes);   // A atoms, then B atoms
+  static constexpr int kStages = 6 / kAtoms;
   static constexpr int kBarOffset = kStages * kStageBytes;
   // full[S], empty[S], tfull[2], tempty[2], drain, tmem ptr, abort
   static constexpr int kPrefixOffset = kBarOffset + (2 * kStages + 5) * 8 + 16;
@@ -276,23 +277,26 @@ __global__ void __launch_bounds__(192, 1)
                      : ti.act0 + S::kTokens < __ldg(p.padded_offsets + ti.expert) +
                                                   (__ldg(p.offsets + ti.expert + 1) - __ldg(p.offsets + ti.expert));
         const uint64_t pa = wshared ? pol_keep : pol_stream;
-        for (int kb = 0; kb < ti.kblocks; ++kb) {
+        for (int kb = 0; kb < ti.kblocks; kb += S::kAtoms) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x2100 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStageBytes;
-          uint8_t* sb = sa + S::kABytes;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::kABytes + ti.n * 128);
+          uint8_t* sb = sa + S::kAtoms * S::kABytes;
+          const int na = min(S::kAtoms, ti.kblocks - kb);   // K atoms in this stage
+          if (leader) mbar_arrive_expect_tx(&full[stage], na * (2 * S::kABytes + ti.n * 128));
           const uint32_t bar = cluster_map(smem_u32(&full[stage]), 0);
-          const int k = kb * 64;
           const int kg = ti.extra ? p.kgroup_x : 0;   // K split over the weight tensor's groups
-          tma_load_3d_pair(sa, amap, bar, kg ? k % kg : k, ti.w0 + static_cast<int>(rank) * 128,
-                           kg ? k / kg : ti.expert, pa);
-          int done = 0;
+          for (int q = 0; q < na; ++q) {
+            const int k = (kb + q) * 64;
+            tma_load_3d_pair(sa + q * S::kABytes, amap, bar, kg ? k % kg : k, ti.w0 + static_cast<int>(rank) * 128,
+                             kg ? k / kg : ti.expert, pa);
+            int done = 0;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int box = 128 >> i;
-            if (half - done >= box) {
-              tma_load_3d_pair(sb + done * 128, bmap0 + i, bar, k, b_row0 + done, 0, pol_norm);
-              done += box;
+            for (int i = 0; i < 4; ++i) {
+              const int box = 128 >> i;
+              if (half - done >= box) {
+                tma_load_3d_pair(sb + q * S::kBBytes + done * 128, bmap0 + i, bar, k, b_row0 + done, 0, pol_norm);
+                done += box;
+              }
             }
           }
           issued = true;
@@ -321,15 +325,17 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
         const uint32_t idesc = idesc_bf16_f32(256, ti.n);
-        for (int kb = 0; kb < ti.kblocks; ++kb) {
+        for (int kb = 0; kb < ti.kblocks; kb += S::kAtoms) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x2300 + stage)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
-          const uint32_t sb = sa + S::kABytes;
+          const uint32_t sb = sa + S::kAtoms * S::kABytes;
+          const int na = min(S::kAtoms, ti.kblocks - kb);
+          for (int q = 0; q < na; ++q)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(sa + kk * 32), sdesc_kmajor_sw128(sb + kk * 32), idesc,
-                          (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(sa + q * S::kABytes + kk * 32),
+                            sdesc_kmajor_sw128(sb + q * S::kBBytes + kk * 32), idesc, (kb | q | kk) != 0 ? 1u : 0u);
           any = true;
           mma_commit_pair(&empty[stage], 0x3);
           if (++stage == S::kStages) { stage = 0; phase ^= 1; }

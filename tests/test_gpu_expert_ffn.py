@@ -76,9 +76,16 @@ def _check(wl, tol):
     assert excess <= tol
 
 
-@pytest.mark.parametrize("T", [130, 700])
+@pytest.mark.parametrize("T", [130, 700, 2100])
 def test_expert_ffn_nvfp4(T):
+    # T = 130: single-CTA token-major tiles; 700, 2100: CTA-pair weight-major
+    # tiles (2100: several 256-token tiles per expert and a ragged last one)
     _check(LI.reduced("ultra_nvfp4", T=T, d=512, l=256, N=16, K=4, m=512), 8e-2)
+
+
+def test_expert_ffn_nvfp4_pair_tiles_skewed():
+    # Zipf-biased routing on the NVFP4 path: experts with many 256-token tiles next to one-row experts
+    _check(LI.replace(LI.reduced("ultra_nvfp4", T=1500, d=512, l=256, N=16, K=4, m=512), zipf_bias=True), 8e-2)
 
 
 @pytest.mark.parametrize("T", [20, 300])

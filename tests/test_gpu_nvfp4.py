@@ -225,7 +225,7 @@ def test_nvfp4_weights_quantised_bit_exact_per_expert():
         assert gs[e] == np.float32(rg)
 
 
-@pytest.mark.parametrize("T", [130, 700, 1000])
+@pytest.mark.parametrize("T", [130, 700, 1000, 2100])
 def test_nvfp4_forward_reduced(T):
     wl = LI.reduced("ultra_nvfp4", T=T, d=512, l=256, N=16, K=4, m=512)
     _nvfp4_layer(wl)
