@@ -3,7 +3,7 @@
 //
 //   D[w, t] = sum_k (q_w[w,k] s_w[w,k/16]) (q_a[t,k] s_a[t,k/16])
 //     w: 256 output features of expert e (128 per CTA of the pair)
-//     t: up to 256 of the expert's tokens (the MMA's N, rounded up to 32)
+//     t: up to 256 of the expert's tokens (the MMA's N, rounded up to 64)
 //
 // Each CTA loads its 128 weight rows and their scales, its half of the token
 // rows, and the scales of all N tokens (the pair's MMA reads B's scales in
@@ -80,20 +80,11 @@ struct Fp4pMaps {
 };
 
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
-                                                 int c1) {
+                                                 int c1, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d_pair_nohint(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
-                                                        int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
       : "memory");
 }
 
@@ -120,7 +111,7 @@ struct Tile4p {
   int act0;    // first padded token row of the tile
   int act_n;   // tokens in the tile
   int w0;      // first feature of the pair's 256
-  int n;       // MMA N: act_n rounded up to 32
+  int n;       // MMA N: act_n rounded up to 64
 };
 
 // Pair tile t: expert e, token tile tt (256 tokens), weight tile of 256
@@ -142,7 +133,9 @@ __device__ __forceinline__ Tile4p fp4p_tile(const Fp4pParams& p, int t, const in
   ti.act0 = __ldg(p.padded_offsets + e) + tt * Fp4pSmem::kTokens;
   ti.act_n = min(Fp4pSmem::kTokens, n_e - tt * Fp4pSmem::kTokens);
   ti.valid = ti.act_n > 0;
-  ti.n = (ti.act_n + 31) & ~31;
+  // block-scaled MMA widths step in 64 columns (the token scales sit in 128-row
+  // atoms, read 64 columns at a time): N in {64, 128, 192, 256}
+  ti.n = (ti.act_n + 63) & ~63;
   return ti;
 }
 
@@ -225,6 +218,7 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs) ----------------
+      const uint64_t pol = policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, issued = false;
@@ -246,20 +240,20 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           uint8_t* ssfb = ssfa + S::kSFA;
           if (leader) mbar_arrive_expect_tx(&full[stage], stage_bytes);
           const uint32_t bar = cluster_map(smem_u32(&full[stage]), 0);
-          tma_load_3d_pair_nohint(sa, &maps.m[0], bar, kb * 128, ti.w0 + static_cast<int>(rank) * 128, ti.expert);
+          tma_load_3d_pair(sa, &maps.m[0], bar, kb * 128, ti.w0 + static_cast<int>(rank) * 128, ti.expert, pol);
           int done = 0;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 3; ++i) {   // half is 32, 64, 96 or 128 rows
             const int box = 128 >> i;
             if (half - done >= box) {
-              tma_load_3d_pair_nohint(sb + done * 128, &maps.m[1 + i], bar, kb * 128, b_row0 + done, 0);
+              tma_load_3d_pair(sb + done * 128, &maps.m[1 + i], bar, kb * 128, b_row0 + done, 0, pol);
               done += box;
             }
           }
           // scale atoms (4 per row block and K block) as 8 rows of 256 bytes
-          tma_load_3d_pair_nohint(ssfa, &maps.m[5], bar, 0, (rb_w * p.groups64 + kb * 4) * 2, ti.expert);
-          tma_load_2d_pair(ssfb, &maps.m[6], bar, 0, (rb_t * p.groups64 + kb * 4) * 2);
-          if (two_rb) tma_load_2d_pair(ssfb + 2048, &maps.m[6], bar, 0, ((rb_t + 1) * p.groups64 + kb * 4) * 2);
+          tma_load_3d_pair(ssfa, &maps.m[5], bar, 0, (rb_w * p.groups64 + kb * 4) * 2, ti.expert, pol);
+          tma_load_2d_pair(ssfb, &maps.m[6], bar, 0, (rb_t * p.groups64 + kb * 4) * 2, pol);
+          if (two_rb) tma_load_2d_pair(ssfb + 2048, &maps.m[6], bar, 0, ((rb_t + 1) * p.groups64 + kb * 4) * 2, pol);
           issued = true;
           if (++stage == S::kStages) { stage = 0; phase ^= 1; }
         }

@@ -97,7 +97,10 @@ struct TcSmem {
   static constexpr int kMaxGroups = 1024;
   // weight-major epilogue: one 32 x 32 BF16 transpose tile per epilogue warp
   static constexpr int kEpiOffset = (kPrefixOffset + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
-  static constexpr int kBytes = kEpiOffset + 4 * 32 * 32 * 2 + 1024;  // +1024 alignment slack
+  // per epilogue warp: a 32 x 32 BF16 transpose tile, or a staged 32-row x 64-byte chunk at an
+  // 80-byte row pitch (bank-conflict free) for the scatter epilogue
+  static constexpr int kEpiWarpBytes = 32 * 80;
+  static constexpr int kBytes = kEpiOffset + 4 * kEpiWarpBytes + 1024;  // +1024 alignment slack
 };
 
 struct TileInfo {
@@ -425,7 +428,41 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + c * 32, v);
         tmem_ld_wait();
-        if (!p.swap) {
+        if (!p.swap && EPI == EPI_SCATTER) {
+          // each token row goes to its K slots' padded rows (the expert-grouped
+          // GEMM input): the warp stages its 32 rows x 32 columns (64 bytes a
+          // row) in shared memory, then writes 64-byte row segments, eight
+          // destinations per store instruction (whole sectors), streamed past L2
+          uint4* st = reinterpret_cast<uint4*>(epi_tile + (warp & 3) * (S::kEpiWarpBytes / 2));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+            u.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+            u.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+            u.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+            st[lane * 5 + j] = u;
+          }
+          __syncwarp();
+          const uint64_t pol = policy_evict_first();
+          const int K = p.scatter_k;
+          const int col0 = ti.w0 + c * 32;
+          const int part = lane & 3;                 // 16 bytes of the 64-byte segment
+          int rr = 0, kk = lane >> 2;                // segment s = rr * K + kk, eight per step
+          while (kk >= K) { kk -= K; ++rr; }
+          const int rows_here = min(32, ti.act_n - q * 32);
+          for (; rr < rows_here;) {
+            const long long tok = ti.act0 + q * 32 + rr;
+            const int pr = __ldg(p.scatter_rows + tok * K + kk);
+            if (pr >= 0 && col0 + part * 8 < p.cols)
+              st_global_v4_hint(reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(pr) * p.ld_out + col0 +
+                                    part * 8,
+                                st[rr * 5 + part], pol);
+            kk += 8;
+            while (kk >= K) { kk -= K; ++rr; }
+          }
+          __syncwarp();
+        } else if (!p.swap) {
           const long long row = ti.act0 + r;
           if (r < ti.act_n) {
             const int col0 = ti.w0 + c * 32;
@@ -449,27 +486,6 @@ __global__ void __launch_bounds__(192, 1)
               uint8_t* o = reinterpret_cast<uint8_t*>(p.out) + row * p.ld_out + col0;
               if (col0 + 16 <= p.cols) *reinterpret_cast<uint4*>(o) = make_uint4(w[0], w[1], w[2], w[3]);
               if (col0 + 32 <= p.cols) *reinterpret_cast<uint4*>(o + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-            } else if (EPI == EPI_SCATTER) {
-              // the token's row goes to each of its K slots' padded rows (the
-              // expert-grouped GEMM input), streamed past L2
-              uint4 u[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                u[j].x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-                u[j].y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-                u[j].z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-                u[j].w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-              }
-              const uint64_t pol = policy_evict_first();
-              const int* dst = p.scatter_rows + row * p.scatter_k;
-              for (int kk = 0; kk < p.scatter_k; ++kk) {
-                const int pr = __ldg(dst + kk);
-                if (pr < 0) continue;
-                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(pr) * p.ld_out + col0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  if (col0 + 8 * j < p.cols) st_global_v4_hint(o + 8 * j, u[j], pol);
-              }
             } else if (EPI == EPI_F32_BIAS) {
               float* o = reinterpret_cast<float*>(p.out) + row * p.ld_out + col0;
 #pragma unroll
@@ -506,7 +522,7 @@ __global__ void __launch_bounds__(192, 1)
           // weight-major, BF16 out: this lane owns output feature w0 + r and 32
           // tokens; transpose the warp's 32 x 32 block through shared memory so
           // each token's 32 features go out as 16-byte stores
-          __nv_bfloat16* tb = epi_tile + (warp & 3) * 32 * 32;
+          __nv_bfloat16* tb = epi_tile + (warp & 3) * (S::kEpiWarpBytes / 2);
           const int col = ti.w0 + r;
           // per-token operands of the chunk are fetched before any store: the
           // gate of token c*32+lane by this lane (one coalesced load, then
