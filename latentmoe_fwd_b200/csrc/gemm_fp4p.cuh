@@ -44,7 +44,9 @@ struct Fp4pSmem {
   static constexpr int kEpiOffset = (kPrefixOffset + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
   static constexpr int kEpiPitch = 33;        // floats per transposed row (bank-conflict free)
   static constexpr int kEpiWarpBytes = 32 * kEpiPitch * 4;
-  static constexpr int kBytes = kEpiOffset + 8 * kEpiWarpBytes + 1024;
+  // per expert: row count and first padded row (read from global memory once)
+  static constexpr int kExpertOffset = kEpiOffset + 8 * kEpiWarpBytes;
+  static constexpr int kBytes = kExpertOffset + 2 * kMaxGroups * 4 + 1024;
   static constexpr int kThreads = 64 + 256;   // producer, MMA, eight epilogue warps
   static constexpr int kAcc1 = 192;           // second accumulator starts here
   static constexpr int kSfaCol = 448;
@@ -79,15 +81,6 @@ struct Fp4pMaps {
   CUtensorMap m[7];
 };
 
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
-                                                 int c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
-      : "memory");
-}
-
 // Scale atom -> tensor memory of both CTAs of the pair (each from its own
 // shared memory at the same offset).
 __device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
@@ -116,7 +109,8 @@ struct Tile4p {
 
 // Pair tile t: expert e, token tile tt (256 tokens), weight tile of 256
 // features; the weight tiles of one token tile are consecutive.
-__device__ __forceinline__ Tile4p fp4p_tile(const Fp4pParams& p, int t, const int* prefix) {
+__device__ __forceinline__ Tile4p fp4p_tile(const Fp4pParams& p, int t, const int* prefix, const int* ecount,
+                                            const int* epoff) {
   Tile4p ti;
   const int ntw = p.cols / 256;
   int lo = 0, hi = p.groups - 1;   // largest e with prefix[e] <= t
@@ -125,12 +119,12 @@ __device__ __forceinline__ Tile4p fp4p_tile(const Fp4pParams& p, int t, const in
     if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
   }
   const int e = lo;
-  const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+  const int n_e = ecount[e];
   const int local = t - prefix[e];
   const int tt = local / ntw, mw = local % ntw;
   ti.expert = e;
   ti.w0 = mw * 256;
-  ti.act0 = __ldg(p.padded_offsets + e) + tt * Fp4pSmem::kTokens;
+  ti.act0 = epoff[e] + tt * Fp4pSmem::kTokens;
   ti.act_n = min(Fp4pSmem::kTokens, n_e - tt * Fp4pSmem::kTokens);
   ti.valid = ti.act_n > 0;
   // block-scaled MMA widths step in 64 columns (the token scales sit in 128-row
@@ -155,6 +149,8 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
   int* prefix = reinterpret_cast<int*>(smem + S::kPrefixOffset);
   float* epi = reinterpret_cast<float*>(smem + S::kEpiOffset);
+  int* ecount = reinterpret_cast<int*>(smem + S::kExpertOffset);
+  int* epoff = ecount + S::kMaxGroups;
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -176,6 +172,8 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
         }
       }
       prefix[e + 1] = ((n_e + S::kTokens - 1) / S::kTokens) * ntw;
+      ecount[e] = n_e;
+      epoff[e] = __ldg(p.padded_offsets + e);
     }
     if (threadIdx.x == 0) prefix[0] = 0;
     __syncthreads();
@@ -223,7 +221,7 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
       uint32_t phase = 0;
       bool ok = true, issued = false;
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
-        const Tile4p ti = fp4p_tile(p, t, prefix);
+        const Tile4p ti = fp4p_tile(p, t, prefix, ecount, epoff);
         if (!ti.valid) continue;
         const int half = ti.n >> 1;
         const int b_row0 = ti.act0 + static_cast<int>(rank) * half;
@@ -252,8 +250,10 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           }
           // scale atoms (4 per row block and K block) as 8 rows of 256 bytes
           tma_load_3d_pair(ssfa, &maps.m[5], bar, 0, (rb_w * p.groups64 + kb * 4) * 2, ti.expert, pol);
-          tma_load_2d_pair(ssfb, &maps.m[6], bar, 0, (rb_t * p.groups64 + kb * 4) * 2, pol);
-          if (two_rb) tma_load_2d_pair(ssfb + 2048, &maps.m[6], bar, 0, ((rb_t + 1) * p.groups64 + kb * 4) * 2, pol);
+          // (every map here is three-dimensional, the token maps with one group)
+          tma_load_3d_pair(ssfb, &maps.m[6], bar, 0, (rb_t * p.groups64 + kb * 4) * 2, 0, pol);
+          if (two_rb)
+            tma_load_3d_pair(ssfb + 2048, &maps.m[6], bar, 0, ((rb_t + 1) * p.groups64 + kb * 4) * 2, 0, pol);
           issued = true;
           if (++stage == S::kStages) { stage = 0; phase ^= 1; }
         }
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
       int local = 0;
       bool ok = true, any = false;
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
-        const Tile4p ti = fp4p_tile(p, t, prefix);
+        const Tile4p ti = fp4p_tile(p, t, prefix, ecount, epoff);
         if (!ti.valid) continue;
         if (local > 0) {
           if (!mbar_wait(overlap_free, (local - 1) & 1, abort_flag, p.err, 0x1600)) { ok = false; break; }
@@ -327,12 +327,21 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
     const uint32_t overlap_bar = cluster_map(smem_u32(overlap_free), 0);
     int local = 0;
     for (int t = cluster; t < ntiles; t += nclusters) {
-      const Tile4p ti = fp4p_tile(p, t, prefix);
+      const Tile4p ti = fp4p_tile(p, t, prefix, ecount, epoff);
       if (!ti.valid) continue;
       const int buf = local & 1;
       const float in_s = p.in_scale_grouped ? __ldg(p.in_scale + ti.expert) : in_s0;
       const float scale = __fmul_rn(in_s, __ldg(p.w_scale + ti.expert));
       const int f0 = ti.w0 + static_cast<int>(rank) * 128 + q * 32;   // first feature of this warp
+      // GEMM 2: the gates of this warp's four chunks (chunk half * 4 + i, token
+      // (half * 4 + i) * 32 + lane), requested before the accumulator wait
+      float gates[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tk = (half * 4 + i) * 32 + lane;
+        gates[i] = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && tk < ti.act_n) ? __ldg(p.row_scale + ti.act0 + tk)
+                                                                                : 1.0f;
+      }
       if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1800 + buf)) break;
       tc_fence_after();
       const uint32_t acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (buf ? S::kAcc1 : 0);
@@ -371,7 +380,8 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           p.out_sf[fp4_sf_offset(row, j0, groups64_out)] = static_cast<uint8_t>(s0);
           p.out_sf[fp4_sf_offset(row, j0 + 1, groups64_out)] = static_cast<uint8_t>(s1);
         } else {
-          const float g = p.row_scale ? __ldg(p.row_scale + row) : 1.0f;
+          const int gi = c & 3;   // chunk c is half * 4 + gi
+          const float g = gi == 0 ? gates[0] : gi == 1 ? gates[1] : gi == 2 ? gates[2] : gates[3];
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + f0;
 #pragma unroll
           for (int j = 0; j < 32; j += 16) {

@@ -51,15 +51,17 @@ static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const
                              cudaStream_t s) {
   using Sm = TcSmem<BN, STAGES>;
   auto kern = tc_gemm_kernel<BN, STAGES, EPI>;
+  constexpr int smem = Sm::kBytes + (EPI == EPI_SCATTER ? Sm::kScatterBytes : 0);
+  static_assert(EPI != EPI_SCATTER || BN < 64 || smem <= 232448, "scatter epilogue exceeds shared memory");
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!device_configured(configured, dev)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return LMOE_ERR_CUDA;
     mark_configured(configured, dev);
   }
-  launch_k(kern, dim3(grid), dim3(192), Sm::kBytes, s, a0, b0, a1, b1, bs, p);
+  launch_k(kern, dim3(grid), dim3(192), smem, s, a0, b0, a1, b1, bs, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -136,7 +138,8 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
     return LMOE_ERR_INVALID_ARG;
   if (L.fp8 && L.grouped) return LMOE_ERR_UNSUPPORTED;
   if (p.ksplit > 1 && (L.grouped || !L.partial)) return LMOE_ERR_INVALID_ARG;
-  if (L.epi == EPI_SCATTER && (L.swap || L.ksplit > 1 || !L.scatter_rows || L.scatter_k <= 0))
+  if (L.epi == EPI_SCATTER &&
+      (L.swap || L.ksplit > 1 || !L.scatter_rows || L.scatter_k <= 0 || L.scatter_k > 32 || L.bn < 64))
     return LMOE_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   const int64_t tiles = L.max_tiles * p.ksplit;

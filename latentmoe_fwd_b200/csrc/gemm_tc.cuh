@@ -101,6 +101,10 @@ struct TcSmem {
   // 80-byte row pitch (bank-conflict free) for the scatter epilogue
   static constexpr int kEpiWarpBytes = 32 * 80;
   static constexpr int kBytes = kEpiOffset + 4 * kEpiWarpBytes + 1024;  // +1024 alignment slack
+  // scatter epilogue only (launched with kBytes + kScatterBytes): each epilogue
+  // warp's 32 token rows x up to 32 destination rows, loaded once per tile
+  static constexpr int kScatterOffset = kEpiOffset + 4 * kEpiWarpBytes;
+  static constexpr int kScatterBytes = 4 * 32 * 32 * 4;
 };
 
 struct TileInfo {
@@ -423,6 +427,15 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
       const int nchunks = p.swap ? (ti.act_n + 31) / 32 : BN / 32;
+      int* srow = reinterpret_cast<int*>(smem + S::kScatterOffset) + (warp & 3) * 32 * 32;
+      if (EPI == EPI_SCATTER) {
+        // the destination rows of this warp's 32 tokens (contiguous in
+        // scatter_rows), read once per tile so the stores below wait on none
+        const int nrow = max(0, min(32, ti.act_n - q * 32)) * p.scatter_k;
+        const int* src = p.scatter_rows + static_cast<long long>(ti.act0 + q * 32) * p.scatter_k;
+        for (int i = lane; i < nrow; i += 32) srow[i] = __ldg(src + i);
+        __syncwarp();
+      }
 #pragma unroll 1
       for (int c = 0; c < nchunks; ++c) {
         uint32_t v[32];
@@ -452,8 +465,7 @@ __global__ void __launch_bounds__(192, 1)
           while (kk >= K) { kk -= K; ++rr; }
           const int rows_here = min(32, ti.act_n - q * 32);
           for (; rr < rows_here;) {
-            const long long tok = ti.act0 + q * 32 + rr;
-            const int pr = __ldg(p.scatter_rows + tok * K + kk);
+            const int pr = srow[rr * K + kk];
             if (pr >= 0 && col0 + part * 8 < p.cols)
               st_global_v4_hint(reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(pr) * p.ld_out + col0 +
                                     part * 8,
@@ -540,6 +552,7 @@ __global__ void __launch_bounds__(192, 1)
               res[j] = live ? __bfloat162float(p.residual[(ti.act0 + c * 32 + j) * p.ld_res + col]) : 0.0f;
             }
           }
+          const float fp8_sc = EPI == EPI_SCALE ? fp8_acc_scale(p) : 1.0f;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float val = __uint_as_float(v[j]);
@@ -550,6 +563,8 @@ __global__ void __launch_bounds__(192, 1)
               val = val * __shfl_sync(0xffffffffu, gate, j);
             } else if (EPI == EPI_ADD_RES) {
               val = val + res[j];
+            } else if (EPI == EPI_SCALE) {
+              val = __fmul_rn(val, fp8_sc);
             }
             tb[j * 32 + lane] = __float2bfloat16_rn(val);
           }

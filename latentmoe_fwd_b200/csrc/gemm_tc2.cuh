@@ -102,7 +102,10 @@ struct Tc2Smem {
   static constexpr int kPrefixOffset = kBarOffset + (2 * kStages + 5) * 8 + 16;
   static constexpr int kMaxGroups = 1024;
   static constexpr int kEpiOffset = (kPrefixOffset + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
-  static constexpr int kBytes = kEpiOffset + 4 * 32 * 32 * 2 + 1024;   // +1024 alignment slack
+  // per expert: its row count and first padded row, copied from global memory
+  // once, so that no role waits on a global load at a tile boundary
+  static constexpr int kExpertOffset = kEpiOffset + 4 * 32 * 32 * 2;
+  static constexpr int kBytes = kExpertOffset + 2 * kMaxGroups * 4 + 1024;   // +1024 alignment slack
   static constexpr int kTmemCols = 512;       // two 256-column accumulators
   static constexpr int kTokens = 256;         // tokens per tile (MMA N <= 256)
 };
@@ -127,7 +130,8 @@ __device__ __forceinline__ int tc2_extra_tiles(const TcParams& p) {
   return p.rows_x > 0 ? ((p.rows_x + 255) / 256) * ((p.cols_x + 255) / 256) : 0;
 }
 
-__device__ __forceinline__ Tile2 tc2_tile(const TcParams& p, int i, int ntiles, int nextra, const int* prefix) {
+__device__ __forceinline__ Tile2 tc2_tile(const TcParams& p, int i, int ntiles, int nextra, const int* prefix,
+                                          const int* ecount, const int* epoff) {
   Tile2 ti;
   const long long before = static_cast<long long>(i) * nextra / ntiles;
   if (nextra > 0 && static_cast<long long>(i + 1) * nextra / ntiles > before) {
@@ -153,12 +157,12 @@ __device__ __forceinline__ Tile2 tc2_tile(const TcParams& p, int i, int ntiles, 
     if (prefix[mid] <= t) lo = mid; else hi = mid - 1;
   }
   const int e = lo;
-  const int n_e = __ldg(p.offsets + e + 1) - __ldg(p.offsets + e);
+  const int n_e = ecount[e];
   const int local = t - prefix[e];
   const int tt = local / ntw, mw = local % ntw;
   ti.expert = e;
   ti.w0 = mw * 256;
-  ti.act0 = __ldg(p.padded_offsets + e) + tt * Tc2Smem::kTokens;
+  ti.act0 = epoff[e] + tt * Tc2Smem::kTokens;
   ti.act_n = min(Tc2Smem::kTokens, n_e - tt * Tc2Smem::kTokens);
   ti.valid = ti.act_n > 0;
   ti.n = (ti.act_n + 31) & ~31;
@@ -187,6 +191,8 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
   int* prefix = reinterpret_cast<int*>(smem + S::kPrefixOffset);
   __nv_bfloat16* epi_tile = reinterpret_cast<__nv_bfloat16*>(smem + S::kEpiOffset);
+  int* ecount = reinterpret_cast<int*>(smem + S::kExpertOffset);
+  int* epoff = ecount + S::kMaxGroups;
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -208,6 +214,8 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       prefix[e + 1] = ((n_e + S::kTokens - 1) / S::kTokens) * ntw;
+      ecount[e] = n_e;
+      epoff[e] = __ldg(p.padded_offsets + e);
     }
     if (threadIdx.x == 0) prefix[0] = 0;
     __syncthreads();
@@ -264,7 +272,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       bool ok = true, issued = false;
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
-        const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix);
+        const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix, ecount, epoff);
         if (!ti.valid) continue;
         const int half = ti.n >> 1;
         const int b_row0 = ti.act0 + static_cast<int>(rank) * half;
@@ -274,8 +282,7 @@ __global__ void __launch_bounds__(192, 1)
         // expert's next token tile; every token tile of the extra problem)
         const bool wshared =
             ti.extra ? p.rows_x > S::kTokens
-                     : ti.act0 + S::kTokens < __ldg(p.padded_offsets + ti.expert) +
-                                                  (__ldg(p.offsets + ti.expert + 1) - __ldg(p.offsets + ti.expert));
+                     : ti.act0 + S::kTokens < epoff[ti.expert] + ecount[ti.expert];
         const uint64_t pa = wshared ? pol_keep : pol_stream;
         for (int kb = 0; kb < ti.kblocks; kb += S::kAtoms) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x2100 + stage)) { ok = false; break; }
@@ -318,7 +325,7 @@ __global__ void __launch_bounds__(192, 1)
       int local = 0;
       bool ok = true, any = false;
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
-        const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix);
+        const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix, ecount, epoff);
         if (!ti.valid) continue;
         const int acc = local & 1;
         if (!mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.err, 0x2200 + acc)) { ok = false; break; }
@@ -356,9 +363,19 @@ __global__ void __launch_bounds__(192, 1)
     const int r = q * 32 + lane;   // feature row of this thread within the CTA's 128
     int local = 0;
     for (int t = cluster; t < ntiles; t += nclusters) {
-      const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix);
+      const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix, ecount, epoff);
       if (!ti.valid) continue;
       const int acc = local & 1;
+      const float* const row_scale = ti.extra ? nullptr : p.row_scale;
+      // the gates of the tile's tokens, all requested at once and before the
+      // wait for the accumulator (lane: token c * 32 + lane of chunk c), so
+      // their latency hides behind the tile's MMAs
+      float gates[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int tk = c * 32 + lane;
+        gates[c] = (EPI == EPI_GATE && row_scale && tk < ti.act_n) ? __ldg(row_scale + ti.act0 + tk) : 1.0f;
+      }
       if (!mbar_wait(&tfull[acc], (local >> 1) & 1, abort_flag, p.err, 0x2400 + acc)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
@@ -367,22 +384,12 @@ __global__ void __launch_bounds__(192, 1)
       const int cols = ti.extra ? p.cols_x : p.cols;
       __nv_bfloat16* const out = reinterpret_cast<__nv_bfloat16*>(ti.extra ? p.out_x : p.out);
       const long long ld_out = ti.extra ? p.ld_out_x : p.ld_out;
-      const float* const row_scale = ti.extra ? nullptr : p.row_scale;
       const int nchunks = (ti.act_n + 31) / 32;
       __nv_bfloat16* tb = epi_tile + q * 32 * 32;
-#pragma unroll 1
-      for (int c = 0; c < nchunks; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
-        tmem_ld_wait();
-        // this lane owns feature wbase + r for 32 tokens; transpose the warp's
-        // 32 x 32 block through shared memory so each token's 32 features go
-        // out as 16-byte stores
-        float gate = 1.0f;
-        if (EPI == EPI_GATE && row_scale) {
-          const int tk = c * 32 + lane;
-          gate = tk < ti.act_n ? __ldg(row_scale + ti.act0 + tk) : 0.0f;
-        }
+      // this lane owns feature wbase + r for 32 tokens a chunk; each warp's
+      // 32 x 32 block is transposed through shared memory so each token's 32
+      // features go out as 16-byte stores
+      auto emit = [&](int c, const uint32_t (&v)[32], float gate) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           float val = __uint_as_float(v[j]);
@@ -407,6 +414,17 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         __syncwarp();
+      };
+      // two chunks per tensor-memory wait
+#pragma unroll
+      for (int c = 0; c < 8; c += 2) {
+        if (c >= nchunks) break;
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, v0);
+        if (c + 1 < nchunks) tmem_ld_32x32b_x32(t_row + (c + 1) * 32, v1);
+        tmem_ld_wait();
+        emit(c, v0, gates[c]);
+        if (c + 1 < nchunks) emit(c + 1, v1, gates[c + 1]);
       }
       tc_fence_before();
       __syncwarp();

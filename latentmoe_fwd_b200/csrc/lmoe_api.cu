@@ -88,7 +88,7 @@ int64_t splitk_floats(const lmoe_config* c, int op) { return c->T * max_dense_co
 struct Layout {
   size_t splitk = 0;        // fp32 split-K partial sums of the weight-major dense GEMMs (T <= 64)
   size_t rsplit = 0;        // fp32 split-K partial sums of the token-major router GEMM (few tiles)
-  size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, zq = 0, zq_sf = 0, z_gs = 0, partials = 0, xq = 0,
+  size_t err = 0, logits = 0, idx = 0, w = 0, z = 0, z_gs = 0, partials = 0, xq = 0,
          offsets = 0, poff = 0, perm_src = 0, inv_perm = 0, slot_row = 0, scratch = 0, gate = 0, zp = 0,
          zp_sf = 0, a = 0, a_sf = 0, y = 0, c = 0, hs = 0, ys = 0, total = 0;
 };
@@ -129,8 +129,6 @@ Layout layout(const lmoe_config* c, int op) {
     L.w = take(T * K * 4);
     if (!identity(c)) L.z = take(T * c->l * ab);
     if (fp4) {
-      L.zq = take(T * c->l / 2);
-      L.zq_sf = take(T * c->l / 16);
       L.z_gs = take(16);
       L.partials = take(nvfp4_partials(T * c->l) * 4);
     }
@@ -819,12 +817,11 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   float* gate = at<float>(ws, L.gate);
   void* zp = at<void>(ws, L.zp);
-  uint8_t* zq_sf = nullptr;
   float* z_gs = nullptr;
   // BF16 latent layer with token-major tiles: the permutation runs first and
   // the down-projection's epilogue writes each token's z row straight to the
   // padded rows of its K slots, so z is never stored and gathered
-  const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens;
+  const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens && l >= 64;
   if (scatter_z) {
     int32_t* slot_row = at<int32_t>(ws, L.slot_row);
     if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
@@ -844,6 +841,26 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     D.scatter_rows = slot_row;
     D.scatter_k = K;
     if ((st = tc_gemm(D, err, s)) != LMOE_OK) return st;
+    mark(3);
+  } else if (fp4) {
+    // NVFP4 latent activations (current per-tensor amax): the permutation runs
+    // first and the quantiser writes each token's codes and scales straight to
+    // the padded rows of its K slots
+    int32_t* slot_row = at<int32_t>(ws, L.slot_row);
+    if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
+                             err, s, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
+      return st;
+    const void* z = x;
+    if (!ident) {
+      void* zb = at<void>(ws, L.z);
+      if ((st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s)) != LMOE_OK)
+        return st;
+      z = zb;
+    }
+    z_gs = at<float>(ws, L.z_gs);
+    if ((st = launch_nvfp4_quantize_scatter(z, T, l, slot_row, K, static_cast<uint8_t*>(zp), at<uint8_t>(ws, L.zp_sf),
+                                            z_gs, at<float>(ws, L.partials), nvfp4_partials(T * l), s)) != LMOE_OK)
+      return st;
     mark(3);
   } else {
     // 2. latent down-projection d -> l
@@ -867,25 +884,14 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
       if (st != LMOE_OK) return st;
       z = zb;
     }
-    if (fp4) {
-      // NVFP4 latent activations: current per-tensor amax, row-major block scales
-      zq_sf = at<uint8_t>(ws, L.zq_sf);
-      z_gs = at<float>(ws, L.z_gs);
-      if ((st = launch_nvfp4_quantize(z, LMOE_BF16, T, l, nullptr, at<uint8_t>(ws, L.zq), zq_sf, z_gs,
-                                      LMOE_SF_ROWMAJOR, at<float>(ws, L.partials), nvfp4_partials(T * l), err, s)) !=
-          LMOE_OK)
-        return st;
-      z = at<void>(ws, L.zq);
-    }
     mark(2);
 
     // 3. dispatch grouped by expert (padded rows), gates per padded row
     if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
                              err, s)) != LMOE_OK)
       return st;
-    const int64_t row_bytes = fp4 ? l / 2 : static_cast<int64_t>(l) * ab;
-    uint8_t* zp_sf = fp4 ? at<uint8_t>(ws, L.zp_sf) : nullptr;
-    if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, zq_sf, zp_sf, N, s)) !=
+    const int64_t row_bytes = static_cast<int64_t>(l) * ab;
+    if ((st = launch_gather(idx, perm_src, offsets, poff, T * K, K, z, row_bytes, zp, nullptr, nullptr, N, s)) !=
         LMOE_OK)
       return st;
     mark(3);

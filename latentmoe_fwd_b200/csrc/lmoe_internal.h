@@ -174,6 +174,11 @@ lmoe_status launch_selftest_wait(uint32_t* err, long long limit_cycles, cudaStre
 lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int32_t* inv_perm,
                            const int32_t* offsets, const int32_t* padded_offsets, const float* w,
                            const void* resid, void* c, int64_t T, int K, int N, int l, cudaStream_t s);
+// BF16 rows -> NVFP4 (current amax) written at each row's K slot rows
+// (slot_row [rows][K], -1 skips) with MMA-tiled scales; cols % 64 == 0, K <= 32.
+lmoe_status launch_nvfp4_quantize_scatter(const void* in, int64_t rows, int cols, const int32_t* slot_row, int K,
+                                          uint8_t* codes, uint8_t* sf, float* global_out, float* partials,
+                                          int npartials, cudaStream_t s);
 lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                   const float* global_in, uint8_t* codes, uint8_t* sf,
                                   float* global_out, int sf_layout, float* partials,
