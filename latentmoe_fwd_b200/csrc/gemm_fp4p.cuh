@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(overlap_bar);
       };
       // chunk c (32 tokens): transpose so that lane j holds token c*32+j's 32 features
-      auto emit = [&](int c, const uint32_t (&v)[32]) {
+      auto emit = [&](int c, const uint32_t (&v)[32], float g) {
         if (c * 32 >= ti.act_n) return;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -380,8 +380,6 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           p.out_sf[fp4_sf_offset(row, j0, groups64_out)] = static_cast<uint8_t>(s0);
           p.out_sf[fp4_sf_offset(row, j0 + 1, groups64_out)] = static_cast<uint8_t>(s1);
         } else {
-          const int gi = c & 3;   // chunk c is half * 4 + gi
-          const float g = gi == 0 ? gates[0] : gi == 1 ? gates[1] : gi == 2 ? gates[2] : gates[3];
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + f0;
 #pragma unroll
           for (int j = 0; j < 32; j += 16) {
@@ -392,40 +390,25 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           }
         }
       };
-      // The slice shared with the other accumulator (chunks 6,7 of buffer 0,
-      // chunks 0,1 of buffer 1) is read first, both chunks at once, and the
-      // MMA released before any arithmetic; the other warps release at once.
+      // The warp's four chunks are read two at a time (one wait per pair). The
+      // next tile's accumulator overlaps chunks 6,7 of buffer 0 / chunks 0,1
+      // of buffer 1: the pair holding those is read first and the MMA released
+      // before any arithmetic (a warp arrives for this tile only after
+      // finishing the previous one, so the release also frees the rest of the
+      // buffer for the tile after next).
       const int nch = (ti.act_n + 31) / 32;
-      const bool owns_shared = buf ? half == 0 : half == 1;
-      if (owns_shared) {
-        const int c0 = buf ? 0 : 6;
+      const int i0 = buf ? 0 : 2;   // first pair (of the warp's chunks half * 4 + i)
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int i = pr == 0 ? i0 : 2 - i0;
+        const int c = half * 4 + i;
         uint32_t v0[32], v1[32];
-        tmem_ld_32x32b_x32(acc + c0 * 32, v0);
-        tmem_ld_32x32b_x32(acc + (c0 + 1) * 32, v1);
+        if (c < nch) tmem_ld_32x32b_x32(acc + c * 32, v0);
+        if (c + 1 < nch) tmem_ld_32x32b_x32(acc + (c + 1) * 32, v1);
         tmem_ld_wait();
-        release();
-        if (c0 < nch) emit(c0, v0);
-        if (c0 + 1 < nch) emit(c0 + 1, v1);
-        const int c2 = buf ? 2 : 4;
-#pragma unroll 1
-        for (int i = 0; i < 2; ++i) {
-          if (c2 + i >= nch) break;
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(acc + (c2 + i) * 32, v);
-          tmem_ld_wait();
-          emit(c2 + i, v);
-        }
-      } else {
-        release();
-#pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
-          const int c = half * 4 + i;
-          if (c >= nch) break;
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(acc + c * 32, v);
-          tmem_ld_wait();
-          emit(c, v);
-        }
+        if (pr == 0) release();
+        emit(c, v0, i == 0 ? gates[0] : gates[2]);
+        emit(c + 1, v1, i == 0 ? gates[1] : gates[3]);
       }
       ++local;
     }
