@@ -127,8 +127,9 @@ static lmoe_status fp4p_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_
   p.out_sf = L.out_sf;
   p.ld_out = L.ld_out;
   p.err = DevErr{err_word};
-  // tiles: at most (a_rows / 256 + groups) token tiles, each with cols / 256 weight tiles
-  const int64_t tiles = (L.a_rows / 256 + L.groups) * (L.cols / 256);
+  // tiles: at most a_rows / 128 token tiles (each expert's padded range is a
+  // multiple of 128 rows), each with cols / 256 weight tiles
+  const int64_t tiles = (L.a_rows / 128) * (L.cols / 256);
   if (L.quant_out) return launch_fp4p<FP4_EPI_SQRELU_QUANT>(maps, p, tiles, stream);
   return launch_fp4p<FP4_EPI_GATE_BF16>(maps, p, tiles, stream);
 }

@@ -3,23 +3,26 @@
 //
 //   D[w, t] = sum_k (q_w[w,k] s_w[w,k/16]) (q_a[t,k] s_a[t,k/16])
 //     w: 256 output features of expert e (128 per CTA of the pair)
-//     t: up to 256 of the expert's tokens (the MMA's N, rounded up to 64)
+//     t: up to 128 of the expert's tokens (the MMA's N, 64 or 128)
 //
 // Each CTA loads its 128 weight rows and their scales, its half of the token
 // rows, and the scales of all N tokens (the pair's MMA reads B's scales in
 // both CTAs); every load is a TMA load with .cta_group::2 that completes on
 // the even CTA's barrier (no multicast). The even CTA's single MMA thread
 // moves the scales to both CTAs' tensor memory with tcgen05.cp.cta_group::2
-// and issues the pair's MMAs. Against the single-CTA token-major kernel this
-// halves the scale copies and MMA issues per SM, moves ~30% fewer bytes per
-// multiply, and pads no token rows (N follows the tile's token count).
+// and issues the pair's MMAs.
 //
-// Tensor memory per CTA: two accumulators of up to 256 columns overlapping in
-// columns [192, 256) ([0,256) and [192,448)), scales at [448, 512): 4 x 4
-// columns of weight scales and 4 x 8 of token scales per stage.
+// Tensor memory per CTA: two accumulators of 128 columns ([0,128) and
+// [128,256)), so the MMAs of a tile wait only for the epilogue of the tile
+// two before it; scales at [256, 288): 4 x 4 columns of weight scales and
+// 4 x 4 of token scales per stage. (An FP4 tile of 256 tokens would need two
+// 256-column accumulators and leave no columns for the scales; letting them
+// overlap made every tile's MMAs wait for the previous tile's epilogue, and
+// with FP4's short tiles that wait was most of the time.)
 // Epilogue: eight warps, two per TMEM lane quarter (one feature per lane),
-// each draining 32-token chunks; a chunk is transposed through shared memory
-// so that each lane then holds one token's 32 features:
+// each reading its two 32-token chunks with one wait and releasing the
+// accumulator before any arithmetic; a chunk is transposed through shared
+// memory so that each lane then holds one token's 32 features:
 //   GEMM 1: a = relu(acc * s_z * s_w1[e])^2 quantised to NVFP4 with the static
 //           scale s_a (16-feature blocks along the token's row)
 //   GEMM 2: y = acc * s_a * s_w2[e] * gate[token], BF16
@@ -33,11 +36,11 @@ namespace lmoe {
 
 struct Fp4pSmem {
   static constexpr int kA = 128 * 128;        // 128 weight rows x 256 fp4
-  static constexpr int kB = 128 * 128;        // up to 128 token rows x 256 fp4
+  static constexpr int kB = 64 * 128;         // up to 64 token rows (this CTA's half) x 256 fp4
   static constexpr int kSFA = 4 * 512;        // 4 atoms (4 K-groups of 64) of this CTA's 128 weight rows
-  static constexpr int kSFB = 8 * 512;        // 4 K-groups x 2 row blocks of the tile's tokens
-  static constexpr int kStage = kA + kB + kSFA + kSFB;   // 38912 = 38 KB, a multiple of 1024
-  static constexpr int kStages = 4;
+  static constexpr int kSFB = 4 * 512;        // 4 atoms of the tile's (up to) 128 tokens
+  static constexpr int kStage = kA + kB + kSFA + kSFB;   // 28672 = 28 KB, a multiple of 1024
+  static constexpr int kStages = 6;
   static constexpr int kBarOffset = kStages * kStage;
   static constexpr int kMaxGroups = 1024;
   static constexpr int kPrefixOffset = kBarOffset + 256;
@@ -48,10 +51,10 @@ struct Fp4pSmem {
   static constexpr int kExpertOffset = kEpiOffset + 8 * kEpiWarpBytes;
   static constexpr int kBytes = kExpertOffset + 2 * kMaxGroups * 4 + 1024;
   static constexpr int kThreads = 64 + 256;   // producer, MMA, eight epilogue warps
-  static constexpr int kAcc1 = 192;           // second accumulator starts here
-  static constexpr int kSfaCol = 448;
-  static constexpr int kSfbCol = 464;
-  static constexpr int kTokens = 256;
+  static constexpr int kAccCols = 128;        // accumulator b at columns [128 b, 128 b + 128)
+  static constexpr int kSfaCol = 256;
+  static constexpr int kSfbCol = 272;
+  static constexpr int kTokens = 128;
 };
 
 struct Fp4pParams {
@@ -107,7 +110,7 @@ struct Tile4p {
   int n;       // MMA N: act_n rounded up to 64
 };
 
-// Pair tile t: expert e, token tile tt (256 tokens), weight tile of 256
+// Pair tile t: expert e, token tile tt (128 tokens), weight tile of 256
 // features; the weight tiles of one token tile are consecutive.
 __device__ __forceinline__ Tile4p fp4p_tile(const Fp4pParams& p, int t, const int* prefix, const int* ecount,
                                             const int* epoff) {
@@ -127,9 +130,8 @@ __device__ __forceinline__ Tile4p fp4p_tile(const Fp4pParams& p, int t, const in
   ti.act0 = epoff[e] + tt * Fp4pSmem::kTokens;
   ti.act_n = min(Fp4pSmem::kTokens, n_e - tt * Fp4pSmem::kTokens);
   ti.valid = ti.act_n > 0;
-  // block-scaled MMA widths step in 64 columns (the token scales sit in 128-row
-  // atoms, read 64 columns at a time): N in {64, 128, 192, 256}
-  ti.n = (ti.act_n + 63) & ~63;
+  // the MMA's N: 64 or 128 (the token scales sit in one 128-row atom)
+  ti.n = ti.act_n <= 64 ? 64 : 128;
   return ti;
 }
 
@@ -143,8 +145,8 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
   uint64_t* empty = full + S::kStages;
   uint64_t* tfull = empty + S::kStages;   // [2]
-  uint64_t* overlap_free = tfull + 2;     // [1], even CTA: both CTAs' epilogue warps arrive
-  uint64_t* drain = overlap_free + 1;
+  uint64_t* tempty = tfull + 2;           // [2], even CTA: both CTAs' 16 epilogue warps arrive
+  uint64_t* drain = tempty + 2;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
   int* prefix = reinterpret_cast<int*>(smem + S::kPrefixOffset);
@@ -197,9 +199,10 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&tfull[0], 1);
-    mbar_init(&tfull[1], 1);
-    mbar_init(overlap_free, 16);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 16);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -226,10 +229,8 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
         const int half = ti.n >> 1;
         const int b_row0 = ti.act0 + static_cast<int>(rank) * half;
         const int rb_w = (ti.w0 >> 7) + static_cast<int>(rank);   // this CTA's weight row block
-        const int rb_t = ti.act0 >> 7;                              // the tile's first token row block
-        const int two_rb = ti.n > 128;
-        const uint32_t stage_bytes =
-            2u * (S::kA + S::kSFA) + static_cast<uint32_t>(ti.n) * 128u + 2u * (two_rb ? 2u : 1u) * 2048u;
+        const int rb_t = ti.act0 >> 7;                              // the tile's token row block
+        const uint32_t stage_bytes = 2u * (S::kA + S::kSFA + S::kSFB) + static_cast<uint32_t>(ti.n) * 128u;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x1500 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStage;
@@ -239,21 +240,12 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], stage_bytes);
           const uint32_t bar = cluster_map(smem_u32(&full[stage]), 0);
           tma_load_3d_pair(sa, &maps.m[0], bar, kb * 128, ti.w0 + static_cast<int>(rank) * 128, ti.expert, pol);
-          int done = 0;
-#pragma unroll
-          for (int i = 0; i < 3; ++i) {   // half is 32, 64, 96 or 128 rows
-            const int box = 128 >> i;
-            if (half - done >= box) {
-              tma_load_3d_pair(sb + done * 128, &maps.m[1 + i], bar, kb * 128, b_row0 + done, 0, pol);
-              done += box;
-            }
-          }
-          // scale atoms (4 per row block and K block) as 8 rows of 256 bytes
+          // half is 32 or 64 rows: maps 2 (64-row boxes) and 3 (32-row boxes)
+          tma_load_3d_pair(sb, &maps.m[half == 64 ? 2 : 3], bar, kb * 128, b_row0, 0, pol);
+          // scale atoms (4 per row block and K block) as 8 rows of 256 bytes; every
+          // map here is three-dimensional, the token maps with one group
           tma_load_3d_pair(ssfa, &maps.m[5], bar, 0, (rb_w * p.groups64 + kb * 4) * 2, ti.expert, pol);
-          // (every map here is three-dimensional, the token maps with one group)
           tma_load_3d_pair(ssfb, &maps.m[6], bar, 0, (rb_t * p.groups64 + kb * 4) * 2, 0, pol);
-          if (two_rb)
-            tma_load_3d_pair(ssfb + 2048, &maps.m[6], bar, 0, ((rb_t + 1) * p.groups64 + kb * 4) * 2, 0, pol);
           issued = true;
           if (++stage == S::kStages) { stage = 0; phase ^= 1; }
         }
@@ -277,13 +269,11 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
       for (int t = cluster; t < ntiles && ok; t += nclusters) {
         const Tile4p ti = fp4p_tile(p, t, prefix, ecount, epoff);
         if (!ti.valid) continue;
-        if (local > 0) {
-          if (!mbar_wait(overlap_free, (local - 1) & 1, abort_flag, p.err, 0x1600)) { ok = false; break; }
-        }
+        const int acc = local & 1;
+        if (!mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, abort_flag, p.err, 0x1600 + acc)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ((local & 1) ? S::kAcc1 : 0);
+        const uint32_t d_tmem = tmem_base + acc * S::kAccCols;
         const uint32_t idesc = idesc_nvfp4(256, ti.n);
-        const int two_rb = ti.n > 128;
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x1700 + stage)) { ok = false; break; }
           tc_fence_after();
@@ -294,19 +284,18 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             tmem_cp_sf_pair(sfa_t + kk * 4, sdesc_sf_atom(sfa_s + kk * 512));
-            tmem_cp_sf_pair(sfb_t + kk * 8, sdesc_sf_atom(sfb_s + kk * 512));
-            if (two_rb) tmem_cp_sf_pair(sfb_t + kk * 8 + 4, sdesc_sf_atom(sfb_s + 2048 + kk * 512));
+            tmem_cp_sf_pair(sfb_t + kk * 4, sdesc_sf_atom(sfb_s + kk * 512));
           }
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_nvfp4_pair(d_tmem, sdesc_kmajor_sw128(a_s + kk * 32), sdesc_kmajor_sw128(b_s + kk * 32), idesc,
-                           sfa_t + kk * 4, sfb_t + kk * 8, (kb | kk) != 0 ? 1u : 0u);
+                           sfa_t + kk * 4, sfb_t + kk * 4, (kb | kk) != 0 ? 1u : 0u);
           any = true;
           mma_commit_pair(&empty[stage], 0x3);
           if (++stage == S::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        mma_commit_pair(&tfull[local & 1], 0x3);
+        mma_commit_pair(&tfull[acc], 0x3);
         ++local;
       }
       if (any) {
@@ -318,13 +307,12 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
   } else if (warp >= 2) {
     // ---------------- epilogue (warps 2..9, both CTAs) ----------------
     const int q = warp & 3;             // TMEM lane quarter
-    const int half = (warp - 2) >> 2;   // which four of the eight 32-token chunks
+    const int half = (warp - 2) >> 2;   // which two of the four 32-token chunks
     float* tb = epi + (warp - 2) * (S::kEpiWarpBytes / 4);
     const float in_s0 = __ldg(p.in_scale);
     const float out_s = (EPI == FP4_EPI_SQRELU_QUANT) ? __ldg(p.out_scale) : 0.0f;
     const int groups64_out = p.cols / 64;
     const uint64_t pol_out = policy_evict_first();
-    const uint32_t overlap_bar = cluster_map(smem_u32(overlap_free), 0);
     int local = 0;
     for (int t = cluster; t < ntiles; t += nclusters) {
       const Tile4p ti = fp4p_tile(p, t, prefix, ecount, epoff);
@@ -333,23 +321,18 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
       const float in_s = p.in_scale_grouped ? __ldg(p.in_scale + ti.expert) : in_s0;
       const float scale = __fmul_rn(in_s, __ldg(p.w_scale + ti.expert));
       const int f0 = ti.w0 + static_cast<int>(rank) * 128 + q * 32;   // first feature of this warp
-      // GEMM 2: the gates of this warp's four chunks (chunk half * 4 + i, token
-      // (half * 4 + i) * 32 + lane), requested before the accumulator wait
-      float gates[4];
+      // GEMM 2: the gates of this warp's two chunks (chunk half * 2 + i, token
+      // (half * 2 + i) * 32 + lane), requested before the accumulator wait
+      float gates[2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tk = (half * 4 + i) * 32 + lane;
+      for (int i = 0; i < 2; ++i) {
+        const int tk = (half * 2 + i) * 32 + lane;
         gates[i] = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && tk < ti.act_n) ? __ldg(p.row_scale + ti.act0 + tk)
                                                                                 : 1.0f;
       }
       if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1800 + buf)) break;
       tc_fence_after();
-      const uint32_t acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (buf ? S::kAcc1 : 0);
-      auto release = [&]() {   // this warp no longer reads the TMEM slice the next tile overwrites
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(overlap_bar);
-      };
+      const uint32_t acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * S::kAccCols;
       // chunk c (32 tokens): transpose so that lane j holds token c*32+j's 32 features
       auto emit = [&](int c, const uint32_t (&v)[32], float g) {
         if (c * 32 >= ti.act_n) return;
@@ -390,26 +373,19 @@ __global__ void __launch_bounds__(Fp4pSmem::kThreads, 1)
           }
         }
       };
-      // The warp's four chunks are read two at a time (one wait per pair). The
-      // next tile's accumulator overlaps chunks 6,7 of buffer 0 / chunks 0,1
-      // of buffer 1: the pair holding those is read first and the MMA released
-      // before any arithmetic (a warp arrives for this tile only after
-      // finishing the previous one, so the release also frees the rest of the
-      // buffer for the tile after next).
+      // both chunks with one wait, then the accumulator goes back to the MMA
+      // (on the even CTA's barrier) before any arithmetic
       const int nch = (ti.act_n + 31) / 32;
-      const int i0 = buf ? 0 : 2;   // first pair (of the warp's chunks half * 4 + i)
-#pragma unroll
-      for (int pr = 0; pr < 2; ++pr) {
-        const int i = pr == 0 ? i0 : 2 - i0;
-        const int c = half * 4 + i;
-        uint32_t v0[32], v1[32];
-        if (c < nch) tmem_ld_32x32b_x32(acc + c * 32, v0);
-        if (c + 1 < nch) tmem_ld_32x32b_x32(acc + (c + 1) * 32, v1);
-        tmem_ld_wait();
-        if (pr == 0) release();
-        emit(c, v0, i == 0 ? gates[0] : gates[2]);
-        emit(c + 1, v1, i == 0 ? gates[1] : gates[3]);
-      }
+      const int c = half * 2;
+      uint32_t v0[32], v1[32];
+      if (c < nch) tmem_ld_32x32b_x32(acc + c * 32, v0);
+      if (c + 1 < nch) tmem_ld_32x32b_x32(acc + (c + 1) * 32, v1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_map(smem_u32(&tempty[buf]), 0));
+      emit(c, v0, gates[0]);
+      emit(c + 1, v1, gates[1]);
       ++local;
     }
   }

@@ -124,6 +124,11 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// The float an order key came from (+0 for either zero, a NaN for 1u).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 template <int NPL, typename TA>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits, int64_t T, int N,
                                                                int K, int tpb, int32_t* __restrict__ idx,
@@ -170,69 +175,81 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
       }
       tau = ldexpf(sqrtf(sq / static_cast<float>(N)), -12) + ldexpf(vmax_abs, -22);
     }
-    // this lane's best and second-best remaining entries (largest key, lowest
-    // column on ties); a lane that wins moves its second up, and scans its
-    // entries again only when it wins without a known second
+    // this lane's four best remaining entries, best first (largest key; the
+    // lower column first among equal keys); a lane that wins passes on to its
+    // next one and scans its entries again only when all four are gone
     uint32_t taken = 0;
-    uint32_t hk = 0, hk2 = 0;
-    int hi_i = 0, hi2 = 0;
-    float hv = -INFINITY, hv2 = -INFINITY;
-    auto top2 = [&]() {
-      hk = 0;
-      hk2 = 0;
-      hv = -INFINITY;
-      hv2 = -INFINITY;
+    uint32_t bk[4];
+    int bi[4];
+    auto rebuild = [&]() {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bk[j] = 0u;
+        bi[j] = 0;
+      }
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
         const uint32_t ki = ((taken >> i) & 1u) ? 0u : key[i];
-        if (ki > hk) {
-          hk2 = hk;
-          hi2 = hi_i;
-          hv2 = hv;
-          hk = ki;
-          hi_i = i;
-          hv = v[i];
-        } else if (ki > hk2) {
-          hk2 = ki;
-          hi2 = i;
-          hv2 = v[i];
+        if (ki > bk[3]) {   // strictly greater: an equal key stays behind the lower column
+          if (ki > bk[2]) {
+            bk[3] = bk[2];
+            bi[3] = bi[2];
+            if (ki > bk[1]) {
+              bk[2] = bk[1];
+              bi[2] = bi[1];
+              if (ki > bk[0]) {
+                bk[1] = bk[0];
+                bi[1] = bi[0];
+                bk[0] = ki;
+                bi[0] = i;
+              } else {
+                bk[1] = ki;
+                bi[1] = i;
+              }
+            } else {
+              bk[2] = ki;
+              bi[2] = i;
+            }
+          } else {
+            bk[3] = ki;
+            bi[3] = i;
+          }
         }
       }
     };
-    top2();
-    bool second = true;   // hk2 is the best entry after hk (0: none left)
+    rebuild();
     // extract candidates in (approximate) order: the K best, the (K+1)-th, and
     // while refining, further experts within 2 tau of the K-th (at most 32)
     float kth = -INFINITY;
     const int cmax = min(N, 32);
     while (C < cmax) {
-      const uint32_t mk = __reduce_max_sync(FULL, hk);
+      const uint32_t mk = __reduce_max_sync(FULL, bk[0]);
       if (mk == 0u) break;
-      const unsigned bal = __ballot_sync(FULL, hk == mk);
+      const unsigned bal = __ballot_sync(FULL, bk[0] == mk);
       int wl = __ffs(bal) - 1;
       if (bal & (bal - 1u))   // equal values in several lanes: the lowest column wins
-        wl = static_cast<int>(__reduce_min_sync(FULL, hk == mk ? static_cast<uint32_t>(hi_i * 32 + lane) : ~0u) & 31u);
-      const float bv = __shfl_sync(FULL, hv, wl);
-      const int bi = __shfl_sync(FULL, hi_i * 32 + lane, wl);
+        wl = static_cast<int>(__reduce_min_sync(FULL, bk[0] == mk ? static_cast<uint32_t>(bi[0] * 32 + lane) : ~0u) &
+                              31u);
+      const float bv = key_value(mk);
+      const int bidx = __shfl_sync(FULL, bi[0] * 32 + lane, wl);
       if (C >= K && !(refine && bv >= kth - 2.0f * tau)) break;   // not a boundary candidate
       if (lane == C) {
         my_v = bv;
-        my_i = bi;
+        my_i = bidx;
       }
       if (C == K - 1) kth = bv;
       ++C;
       if (!refine && C >= K) break;
       if (lane == wl) {   // the winning lane moves on to its next entry
-        taken |= 1u << hi_i;
-        if (second) {
-          hk = hk2;
-          hi_i = hi2;
-          hv = hv2;
-          second = false;
-        } else {
-          top2();
-          second = true;
-        }
+        taken |= 1u << bi[0];
+        bk[0] = bk[1];
+        bi[0] = bi[1];
+        bk[1] = bk[2];
+        bi[1] = bi[2];
+        bk[2] = bk[3];
+        bi[2] = bi[3];
+        bk[3] = 0u;
+        if (bk[0] == 0u) rebuild();
       }
     }
     if (refine) {
@@ -290,12 +307,16 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
     }
   }
   if (!has_token) return;
-  // rank of each candidate among the C
-  int rank = 0;
-  for (int c = 0; c < C; ++c) {
-    const float ov = __shfl_sync(FULL, my_v, c);
-    const int oi = __shfl_sync(FULL, my_i, c);
-    if (lane < C && c != lane && before(ov, oi, my_v, my_i)) ++rank;
+  // rank of each candidate among the C: the extraction order, unless the
+  // exact refinement changed some of the values
+  int rank = lane;
+  if (todo != 0u) {
+    rank = 0;
+    for (int c = 0; c < C; ++c) {
+      const float ov = __shfl_sync(FULL, my_v, c);
+      const int oi = __shfl_sync(FULL, my_i, c);
+      if (lane < C && c != lane && before(ov, oi, my_v, my_i)) ++rank;
+    }
   }
   const bool chosen = lane < C && rank < K;
   // the largest logit is rank 0
