@@ -3,7 +3,6 @@
 #include <mutex>
 
 #include "gemm_fp4.cuh"
-#include "gemm_fp4p.cuh"
 #include "gemm_tc.cuh"
 #include "lmoe_internal.h"
 
@@ -42,98 +41,6 @@ static bool make_map_fp4(CUtensorMap* map, const void* ptr, int64_t k, int64_t r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over bytes [d2][d1][d0] (d0 contiguous), no swizzle, box {box0, box1, 1}.
-static bool make_map_u8(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
-                        uint32_t box1) {
-  EncodeTiledFn enc = encode_fn_fp4();
-  if (!enc || !ptr || (reinterpret_cast<uintptr_t>(ptr) & 15) || d0 % 16) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0, d0 * d1};
-  cuuint32_t box[3] = {box0, box1, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <int EPI>
-static lmoe_status launch_fp4p(const Fp4pMaps& m, const Fp4pParams& p, int64_t max_tiles, cudaStream_t s) {
-  auto kern = fp4p_gemm_kernel<EPI>;
-  static std::atomic<uint64_t> configured{0};
-  static std::atomic<int> max_clusters_dev[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(Fp4pSmem::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Fp4pSmem::kBytes;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int max_clusters = 0;
-  if (device_configured(configured, dev)) {
-    max_clusters = max_clusters_dev[dev].load(std::memory_order_relaxed);
-  } else {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp4pSmem::kBytes) != cudaSuccess)
-      return LMOE_ERR_CUDA;
-    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess || max_clusters <= 0)
-      return LMOE_ERR_CUDA;
-    if (dev >= 0 && dev < 64) max_clusters_dev[dev].store(max_clusters, std::memory_order_relaxed);
-    mark_configured(configured, dev);
-  }
-  const int64_t clusters = max_tiles < max_clusters ? max_tiles : max_clusters;
-  if (clusters <= 0) return LMOE_OK;
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.numAttrs = 2;   // cluster shape + programmatic serialisation (occupancy was queried with the shape only)
-  if (cudaLaunchKernelEx(&cfg, kern, m, p) != cudaSuccess) return LMOE_ERR_CUDA;
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
-}
-
-// The CTA-pair weight-major kernel (see gemm_fp4p.cuh).
-static lmoe_status fp4p_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream) {
-  if (L.groups > Fp4pSmem::kMaxGroups) return LMOE_ERR_UNSUPPORTED;
-  Fp4pMaps maps;
-  if (!make_map_fp4(&maps.m[0], L.b_codes, L.k, L.cols, L.groups, 128)) return LMOE_ERR_INVALID_ARG;
-  for (int i = 0; i < 4; ++i)
-    if (!make_map_fp4(&maps.m[1 + i], L.a_codes, L.k, L.a_rows, 1, 128 >> i)) return LMOE_ERR_INVALID_ARG;
-  const uint64_t g64 = static_cast<uint64_t>(L.k / 64);
-  // scale atoms viewed as rows of 256 bytes: two rows per 512-byte atom
-  if (!make_map_u8(&maps.m[5], L.b_sf, 256, static_cast<uint64_t>(L.cols / 128) * g64 * 2, L.groups, 256, 8))
-    return LMOE_ERR_INVALID_ARG;
-  if (!make_map_u8(&maps.m[6], L.a_sf, 256, static_cast<uint64_t>(L.a_rows / 128) * g64 * 2, 1, 256, 8))
-    return LMOE_ERR_INVALID_ARG;
-  Fp4pParams p = {};
-  p.rows = static_cast<int>(L.a_rows);
-  p.cols = L.cols;
-  p.kblocks = static_cast<int>(L.k / 256);
-  p.groups64 = static_cast<int>(g64);
-  p.offsets = L.offsets;
-  p.padded_offsets = L.padded_offsets;
-  p.groups = L.groups;
-  p.in_scale = L.in_scale;
-  p.in_scale_grouped = L.in_scale_grouped;
-  p.w_scale = L.w_scale;
-  p.out_scale = L.out_scale;
-  p.row_scale = L.row_scale;
-  p.out = L.out;
-  p.out_sf = L.out_sf;
-  p.ld_out = L.ld_out;
-  p.err = DevErr{err_word};
-  // tiles: at most a_rows / 128 token tiles (each expert's padded range is a
-  // multiple of 128 rows), each with cols / 256 weight tiles
-  const int64_t tiles = (L.a_rows / 128) * (L.cols / 256);
-  if (L.quant_out) return launch_fp4p<FP4_EPI_SQRELU_QUANT>(maps, p, tiles, stream);
-  return launch_fp4p<FP4_EPI_GATE_BF16>(maps, p, tiles, stream);
-}
-
 template <int EPI>
 static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const Fp4Params& p, int grid,
                               cudaStream_t s) {
@@ -153,8 +60,6 @@ static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const 
 
 lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream) {
   if (L.k % 256 || L.cols % 256 || L.groups > Fp4Smem::kMaxGroups) return LMOE_ERR_UNSUPPORTED;
-  const bool vec32 = (reinterpret_cast<uintptr_t>(L.out) % 32 == 0) && (L.ld_out * 2) % 32 == 0;
-  if (L.pairs && (L.quant_out || vec32)) return fp4p_gemm(L, err_word, stream);
   CUtensorMap ma, mb;
   if (!make_map_fp4(&ma, L.a_codes, L.k, L.a_rows, 1, 128)) return LMOE_ERR_INVALID_ARG;
   if (!make_map_fp4(&mb, L.b_codes, L.k, L.cols, L.groups, 256)) return LMOE_ERR_INVALID_ARG;

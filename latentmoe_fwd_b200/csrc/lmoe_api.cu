@@ -583,8 +583,6 @@ lmoe_status expert_ffn_fp4(const lmoe_config* cfg, const lmoe_weights* w, const 
   g1.quant_out = 1;
   g1.out = a_codes;
   g1.out_sf = a_sf;
-  // enough rows per expert on average: CTA pairs, 256 features x up to 256 tokens per tile
-  g1.pairs = cfg->T > 64 && static_cast<int64_t>(cfg->T) * cfg->K >= 64LL * cfg->N;
   lmoe_status st = fp4_gemm(g1, err, s);
   if (st != LMOE_OK) return st;
   if (between) between();

@@ -118,7 +118,6 @@ struct Fp4Launch {
   const float* out_scale = nullptr;  // device scalar (quant_out)
   const float* row_scale = nullptr;  // gates (GEMM 2)
   int quant_out = 0;                 // 1: relu^2 + NVFP4 codes/scales out; 0: BF16 out * gate
-  int pairs = 0;                     // 1: CTA-pair weight-major tiles (many rows per expert)
   void* out = nullptr;
   uint8_t* out_sf = nullptr;
   int64_t ld_out = 0;
