@@ -382,37 +382,24 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
           }
         }
       };
-      // The slice shared with the other accumulator (chunks 6,7 of buffer 0,
-      // chunks 0,1 of buffer 1) is read first, both chunks at once, and the
-      // MMA released before any arithmetic; the other warps release at once.
+      // The warp's four chunks are read two at a time (one wait per pair). The
+      // slice shared with the other accumulator (chunks 6,7 of buffer 0,
+      // chunks 0,1 of buffer 1) belongs to one warp of each lane quarter: it
+      // reads that pair first and releases the MMA before any arithmetic; the
+      // other warps release at once.
       const bool owns_shared = buf ? half == 0 : half == 1;
-      if (owns_shared) {
-        const int c0 = buf ? 0 : 6;
+      if (!owns_shared) release();
+      const int i0 = buf ? 0 : 2;   // first pair (of the warp's chunks half * 4 + i)
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int c = half * 4 + (pr == 0 ? i0 : 2 - i0);
         uint32_t v0[32], v1[32];
-        tmem_ld_32x32b_x32(acc + c0 * 32, v0);
-        tmem_ld_32x32b_x32(acc + (c0 + 1) * 32, v1);
+        tmem_ld_32x32b_x32(acc + c * 32, v0);
+        tmem_ld_32x32b_x32(acc + (c + 1) * 32, v1);
         tmem_ld_wait();
-        release();
-        emit(c0, v0);
-        emit(c0 + 1, v1);
-        const int c2 = buf ? 2 : 4;
-#pragma unroll 1
-        for (int i = 0; i < 2; ++i) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(acc + (c2 + i) * 32, v);
-          tmem_ld_wait();
-          emit(c2 + i, v);
-        }
-      } else {
-        release();
-#pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
-          const int c = half * 4 + i;
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(acc + c * 32, v);
-          tmem_ld_wait();
-          emit(c, v);
-        }
+        if (pr == 0 && owns_shared) release();
+        emit(c, v0);
+        emit(c + 1, v1);
       }
       ++local;
     }
