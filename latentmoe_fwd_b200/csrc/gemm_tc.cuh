@@ -338,13 +338,20 @@ __global__ void __launch_bounds__(192, 1)
           } else {
             a_row = ti.w0; a_grp = ti.expert; b_row = ti.act0; b_grp = 0;
           }
-          // weights are streamed (evict first) unless several tiles of this
-          // expert share them (weight-major tiles of an expert with more tokens
-          // than one tile holds); activation rows are kept (evict last)
-          // weight-major tiles: the weights are kept when other token tiles of
-          // the expert will read them again, streamed otherwise
-          const uint64_t pa = p.swap ? (ti.wshared ? pol_a : pol_w) : pol_a;
-          const uint64_t pb = p.swap ? (ti.wshared ? pol_n : pol_a) : pol_w;
+          // L2 policy per operand:
+          //  * dense token-major tiles (the projections and the router at large
+          //    T): every row block reads all of the weight matrix, while a row
+          //    block of activations is read only by the tiles next to it in the
+          //    tile order, which run at the same time: weights kept (evict
+          //    last), activations normal, so a long activation stream cannot
+          //    push the weights out;
+          //  * grouped token-major tiles: an expert's weights serve only its
+          //    own row blocks: weights streamed, activations kept;
+          //  * weight-major tiles: weights kept when other token tiles of the
+          //    expert read them again, streamed otherwise; activations kept.
+          const bool dense_tm = !p.swap && !p.grouped;
+          const uint64_t pa = p.swap ? (ti.wshared ? pol_a : pol_w) : (dense_tm ? pol_n : pol_a);
+          const uint64_t pb = p.swap ? (ti.wshared ? pol_n : pol_a) : (dense_tm ? pol_a : pol_w);
           if (akg > 0) tma_load_3d(sa, ma, &full[stage], k % akg, a_row, k / akg, pa);
           else tma_load_3d(sa, ma, &full[stage], k, a_row, a_grp, pa);
           if (bkg > 0) tma_load_3d(sb, mb, &full[stage], k % bkg, b_row, k / bkg, pb);
