@@ -416,6 +416,48 @@ lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* p
                             const float* b_global, int cols, int64_t k, const float* row_scale, void* out,
                             int64_t ld_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Backward of the routed experts under the NVFP4 training recipe
+ * (greeksharifa page on the Nemotron 3 whitepaper, section 2.4 "NVFP4
+ * Training"; notes.yuuk.io page, section 4: fprop, dgrad and wgrad as NVFP4
+ * GEMMs, 16 x 16 weight blocks, stochastic rounding of gradients, a random
+ * Hadamard transform on the wgrad inputs; the details are readings). Slots
+ * are in lmoe_permute's padded layout: expert e owns rows
+ * padded_offsets[e] .. padded_offsets[e] + counts[e] - 1, padded_offsets[e]
+ * = sum over e' < e of counts[e'] rounded up to 128. Per expert, over its n
+ * rows (zero rows up to R = n rounded up to 16 wherever a quantiser runs
+ * along the rows):
+ *   W1q, W2q = the BF16 masters w1[e] [m][l], w2[e] [l][m] quantised with
+ *     16 x 16 blocks (current amax); h = zq W1q^T (BF16), aq = NVFP4(relu(h)^2)
+ *     with the static global scale a_global, o = aq W2q^T (BF16);
+ *   dgate[r] = dy[r] . o[r];  do = gate[r] dy[r]  (fp32);
+ *   dA = SR(do) W2q;  dh = dA * 2 max(h, 0);  dz = SR(dh) W1q;
+ *   dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T;  dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T;
+ *   SR: lmoe_nvfp4_quantize_ex's stochastic rounding with sr_stream
+ *   4 e + 2 g + j (g: 0 first GEMM, 1 second; j: 0 dgrad, 1 wgrad) and
+ *   `seed`; RHT with rht_signs; every quantiser takes its tensor's current
+ *   amax (per expert).
+ *  counts [N]: HOST array of rows per expert. offsets, padded_offsets [N+1]:
+ *    DEVICE arrays as lmoe_permute writes them.
+ *  z_codes [P][l/2], z_sf (MMA-tiled over the P padded rows), z_global
+ *    (device F32): the NVFP4 latent rows as lmoe_permute moves them.
+ *  w1, w2: BF16 masters [N][m][l], [N][l][m]. a_global: device F32.
+ *  gate [P] F32, dy [P][l] BF16: each slot row's gate and upstream gradient.
+ *  Outputs (device): dz [P][l] BF16 (padding rows unspecified), dgate [P] F32
+ *    (set for real rows only), dw1 [N][m][l] and dw2 [N][l][m] BF16.
+ *  l and m multiples of 256; 16-byte aligned buffers; ws of at least
+ *  lmoe_expert_backward_nvfp4_workspace(cfg, counts) bytes, its first 256
+ *  zeroed before first use (the error word).
+ *  Errors: LMOE_ERR_INVALID_ARG for null or unaligned pointers, negative
+ *  counts, N outside 1..1024; LMOE_ERR_UNSUPPORTED for l or m not multiples
+ *  of 256; LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT. */
+size_t lmoe_expert_backward_nvfp4_workspace(const lmoe_config* cfg, const int32_t* counts);
+lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* counts, const int32_t* offsets,
+                                       const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
+                                       const float* z_global, const void* w1, const void* w2,
+                                       const float* a_global, const float* gate, const void* dy, uint64_t seed,
+                                       uint32_t rht_signs, void* dz, float* dgate, void* dw1, void* dw2, void* ws,
+                                       size_t ws_bytes, void* stream);
+
 /* Expert parallelism in the latent dimension (greeksharifa page on the
  * Nemotron 3 whitepaper, section 2.2 "LatentMoE": the rows that cross GPUs
  * between the projections are l-dim, so the all-to-all volume falls by d/l).

@@ -37,7 +37,8 @@ EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permut
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
            "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize",
            "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_gemm",
-           "lmoe_ep_plan", "lmoe_ep_reorder")
+           "lmoe_ep_plan", "lmoe_ep_reorder", "lmoe_expert_backward_nvfp4",
+           "lmoe_expert_backward_nvfp4_workspace")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -95,6 +96,9 @@ def _load():
         "lmoe_nvfp4_quantize_ex": (ctypes.c_int, [P, ctypes.c_int, I64, I64, ctypes.c_uint32, ctypes.c_uint32,
                                                   ctypes.c_uint64, ctypes.c_uint32, P, P, P, P, ctypes.c_int, P,
                                                   ctypes.c_size_t, P]),
+        "lmoe_expert_backward_nvfp4_workspace": (ctypes.c_size_t, [C, P]),
+        "lmoe_expert_backward_nvfp4": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_uint64,
+                                                      ctypes.c_uint32, P, P, P, P, P, ctypes.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -258,6 +262,32 @@ def nvfp4_gemm(groups, offsets, padded_offsets, a_rows, a_codes, a_sf, a_global,
                                _p(a_global), int(a_global_per_group), _p(b_codes), _p(b_sf), _p(b_global),
                                int(cols), int(k), _p(row_scale), _p(out), int(ld_out), _p(ws), ws.numel(),
                                _stream(stream)), "lmoe_nvfp4_gemm")
+
+
+def expert_backward_nvfp4_workspace(cfg: Config, counts) -> int:
+    """lmoe_expert_backward_nvfp4_workspace (counts: host int32 array [N])."""
+    import numpy as np
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    return int(lib.lmoe_expert_backward_nvfp4_workspace(ctypes.byref(cfg),
+                                                        counts.ctypes.data_as(ctypes.c_void_p)))
+
+
+def expert_backward_nvfp4(cfg: Config, counts, offsets, padded_offsets, z_codes, z_sf, z_global, w1, w2, a_global,
+                          gate, dy, seed, rht_signs, dz, dgate, dw1, dw2, ws=None, stream=None):
+    """lmoe_expert_backward_nvfp4: the routed experts' backward under the NVFP4
+    training recipe (see the header). counts: host int32 array [N]; the rest
+    device tensors. Allocates the workspace when none is given."""
+    import numpy as np
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    if ws is None:
+        import torch
+        ws = torch.zeros(expert_backward_nvfp4_workspace(cfg, counts), dtype=torch.uint8, device="cuda")
+    _check(lib.lmoe_expert_backward_nvfp4(ctypes.byref(cfg), counts.ctypes.data_as(ctypes.c_void_p), _p(offsets),
+                                          _p(padded_offsets), _p(z_codes), _p(z_sf), _p(z_global), _p(w1), _p(w2),
+                                          _p(a_global), _p(gate), _p(dy), int(seed), int(rht_signs), _p(dz),
+                                          _p(dgate), _p(dw1), _p(dw2), _p(ws), ws.numel(), _stream(stream)),
+           "lmoe_expert_backward_nvfp4")
+    return ws
 
 
 def ep_plan(G: int, rank: int, counts):

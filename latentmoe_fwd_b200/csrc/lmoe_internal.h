@@ -189,7 +189,7 @@ int nvfp4x_partials(int64_t blocks);
 lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
-                                     cudaStream_t s);
+                                     cudaStream_t s, int64_t out_pitch = 0);
 // FP8 E4M3 codes of in / s with one FP32 scale per tensor (scale_in, or the
 // tensor's amax / 448 when scale_in is null; scale_out receives it).
 lmoe_status launch_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,

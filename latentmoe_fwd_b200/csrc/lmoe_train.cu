@@ -83,6 +83,7 @@ struct QxParams {
   uint8_t* codes;
   uint8_t* sf;
   float* global_out;
+  int64_t pitch;         // elements per stored output row (>= out cols; the rest stored as zero codes and scales)
 };
 
 __device__ __forceinline__ double load_in(const QxParams& p, int64_t r, int64_t c) {
@@ -200,9 +201,10 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p) 
   if (blockIdx.x == 0 && threadIdx.x == 0 && p.global_out) *p.global_out = s_g;
   const float t = __fmul_rn(s_g, 6.0f);
   const int64_t R = out_rows(p), C = out_cols(p), nb = C / 16;
-  const int64_t groups64 = (C + 63) / 64;
+  const int64_t nb_store = p.pitch / 16;   // stored blocks per row; those past nb are zero
+  const int64_t groups64 = (p.pitch + 63) / 64;
   const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;   // 16-row groups, tiled padding
-  const int64_t nb_cov = p.tiled ? groups64 * 4 : nb;
+  const int64_t nb_cov = p.tiled ? groups64 * 4 : nb_store;
   const int64_t total = rg_cov * nb_cov;
   for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
        b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -255,12 +257,14 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p) 
             hi = cvt_e2m1_x8(q + 8);
           }
         }
-        *reinterpret_cast<uint2*>(p.codes + ro * (C / 2) + j * 8) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(lo, hi);
+      } else if (ro < R && j < nb_store) {
+        *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(0u, 0u);
       }
       if (p.tiled) {
         if (ro < ((R + 127) / 128) * 128) p.sf[tiled_off(ro, j, groups64)] = static_cast<uint8_t>(scode);
-      } else if (ro < R && j < nb) {
-        p.sf[ro * nb + j] = static_cast<uint8_t>(scode);
+      } else if (ro < R && j < nb_store) {
+        p.sf[ro * nb_store + j] = static_cast<uint8_t>(scode);
       }
     }
   }
@@ -276,7 +280,7 @@ int nvfp4x_partials(int64_t blocks) {
 lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
-                                     cudaStream_t s) {
+                                     cudaStream_t s, int64_t out_pitch) {
   QxParams p = {};
   p.in = in;
   p.bf16 = in_dtype == LMOE_BF16;
@@ -295,6 +299,8 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   p.sf = sf;
   p.global_out = global_out;
   const int64_t R = p.transpose ? cols : rows, C = p.transpose ? rows : cols;
+  p.pitch = out_pitch > 0 ? out_pitch : C;
+  if (p.pitch < C || p.pitch % 16) return LMOE_ERR_INVALID_ARG;
   if (R == 0) return LMOE_OK;
   const int sms = device_sm_count();
   const int np = nvfp4x_partials(R * (C / 16));
@@ -305,7 +311,7 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   p.partials = partials;
   p.np = global_in ? 0 : np;
   const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;
-  const int64_t nb_cov = p.tiled ? (C + 63) / 64 * 4 : C / 16;
+  const int64_t nb_cov = p.tiled ? (p.pitch + 63) / 64 * 4 : p.pitch / 16;
   int64_t blocks = (rg_cov * nb_cov + kXThreads - 1) / kXThreads;
   if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
   if (blocks < 1) blocks = 1;

@@ -304,38 +304,33 @@ def _fake_quant(A, s_g=None):
     return O.nvfp4_fake_quant(A, s_g)[0]
 
 
-def backward_nvfp4(params: dict, K: int, dout, signs, seed: int, a_global_scale=None,
-                   quantize: bool = True) -> dict:
-    """The layer's gradients with its routed experts trained under the NVFP4
-    recipe: the expert GEMMs' forward reads NVFP4 z (current amax), NVFP4 a
-    (``a_global_scale``, else its current amax) and 2-D-block NVFP4 weights;
-    their dgrad and wgrad are ``nvfp4_linear_backward``, with each expert's
-    rows padded by zero rows to a multiple of 16 for the token transform. The
-    router, the latent projections and the shared experts stay unquantised
-    (the recipe keeps such layers in higher precision; the latent projections
-    stay BF16 on the pages), and every quantiser passes its gradient straight
-    through. Uniforms come from ``sr_uniforms(seed, stream)`` with stream
-    4 e + 2 g + j for expert e, GEMM g (0: first, 1: second) and j (0: dgrad,
-    1: wgrad). quantize=False turns every quantiser into the identity.
-    Returns the same keys as ``backward``.
+def routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, signs, seed: int, a_global_scale=None,
+                                  quantize: bool = True) -> dict:
+    """The routed experts' part of ``backward_nvfp4``, per expert e over the
+    slots routed to it (t, k with idx[t, k] == e, in token order):
+
+      forward (recomputed): h = ze W1q^T, aq = NVFP4(relu(h)^2, a_global_scale
+        or the current amax), o = aq W2q^T, with ze = zq[t] (the NVFP4 latent
+        rows) and W1q, W2q the experts' matrices quantised with 16 x 16 blocks;
+      dgate[t, k] = dy . o with dy = dc[t];  do = gate * dy;
+      dgrad and wgrad of the two GEMMs by ``nvfp4_linear_backward``, each
+        expert's rows padded by zero rows to a multiple of 16, uniforms from
+        ``sr_uniforms(seed, 4 e + 2 g + j)`` (g: 0 first GEMM, 1 second; j: 0
+        dgrad, 1 wgrad);  dh = dA * 2 max(h, 0).
+
+    Returns c [T, l] (the gated sum of the experts' outputs), dz [T, l] (the
+    gradient reaching zq), dgate [T, K], dw1 [N, m, l] and dw2 [N, l, m].
+    quantize=False turns every quantiser into the identity.
     """
-    x = np.asarray(params["x"], dtype=np.float64)
-    dout = np.asarray(dout, dtype=np.float64)
-    T = x.shape[0]
-    wr, bias = params["w_router"], params.get("router_bias")
-    w_down, w_up = params.get("w_down"), params.get("w_up")
-    w1, w2 = params["w1"], params["w2"]
-    N, m, l = w1.shape
+    zq, dc, gates = (np.asarray(a, dtype=np.float64) for a in (zq, dc, gates))
+    w1, w2 = np.asarray(w1, dtype=np.float64), np.asarray(w2, dtype=np.float64)
+    T, l = zq.shape
+    K = idx.shape[1]
+    N = w1.shape[0]
     fq = _fake_quant if quantize else (lambda A, s_g=None: A)
     fq2 = (lambda A: _deq(O.nvfp4_quantize_2d(A))) if quantize else (lambda A: A)
-
-    logits = O.router_logits(x, wr, bias)
-    idx, gates = O.route_topk(logits, K)
-    z = x if w_down is None else x @ w_down.T
-    zq = fq(z)
-    dc = dout if w_up is None else dout @ w_up
     c = np.zeros((T, l))
-    dz = np.zeros_like(z)
+    dz = np.zeros((T, l))
     dgate = np.zeros((T, K))
     dw1, dw2 = np.zeros_like(w1), np.zeros_like(w2)
 
@@ -367,10 +362,44 @@ def backward_nvfp4(params: dict, K: int, dout, signs, seed: int, a_global_scale=
                                    uni(l, R, 4 * e + 3), quantize)
         dw2[e] = r2["dW"]
         dh = r2["dX"][:n] * 2.0 * np.maximum(h, 0.0)
-        r1 = nvfp4_linear_backward(pad16(ze), w1[e], pad16(dh), signs, uni(R, m, 4 * e + 0),
-                                   uni(m, R, 4 * e + 1), quantize)
+        r1 = nvfp4_linear_backward(pad16(ze), w1[e], pad16(dh), signs, uni(R, w1.shape[1], 4 * e + 0),
+                                   uni(w1.shape[1], R, 4 * e + 1), quantize)
         dw1[e] = r1["dW"]
         np.add.at(dz, t, r1["dX"][:n])
+    return dict(c=c, dz=dz, dgate=dgate, dw1=dw1, dw2=dw2)
+
+
+def backward_nvfp4(params: dict, K: int, dout, signs, seed: int, a_global_scale=None,
+                   quantize: bool = True) -> dict:
+    """The layer's gradients with its routed experts trained under the NVFP4
+    recipe: the expert GEMMs' forward reads NVFP4 z (current amax), NVFP4 a
+    (``a_global_scale``, else its current amax) and 2-D-block NVFP4 weights;
+    their dgrad and wgrad are ``nvfp4_linear_backward``, with each expert's
+    rows padded by zero rows to a multiple of 16 for the token transform. The
+    router, the latent projections and the shared experts stay unquantised
+    (the recipe keeps such layers in higher precision; the latent projections
+    stay BF16 on the pages), and every quantiser passes its gradient straight
+    through. Uniforms come from ``sr_uniforms(seed, stream)`` with stream
+    4 e + 2 g + j for expert e, GEMM g (0: first, 1: second) and j (0: dgrad,
+    1: wgrad). quantize=False turns every quantiser into the identity.
+    Returns the same keys as ``backward``.
+    """
+    x = np.asarray(params["x"], dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    T = x.shape[0]
+    wr, bias = params["w_router"], params.get("router_bias")
+    w_down, w_up = params.get("w_down"), params.get("w_up")
+    w1, w2 = params["w1"], params["w2"]
+    N = w1.shape[0]
+    fq = _fake_quant if quantize else (lambda A, s_g=None: A)
+
+    logits = O.router_logits(x, wr, bias)
+    idx, gates = O.route_topk(logits, K)
+    z = x if w_down is None else x @ w_down.T
+    zq = fq(z)
+    dc = dout if w_up is None else dout @ w_up
+    r = routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, signs, seed, a_global_scale, quantize)
+    c, dz, dgate, dw1, dw2 = r["c"], r["dz"], r["dgate"], r["dw1"], r["dw2"]
     dw_up = None if w_up is None else dout.T @ c
 
     dsel = gates * (dgate - np.sum(gates * dgate, axis=1, keepdims=True))

@@ -165,3 +165,88 @@ def test_linear_layer_dgrad_and_wgrad_match_the_oracle():
     exact = B.nvfp4_linear_backward(X, W, dY, SIGNS, None, None, quantize=False)
     rel = np.sqrt(np.mean((dW - exact["dW"]) ** 2) / np.mean(exact["dW"] ** 2))
     assert 1e-3 < rel < 0.5
+
+
+@pytest.mark.parametrize("T,N,K,zero_expert", [(160, 4, 2, False), (96, 8, 3, True)])
+def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
+    """lmoe_expert_backward_nvfp4 (recomputed NVFP4 forward, SR dgrad, RHT +
+    SR wgrad for both expert GEMMs, every step a kernel of the library) against
+    the oracle's routed_experts_backward_nvfp4 on the same NVFP4 latent rows,
+    routing, gates and upstream gradient. Outputs are BF16 (dz, dW1, dW2) or
+    fp32 from BF16 operands (dgate): checked beyond half a BF16 step against
+    the oracle, with the 8e-2 * RMS bar of the NVFP4 forward (a quantiser
+    decision can flip where the GPU's fp32 input sits within a rounding of a
+    threshold), and the whole within 1e-2 in relative Frobenius norm."""
+    from gpu_util import bf16_parity, quantize_dev
+    l = m = 256
+    rng = np.random.default_rng(T * 7 + N)
+    zb = LI.bf16_bits(rng.standard_normal((T, l)))
+    w1b = LI.bf16_bits(rng.standard_normal((N, m, l)) / np.sqrt(l))
+    w2b = LI.bf16_bits(rng.standard_normal((N, l, m)) / np.sqrt(m))
+    dcb = LI.bf16_bits(rng.standard_normal((T, l)) * 0.05)
+    logits = rng.standard_normal((T, N))
+    if zero_expert:
+        logits[:, N - 1] = -50.0                            # an expert no token reaches
+    idx, gates = O.route_topk(logits, K)
+    s_a = float(np.float32(20.0 / 2688.0))                  # static global scale of a
+    seed = 0x5EED
+    z, w1, w2, dc = (O.from_bf16_bits(b) for b in (zb, w1b, w2b, dcb))
+
+    # oracle, on the NVFP4 latent rows the GPU quantiser produces (bit-exact, pinned elsewhere)
+    zq, _ = O.nvfp4_fake_quant(z)
+    ref = B.routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, SIGNS, seed, s_a)
+
+    # device: quantise z, permute rows (NVFP4 codes + tiled scales) and gates
+    cfg = L.config(T=T, d=l, l=l, N=N, K=K, m=m, expert=L.NVFP4)
+    P = L.padded_rows(cfg)
+    codes, sf, zgs = quantize_dev(to_dev(zb, "bf16"), T, l)
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device="cuda")
+    offsets, poff, perm_src, inv_perm = i32(N + 1), i32(N + 1), i32(T * K), i32(T * K)
+    zp = torch.zeros((P, l // 2), dtype=torch.uint8, device="cuda")
+    zp_sf = torch.zeros(P * l // 16, dtype=torch.uint8, device="cuda")
+    pgate = torch.zeros(P, dtype=torch.float32, device="cuda")
+    idx_d = torch.from_numpy(idx.astype(np.int32)).cuda()
+    gates_d = torch.from_numpy(gates.astype(np.float32)).cuda()
+    ws = L.workspace(cfg, L.OP_PERMUTE)
+    L.permute(cfg, idx_d, offsets, perm_src, inv_perm, poff, codes, l // 2, zp, sf, zp_sf, gates_d, pgate, ws=ws)
+    assert L.read_device_error(ws)[0] == L.OK
+    # each padded row's upstream gradient: dc of its token
+    counts = np.bincount(idx.reshape(-1), minlength=N).astype(np.int32)
+    off_h, poff_h, src_h = offsets.cpu().numpy(), poff.cpu().numpy(), perm_src.cpu().numpy()
+    row_of = np.empty(T * K, dtype=np.int64)                # slot f -> padded row
+    for r, f in enumerate(src_h):
+        e = idx.reshape(-1)[f]
+        row_of[f] = r - off_h[e] + poff_h[e]
+    dy_pad = np.zeros((P, l), dtype=np.uint16)
+    dy_pad[row_of] = dcb[np.arange(T * K) // K]
+    dy = to_dev(dy_pad, "bf16")
+    a_g = torch.tensor([s_a], dtype=torch.float32, device="cuda")
+    dz = torch.zeros((P, l), dtype=torch.bfloat16, device="cuda")
+    dgate = torch.zeros(P, dtype=torch.float32, device="cuda")
+    dw1 = torch.empty((N, m, l), dtype=torch.bfloat16, device="cuda")
+    dw2 = torch.empty((N, l, m), dtype=torch.bfloat16, device="cuda")
+    bws = L.expert_backward_nvfp4(cfg, counts, offsets, poff, zp, zp_sf, zgs, to_dev(w1b, "bf16"),
+                                  to_dev(w2b, "bf16"), a_g, pgate, dy, seed, SIGN_BITS, dz, dgate, dw1, dw2)
+    st, info = L.read_device_error(bws)
+    assert st == L.OK, (L.status_string(st), hex(info))
+
+    # back to tokens: dz summed over each token's slots, dgate per (token, k)
+    dz_rows = dz.float().cpu().numpy().astype(np.float64)
+    dz_tok = np.zeros((T, l))
+    np.add.at(dz_tok, np.arange(T * K) // K, dz_rows[row_of])
+    dgate_tk = dgate.cpu().numpy().astype(np.float64)[row_of].reshape(T, K)
+    got = dict(dz=dz_tok, dgate=dgate_tk, dw1=dw1.float().cpu().numpy().astype(np.float64),
+               dw2=dw2.float().cpu().numpy().astype(np.float64))
+    exact = B.routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, SIGNS, seed, s_a, quantize=False)
+    for name in ("dz", "dgate", "dw1", "dw2"):
+        g, r = got[name], ref[name]
+        excess, raw = bf16_parity(g, r, O.round_bf16(r))
+        fro = np.linalg.norm(g - r) / np.linalg.norm(r)
+        qerr = np.linalg.norm(exact[name] - r) / np.linalg.norm(r)
+        print(f"experts backward {name}: excess {excess:.3e} * RMS, raw {raw:.3e} * RMS, rel {fro:.3e} "
+              f"(recipe vs unquantised: {qerr:.3e})")
+        assert excess <= 8e-2, name
+        assert fro <= 1e-2, name
+        assert fro < 0.2 * qerr or name == "dgate", name   # far closer to the oracle than to the unquantised value
+    if zero_expert:
+        assert not np.any(got["dw1"][N - 1]) and not np.any(got["dw2"][N - 1])
