@@ -95,11 +95,6 @@ struct Tc2Smem {
   static constexpr int kABytes = 128 * 128;   // 128 weight rows x 64 bf16 (one K atom)
   static constexpr int kBBytes = 128 * 128;   // up to 128 token rows x 64 bf16
   static constexpr int kAtoms = 2;            // 64-wide K atoms per stage (measured 9% faster than 1)
-  // tiles of at most 64 tokens stream their weights from HBM with little math
-  // per byte: their stages hold three K atoms (the B atoms, at most 32 rows a
-  // CTA, packed at 4 KB), half as many bytes again in flight
-  static constexpr int kAtomsThin = 3;
-  static constexpr int kBBytesThin = 32 * 128;
   static constexpr int kStageBytes = kAtoms * (kABytes + kBBytes);   // A atoms, then B atoms
   static constexpr int kStages = 6 / kAtoms;
   static constexpr int kBarOffset = kStages * kStageBytes;
@@ -111,7 +106,6 @@ struct Tc2Smem {
   // once, so that no role waits on a global load at a tile boundary
   static constexpr int kExpertOffset = kEpiOffset + 4 * 32 * 32 * 2;
   static constexpr int kBytes = kExpertOffset + 2 * kMaxGroups * 4 + 1024;   // +1024 alignment slack
-  static_assert(kAtomsThin * (kABytes + kBBytesThin) <= kStageBytes, "thin stage exceeds a stage");
   static constexpr int kTmemCols = 512;       // two 256-column accumulators
   static constexpr int kTokens = 256;         // tokens per tile (MMA N <= 256)
 };
@@ -290,14 +284,11 @@ __global__ void __launch_bounds__(192, 1)
             ti.extra ? p.rows_x > S::kTokens
                      : ti.act0 + S::kTokens < epoff[ti.expert] + ecount[ti.expert];
         const uint64_t pa = wshared ? pol_keep : pol_stream;
-        const bool thin = ti.n <= 64;
-        const int atoms = thin ? S::kAtomsThin : S::kAtoms;
-        const int bpitch = thin ? S::kBBytesThin : S::kBBytes;
-        for (int kb = 0; kb < ti.kblocks; kb += atoms) {
+        for (int kb = 0; kb < ti.kblocks; kb += S::kAtoms) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x2100 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStageBytes;
-          uint8_t* sb = sa + atoms * S::kABytes;
-          const int na = min(atoms, ti.kblocks - kb);   // K atoms in this stage
+          uint8_t* sb = sa + S::kAtoms * S::kABytes;
+          const int na = min(S::kAtoms, ti.kblocks - kb);   // K atoms in this stage
           if (leader) mbar_arrive_expect_tx(&full[stage], na * (2 * S::kABytes + ti.n * 128));
           const uint32_t bar = cluster_map(smem_u32(&full[stage]), 0);
           const int kg = ti.extra ? p.kgroup_x : 0;   // K split over the weight tensor's groups
@@ -310,7 +301,7 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < 4; ++i) {
               const int box = 128 >> i;
               if (half - done >= box) {
-                tma_load_3d_pair(sb + q * bpitch + done * 128, bmap0 + i, bar, k, b_row0 + done, 0, pol_norm);
+                tma_load_3d_pair(sb + q * S::kBBytes + done * 128, bmap0 + i, bar, k, b_row0 + done, 0, pol_norm);
                 done += box;
               }
             }
@@ -341,20 +332,17 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
         const uint32_t idesc = idesc_bf16_f32(256, ti.n);
-        const bool thin = ti.n <= 64;
-        const int atoms = thin ? S::kAtomsThin : S::kAtoms;
-        const int bpitch = thin ? S::kBBytesThin : S::kBBytes;
-        for (int kb = 0; kb < ti.kblocks; kb += atoms) {
+        for (int kb = 0; kb < ti.kblocks; kb += S::kAtoms) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x2300 + stage)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * S::kStageBytes);
-          const uint32_t sb = sa + atoms * S::kABytes;
-          const int na = min(atoms, ti.kblocks - kb);
+          const uint32_t sb = sa + S::kAtoms * S::kABytes;
+          const int na = min(S::kAtoms, ti.kblocks - kb);
           for (int q = 0; q < na; ++q)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_pair(d_tmem, sdesc_kmajor_sw128(sa + q * S::kABytes + kk * 32),
-                            sdesc_kmajor_sw128(sb + q * bpitch + kk * 32), idesc, (kb | q | kk) != 0 ? 1u : 0u);
+                            sdesc_kmajor_sw128(sb + q * S::kBBytes + kk * 32), idesc, (kb | q | kk) != 0 ? 1u : 0u);
           any = true;
           mma_commit_pair(&empty[stage], 0x3);
           if (++stage == S::kStages) { stage = 0; phase ^= 1; }
