@@ -427,8 +427,8 @@ lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* p
  * rows (zero rows up to R = n rounded up to 16 wherever a quantiser runs
  * along the rows):
  *   W1q, W2q = the BF16 masters w1[e] [m][l], w2[e] [l][m] quantised with
- *     16 x 16 blocks (current amax); h = zq W1q^T (BF16), aq = NVFP4(relu(h)^2)
- *     with the static global scale a_global, o = aq W2q^T (BF16);
+ *     16 x 16 blocks (current amax); h = zq W1q^T (fp32), aq = NVFP4(relu(h)^2)
+ *     with the static global scale a_global, o = aq W2q^T (fp32);
  *   dgate[r] = dy[r] . o[r];  do = gate[r] dy[r]  (fp32);
  *   dA = SR(do) W2q;  dh = dA * 2 max(h, 0);  dz = SR(dh) W1q;
  *   dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T;  dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T;

@@ -84,12 +84,14 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   p.out_sf = L.out_sf;
   p.ld_out = L.ld_out;
   p.out_vec32 = (reinterpret_cast<uintptr_t>(L.out) % 32 == 0) && (L.ld_out * 2) % 32 == 0;
+  if (L.f32_out && ((reinterpret_cast<uintptr_t>(L.out) & 15) || L.ld_out % 4)) return LMOE_ERR_INVALID_ARG;
   p.err = DevErr{err_word};
   const int sms = device_sm_count();
   const int64_t tiles = (L.a_rows / 128) * (L.cols / 256);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   if (grid <= 0) return LMOE_OK;
   if (L.quant_out) return launch_fp4<FP4_EPI_SQRELU_QUANT>(ma, mb, p, grid, stream);
+  if (L.f32_out) return launch_fp4<FP4_EPI_F32>(ma, mb, p, grid, stream);
   return launch_fp4<FP4_EPI_GATE_BF16>(ma, mb, p, grid, stream);
 }
 

@@ -25,7 +25,9 @@
 
 namespace lmoe {
 
-enum Fp4Epi : int { FP4_EPI_SQRELU_QUANT = 0, FP4_EPI_GATE_BF16 = 1 };
+// FP4_EPI_F32: out = acc * scales in fp32 (the training recipe's backward
+// feeds such results to its stochastic quantisers, which need them unrounded)
+enum Fp4Epi : int { FP4_EPI_SQRELU_QUANT = 0, FP4_EPI_GATE_BF16 = 1, FP4_EPI_F32 = 2 };
 
 struct Fp4Params {
   int rows;                   // padded rows of A (a multiple of 128)
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
       const long long row = act0 + r;
       const bool row_ok = r < act_n;
       // per-tile scalars fetched before the accumulator is ready
-      const float gate = (EPI == FP4_EPI_GATE_BF16 && p.row_scale && row_ok) ? __ldg(p.row_scale + row) : 1.0f;
+      const float gate = (EPI != FP4_EPI_SQRELU_QUANT && p.row_scale && row_ok) ? __ldg(p.row_scale + row) : 1.0f;
       const float in_s = p.in_scale_grouped ? __ldg(p.in_scale + e) : in_s0;
       const float scale = __fmul_rn(in_s, __ldg(p.w_scale + e));
       if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag, p.err, 0x1400 + buf)) break;
@@ -357,6 +359,14 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
           const int j0 = col0 / 16;
           p.out_sf[fp4_sf_offset(row, j0, groups64_out)] = static_cast<uint8_t>(s0);
           p.out_sf[fp4_sf_offset(row, j0 + 1, groups64_out)] = static_cast<uint8_t>(s1);
+        } else if (EPI == FP4_EPI_F32) {
+          float* o = reinterpret_cast<float*>(p.out) + row * p.ld_out + col0;
+          const float sg = scale * gate;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(o + j) =
+                make_float4(__uint_as_float(v[j]) * sg, __uint_as_float(v[j + 1]) * sg,
+                            __uint_as_float(v[j + 2]) * sg, __uint_as_float(v[j + 3]) * sg);
         } else {
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
           const float sg = scale * gate;

@@ -118,6 +118,7 @@ struct Fp4Launch {
   const float* out_scale = nullptr;  // device scalar (quant_out)
   const float* row_scale = nullptr;  // gates (GEMM 2)
   int quant_out = 0;                 // 1: relu^2 + NVFP4 codes/scales out; 0: BF16 out * gate
+  int f32_out = 0;                   // with quant_out 0: fp32 out * gate instead of BF16
   void* out = nullptr;
   uint8_t* out_sf = nullptr;
   int64_t ld_out = 0;

@@ -8,7 +8,9 @@
 //
 // Per expert e, over its n slot rows (padded with zero rows to R, a multiple
 // of 16, wherever a quantiser runs along the tokens):
-//   h = zq W1q^T, aq = NVFP4(relu(h)^2, s_a), o = aq W2q^T  (recomputed)
+//   h = zq W1q^T, aq = NVFP4(relu(h)^2, s_a), o = aq W2q^T  (recomputed;
+//   h, o and dA kept in fp32: a stochastic quantiser turns any rounding of
+//   its input into changed codes, so its inputs stay unrounded)
 //   dgate = dy . o per row, do = gate * dy
 //   dA = SR(do) W2q,          dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T
 //   dh = dA * 2 max(h, 0)
@@ -35,7 +37,7 @@ int64_t ceil_to(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 // do[r][:] = gate * dy for r < n (fp32; rows n..R-1 zero); dgate[r] = dy . o.
 // A block per row r < R.
 __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const __nv_bfloat16* __restrict__ dy,
-                                                              const __nv_bfloat16* __restrict__ o,
+                                                              const float* __restrict__ o,
                                                               const float* __restrict__ gate, int64_t row0, int n,
                                                               int l, float* __restrict__ d_o,
                                                               float* __restrict__ dgate) {
@@ -52,7 +54,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const __nv_bfloat16
   float dot = 0.0f;
   for (int j = threadIdx.x; j < l; j += blockDim.x) {
     const float d = __bfloat162float(dy[row * l + j]);
-    dot = fmaf(d, __bfloat162float(o[row * l + j]), dot);
+    dot = fmaf(d, o[row * l + j], dot);
     out[j] = __fmul_rn(g, d);
   }
 #pragma unroll
@@ -67,8 +69,8 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const __nv_bfloat16
 }
 
 // dh[r][c] = dA[r][c] * 2 max(h[row0 + r][c], 0) for r < n, 0 for n <= r < R.
-__global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const __nv_bfloat16* __restrict__ dA,
-                                                            const __nv_bfloat16* __restrict__ h, int64_t row0,
+__global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const float* __restrict__ dA,
+                                                            const float* __restrict__ h, int64_t row0,
                                                             int n, int R, int m, float* __restrict__ dh) {
   pdl_begin();
   const int64_t total = static_cast<int64_t>(R) * m;
@@ -77,8 +79,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const __nv_bfloat16* 
     const int64_t r = i / m, c = i % m;
     float v = 0.0f;
     if (r < n) {
-      const float hv = __bfloat162float(h[(row0 + r) * m + c]);
-      v = __bfloat162float(dA[r * m + c]) * (2.0f * fmaxf(hv, 0.0f));
+      v = dA[r * m + c] * (2.0f * fmaxf(h[(row0 + r) * m + c], 0.0f));
     }
     dh[i] = v;
   }
@@ -170,17 +171,17 @@ BwLayout bw_layout(const lmoe_config* c, const int32_t* counts) {
   L.wtc = take(l * m / 2);
   L.wts = take(l * m / 16);
   L.wtg = take(4);
-  L.h = take(P * m * 2);
+  L.h = take(P * m * 4);
   L.aqc = take(P * m / 2);
   L.aqs = take(P * m / 16);
-  L.o = take(P * l * 2);
+  L.o = take(P * l * 4);
   L.d_o = take(Rmax * l * 4);
   L.dh = take(Rmax * m * 4);
   L.deq = take(Rmax * lm * 4);
   L.qac = take(L.R128max * lm / 2);
   L.qas = take(L.R128max * lm / 16);
   L.qag = take(4);
-  L.dA = take(L.R128max * m * 2);
+  L.dA = take(L.R128max * m * 4);
   L.t1c = take(lm * L.K256max / 2);
   L.t1s = take(lm * L.K256max / 16);
   L.t1g = take(4);
@@ -296,14 +297,16 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
   f.w_scale = at<float>(ws, L.w1g);
   f.out = at<void>(ws, L.h);
   f.ld_out = m;
+  f.f32_out = 1;
   if (L.P > 0 && (st = fp4_gemm(f, err, s)) != LMOE_OK) return st;
   Fp4Launch fq = f;
   fq.quant_out = 1;
+  fq.f32_out = 0;
   fq.out_scale = a_global;
   fq.out = at<void>(ws, L.aqc);
   fq.out_sf = at<uint8_t>(ws, L.aqs);
   if (L.P > 0 && (st = fp4_gemm(fq, err, s)) != LMOE_OK) return st;
-  Fp4Launch f2 = f;
+  Fp4Launch f2 = f;   // fp32 out, as f
   f2.a_codes = at<uint8_t>(ws, L.aqc);
   f2.a_sf = at<uint8_t>(ws, L.aqs);
   f2.b_codes = at<uint8_t>(ws, L.w2c);
@@ -326,14 +329,14 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
   uint8_t *t1c = at<uint8_t>(ws, L.t1c), *t1s = at<uint8_t>(ws, L.t1s);
   uint8_t *t2c = at<uint8_t>(ws, L.t2c), *t2s = at<uint8_t>(ws, L.t2s);
   float *t1g = at<float>(ws, L.t1g), *t2g = at<float>(ws, L.t2g);
-  __nv_bfloat16* dA = at<__nv_bfloat16>(ws, L.dA);
-  const __nv_bfloat16* h = at<__nv_bfloat16>(ws, L.h);
-  const __nv_bfloat16* o = at<__nv_bfloat16>(ws, L.o);
+  float* dA = at<float>(ws, L.dA);
+  const float* h = at<float>(ws, L.h);
+  const float* o = at<float>(ws, L.o);
 
   // a single-group GEMM out[rows][cols] = A[rows][k] . B[cols][k]^T (BF16 out)
   auto gemm1 = [&](const uint8_t* ac, const uint8_t* as, const float* ag, int64_t a_rows, const int32_t* off,
                    const uint8_t* bc, const uint8_t* bs, const float* bg, int64_t cols, int64_t k, void* out,
-                   int64_t ld) {
+                   int64_t ld, int f32) {
     Fp4Launch g;
     g.a_codes = ac;
     g.a_sf = as;
@@ -349,6 +352,7 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     g.w_scale = bg;
     g.out = out;
     g.ld_out = ld;
+    g.f32_out = f32;
     return fp4_gemm(g, err, s);
   };
 
@@ -377,7 +381,7 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     if ((st = launch_nvfp4_quantize_ex(W2 + e * l * m, LMOE_BF16, l, m, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr, wtc, wts,
                                        wtg, tiled2d, part, s)) != LMOE_OK)
       break;
-    if ((st = gemm1(qac, qas, qag, R128, off_e, wtc, wts, wtg, m, l, dA, m)) != LMOE_OK) break;
+    if ((st = gemm1(qac, qas, qag, R128, off_e, wtc, wts, wtg, m, l, dA, m, 1)) != LMOE_OK) break;
     // dh
     launch_k(bw_dh_kernel, dim3(grid_for(static_cast<int64_t>(R) * m)), dim3(kBwThreads), 0, s, dA, h, p0, n, R,
              static_cast<int>(m), dh);
@@ -395,7 +399,7 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
                                        nullptr, t2c, t2s, t2g, LMOE_SF_MMA_TILED, part, s, K256)) != LMOE_OK)
       break;
     if ((st = gemm1(t1c, t1s, t1g, l, off_l, t2c, t2s, t2g, m, K256, static_cast<__nv_bfloat16*>(dw2) + e * l * m,
-                    m)) != LMOE_OK)
+                    m, 0)) != LMOE_OK)
       break;
     // first GEMM, dgrad: dz = SR(dh) W1q  (W1^T [l][m] with 16 x 16 blocks), into the expert's slot rows
     if ((st = launch_nvfp4_quantize_ex(dh, LMOE_F32, R, m, LMOE_QX_SR, rht_signs, seed, st_dg1, nullptr, qac, qas,
@@ -404,8 +408,8 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     if ((st = launch_nvfp4_quantize_ex(W1 + e * m * l, LMOE_BF16, m, l, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr, wtc, wts,
                                        wtg, tiled2d, part, s)) != LMOE_OK)
       break;
-    if ((st = gemm1(qac, qas, qag, R128, off_e, wtc, wts, wtg, l, m, static_cast<__nv_bfloat16*>(dz) + p0 * l, l)) !=
-        LMOE_OK)
+    if ((st = gemm1(qac, qas, qag, R128, off_e, wtc, wts, wtg, l, m, static_cast<__nv_bfloat16*>(dz) + p0 * l, l,
+                    0)) != LMOE_OK)
       break;
     // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
     launch_k(bw_dequant_kernel, dim3(grid_for(static_cast<int64_t>(R) * l / 2)), dim3(kBwThreads), 0, s, z_codes,
@@ -418,7 +422,7 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     if ((st = launch_nvfp4_quantize_ex(deq, LMOE_F32, R, l, LMOE_QX_TRANSPOSE | LMOE_QX_RHT, rht_signs, seed, 0,
                                        nullptr, t2c, t2s, t2g, LMOE_SF_MMA_TILED, part, s, K256)) != LMOE_OK)
       break;
-    st = gemm1(t1c, t1s, t1g, m, off_m, t2c, t2s, t2g, l, K256, static_cast<__nv_bfloat16*>(dw1) + e * m * l, l);
+    st = gemm1(t1c, t1s, t1g, m, off_m, t2c, t2s, t2g, l, K256, static_cast<__nv_bfloat16*>(dw1) + e * m * l, l, 0);
   }
   if (st != LMOE_OK) return st;
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
