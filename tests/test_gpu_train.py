@@ -172,11 +172,20 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
     """lmoe_expert_backward_nvfp4 (recomputed NVFP4 forward, SR dgrad, RHT +
     SR wgrad for both expert GEMMs, every step a kernel of the library) against
     the oracle's routed_experts_backward_nvfp4 on the same NVFP4 latent rows,
-    routing, gates and upstream gradient. Outputs are BF16 (dz, dW1, dW2) or
-    fp32 from BF16 operands (dgate): checked beyond half a BF16 step against
-    the oracle, with the 8e-2 * RMS bar of the NVFP4 forward (a quantiser
-    decision can flip where the GPU's fp32 input sits within a rounding of a
-    threshold), and the whole within 1e-2 in relative Frobenius norm."""
+    routing, gates and upstream gradient.
+
+    The GPU forms a stochastic quantiser's input (dh = dA * 2 relu(h)) with
+    fp32 GEMMs where the oracle is exact, so an element whose value sits
+    within that rounding (~2^-20 relative) of its uniform's threshold takes the
+    other grid neighbour: a probability of ~1e-5 per element. In dz and dgate
+    such a flip is one term of a long sum; in a weight gradient it moves one
+    whole row (a flip in the gradient operand) or column (in the activation
+    operand) of that expert's dW by one quantisation step times the other
+    operand, up to several tenths of RMS(dW). So: dz and dgate within the NVFP4
+    forward's 8e-2 * RMS bar beyond half a BF16 step everywhere; dW within it
+    outside at most two such lines per expert; every output within 1e-2 in
+    relative Frobenius norm, and at least 5x closer to the oracle than the
+    oracle is to the unquantised gradient (dz, dW)."""
     from gpu_util import bf16_parity, quantize_dev
     l = m = 256
     rng = np.random.default_rng(T * 7 + N)
@@ -238,6 +247,7 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
     got = dict(dz=dz_tok, dgate=dgate_tk, dw1=dw1.float().cpu().numpy().astype(np.float64),
                dw2=dw2.float().cpu().numpy().astype(np.float64))
     exact = B.routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, SIGNS, seed, s_a, quantize=False)
+    from gpu_util import bf16_ulp
     for name in ("dz", "dgate", "dw1", "dw2"):
         g, r = got[name], ref[name]
         excess, raw = bf16_parity(g, r, O.round_bf16(r))
@@ -245,8 +255,20 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
         qerr = np.linalg.norm(exact[name] - r) / np.linalg.norm(r)
         print(f"experts backward {name}: excess {excess:.3e} * RMS, raw {raw:.3e} * RMS, rel {fro:.3e} "
               f"(recipe vs unquantised: {qerr:.3e})")
-        assert excess <= 8e-2, name
         assert fro <= 1e-2, name
-        assert fro < 0.2 * qerr or name == "dgate", name   # far closer to the oracle than to the unquantised value
+        if name in ("dz", "dgate"):
+            assert excess <= 8e-2, name
+        else:
+            # elements beyond the bar, per expert: covered by at most two rows or two columns
+            rms = np.sqrt(np.mean(O.round_bf16(r) ** 2))
+            over = (np.abs(g - r) - bf16_ulp(O.round_bf16(r)) / 2) > 8e-2 * rms
+            for e in range(N):
+                rows, cols = np.nonzero(over[e])
+                lines = min(np.unique(rows).size, np.unique(cols).size)
+                if lines:
+                    print(f"  {name}[{e}]: {rows.size} elements beyond the bar on {lines} line(s)")
+                assert lines <= 2, (name, e)
+        if name != "dgate":
+            assert fro < 0.2 * qerr, name   # far closer to the oracle than to the unquantised value
     if zero_expert:
         assert not np.any(got["dw1"][N - 1]) and not np.any(got["dw2"][N - 1])
