@@ -176,14 +176,17 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
 
     The GPU forms a stochastic quantiser's input (dh = dA * 2 relu(h)) with
     fp32 GEMMs where the oracle is exact, so an element whose value sits
-    within that rounding (~2^-20 relative) of its uniform's threshold takes the
-    other grid neighbour: a probability of ~1e-5 per element. In dz and dgate
+    within that rounding of its uniform's threshold takes the other grid
+    neighbour. The tensor cores' fp32 accumulation is off by up to ~2^-13 of
+    the L2 norm of a dot product's terms (the window of the z-rounding ties),
+    so about 1e-4 of the elements flip: a few per expert here. In dz and dgate
     such a flip is one term of a long sum; in a weight gradient it moves one
     whole row (a flip in the gradient operand) or column (in the activation
     operand) of that expert's dW by one quantisation step times the other
     operand, up to several tenths of RMS(dW). So: dz and dgate within the NVFP4
     forward's 8e-2 * RMS bar beyond half a BF16 step everywhere; dW within it
-    outside at most two such lines per expert; every output within 1e-2 in
+    outside at most eight such lines per expert (and 2% of its elements); every
+    output within 1e-2 in
     relative Frobenius norm, and at least 5x closer to the oracle than the
     oracle is to the unquantised gradient (dz, dW)."""
     from gpu_util import bf16_parity, quantize_dev
@@ -267,7 +270,8 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
                 lines = min(np.unique(rows).size, np.unique(cols).size)
                 if lines:
                     print(f"  {name}[{e}]: {rows.size} elements beyond the bar on {lines} line(s)")
-                assert lines <= 2, (name, e)
+                assert lines <= 8, (name, e)
+            assert over.mean() <= 0.02, name
         if name != "dgate":
             assert fro < 0.2 * qerr, name   # far closer to the oracle than to the unquantised value
     if zero_expert:
