@@ -441,7 +441,8 @@ lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* p
  *  z_codes [P][l/2], z_sf (MMA-tiled over the P padded rows), z_global
  *    (device F32): the NVFP4 latent rows as lmoe_permute moves them.
  *  w1, w2: BF16 masters [N][m][l], [N][l][m]. a_global: device F32.
- *  gate [P] F32, dy [P][l] BF16: each slot row's gate and upstream gradient.
+ *  gate [P] F32, dy [P][l] F32: each slot row's gate and upstream gradient
+ *    (fp32: the stochastic quantiser of do = gate * dy must see it unrounded).
  *  Outputs (device): dz [P][l] BF16 (padding rows unspecified), dgate [P] F32
  *    (set for real rows only), dw1 [N][m][l] and dw2 [N][l][m] BF16.
  *  l and m multiples of 256; 16-byte aligned buffers; ws of at least
@@ -454,7 +455,7 @@ size_t lmoe_expert_backward_nvfp4_workspace(const lmoe_config* cfg, const int32_
 lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* counts, const int32_t* offsets,
                                        const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
                                        const float* z_global, const void* w1, const void* w2,
-                                       const float* a_global, const float* gate, const void* dy, uint64_t seed,
+                                       const float* a_global, const float* gate, const float* dy, uint64_t seed,
                                        uint32_t rht_signs, void* dz, float* dgate, void* dw1, void* dw2, void* ws,
                                        size_t ws_bytes, void* stream);
 

@@ -36,7 +36,7 @@ int64_t ceil_to(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 // do[r][:] = gate * dy for r < n (fp32; rows n..R-1 zero); dgate[r] = dy . o.
 // A block per row r < R.
-__global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const __nv_bfloat16* __restrict__ dy,
+__global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const float* __restrict__ dy,
                                                               const float* __restrict__ o,
                                                               const float* __restrict__ gate, int64_t row0, int n,
                                                               int l, float* __restrict__ d_o,
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const __nv_bfloat16
   const float g = __ldg(gate + row);
   float dot = 0.0f;
   for (int j = threadIdx.x; j < l; j += blockDim.x) {
-    const float d = __bfloat162float(dy[row * l + j]);
+    const float d = dy[row * l + j];
     dot = fmaf(d, o[row * l + j], dot);
     out[j] = __fmul_rn(g, d);
   }
@@ -219,7 +219,7 @@ size_t lmoe_expert_backward_nvfp4_workspace(const lmoe_config* cfg, const int32_
 lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* counts, const int32_t* offsets,
                                        const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
                                        const float* z_global, const void* w1, const void* w2,
-                                       const float* a_global, const float* gate, const void* dy, uint64_t seed,
+                                       const float* a_global, const float* gate, const float* dy, uint64_t seed,
                                        uint32_t rht_signs, void* dz, float* dgate, void* dw1, void* dw2, void* ws,
                                        size_t ws_bytes, void* stream) {
   if (!cfg || !counts || !offsets || !padded_offsets || !z_codes || !z_sf || !z_global || !w1 || !w2 ||
@@ -233,9 +233,29 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     if (counts[e] < 0) return LMOE_ERR_INVALID_ARG;
   if (!a16(z_codes) || !a16(z_sf) || !a16(w1) || !a16(w2) || !a16(dy) || !a16(dz) || !a16(dw1) || !a16(dw2))
     return LMOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < bw_layout(cfg, counts).total) return LMOE_ERR_WORKSPACE;
+  return expert_backward_core(cfg, counts, offsets, padded_offsets, z_codes, z_sf, z_global, w1, w2, a_global, gate,
+                              dy, seed, rht_signs, dz, dgate, dw1, dw2, ws, nullptr,
+                              static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace lmoe {
+
+size_t expert_backward_ws(const lmoe_config* cfg, const int32_t* counts) { return bw_layout(cfg, counts).total; }
+
+// The routed experts' backward (see lmoe_expert_backward_nvfp4), arguments
+// checked by the caller; ws holds at least expert_backward_ws() bytes. With
+// o_out, the recomputed expert outputs o (fp32, [P][l]) are copied there.
+lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, const int32_t* offsets,
+                                 const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
+                                 const float* z_global, const void* w1, const void* w2, const float* a_global,
+                                 const float* gate, const float* dy, uint64_t seed, uint32_t rht_signs, void* dz,
+                                 float* dgate, void* dw1, void* dw2, void* ws, float* o_out, cudaStream_t s) {
+  const int N = cfg->N;
+  const int64_t l = cfg->l, m = cfg->m;
   const BwLayout L = bw_layout(cfg, counts);
-  if (!ws || ws_bytes < L.total) return LMOE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = at<uint32_t>(ws, L.err);
   double* part = at<double>(ws, L.part);
   lmoe_status st = LMOE_OK;
@@ -371,7 +391,7 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     const uint32_t st_dg1 = 4u * e + 0, st_wg1 = 4u * e + 1, st_dg2 = 4u * e + 2, st_wg2 = 4u * e + 3;
 
     // do, dgate
-    launch_k(bw_prep_kernel, dim3(R), dim3(kBwThreads), 0, s, static_cast<const __nv_bfloat16*>(dy), o, gate, p0, n,
+    launch_k(bw_prep_kernel, dim3(R), dim3(kBwThreads), 0, s, static_cast<const float*>(dy), o, gate, p0, n,
              static_cast<int>(l), d_o, dgate);
     count_launch();
     // second GEMM, dgrad: dA = SR(do) W2q  (W2^T [m][l] with 16 x 16 blocks)
@@ -425,7 +445,10 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     st = gemm1(t1c, t1s, t1g, m, off_m, t2c, t2s, t2g, l, K256, static_cast<__nv_bfloat16*>(dw1) + e * m * l, l, 0);
   }
   if (st != LMOE_OK) return st;
+  if (o_out && L.P > 0 &&
+      cudaMemcpyAsync(o_out, o, static_cast<size_t>(L.P) * l * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return LMOE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
-}  // extern "C"
+}  // namespace lmoe

@@ -229,9 +229,9 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
     for r, f in enumerate(src_h):
         e = idx.reshape(-1)[f]
         row_of[f] = r - off_h[e] + poff_h[e]
-    dy_pad = np.zeros((P, l), dtype=np.uint16)
-    dy_pad[row_of] = dcb[np.arange(T * K) // K]
-    dy = to_dev(dy_pad, "bf16")
+    dy_pad = np.zeros((P, l), dtype=np.float32)
+    dy_pad[row_of] = dc[np.arange(T * K) // K]
+    dy = to_dev(dy_pad, "f32")
     a_g = torch.tensor([s_a], dtype=torch.float32, device="cuda")
     dz = torch.zeros((P, l), dtype=torch.bfloat16, device="cuda")
     dgate = torch.zeros(P, dtype=torch.float32, device="cuda")
