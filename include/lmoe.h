@@ -459,6 +459,55 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
                                        uint32_t rht_signs, void* dz, float* dgate, void* dw1, void* dw2, void* ws,
                                        size_t ws_bytes, void* stream);
 
+/* Gradients of the layer, written by lmoe_backward_nvfp4 (device buffers,
+ * BF16 unless noted; the ones a configuration does not have may be NULL). */
+typedef struct {
+  void* dx;             /* [T][d] */
+  void* dw_router;      /* [N][d] */
+  float* drouter_bias;  /* [N] F32; needed with a router bias */
+  void* dw_down;        /* [l][d]; latent projections only */
+  void* dw_up;          /* [d][l]; latent projections only */
+  void* dw1;            /* [N][m][l] */
+  void* dw2;            /* [N][l][m] */
+  void* dws1;           /* [S][m_shared][d]; with shared experts */
+  void* dws2;           /* [S][d][m_shared] */
+} lmoe_grads;
+
+/* The layer's backward pass with its routed experts trained under the NVFP4
+ * recipe (greeksharifa page, sections 2.2 "LatentMoE" and 2.4 "NVFP4
+ * Training"; notes.yuuk.io page, section 4). The forward pieces the gradients
+ * need are recomputed from x: router logits (+ bias) and the top-K gates, z
+ * (down-projection), z quantised to NVFP4 with its current amax, the slots
+ * permuted by expert. Then, for the upstream gradient dout [T][d]:
+ *   dc = dout W_up (identity projections: dout);
+ *   the routed experts: lmoe_expert_backward_nvfp4 on the slot rows (BF16
+ *     masters w1, w2; a_global, seed and rht_signs as there), giving dz per
+ *     slot, dgate, dW1, dW2 and the experts' outputs o;
+ *   c = sum_k g_k o_k;  dW_up = dout^T c;
+ *   dsel_k = g_k (dgate_k - sum_j g_j dgate_j) at the K chosen experts (top-K
+ *     selection passes no gradient), dW_router = dsel^T x, drouter_bias =
+ *     sum over tokens of dsel;
+ *   dz_t = sum_k dz(t, k);  dW_down = dz^T x;
+ *   each shared expert s: pre = x Ws1_s^T, dWs2_s = dout^T relu(pre)^2,
+ *     dpre = (dout Ws2_s) 2 max(pre, 0), dWs1_s = dpre^T x;
+ *   dx = dsel W_router + dz W_down + sum_s dpre_s Ws1_s (dz W_down -> dz with
+ *     identity projections).
+ * The router, the projections and the shared experts (kept in higher
+ * precision by the recipe) are BF16 tensor-core GEMMs with fp32 accumulation.
+ *  cfg: act and expert BF16 (w->w1, w->w2 are the BF16 masters), no
+ *    LMOE_FLAG_SHARED_FP8; d % 64, l and m multiples of 256, N % 8,
+ *    m_shared % 64. w: the forward's weights. x, dout [T][d] BF16.
+ *  The call synchronises its stream once (the experts' row counts are read
+ *  on the host). ws: lmoe_backward_nvfp4_workspace(cfg) bytes, the first 256
+ *  zeroed before first use (the error word).
+ *  Errors: LMOE_ERR_INVALID_ARG for null or unaligned pointers and missing
+ *  weights or gradients; LMOE_ERR_UNSUPPORTED for the dtype, flag and size
+ *  conditions above; LMOE_ERR_WORKSPACE; LMOE_ERR_CUDA. */
+size_t lmoe_backward_nvfp4_workspace(const lmoe_config* cfg);
+lmoe_status lmoe_backward_nvfp4(const lmoe_config* cfg, const lmoe_weights* w, const void* x, const void* dout,
+                                const float* a_global, uint64_t seed, uint32_t rht_signs, const lmoe_grads* g,
+                                void* ws, size_t ws_bytes, void* stream);
+
 /* Expert parallelism in the latent dimension (greeksharifa page on the
  * Nemotron 3 whitepaper, section 2.2 "LatentMoE": the rows that cross GPUs
  * between the projections are l-dim, so the all-to-all volume falls by d/l).

@@ -38,7 +38,7 @@ EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permut
            "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize",
            "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_gemm",
            "lmoe_ep_plan", "lmoe_ep_reorder", "lmoe_expert_backward_nvfp4",
-           "lmoe_expert_backward_nvfp4_workspace")
+           "lmoe_expert_backward_nvfp4_workspace", "lmoe_backward_nvfp4", "lmoe_backward_nvfp4_workspace")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
 
@@ -55,6 +55,11 @@ class Weights(ctypes.Structure):
         "w_router", "router_bias", "w_down", "w_up", "w1", "w2", "w1_sf", "w2_sf",
         "w1_gs", "w2_gs", "a_global_scale", "ws1", "ws2", "ws1_scale", "ws2_scale", "shared_x_scale",
         "shared_h_scale")]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "dx", "dw_router", "drouter_bias", "dw_down", "dw_up", "dw1", "dw2", "dws1", "dws2")]
 
 
 class LmoeError(RuntimeError):
@@ -97,6 +102,9 @@ def _load():
                                                   ctypes.c_uint64, ctypes.c_uint32, P, P, P, P, ctypes.c_int, P,
                                                   ctypes.c_size_t, P]),
         "lmoe_expert_backward_nvfp4_workspace": (ctypes.c_size_t, [C, P]),
+        "lmoe_backward_nvfp4_workspace": (ctypes.c_size_t, [C]),
+        "lmoe_backward_nvfp4": (ctypes.c_int, [C, W, P, P, P, ctypes.c_uint64, ctypes.c_uint32,
+                                               ctypes.POINTER(Grads), P, ctypes.c_size_t, P]),
         "lmoe_expert_backward_nvfp4": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_uint64,
                                                       ctypes.c_uint32, P, P, P, P, P, ctypes.c_size_t, P]),
     }
@@ -287,6 +295,24 @@ def expert_backward_nvfp4(cfg: Config, counts, offsets, padded_offsets, z_codes,
                                           _p(a_global), _p(gate), _p(dy), int(seed), int(rht_signs), _p(dz),
                                           _p(dgate), _p(dw1), _p(dw2), _p(ws), ws.numel(), _stream(stream)),
            "lmoe_expert_backward_nvfp4")
+    return ws
+
+
+def grads(**kw) -> Grads:
+    """lmoe_grads from device tensors (missing ones NULL)."""
+    return Grads(**{k: (None if v is None else v.data_ptr()) for k, v in kw.items()})
+
+
+def backward_nvfp4(cfg: Config, w: Weights, x, dout, a_global, seed, rht_signs, g: Grads, ws=None, stream=None):
+    """lmoe_backward_nvfp4: the layer's gradients, routed experts under the
+    NVFP4 training recipe (see the header). Allocates the workspace when none
+    is given; returns it (its error word holds device errors)."""
+    if ws is None:
+        import torch
+        ws = torch.zeros(int(lib.lmoe_backward_nvfp4_workspace(ctypes.byref(cfg))), dtype=torch.uint8, device="cuda")
+    _check(lib.lmoe_backward_nvfp4(ctypes.byref(cfg), ctypes.byref(w), _p(x), _p(dout), _p(a_global), int(seed),
+                                   int(rht_signs), ctypes.byref(g), _p(ws), ws.numel(), _stream(stream)),
+           "lmoe_backward_nvfp4")
     return ws
 
 

@@ -202,6 +202,8 @@ int tokmajor_splits(int64_t rows, int cols, int64_t k) {
   return sp > 1 ? sp : 1;
 }
 
+}  // namespace
+
 // out[rows, cols] = epi(x[rows, k] . W[cols, k]^T) with BF16 operands.
 lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int64_t k, void* out,
                        int64_t ld_out, int epi, const float* bias, const void* residual, int64_t ld_res,
@@ -240,6 +242,8 @@ lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int
   L.ld_res = ld_res;
   return tc_gemm(L, err, s);
 }
+
+namespace {
 
 // out[rows, cols] = epi(x[rows, k] . W^T) with E4M3 operands; W is [cols][k],
 // or [k / wgroup][cols][wgroup] (the K axis split over a stack of matrices)

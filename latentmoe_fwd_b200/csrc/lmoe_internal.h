@@ -191,16 +191,25 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
                                      cudaStream_t s, int64_t out_pitch = 0);
+// Dense BF16 GEMM on the tensor cores (lmoe_api.cu): out[rows][cols] =
+// epi(x[rows][k] . w[cols][k]^T), token-major tiles, or weight-major ones for
+// rows <= 64 (split-K into `partial` when given). epi: EPI_* of gemm_tc.cuh
+// (EPI_F32_BIAS: fp32 out (+ bias); EPI_BF16; EPI_ADD_RES: + residual, BF16).
+lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int64_t k, void* out,
+                       int64_t ld_out, int epi, const float* bias, const void* residual, int64_t ld_res,
+                       float* partial, uint32_t* err, cudaStream_t s);
 // Routed experts' backward under the NVFP4 training recipe (lmoe_train_experts.cu):
 // the body of lmoe_expert_backward_nvfp4 without its argument checks; ws holds
 // at least expert_backward_ws(cfg, counts) bytes (first 256 the error word);
-// o_out (nullable): receives the recomputed expert outputs o, fp32 [P][l].
+// o_out (nullable): receives the recomputed expert outputs o, fp32 [P][l];
+// err_word (nullable): the error word to report into instead of ws's own.
 size_t expert_backward_ws(const lmoe_config* cfg, const int32_t* counts);
 lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, const int32_t* offsets,
                                  const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
                                  const float* z_global, const void* w1, const void* w2, const float* a_global,
                                  const float* gate, const float* dy, uint64_t seed, uint32_t rht_signs, void* dz,
-                                 float* dgate, void* dw1, void* dw2, void* ws, float* o_out, cudaStream_t s);
+                                 float* dgate, void* dw1, void* dw2, void* ws, float* o_out, uint32_t* err_word,
+                                 cudaStream_t s);
 // FP8 E4M3 codes of in / s with one FP32 scale per tensor (scale_in, or the
 // tensor's amax / 448 when scale_in is null; scale_out receives it).
 lmoe_status launch_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,

@@ -235,7 +235,7 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
     return LMOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < bw_layout(cfg, counts).total) return LMOE_ERR_WORKSPACE;
   return expert_backward_core(cfg, counts, offsets, padded_offsets, z_codes, z_sf, z_global, w1, w2, a_global, gate,
-                              dy, seed, rht_signs, dz, dgate, dw1, dw2, ws, nullptr,
+                              dy, seed, rht_signs, dz, dgate, dw1, dw2, ws, nullptr, nullptr,
                               static_cast<cudaStream_t>(stream));
 }
 
@@ -252,11 +252,12 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                                  const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
                                  const float* z_global, const void* w1, const void* w2, const float* a_global,
                                  const float* gate, const float* dy, uint64_t seed, uint32_t rht_signs, void* dz,
-                                 float* dgate, void* dw1, void* dw2, void* ws, float* o_out, cudaStream_t s) {
+                                 float* dgate, void* dw1, void* dw2, void* ws, float* o_out, uint32_t* err_word,
+                                 cudaStream_t s) {
   const int N = cfg->N;
   const int64_t l = cfg->l, m = cfg->m;
   const BwLayout L = bw_layout(cfg, counts);
-  uint32_t* err = at<uint32_t>(ws, L.err);
+  uint32_t* err = err_word ? err_word : at<uint32_t>(ws, L.err);
   double* part = at<double>(ws, L.part);
   lmoe_status st = LMOE_OK;
   const __nv_bfloat16* W1 = static_cast<const __nv_bfloat16*>(w1);

@@ -276,3 +276,78 @@ def test_routed_experts_backward_matches_the_oracle(T, N, K, zero_expert):
             assert fro < 0.2 * qerr, name   # far closer to the oracle than to the unquantised value
     if zero_expert:
         assert not np.any(got["dw1"][N - 1]) and not np.any(got["dw2"][N - 1])
+
+
+def _weight_grad_check(name, g, r, N_groups=None):
+    """The weight-gradient bar of the expert test: 1e-2 relative Frobenius error,
+    and elements beyond 8e-2 * RMS (past half a BF16 step) confined to at most
+    eight rows or columns of each expert's matrix (stochastic-rounding flips)."""
+    from gpu_util import bf16_ulp
+    fro = np.linalg.norm(g - r) / np.linalg.norm(r)
+    rms = np.sqrt(np.mean(O.round_bf16(r) ** 2))
+    over = (np.abs(g - r) - bf16_ulp(O.round_bf16(r)) / 2) > 8e-2 * rms
+    for e in range(over.shape[0]):
+        rows, cols = np.nonzero(over[e])
+        assert min(np.unique(rows).size, np.unique(cols).size) <= 8, (name, e)
+    assert over.mean() <= 0.02, name
+    assert fro <= 1e-2, name
+    return fro
+
+
+@pytest.mark.parametrize("case", ["latent", "latent_shared_bias", "identity_shared"])
+def test_layer_backward_matches_the_oracle(case):
+    """lmoe_backward_nvfp4 (the whole layer's gradients: recomputed routing and
+    NVFP4 latent rows, the routed experts under the recipe, the router, the
+    latent projections and the shared experts as BF16 GEMMs) against the
+    oracle's backward_nvfp4 on the same inputs. The dense gradients are BF16
+    GEMMs of BF16-rounded gradient tensors: within 2e-2 * RMS beyond half a
+    BF16 step (the BF16 forward's bar); dW1 and dW2 as in the expert test."""
+    from gpu_util import DevLayer, bf16_parity
+    if case == "latent":
+        wl = LI.reduced("ultra_decode", T=160, d=512, l=256, N=8, K=2, m=256)
+    elif case == "latent_shared_bias":
+        wl = LI.replace(LI.reduced("ultra_zipf", T=96, d=512, l=256, N=8, K=3, m=256, n_shared=1, m_shared=128))
+    else:
+        wl = LI.reduced("std_moe_bf16", T=128, d=256, l=256, N=8, K=2, m=256, n_shared=2, m_shared=64)
+    inp = LI.make_inputs(wl)
+    p = B.params_from_inputs(wl, inp)
+    rng = np.random.default_rng(11)
+    doutb = LI.bf16_bits(rng.standard_normal((wl.T, wl.d)) * 0.05)
+    dout = O.from_bf16_bits(doutb)
+    # static global scale of a from the unquantised expert pre-activations
+    x = p["x"]
+    z = x if p["w_down"] is None else x @ p["w_down"].T
+    amax = max(np.max(O.sq_relu(z @ p["w1"][e].T)) for e in range(wl.N))
+    s_a = float(np.float32(amax / 2688.0))
+    seed = 0xBEEF
+    logits = O.router_logits(x, p["w_router"], p["router_bias"])
+    assert not np.any(O.near_tie_tokens(logits, wl.K)), "near-tie routing in the test data"
+    ref = B.backward_nvfp4(p, wl.K, dout, SIGNS, seed, a_global_scale=s_a)
+
+    dev = DevLayer(wl, inp)
+    bf = lambda *shape: torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+    S, ms = wl.n_shared, wl.m_shared
+    out = dict(dx=bf(wl.T, wl.d), dw_router=bf(wl.N, wl.d), dw1=bf(wl.N, wl.m, wl.l), dw2=bf(wl.N, wl.l, wl.m))
+    if inp["router_bias"] is not None:
+        out["drouter_bias"] = torch.zeros(wl.N, dtype=torch.float32, device="cuda")
+    if not wl.identity:
+        out.update(dw_down=bf(wl.l, wl.d), dw_up=bf(wl.d, wl.l))
+    if S:
+        out.update(dws1=bf(S, ms, wl.d), dws2=bf(S, wl.d, ms))
+    g = L.grads(**out)
+    a_g = torch.tensor([s_a], dtype=torch.float32, device="cuda")
+    ws = L.backward_nvfp4(dev.cfg, dev.w, dev.x, to_dev(doutb, "bf16"), a_g, seed, SIGN_BITS, g)
+    st, info = L.read_device_error(ws)
+    assert st == L.OK, (L.status_string(st), hex(info))
+    got = {k: v.float().cpu().numpy().astype(np.float64) for k, v in out.items()}
+    for name in ("dx", "dw_router", "drouter_bias", "dw_down", "dw_up", "dws1", "dws2"):
+        if name not in got:
+            continue
+        r = ref[name]
+        excess, raw = bf16_parity(got[name], r, O.round_bf16(r))
+        fro = np.linalg.norm(got[name] - r) / np.linalg.norm(r)
+        print(f"layer backward {case} {name}: excess {excess:.3e} * RMS, raw {raw:.3e} * RMS, rel {fro:.3e}")
+        assert excess <= 2e-2, name
+    for name in ("dw1", "dw2"):
+        fro = _weight_grad_check(name, got[name], ref[name])
+        print(f"layer backward {case} {name}: rel {fro:.3e}")
