@@ -151,9 +151,11 @@ struct SimtLaunch {
 lmoe_status simt_gemm(const SimtLaunch& L, uint32_t* err_word, cudaStream_t stream);
 
 // ----- small kernels (lmoe_kernels.cu) -----
-// x / w_router non-null: refine near-tied decisions with exact logits (see the kernel).
+// x / w_router non-null: refine near-tied decisions with exact logits (see the
+// kernel); refine_all: every candidate's logit exact (gates to fp32 rounding).
 lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w, const void* x,
-                        const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s);
+                        const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s,
+                        int refine_all = 0);
 // Slots per warp of the counting sort: the workspace path uses short chunks
 // (more CTAs in flight); the fixed-scratch path keeps 1024 (fewer counters).
 constexpr int kPermSlotsPerWarp = 128;

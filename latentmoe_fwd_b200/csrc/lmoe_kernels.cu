@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
                                                                int K, int tpb, int32_t* __restrict__ idx,
                                                                float* __restrict__ w, const TA* __restrict__ x,
                                                                const TA* __restrict__ wr,
-                                                               const float* __restrict__ bias, int d) {
+                                                               const float* __restrict__ bias, int d,
+                                                               int refine_all) {
   pdl_begin();
   __shared__ int s_njobs[kTopkWarps];
   __shared__ int s_expert[kTopkWarps * 32];
@@ -253,11 +254,12 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
       }
     }
     if (refine) {
-      // mark candidates that have a neighbour within 2 tau
+      // mark candidates that have a neighbour within 2 tau (every candidate
+      // with refine_all: exact logits, hence gates to fp32 rounding)
       const float up = __shfl_up_sync(FULL, my_v, 1);
       const float dn = __shfl_down_sync(FULL, my_v, 1);
-      const bool mark =
-          lane < C && ((lane > 0 && up - my_v <= 2.0f * tau) || (lane + 1 < C && my_v - dn <= 2.0f * tau));
+      const bool mark = lane < C && (refine_all || (lane > 0 && up - my_v <= 2.0f * tau) ||
+                                     (lane + 1 < C && my_v - dn <= 2.0f * tau));
       todo = __ballot_sync(FULL, mark);
       if (mark) s_expert[warp * 32 + __popc(todo & ((1u << lane) - 1u))] = my_i;
     }
@@ -333,7 +335,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
 }
 
 lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* idx, float* w, const void* x,
-                        const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s) {
+                        const void* w_router, const float* bias, int d, int act, uint32_t* err, cudaStream_t s,
+                        int refine_all) {
   (void)err;
   if (T == 0) return LMOE_OK;
   // few tokens: one token per block, so the block's eight warps share its dots
@@ -346,11 +349,11 @@ lmoe_status launch_topk(const float* logits, int64_t T, int N, int K, int32_t* i
   do {                                                                                                       \
     if (act == LMOE_F32)                                                                                     \
       launch_k(topk_kernel<NPLV, float>, dim3(blocks), dim3(kTopkWarps * 32), 0, s, logits, T, N, K, tpb, idx, \
-               w, static_cast<const float*>(x), static_cast<const float*>(w_router), bias, d);               \
+               w, static_cast<const float*>(x), static_cast<const float*>(w_router), bias, d, refine_all);   \
     else                                                                                                     \
       launch_k(topk_kernel<NPLV, __nv_bfloat16>, dim3(blocks), dim3(kTopkWarps * 32), 0, s, logits, T, N, K,   \
                tpb, idx, w, static_cast<const __nv_bfloat16*>(x),                                            \
-               static_cast<const __nv_bfloat16*>(w_router), bias, d);                                        \
+               static_cast<const __nv_bfloat16*>(w_router), bias, d, refine_all);                            \
   } while (0)
   if (npl <= 1) LMOE_TOPK(1);
   else if (npl <= 2) LMOE_TOPK(2);

@@ -274,8 +274,9 @@ lmoe_status lmoe_backward_nvfp4(const lmoe_config* cfg, const lmoe_weights* w, c
   if (!ok(dense_bf16(x, T, w->w_router, static_cast<int>(N), d, logits, N, EPI_F32_BIAS, w->router_bias, nullptr, 0,
                      nullptr, err, s)))
     return st;
+  // gates from exact logits: the experts' stochastic quantisers read gate * dy
   if (!ok(launch_topk(logits, T, static_cast<int>(N), static_cast<int>(K), idx, gates, x, w->w_router,
-                      w->router_bias, static_cast<int>(d), LMOE_BF16, err, s)))
+                      w->router_bias, static_cast<int>(d), LMOE_BF16, err, s, 1)))
     return st;
   const void* z = x;
   if (!ident) {

@@ -372,7 +372,8 @@ def routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, signs, seed: int, 
 def backward_nvfp4(params: dict, K: int, dout, signs, seed: int, a_global_scale=None,
                    quantize: bool = True) -> dict:
     """The layer's gradients with its routed experts trained under the NVFP4
-    recipe: the expert GEMMs' forward reads NVFP4 z (current amax), NVFP4 a
+    recipe: the expert GEMMs' forward reads NVFP4 z (of z rounded to BF16, the
+    forward's rounding point; current amax), NVFP4 a
     (``a_global_scale``, else its current amax) and 2-D-block NVFP4 weights;
     their dgrad and wgrad are ``nvfp4_linear_backward``, with each expert's
     rows padded by zero rows to a multiple of 16 for the token transform. The
@@ -396,7 +397,9 @@ def backward_nvfp4(params: dict, K: int, dout, signs, seed: int, a_global_scale=
     logits = O.router_logits(x, wr, bias)
     idx, gates = O.route_topk(logits, K)
     z = x if w_down is None else x @ w_down.T
-    zq = fq(z)
+    # the experts read NVFP4 of z as the forward stores it: rounded to BF16
+    # first (its rounding point), then quantised with the current amax
+    zq = fq(O.round_bf16(z)) if quantize else z
     dc = dout if w_up is None else dout @ w_up
     r = routed_experts_backward_nvfp4(zq, w1, w2, idx, gates, dc, signs, seed, a_global_scale, quantize)
     c, dz, dgate, dw1, dw2 = r["c"], r["dz"], r["dgate"], r["dw1"], r["dw2"]
