@@ -30,6 +30,7 @@ barrier and the max over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -374,6 +375,92 @@ def workload_config(wl):
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
+def run_backward(args, wl):
+    """--backward: time lmoe_backward_nvfp4, the layer's backward pass with its
+    routed experts under the NVFP4 training recipe (BF16 masters of every
+    weight; one step = one backward over the workload's T tokens, inputs
+    resident). Roofline: the six NVFP4 expert GEMMs (forward recompute, dgrad,
+    wgrad of both layers) at the FP4 peak plus the BF16 GEMMs of the router,
+    the projections and the shared experts at the BF16 peak, against the
+    measured step. One JSON line, rank 0, N = 1."""
+    import torch
+
+    import latentmoe_fwd_b200 as L
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    inp = LI.make_inputs(wl)
+    bits = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+        torch.bfloat16).cuda()
+    t = {k: bits(inp[k]) for k in ("x", "w_router", "w_down", "w_up", "w1", "w2", "ws1", "ws2")}
+    bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).cuda()
+    cfg = L.config(T=wl.T, d=wl.d, l=wl.l, N=wl.N, K=wl.K, m=wl.m, n_shared=wl.n_shared, m_shared=wl.m_shared,
+                   identity=wl.identity)
+    w = L.weights(w_router=t["w_router"], router_bias=bias, w_down=t["w_down"], w_up=t["w_up"], w1=t["w1"],
+                  w2=t["w2"], ws1=t["ws1"], ws2=t["ws2"])
+    rng = np.random.default_rng(5)
+    dout = bits(LI.bf16_bits(rng.standard_normal((wl.T, wl.d)) * 0.05))
+    s_a = inp["a_global_scale"] if inp.get("a_global_scale") is not None else float(np.float32(256.0 / 2688.0))
+    a_g = torch.tensor([s_a], dtype=torch.float32, device="cuda")
+    bf = lambda *shape: torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    S, ms = wl.n_shared, wl.m_shared
+    out = dict(dx=bf(wl.T, wl.d), dw_router=bf(wl.N, wl.d), dw1=bf(wl.N, wl.m, wl.l), dw2=bf(wl.N, wl.l, wl.m))
+    if bias is not None:
+        out["drouter_bias"] = torch.empty(wl.N, dtype=torch.float32, device="cuda")
+    if not wl.identity:
+        out.update(dw_down=bf(wl.l, wl.d), dw_up=bf(wl.d, wl.l))
+    if S:
+        out.update(dws1=bf(S, ms, wl.d), dws2=bf(S, wl.d, ms))
+    g = L.grads(**out)
+    ws = torch.zeros(int(L.lib.lmoe_backward_nvfp4_workspace(ctypes.byref(cfg))), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        L.backward_nvfp4(cfg, w, t["x"], dout, a_g, 1, 0x5A5A, g, ws)
+    torch.cuda.synchronize()
+    stv, info = L.read_device_error(ws)
+    if stv != L.OK:
+        raise RuntimeError(f"device error during warm-up: {L.status_string(stv)} info={info:#x}")
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    launches0 = L.kernel_launch_count()
+    start.record(stream)
+    for i in range(K):
+        L.backward_nvfp4(cfg, w, t["x"], dout, a_g, 1 + i, 0x5A5A, g, ws, stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    launches = L.kernel_launch_count() - launches0
+    clocks = sampler.stop()
+    stv, info = L.read_device_error(ws)
+    if stv != L.OK:
+        raise RuntimeError(f"device error in the timed region: {L.status_string(stv)} info={info:#x}")
+    ms_step = start.elapsed_time(end) / K
+    TK = wl.T * wl.K
+    fp4_flops = 3 * 2 * (2.0 * TK * wl.l * wl.m)
+    dense = 2.0 * wl.T * wl.d * wl.N * 3                      # router logits, dW_router, dx's router term
+    if not wl.identity:
+        dense += 2.0 * wl.T * wl.d * wl.l * 5                 # z, dc, dW_up, dW_down, dx's projection term
+    if S:
+        dense += 2.0 * wl.T * wl.d * S * ms * 5                # pre, dout Ws2, dWs2, dWs1, dx's shared term
+    peaks, src = load_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops"]
+    t_peak = fp4_flops / (fp4_peak * 1e9) + dense / (peaks["bf16_tflops"] * 1e9)
+    line = {
+        "metric": "LatentMoE layer backward tokens/s on 1 B200 (routed experts under the NVFP4 training recipe)",
+        "value": wl.T / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "dtype": "nvfp4+bf16", "data": "synthetic",
+        "config": workload_config(wl),
+        "roofline": {"bound": "tensor", "achieved_tflops": (fp4_flops + dense) / (ms_step * 1e9),
+                     "fp4_flops": fp4_flops, "bf16_flops": dense, "time_at_peak_ms": t_peak,
+                     "frac": t_peak / ms_step, "peak_fp4_tflops": fp4_peak, "peak_bf16_tflops": peaks["bf16_tflops"],
+                     "peak_source": src,
+                     "note": "the host walks the experts (about 20 launches each) and reads their row counts once"},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -387,6 +474,8 @@ def main():
                     help="override the workload's token count (smaller captures for ncu)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override the workload's expert count (smaller captures for ncu)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer backward (NVFP4 training recipe for the routed experts) instead")
     args = ap.parse_args()
     wl = LI.WORKLOADS[args.workload]
     if args.tokens is not None:
@@ -395,6 +484,8 @@ def main():
         wl = LI.replace(wl, N=args.experts)
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.backward:
+        return run_backward(args, wl)
 
     import torch
     import torch.distributed as dist

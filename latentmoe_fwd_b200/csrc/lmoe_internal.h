@@ -206,6 +206,7 @@ lmoe_status dense_bf16(const void* x, int64_t rows, const void* w, int cols, int
 // o_out (nullable): receives the recomputed expert outputs o, fp32 [P][l];
 // err_word (nullable): the error word to report into instead of ws's own.
 size_t expert_backward_ws(const lmoe_config* cfg, const int32_t* counts);
+size_t expert_backward_ws_bound(const lmoe_config* cfg);   // any routing of cfg->T tokens
 lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, const int32_t* offsets,
                                  const int32_t* padded_offsets, const uint8_t* z_codes, const uint8_t* z_sf,
                                  const float* z_global, const void* w1, const void* w2, const float* a_global,

@@ -142,14 +142,10 @@ struct BwLayout {
   int64_t P, Rmax, R128max, K256max;
 };
 
-BwLayout bw_layout(const lmoe_config* c, const int32_t* counts) {
+// P: padded slot rows; Rmax: the largest expert's rows rounded up to 16.
+BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax) {
   BwLayout L = {};
   const int64_t N = c->N, l = c->l, m = c->m;
-  int64_t P = 0, Rmax = 0;
-  for (int e = 0; e < N; ++e) {
-    P += ceil_to(counts[e], 128);
-    Rmax = counts[e] > 0 ? (ceil_to(counts[e], 16) > Rmax ? ceil_to(counts[e], 16) : Rmax) : Rmax;
-  }
   L.P = P;
   L.Rmax = Rmax;
   L.R128max = ceil_to(Rmax, 128);
@@ -193,6 +189,15 @@ BwLayout bw_layout(const lmoe_config* c, const int32_t* counts) {
   L.tab = take((N * 4 + 8) * 4);   // per expert {0, n, 0, R128}; then {0, l, 0, l}, {0, m, 0, m}
   L.total = off;
   return L;
+}
+
+BwLayout bw_layout(const lmoe_config* c, const int32_t* counts) {
+  int64_t P = 0, Rmax = 0;
+  for (int e = 0; e < c->N; ++e) {
+    P += ceil_to(counts[e], 128);
+    if (counts[e] > 0 && ceil_to(counts[e], 16) > Rmax) Rmax = ceil_to(counts[e], 16);
+  }
+  return bw_layout_for(c, P, Rmax);
 }
 
 template <typename T>
@@ -244,6 +249,12 @@ lmoe_status lmoe_expert_backward_nvfp4(const lmoe_config* cfg, const int32_t* co
 namespace lmoe {
 
 size_t expert_backward_ws(const lmoe_config* cfg, const int32_t* counts) { return bw_layout(cfg, counts).total; }
+
+// Enough for any routing of cfg->T tokens: at most padded_rows slot rows, and
+// no expert with more than T rows (a token picks an expert once).
+size_t expert_backward_ws_bound(const lmoe_config* cfg) {
+  return bw_layout_for(cfg, lmoe_padded_rows(cfg), ceil_to(cfg->T > 0 ? cfg->T : 1, 16)).total;
+}
 
 // The routed experts' backward (see lmoe_expert_backward_nvfp4), arguments
 // checked by the caller; ws holds at least expert_backward_ws() bytes. With

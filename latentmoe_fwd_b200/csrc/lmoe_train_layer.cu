@@ -193,9 +193,7 @@ LbLayout lb_layout(const lmoe_config* c) {
     L.ws2T = take(Sms * d * 2);
     L.ws1T = take(d * Sms * 2);
   }
-  // the experts' workspace for the worst case: every expert with T rows
-  std::vector<int32_t> worst(N > 0 ? N : 1, static_cast<int32_t>(T));
-  L.ex = take(expert_backward_ws(c, worst.data()));
+  L.ex = take(expert_backward_ws_bound(c));   // any routing of the T tokens
   L.total = off;
   return L;
 }
