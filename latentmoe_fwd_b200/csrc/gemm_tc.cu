@@ -51,8 +51,7 @@ static lmoe_status launch_tc(const CUtensorMap& a0, const CUtensorMap& b0, const
                              cudaStream_t s) {
   using Sm = TcSmem<BN, STAGES>;
   auto kern = tc_gemm_kernel<BN, STAGES, EPI>;
-  constexpr int smem = Sm::kBytes + (EPI == EPI_SCATTER ? Sm::kScatterBytes : 0);
-  static_assert(EPI != EPI_SCATTER || BN < 64 || smem <= 232448, "scatter epilogue exceeds shared memory");
+  constexpr int smem = Sm::kBytes;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -75,7 +74,6 @@ static lmoe_status dispatch_epi(int epi, const CUtensorMap* m, const TcParams& p
     case EPI_GATE: return launch_tc<BN, STAGES, EPI_GATE>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_ADD_RES: return launch_tc<BN, STAGES, EPI_ADD_RES>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_PARTIAL: return launch_tc<BN, STAGES, EPI_PARTIAL>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
-    case EPI_SCATTER: return launch_tc<BN, STAGES, EPI_SCATTER>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_SQRELU_Q8: return launch_tc<BN, STAGES, EPI_SQRELU_Q8>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
     case EPI_SCALE: return launch_tc<BN, STAGES, EPI_SCALE>(m[0], m[1], m[2], m[3], m[4], p, grid, s);
   }
@@ -125,8 +123,6 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
   p.ld_res = L.ld_res;
   p.ksplit = L.ksplit > 1 ? L.ksplit : 1;
   p.partial = L.partial;
-  p.scatter_rows = L.scatter_rows;
-  p.scatter_k = L.scatter_k;
   p.fp8 = L.fp8;
   p.scale_a = L.scale_a;
   p.scale_w = L.scale_w;
@@ -138,9 +134,6 @@ lmoe_status tc_gemm(const TcLaunch& L, uint32_t* err_word, cudaStream_t stream) 
     return LMOE_ERR_INVALID_ARG;
   if (L.fp8 && L.grouped) return LMOE_ERR_UNSUPPORTED;
   if (p.ksplit > 1 && (L.grouped || !L.partial)) return LMOE_ERR_INVALID_ARG;
-  if (L.epi == EPI_SCATTER &&
-      (L.swap || L.ksplit > 1 || !L.scatter_rows || L.scatter_k <= 0 || L.scatter_k > 32 || L.bn < 64))
-    return LMOE_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   const int64_t tiles = L.max_tiles * p.ksplit;
   int64_t grid = tiles < sms ? tiles : sms;

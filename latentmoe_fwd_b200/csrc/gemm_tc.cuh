@@ -35,8 +35,6 @@ enum EpiKind : int {
   EPI_GATE = 3,       // out bf16 = acc * row_scale[row]
   EPI_ADD_RES = 4,    // out bf16 = acc + residual[row][col]
   EPI_PARTIAL = 5,    // split-K: fp32 partial sums, the epilogue runs in the reduction
-  EPI_SCATTER = 6,    // out bf16 = acc, row t stored at each padded row scatter_rows[t*K + k]
-                      // (k < scatter_k; negative entries skipped): token-major tiles only
   EPI_SQRELU_Q8 = 7,  // out E4M3 byte = E4M3(relu(acc * s_a * s_w)^2 / out_scale)
   EPI_SCALE = 8       // out bf16 = acc * s_a * s_w
 };
@@ -65,8 +63,6 @@ struct TcParams {
   long long ld_res;
   int ksplit;                 // >1: split the K blocks of every tile; partial sums go to `partial`
   float* partial;             // [ksplit][rows][cols] fp32 (split-K only)
-  const int* scatter_rows;    // EPI_SCATTER: [rows][scatter_k] destination rows of each row
-  int scatter_k;
   // FP8 operands (E4M3 codes, 1 byte each; K blocks of 128 elements, the same
   // 128 bytes per row per stage as BF16): tcgen05.mma kind::f8f6f4
   int fp8;
@@ -97,14 +93,9 @@ struct TcSmem {
   static constexpr int kMaxGroups = 1024;
   // weight-major epilogue: one 32 x 32 BF16 transpose tile per epilogue warp
   static constexpr int kEpiOffset = (kPrefixOffset + (kMaxGroups + 1) * 4 + 15) / 16 * 16;
-  // per epilogue warp: a 32 x 32 BF16 transpose tile, or a staged 32-row x 64-byte chunk at an
-  // 80-byte row pitch (bank-conflict free) for the scatter epilogue
+  // per epilogue warp: a 32 x 32 BF16 transpose tile (80-byte row pitch, bank-conflict free)
   static constexpr int kEpiWarpBytes = 32 * 80;
   static constexpr int kBytes = kEpiOffset + 4 * kEpiWarpBytes + 1024;  // +1024 alignment slack
-  // scatter epilogue only (launched with kBytes + kScatterBytes): each epilogue
-  // warp's 32 token rows x up to 32 destination rows, loaded once per tile
-  static constexpr int kScatterOffset = kEpiOffset + 4 * kEpiWarpBytes;
-  static constexpr int kScatterBytes = 4 * 32 * 32 * 4;
 };
 
 struct TileInfo {
@@ -434,54 +425,12 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
       const int nchunks = p.swap ? (ti.act_n + 31) / 32 : BN / 32;
-      int* srow = reinterpret_cast<int*>(smem + S::kScatterOffset) + (warp & 3) * 32 * 32;
-      if (EPI == EPI_SCATTER) {
-        // the destination rows of this warp's 32 tokens (contiguous in
-        // scatter_rows), read once per tile so the stores below wait on none
-        const int nrow = max(0, min(32, ti.act_n - q * 32)) * p.scatter_k;
-        const int* src = p.scatter_rows + static_cast<long long>(ti.act0 + q * 32) * p.scatter_k;
-        for (int i = lane; i < nrow; i += 32) srow[i] = __ldg(src + i);
-        __syncwarp();
-      }
 #pragma unroll 1
       for (int c = 0; c < nchunks; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + c * 32, v);
         tmem_ld_wait();
-        if (!p.swap && EPI == EPI_SCATTER) {
-          // each token row goes to its K slots' padded rows (the expert-grouped
-          // GEMM input): the warp stages its 32 rows x 32 columns (64 bytes a
-          // row) in shared memory, then writes 64-byte row segments, eight
-          // destinations per store instruction (whole sectors), streamed past L2
-          uint4* st = reinterpret_cast<uint4*>(epi_tile + (warp & 3) * (S::kEpiWarpBytes / 2));
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-            u.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-            u.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-            u.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
-            st[lane * 5 + j] = u;
-          }
-          __syncwarp();
-          const uint64_t pol = policy_evict_first();
-          const int K = p.scatter_k;
-          const int col0 = ti.w0 + c * 32;
-          const int part = lane & 3;                 // 16 bytes of the 64-byte segment
-          int rr = 0, kk = lane >> 2;                // segment s = rr * K + kk, eight per step
-          while (kk >= K) { kk -= K; ++rr; }
-          const int rows_here = min(32, ti.act_n - q * 32);
-          for (; rr < rows_here;) {
-            const int pr = srow[rr * K + kk];
-            if (pr >= 0 && col0 + part * 8 < p.cols)
-              st_global_v4_hint(reinterpret_cast<__nv_bfloat16*>(p.out) + static_cast<long long>(pr) * p.ld_out + col0 +
-                                    part * 8,
-                                st[rr * 5 + part], pol);
-            kk += 8;
-            while (kk >= K) { kk -= K; ++rr; }
-          }
-          __syncwarp();
-        } else if (!p.swap) {
+        if (!p.swap) {
           const long long row = ti.act0 + r;
           if (r < ti.act_n) {
             const int col0 = ti.w0 + c * 32;

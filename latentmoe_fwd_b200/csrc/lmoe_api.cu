@@ -820,29 +820,20 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   float* gate = at<float>(ws, L.gate);
   void* zp = at<void>(ws, L.zp);
   float* z_gs = nullptr;
-  // BF16 latent layer with token-major tiles: the permutation runs first and
-  // the down-projection's epilogue writes each token's z row straight to the
-  // padded rows of its K slots, so z is never stored and gathered
+  // BF16 latent layer at prefill sizes: the permutation runs first, then the
+  // down-projection stores z once and a token-order copy reads each z row once
+  // and writes it to the padded rows of its K slots
   const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens && l >= 64;
   if (scatter_z) {
     int32_t* slot_row = at<int32_t>(ws, L.slot_row);
     if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
                              err, s, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
       return st;
-    TcLaunch D;
-    D.rows = static_cast<int>(T);
-    D.cols = l;
-    D.kblocks[0] = kblocks(d);
-    D.bn = normal_bn(l);
-    D.a[0] = TcOperand{x, d, T, 1};
-    D.b[0] = TcOperand{w->w_down, d, l, 1};
-    D.max_tiles = ((T + 127) / 128) * ((l + D.bn - 1) / D.bn);
-    D.out = zp;
-    D.ld_out = l;
-    D.epi = EPI_SCATTER;
-    D.scatter_rows = slot_row;
-    D.scatter_k = K;
-    if ((st = tc_gemm(D, err, s)) != LMOE_OK) return st;
+    void* zb = at<void>(ws, L.z);
+    if ((st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s)) != LMOE_OK)
+      return st;
+    mark(2);
+    if ((st = launch_scatter_rows(zb, T, static_cast<int64_t>(l) * ab, slot_row, K, zp, s)) != LMOE_OK) return st;
     mark(3);
   } else if (fp4) {
     // NVFP4 latent activations (current per-tensor amax): the permutation runs

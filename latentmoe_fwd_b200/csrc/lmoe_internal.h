@@ -79,8 +79,6 @@ struct TcLaunch {
   int bn = 256;
   int ksplit = 1;                // >1: split-K with fp32 partials in `partial`, then a reduction
   float* partial = nullptr;      // [ksplit][rows][cols]
-  const int* scatter_rows = nullptr;   // EPI_SCATTER (token-major only): [rows][scatter_k] destination rows
-  int scatter_k = 0;
   int fp8 = 0;                   // 1: E4M3 operands (every segment), K blocks of 128
   const float* scale_a = nullptr;     // EPI_SQRELU_Q8 / EPI_SCALE: operand scales (device scalars)
   const float* scale_w = nullptr;
@@ -181,6 +179,10 @@ lmoe_status launch_combine(const void* y, int act, const int32_t* idx, const int
 lmoe_status launch_nvfp4_quantize_scatter(const void* in, int64_t rows, int cols, const int32_t* slot_row, int K,
                                           uint8_t* codes, uint8_t* sf, float* global_out, float* partials,
                                           int npartials, cudaStream_t s);
+// Each of the n rows (row_bytes, a multiple of 16) copied to the padded rows
+// of its K slots (slot_row[t*K+k]; -1 skips the slot).
+lmoe_status launch_scatter_rows(const void* rows, int64_t n, int64_t row_bytes, const int32_t* slot_row, int K,
+                                void* out, cudaStream_t s);
 lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                   const float* global_in, uint8_t* codes, uint8_t* sf,
                                   float* global_out, int sf_layout, float* partials,

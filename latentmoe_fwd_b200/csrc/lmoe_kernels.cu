@@ -1061,6 +1061,56 @@ lmoe_status launch_nvfp4_quantize_scatter(const void* in, int64_t rows, int cols
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
+// Dispatch copy in token order: each token's row is read once and written to
+// the padded rows of its K slots (the permutation's slot_row; -1 marks a slot
+// left out). A warp per token; each pass holds 2 KB of the row in registers
+// (four 16-byte loads per lane) and stores it at every slot row.
+__global__ void __launch_bounds__(256) scatter_rows_kernel(const uint8_t* __restrict__ rows, int64_t n,
+                                                           int64_t row_bytes, const int32_t* __restrict__ slot_row,
+                                                           int K, uint8_t* __restrict__ out) {
+  pdl_begin();
+  constexpr unsigned FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const int64_t n16 = row_bytes >> 4;
+  const uint64_t pol = policy_evict_first();   // the expert GEMM reads the slot rows much later
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < n; t += warps) {
+    const int my_row = lane < K ? __ldg(slot_row + t * K + lane) : -1;
+    const uint4* src = reinterpret_cast<const uint4*>(rows + t * row_bytes);
+    for (int64_t i0 = 0; i0 < n16; i0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + u * 32 + lane;
+        v[u] = i < n16 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      for (int k = 0; k < K; ++k) {
+        const int p = __shfl_sync(FULL, my_row, k);
+        if (p < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(p) * row_bytes);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + u * 32 + lane;
+          if (i < n16) st_global_v4_hint(dst + i, v[u], pol);
+        }
+      }
+    }
+  }
+}
+
+lmoe_status launch_scatter_rows(const void* rows, int64_t n, int64_t row_bytes, const int32_t* slot_row, int K,
+                                void* out, cudaStream_t s) {
+  if (n == 0) return LMOE_OK;
+  if (row_bytes <= 0 || row_bytes % 16 || K < 1 || K > 32) return LMOE_ERR_UNSUPPORTED;
+  const int sms = device_sm_count();
+  int64_t blocks = (n * 32 + 255) / 256;
+  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  launch_k(scatter_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+           static_cast<const uint8_t*>(rows), n, row_bytes, slot_row, K, static_cast<uint8_t*>(out));
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
 lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols,
                                   const float* global_in, uint8_t* codes, uint8_t* sf,
                                   float* global_out, int sf_layout, float* partials, int npartials,
