@@ -189,12 +189,14 @@ lmoe_status launch_nvfp4_quantize(const void* in, int in_dtype, int64_t rows, in
                                   int npartials, uint32_t* err, cudaStream_t s);
 int nvfp4_partials(int64_t elems);
 // Training-recipe NVFP4 quantiser (lmoe_train.cu): partials holds
-// nvfp4x_partials(out_rows * out_cols / 16) doubles.
+// groups * nvfp4x_partials(out_rows * out_cols / 16) doubles. groups > 1:
+// that many matrices of rows x cols, contiguous in `in`, codes and sf, each
+// with its own global scale (global_out[g]); round to nearest only.
 int nvfp4x_partials(int64_t blocks);
 lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
-                                     cudaStream_t s, int64_t out_pitch = 0);
+                                     cudaStream_t s, int64_t out_pitch = 0, int groups = 1);
 // Dense BF16 GEMM on the tensor cores (lmoe_api.cu): out[rows][cols] =
 // epi(x[rows][k] . w[cols][k]^T), token-major tiles, or weight-major ones for
 // rows <= 64 (split-K into `partial` when given). epi: EPI_* of gemm_tc.cuh

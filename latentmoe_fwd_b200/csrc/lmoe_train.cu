@@ -84,7 +84,25 @@ struct QxParams {
   uint8_t* sf;
   float* global_out;
   int64_t pitch;         // elements per stored output row (>= out cols; the rest stored as zero codes and scales)
+  // grouped launches (gridDim.y groups, one matrix each, with its own global
+  // scale): strides between the groups' inputs (elements), codes and scales (bytes)
+  int64_t gs_in, gs_codes, gs_sf;
 };
+
+// The parameters of group blockIdx.y: its input, outputs, global scale and
+// amax partials.
+__device__ __forceinline__ QxParams qx_group(const QxParams& p0) {
+  QxParams p = p0;
+  const int64_t g = blockIdx.y;
+  if (g) {
+    p.in = static_cast<const uint8_t*>(p0.in) + g * p0.gs_in * (p0.bf16 ? 2 : 4);
+    p.codes += g * p0.gs_codes;
+    p.sf += g * p0.gs_sf;
+    if (p.global_out) p.global_out += g;
+    if (p.partials) p.partials += g * p0.np;
+  }
+  return p;
+}
 
 __device__ __forceinline__ double load_in(const QxParams& p, int64_t r, int64_t c) {
   if (p.bf16) return static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(p.in)[r * p.cols + c]));
@@ -119,8 +137,10 @@ __device__ __forceinline__ int64_t out_rows(const QxParams& p) { return p.transp
 __device__ __forceinline__ int64_t out_cols(const QxParams& p) { return p.transpose ? p.rows : p.cols; }
 
 // Pass 1: per-CTA maxima of |out| (fp64, exact).
-__global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p, double* __restrict__ partials) {
+__global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, double* __restrict__ partials) {
   pdl_begin();
+  const QxParams p = qx_group(p0);
+  partials += static_cast<int64_t>(blockIdx.y) * gridDim.x;
   __shared__ double red[kXThreads / 32];
   const int64_t nb = out_cols(p) / 16, total = out_rows(p) * nb;
   double m = 0.0;
@@ -175,9 +195,13 @@ __device__ __forceinline__ int64_t tiled_off(int64_t row, int64_t j, int64_t gro
   return ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
 }
 
-// Pass 2: a thread per 16 output rows x one 16-column block.
-__global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p) {
+// Pass 2: a thread per output row and 16-column block; the 16 rows of a
+// 16-row group sit in one half-warp (lane & 15 = row in the group), so a
+// 16 x 16 block's amax is a half-warp reduction. The item count is rounded up
+// to whole warps; items past the end take part in the reductions only.
+__global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0) {
   pdl_begin();
+  const QxParams p = qx_group(p0);
   __shared__ double red[kXThreads / 32];
   __shared__ float s_gs;
   // global scale: s_g = fp32(amax / 2688) from the fp64 amax (1 when 0)
@@ -205,67 +229,62 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p) 
   const int64_t groups64 = (p.pitch + 63) / 64;
   const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;   // 16-row groups, tiled padding
   const int64_t nb_cov = p.tiled ? groups64 * 4 : nb_store;
-  const int64_t total = rg_cov * nb_cov;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
-       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t items = rg_cov * nb_cov * 16;
+  const int64_t items32 = (items + 31) / 32 * 32;
+  const int i16 = threadIdx.x & 15;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items32;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool live = it < items;
+    const int64_t b = it >> 4;   // (16-row group, block) of this half-warp
+    // transposed input: consecutive groups are consecutive input columns
     const int64_t g = p.transpose ? b % rg_cov : b / nb_cov;
     const int64_t j = p.transpose ? b / rg_cov : b % nb_cov;
-    const int64_t r0 = g * 16;
-    uint32_t code2d = 0;
-    if (p.block2d && j < nb && r0 < R) {   // one scale from the amax of the 16 x 16 block
-      double m = 0.0;
-      for (int i = 0; i < 16 && r0 + i < R; ++i) {
-        double v[16];
-        load_block(p, r0 + i, j, v);
+    const int64_t ro = g * 16 + i16;
+    const bool has = live && ro < R && j < nb;
+    double v[16];
+    double m = 0.0;
+    if (has) {
+      load_block(p, ro, j, v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
-      }
-      code2d = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
+      for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
     }
-    for (int i = 0; i < 16; ++i) {
-      const int64_t ro = r0 + i;
-      uint32_t scode = 0;
-      if (ro < R && j < nb) {
-        double v[16];
-        load_block(p, ro, j, v);
-        if (p.block2d) {
-          scode = code2d;
-        } else {
-          double m = 0.0;
+    if (p.block2d) {   // one scale from the amax of the 16 x 16 block
 #pragma unroll
-          for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
-          scode = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
-        }
-        const double dec = e4m3_exact(scode);
-        uint32_t lo = 0, hi = 0;
-        if (dec != 0.0) {
-          const float sc = __fmul_rn(static_cast<float>(dec), s_g);
-          float q[16];
+      for (int off = 8; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+    }
+    if (!live) continue;
+    uint32_t scode = 0;
+    if (has) {
+      scode = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
+      const double dec = e4m3_exact(scode);
+      uint32_t lo = 0, hi = 0;
+      if (dec != 0.0) {
+        const float sc = __fmul_rn(static_cast<float>(dec), s_g);
+        float q[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(v[e] / static_cast<double>(sc));
-          if (p.sr) {
-            float u[16];
-            sr_uniforms16(static_cast<uint64_t>(ro) * C + j * 16, p.seed, p.stream, u);
+        for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(v[e] / static_cast<double>(sc));
+        if (p.sr) {
+          float u[16];
+          sr_uniforms16(static_cast<uint64_t>(ro) * C + j * 16, p.seed, p.stream, u);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const uint32_t c = e2m1_sr(q[e], u[e]);
-              if (e < 8) lo |= c << (4 * e);
-              else hi |= c << (4 * (e - 8));
-            }
-          } else {   // round to nearest even (hardware conversion, element 2k in the low nibble)
-            lo = cvt_e2m1_x8(q);
-            hi = cvt_e2m1_x8(q + 8);
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t c = e2m1_sr(q[e], u[e]);
+            if (e < 8) lo |= c << (4 * e);
+            else hi |= c << (4 * (e - 8));
           }
+        } else {   // round to nearest even (hardware conversion, element 2k in the low nibble)
+          lo = cvt_e2m1_x8(q);
+          hi = cvt_e2m1_x8(q + 8);
         }
-        *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(lo, hi);
-      } else if (ro < R && j < nb_store) {
-        *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(0u, 0u);
       }
-      if (p.tiled) {
-        if (ro < ((R + 127) / 128) * 128) p.sf[tiled_off(ro, j, groups64)] = static_cast<uint8_t>(scode);
-      } else if (ro < R && j < nb_store) {
-        p.sf[ro * nb_store + j] = static_cast<uint8_t>(scode);
-      }
+      *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(lo, hi);
+    } else if (ro < R && j < nb_store) {
+      *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(0u, 0u);
+    }
+    if (p.tiled) {
+      if (ro < ((R + 127) / 128) * 128) p.sf[tiled_off(ro, j, groups64)] = static_cast<uint8_t>(scode);
+    } else if (ro < R && j < nb_store) {
+      p.sf[ro * nb_store + j] = static_cast<uint8_t>(scode);
     }
   }
 }
@@ -280,7 +299,7 @@ int nvfp4x_partials(int64_t blocks) {
 lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, int64_t cols, uint32_t flags,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
-                                     cudaStream_t s, int64_t out_pitch) {
+                                     cudaStream_t s, int64_t out_pitch, int groups) {
   QxParams p = {};
   p.in = in;
   p.bf16 = in_dtype == LMOE_BF16;
@@ -301,21 +320,28 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   const int64_t R = p.transpose ? cols : rows, C = p.transpose ? rows : cols;
   p.pitch = out_pitch > 0 ? out_pitch : C;
   if (p.pitch < C || p.pitch % 16) return LMOE_ERR_INVALID_ARG;
+  // groups share one SR stream, so stochastic rounding stays one group per launch
+  if (groups < 1 || groups > 65535 || (groups > 1 && (p.sr || global_in))) return LMOE_ERR_INVALID_ARG;
   if (R == 0) return LMOE_OK;
+  const int64_t groups64 = (p.pitch + 63) / 64;
+  p.gs_in = rows * cols;
+  p.gs_codes = R * p.pitch / 2;
+  p.gs_sf = p.tiled ? (R + 127) / 128 * groups64 * 512 : R * (p.pitch / 16);
   const int sms = device_sm_count();
   const int np = nvfp4x_partials(R * (C / 16));
   if (!global_in) {
-    launch_k(qx_amax_kernel, dim3(np), dim3(kXThreads), 0, s, p, partials);
+    launch_k(qx_amax_kernel, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);
     count_launch();
   }
   p.partials = partials;
   p.np = global_in ? 0 : np;
   const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;
-  const int64_t nb_cov = p.tiled ? (p.pitch + 63) / 64 * 4 : p.pitch / 16;
-  int64_t blocks = (rg_cov * nb_cov + kXThreads - 1) / kXThreads;
-  if (blocks > static_cast<int64_t>(sms) * 8) blocks = static_cast<int64_t>(sms) * 8;
+  const int64_t nb_cov = p.tiled ? groups64 * 4 : p.pitch / 16;
+  int64_t blocks = (rg_cov * nb_cov * 16 + kXThreads - 1) / kXThreads;
+  const int64_t cap = (static_cast<int64_t>(sms) * 8 + groups - 1) / groups;
+  if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  launch_k(qx_encode_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kXThreads), 0, s, p);
+  launch_k(qx_encode_kernel, dim3(static_cast<unsigned>(blocks), groups), dim3(kXThreads), 0, s, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

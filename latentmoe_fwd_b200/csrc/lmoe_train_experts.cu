@@ -137,7 +137,7 @@ unsigned grid_for(int64_t items) {
 
 // Workspace carve-up (all offsets 256-byte aligned).
 struct BwLayout {
-  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, wtc, wts, wtg, h, aqc, aqs, o, d_o, dh, deq, qac, qas, qag, dA,
+  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w1tg, w2tc, w2ts, w2tg, h, aqc, aqs, o, d_o, dh, deq, qac, qas, qag, dA,
       t1c, t1s, t1g, t2c, t2s, t2g, part, tab, total;
   int64_t P, Rmax, R128max, K256max;
 };
@@ -164,9 +164,12 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax) {
   L.w2c = take(N * l * m / 2);
   L.w2s = take(N * l * m / 16);
   L.w2g = take(N * 4);
-  L.wtc = take(l * m / 2);
-  L.wts = take(l * m / 16);
-  L.wtg = take(4);
+  L.w1tc = take(N * l * m / 2);   // transposed weights (dgrad operands), every expert
+  L.w1ts = take(N * l * m / 16);
+  L.w1tg = take(N * 4);
+  L.w2tc = take(N * l * m / 2);
+  L.w2ts = take(N * l * m / 16);
+  L.w2tg = take(N * 4);
   L.h = take(P * m * 4);
   L.aqc = take(P * m / 2);
   L.aqs = take(P * m / 16);
@@ -184,8 +187,10 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax) {
   L.t2c = take(lm * L.K256max / 2);
   L.t2s = take(lm * L.K256max / 16);
   L.t2g = take(4);
-  const int64_t qx_blocks = (m * l > Rmax * lm ? m * l : Rmax * lm) / 16;
-  L.part = take(static_cast<size_t>(nvfp4x_partials(qx_blocks > 0 ? qx_blocks : 1)) * 8);
+  // amax partials: the grouped weight launches (N groups) or one gradient operand
+  const int64_t np_w = N * nvfp4x_partials(m * l / 16 > 0 ? m * l / 16 : 1);
+  const int64_t np_g = nvfp4x_partials(Rmax * lm / 16 > 0 ? Rmax * lm / 16 : 1);
+  L.part = take(static_cast<size_t>(np_w > np_g ? np_w : np_g) * 8);
   L.tab = take((N * 4 + 8) * 4);   // per expert {0, n, 0, R128}; then {0, l, 0, l}, {0, m, 0, m}
   L.total = off;
   return L;
@@ -301,17 +306,25 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   const int32_t* off_l = dtab + 4 * N;       // {0, l}
   const int32_t* off_m = dtab + 4 * N + 4;   // {0, m}
 
-  // forward weights: every expert's W1 [m][l] and W2 [l][m] with 16 x 16 blocks (current amax)
-  for (int e = 0; e < N && st == LMOE_OK; ++e) {
-    st = launch_nvfp4_quantize_ex(W1 + e * m * l, LMOE_BF16, m, l, 0, 0, 0, 0, nullptr,
-                                  at<uint8_t>(ws, L.w1c) + e * m * l / 2, at<uint8_t>(ws, L.w1s) + e * m * l / 16,
-                                  at<float>(ws, L.w1g) + e, tiled2d, part, s);
-    if (st == LMOE_OK)
-      st = launch_nvfp4_quantize_ex(W2 + e * l * m, LMOE_BF16, l, m, 0, 0, 0, 0, nullptr,
-                                    at<uint8_t>(ws, L.w2c) + e * l * m / 2, at<uint8_t>(ws, L.w2s) + e * l * m / 16,
-                                    at<float>(ws, L.w2g) + e, tiled2d, part, s);
-  }
-  if (st != LMOE_OK) return st;
+  // every expert's weights with 16 x 16 blocks (current amax per expert and
+  // matrix), one grouped launch each: W1 [m][l] and W2 [l][m] for the forward,
+  // W2^T [m][l] and W1^T [l][m] for the dgrads
+  if ((st = launch_nvfp4_quantize_ex(W1, LMOE_BF16, m, l, 0, 0, 0, 0, nullptr, at<uint8_t>(ws, L.w1c),
+                                     at<uint8_t>(ws, L.w1s), at<float>(ws, L.w1g), tiled2d, part, s, 0, N)) !=
+      LMOE_OK)
+    return st;
+  if ((st = launch_nvfp4_quantize_ex(W2, LMOE_BF16, l, m, 0, 0, 0, 0, nullptr, at<uint8_t>(ws, L.w2c),
+                                     at<uint8_t>(ws, L.w2s), at<float>(ws, L.w2g), tiled2d, part, s, 0, N)) !=
+      LMOE_OK)
+    return st;
+  if ((st = launch_nvfp4_quantize_ex(W2, LMOE_BF16, l, m, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr,
+                                     at<uint8_t>(ws, L.w2tc), at<uint8_t>(ws, L.w2ts), at<float>(ws, L.w2tg), tiled2d,
+                                     part, s, 0, N)) != LMOE_OK)
+    return st;
+  if ((st = launch_nvfp4_quantize_ex(W1, LMOE_BF16, m, l, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr,
+                                     at<uint8_t>(ws, L.w1tc), at<uint8_t>(ws, L.w1ts), at<float>(ws, L.w1tg), tiled2d,
+                                     part, s, 0, N)) != LMOE_OK)
+    return st;
 
   // recomputed forward over all slots: h (BF16), aq (NVFP4 with the static s_a), o (BF16)
   Fp4Launch f;
@@ -356,8 +369,6 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   float* deq = at<float>(ws, L.deq);
   uint8_t *qac = at<uint8_t>(ws, L.qac), *qas = at<uint8_t>(ws, L.qas);
   float* qag = at<float>(ws, L.qag);
-  uint8_t *wtc = at<uint8_t>(ws, L.wtc), *wts = at<uint8_t>(ws, L.wts);
-  float* wtg = at<float>(ws, L.wtg);
   uint8_t *t1c = at<uint8_t>(ws, L.t1c), *t1s = at<uint8_t>(ws, L.t1s);
   uint8_t *t2c = at<uint8_t>(ws, L.t2c), *t2s = at<uint8_t>(ws, L.t2s);
   float *t1g = at<float>(ws, L.t1g), *t2g = at<float>(ws, L.t2g);
@@ -410,10 +421,9 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
     if ((st = launch_nvfp4_quantize_ex(d_o, LMOE_F32, R, l, LMOE_QX_SR, rht_signs, seed, st_dg2, nullptr, qac, qas,
                                        qag, LMOE_SF_MMA_TILED, part, s)) != LMOE_OK)
       break;
-    if ((st = launch_nvfp4_quantize_ex(W2 + e * l * m, LMOE_BF16, l, m, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr, wtc, wts,
-                                       wtg, tiled2d, part, s)) != LMOE_OK)
+    if ((st = gemm1(qac, qas, qag, R128, off_e, at<uint8_t>(ws, L.w2tc) + e * l * m / 2,
+                    at<uint8_t>(ws, L.w2ts) + e * l * m / 16, at<float>(ws, L.w2tg) + e, m, l, dA, m, 1)) != LMOE_OK)
       break;
-    if ((st = gemm1(qac, qas, qag, R128, off_e, wtc, wts, wtg, m, l, dA, m, 1)) != LMOE_OK) break;
     // dh
     launch_k(bw_dh_kernel, dim3(grid_for(static_cast<int64_t>(R) * m)), dim3(kBwThreads), 0, s, dA, h, p0, n, R,
              static_cast<int>(m), dh);
@@ -437,11 +447,9 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
     if ((st = launch_nvfp4_quantize_ex(dh, LMOE_F32, R, m, LMOE_QX_SR, rht_signs, seed, st_dg1, nullptr, qac, qas,
                                        qag, LMOE_SF_MMA_TILED, part, s)) != LMOE_OK)
       break;
-    if ((st = launch_nvfp4_quantize_ex(W1 + e * m * l, LMOE_BF16, m, l, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr, wtc, wts,
-                                       wtg, tiled2d, part, s)) != LMOE_OK)
-      break;
-    if ((st = gemm1(qac, qas, qag, R128, off_e, wtc, wts, wtg, l, m, static_cast<__nv_bfloat16*>(dz) + p0 * l, l,
-                    0)) != LMOE_OK)
+    if ((st = gemm1(qac, qas, qag, R128, off_e, at<uint8_t>(ws, L.w1tc) + e * l * m / 2,
+                    at<uint8_t>(ws, L.w1ts) + e * l * m / 16, at<float>(ws, L.w1tg) + e, l, m,
+                    static_cast<__nv_bfloat16*>(dz) + p0 * l, l, 0)) != LMOE_OK)
       break;
     // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
     launch_k(bw_dequant_kernel, dim3(grid_for(static_cast<int64_t>(R) * l / 2)), dim3(kBwThreads), 0, s, z_codes,

@@ -90,6 +90,29 @@ def test_transposed_weight_2d_blocks_bit_exact():
     assert np.array_equal(O.nvfp4_dequantize(rc, rsf, rg), O.nvfp4_dequantize(wc, wsf, rg).T)
 
 
+@pytest.mark.parametrize("layout", ["rowmajor", "tiled"])
+def test_ragged_2d_blocks_bit_exact(layout):
+    # 40 rows: the last 16 x 16 blocks hold 8 rows (the rest count as 0)
+    W = _data(40, 96, 9)
+    lay = (L.SF_ROWMAJOR if layout == "rowmajor" else L.SF_MMA_TILED) | L.SF_BLOCK_16X16
+    if layout == "tiled":
+        codes = torch.empty((40, 48), dtype=torch.uint8, device="cuda")
+        sf = torch.zeros((40 + 127) // 128 * ((96 + 63) // 64) * 512, dtype=torch.uint8, device="cuda")
+        g = torch.empty(1, dtype=torch.float32, device="cuda")
+        L.nvfp4_quantize_ex(to_dev(W, "bf16"), L.BF16, 40, 96, 0, SIGN_BITS, 0, 0, None, codes, sf, g, lay)
+        torch.cuda.synchronize()
+        codes, sf, g = codes.cpu().numpy(), sf.cpu().numpy(), float(g.item())
+        rc, rsf, rg = O.nvfp4_quantize_2d(O.from_bf16_bits(W))
+        assert g == np.float32(rg) and np.array_equal(codes, rc)
+        r, j = np.arange(40)[:, None], np.arange(96 // 16)[None, :]   # the documented MMA-tiled offsets
+        off = ((r >> 7) * ((96 + 63) // 64) + (j >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (j & 3)
+        assert np.array_equal(sf[off], rsf)
+        return
+    codes, sf, g = _quantize_ex(W, 40, 96, 0, layout=lay)
+    rc, rsf, rg = O.nvfp4_quantize_2d(O.from_bf16_bits(W))
+    assert g == np.float32(rg) and np.array_equal(sf, rsf) and np.array_equal(codes, rc)
+
+
 def test_plain_mode_equals_nvfp4_quantize():
     bits = _data(130, 64, 2)
     codes, sf, g = _quantize_ex(bits, 130, 64, 0)
