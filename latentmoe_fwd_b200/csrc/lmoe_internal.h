@@ -197,6 +197,17 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
                                      cudaStream_t s, int64_t out_pitch = 0, int groups = 1);
+// Ragged groups: group g quantises input rows [gtab[5g], gtab[5g] + gtab[5g+1])
+// of a [*][cols] input as one matrix (own global scale global_out[g], SR
+// stream stream0 + g * stream_step), codes at codes + gtab[5g+2], scales at
+// sf + gtab[5g+3], output pitch gtab[5g+4] (0: the output's columns).
+// rows_max / pitch_max bound every group's rows and pitch (grid sizing);
+// partials holds groups * nvfp4x_partials(out_rows_max * pitch_max / 16) doubles.
+lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t rows_max, int64_t cols,
+                                         uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
+                                         uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
+                                         uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
+                                         double* partials, cudaStream_t s);
 // Dense BF16 GEMM on the tensor cores (lmoe_api.cu): out[rows][cols] =
 // epi(x[rows][k] . w[cols][k]^T), token-major tiles, or weight-major ones for
 // rows <= 64 (split-K into `partial` when given). epi: EPI_* of gemm_tc.cuh

@@ -87,6 +87,11 @@ struct QxParams {
   // grouped launches (gridDim.y groups, one matrix each, with its own global
   // scale): strides between the groups' inputs (elements), codes and scales (bytes)
   int64_t gs_in, gs_codes, gs_sf;
+  // ragged groups instead (gtab non-null): per group {first input row, input
+  // rows, codes offset, scales offset (bytes), output pitch (0: out cols)};
+  // group g draws its SR uniforms on stream + g * stream_step
+  const int64_t* gtab;
+  uint32_t stream_step;
 };
 
 // The parameters of group blockIdx.y: its input, outputs, global scale and
@@ -94,7 +99,17 @@ struct QxParams {
 __device__ __forceinline__ QxParams qx_group(const QxParams& p0) {
   QxParams p = p0;
   const int64_t g = blockIdx.y;
-  if (g) {
+  if (p0.gtab) {
+    const int64_t* t = p0.gtab + g * 5;
+    p.in = static_cast<const uint8_t*>(p0.in) + t[0] * p0.cols * (p0.bf16 ? 2 : 4);
+    p.rows = t[1];
+    p.codes += t[2];
+    p.sf += t[3];
+    p.pitch = t[4] > 0 ? t[4] : (p0.transpose ? t[1] : p0.cols);
+    p.stream = p0.stream + static_cast<uint32_t>(g) * p0.stream_step;
+    if (p.global_out) p.global_out += g;
+    if (p.partials) p.partials += g * p0.np;
+  } else if (g) {
     p.in = static_cast<const uint8_t*>(p0.in) + g * p0.gs_in * (p0.bf16 ? 2 : 4);
     p.codes += g * p0.gs_codes;
     p.sf += g * p0.gs_sf;
@@ -166,29 +181,25 @@ __global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, d
   }
 }
 
-// E2M1 grid magnitudes by code.
-__device__ __forceinline__ double e2m1_mag(int c) {
-  constexpr double g[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
-  return g[c];
-}
-
 // Stochastic E2M1 code of v (fp32 value): |v| >= 6 -> 6; else, between grid
 // neighbours lo <= |v| < hi, hi when u * (hi - lo) < |v| - lo (exact
-// comparison), else lo; the sign bit is the sign of v.
+// comparison), else lo; the sign bit is the sign of v. The grid (0, 0.5, 1,
+// 1.5, 2, 3, 4, 6) is walked with compares and selects, so nothing is indexed
+// at run time.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, float u) {
   const double a = fabs(static_cast<double>(v));
-  int lo = 0;
-#pragma unroll
-  for (int c = 1; c < 8; ++c)
-    if (a >= e2m1_mag(c)) lo = c;
-  int code = lo;
-  if (a >= 6.0) {
-    code = 7;
-  } else {
-    const double l = e2m1_mag(lo), h = e2m1_mag(lo + 1);
-    if (static_cast<double>(u) * (h - l) < a - l) code = lo + 1;
-  }
-  return static_cast<uint32_t>(code) | (signbit(v) ? 8u : 0u);
+  uint32_t lo = 0;
+  double l = 0.0, h = 0.5;
+  if (a >= 0.5) { lo = 1; l = 0.5; h = 1.0; }
+  if (a >= 1.0) { lo = 2; l = 1.0; h = 1.5; }
+  if (a >= 1.5) { lo = 3; l = 1.5; h = 2.0; }
+  if (a >= 2.0) { lo = 4; l = 2.0; h = 3.0; }
+  if (a >= 3.0) { lo = 5; l = 3.0; h = 4.0; }
+  if (a >= 4.0) { lo = 6; l = 4.0; h = 6.0; }
+  uint32_t code = lo;
+  if (a >= 6.0) code = 7;
+  else if (static_cast<double>(u) * (h - l) < a - l) code = lo + 1;
+  return code | (signbit(v) ? 8u : 0u);
 }
 
 __device__ __forceinline__ int64_t tiled_off(int64_t row, int64_t j, int64_t groups64) {
@@ -337,6 +348,51 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   p.np = global_in ? 0 : np;
   const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;
   const int64_t nb_cov = p.tiled ? groups64 * 4 : p.pitch / 16;
+  int64_t blocks = (rg_cov * nb_cov * 16 + kXThreads - 1) / kXThreads;
+  const int64_t cap = (static_cast<int64_t>(sms) * 8 + groups - 1) / groups;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  launch_k(qx_encode_kernel, dim3(static_cast<unsigned>(blocks), groups), dim3(kXThreads), 0, s, p);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t rows_max, int64_t cols,
+                                         uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
+                                         uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
+                                         uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
+                                         double* partials, cudaStream_t s) {
+  if (groups < 1 || groups > 65535 || !gtab || !global_out || rows_max < 0 || cols <= 0 || cols % 16)
+    return LMOE_ERR_INVALID_ARG;
+  QxParams p = {};
+  p.in = in;
+  p.bf16 = in_dtype == LMOE_BF16;
+  p.rows = rows_max;
+  p.cols = cols;
+  p.transpose = (flags & LMOE_QX_TRANSPOSE) != 0;
+  p.rht = (flags & LMOE_QX_RHT) != 0;
+  p.signs = rht_signs & 0xFFFFu;
+  p.sr = (flags & LMOE_QX_SR) != 0;
+  p.seed = seed;
+  p.stream = stream0;
+  p.stream_step = stream_step;
+  p.block2d = (sf_layout & LMOE_SF_BLOCK_16X16) != 0;
+  p.tiled = (sf_layout & ~LMOE_SF_BLOCK_16X16) == LMOE_SF_MMA_TILED;
+  p.codes = codes;
+  p.sf = sf;
+  p.global_out = global_out;
+  p.gtab = gtab;
+  const int64_t R = p.transpose ? cols : rows_max, C = p.transpose ? rows_max : cols;
+  const int64_t pitch = pitch_max > C ? pitch_max : C;
+  if (pitch % 16) return LMOE_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const int np = nvfp4x_partials(R * (pitch / 16) > 0 ? R * (pitch / 16) : 1);
+  launch_k(qx_amax_kernel, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);
+  count_launch();
+  p.partials = partials;
+  p.np = np;
+  const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;
+  const int64_t nb_cov = p.tiled ? (pitch + 63) / 64 * 4 : pitch / 16;
   int64_t blocks = (rg_cov * nb_cov * 16 + kXThreads - 1) / kXThreads;
   const int64_t cap = (static_cast<int64_t>(sms) * 8 + groups - 1) / groups;
   if (blocks > cap) blocks = cap;

@@ -16,9 +16,12 @@
 //   dh = dA * 2 max(h, 0)
 //   dz = SR(dh) W1q,          dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
 // with SR uniforms from Philox-4x32-10 on stream 4 e + 2 g + j (g: 0 first
-// GEMM, 1 second; j: 0 dgrad, 1 wgrad). The host walks the experts; every
-// step is a kernel of this library (the training quantiser, the grouped
-// NVFP4 GEMM, and the three small kernels below).
+// GEMM, 1 second; j: 0 dgrad, 1 wgrad). Every step but the wgrads runs as one
+// launch over all experts: the quantiser with a group per expert (its own
+// global scale and SR stream), the grouped NVFP4 GEMM for the forward
+// recompute and both dgrads, and the three small kernels below with a grid
+// row per expert. The wgrads contract over each expert's own token count, so
+// the host issues one GEMM per expert and wgrad.
 #include <cuda_bf16.h>
 
 #include <vector>
@@ -34,54 +37,61 @@ constexpr int kBwThreads = 256;
 size_t up256(size_t b) { return (b + 255) / 256 * 256; }
 int64_t ceil_to(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
-// do[r][:] = gate * dy for r < n (fp32; rows n..R-1 zero); dgate[r] = dy . o.
-// A block per row r < R.
+// Per expert e (blockIdx.y), etab[4e..4e+3] = {first padded row p0, rows n,
+// rows R (n rounded up to 16), first wgrad K column}.
+
+// do[p0 + r][:] = gate * dy for r < n (fp32; rows n..R-1 zero); dgate[p0 + r]
+// = dy . o. A block per row.
 __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const float* __restrict__ dy,
                                                               const float* __restrict__ o,
-                                                              const float* __restrict__ gate, int64_t row0, int n,
-                                                              int l, float* __restrict__ d_o,
-                                                              float* __restrict__ dgate) {
+                                                              const float* __restrict__ gate,
+                                                              const int64_t* __restrict__ etab, int l,
+                                                              float* __restrict__ d_o, float* __restrict__ dgate) {
   pdl_begin();
   __shared__ float red[kBwThreads / 32];
-  const int r = blockIdx.x;
-  float* out = d_o + static_cast<int64_t>(r) * l;
-  if (r >= n) {
-    for (int j = threadIdx.x; j < l; j += blockDim.x) out[j] = 0.0f;
-    return;
-  }
-  const int64_t row = row0 + r;
-  const float g = __ldg(gate + row);
-  float dot = 0.0f;
-  for (int j = threadIdx.x; j < l; j += blockDim.x) {
-    const float d = dy[row * l + j];
-    dot = fmaf(d, o[row * l + j], dot);
-    out[j] = __fmul_rn(g, d);
-  }
+  const int64_t* t = etab + 4 * blockIdx.y;
+  const int64_t p0 = t[0], n = t[1], R = t[2];
+  for (int64_t r = blockIdx.x; r < R; r += gridDim.x) {
+    const int64_t row = p0 + r;
+    float* out = d_o + row * l;
+    if (r >= n) {
+      for (int j = threadIdx.x; j < l; j += blockDim.x) out[j] = 0.0f;
+      continue;
+    }
+    const float g = __ldg(gate + row);
+    float dot = 0.0f;
+    for (int j = threadIdx.x; j < l; j += blockDim.x) {
+      const float d = dy[row * l + j];
+      dot = fmaf(d, o[row * l + j], dot);
+      out[j] = __fmul_rn(g, d);
+    }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dot;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.0f;
-    for (int i = 0; i < kBwThreads / 32; ++i) s += red[i];
-    dgate[row] = s;
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dot;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.0f;
+      for (int i = 0; i < kBwThreads / 32; ++i) s += red[i];
+      dgate[row] = s;
+    }
+    __syncthreads();   // red is reused by the block's next row
   }
 }
 
-// dh[r][c] = dA[r][c] * 2 max(h[row0 + r][c], 0) for r < n, 0 for n <= r < R.
+// dh[p0 + r][c] = dA[p0 + r][c] * 2 max(h[p0 + r][c], 0) for r < n, 0 for n <= r < R.
 __global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const float* __restrict__ dA,
-                                                            const float* __restrict__ h, int64_t row0,
-                                                            int n, int R, int m, float* __restrict__ dh) {
+                                                            const float* __restrict__ h,
+                                                            const int64_t* __restrict__ etab, int m,
+                                                            float* __restrict__ dh) {
   pdl_begin();
-  const int64_t total = static_cast<int64_t>(R) * m;
+  const int64_t* t = etab + 4 * blockIdx.y;
+  const int64_t p0 = t[0], n = t[1], R = t[2];
+  const int64_t total = R * m;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = i / m, c = i % m;
-    float v = 0.0f;
-    if (r < n) {
-      v = dA[r * m + c] * (2.0f * fmaxf(h[(row0 + r) * m + c], 0.0f));
-    }
-    dh[i] = v;
+    const int64_t at = (p0 + r) * m + c;
+    dh[at] = r < n ? dA[at] * (2.0f * fmaxf(h[at], 0.0f)) : 0.0f;
   }
 }
 
@@ -96,25 +106,28 @@ __device__ __forceinline__ double e4m3_val(uint32_t c) {
   return e == 0 ? ldexp(static_cast<double>(f), -9) : ldexp(static_cast<double>(8 + f), e - 10);
 }
 
-// Rows row0 .. row0 + R - 1 of NVFP4 codes [*, cols/2] with MMA-tiled scales
-// (groups64 = cols / 64) and a global scale, as fp32 [R][cols]; rows >= n are
-// zero. Each value is code * block scale * global, formed exactly in fp64
-// (2 + 4 + 24 significant bits) and rounded once to fp32.
+// Rows p0 .. p0 + R - 1 of NVFP4 codes [*, cols/2] with MMA-tiled scales
+// (groups64 = cols / 64) and a global scale, as fp32 [*][cols] at the same
+// rows; rows >= p0 + n are zero. Each value is code * block scale * global,
+// formed exactly in fp64 (2 + 4 + 24 significant bits) and rounded once to fp32.
 __global__ void __launch_bounds__(kBwThreads) bw_dequant_kernel(const uint8_t* __restrict__ codes,
                                                                  const uint8_t* __restrict__ sf,
-                                                                 const float* __restrict__ global, int64_t row0,
-                                                                 int n, int R, int cols, float* __restrict__ out) {
+                                                                 const float* __restrict__ global,
+                                                                 const int64_t* __restrict__ etab, int cols,
+                                                                 float* __restrict__ out) {
   pdl_begin();
+  const int64_t* t = etab + 4 * blockIdx.y;
+  const int64_t p0 = t[0], n = t[1], R = t[2];
   const double s_g = static_cast<double>(__ldg(global));
   const int groups64 = cols / 64;
-  const int64_t total = static_cast<int64_t>(R) * (cols / 2);
+  const int64_t total = R * (cols / 2);
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = i / (cols / 2);
     const int cb = static_cast<int>(i % (cols / 2));   // byte: elements 2 cb, 2 cb + 1
+    const int64_t row = p0 + r;
     float v0 = 0.0f, v1 = 0.0f;
     if (r < n) {
-      const int64_t row = row0 + r;
       const uint32_t b = codes[row * (cols / 2) + cb];
       const int j = (2 * cb) / 16;
       const int64_t so = ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
@@ -123,33 +136,36 @@ __global__ void __launch_bounds__(kBwThreads) bw_dequant_kernel(const uint8_t* _
       v0 = __double2float_rn((c0 & 8u ? -1.0 : 1.0) * e2m1_mag(c0 & 7u) * sc);
       v1 = __double2float_rn((c1 & 8u ? -1.0 : 1.0) * e2m1_mag(c1 & 7u) * sc);
     }
-    out[r * cols + 2 * cb] = v0;
-    out[r * cols + 2 * cb + 1] = v1;
+    out[row * cols + 2 * cb] = v0;
+    out[row * cols + 2 * cb + 1] = v1;
   }
 }
 
-unsigned grid_for(int64_t items) {
+// Grid for a per-expert loop over `items` (x), one row per expert (y): about
+// eight resident CTAs per SM over all experts.
+dim3 grid_per_expert(int64_t items, int N) {
   const int64_t sms = device_sm_count();
   int64_t b = (items + kBwThreads - 1) / kBwThreads;
-  if (b > sms * 8) b = sms * 8;
-  return static_cast<unsigned>(b < 1 ? 1 : b);
+  const int64_t cap = (sms * 8 + N - 1) / N;
+  if (b > cap) b = cap;
+  return dim3(static_cast<unsigned>(b < 1 ? 1 : b), static_cast<unsigned>(N));
 }
 
 // Workspace carve-up (all offsets 256-byte aligned).
 struct BwLayout {
-  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w1tg, w2tc, w2ts, w2tg, h, aqc, aqs, o, d_o, dh, deq, qac, qas, qag, dA,
-      t1c, t1s, t1g, t2c, t2s, t2g, part, tab, total;
-  int64_t P, Rmax, R128max, K256max;
+  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w1tg, w2tc, w2ts, w2tg, h, aqc, aqs, o, d_o, dh, deq, qac,
+      qas, qag, dA, t1c, t1s, t1g, t2c, t2s, t2g, part, etab, gtab, itab, total;
+  int64_t P, Rmax, Ksum;
 };
 
-// P: padded slot rows; Rmax: the largest expert's rows rounded up to 16.
-BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax) {
+// P: padded slot rows; Rmax: the largest expert's rows rounded up to 16;
+// Ksum: the experts' wgrad contraction lengths (rows rounded up to 256), summed.
+BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ksum) {
   BwLayout L = {};
   const int64_t N = c->N, l = c->l, m = c->m;
   L.P = P;
   L.Rmax = Rmax;
-  L.R128max = ceil_to(Rmax, 128);
-  L.K256max = ceil_to(Rmax, 256);
+  L.Ksum = Ksum;
   const int64_t lm = l > m ? l : m;
   size_t off = 0;
   auto take = [&](size_t b) {
@@ -170,39 +186,48 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax) {
   L.w2tc = take(N * l * m / 2);
   L.w2ts = take(N * l * m / 16);
   L.w2tg = take(N * 4);
+  // every expert's rows at its padded offset
   L.h = take(P * m * 4);
   L.aqc = take(P * m / 2);
   L.aqs = take(P * m / 16);
   L.o = take(P * l * 4);
-  L.d_o = take(Rmax * l * 4);
-  L.dh = take(Rmax * m * 4);
-  L.deq = take(Rmax * lm * 4);
-  L.qac = take(L.R128max * lm / 2);
-  L.qas = take(L.R128max * lm / 16);
-  L.qag = take(4);
-  L.dA = take(L.R128max * m * 4);
-  L.t1c = take(lm * L.K256max / 2);
-  L.t1s = take(lm * L.K256max / 16);
-  L.t1g = take(4);
-  L.t2c = take(lm * L.K256max / 2);
-  L.t2s = take(lm * L.K256max / 16);
-  L.t2g = take(4);
-  // amax partials: the grouped weight launches (N groups) or one gradient operand
-  const int64_t np_w = N * nvfp4x_partials(m * l / 16 > 0 ? m * l / 16 : 1);
-  const int64_t np_g = nvfp4x_partials(Rmax * lm / 16 > 0 ? Rmax * lm / 16 : 1);
-  L.part = take(static_cast<size_t>(np_w > np_g ? np_w : np_g) * 8);
-  L.tab = take((N * 4 + 8) * 4);   // per expert {0, n, 0, R128}; then {0, l, 0, l}, {0, m, 0, m}
+  L.d_o = take(P * l * 4);
+  L.dh = take(P * m * 4);
+  L.deq = take(P * lm * 4);
+  L.qac = take(P * lm / 2);
+  L.qas = take(P * lm / 16);
+  L.qag = take(N * 4);
+  L.dA = take(P * m * 4);
+  // wgrad operands: expert e's [lm][K256_e] matrices back to back
+  L.t1c = take(lm * Ksum / 2);
+  L.t1s = take(lm * Ksum / 16);
+  L.t1g = take(N * 4);
+  L.t2c = take(lm * Ksum / 2);
+  L.t2s = take(lm * Ksum / 16);
+  L.t2g = take(N * 4);
+  // amax partials of the largest grouped quantiser launch
+  const int64_t K256max = ceil_to(Rmax, 256);
+  int64_t np = N * nvfp4x_partials(m * l / 16 > 0 ? m * l / 16 : 1);
+  const int64_t np_rows = N * nvfp4x_partials(Rmax * lm / 16 > 0 ? Rmax * lm / 16 : 1);
+  const int64_t np_t = N * nvfp4x_partials(lm * K256max / 16 > 0 ? lm * K256max / 16 : 1);
+  if (np_rows > np) np = np_rows;
+  if (np_t > np) np = np_t;
+  L.part = take(static_cast<size_t>(np) * 8);
+  L.etab = take(N * 4 * 8);       // per expert {p0, n, R, K offset}
+  L.gtab = take(6 * N * 5 * 8);   // six quantiser group tables
+  L.itab = take(8 * 4);           // wgrad problem offsets
   L.total = off;
   return L;
 }
 
 BwLayout bw_layout(const lmoe_config* c, const int32_t* counts) {
-  int64_t P = 0, Rmax = 0;
+  int64_t P = 0, Rmax = 0, Ksum = 0;
   for (int e = 0; e < c->N; ++e) {
     P += ceil_to(counts[e], 128);
+    Ksum += ceil_to(counts[e], 256);
     if (counts[e] > 0 && ceil_to(counts[e], 16) > Rmax) Rmax = ceil_to(counts[e], 16);
   }
-  return bw_layout_for(c, P, Rmax);
+  return bw_layout_for(c, P, Rmax, Ksum);
 }
 
 template <typename T>
@@ -258,7 +283,9 @@ size_t expert_backward_ws(const lmoe_config* cfg, const int32_t* counts) { retur
 // Enough for any routing of cfg->T tokens: at most padded_rows slot rows, and
 // no expert with more than T rows (a token picks an expert once).
 size_t expert_backward_ws_bound(const lmoe_config* cfg) {
-  return bw_layout_for(cfg, lmoe_padded_rows(cfg), ceil_to(cfg->T > 0 ? cfg->T : 1, 16)).total;
+  const int64_t P = lmoe_padded_rows(cfg);
+  // ceil256(n) <= ceil128(n) + 128 for every expert
+  return bw_layout_for(cfg, P, ceil_to(cfg->T > 0 ? cfg->T : 1, 16), P + 128 * static_cast<int64_t>(cfg->N)).total;
 }
 
 // The routed experts' backward (see lmoe_expert_backward_nvfp4), arguments
@@ -280,31 +307,53 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   const __nv_bfloat16* W2 = static_cast<const __nv_bfloat16*>(w2);
   const int tiled2d = LMOE_SF_MMA_TILED | LMOE_SF_BLOCK_16X16;
 
-  // per-expert GEMM offsets: {0, n, 0, R128}; wgrad problems {0, l, 0, l} and {0, m, 0, m}
-  std::vector<int32_t> tab(static_cast<size_t>(N) * 4 + 8);
-  std::vector<int64_t> poff(N + 1, 0);
+  // per expert {p0, n, R, K offset}; six quantiser group tables {first input
+  // row, rows, codes offset, scales offset, pitch}: 0 SR(do), 1 RHT(do)^T,
+  // 2 RHT(aq)^T, 3 SR(dh), 4 RHT(dh)^T, 5 RHT(zq)^T
+  std::vector<int64_t> etab(static_cast<size_t>(N) * 4), gtab(static_cast<size_t>(6) * N * 5);
+  int64_t p0 = 0, koff = 0;
   for (int e = 0; e < N; ++e) {
-    const int64_t n = counts[e];
-    tab[4 * e + 0] = 0;
-    tab[4 * e + 1] = static_cast<int32_t>(n);
-    tab[4 * e + 2] = 0;
-    tab[4 * e + 3] = static_cast<int32_t>(ceil_to(ceil_to(n, 16), 128));
-    poff[e + 1] = poff[e] + ceil_to(n, 128);
+    const int64_t n = counts[e], R = ceil_to(n, 16), K256 = ceil_to(n, 256);
+    etab[4 * e + 0] = p0;
+    etab[4 * e + 1] = n;
+    etab[4 * e + 2] = R;
+    etab[4 * e + 3] = koff;
+    auto row_group = [&](int t, int64_t cols) {   // [R][cols] at the expert's padded rows
+      int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 5;
+      g[0] = p0;
+      g[1] = R;
+      g[2] = p0 * cols / 2;
+      g[3] = p0 * cols / 16;   // p0 is a multiple of 128: whole scale atoms
+      g[4] = 0;
+    };
+    auto t_group = [&](int t, int64_t out_rows) {   // [out_rows][K256] after the expert's predecessors
+      int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 5;
+      g[0] = p0;
+      g[1] = R;
+      g[2] = out_rows * koff / 2;
+      g[3] = out_rows * koff / 16;
+      g[4] = K256;
+    };
+    row_group(0, l);
+    t_group(1, l);
+    t_group(2, m);
+    row_group(3, m);
+    t_group(4, m);
+    t_group(5, l);
+    p0 += ceil_to(n, 128);
+    koff += K256;
   }
-  int32_t* tail = tab.data() + 4 * N;
-  tail[0] = 0;
-  tail[1] = static_cast<int32_t>(l);
-  tail[2] = 0;
-  tail[3] = static_cast<int32_t>(l);
-  tail[4] = 0;
-  tail[5] = static_cast<int32_t>(m);
-  tail[6] = 0;
-  tail[7] = static_cast<int32_t>(m);
-  int32_t* dtab = at<int32_t>(ws, L.tab);
-  if (cudaMemcpyAsync(dtab, tab.data(), tab.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  // wgrad problems: one group of l (or m) rows, {0, rows, 0, rows}
+  const int32_t itab[8] = {0, static_cast<int32_t>(l), 0, static_cast<int32_t>(l),
+                           0, static_cast<int32_t>(m), 0, static_cast<int32_t>(m)};
+  int64_t* d_etab = at<int64_t>(ws, L.etab);
+  int64_t* d_gtab = at<int64_t>(ws, L.gtab);
+  int32_t* d_itab = at<int32_t>(ws, L.itab);
+  if (cudaMemcpyAsync(d_etab, etab.data(), etab.size() * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(d_gtab, gtab.data(), gtab.size() * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(d_itab, itab, sizeof(itab), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return LMOE_ERR_CUDA;
-  const int32_t* off_l = dtab + 4 * N;       // {0, l}
-  const int32_t* off_m = dtab + 4 * N + 4;   // {0, m}
+  auto gt = [&](int t) { return d_gtab + static_cast<size_t>(t) * N * 5; };
 
   // every expert's weights with 16 x 16 blocks (current amax per expert and
   // matrix), one grouped launch each: W1 [m][l] and W2 [l][m] for the forward,
@@ -326,43 +375,57 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                                      part, s, 0, N)) != LMOE_OK)
     return st;
 
-  // recomputed forward over all slots: h (BF16), aq (NVFP4 with the static s_a), o (BF16)
-  Fp4Launch f;
-  f.a_codes = z_codes;
-  f.a_sf = z_sf;
-  f.a_rows = L.P;
-  f.b_codes = at<uint8_t>(ws, L.w1c);
-  f.b_sf = at<uint8_t>(ws, L.w1s);
-  f.k = l;
-  f.cols = static_cast<int>(m);
-  f.groups = N;
-  f.offsets = offsets;
-  f.padded_offsets = padded_offsets;
-  f.in_scale = z_global;
-  f.w_scale = at<float>(ws, L.w1g);
-  f.out = at<void>(ws, L.h);
-  f.ld_out = m;
-  f.f32_out = 1;
-  if (L.P > 0 && (st = fp4_gemm(f, err, s)) != LMOE_OK) return st;
-  Fp4Launch fq = f;
-  fq.quant_out = 1;
-  fq.f32_out = 0;
-  fq.out_scale = a_global;
-  fq.out = at<void>(ws, L.aqc);
-  fq.out_sf = at<uint8_t>(ws, L.aqs);
-  if (L.P > 0 && (st = fp4_gemm(fq, err, s)) != LMOE_OK) return st;
-  Fp4Launch f2 = f;   // fp32 out, as f
-  f2.a_codes = at<uint8_t>(ws, L.aqc);
-  f2.a_sf = at<uint8_t>(ws, L.aqs);
-  f2.b_codes = at<uint8_t>(ws, L.w2c);
-  f2.b_sf = at<uint8_t>(ws, L.w2s);
-  f2.k = m;
-  f2.cols = static_cast<int>(l);
-  f2.in_scale = a_global;
-  f2.w_scale = at<float>(ws, L.w2g);
-  f2.out = at<void>(ws, L.o);
-  f2.ld_out = l;
-  if (L.P > 0 && (st = fp4_gemm(f2, err, s)) != LMOE_OK) return st;
+  // the expert-grouped NVFP4 GEMM over every expert's padded rows
+  auto grouped = [&](const void* ac, const uint8_t* as, const float* ag, int ag_grouped, const void* bc,
+                     const uint8_t* bs, const float* bg, int64_t cols, int64_t k, void* out, int64_t ld, int f32) {
+    Fp4Launch g;
+    g.a_codes = ac;
+    g.a_sf = as;
+    g.a_rows = L.P;
+    g.b_codes = bc;
+    g.b_sf = bs;
+    g.k = k;
+    g.cols = static_cast<int>(cols);
+    g.groups = N;
+    g.offsets = offsets;
+    g.padded_offsets = padded_offsets;
+    g.in_scale = ag;
+    g.in_scale_grouped = ag_grouped;
+    g.w_scale = bg;
+    g.out = out;
+    g.ld_out = ld;
+    g.f32_out = f32;
+    return L.P > 0 ? fp4_gemm(g, err, s) : LMOE_OK;
+  };
+
+  // recomputed forward over all slots: h (fp32), aq (NVFP4 with the static s_a), o (fp32)
+  if ((st = grouped(z_codes, z_sf, z_global, 0, at<uint8_t>(ws, L.w1c), at<uint8_t>(ws, L.w1s),
+                    at<float>(ws, L.w1g), m, l, at<void>(ws, L.h), m, 1)) != LMOE_OK)
+    return st;
+  {
+    Fp4Launch fq;
+    fq.a_codes = z_codes;
+    fq.a_sf = z_sf;
+    fq.a_rows = L.P;
+    fq.b_codes = at<uint8_t>(ws, L.w1c);
+    fq.b_sf = at<uint8_t>(ws, L.w1s);
+    fq.k = l;
+    fq.cols = static_cast<int>(m);
+    fq.groups = N;
+    fq.offsets = offsets;
+    fq.padded_offsets = padded_offsets;
+    fq.in_scale = z_global;
+    fq.w_scale = at<float>(ws, L.w1g);
+    fq.quant_out = 1;
+    fq.out_scale = a_global;
+    fq.out = at<void>(ws, L.aqc);
+    fq.out_sf = at<uint8_t>(ws, L.aqs);
+    fq.ld_out = m;
+    if (L.P > 0 && (st = fp4_gemm(fq, err, s)) != LMOE_OK) return st;
+  }
+  if ((st = grouped(at<uint8_t>(ws, L.aqc), at<uint8_t>(ws, L.aqs), a_global, 0, at<uint8_t>(ws, L.w2c),
+                    at<uint8_t>(ws, L.w2s), at<float>(ws, L.w2g), l, m, at<void>(ws, L.o), l, 1)) != LMOE_OK)
+    return st;
 
   float* d_o = at<float>(ws, L.d_o);
   float* dh = at<float>(ws, L.dh);
@@ -375,96 +438,78 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   float* dA = at<float>(ws, L.dA);
   const float* h = at<float>(ws, L.h);
   const float* o = at<float>(ws, L.o);
-
-  // a single-group GEMM out[rows][cols] = A[rows][k] . B[cols][k]^T (BF16 out)
-  auto gemm1 = [&](const uint8_t* ac, const uint8_t* as, const float* ag, int64_t a_rows, const int32_t* off,
-                   const uint8_t* bc, const uint8_t* bs, const float* bg, int64_t cols, int64_t k, void* out,
-                   int64_t ld, int f32) {
-    Fp4Launch g;
-    g.a_codes = ac;
-    g.a_sf = as;
-    g.a_rows = a_rows;
-    g.b_codes = bc;
-    g.b_sf = bs;
-    g.k = k;
-    g.cols = static_cast<int>(cols);
-    g.groups = 1;
-    g.offsets = off;
-    g.padded_offsets = off + 2;
-    g.in_scale = ag;
-    g.w_scale = bg;
-    g.out = out;
-    g.ld_out = ld;
-    g.f32_out = f32;
-    return fp4_gemm(g, err, s);
+  const int64_t K256max = ceil_to(L.Rmax, 256);
+  const uint32_t T_RHT = LMOE_QX_TRANSPOSE | LMOE_QX_RHT;
+  auto quant = [&](int t, const float* in, int64_t cols, uint32_t flags, uint32_t stream0, uint8_t* c, uint8_t* sf,
+                   float* g) {
+    const bool tr = (flags & LMOE_QX_TRANSPOSE) != 0;
+    return launch_nvfp4_quantize_groups(in, LMOE_F32, L.Rmax, cols, flags, rht_signs, seed, stream0, 4, gt(t), N,
+                                        tr ? K256max : cols, c, sf, g, LMOE_SF_MMA_TILED, part, s);
+  };
+  // the wgrad of every expert with rows: out[rows][cols] = A[rows][K256] . B[cols][K256]^T
+  auto wgrads = [&](int64_t rows, int64_t cols, void* dw) -> lmoe_status {
+    for (int e = 0; e < N; ++e) {
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(dw) + e * rows * cols;
+      const int64_t K256 = ceil_to(counts[e], 256), ko = etab[4 * e + 3];
+      if (K256 == 0) {   // no rows: zero weight gradient
+        if (cudaMemsetAsync(out, 0, rows * cols * 2, s) != cudaSuccess) return LMOE_ERR_CUDA;
+        continue;
+      }
+      Fp4Launch g;
+      g.a_codes = t1c + rows * ko / 2;
+      g.a_sf = t1s + rows * ko / 16;
+      g.a_rows = rows;
+      g.b_codes = t2c + cols * ko / 2;
+      g.b_sf = t2s + cols * ko / 16;
+      g.k = K256;
+      g.cols = static_cast<int>(cols);
+      g.groups = 1;
+      g.offsets = d_itab + (rows == l ? 0 : 4);   // {0, rows}
+      g.padded_offsets = g.offsets + 2;
+      g.in_scale = t1g + e;
+      g.w_scale = t2g + e;
+      g.out = out;
+      g.ld_out = cols;
+      lmoe_status r = fp4_gemm(g, err, s);
+      if (r != LMOE_OK) return r;
+    }
+    return LMOE_OK;
   };
 
-  for (int e = 0; e < N && st == LMOE_OK; ++e) {
-    const int n = counts[e];
-    if (n == 0) {   // no rows: zero weight gradients
-      if (cudaMemsetAsync(static_cast<__nv_bfloat16*>(dw1) + e * m * l, 0, m * l * 2, s) != cudaSuccess ||
-          cudaMemsetAsync(static_cast<__nv_bfloat16*>(dw2) + e * l * m, 0, l * m * 2, s) != cudaSuccess)
-        return LMOE_ERR_CUDA;
-      continue;
-    }
-    const int R = static_cast<int>(ceil_to(n, 16));
-    const int64_t R128 = ceil_to(R, 128), K256 = ceil_to(R, 256);
-    const int64_t p0 = poff[e];
-    const int32_t* off_e = dtab + 4 * e;
-    const uint32_t st_dg1 = 4u * e + 0, st_wg1 = 4u * e + 1, st_dg2 = 4u * e + 2, st_wg2 = 4u * e + 3;
-
-    // do, dgate
-    launch_k(bw_prep_kernel, dim3(R), dim3(kBwThreads), 0, s, static_cast<const float*>(dy), o, gate, p0, n,
-             static_cast<int>(l), d_o, dgate);
-    count_launch();
-    // second GEMM, dgrad: dA = SR(do) W2q  (W2^T [m][l] with 16 x 16 blocks)
-    if ((st = launch_nvfp4_quantize_ex(d_o, LMOE_F32, R, l, LMOE_QX_SR, rht_signs, seed, st_dg2, nullptr, qac, qas,
-                                       qag, LMOE_SF_MMA_TILED, part, s)) != LMOE_OK)
-      break;
-    if ((st = gemm1(qac, qas, qag, R128, off_e, at<uint8_t>(ws, L.w2tc) + e * l * m / 2,
-                    at<uint8_t>(ws, L.w2ts) + e * l * m / 16, at<float>(ws, L.w2tg) + e, m, l, dA, m, 1)) != LMOE_OK)
-      break;
-    // dh
-    launch_k(bw_dh_kernel, dim3(grid_for(static_cast<int64_t>(R) * m)), dim3(kBwThreads), 0, s, dA, h, p0, n, R,
-             static_cast<int>(m), dh);
-    count_launch();
-    // second GEMM, wgrad: dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T  (contraction over R tokens, stored K256 wide)
-    launch_k(bw_dequant_kernel, dim3(grid_for(static_cast<int64_t>(R) * m / 2)), dim3(kBwThreads), 0, s,
-             static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqc)), static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqs)),
-             a_global, p0, n, R, static_cast<int>(m), deq);
-    count_launch();
-    if ((st = launch_nvfp4_quantize_ex(d_o, LMOE_F32, R, l, LMOE_QX_TRANSPOSE | LMOE_QX_RHT | LMOE_QX_SR, rht_signs,
-                                       seed, st_wg2, nullptr, t1c, t1s, t1g, LMOE_SF_MMA_TILED, part, s, K256)) !=
-        LMOE_OK)
-      break;
-    if ((st = launch_nvfp4_quantize_ex(deq, LMOE_F32, R, m, LMOE_QX_TRANSPOSE | LMOE_QX_RHT, rht_signs, seed, 0,
-                                       nullptr, t2c, t2s, t2g, LMOE_SF_MMA_TILED, part, s, K256)) != LMOE_OK)
-      break;
-    if ((st = gemm1(t1c, t1s, t1g, l, off_l, t2c, t2s, t2g, m, K256, static_cast<__nv_bfloat16*>(dw2) + e * l * m,
-                    m, 0)) != LMOE_OK)
-      break;
-    // first GEMM, dgrad: dz = SR(dh) W1q  (W1^T [l][m] with 16 x 16 blocks), into the expert's slot rows
-    if ((st = launch_nvfp4_quantize_ex(dh, LMOE_F32, R, m, LMOE_QX_SR, rht_signs, seed, st_dg1, nullptr, qac, qas,
-                                       qag, LMOE_SF_MMA_TILED, part, s)) != LMOE_OK)
-      break;
-    if ((st = gemm1(qac, qas, qag, R128, off_e, at<uint8_t>(ws, L.w1tc) + e * l * m / 2,
-                    at<uint8_t>(ws, L.w1ts) + e * l * m / 16, at<float>(ws, L.w1tg) + e, l, m,
-                    static_cast<__nv_bfloat16*>(dz) + p0 * l, l, 0)) != LMOE_OK)
-      break;
-    // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
-    launch_k(bw_dequant_kernel, dim3(grid_for(static_cast<int64_t>(R) * l / 2)), dim3(kBwThreads), 0, s, z_codes,
-             z_sf, z_global, p0, n, R, static_cast<int>(l), deq);
-    count_launch();
-    if ((st = launch_nvfp4_quantize_ex(dh, LMOE_F32, R, m, LMOE_QX_TRANSPOSE | LMOE_QX_RHT | LMOE_QX_SR, rht_signs,
-                                       seed, st_wg1, nullptr, t1c, t1s, t1g, LMOE_SF_MMA_TILED, part, s, K256)) !=
-        LMOE_OK)
-      break;
-    if ((st = launch_nvfp4_quantize_ex(deq, LMOE_F32, R, l, LMOE_QX_TRANSPOSE | LMOE_QX_RHT, rht_signs, seed, 0,
-                                       nullptr, t2c, t2s, t2g, LMOE_SF_MMA_TILED, part, s, K256)) != LMOE_OK)
-      break;
-    st = gemm1(t1c, t1s, t1g, m, off_m, t2c, t2s, t2g, l, K256, static_cast<__nv_bfloat16*>(dw1) + e * m * l, l, 0);
-  }
-  if (st != LMOE_OK) return st;
+  // do, dgate
+  launch_k(bw_prep_kernel, grid_per_expert(L.Rmax * kBwThreads, N), dim3(kBwThreads), 0, s,
+           static_cast<const float*>(dy), o, gate, static_cast<const int64_t*>(d_etab), static_cast<int>(l), d_o,
+           dgate);
+  count_launch();
+  // second GEMM, dgrad: dA = SR(do) W2q  (W2^T [m][l] with 16 x 16 blocks)
+  if ((st = quant(0, d_o, l, LMOE_QX_SR, 2, qac, qas, qag)) != LMOE_OK) return st;
+  if ((st = grouped(qac, qas, qag, 1, at<uint8_t>(ws, L.w2tc), at<uint8_t>(ws, L.w2ts), at<float>(ws, L.w2tg), m, l,
+                    dA, m, 1)) != LMOE_OK)
+    return st;
+  // dh
+  launch_k(bw_dh_kernel, grid_per_expert(L.Rmax * m, N), dim3(kBwThreads), 0, s, static_cast<const float*>(dA), h,
+           static_cast<const int64_t*>(d_etab), static_cast<int>(m), dh);
+  count_launch();
+  // second GEMM, wgrad: dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T  (contraction over the expert's K256 tokens)
+  launch_k(bw_dequant_kernel, grid_per_expert(L.Rmax * m / 2, N), dim3(kBwThreads), 0, s,
+           static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqc)), static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqs)),
+           a_global, static_cast<const int64_t*>(d_etab), static_cast<int>(m), deq);
+  count_launch();
+  if ((st = quant(1, d_o, l, T_RHT | LMOE_QX_SR, 3, t1c, t1s, t1g)) != LMOE_OK) return st;
+  if ((st = quant(2, deq, m, T_RHT, 0, t2c, t2s, t2g)) != LMOE_OK) return st;
+  if ((st = wgrads(l, m, dw2)) != LMOE_OK) return st;
+  // first GEMM, dgrad: dz = SR(dh) W1q  (W1^T [l][m] with 16 x 16 blocks), at the slot rows
+  if ((st = quant(3, dh, m, LMOE_QX_SR, 0, qac, qas, qag)) != LMOE_OK) return st;
+  if ((st = grouped(qac, qas, qag, 1, at<uint8_t>(ws, L.w1tc), at<uint8_t>(ws, L.w1ts), at<float>(ws, L.w1tg), l, m,
+                    dz, l, 0)) != LMOE_OK)
+    return st;
+  // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
+  launch_k(bw_dequant_kernel, grid_per_expert(L.Rmax * l / 2, N), dim3(kBwThreads), 0, s, z_codes, z_sf, z_global,
+           static_cast<const int64_t*>(d_etab), static_cast<int>(l), deq);
+  count_launch();
+  if ((st = quant(4, dh, m, T_RHT | LMOE_QX_SR, 1, t1c, t1s, t1g)) != LMOE_OK) return st;
+  if ((st = quant(5, deq, l, T_RHT, 0, t2c, t2s, t2g)) != LMOE_OK) return st;
+  if ((st = wgrads(m, l, dw1)) != LMOE_OK) return st;
   if (o_out && L.P > 0 &&
       cudaMemcpyAsync(o_out, o, static_cast<size_t>(L.P) * l * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return LMOE_ERR_CUDA;
