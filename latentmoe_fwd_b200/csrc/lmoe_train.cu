@@ -92,6 +92,7 @@ struct QxParams {
   // group g draws its SR uniforms on stream + g * stream_step
   const int64_t* gtab;
   uint32_t stream_step;
+  int vec;               // input 16-byte aligned: row segments read with 16-byte loads
 };
 
 // The parameters of group blockIdx.y: its input, outputs, global scale and
@@ -148,6 +149,48 @@ __device__ __forceinline__ void load_block(const QxParams& p, int64_t ro, int64_
   }
 }
 
+// Without the transform every value is an fp32 number, and so is each step
+// below (fp32 IEEE division gives the correctly rounded quotient, which the
+// fp64 quotient rounded to fp32 equals: 53 >= 2 * 24 + 2 bits), so this path
+// takes the same decisions in fp32.
+__device__ __forceinline__ void load_block_f32(const QxParams& p, int64_t ro, int64_t j, float (&v)[16]) {
+  if (!p.transpose && p.vec) {
+    if (p.bf16) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.in) + ro * p.cols + j * 16);
+      const uint4 a = __ldg(src), b = __ldg(src + 1);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.in) + ro * p.cols + j * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 f = __ldg(src + i);
+        v[4 * i] = f.x;
+        v[4 * i + 1] = f.y;
+        v[4 * i + 2] = f.z;
+        v[4 * i + 3] = f.w;
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int64_t r = p.transpose ? j * 16 + i : ro, c = p.transpose ? ro : j * 16 + i;
+    v[i] = p.bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.in)[r * p.cols + c])
+                  : static_cast<const float*>(p.in)[r * p.cols + c];
+  }
+}
+
+// E4M3 code -> value in fp32 (exact: at most 4 significant bits).
+__device__ __forceinline__ float e4m3_exact_f(uint32_t c) {
+  const int e = (c >> 3) & 15, f = c & 7;
+  return e == 0 ? ldexpf(static_cast<float>(f), -9) : ldexpf(static_cast<float>(8 + f), e - 10);
+}
+
 __device__ __forceinline__ int64_t out_rows(const QxParams& p) { return p.transpose ? p.cols : p.rows; }
 __device__ __forceinline__ int64_t out_cols(const QxParams& p) { return p.transpose ? p.rows : p.cols; }
 
@@ -165,10 +208,19 @@ __global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, d
     // (consecutive input columns) of one block column, so loads coalesce
     const int64_t ro = p.transpose ? b % out_rows(p) : b / nb;
     const int64_t j = p.transpose ? b / out_rows(p) : b % nb;
-    double v[16];
-    load_block(p, ro, j, v);
+    if (p.rht) {
+      double v[16];
+      load_block(p, ro, j, v);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmax(m, fabs(v[i]));
+      for (int i = 0; i < 16; ++i) m = fmax(m, fabs(v[i]));
+    } else {
+      float v[16];
+      load_block_f32(p, ro, j, v);
+      float mf = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mf = fmaxf(mf, fabsf(v[i]));
+      m = fmax(m, static_cast<double>(mf));
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -182,23 +234,24 @@ __global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, d
 }
 
 // Stochastic E2M1 code of v (fp32 value): |v| >= 6 -> 6; else, between grid
-// neighbours lo <= |v| < hi, hi when u * (hi - lo) < |v| - lo (exact
-// comparison), else lo; the sign bit is the sign of v. The grid (0, 0.5, 1,
-// 1.5, 2, 3, 4, 6) is walked with compares and selects, so nothing is indexed
-// at run time.
+// neighbours lo <= |v| < hi, hi when u * (hi - lo) < |v| - lo, else lo; the
+// sign bit is the sign of v. Both sides are exact in fp32: hi - lo is a power
+// of two, u has 24 bits, and lo <= |v| < hi <= 2 lo (or lo = 0) makes the
+// difference exact. The grid (0, 0.5, 1, 1.5, 2, 3, 4, 6) is walked with
+// compares and selects, so nothing is indexed at run time.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, float u) {
-  const double a = fabs(static_cast<double>(v));
+  const float a = fabsf(v);
   uint32_t lo = 0;
-  double l = 0.0, h = 0.5;
-  if (a >= 0.5) { lo = 1; l = 0.5; h = 1.0; }
-  if (a >= 1.0) { lo = 2; l = 1.0; h = 1.5; }
-  if (a >= 1.5) { lo = 3; l = 1.5; h = 2.0; }
-  if (a >= 2.0) { lo = 4; l = 2.0; h = 3.0; }
-  if (a >= 3.0) { lo = 5; l = 3.0; h = 4.0; }
-  if (a >= 4.0) { lo = 6; l = 4.0; h = 6.0; }
+  float l = 0.0f, h = 0.5f;
+  if (a >= 0.5f) { lo = 1; l = 0.5f; h = 1.0f; }
+  if (a >= 1.0f) { lo = 2; l = 1.0f; h = 1.5f; }
+  if (a >= 1.5f) { lo = 3; l = 1.5f; h = 2.0f; }
+  if (a >= 2.0f) { lo = 4; l = 2.0f; h = 3.0f; }
+  if (a >= 3.0f) { lo = 5; l = 3.0f; h = 4.0f; }
+  if (a >= 4.0f) { lo = 6; l = 4.0f; h = 6.0f; }
   uint32_t code = lo;
-  if (a >= 6.0) code = 7;
-  else if (static_cast<double>(u) * (h - l) < a - l) code = lo + 1;
+  if (a >= 6.0f) code = 7;
+  else if (__fmul_rn(u, h - l) < __fsub_rn(a, l)) code = lo + 1;
   return code | (signbit(v) ? 8u : 0u);
 }
 
@@ -210,6 +263,7 @@ __device__ __forceinline__ int64_t tiled_off(int64_t row, int64_t j, int64_t gro
 // 16-row group sit in one half-warp (lane & 15 = row in the group), so a
 // 16 x 16 block's amax is a half-warp reduction. The item count is rounded up
 // to whole warps; items past the end take part in the reductions only.
+template <bool RHT>
 __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0) {
   pdl_begin();
   const QxParams p = qx_group(p0);
@@ -253,11 +307,20 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
     const int64_t ro = g * 16 + i16;
     const bool has = live && ro < R && j < nb;
     double v[16];
+    float vf[16];
     double m = 0.0;
     if (has) {
-      load_block(p, ro, j, v);
+      if (RHT) {
+        load_block(p, ro, j, v);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
+        for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
+      } else {
+        load_block_f32(p, ro, j, vf);
+        float mf = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) mf = fmaxf(mf, fabsf(vf[e]));
+        m = static_cast<double>(mf);
+      }
     }
     if (p.block2d) {   // one scale from the amax of the 16 x 16 block
 #pragma unroll
@@ -266,14 +329,29 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
     if (!live) continue;
     uint32_t scode = 0;
     if (has) {
-      scode = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
-      const double dec = e4m3_exact(scode);
       uint32_t lo = 0, hi = 0;
-      if (dec != 0.0) {
-        const float sc = __fmul_rn(static_cast<float>(dec), s_g);
-        float q[16];
+      float q[16];
+      bool nz;
+      if (RHT) {
+        scode = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
+        const double dec = e4m3_exact(scode);
+        nz = dec != 0.0;
+        if (nz) {
+          const float sc = __fmul_rn(static_cast<float>(dec), s_g);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(v[e] / static_cast<double>(sc));
+          for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(v[e] / static_cast<double>(sc));
+        }
+      } else {
+        scode = cvt_to_e4m3(__fdiv_rn(static_cast<float>(m), t));
+        const float dec = e4m3_exact_f(scode);
+        nz = dec != 0.0f;
+        if (nz) {
+          const float sc = __fmul_rn(dec, s_g);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(vf[e], sc);
+        }
+      }
+      if (nz) {
         if (p.sr) {
           float u[16];
           sr_uniforms16(static_cast<uint64_t>(ro) * C + j * 16, p.seed, p.stream, u);
@@ -328,6 +406,7 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   p.codes = codes;
   p.sf = sf;
   p.global_out = global_out;
+  p.vec = (reinterpret_cast<uintptr_t>(in) & 15) == 0;
   const int64_t R = p.transpose ? cols : rows, C = p.transpose ? rows : cols;
   p.pitch = out_pitch > 0 ? out_pitch : C;
   if (p.pitch < C || p.pitch % 16) return LMOE_ERR_INVALID_ARG;
@@ -352,7 +431,8 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   const int64_t cap = (static_cast<int64_t>(sms) * 8 + groups - 1) / groups;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  launch_k(qx_encode_kernel, dim3(static_cast<unsigned>(blocks), groups), dim3(kXThreads), 0, s, p);
+  launch_k(p.rht ? qx_encode_kernel<true> : qx_encode_kernel<false>, dim3(static_cast<unsigned>(blocks), groups),
+           dim3(kXThreads), 0, s, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -381,6 +461,7 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
   p.codes = codes;
   p.sf = sf;
   p.global_out = global_out;
+  p.vec = (reinterpret_cast<uintptr_t>(in) & 15) == 0;
   p.gtab = gtab;
   const int64_t R = p.transpose ? cols : rows_max, C = p.transpose ? rows_max : cols;
   const int64_t pitch = pitch_max > C ? pitch_max : C;
@@ -397,7 +478,8 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
   const int64_t cap = (static_cast<int64_t>(sms) * 8 + groups - 1) / groups;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  launch_k(qx_encode_kernel, dim3(static_cast<unsigned>(blocks), groups), dim3(kXThreads), 0, s, p);
+  launch_k(p.rht ? qx_encode_kernel<true> : qx_encode_kernel<false>, dim3(static_cast<unsigned>(blocks), groups),
+           dim3(kXThreads), 0, s, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
