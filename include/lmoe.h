@@ -393,6 +393,22 @@ lmoe_status lmoe_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, i
                                    const float* global_in, uint8_t* codes, uint8_t* sf, float* global_out,
                                    int sf_layout, void* ws, size_t ws_bytes, void* stream);
 
+/* Transpose of NVFP4 weights quantised with 16 x 16 scale blocks (the
+ * training recipe's 2-D weight blocks: greeksharifa page, section 2.4 "NVFP4
+ * Training"; the dgrads read W^T). With square blocks W^T quantises to W's
+ * codes and scales transposed: every element keeps its block's scale and the
+ * global scale is W's, so this replaces quantising the transpose.
+ *  codes: `groups` matrices [rows][cols/2] back to back (element 2k in the
+ *  low nibble), sf: their MMA-tiled scales (rows * cols / 16 bytes each), as
+ *  lmoe_nvfp4_quantize_ex writes with LMOE_SF_MMA_TILED | LMOE_SF_BLOCK_16X16;
+ *  codes_t [groups][cols][rows/2] and sf_t (same sizes) receive W^T's; the
+ *  global scales are unchanged. Device pointers, 16-byte aligned, no overlap.
+ *  Errors: LMOE_ERR_INVALID_ARG for null or unaligned pointers or negative
+ *  sizes; LMOE_ERR_UNSUPPORTED unless rows and cols are multiples of 128
+ *  (whole scale atoms) and groups <= 65535. Nothing to do for zero sizes. */
+lmoe_status lmoe_nvfp4_transpose_2d(const uint8_t* codes, const uint8_t* sf, int64_t groups, int64_t rows,
+                                    int64_t cols, uint8_t* codes_t, uint8_t* sf_t, void* stream);
+
 /* Grouped block-scaled NVFP4 GEMM (the kernel of the routed experts, exposed
  * for the training recipe's dgrad and wgrad; greeksharifa page, section 2.4
  * "NVFP4 Training": fprop, dgrad and wgrad run as NVFP4 GEMMs):

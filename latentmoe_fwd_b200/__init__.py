@@ -7,7 +7,8 @@ loads the shared library and fails loudly if it has not been built
 
 Entry points mirror include/lmoe.h: ``route``, ``permute`` (and
 ``permute_noalloc``), ``expert_ffn``, ``combine``, ``forward`` (and
-``forward_traced``), ``nvfp4_quantize``, ``nvfp4_quantize_ex``, ``fp8_quantize``, plus ``workspace_size``,
+``forward_traced``), ``nvfp4_quantize``, ``nvfp4_quantize_ex``, ``nvfp4_transpose_2d``, ``fp8_quantize``,
+plus ``workspace_size``,
 ``padded_rows``, ``workspace``, ``read_device_error``,
 ``selftest_wait_timeout`` and ``kernel_launch_count``.
 Tensor arguments are torch tensors (or None); their ``data_ptr()`` is passed.
@@ -36,7 +37,8 @@ EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permut
            "lmoe_expert_ffn", "lmoe_combine", "lmoe_forward", "lmoe_nvfp4_quantize",
            "lmoe_read_device_error", "lmoe_status_string", "lmoe_kernel_launch_count",
            "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize",
-           "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_gemm",
+           "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_transpose_2d",
+           "lmoe_nvfp4_gemm",
            "lmoe_ep_plan", "lmoe_ep_reorder", "lmoe_expert_backward_nvfp4",
            "lmoe_expert_backward_nvfp4_workspace", "lmoe_backward_nvfp4", "lmoe_backward_nvfp4_workspace")
 TRACE_EVENTS = 8
@@ -94,6 +96,7 @@ def _load():
         "lmoe_selftest_wait_timeout": (ctypes.c_int, [P, ctypes.c_size_t, ctypes.c_uint64, P]),
         "lmoe_fp8_quantize": (ctypes.c_int, [P, ctypes.c_int, I64, I64, P, P, P, P, ctypes.c_size_t, P]),
         "lmoe_nvfp4_quantize_ex_workspace": (ctypes.c_size_t, [I64, I64]),
+        "lmoe_nvfp4_transpose_2d": (ctypes.c_int, [P, P, I64, I64, I64, P, P, P]),
         "lmoe_ep_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int] + [P] * 12),
         "lmoe_ep_reorder": (ctypes.c_int, [P, P, I64, ctypes.c_int, P, P, P, I64, P]),
         "lmoe_nvfp4_gemm": (ctypes.c_int, [ctypes.c_int, P, P, I64, P, P, P, ctypes.c_int, P, P, P, ctypes.c_int,
@@ -261,6 +264,13 @@ def nvfp4_quantize_ex(x, in_dtype, rows, cols, flags, rht_signs, seed, sr_stream
                                       int(seed), int(sr_stream), _p(global_in), _p(codes), _p(sf), _p(global_out),
                                       int(sf_layout), _p(ws), 0 if ws is None else ws.numel(), _stream(stream)),
            "lmoe_nvfp4_quantize_ex")
+
+
+def nvfp4_transpose_2d(codes, sf, groups, rows, cols, codes_t, sf_t, stream=None):
+    """lmoe_nvfp4_transpose_2d: codes and MMA-tiled scales of NVFP4 matrices
+    with 16 x 16 blocks -> those of their transposes."""
+    _check(lib.lmoe_nvfp4_transpose_2d(_p(codes), _p(sf), int(groups), int(rows), int(cols), _p(codes_t), _p(sf_t),
+                                       _stream(stream)), "lmoe_nvfp4_transpose_2d")
 
 
 def nvfp4_gemm(groups, offsets, padded_offsets, a_rows, a_codes, a_sf, a_global, a_global_per_group, b_codes, b_sf,

@@ -717,6 +717,11 @@ lmoe_status lmoe_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows, i
                                   global_out, sf_layout, partials, static_cast<cudaStream_t>(stream));
 }
 
+lmoe_status lmoe_nvfp4_transpose_2d(const uint8_t* codes, const uint8_t* sf, int64_t groups, int64_t rows,
+                                    int64_t cols, uint8_t* codes_t, uint8_t* sf_t, void* stream) {
+  return launch_nvfp4_transpose2d(codes, sf, groups, rows, cols, codes_t, sf_t, static_cast<cudaStream_t>(stream));
+}
+
 lmoe_status lmoe_nvfp4_gemm(int groups, const int32_t* offsets, const int32_t* padded_offsets, int64_t a_rows,
                             const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
                             int a_global_per_group, const uint8_t* b_codes, const uint8_t* b_sf,

@@ -197,6 +197,10 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
                                      uint32_t rht_signs, uint64_t seed, uint32_t sr_stream, const float* global_in,
                                      uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout, double* partials,
                                      cudaStream_t s, int64_t out_pitch = 0, int groups = 1);
+// Codes and MMA-tiled scales of `groups` [rows][cols] matrices quantised with
+// 16 x 16 blocks -> those of their transposes (rows, cols multiples of 128).
+lmoe_status launch_nvfp4_transpose2d(const uint8_t* codes, const uint8_t* sf, int64_t groups, int64_t rows,
+                                     int64_t cols, uint8_t* codes_t, uint8_t* sf_t, cudaStream_t s);
 // Ragged groups: group g quantises input rows [gtab[5g], gtab[5g] + gtab[5g+1])
 // of a [*][cols] input as one matrix (own global scale global_out[g], SR
 // stream stream0 + g * stream_step), codes at codes + gtab[5g+2], scales at

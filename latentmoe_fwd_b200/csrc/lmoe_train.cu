@@ -378,7 +378,77 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
   }
 }
 
+// Transpose of NVFP4 data with 16 x 16 scale blocks: a CTA per 128 x 128
+// tile of one group. The tile's codes (128 rows x 64 bytes) are staged in
+// shared memory; thread (c = tid % 128, half = tid / 128) then gathers input
+// rows half * 64 .. half * 64 + 63 of column c (64 nibbles, element 2k in the
+// low nibble) into 32 bytes of output row c, and writes the four scales of
+// those rows' 16-row groups as one word of the output's MMA-tiled layout.
+__global__ void __launch_bounds__(256) nvfp4_transpose2d_kernel(const uint8_t* __restrict__ codes,
+                                                                 const uint8_t* __restrict__ sf, int64_t rows,
+                                                                 int64_t cols, uint8_t* __restrict__ codes_t,
+                                                                 uint8_t* __restrict__ sf_t) {
+  pdl_begin();
+  __shared__ __align__(16) uint8_t tile[128 * 64];
+  const int64_t g = blockIdx.z;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 128, c0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const uint8_t* in = codes + g * rows * cols / 2;
+  const uint8_t* in_sf = sf + g * rows * cols / 16;
+  uint8_t* out = codes_t + g * rows * cols / 2;
+  uint8_t* out_sf = sf_t + g * rows * cols / 16;
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int idx = tid + k * 256;
+    const int row = idx >> 2, part = idx & 3;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(in + (r0 + row) * (cols / 2) + c0 / 2) + part);
+    *reinterpret_cast<uint4*>(tile + row * 64 + part * 16) = v;
+  }
+  __syncthreads();
+  const int c = tid & 127, half = tid >> 7;
+  const int shift = (c & 1) * 4;
+  uint32_t w[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {   // nibble b of the word: input row half * 64 + q * 8 + b
+      const int r = half * 64 + q * 8 + b;
+      word |= static_cast<uint32_t>((tile[r * 64 + (c >> 1)] >> shift) & 15u) << (4 * b);
+    }
+    w[q] = word;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out + (c0 + c) * (rows / 2) + r0 / 2 + half * 32);
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  // scales: output row c0 + c, blocks j = (r0 + half * 64) / 16 + 0..3
+  const int64_t g64_in = cols / 64, g64_out = rows / 64;
+  const int64_t jc = (c0 + c) / 16;   // the input's scale column of this output row
+  uint32_t sw = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+    sw |= static_cast<uint32_t>(__ldg(in_sf + tiled_off(r0 + half * 64 + b * 16, jc, g64_in))) << (8 * b);
+  *reinterpret_cast<uint32_t*>(out_sf + tiled_off(c0 + c, (r0 + half * 64) / 16, g64_out)) = sw;
+}
+
 }  // namespace
+
+lmoe_status launch_nvfp4_transpose2d(const uint8_t* codes, const uint8_t* sf, int64_t groups, int64_t rows,
+                                     int64_t cols, uint8_t* codes_t, uint8_t* sf_t, cudaStream_t s) {
+  if (groups < 0 || rows < 0 || cols < 0) return LMOE_ERR_INVALID_ARG;
+  if (groups == 0 || rows == 0 || cols == 0) return LMOE_OK;
+  if (!codes || !sf || !codes_t || !sf_t) return LMOE_ERR_INVALID_ARG;
+  if (rows % 128 || cols % 128 || groups > 65535 || rows / 128 > 65535 || cols / 128 > 0x7fffffff)
+    return LMOE_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(codes) | reinterpret_cast<uintptr_t>(codes_t) | reinterpret_cast<uintptr_t>(sf) |
+       reinterpret_cast<uintptr_t>(sf_t)) & 15)
+    return LMOE_ERR_INVALID_ARG;
+  launch_k(nvfp4_transpose2d_kernel, dim3(static_cast<unsigned>(cols / 128), static_cast<unsigned>(rows / 128),
+                                          static_cast<unsigned>(groups)),
+           dim3(256), 0, s, codes, sf, rows, cols, codes_t, sf_t);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
 
 int nvfp4x_partials(int64_t blocks) {
   const int64_t want = (blocks + 4 * kXThreads - 1) / (4 * kXThreads);

@@ -153,7 +153,7 @@ dim3 grid_per_expert(int64_t items, int N) {
 
 // Workspace carve-up (all offsets 256-byte aligned).
 struct BwLayout {
-  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w1tg, w2tc, w2ts, w2tg, h, aqc, aqs, o, d_o, dh, deq, qac,
+  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w2tc, w2ts, h, aqc, aqs, o, d_o, dh, deq, qac,
       qas, qag, dA, t1c, t1s, t1g, t2c, t2s, t2g, part, etab, gtab, itab, total;
   int64_t P, Rmax, Ksum;
 };
@@ -182,10 +182,8 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ks
   L.w2g = take(N * 4);
   L.w1tc = take(N * l * m / 2);   // transposed weights (dgrad operands), every expert
   L.w1ts = take(N * l * m / 16);
-  L.w1tg = take(N * 4);
   L.w2tc = take(N * l * m / 2);
   L.w2ts = take(N * l * m / 16);
-  L.w2tg = take(N * 4);
   // every expert's rows at its padded offset
   L.h = take(P * m * 4);
   L.aqc = take(P * m / 2);
@@ -357,7 +355,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
 
   // every expert's weights with 16 x 16 blocks (current amax per expert and
   // matrix), one grouped launch each: W1 [m][l] and W2 [l][m] for the forward,
-  // W2^T [m][l] and W1^T [l][m] for the dgrads
+  // then W2^T [m][l] and W1^T [l][m] for the dgrads
   if ((st = launch_nvfp4_quantize_ex(W1, LMOE_BF16, m, l, 0, 0, 0, 0, nullptr, at<uint8_t>(ws, L.w1c),
                                      at<uint8_t>(ws, L.w1s), at<float>(ws, L.w1g), tiled2d, part, s, 0, N)) !=
       LMOE_OK)
@@ -366,13 +364,13 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                                      at<uint8_t>(ws, L.w2s), at<float>(ws, L.w2g), tiled2d, part, s, 0, N)) !=
       LMOE_OK)
     return st;
-  if ((st = launch_nvfp4_quantize_ex(W2, LMOE_BF16, l, m, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr,
-                                     at<uint8_t>(ws, L.w2tc), at<uint8_t>(ws, L.w2ts), at<float>(ws, L.w2tg), tiled2d,
-                                     part, s, 0, N)) != LMOE_OK)
+  // with 16 x 16 blocks the transposes quantise to the transposed codes and
+  // scales, under the same global scales
+  if ((st = launch_nvfp4_transpose2d(at<uint8_t>(ws, L.w2c), at<uint8_t>(ws, L.w2s), N, l, m,
+                                     at<uint8_t>(ws, L.w2tc), at<uint8_t>(ws, L.w2ts), s)) != LMOE_OK)
     return st;
-  if ((st = launch_nvfp4_quantize_ex(W1, LMOE_BF16, m, l, LMOE_QX_TRANSPOSE, 0, 0, 0, nullptr,
-                                     at<uint8_t>(ws, L.w1tc), at<uint8_t>(ws, L.w1ts), at<float>(ws, L.w1tg), tiled2d,
-                                     part, s, 0, N)) != LMOE_OK)
+  if ((st = launch_nvfp4_transpose2d(at<uint8_t>(ws, L.w1c), at<uint8_t>(ws, L.w1s), N, m, l,
+                                     at<uint8_t>(ws, L.w1tc), at<uint8_t>(ws, L.w1ts), s)) != LMOE_OK)
     return st;
 
   // the expert-grouped NVFP4 GEMM over every expert's padded rows
@@ -483,7 +481,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   count_launch();
   // second GEMM, dgrad: dA = SR(do) W2q  (W2^T [m][l] with 16 x 16 blocks)
   if ((st = quant(0, d_o, l, LMOE_QX_SR, 2, qac, qas, qag)) != LMOE_OK) return st;
-  if ((st = grouped(qac, qas, qag, 1, at<uint8_t>(ws, L.w2tc), at<uint8_t>(ws, L.w2ts), at<float>(ws, L.w2tg), m, l,
+  if ((st = grouped(qac, qas, qag, 1, at<uint8_t>(ws, L.w2tc), at<uint8_t>(ws, L.w2ts), at<float>(ws, L.w2g), m, l,
                     dA, m, 1)) != LMOE_OK)
     return st;
   // dh
@@ -500,7 +498,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   if ((st = wgrads(l, m, dw2)) != LMOE_OK) return st;
   // first GEMM, dgrad: dz = SR(dh) W1q  (W1^T [l][m] with 16 x 16 blocks), at the slot rows
   if ((st = quant(3, dh, m, LMOE_QX_SR, 0, qac, qas, qag)) != LMOE_OK) return st;
-  if ((st = grouped(qac, qas, qag, 1, at<uint8_t>(ws, L.w1tc), at<uint8_t>(ws, L.w1ts), at<float>(ws, L.w1tg), l, m,
+  if ((st = grouped(qac, qas, qag, 1, at<uint8_t>(ws, L.w1tc), at<uint8_t>(ws, L.w1ts), at<float>(ws, L.w1g), l, m,
                     dz, l, 0)) != LMOE_OK)
     return st;
   // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T

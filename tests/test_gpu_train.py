@@ -113,6 +113,30 @@ def test_ragged_2d_blocks_bit_exact(layout):
     assert g == np.float32(rg) and np.array_equal(sf, rsf) and np.array_equal(codes, rc)
 
 
+@pytest.mark.parametrize("groups,rows,cols", [(1, 128, 128), (3, 256, 384)])
+def test_transpose_2d_equals_quantising_the_transpose(groups, rows, cols):
+    # W^T with 16 x 16 blocks quantises to W's codes and scales transposed
+    lay = L.SF_MMA_TILED | L.SF_BLOCK_16X16
+    Ws = [_data(rows, cols, 40 + g) for g in range(groups)]
+    codes = torch.empty((groups, rows, cols // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.zeros((groups, rows * cols // 16), dtype=torch.uint8, device="cuda")
+    ref_c = torch.empty((groups, cols, rows // 2), dtype=torch.uint8, device="cuda")
+    ref_s = torch.zeros((groups, rows * cols // 16), dtype=torch.uint8, device="cuda")
+    gl = torch.empty(2 * groups, dtype=torch.float32, device="cuda")
+    for g, W in enumerate(Ws):
+        x = to_dev(W, "bf16")
+        L.nvfp4_quantize_ex(x, L.BF16, rows, cols, 0, 0, 0, 0, None, codes[g], sf[g], gl[2 * g:], lay)
+        L.nvfp4_quantize_ex(x, L.BF16, rows, cols, L.QX_TRANSPOSE, 0, 0, 0, None, ref_c[g], ref_s[g],
+                            gl[2 * g + 1:], lay)
+    ct = torch.full_like(ref_c, 0xAA)
+    st = torch.full_like(ref_s, 0xAA)
+    L.nvfp4_transpose_2d(codes, sf, groups, rows, cols, ct, st)
+    torch.cuda.synchronize()
+    g = gl.cpu().numpy()
+    assert np.array_equal(g[0::2], g[1::2])
+    assert torch.equal(ct, ref_c) and torch.equal(st, ref_s)
+
+
 def test_plain_mode_equals_nvfp4_quantize():
     bits = _data(130, 64, 2)
     codes, sf, g = _quantize_ex(bits, 130, 64, 0)
