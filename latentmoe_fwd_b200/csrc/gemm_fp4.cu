@@ -41,10 +41,10 @@ static bool make_map_fp4(CUtensorMap* map, const void* ptr, int64_t k, int64_t r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool BATCH = false>
 static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const Fp4Params& p, int grid,
                               cudaStream_t s) {
-  auto kern = fp4_gemm_kernel<EPI>;
+  auto kern = fp4_gemm_kernel<EPI, BATCH>;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -60,9 +60,11 @@ static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const 
 
 lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream) {
   if (L.k % 256 || L.cols % 256 || L.groups > Fp4Smem::kMaxGroups) return LMOE_ERR_UNSUPPORTED;
+  const bool batch = L.kgroups != nullptr;
+  if (batch && (L.quant_out || L.f32_out || L.row_scale || L.a_rows % 128 || L.groups < 1)) return LMOE_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
   if (!make_map_fp4(&ma, L.a_codes, L.k, L.a_rows, 1, 128)) return LMOE_ERR_INVALID_ARG;
-  if (!make_map_fp4(&mb, L.b_codes, L.k, L.cols, L.groups, 256)) return LMOE_ERR_INVALID_ARG;
+  if (!make_map_fp4(&mb, L.b_codes, L.k, L.cols, batch ? 1 : L.groups, 256)) return LMOE_ERR_INVALID_ARG;
   Fp4Params p;
   p.rows = static_cast<int>(L.a_rows);
   p.cols = L.cols;
@@ -71,7 +73,9 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   p.sf_groups_b = static_cast<int>(L.k / 64);
   p.sfa = L.a_sf;
   p.sfb = L.b_sf;
-  p.sfb_expert_bytes = static_cast<long long>(L.cols) * (L.k / 16);
+  p.sfb_expert_bytes = batch ? 0 : static_cast<long long>(L.cols) * (L.k / 16);
+  p.kgroup_tab = L.kgroups;
+  p.out_group_stride = L.out_group_stride;
   p.offsets = L.offsets;
   p.padded_offsets = L.padded_offsets;
   p.groups = L.groups;
@@ -87,9 +91,11 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   if (L.f32_out && ((reinterpret_cast<uintptr_t>(L.out) & 15) || L.ld_out % 4)) return LMOE_ERR_INVALID_ARG;
   p.err = DevErr{err_word};
   const int sms = device_sm_count();
-  const int64_t tiles = (L.a_rows / 128) * (L.cols / 256);
+  const int64_t tiles = (L.a_rows / 128) * (L.cols / 256) * (batch ? L.groups : 1);
+  if (tiles > 0x7fffffff) return LMOE_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   if (grid <= 0) return LMOE_OK;
+  if (batch) return launch_fp4<FP4_EPI_GATE_BF16, true>(ma, mb, p, grid, stream);
   if (L.quant_out) return launch_fp4<FP4_EPI_SQRELU_QUANT>(ma, mb, p, grid, stream);
   if (L.f32_out) return launch_fp4<FP4_EPI_F32>(ma, mb, p, grid, stream);
   return launch_fp4<FP4_EPI_GATE_BF16>(ma, mb, p, grid, stream);

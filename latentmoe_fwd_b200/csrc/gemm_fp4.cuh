@@ -50,6 +50,12 @@ struct Fp4Params {
   uint8_t* out_sf;            // GEMM1: MMA-tiled scales of a
   long long ld_out;           // GEMM2: elements per row
   int out_vec32;              // GEMM2: rows start on 32-byte boundaries (32-byte stores)
+  // K-batched problems (the kernel's BATCH form): group g multiplies K
+  // columns [kgroup_tab[2g], + 256 * kgroup_tab[2g+1]) of A [rows][K] and of
+  // B [cols][K] (shared matrices, K the sum over groups) into its own output
+  // at out + g * out_group_stride
+  const int* kgroup_tab;
+  long long out_group_stride;
   DevErr err;
 };
 
@@ -147,7 +153,7 @@ __device__ __forceinline__ long long fp4_sf_offset(long long row, int j, int gro
   return ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
 }
 
-template <int EPI>
+template <int EPI, bool BATCH = false>
 __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Fp4Params p) {
@@ -181,7 +187,18 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
   }
   int* s_pstart = reinterpret_cast<int*>(smem + S::kRowsOffset);   // [groups + 1] padded starts
   int* s_rend = s_pstart + S::kMaxGroups + 1;                          // [groups] real ends
-  for (int g = threadIdx.x; g <= p.groups; g += blockDim.x) {
+  // BATCH: s_pstart[g] = first K column of group g, s_rend[g] = its K blocks
+  for (int g = threadIdx.x; BATCH && g < p.groups; g += blockDim.x) {
+    int k0 = __ldg(p.kgroup_tab + 2 * g), nk = __ldg(p.kgroup_tab + 2 * g + 1);
+    if (kChecks && (k0 < 0 || (k0 & 255) || nk < 0 || k0 / 256 + nk > p.kblocks)) {   // within K
+      dev_report(p.err, kErrBounds, 0x5302);
+      k0 = 0;
+      nk = 0;
+    }
+    s_pstart[g] = k0;
+    s_rend[g] = nk;
+  }
+  for (int g = threadIdx.x; !BATCH && g <= p.groups; g += blockDim.x) {
     int ps = __ldg(p.padded_offsets + g);
     if (kChecks && (ps < 0 || ps > p.rows || (ps & 127))) {
       dev_report(p.err, kErrBounds, 0x5300);
@@ -207,17 +224,31 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
   const uint32_t tmem_base = *tmem_ptr;
 
   const int ntw = (p.cols + 255) / 256;
-  const int ntiles = (s_pstart[p.groups] >> 7) * ntw;
+  const int tpg = (p.rows >> 7) * ntw;   // BATCH: tiles per group
+  const int ntiles = BATCH ? p.groups * tpg : (s_pstart[p.groups] >> 7) * ntw;
 
   // a CTA visits its tiles in increasing order, so the owning expert (the
-  // largest e with padded start <= act0) only moves forward
+  // largest e with padded start <= act0) only moves forward. nkb: the tile's
+  // 256-element K blocks from K column koff.
   int cur_e = 0;
-  auto tile_of = [&](int t, int& e, int& act0, int& act_n, int& w0) {
-    w0 = (t % ntw) * 256;
-    act0 = (t / ntw) * 128;
-    while (cur_e + 1 < p.groups && s_pstart[cur_e + 1] <= act0) ++cur_e;
-    e = cur_e;
-    act_n = min(128, s_rend[e] - act0);
+  auto tile_of = [&](int t, int& e, int& act0, int& act_n, int& w0, int& nkb, int& koff) {
+    if (BATCH) {
+      e = t / tpg;
+      const int rem = t - e * tpg;
+      w0 = (rem % ntw) * 256;
+      act0 = (rem / ntw) * 128;
+      koff = s_pstart[e];
+      nkb = s_rend[e];
+      act_n = nkb > 0 ? 128 : 0;
+    } else {
+      w0 = (t % ntw) * 256;
+      act0 = (t / ntw) * 128;
+      while (cur_e + 1 < p.groups && s_pstart[cur_e + 1] <= act0) ++cur_e;
+      e = cur_e;
+      act_n = min(128, s_rend[e] - act0);
+      nkb = p.kblocks;
+      koff = 0;
+    }
   };
 
   if (warp == 0) {
@@ -229,20 +260,20 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
       uint32_t issued_mask = 0, last_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        int e, act0, act_n, w0;
-        tile_of(t, e, act0, act_n, w0);
+        int e, act0, act_n, w0, nkb, koff;
+        tile_of(t, e, act0, act_n, w0, nkb, koff);
         if (act_n <= 0) continue;
-        const uint8_t* sfa_blk = p.sfa + static_cast<long long>(act0 >> 7) * p.sf_groups_a * 512;
-        const uint8_t* sfb_e = p.sfb + static_cast<long long>(e) * p.sfb_expert_bytes;
-        for (int kb = 0; kb < p.kblocks; ++kb) {
+        const uint8_t* sfa_blk = p.sfa + (static_cast<long long>(act0 >> 7) * p.sf_groups_a + koff / 64) * 512;
+        const uint8_t* sfb_e = p.sfb + static_cast<long long>(e) * p.sfb_expert_bytes + (koff / 64) * 512;
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, 0x1100 + stage)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::kStage;
           uint8_t* sb = sa + S::kA;
           uint8_t* ssfa = sb + S::kB;
           uint8_t* ssfb = ssfa + S::kSFA;
           mbar_arrive_expect_tx(&full[stage], S::kStage);
-          tma_load_3d(sa, &tmA, &full[stage], kb * 128, act0, 0, pol_a);
-          tma_load_3d(sb, &tmB, &full[stage], kb * 128, w0, e, pol_w);
+          tma_load_3d(sa, &tmA, &full[stage], koff / 2 + kb * 128, act0, 0, pol_a);
+          tma_load_3d(sb, &tmB, &full[stage], koff / 2 + kb * 128, w0, BATCH ? 0 : e, pol_w);
           bulk_load(ssfa, sfa_blk + kb * 4 * 512, S::kSFA, &full[stage]);
 #pragma unroll
           for (int nb = 0; nb < 2; ++nb)
@@ -272,15 +303,15 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
       int local = 0;
       bool ok = true, any = false;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        int e, act0, act_n, w0;
-        tile_of(t, e, act0, act_n, w0);
+        int e, act0, act_n, w0, nkb, koff;
+        tile_of(t, e, act0, act_n, w0, nkb, koff);
         if (act_n <= 0) continue;
         if (local > 0) {
           if (!mbar_wait(overlap_free, (local - 1) & 1, abort_flag, p.err, 0x1200)) { ok = false; break; }
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ((local & 1) ? S::kAcc1 : 0);
-        for (int kb = 0; kb < p.kblocks; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, 0x1300 + stage)) { ok = false; break; }
           tc_fence_after();
           uint8_t* sa = smem + stage * S::kStage;
@@ -323,9 +354,10 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     const int groups64_out = (p.cols + 63) / 64;
     const uint64_t pol_out = policy_evict_first();
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      int e, act0, act_n, w0;
-      tile_of(t, e, act0, act_n, w0);
+      int e, act0, act_n, w0, nkb, koff;
+      tile_of(t, e, act0, act_n, w0, nkb, koff);
       if (act_n <= 0) continue;
+      const long long obase = BATCH ? e * p.out_group_stride : 0;
       const int buf = local & 1;
       const long long row = act0 + r;
       const bool row_ok = r < act_n;
@@ -360,7 +392,7 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
           p.out_sf[fp4_sf_offset(row, j0, groups64_out)] = static_cast<uint8_t>(s0);
           p.out_sf[fp4_sf_offset(row, j0 + 1, groups64_out)] = static_cast<uint8_t>(s1);
         } else if (EPI == FP4_EPI_F32) {
-          float* o = reinterpret_cast<float*>(p.out) + row * p.ld_out + col0;
+          float* o = reinterpret_cast<float*>(p.out) + obase + row * p.ld_out + col0;
           const float sg = scale * gate;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
@@ -368,7 +400,7 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
                 make_float4(__uint_as_float(v[j]) * sg, __uint_as_float(v[j + 1]) * sg,
                             __uint_as_float(v[j + 2]) * sg, __uint_as_float(v[j + 3]) * sg);
         } else {
-          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.ld_out + col0;
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + obase + row * p.ld_out + col0;
           const float sg = scale * gate;
           if (p.out_vec32) {   // whole 32-byte sectors per store
 #pragma unroll

@@ -117,6 +117,12 @@ struct Fp4Launch {
   const float* row_scale = nullptr;  // gates (GEMM 2)
   int quant_out = 0;                 // 1: relu^2 + NVFP4 codes/scales out; 0: BF16 out * gate
   int f32_out = 0;                   // with quant_out 0: fp32 out * gate instead of BF16
+  // K-batched problems (BF16 out only): kgroups[2g], kgroups[2g+1] = first K
+  // column (a multiple of 256) and 256-element K blocks of group g; A [a_rows][k]
+  // and B [cols][k] are single matrices (k the total), group g's output
+  // [a_rows][cols] at out + g * out_group_stride elements
+  const int* kgroups = nullptr;
+  int64_t out_group_stride = 0;
   void* out = nullptr;
   uint8_t* out_sf = nullptr;
   int64_t ld_out = 0;
@@ -205,12 +211,15 @@ lmoe_status launch_nvfp4_transpose2d(const uint8_t* codes, const uint8_t* sf, in
 // of a [*][cols] input as one matrix (own global scale global_out[g], SR
 // stream stream0 + g * stream_step), codes at codes + gtab[5g+2], scales at
 // sf + gtab[5g+3], output pitch gtab[5g+4] (0: the output's columns).
-// rows_max / pitch_max bound every group's rows and pitch (grid sizing);
-// partials holds groups * nvfp4x_partials(out_rows_max * pitch_max / 16) doubles.
+// ld > 0 (a multiple of 64): every group writes into one matrix of ld-element
+// rows (codes at ld / 2 bytes per row, MMA-tiled atoms over ld / 64 column
+// groups), its offsets naming its first column. rows_max / pitch_max bound
+// every group's rows and pitch (grid sizing); partials holds
+// groups * nvfp4x_partials(out_rows_max * pitch_max / 16) doubles.
 lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t rows_max, int64_t cols,
                                          uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
                                          uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
-                                         uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
+                                         int64_t ld, uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
                                          double* partials, cudaStream_t s);
 // Dense BF16 GEMM on the tensor cores (lmoe_api.cu): out[rows][cols] =
 // epi(x[rows][k] . w[cols][k]^T), token-major tiles, or weight-major ones for

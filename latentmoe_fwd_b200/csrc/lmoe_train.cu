@@ -93,6 +93,7 @@ struct QxParams {
   const int64_t* gtab;
   uint32_t stream_step;
   int vec;               // input 16-byte aligned: row segments read with 16-byte loads
+  int64_t ld;            // elements per destination row (codes, and tiled scale atoms); 0: pitch
 };
 
 // The parameters of group blockIdx.y: its input, outputs, global scale and
@@ -292,6 +293,8 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
   const int64_t R = out_rows(p), C = out_cols(p), nb = C / 16;
   const int64_t nb_store = p.pitch / 16;   // stored blocks per row; those past nb are zero
   const int64_t groups64 = (p.pitch + 63) / 64;
+  const int64_t ld = p.ld > 0 ? p.ld : p.pitch;
+  const int64_t ld64 = (ld + 63) / 64;
   const int64_t rg_cov = p.tiled ? (R + 127) / 128 * 8 : (R + 15) / 16;   // 16-row groups, tiled padding
   const int64_t nb_cov = p.tiled ? groups64 * 4 : nb_store;
   const int64_t items = rg_cov * nb_cov * 16;
@@ -366,14 +369,14 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
           hi = cvt_e2m1_x8(q + 8);
         }
       }
-      *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(lo, hi);
+      *reinterpret_cast<uint2*>(p.codes + ro * (ld / 2) + j * 8) = make_uint2(lo, hi);
     } else if (ro < R && j < nb_store) {
-      *reinterpret_cast<uint2*>(p.codes + ro * (p.pitch / 2) + j * 8) = make_uint2(0u, 0u);
+      *reinterpret_cast<uint2*>(p.codes + ro * (ld / 2) + j * 8) = make_uint2(0u, 0u);
     }
     if (p.tiled) {
-      if (ro < ((R + 127) / 128) * 128) p.sf[tiled_off(ro, j, groups64)] = static_cast<uint8_t>(scode);
+      if (ro < ((R + 127) / 128) * 128) p.sf[tiled_off(ro, j, ld64)] = static_cast<uint8_t>(scode);
     } else if (ro < R && j < nb_store) {
-      p.sf[ro * nb_store + j] = static_cast<uint8_t>(scode);
+      p.sf[ro * (ld / 16) + j] = static_cast<uint8_t>(scode);
     }
   }
 }
@@ -510,7 +513,7 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
 lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t rows_max, int64_t cols,
                                          uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
                                          uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
-                                         uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
+                                         int64_t ld, uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
                                          double* partials, cudaStream_t s) {
   if (groups < 1 || groups > 65535 || !gtab || !global_out || rows_max < 0 || cols <= 0 || cols % 16)
     return LMOE_ERR_INVALID_ARG;
@@ -535,7 +538,8 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
   p.gtab = gtab;
   const int64_t R = p.transpose ? cols : rows_max, C = p.transpose ? rows_max : cols;
   const int64_t pitch = pitch_max > C ? pitch_max : C;
-  if (pitch % 16) return LMOE_ERR_INVALID_ARG;
+  if (pitch % 16 || ld < 0 || ld % 64) return LMOE_ERR_INVALID_ARG;
+  p.ld = ld;
   const int sms = device_sm_count();
   const int np = nvfp4x_partials(R * (pitch / 16) > 0 ? R * (pitch / 16) : 1);
   launch_k(qx_amax_kernel, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);

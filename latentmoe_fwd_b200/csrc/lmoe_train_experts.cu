@@ -154,7 +154,7 @@ dim3 grid_per_expert(int64_t items, int N) {
 // Workspace carve-up (all offsets 256-byte aligned).
 struct BwLayout {
   size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w2tc, w2ts, h, aqc, aqs, o, d_o, dh, deq, qac,
-      qas, qag, dA, t1c, t1s, t1g, t2c, t2s, t2g, part, etab, gtab, itab, total;
+      qas, qag, dA, t1c, t1s, t1g, t2c, t2s, t2g, part, etab, gtab, ktab, total;
   int64_t P, Rmax, Ksum;
 };
 
@@ -196,7 +196,7 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ks
   L.qas = take(P * lm / 16);
   L.qag = take(N * 4);
   L.dA = take(P * m * 4);
-  // wgrad operands: expert e's [lm][K256_e] matrices back to back
+  // wgrad operands: [lm][Ksum] matrices, expert e's K256_e columns at its offset
   L.t1c = take(lm * Ksum / 2);
   L.t1s = take(lm * Ksum / 16);
   L.t1g = take(N * 4);
@@ -213,7 +213,7 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ks
   L.part = take(static_cast<size_t>(np) * 8);
   L.etab = take(N * 4 * 8);       // per expert {p0, n, R, K offset}
   L.gtab = take(6 * N * 5 * 8);   // six quantiser group tables
-  L.itab = take(8 * 4);           // wgrad problem offsets
+  L.ktab = take(N * 2 * 4);       // wgrad K range per expert
   L.total = off;
   return L;
 }
@@ -309,6 +309,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   // row, rows, codes offset, scales offset, pitch}: 0 SR(do), 1 RHT(do)^T,
   // 2 RHT(aq)^T, 3 SR(dh), 4 RHT(dh)^T, 5 RHT(zq)^T
   std::vector<int64_t> etab(static_cast<size_t>(N) * 4), gtab(static_cast<size_t>(6) * N * 5);
+  std::vector<int32_t> ktab(static_cast<size_t>(N) * 2);   // wgrad K range per expert: {first column, blocks}
   int64_t p0 = 0, koff = 0;
   for (int e = 0; e < N; ++e) {
     const int64_t n = counts[e], R = ceil_to(n, 16), K256 = ceil_to(n, 256);
@@ -324,32 +325,31 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
       g[3] = p0 * cols / 16;   // p0 is a multiple of 128: whole scale atoms
       g[4] = 0;
     };
-    auto t_group = [&](int t, int64_t out_rows) {   // [out_rows][K256] after the expert's predecessors
+    auto t_group = [&](int t) {   // columns [koff, koff + K256) of a [out_rows][Ksum] matrix
       int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 5;
       g[0] = p0;
       g[1] = R;
-      g[2] = out_rows * koff / 2;
-      g[3] = out_rows * koff / 16;
+      g[2] = koff / 2;
+      g[3] = koff / 64 * 512;   // koff is a multiple of 256: whole scale atoms
       g[4] = K256;
     };
     row_group(0, l);
-    t_group(1, l);
-    t_group(2, m);
+    t_group(1);
+    t_group(2);
     row_group(3, m);
-    t_group(4, m);
-    t_group(5, l);
+    t_group(4);
+    t_group(5);
+    ktab[2 * e] = static_cast<int32_t>(koff);
+    ktab[2 * e + 1] = static_cast<int32_t>(K256 / 256);
     p0 += ceil_to(n, 128);
     koff += K256;
   }
-  // wgrad problems: one group of l (or m) rows, {0, rows, 0, rows}
-  const int32_t itab[8] = {0, static_cast<int32_t>(l), 0, static_cast<int32_t>(l),
-                           0, static_cast<int32_t>(m), 0, static_cast<int32_t>(m)};
   int64_t* d_etab = at<int64_t>(ws, L.etab);
   int64_t* d_gtab = at<int64_t>(ws, L.gtab);
-  int32_t* d_itab = at<int32_t>(ws, L.itab);
+  int32_t* d_ktab = at<int32_t>(ws, L.ktab);
   if (cudaMemcpyAsync(d_etab, etab.data(), etab.size() * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(d_gtab, gtab.data(), gtab.size() * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(d_itab, itab, sizeof(itab), cudaMemcpyHostToDevice, s) != cudaSuccess)
+      cudaMemcpyAsync(d_ktab, ktab.data(), ktab.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return LMOE_ERR_CUDA;
   auto gt = [&](int t) { return d_gtab + static_cast<size_t>(t) * N * 5; };
 
@@ -442,36 +442,35 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                    float* g) {
     const bool tr = (flags & LMOE_QX_TRANSPOSE) != 0;
     return launch_nvfp4_quantize_groups(in, LMOE_F32, L.Rmax, cols, flags, rht_signs, seed, stream0, 4, gt(t), N,
-                                        tr ? K256max : cols, c, sf, g, LMOE_SF_MMA_TILED, part, s);
+                                        tr ? K256max : cols, tr ? L.Ksum : 0, c, sf, g, LMOE_SF_MMA_TILED, part,
+                                        s);
   };
-  // the wgrad of every expert with rows: out[rows][cols] = A[rows][K256] . B[cols][K256]^T
+  // every expert's wgrad in one K-batched launch: dW[e] [rows][cols] =
+  // A[:, K_e] . B[:, K_e]^T over the expert's K256 columns (experts without
+  // rows get a zero gradient)
   auto wgrads = [&](int64_t rows, int64_t cols, void* dw) -> lmoe_status {
-    for (int e = 0; e < N; ++e) {
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(dw) + e * rows * cols;
-      const int64_t K256 = ceil_to(counts[e], 256), ko = etab[4 * e + 3];
-      if (K256 == 0) {   // no rows: zero weight gradient
-        if (cudaMemsetAsync(out, 0, rows * cols * 2, s) != cudaSuccess) return LMOE_ERR_CUDA;
-        continue;
-      }
-      Fp4Launch g;
-      g.a_codes = t1c + rows * ko / 2;
-      g.a_sf = t1s + rows * ko / 16;
-      g.a_rows = rows;
-      g.b_codes = t2c + cols * ko / 2;
-      g.b_sf = t2s + cols * ko / 16;
-      g.k = K256;
-      g.cols = static_cast<int>(cols);
-      g.groups = 1;
-      g.offsets = d_itab + (rows == l ? 0 : 4);   // {0, rows}
-      g.padded_offsets = g.offsets + 2;
-      g.in_scale = t1g + e;
-      g.w_scale = t2g + e;
-      g.out = out;
-      g.ld_out = cols;
-      lmoe_status r = fp4_gemm(g, err, s);
-      if (r != LMOE_OK) return r;
-    }
-    return LMOE_OK;
+    for (int e = 0; e < N; ++e)
+      if (counts[e] == 0 &&
+          cudaMemsetAsync(static_cast<__nv_bfloat16*>(dw) + e * rows * cols, 0, rows * cols * 2, s) != cudaSuccess)
+        return LMOE_ERR_CUDA;
+    if (L.Ksum == 0) return LMOE_OK;
+    Fp4Launch g;
+    g.a_codes = t1c;
+    g.a_sf = t1s;
+    g.a_rows = rows;
+    g.b_codes = t2c;
+    g.b_sf = t2s;
+    g.k = L.Ksum;
+    g.cols = static_cast<int>(cols);
+    g.groups = N;
+    g.kgroups = d_ktab;
+    g.in_scale = t1g;
+    g.in_scale_grouped = 1;
+    g.w_scale = t2g;
+    g.out = dw;
+    g.ld_out = cols;
+    g.out_group_stride = rows * cols;
+    return fp4_gemm(g, err, s);
   };
 
   // do, dgate
