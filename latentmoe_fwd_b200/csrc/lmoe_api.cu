@@ -35,6 +35,38 @@ size_t act_bytes(const lmoe_config* c) { return c->act == LMOE_F32 ? 4 : 2; }
 
 bool identity(const lmoe_config* c) { return (c->flags & LMOE_FLAG_IDENTITY_PROJ) != 0; }
 
+// A host thread's second stream on a device (highest priority) with the two
+// events that fork work onto it and join it back, created on first use and
+// kept for the thread's life. Per thread, so that concurrent callers never
+// record one another's events.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+bool side_stream(SideStream* out) {
+  thread_local SideStream per_device[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  SideStream& ss = per_device[dev];
+  if (!ss.stream) {
+    int lo = 0, hi = 0;
+    SideStream made;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&made.stream, cudaStreamNonBlocking, hi) != cudaSuccess)
+      return false;
+    if (cudaEventCreateWithFlags(&made.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&made.join, cudaEventDisableTiming) != cudaSuccess) {
+      if (made.fork) cudaEventDestroy(made.fork);
+      cudaStreamDestroy(made.stream);
+      return false;
+    }
+    ss = made;
+  }
+  *out = ss;
+  return true;
+}
+
 int64_t padded_rows(const lmoe_config* c) {
   const int64_t slots = c->T * c->K;
   const int64_t nonempty = slots < c->N ? slots : c->N;
@@ -796,6 +828,18 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   float* gw = at<float>(ws, L.w);
   float* logits = at<float>(ws, L.logits);
 
+  // BF16 latent layer at prefill sizes: the permutation runs first, then the
+  // down-projection stores z once and a token-order copy reads each z row once
+  // and writes it to the padded rows of its K slots
+  const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens && l >= 64;
+  // The top-K and the permutation need only the router logits, the
+  // down-projection only x: when both follow, the routing runs on a side
+  // stream beside the down-projection GEMM (whose persistent CTAs leave room
+  // on every SM for the routing's small ones). Not while tracing stages.
+  SideStream side;
+  const bool overlap = !events && (scatter_z || (fp4 && !ident)) && side_stream(&side);
+  cudaStream_t rs = overlap ? side.stream : s;
+
   // 1. router logits (+ bias) and top-K gates
   if (f32) {
     SimtLaunch S;
@@ -814,9 +858,16 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
                     L.rsplit ? at<float>(ws, L.rsplit) : splitk, err, s);
   }
   if (st != LMOE_OK) return st;
-  if ((st = launch_topk(logits, T, N, K, idx, gw, x, w->w_router, w->router_bias, d, cfg->act, err, s)) != LMOE_OK)
+  if (overlap && (cudaEventRecord(side.fork, s) != cudaSuccess || cudaStreamWaitEvent(rs, side.fork, 0) != cudaSuccess))
+    return LMOE_ERR_CUDA;
+  if ((st = launch_topk(logits, T, N, K, idx, gw, x, w->w_router, w->router_bias, d, cfg->act, err, rs)) != LMOE_OK)
     return st;
   mark(1);
+  // the main stream waits for the routing (no-op without the side stream)
+  auto join_routing = [&]() {
+    return !overlap || (cudaEventRecord(side.join, rs) == cudaSuccess && cudaStreamWaitEvent(s, side.join, 0) ==
+                        cudaSuccess);
+  };
 
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* poff = at<int32_t>(ws, L.poff);
@@ -825,18 +876,15 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   float* gate = at<float>(ws, L.gate);
   void* zp = at<void>(ws, L.zp);
   float* z_gs = nullptr;
-  // BF16 latent layer at prefill sizes: the permutation runs first, then the
-  // down-projection stores z once and a token-order copy reads each z row once
-  // and writes it to the padded rows of its K slots
-  const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens && l >= 64;
   if (scatter_z) {
     int32_t* slot_row = at<int32_t>(ws, L.slot_row);
     if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
-                             err, s, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
+                             err, rs, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
       return st;
     void* zb = at<void>(ws, L.z);
     if ((st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s)) != LMOE_OK)
       return st;
+    if (!join_routing()) return LMOE_ERR_CUDA;
     mark(2);
     if ((st = launch_scatter_rows(zb, T, static_cast<int64_t>(l) * ab, slot_row, K, zp, s)) != LMOE_OK) return st;
     mark(3);
@@ -846,7 +894,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     // the padded rows of its K slots
     int32_t* slot_row = at<int32_t>(ws, L.slot_row);
     if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
-                             err, s, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
+                             err, rs, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
       return st;
     const void* z = x;
     if (!ident) {
@@ -855,6 +903,7 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
         return st;
       z = zb;
     }
+    if (!join_routing()) return LMOE_ERR_CUDA;
     z_gs = at<float>(ws, L.z_gs);
     if ((st = launch_nvfp4_quantize_scatter(z, T, l, slot_row, K, static_cast<uint8_t*>(zp), at<uint8_t>(ws, L.zp_sf),
                                             z_gs, at<float>(ws, L.partials), nvfp4_partials(T * l), s)) != LMOE_OK)
