@@ -563,6 +563,63 @@ lmoe_status lmoe_ep_plan(int G, int rank, int N, const int32_t* counts, int32_t*
 lmoe_status lmoe_ep_reorder(const void* in, void* out, int64_t row_bytes, int nblocks, const int32_t* src_rows,
                             const int32_t* dst_rows, const int64_t* row_prefix, int64_t total_rows, void* stream);
 
+/* The expert-parallel data plane over peer memory (greeksharifa page,
+ * section 2.2 "LatentMoE": the rows that cross GPUs are the l-dim latent
+ * rows). Instead of an all-to-all into a staging buffer and a reorder, each
+ * rank's dispatch kernel stores its token rows straight into the owner
+ * ranks' expert-grouped buffers through peer pointers, and its combine kernel
+ * reads the owners' expert outputs back the same way; the owners run
+ * lmoe_expert_ffn on their received rows between the two. Plain loads and
+ * stores only (no TMA, no multicast). Between the phases the caller
+ * separates the ranks with a barrier of its own (every rank's dispatch done
+ * before any owner's expert FFN; every expert FFN done before any combine):
+ * the kernels do not wait on other GPUs.
+ *
+ * lmoe_ep_slot_bases (HOST arrays, no device work): from counts [G][N] (after
+ * the count exchange) gives, for this rank, expert_owner [N] (the rank that
+ * owns each expert, ownership as lmoe_ep_plan) and dst_base [N]: the owner's
+ * padded row of this rank's first row for the expert in the owner's
+ * expert-grouped buffer (sources in rank order inside an expert, each expert's
+ * range padded to 128 rows: lmoe_ep_plan's local_padded_offsets and
+ * block_dst). Errors as lmoe_ep_plan. */
+lmoe_status lmoe_ep_slot_bases(int G, int rank, int N, const int32_t* counts, int32_t* expert_owner,
+                               int32_t* dst_base);
+
+/* Dispatch: slot f = t*K + k (expert e = topk_idx[f]; slots with e outside
+ * [0, N) are skipped, as lmoe_permute leaves them out) goes to rank
+ * h = expert_owner[e], row dst_base[e] + inv_perm[f] - offsets[e] of that
+ * rank's buffer: the token's row rows[t] (row_bytes, a multiple of 16) is
+ * copied there, and with topk_w its gate to the same row of the rank's gate
+ * buffer (F32, the perm_gate of its lmoe_expert_ffn call).
+ *  topk_idx, inv_perm, offsets: this rank's lmoe_permute results ([T][K],
+ *  [T*K], [N+1]); expert_owner, dst_base [N]: DEVICE copies of
+ *  lmoe_ep_slot_bases's arrays; peer_rows [G], peer_gates [G] (or NULL with
+ *  topk_w NULL): DEVICE arrays of device pointers, rank h's buffers (another
+ *  GPU's memory mapped into this process, or this GPU's own for h = rank),
+ *  each holding peer_rows_cap rows. err_word (device, may be NULL): a row or
+ *  owner out of range is skipped and recorded there (LMOE_ERR_DEVICE_BOUNDS,
+ *  info the slot) as in a workspace's error word. Asynchronous on `stream`.
+ *  Errors: LMOE_ERR_INVALID_ARG for null pointers, K outside [1, 32], sizes,
+ *  unaligned rows, topk_w without peer_gates or the reverse. */
+lmoe_status lmoe_ep_dispatch(int64_t T, int K, int N, int G, const void* rows, int64_t row_bytes,
+                             const int32_t* topk_idx, const int32_t* inv_perm, const int32_t* offsets,
+                             const int32_t* expert_owner, const int32_t* dst_base, void* const* peer_rows,
+                             int64_t peer_rows_cap, const float* topk_w, float* const* peer_gates, uint32_t* err_word,
+                             void* stream);
+
+/* Combine: c[t] = sum over the token's in-range slots, in k order, in fp32,
+ * of the owner's expert-output row (BF16 [*][l], gates applied by the owner's
+ * lmoe_expert_ffn from the dispatched gates) at the slot's row, stored BF16
+ * -- lmoe_combine's arithmetic with topk_w NULL. peer_y [G]: DEVICE array of
+ * the ranks' y buffers (peer_rows_cap rows each); the other arguments as
+ * lmoe_ep_dispatch; c [T][l] (16-byte aligned), l a multiple of 8.
+ *  Errors: LMOE_ERR_INVALID_ARG for null pointers, K outside [1, 32], sizes,
+ *  an unaligned c; LMOE_ERR_UNSUPPORTED for T >= 2^31. */
+lmoe_status lmoe_ep_combine(int64_t T, int K, int N, int G, int l, const void* const* peer_y, int64_t peer_rows_cap,
+                            const int32_t* topk_idx, const int32_t* inv_perm, const int32_t* offsets,
+                            const int32_t* expert_owner, const int32_t* dst_base, void* c, uint32_t* err_word,
+                            void* stream);
+
 /* Synchronises `stream`, returns the device error status recorded in the
  * workspace `ws` (LMOE_OK if none) and clears it (the read and the clear run
  * on `stream`). `info` (host, may be NULL) receives a kernel-specific detail

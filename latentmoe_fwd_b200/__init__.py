@@ -39,7 +39,8 @@ EXPORTS = ("lmoe_workspace_size", "lmoe_padded_rows", "lmoe_route", "lmoe_permut
            "lmoe_forward_traced", "lmoe_permute_noalloc", "lmoe_selftest_wait_timeout", "lmoe_fp8_quantize",
            "lmoe_nvfp4_quantize_ex", "lmoe_nvfp4_quantize_ex_workspace", "lmoe_nvfp4_transpose_2d",
            "lmoe_nvfp4_gemm",
-           "lmoe_ep_plan", "lmoe_ep_reorder", "lmoe_expert_backward_nvfp4",
+           "lmoe_ep_plan", "lmoe_ep_reorder", "lmoe_ep_slot_bases", "lmoe_ep_dispatch", "lmoe_ep_combine",
+           "lmoe_expert_backward_nvfp4",
            "lmoe_expert_backward_nvfp4_workspace", "lmoe_backward_nvfp4", "lmoe_backward_nvfp4_workspace")
 TRACE_EVENTS = 8
 TRACE_STAGES = ("route", "down_proj", "permute", "expert_gemm1", "expert_gemm2", "combine", "up_proj")
@@ -99,6 +100,11 @@ def _load():
         "lmoe_nvfp4_transpose_2d": (ctypes.c_int, [P, P, I64, I64, I64, P, P, P]),
         "lmoe_ep_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int] + [P] * 12),
         "lmoe_ep_reorder": (ctypes.c_int, [P, P, I64, ctypes.c_int, P, P, P, I64, P]),
+        "lmoe_ep_slot_bases": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]),
+        "lmoe_ep_dispatch": (ctypes.c_int, [I64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, I64, P, P, P, P, P, P,
+                                            I64, P, P, P, P]),
+        "lmoe_ep_combine": (ctypes.c_int, [I64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, I64, P, P,
+                                           P, P, P, P, P, P]),
         "lmoe_nvfp4_gemm": (ctypes.c_int, [ctypes.c_int, P, P, I64, P, P, P, ctypes.c_int, P, P, P, ctypes.c_int,
                                            I64, P, P, I64, P, ctypes.c_size_t, P]),
         "lmoe_nvfp4_quantize_ex": (ctypes.c_int, [P, ctypes.c_int, I64, I64, ctypes.c_uint32, ctypes.c_uint32,
@@ -354,6 +360,38 @@ def ep_reorder(x, out, row_bytes, src_rows, dst_rows, row_prefix, total_rows, st
     """lmoe_ep_reorder: copy row blocks (device tensors; row_prefix int64)."""
     _check(lib.lmoe_ep_reorder(_p(x), _p(out), int(row_bytes), int(src_rows.numel()), _p(src_rows), _p(dst_rows),
                                _p(row_prefix), int(total_rows), _stream(stream)), "lmoe_ep_reorder")
+
+
+def ep_slot_bases(G: int, rank: int, counts):
+    """lmoe_ep_slot_bases on host arrays: counts [G][N] int32 (numpy) ->
+    (expert_owner [N], dst_base [N]) numpy int32 arrays for this rank."""
+    import numpy as np
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    N = counts.shape[1]
+    owner = np.zeros(N, dtype=np.int32)
+    base = np.zeros(N, dtype=np.int32)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib.lmoe_ep_slot_bases(G, rank, N, ptr(counts), ptr(owner), ptr(base)), "lmoe_ep_slot_bases")
+    return owner, base
+
+
+def ep_dispatch(T, K, N, G, rows, row_bytes, topk_idx, inv_perm, offsets, expert_owner, dst_base, peer_rows,
+                peer_rows_cap, topk_w=None, peer_gates=None, err_word=None, stream=None):
+    """lmoe_ep_dispatch: this rank's token rows (and gates) stored at their
+    slots' rows in the owners' buffers. peer_rows / peer_gates: int64 device
+    tensors of the G buffers' addresses."""
+    _check(lib.lmoe_ep_dispatch(int(T), int(K), int(N), int(G), _p(rows), int(row_bytes), _p(topk_idx), _p(inv_perm),
+                                _p(offsets), _p(expert_owner), _p(dst_base), _p(peer_rows), int(peer_rows_cap),
+                                _p(topk_w), _p(peer_gates), _p(err_word), _stream(stream)), "lmoe_ep_dispatch")
+
+
+def ep_combine(T, K, N, G, l, peer_y, peer_rows_cap, topk_idx, inv_perm, offsets, expert_owner, dst_base, c,
+               err_word=None, stream=None):
+    """lmoe_ep_combine: c[t] = the k-ordered fp32 sum of the owners' expert
+    rows of the token's slots (peer_y: int64 device tensor of addresses)."""
+    _check(lib.lmoe_ep_combine(int(T), int(K), int(N), int(G), int(l), _p(peer_y), int(peer_rows_cap),
+                               _p(topk_idx), _p(inv_perm), _p(offsets), _p(expert_owner), _p(dst_base), _p(c),
+                               _p(err_word), _stream(stream)), "lmoe_ep_combine")
 
 
 def selftest_wait_timeout(ws, limit_cycles: int, stream=None):

@@ -13,6 +13,7 @@
 // order, each sorted by expert; the expert GEMMs want every local expert's
 // rows together (source rank ascending inside an expert) at padded offsets
 // (multiples of 128), so each (source, expert) block moves as a whole.
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "lmoe_device.cuh"
@@ -50,6 +51,118 @@ __global__ void __launch_bounds__(256) ep_reorder_kernel(const uint8_t* __restri
   const uint4* s = reinterpret_cast<const uint4*>(in + (static_cast<int64_t>(__ldg(src + lo)) + i) * row_bytes);
   uint4* d = reinterpret_cast<uint4*>(out + (static_cast<int64_t>(__ldg(dst + lo)) + i) * row_bytes);
   for (int64_t v = lane; v < row_bytes / 16; v += 32) d[v] = __ldg(s + v);
+}
+
+// Dispatch over peer memory: a warp per token reads its row once (2 KB per
+// pass, four 16-byte loads per lane) and stores it, with its gate, at each of
+// its K slots' rows in the owner rank's expert-grouped buffer. Slot f = t*K+k
+// of expert e goes to rank owner[e], row dst_base[e] + inv_perm[f] - offsets[e].
+// Plain stores to peer-mapped (or local) memory; a slot whose expert or row is
+// out of range is skipped and reported.
+__global__ void __launch_bounds__(256) ep_dispatch_kernel(
+    const uint8_t* __restrict__ rows, int64_t T, int64_t row_bytes, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ inv_perm, const int32_t* __restrict__ offsets, const int32_t* __restrict__ owner,
+    const int32_t* __restrict__ dst_base, uint8_t* const* __restrict__ peer_rows, const float* __restrict__ gates,
+    float* const* __restrict__ peer_gates, int K, int N, int G, int64_t rows_cap, DevErr err) {
+  pdl_begin();
+  constexpr unsigned FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const int64_t n16 = row_bytes >> 4;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    int h = -1;
+    int64_t row = -1;
+    if (lane < K) {
+      const int64_t f = t * K + lane;
+      const int e = __ldg(idx + f);
+      if (e >= 0 && e < N) {
+        h = __ldg(owner + e);
+        row = static_cast<int64_t>(__ldg(dst_base + e)) + __ldg(inv_perm + f) - __ldg(offsets + e);
+        if (h < 0 || h >= G || row < 0 || row >= rows_cap) {
+          dev_report(err, kErrBounds, static_cast<uint32_t>(f));
+          h = -1;
+        }
+      }
+      if (h >= 0 && gates && peer_gates) peer_gates[h][row] = __ldg(gates + f);
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(rows + t * row_bytes);
+    for (int64_t i0 = 0; i0 < n16; i0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = i0 + u * 32 + lane;
+        v[u] = i < n16 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      for (int k = 0; k < K; ++k) {
+        const int hk = __shfl_sync(FULL, h, k);
+        const int64_t rk = __shfl_sync(FULL, row, k);
+        if (hk < 0) continue;
+        uint4* dst = reinterpret_cast<uint4*>(peer_rows[hk] + rk * row_bytes);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t i = i0 + u * 32 + lane;
+          if (i < n16) dst[i] = v[u];
+        }
+      }
+    }
+  }
+}
+
+// Combine over peer memory: c[t] = sum over the token's in-range slots, in k
+// order, of the owner's y row (gates already applied by the owner), in fp32,
+// stored BF16 -- the arithmetic of the single-GPU combine with no gate. A CTA
+// per token.
+__global__ void __launch_bounds__(256) ep_combine_kernel(
+    const __nv_bfloat16* const* __restrict__ peer_y, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ inv_perm, const int32_t* __restrict__ offsets, const int32_t* __restrict__ owner,
+    const int32_t* __restrict__ dst_base, __nv_bfloat16* __restrict__ c, int K, int N, int G, int l,
+    int64_t rows_cap, DevErr err) {
+  pdl_begin();
+  __shared__ const __nv_bfloat16* rowp[32];
+  __shared__ int s_nk;
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < 32) {
+    const int k = threadIdx.x;
+    bool ok = false;
+    const __nv_bfloat16* p = nullptr;
+    if (k < K) {
+      const int64_t f = t * K + k;
+      const int e = __ldg(idx + f);
+      if (e >= 0 && e < N) {
+        const int h = __ldg(owner + e);
+        const int64_t row = static_cast<int64_t>(__ldg(dst_base + e)) + __ldg(inv_perm + f) - __ldg(offsets + e);
+        ok = h >= 0 && h < G && row >= 0 && row < rows_cap;
+        if (ok) p = peer_y[h] + row * l;
+        else dev_report(err, kErrBounds, static_cast<uint32_t>(f));
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    if (ok) rowp[__popc(m & ((1u << k) - 1u))] = p;
+    if (k == 0) s_nk = __popc(m);
+  }
+  __syncthreads();
+  const int nk = s_nk;
+  for (int col = threadIdx.x * 8; col < l; col += blockDim.x * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int k = 0; k < nk; ++k) {
+      const uint4 u = *reinterpret_cast<const uint4*>(rowp[k] + col);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __bfloat1622float2(h2[i]);
+        acc[2 * i] += f2.x;
+        acc[2 * i + 1] += f2.y;
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(c + t * l + col) = o;
+  }
 }
 
 }  // namespace
@@ -141,6 +254,73 @@ lmoe_status lmoe_ep_reorder(const void* in, void* out, int64_t row_bytes, int nb
   launch_k(ep_reorder_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, static_cast<cudaStream_t>(stream),
            static_cast<const uint8_t*>(in), static_cast<uint8_t*>(out), row_bytes, src_rows, dst_rows, row_prefix,
            nblocks, total_rows);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+lmoe_status lmoe_ep_slot_bases(int G, int rank, int N, const int32_t* counts, int32_t* expert_owner,
+                               int32_t* dst_base) {
+  if (G <= 0 || N <= 0 || rank < 0 || rank >= G || !counts || !expert_owner || !dst_base)
+    return LMOE_ERR_INVALID_ARG;
+  if (N > 1024 || G > N) return LMOE_ERR_UNSUPPORTED;
+  for (int64_t i = 0; i < static_cast<int64_t>(G) * N; ++i)
+    if (counts[i] < 0) return LMOE_ERR_INVALID_ARG;
+  for (int h = 0; h < G; ++h) {
+    int f0 = 0, nl = 0;
+    ownership(G, N, h, &f0, &nl);
+    int64_t poff = 0;   // owner h's padded offset of its expert f0 + el
+    for (int el = 0; el < nl; ++el) {
+      const int e = f0 + el;
+      int64_t tot = 0, before = 0;
+      for (int g = 0; g < G; ++g) {
+        const int64_t c = counts[static_cast<int64_t>(g) * N + e];
+        tot += c;
+        if (g < rank) before += c;
+      }
+      if (poff + before > INT32_MAX) return LMOE_ERR_UNSUPPORTED;
+      expert_owner[e] = h;
+      dst_base[e] = static_cast<int32_t>(poff + before);
+      poff += (tot + 127) / 128 * 128;
+    }
+  }
+  return LMOE_OK;
+}
+
+lmoe_status lmoe_ep_dispatch(int64_t T, int K, int N, int G, const void* rows, int64_t row_bytes,
+                             const int32_t* topk_idx, const int32_t* inv_perm, const int32_t* offsets,
+                             const int32_t* expert_owner, const int32_t* dst_base, void* const* peer_rows,
+                             int64_t peer_rows_cap, const float* topk_w, float* const* peer_gates, uint32_t* err_word,
+                             void* stream) {
+  if (T < 0 || K < 1 || K > 32 || N < 1 || G < 1 || peer_rows_cap < 0) return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!rows || !topk_idx || !inv_perm || !offsets || !expert_owner || !dst_base || !peer_rows)
+    return LMOE_ERR_INVALID_ARG;
+  if (row_bytes <= 0 || row_bytes % 16 || (reinterpret_cast<uintptr_t>(rows) & 15)) return LMOE_ERR_INVALID_ARG;
+  if ((topk_w == nullptr) != (peer_gates == nullptr)) return LMOE_ERR_INVALID_ARG;
+  const int64_t sms = device_sm_count();
+  int64_t blocks = (T * 32 + 255) / 256;
+  if (blocks > sms * 8) blocks = sms * 8;
+  launch_k(ep_dispatch_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, static_cast<cudaStream_t>(stream),
+           static_cast<const uint8_t*>(rows), T, row_bytes, topk_idx, inv_perm, offsets, expert_owner, dst_base,
+           reinterpret_cast<uint8_t* const*>(peer_rows), topk_w, peer_gates, K, N, G, peer_rows_cap,
+           DevErr{err_word});
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+lmoe_status lmoe_ep_combine(int64_t T, int K, int N, int G, int l, const void* const* peer_y, int64_t peer_rows_cap,
+                            const int32_t* topk_idx, const int32_t* inv_perm, const int32_t* offsets,
+                            const int32_t* expert_owner, const int32_t* dst_base, void* c, uint32_t* err_word,
+                            void* stream) {
+  if (T < 0 || K < 1 || K > 32 || N < 1 || G < 1 || l <= 0 || l % 8 || peer_rows_cap < 0)
+    return LMOE_ERR_INVALID_ARG;
+  if (T == 0) return LMOE_OK;
+  if (!peer_y || !topk_idx || !inv_perm || !offsets || !expert_owner || !dst_base || !c) return LMOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(c) & 15) return LMOE_ERR_INVALID_ARG;
+  if (T > 0x7fffffff) return LMOE_ERR_UNSUPPORTED;
+  launch_k(ep_combine_kernel, dim3(static_cast<unsigned>(T)), dim3(256), 0, static_cast<cudaStream_t>(stream),
+           reinterpret_cast<const __nv_bfloat16* const*>(peer_y), topk_idx, inv_perm, offsets, expert_owner,
+           dst_base, static_cast<__nv_bfloat16*>(c), K, N, G, l, peer_rows_cap, DevErr{err_word});
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }

@@ -128,3 +128,35 @@ def test_ep_plan_rejects_bad_arguments():
         L.ep_plan(3, 0, np.zeros((3, 2), dtype=np.int32))          # more ranks than experts
     with pytest.raises(L.LmoeError):
         L.ep_plan(2, 0, -np.ones((2, 4), dtype=np.int32))          # negative counts
+
+
+def _owner_first(G, N, h):
+    base, extra = N // G, N % G
+    return h * base + min(h, extra), base + (1 if h < extra else 0)
+
+
+@pytest.mark.parametrize("G,N", [(2, 8), (3, 10), (4, 4)])
+def test_slot_bases_follow_the_ownership_and_padded_layout(G, N):
+    # written out here from the ownership rule and the padded expert-grouped
+    # layout: owner h's expert e starts at the sum of its earlier experts'
+    # totals (over all sources) rounded up to 128, and rank r's rows for e
+    # follow those of ranks < r
+    L = pytest.importorskip("latentmoe_fwd_b200")
+    rng = np.random.default_rng(G * 100 + N)
+    counts = rng.integers(0, 300, size=(G, N)).astype(np.int32)
+    counts[0, 1] = 0
+    for r in range(G):
+        owner, base = L.ep_slot_bases(G, r, counts)
+        for h in range(G):
+            f0, nl = _owner_first(G, N, h)
+            poff = 0
+            for e in range(f0, f0 + nl):
+                assert owner[e] == h
+                assert base[e] == poff + counts[:r, e].sum()
+                poff += -(-int(counts[:, e].sum()) // 128) * 128
+        # the same rows as the plan's (source r, local expert) blocks at each owner
+        for h in range(G):
+            plan = L.ep_plan(G, h, counts)
+            f0, nl = plan["first_expert"], plan["local_experts"]
+            for el in range(nl):
+                assert base[f0 + el] == plan["block_dst"][r * nl + el]
