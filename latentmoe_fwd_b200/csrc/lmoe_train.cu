@@ -28,7 +28,10 @@ constexpr int kXThreads = 256;
 // E4M3 code -> exact value: subnormal f * 2^-9, normal (8 + f) * 2^(e - 10).
 __device__ __forceinline__ double e4m3_exact(uint32_t c) {
   const int e = (c >> 3) & 15, f = c & 7;
-  return e == 0 ? ldexp(static_cast<double>(f), -9) : ldexp(static_cast<double>(8 + f), e - 10);
+  // f * 2^-9 or (8 + f) * 2^(e - 10): a small integer times a power of two
+  // built from its exponent bits (both exact)
+  const int ex = e == 0 ? -9 : e - 10;
+  return static_cast<double>(e == 0 ? f : 8 + f) * __longlong_as_double(static_cast<long long>(ex + 1023) << 52);
 }
 
 // Philox-4x32-10 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
@@ -58,10 +61,11 @@ __device__ __forceinline__ void sr_uniforms16(uint64_t i0, uint64_t seed, uint32
     const uint64_t c = (i0 >> 2) + q;
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), stream, 0u),
                                   static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
-    u[4 * q + 0] = ldexpf(static_cast<float>(w.x >> 8), -24);
-    u[4 * q + 1] = ldexpf(static_cast<float>(w.y >> 8), -24);
-    u[4 * q + 2] = ldexpf(static_cast<float>(w.z >> 8), -24);
-    u[4 * q + 3] = ldexpf(static_cast<float>(w.w >> 8), -24);
+    constexpr float k2m24 = 1.0f / 16777216.0f;   // 2^-24: the products are exact
+    u[4 * q + 0] = static_cast<float>(w.x >> 8) * k2m24;
+    u[4 * q + 1] = static_cast<float>(w.y >> 8) * k2m24;
+    u[4 * q + 2] = static_cast<float>(w.z >> 8) * k2m24;
+    u[4 * q + 3] = static_cast<float>(w.w >> 8) * k2m24;
   }
 }
 
@@ -88,10 +92,19 @@ struct QxParams {
   // scale): strides between the groups' inputs (elements), codes and scales (bytes)
   int64_t gs_in, gs_codes, gs_sf;
   // ragged groups instead (gtab non-null): per group {first input row, input
-  // rows, codes offset, scales offset (bytes), output pitch (0: out cols)};
-  // group g draws its SR uniforms on stream + g * stream_step
+  // rows, codes offset, scales offset (bytes), output pitch (0: out cols),
+  // rows holding data (the rest read as zero; NVFP4 input)}; group g draws
+  // its SR uniforms on stream + g * stream_step
   const int64_t* gtab;
   uint32_t stream_step;
+  // NVFP4 input: `in` holds E2M1 codes [*][cols/2] with MMA-tiled scales in_sf
+  // (over the absolute rows) and the global scale *in_global; an element is
+  // fp32(code * scale * global), formed exactly in fp64 and rounded once
+  int fp4in;
+  const uint8_t* in_sf;
+  const float* in_global;
+  float in_gs;
+  int64_t in_row0, real_rows;
   int vec;               // input 16-byte aligned: row segments read with 16-byte loads
   int64_t ld;            // elements per destination row (codes, and tiled scale atoms); 0: pitch
 };
@@ -102,8 +115,13 @@ __device__ __forceinline__ QxParams qx_group(const QxParams& p0) {
   QxParams p = p0;
   const int64_t g = blockIdx.y;
   if (p0.gtab) {
-    const int64_t* t = p0.gtab + g * 5;
-    p.in = static_cast<const uint8_t*>(p0.in) + t[0] * p0.cols * (p0.bf16 ? 2 : 4);
+    const int64_t* t = p0.gtab + g * 6;
+    if (p0.fp4in) {   // rows are addressed absolutely (the scales' tiling)
+      p.in_row0 = t[0];
+      p.real_rows = t[5];
+    } else {
+      p.in = static_cast<const uint8_t*>(p0.in) + t[0] * p0.cols * (p0.bf16 ? 2 : 4);
+    }
     p.rows = t[1];
     p.codes += t[2];
     p.sf += t[3];
@@ -121,7 +139,22 @@ __device__ __forceinline__ QxParams qx_group(const QxParams& p0) {
   return p;
 }
 
+// E2M1 magnitude by code (0, 0.5, 1, 1.5, 2, 3, 4, 6), without a table.
+__device__ __forceinline__ double e2m1_mag_d(uint32_t c) {
+  return (c < 4) ? 0.5 * static_cast<double>(c) : (c < 6 ? static_cast<double>(c - 2) : (c == 6 ? 4.0 : 6.0));
+}
+
 __device__ __forceinline__ double load_in(const QxParams& p, int64_t r, int64_t c) {
+  if (p.fp4in) {
+    if (r >= p.real_rows) return 0.0;
+    const int64_t row = p.in_row0 + r;
+    const uint32_t byte = static_cast<const uint8_t*>(p.in)[row * (p.cols / 2) + (c >> 1)];
+    const uint32_t code = (c & 1) ? byte >> 4 : byte & 15u;
+    const int64_t j = c >> 4, g64 = p.cols / 64;
+    const uint32_t s = p.in_sf[((row >> 7) * g64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3)];
+    const double sc = e4m3_exact(s) * static_cast<double>(p.in_gs);
+    return static_cast<double>(__double2float_rn((code & 8u ? -1.0 : 1.0) * e2m1_mag_d(code & 7u) * sc));
+  }
   if (p.bf16) return static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(p.in)[r * p.cols + c]));
   return static_cast<double>(static_cast<const float*>(p.in)[r * p.cols + c]);
 }
@@ -186,10 +219,12 @@ __device__ __forceinline__ void load_block_f32(const QxParams& p, int64_t ro, in
   }
 }
 
-// E4M3 code -> value in fp32 (exact: at most 4 significant bits).
+// E4M3 code -> value in fp32 (exact: at most 4 significant bits, a normal
+// power of two between 2^-9 and 2^5).
 __device__ __forceinline__ float e4m3_exact_f(uint32_t c) {
   const int e = (c >> 3) & 15, f = c & 7;
-  return e == 0 ? ldexpf(static_cast<float>(f), -9) : ldexpf(static_cast<float>(8 + f), e - 10);
+  const int ex = e == 0 ? -9 : e - 10;
+  return static_cast<float>(e == 0 ? f : 8 + f) * __int_as_float((ex + 127) << 23);
 }
 
 __device__ __forceinline__ int64_t out_rows(const QxParams& p) { return p.transpose ? p.cols : p.rows; }
@@ -198,7 +233,8 @@ __device__ __forceinline__ int64_t out_cols(const QxParams& p) { return p.transp
 // Pass 1: per-CTA maxima of |out| (fp64, exact).
 __global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, double* __restrict__ partials) {
   pdl_begin();
-  const QxParams p = qx_group(p0);
+  QxParams p = qx_group(p0);
+  if (p.fp4in) p.in_gs = __ldg(p.in_global);
   partials += static_cast<int64_t>(blockIdx.y) * gridDim.x;
   __shared__ double red[kXThreads / 32];
   const int64_t nb = out_cols(p) / 16, total = out_rows(p) * nb;
@@ -267,7 +303,8 @@ __device__ __forceinline__ int64_t tiled_off(int64_t row, int64_t j, int64_t gro
 template <bool RHT>
 __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0) {
   pdl_begin();
-  const QxParams p = qx_group(p0);
+  QxParams p = qx_group(p0);
+  if (p.fp4in) p.in_gs = __ldg(p.in_global);
   __shared__ double red[kXThreads / 32];
   __shared__ float s_gs;
   // global scale: s_g = fp32(amax / 2688) from the fp64 amax (1 when 0)
@@ -300,49 +337,61 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
   const int64_t items = rg_cov * nb_cov * 16;
   const int64_t items32 = (items + 31) / 32 * 32;
   const int i16 = threadIdx.x & 15;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items32;
-       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const bool live = it < items;
+  // One item per thread and pass: output row ro, block j. `fetch` reads its 16
+  // values and their amax; `finish` forms the 16 x 16 amax (half-warp
+  // shuffles, every lane takes part), then encodes and stores. (Two items in
+  // flight per thread measured slower: the extra registers cost occupancy.)
+  struct Item {
+    bool live, has;
+    int64_t ro, j;
+    double m;
+    double v[RHT ? 16 : 1];
+    float vf[RHT ? 1 : 16];
+  };
+  auto fetch = [&](int64_t it, Item& I) {
+    I.live = it < items;
     const int64_t b = it >> 4;   // (16-row group, block) of this half-warp
     // transposed input: consecutive groups are consecutive input columns
     const int64_t g = p.transpose ? b % rg_cov : b / nb_cov;
-    const int64_t j = p.transpose ? b / rg_cov : b % nb_cov;
-    const int64_t ro = g * 16 + i16;
-    const bool has = live && ro < R && j < nb;
-    double v[16];
-    float vf[16];
-    double m = 0.0;
-    if (has) {
-      if (RHT) {
-        load_block(p, ro, j, v);
+    I.j = p.transpose ? b / rg_cov : b % nb_cov;
+    I.ro = g * 16 + i16;
+    I.has = I.live && I.ro < R && I.j < nb;
+    I.m = 0.0;
+    if (I.has) {
+      if constexpr (RHT) {
+        load_block(p, I.ro, I.j, I.v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
+        for (int e = 0; e < 16; ++e) I.m = fmax(I.m, fabs(I.v[e]));
       } else {
-        load_block_f32(p, ro, j, vf);
+        load_block_f32(p, I.ro, I.j, I.vf);
         float mf = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) mf = fmaxf(mf, fabsf(vf[e]));
-        m = static_cast<double>(mf);
+        for (int e = 0; e < 16; ++e) mf = fmaxf(mf, fabsf(I.vf[e]));
+        I.m = static_cast<double>(mf);
       }
     }
+  };
+  auto finish = [&](Item& I) {
+    double m = I.m;
     if (p.block2d) {   // one scale from the amax of the 16 x 16 block
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
     }
-    if (!live) continue;
+    if (!I.live) return;
+    const int64_t ro = I.ro, j = I.j;
     uint32_t scode = 0;
-    if (has) {
+    if (I.has) {
       uint32_t lo = 0, hi = 0;
       float q[16];
       bool nz;
-      if (RHT) {
+      if constexpr (RHT) {
         scode = cvt_to_e4m3(__double2float_rn(m / static_cast<double>(t)));
         const double dec = e4m3_exact(scode);
         nz = dec != 0.0;
         if (nz) {
           const float sc = __fmul_rn(static_cast<float>(dec), s_g);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(v[e] / static_cast<double>(sc));
+          for (int e = 0; e < 16; ++e) q[e] = __double2float_rn(I.v[e] / static_cast<double>(sc));
         }
       } else {
         scode = cvt_to_e4m3(__fdiv_rn(static_cast<float>(m), t));
@@ -351,7 +400,7 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
         if (nz) {
           const float sc = __fmul_rn(dec, s_g);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(vf[e], sc);
+          for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(I.vf[e], sc);
         }
       }
       if (nz) {
@@ -378,6 +427,12 @@ __global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0)
     } else if (ro < R && j < nb_store) {
       p.sf[ro * (ld / 16) + j] = static_cast<uint8_t>(scode);
     }
+  };
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items32; it += stride) {
+    Item I;
+    fetch(it, I);
+    finish(I);
   }
 }
 
@@ -514,12 +569,19 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
                                          uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
                                          uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
                                          int64_t ld, uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
-                                         double* partials, cudaStream_t s) {
+                                         double* partials, cudaStream_t s, const uint8_t* in_sf,
+                                         const float* in_global) {
   if (groups < 1 || groups > 65535 || !gtab || !global_out || rows_max < 0 || cols <= 0 || cols % 16)
+    return LMOE_ERR_INVALID_ARG;
+  // NVFP4 input: scales tiled over 64-column groups, read through the transform path
+  if (in_dtype == LMOE_NVFP4 && (!in_sf || !in_global || cols % 64 || !(flags & LMOE_QX_RHT)))
     return LMOE_ERR_INVALID_ARG;
   QxParams p = {};
   p.in = in;
   p.bf16 = in_dtype == LMOE_BF16;
+  p.fp4in = in_dtype == LMOE_NVFP4;
+  p.in_sf = in_sf;
+  p.in_global = in_global;
   p.rows = rows_max;
   p.cols = cols;
   p.transpose = (flags & LMOE_QX_TRANSPOSE) != 0;

@@ -16,12 +16,12 @@
 //   dh = dA * 2 max(h, 0)
 //   dz = SR(dh) W1q,          dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
 // with SR uniforms from Philox-4x32-10 on stream 4 e + 2 g + j (g: 0 first
-// GEMM, 1 second; j: 0 dgrad, 1 wgrad). Every step but the wgrads runs as one
-// launch over all experts: the quantiser with a group per expert (its own
-// global scale and SR stream), the grouped NVFP4 GEMM for the forward
-// recompute and both dgrads, and the three small kernels below with a grid
-// row per expert. The wgrads contract over each expert's own token count, so
-// the host issues one GEMM per expert and wgrad.
+// GEMM, 1 second; j: 0 dgrad, 1 wgrad). Every step runs as one launch over
+// all experts: the quantiser with a group per expert (its own global scale
+// and SR stream; it reads aq and zq as NVFP4 codes), the grouped NVFP4 GEMM
+// for the forward recompute and both dgrads, its K-batched form for the
+// wgrads (each expert contracts over its own token count), and the two small
+// kernels below with a grid row per expert.
 #include <cuda_bf16.h>
 
 #include <vector>
@@ -95,52 +95,6 @@ __global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const float* __restri
   }
 }
 
-// E2M1 magnitude by code (0, 0.5, 1, 1.5, 2, 3, 4, 6).
-__device__ __forceinline__ double e2m1_mag(uint32_t c) {
-  return (c < 4) ? 0.5 * static_cast<double>(c) : (c < 6 ? static_cast<double>(c - 2) : (c == 6 ? 4.0 : 6.0));
-}
-
-// E4M3 code -> value: subnormal f * 2^-9, normal (8 + f) * 2^(e - 10).
-__device__ __forceinline__ double e4m3_val(uint32_t c) {
-  const int e = (c >> 3) & 15, f = c & 7;
-  return e == 0 ? ldexp(static_cast<double>(f), -9) : ldexp(static_cast<double>(8 + f), e - 10);
-}
-
-// Rows p0 .. p0 + R - 1 of NVFP4 codes [*, cols/2] with MMA-tiled scales
-// (groups64 = cols / 64) and a global scale, as fp32 [*][cols] at the same
-// rows; rows >= p0 + n are zero. Each value is code * block scale * global,
-// formed exactly in fp64 (2 + 4 + 24 significant bits) and rounded once to fp32.
-__global__ void __launch_bounds__(kBwThreads) bw_dequant_kernel(const uint8_t* __restrict__ codes,
-                                                                 const uint8_t* __restrict__ sf,
-                                                                 const float* __restrict__ global,
-                                                                 const int64_t* __restrict__ etab, int cols,
-                                                                 float* __restrict__ out) {
-  pdl_begin();
-  const int64_t* t = etab + 4 * blockIdx.y;
-  const int64_t p0 = t[0], n = t[1], R = t[2];
-  const double s_g = static_cast<double>(__ldg(global));
-  const int groups64 = cols / 64;
-  const int64_t total = R * (cols / 2);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / (cols / 2);
-    const int cb = static_cast<int>(i % (cols / 2));   // byte: elements 2 cb, 2 cb + 1
-    const int64_t row = p0 + r;
-    float v0 = 0.0f, v1 = 0.0f;
-    if (r < n) {
-      const uint32_t b = codes[row * (cols / 2) + cb];
-      const int j = (2 * cb) / 16;
-      const int64_t so = ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
-      const double sc = e4m3_val(sf[so]) * s_g;
-      const uint32_t c0 = b & 15u, c1 = b >> 4;
-      v0 = __double2float_rn((c0 & 8u ? -1.0 : 1.0) * e2m1_mag(c0 & 7u) * sc);
-      v1 = __double2float_rn((c1 & 8u ? -1.0 : 1.0) * e2m1_mag(c1 & 7u) * sc);
-    }
-    out[row * cols + 2 * cb] = v0;
-    out[row * cols + 2 * cb + 1] = v1;
-  }
-}
-
 // Grid for a per-expert loop over `items` (x), one row per expert (y): about
 // eight resident CTAs per SM over all experts.
 dim3 grid_per_expert(int64_t items, int N) {
@@ -153,7 +107,7 @@ dim3 grid_per_expert(int64_t items, int N) {
 
 // Workspace carve-up (all offsets 256-byte aligned).
 struct BwLayout {
-  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w2tc, w2ts, h, aqc, aqs, o, d_o, dh, deq, qac,
+  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w2tc, w2ts, h, aqc, aqs, o, d_o, dh, qac,
       qas, qag, dA, t1c, t1s, t1g, t2c, t2s, t2g, part, etab, gtab, ktab, total;
   int64_t P, Rmax, Ksum;
 };
@@ -191,7 +145,6 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ks
   L.o = take(P * l * 4);
   L.d_o = take(P * l * 4);
   L.dh = take(P * m * 4);
-  L.deq = take(P * lm * 4);
   L.qac = take(P * lm / 2);
   L.qas = take(P * lm / 16);
   L.qag = take(N * 4);
@@ -212,7 +165,7 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ks
   if (np_t > np) np = np_t;
   L.part = take(static_cast<size_t>(np) * 8);
   L.etab = take(N * 4 * 8);       // per expert {p0, n, R, K offset}
-  L.gtab = take(6 * N * 5 * 8);   // six quantiser group tables
+  L.gtab = take(6 * N * 6 * 8);   // six quantiser group tables
   L.ktab = take(N * 2 * 4);       // wgrad K range per expert
   L.total = off;
   return L;
@@ -308,7 +261,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   // per expert {p0, n, R, K offset}; six quantiser group tables {first input
   // row, rows, codes offset, scales offset, pitch}: 0 SR(do), 1 RHT(do)^T,
   // 2 RHT(aq)^T, 3 SR(dh), 4 RHT(dh)^T, 5 RHT(zq)^T
-  std::vector<int64_t> etab(static_cast<size_t>(N) * 4), gtab(static_cast<size_t>(6) * N * 5);
+  std::vector<int64_t> etab(static_cast<size_t>(N) * 4), gtab(static_cast<size_t>(6) * N * 6);
   std::vector<int32_t> ktab(static_cast<size_t>(N) * 2);   // wgrad K range per expert: {first column, blocks}
   int64_t p0 = 0, koff = 0;
   for (int e = 0; e < N; ++e) {
@@ -318,20 +271,22 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
     etab[4 * e + 2] = R;
     etab[4 * e + 3] = koff;
     auto row_group = [&](int t, int64_t cols) {   // [R][cols] at the expert's padded rows
-      int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 5;
+      int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 6;
       g[0] = p0;
       g[1] = R;
       g[2] = p0 * cols / 2;
       g[3] = p0 * cols / 16;   // p0 is a multiple of 128: whole scale atoms
       g[4] = 0;
+      g[5] = n;
     };
     auto t_group = [&](int t) {   // columns [koff, koff + K256) of a [out_rows][Ksum] matrix
-      int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 5;
+      int64_t* g = gtab.data() + (static_cast<size_t>(t) * N + e) * 6;
       g[0] = p0;
       g[1] = R;
       g[2] = koff / 2;
       g[3] = koff / 64 * 512;   // koff is a multiple of 256: whole scale atoms
       g[4] = K256;
+      g[5] = n;
     };
     row_group(0, l);
     t_group(1);
@@ -351,7 +306,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
       cudaMemcpyAsync(d_gtab, gtab.data(), gtab.size() * 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(d_ktab, ktab.data(), ktab.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return LMOE_ERR_CUDA;
-  auto gt = [&](int t) { return d_gtab + static_cast<size_t>(t) * N * 5; };
+  auto gt = [&](int t) { return d_gtab + static_cast<size_t>(t) * N * 6; };
 
   // every expert's weights with 16 x 16 blocks (current amax per expert and
   // matrix), one grouped launch each: W1 [m][l] and W2 [l][m] for the forward,
@@ -427,7 +382,6 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
 
   float* d_o = at<float>(ws, L.d_o);
   float* dh = at<float>(ws, L.dh);
-  float* deq = at<float>(ws, L.deq);
   uint8_t *qac = at<uint8_t>(ws, L.qac), *qas = at<uint8_t>(ws, L.qas);
   float* qag = at<float>(ws, L.qag);
   uint8_t *t1c = at<uint8_t>(ws, L.t1c), *t1s = at<uint8_t>(ws, L.t1s);
@@ -438,12 +392,14 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   const float* o = at<float>(ws, L.o);
   const int64_t K256max = ceil_to(L.Rmax, 256);
   const uint32_t T_RHT = LMOE_QX_TRANSPOSE | LMOE_QX_RHT;
-  auto quant = [&](int t, const float* in, int64_t cols, uint32_t flags, uint32_t stream0, uint8_t* c, uint8_t* sf,
-                   float* g) {
+  // fp32 operands, or NVFP4 codes (in_sf, in_g: the wgrad inputs aq and zq,
+  // decoded exactly by the quantiser as it reads them)
+  auto quant = [&](int t, const void* in, int64_t cols, uint32_t flags, uint32_t stream0, uint8_t* c, uint8_t* sf,
+                   float* g, const uint8_t* in_sf = nullptr, const float* in_g = nullptr) {
     const bool tr = (flags & LMOE_QX_TRANSPOSE) != 0;
-    return launch_nvfp4_quantize_groups(in, LMOE_F32, L.Rmax, cols, flags, rht_signs, seed, stream0, 4, gt(t), N,
-                                        tr ? K256max : cols, tr ? L.Ksum : 0, c, sf, g, LMOE_SF_MMA_TILED, part,
-                                        s);
+    return launch_nvfp4_quantize_groups(in, in_sf ? LMOE_NVFP4 : LMOE_F32, L.Rmax, cols, flags, rht_signs, seed,
+                                        stream0, 4, gt(t), N, tr ? K256max : cols, tr ? L.Ksum : 0, c, sf, g,
+                                        LMOE_SF_MMA_TILED, part, s, in_sf, in_g);
   };
   // every expert's wgrad in one K-batched launch: dW[e] [rows][cols] =
   // A[:, K_e] . B[:, K_e]^T over the expert's K256 columns (experts without
@@ -488,12 +444,9 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
            static_cast<const int64_t*>(d_etab), static_cast<int>(m), dh);
   count_launch();
   // second GEMM, wgrad: dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T  (contraction over the expert's K256 tokens)
-  launch_k(bw_dequant_kernel, grid_per_expert(L.Rmax * m / 2, N), dim3(kBwThreads), 0, s,
-           static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqc)), static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqs)),
-           a_global, static_cast<const int64_t*>(d_etab), static_cast<int>(m), deq);
-  count_launch();
   if ((st = quant(1, d_o, l, T_RHT | LMOE_QX_SR, 3, t1c, t1s, t1g)) != LMOE_OK) return st;
-  if ((st = quant(2, deq, m, T_RHT, 0, t2c, t2s, t2g)) != LMOE_OK) return st;
+  if ((st = quant(2, at<uint8_t>(ws, L.aqc), m, T_RHT, 0, t2c, t2s, t2g, at<uint8_t>(ws, L.aqs), a_global)) != LMOE_OK)
+    return st;
   if ((st = wgrads(l, m, dw2)) != LMOE_OK) return st;
   // first GEMM, dgrad: dz = SR(dh) W1q  (W1^T [l][m] with 16 x 16 blocks), at the slot rows
   if ((st = quant(3, dh, m, LMOE_QX_SR, 0, qac, qas, qag)) != LMOE_OK) return st;
@@ -501,11 +454,8 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                     dz, l, 0)) != LMOE_OK)
     return st;
   // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
-  launch_k(bw_dequant_kernel, grid_per_expert(L.Rmax * l / 2, N), dim3(kBwThreads), 0, s, z_codes, z_sf, z_global,
-           static_cast<const int64_t*>(d_etab), static_cast<int>(l), deq);
-  count_launch();
   if ((st = quant(4, dh, m, T_RHT | LMOE_QX_SR, 1, t1c, t1s, t1g)) != LMOE_OK) return st;
-  if ((st = quant(5, deq, l, T_RHT, 0, t2c, t2s, t2g)) != LMOE_OK) return st;
+  if ((st = quant(5, z_codes, l, T_RHT, 0, t2c, t2s, t2g, z_sf, z_global)) != LMOE_OK) return st;
   if ((st = wgrads(m, l, dw1)) != LMOE_OK) return st;
   if (o_out && L.P > 0 &&
       cudaMemcpyAsync(o_out, o, static_cast<size_t>(L.P) * l * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
