@@ -828,16 +828,17 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
   float* gw = at<float>(ws, L.w);
   float* logits = at<float>(ws, L.logits);
 
-  // BF16 latent layer at prefill sizes: the permutation runs first, then the
-  // down-projection stores z once and a token-order copy reads each z row once
-  // and writes it to the padded rows of its K slots
-  const bool scatter_z = !ident && !fp4 && !f32 && T > kSwapMaxTokens && l >= 64;
+  // BF16 layer at prefill sizes: the permutation runs first, then (latent
+  // projections) the down-projection stores z once, and a token-order copy
+  // reads each z row (x with identity projections) once and writes it to the
+  // padded rows of its K slots
+  const bool scatter_z = !fp4 && !f32 && T > kSwapMaxTokens && l >= 64;
   // The top-K and the permutation need only the router logits, the
   // down-projection only x: when both follow, the routing runs on a side
   // stream beside the down-projection GEMM (whose persistent CTAs leave room
   // on every SM for the routing's small ones). Not while tracing stages.
   SideStream side;
-  const bool overlap = !events && (scatter_z || (fp4 && !ident)) && side_stream(&side);
+  const bool overlap = !events && !ident && (scatter_z || fp4) && side_stream(&side);
   cudaStream_t rs = overlap ? side.stream : s;
 
   // 1. router logits (+ bias) and top-K gates
@@ -881,9 +882,13 @@ lmoe_status lmoe_forward_traced(const lmoe_config* cfg, const lmoe_weights* w, c
     if ((st = launch_permute(idx, T, K, N, offsets, perm_src, inv_perm, poff, at<int32_t>(ws, L.scratch), gw, gate,
                              err, rs, kPermSlotsPerWarp, slot_row)) != LMOE_OK)
       return st;
-    void* zb = at<void>(ws, L.z);
-    if ((st = dense_bf16(x, T, w->w_down, l, d, zb, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s)) != LMOE_OK)
-      return st;
+    const void* zb = x;
+    if (!ident) {
+      void* z = at<void>(ws, L.z);
+      if ((st = dense_bf16(x, T, w->w_down, l, d, z, l, EPI_BF16, nullptr, nullptr, 0, splitk, err, s)) != LMOE_OK)
+        return st;
+      zb = z;
+    }
     if (!join_routing()) return LMOE_ERR_CUDA;
     mark(2);
     if ((st = launch_scatter_rows(zb, T, static_cast<int64_t>(l) * ab, slot_row, K, zp, s)) != LMOE_OK) return st;
