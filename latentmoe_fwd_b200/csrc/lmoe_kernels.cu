@@ -1035,8 +1035,9 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_encode_scatter_kernel(
         const int p = __shfl_sync(FULL, my_row, k);
         if (p < 0 || g >= groups64) continue;
         uint8_t* dst = codes + static_cast<int64_t>(p) * row_bytes + static_cast<int64_t>(g) * 32;
-        st_global_v4_hint(reinterpret_cast<uint4*>(dst), c01, pol);
-        st_global_v4_hint(reinterpret_cast<uint4*>(dst + 16), c23, pol);
+        // the lane's 32 code bytes as one 32-byte store: whole sectors, half the requests
+        const uint32_t u[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
+        st_global_v8_hint(dst, u, pol);
         *reinterpret_cast<uint32_t*>(sf + sf_tiled_offset(p, g * 4, groups64)) = sw;
       }
     }
@@ -1048,6 +1049,7 @@ lmoe_status launch_nvfp4_quantize_scatter(const void* in, int64_t rows, int cols
                                           int npartials, cudaStream_t s) {
   if (rows == 0) return LMOE_OK;
   if (cols % 64 || K < 1 || K > 32) return LMOE_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(codes) & 31) return LMOE_ERR_INVALID_ARG;   // 32-byte code stores
   launch_k(nvfp4_amax_kernel<__nv_bfloat16>, dim3(npartials), dim3(kQThreads), 0, s,
            static_cast<const __nv_bfloat16*>(in), rows * cols, partials);
   count_launch();
