@@ -454,7 +454,7 @@ def run_backward(args, wl):
                      "fp4_flops": fp4_flops, "bf16_flops": dense, "time_at_peak_ms": t_peak,
                      "frac": t_peak / ms_step, "peak_fp4_tflops": fp4_peak, "peak_bf16_tflops": peaks["bf16_tflops"],
                      "peak_source": src,
-                     "note": "the host walks the experts (about 20 launches each) and reads their row counts once"},
+                     "note": "grouped launches over all experts; the host reads their row counts once"},
         "gpu_launches": int(launches), "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
