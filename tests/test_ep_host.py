@@ -5,7 +5,8 @@ their l-dim rows to the experts' owners with all_to_all_single, run the owned
 experts on the expert-grouped rows, send the outputs back and combine. The
 sharded layer must equal the oracle's unsharded forward token for token
 (fp64, no rounding points), which checks ownership, the count exchange, the
-send/receive offsets and both reorders."""
+send/receive offsets and both reorders; the same rank processes check the
+peer-memory data plane's addressing (lmoe_ep_slot_bases) against it."""
 import os
 import sys
 
@@ -76,6 +77,31 @@ def _rank_main(rank, world, port, T_each, result):
     y_slot = np.zeros((T_each * K, l))
     y_slot[perm_src] = ys.numpy()
     c = np.einsum("tk,tkl->tl", gates, y_slot.reshape(T_each, K, l))
+
+    # the peer-memory data plane's addressing (lmoe_ep_slot_bases, as
+    # lmoe_ep_dispatch / lmoe_ep_combine apply it): slot f of expert e goes to
+    # rank owner[e], row base[e] + inv_perm[f] - offsets[e]. The stores are
+    # emulated by gathering (rank, row, data) at every rank; each owner's
+    # buffer must equal the all-to-all + reorder result, and reading the
+    # owners' outputs back at the same rows must give this rank's y rows.
+    owner, base = L.ep_slot_bases(world, rank, torch.stack(parts).numpy())
+    e_slot = idx.reshape(-1)
+    dst_rank = owner[e_slot]
+    dst_row = base[e_slot] + inv_perm - offsets[e_slot]
+    stores = [None] * world
+    dist.all_gather_object(stores, (dst_rank, dst_row, z[np.arange(T_each * K) // K]))
+    mine = np.zeros((P, l))
+    for dr, rr, data in stores:
+        sel = dr == rank
+        mine[rr[sel]] = data[sel]
+    real = np.concatenate([np.arange(plan["local_padded_offsets"][el],
+                                     plan["local_padded_offsets"][el] + plan["local_offsets"][el + 1]
+                                     - plan["local_offsets"][el]) for el in range(plan["local_experts"])])
+    assert np.array_equal(mine[real], grouped[real])
+    ys_all = [None] * world
+    dist.all_gather_object(ys_all, y)
+    y_read = np.stack([ys_all[h][r] for h, r in zip(dst_rank, dst_row)])
+    assert np.array_equal(y_read, y_slot)
     out = c @ wu.T
     ref = O.forward(wl, inp, tokens=tok, precision="f64")["out"]
     result[rank] = float(np.max(np.abs(out - ref)) / np.sqrt(np.mean(ref ** 2)))
