@@ -359,8 +359,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ---------------- epilogue (warps 2..5, both CTAs) ----------------
-    const int q = warp & 3;
-    const int r = q * 32 + lane;   // feature row of this thread within the CTA's 128
+    const int q = warp & 3;        // TMEM lane quarter: feature rows q * 32 .. q * 32 + 31 of the CTA's 128
     int local = 0;
     for (int t = cluster; t < ntiles; t += nclusters) {
       const Tile2 ti = tc2_tile(p, t, ntiles, nextra, prefix, ecount, epoff);

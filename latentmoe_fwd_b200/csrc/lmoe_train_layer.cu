@@ -138,7 +138,7 @@ struct LbLayout {
 
 LbLayout lb_layout(const lmoe_config* c) {
   LbLayout L = {};
-  const int64_t T = c->T, d = c->d, l = c->l, N = c->N, K = c->K, m = c->m;
+  const int64_t T = c->T, d = c->d, l = c->l, N = c->N, K = c->K;
   const int64_t Sms = static_cast<int64_t>(c->n_shared) * c->m_shared;
   const bool ident = (c->flags & LMOE_FLAG_IDENTITY_PROJ) != 0;
   L.P = lmoe_padded_rows(c);
