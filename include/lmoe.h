@@ -220,6 +220,8 @@ lmoe_status lmoe_route(const lmoe_config* cfg, const void* x, const void* w_rout
  *    of `rows`, re-laid to LMOE_SF_MMA_TILED at the padded rows; row_cols is
  *    2*row_bytes (the rows then hold packed E2M1 codes).
  *  topk_w / perm_gate (optional): the gate of each padded row ([padded] F32).
+ *  With T = 0 only offsets and padded_offsets are needed (written as zeros);
+ *  the other buffers may be NULL.
  *  Errors: the config checks above; LMOE_ERR_INVALID_ARG for a NULL index
  *  buffer, rows without permuted_rows (or scales, gates without their
  *  destination), row_bytes not a positive multiple of 16, unaligned rows,

@@ -442,7 +442,8 @@ lmoe_status lmoe_permute(const lmoe_config* cfg, const int32_t* topk_idx, int32_
                          const float* topk_w, float* perm_gate, void* ws, size_t ws_bytes, void* stream) {
   lmoe_status st = check_config(cfg);
   if (st != LMOE_OK) return st;
-  if (!topk_idx || !offsets || !perm_src || !inv_perm || !padded_offsets) return LMOE_ERR_INVALID_ARG;
+  if (!offsets || !padded_offsets) return LMOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!topk_idx || !perm_src || !inv_perm)) return LMOE_ERR_INVALID_ARG;   // T = 0: offsets only
   if ((rows == nullptr) != (permuted_rows == nullptr)) return LMOE_ERR_INVALID_ARG;
   if (rows && (row_bytes <= 0 || row_bytes % 16 || !aligned16(rows) || !aligned16(permuted_rows)))
     return LMOE_ERR_INVALID_ARG;

@@ -35,13 +35,16 @@ def test_ep_reorder_both_directions_bit_exact():
     assert torch.equal(back.cpu(), r)                   # the way back restores the received order
 
 
-def _ep_case(G=3, N=12, K=3, l=256, m=256, Ts=(100, 150, 80), seed=7):
+def _ep_case(G=3, N=12, K=3, l=256, m=256, Ts=(100, 150, 80), seed=7, unused=()):
     """Routing, latent rows and expert weights of a small layer whose tokens
-    are split over G emulated ranks (consecutive chunks)."""
+    are split over G emulated ranks (consecutive chunks); experts in `unused`
+    receive no token."""
     rng = np.random.default_rng(seed)
     T = sum(Ts)
     p = 1.0 / np.arange(1, N + 1) ** 1.1
-    p = p[rng.permutation(N)] / p.sum()                 # skewed expert loads
+    p = p[rng.permutation(N)]
+    p[list(unused)] = 0.0
+    p = p / p.sum()                                     # skewed expert loads
     idx = np.stack([rng.choice(N, K, replace=False, p=p) for _ in range(T)]).astype(np.int32)
     g = rng.random((T, K)).astype(np.float32) + 0.1
     g = (g / g.sum(axis=1, keepdims=True)).astype(np.float32)
@@ -128,8 +131,13 @@ def _expert_parallel(c, corrupt_base=False):
     return torch.cat(outs), L.read_device_error(err.view(torch.uint8))
 
 
-def test_ep_dispatch_and_combine_equal_the_one_gpu_layer():
-    c = _ep_case()
+@pytest.mark.parametrize("case", ["three_ranks", "one_rank", "empty_rank_unused_expert"])
+def test_ep_dispatch_and_combine_equal_the_one_gpu_layer(case):
+    # (tokens x K >= 64 x experts in every case, so the owners' expert GEMMs
+    # take the same CTA-pair kernel as the single-GPU reference)
+    c = {"three_ranks": lambda: _ep_case(),
+         "one_rank": lambda: _ep_case(G=1, Ts=(300,), seed=3),
+         "empty_rank_unused_expert": lambda: _ep_case(Ts=(150, 0, 120), seed=5, unused=(4,))}[case]()
     ref = _one_gpu(c)
     got, (st, info) = _expert_parallel(c)
     assert st == L.OK, (st, info)
