@@ -467,6 +467,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(LI.WORKLOADS))
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one forward captured in a CUDA graph (the e2e leg stays eager)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample", type=int, default=None, help="oracle tokens per call of cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -574,6 +576,21 @@ def main():
     if stv != L.OK:
         raise RuntimeError(f"device error during warm-up: {L.status_string(stv)} info={info:#x}")
 
+    # --graph: one forward captured in a CUDA graph, replayed once per step
+    graph, graph_launches = None, 0
+    if args.graph:
+        gs = torch.cuda.Stream()
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            L.forward(cfg, w, x, out, ws, gs)   # first use on the capture stream
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        n0 = L.kernel_launch_count()
+        with torch.cuda.graph(graph, stream=gs):
+            L.forward(cfg, w, x, out, ws, gs)
+        graph_launches = L.kernel_launch_count() - n0
+        torch.cuda.synchronize()
+
     # ---- device-resident timed region ----
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(L.TRACE_EVENTS)] for _ in range(K)]
@@ -585,10 +602,13 @@ def main():
     launches0 = L.kernel_launch_count()
     start.record(stream)
     for i in range(K):
-        L.forward(cfg, w, x, out, ws, stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            L.forward(cfg, w, x, out, ws, stream)
     end.record(stream)
     torch.cuda.synchronize()
-    launches = L.kernel_launch_count() - launches0
+    launches = L.kernel_launch_count() - launches0 + graph_launches * K
     clocks = sampler.stop()
     barrier()
     stv, info = L.read_device_error(ws)
@@ -685,6 +705,7 @@ def main():
                                                                                      x_host.element_size()),
                     "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())},
             "gpu_launches": int(launches),
+            "launch": "cuda_graph" if graph is not None else "stream",
             "clocks": clocks,
             "stage_ms": {n: float(v) for n, v in zip(L.TRACE_STAGES, stage_ms)},
         }
