@@ -598,7 +598,7 @@ lmoe_status lmoe_ep_slot_bases(int G, int rank, int N, const int32_t* counts, in
  *  lmoe_ep_slot_bases's arrays; peer_rows [G], peer_gates [G] (or NULL with
  *  topk_w NULL): DEVICE arrays of device pointers, rank h's buffers (another
  *  GPU's memory mapped into this process, or this GPU's own for h = rank),
- *  each holding peer_rows_cap rows. err_word (device, may be NULL): a row or
+ *  each 16-byte aligned and holding peer_rows_cap rows. err_word (device, may be NULL): a row or
  *  owner out of range is skipped and recorded there (LMOE_ERR_DEVICE_BOUNDS,
  *  info the slot) as in a workspace's error word. Asynchronous on `stream`.
  *  Errors: LMOE_ERR_INVALID_ARG for null pointers, K outside [1, 32], sizes,
@@ -613,7 +613,8 @@ lmoe_status lmoe_ep_dispatch(int64_t T, int K, int N, int G, const void* rows, i
  * of the owner's expert-output row (BF16 [*][l], gates applied by the owner's
  * lmoe_expert_ffn from the dispatched gates) at the slot's row, stored BF16
  * -- lmoe_combine's arithmetic with topk_w NULL. peer_y [G]: DEVICE array of
- * the ranks' y buffers (peer_rows_cap rows each); the other arguments as
+ * the ranks' y buffers (16-byte aligned, peer_rows_cap rows each); the
+ * other arguments as
  * lmoe_ep_dispatch; c [T][l] (16-byte aligned), l a multiple of 8.
  *  Errors: LMOE_ERR_INVALID_ARG for null pointers, K outside [1, 32], sizes,
  *  an unaligned c; LMOE_ERR_UNSUPPORTED for T >= 2^31. */

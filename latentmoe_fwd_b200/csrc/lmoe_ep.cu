@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(
       if (e >= 0 && e < N) {
         h = __ldg(owner + e);
         row = static_cast<int64_t>(__ldg(dst_base + e)) + __ldg(inv_perm + f) - __ldg(offsets + e);
-        if (h < 0 || h >= G || row < 0 || row >= rows_cap) {
+        // a rank, row or buffer (16-byte stores) out of range is skipped and reported
+        if (h < 0 || h >= G || row < 0 || row >= rows_cap || (reinterpret_cast<uintptr_t>(peer_rows[h]) & 15)) {
           dev_report(err, kErrBounds, static_cast<uint32_t>(f));
           h = -1;
         }
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(
       if (e >= 0 && e < N) {
         const int h = __ldg(owner + e);
         const int64_t row = static_cast<int64_t>(__ldg(dst_base + e)) + __ldg(inv_perm + f) - __ldg(offsets + e);
-        ok = h >= 0 && h < G && row >= 0 && row < rows_cap;
+        ok = h >= 0 && h < G && row >= 0 && row < rows_cap && !(reinterpret_cast<uintptr_t>(peer_y[h]) & 15);
         if (ok) p = peer_y[h] + row * l;
         else dev_report(err, kErrBounds, static_cast<uint32_t>(f));
       }
