@@ -55,15 +55,22 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const float* __rest
     const int64_t row = p0 + r;
     float* out = d_o + row * l;
     if (r >= n) {
-      for (int j = threadIdx.x; j < l; j += blockDim.x) out[j] = 0.0f;
+      for (int j = threadIdx.x; j < l / 4; j += blockDim.x) reinterpret_cast<float4*>(out)[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       continue;
     }
     const float g = __ldg(gate + row);
     float dot = 0.0f;
-    for (int j = threadIdx.x; j < l; j += blockDim.x) {
-      const float d = dy[row * l + j];
-      dot = fmaf(d, o[row * l + j], dot);
-      out[j] = __fmul_rn(g, d);
+    // 16-byte accesses (l is a multiple of 256)
+    const float4* dy4 = reinterpret_cast<const float4*>(dy + row * l);
+    const float4* o4 = reinterpret_cast<const float4*>(o + row * l);
+    float4* out4 = reinterpret_cast<float4*>(out);
+    for (int j = threadIdx.x; j < l / 4; j += blockDim.x) {
+      const float4 d = dy4[j], v = o4[j];
+      dot = fmaf(d.x, v.x, dot);
+      dot = fmaf(d.y, v.y, dot);
+      dot = fmaf(d.z, v.z, dot);
+      dot = fmaf(d.w, v.w, dot);
+      out4[j] = make_float4(__fmul_rn(g, d.x), __fmul_rn(g, d.y), __fmul_rn(g, d.z), __fmul_rn(g, d.w));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
@@ -86,12 +93,18 @@ __global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const float* __restri
   pdl_begin();
   const int64_t* t = etab + 4 * blockIdx.y;
   const int64_t p0 = t[0], n = t[1], R = t[2];
-  const int64_t total = R * m;
+  const int64_t total = R * m / 4;   // float4 groups (m is a multiple of 256)
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / m, c = i % m;
-    const int64_t at = (p0 + r) * m + c;
-    dh[at] = r < n ? dA[at] * (2.0f * fmaxf(h[at], 0.0f)) : 0.0f;
+    const int64_t r = (4 * i) / m;
+    const int64_t at = p0 * m / 4 + i;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < n) {
+      const float4 a = reinterpret_cast<const float4*>(dA)[at], hv = reinterpret_cast<const float4*>(h)[at];
+      v = make_float4(a.x * (2.0f * fmaxf(hv.x, 0.0f)), a.y * (2.0f * fmaxf(hv.y, 0.0f)),
+                      a.z * (2.0f * fmaxf(hv.z, 0.0f)), a.w * (2.0f * fmaxf(hv.w, 0.0f)));
+    }
+    reinterpret_cast<float4*>(dh)[at] = v;
   }
 }
 
