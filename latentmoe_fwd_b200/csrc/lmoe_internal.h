@@ -244,7 +244,8 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                                  const float* z_global, const void* w1, const void* w2, const float* a_global,
                                  const float* gate, const float* dy, uint64_t seed, uint32_t rht_signs, void* dz,
                                  float* dgate, void* dw1, void* dw2, void* ws, float* o_out, uint32_t* err_word,
-                                 cudaStream_t s);
+                                 cudaStream_t s, const float* dy_tok = nullptr, const int32_t* perm_src = nullptr,
+                                 int K = 0);
 // FP8 E4M3 codes of in / s with one FP32 scale per tensor (scale_in, or the
 // tensor's amax / 448 when scale_in is null; scale_out receives it).
 lmoe_status launch_fp8_quantize(const void* in, int in_dtype, int64_t rows, int64_t cols, const float* scale_in,

@@ -41,12 +41,18 @@ int64_t ceil_to(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 // rows R (n rounded up to 16), first wgrad K column}.
 
 // do[p0 + r][:] = gate * dy for r < n (fp32; rows n..R-1 zero); dgate[p0 + r]
-// = dy . o. A block per row.
+// = dy . o. A block per row. dy is the slot row's upstream gradient: row
+// p0 + r of `dy`, or with dy_tok the row of the slot's token (the slot at
+// sorted position offsets[e] + r, token perm_src[...] / K) of the token-major
+// dy_tok.
 __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const float* __restrict__ dy,
                                                               const float* __restrict__ o,
                                                               const float* __restrict__ gate,
                                                               const int64_t* __restrict__ etab, int l,
-                                                              float* __restrict__ d_o, float* __restrict__ dgate) {
+                                                              float* __restrict__ d_o, float* __restrict__ dgate,
+                                                              const float* __restrict__ dy_tok,
+                                                              const int32_t* __restrict__ perm_src,
+                                                              const int32_t* __restrict__ offsets, int K) {
   pdl_begin();
   __shared__ float red[kBwThreads / 32];
   const int64_t* t = etab + 4 * blockIdx.y;
@@ -61,7 +67,9 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep_kernel(const float* __rest
     const float g = __ldg(gate + row);
     float dot = 0.0f;
     // 16-byte accesses (l is a multiple of 256)
-    const float4* dy4 = reinterpret_cast<const float4*>(dy + row * l);
+    const float* dyr = dy_tok ? dy_tok + static_cast<int64_t>(__ldg(perm_src + __ldg(offsets + blockIdx.y) + r) / K) * l
+                              : dy + row * l;
+    const float4* dy4 = reinterpret_cast<const float4*>(dyr);
     const float4* o4 = reinterpret_cast<const float4*>(o + row * l);
     float4* out4 = reinterpret_cast<float4*>(out);
     for (int j = threadIdx.x; j < l / 4; j += blockDim.x) {
@@ -260,7 +268,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                                  const float* z_global, const void* w1, const void* w2, const float* a_global,
                                  const float* gate, const float* dy, uint64_t seed, uint32_t rht_signs, void* dz,
                                  float* dgate, void* dw1, void* dw2, void* ws, float* o_out, uint32_t* err_word,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, const float* dy_tok, const int32_t* perm_src, int K) {
   const int N = cfg->N;
   const int64_t l = cfg->l, m = cfg->m;
   const BwLayout L = bw_layout(cfg, counts);
@@ -445,7 +453,7 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   // do, dgate
   launch_k(bw_prep_kernel, grid_per_expert(L.Rmax * kBwThreads, N), dim3(kBwThreads), 0, s,
            static_cast<const float*>(dy), o, gate, static_cast<const int64_t*>(d_etab), static_cast<int>(l), d_o,
-           dgate);
+           dgate, dy_tok, perm_src, offsets, K);
   count_launch();
   // second GEMM, dgrad: dA = SR(do) W2q  (W2^T [m][l] with 16 x 16 blocks)
   if ((st = quant(0, d_o, l, LMOE_QX_SR, 2, qac, qas, qag)) != LMOE_OK) return st;

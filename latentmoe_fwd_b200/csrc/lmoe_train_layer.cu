@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kLbThreads) colsum_kernel(const float* __restr
 }
 
 struct LbLayout {
-  size_t err, logits, idx, gates, z, zq, zsf, zgs, qpart, offs, poff, psrc, iperm, scratch, pgate, zp, zpsf, dc, dy,
+  size_t err, logits, idx, gates, z, zq, zsf, zgs, qpart, offs, poff, psrc, iperm, scratch, pgate, zp, zpsf, dc,
       dzr, dgate, o, c, dzt, dl32, dl16, dlT, xT, doT, cT, dzT, wupT, wrT, wdnT, pre, hs, hsT, tmp, dpre, dpreT, ws2T,
       ws1T, ex, total;
   int64_t P, T64;
@@ -167,7 +167,6 @@ LbLayout lb_layout(const lmoe_config* c) {
   L.zp = take(L.P * l / 2);
   L.zpsf = take(L.P * l / 16);
   L.dc = take(T * l * 4);
-  L.dy = take(L.P * l * 4);
   L.dzr = take(L.P * l * 2);
   L.dgate = take(L.P * 4);
   L.o = take(L.P * l * 4);
@@ -310,11 +309,8 @@ lmoe_status lmoe_backward_nvfp4(const lmoe_config* cfg, const lmoe_weights* w, c
              T * l, dc);
     count_launch();
   }
-  // each slot row's upstream gradient: dc of its token, fp32, in the experts' padded layout
-  float* dy = at<float>(ws, L.dy);
-  if (!ok(launch_gather(idx, psrc, offs, poff, T * K, static_cast<int>(K), dc, l * 4, dy, nullptr, nullptr,
-                        static_cast<int>(N), s)))
-    return st;
+  // each slot row's upstream gradient is dc of its token (fp32): the experts'
+  // backward reads it through the permutation, no per-slot copy
 
   // ---- the routed experts (NVFP4 recipe); they need their row counts on the host ----
   std::vector<int32_t> off_h(N + 1);
@@ -328,8 +324,8 @@ lmoe_status lmoe_backward_nvfp4(const lmoe_config* cfg, const lmoe_weights* w, c
   float* dgate = at<float>(ws, L.dgate);
   __nv_bfloat16* dzr = at<__nv_bfloat16>(ws, L.dzr);
   if (!ok(expert_backward_core(cfg, counts.data(), offs, poff, at<uint8_t>(ws, L.zp), at<uint8_t>(ws, L.zpsf), zgs,
-                               w->w1, w->w2, a_global, pgate, dy, seed, rht_signs, dzr, dgate, g->dw1, g->dw2, ex, o,
-                               err, s)))
+                               w->w1, w->w2, a_global, pgate, nullptr, seed, rht_signs, dzr, dgate, g->dw1, g->dw2,
+                               ex, o, err, s, dc, psrc, static_cast<int>(K))))
     return st;
 
   // c = sum_k g_k o_k (fp32), dz_t = sum_k dz(t, k) (BF16)
