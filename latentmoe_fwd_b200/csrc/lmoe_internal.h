@@ -210,10 +210,8 @@ lmoe_status launch_nvfp4_transpose2d(const uint8_t* codes, const uint8_t* sf, in
 // Ragged groups: group g quantises input rows [gtab[6g], gtab[6g] + gtab[6g+1])
 // of a [*][cols] input as one matrix (own global scale global_out[g], SR
 // stream stream0 + g * stream_step), codes at codes + gtab[6g+2], scales at
-// sf + gtab[6g+3], output pitch gtab[6g+4] (0: the output's columns).
-// in_dtype LMOE_NVFP4 (with LMOE_QX_RHT): `in` holds E2M1 codes [*][cols/2],
-// in_sf their MMA-tiled scales, in_global their global scale; the group's
-// rows from gtab[6g+5] on read as zero.
+// sf + gtab[6g+3], output pitch gtab[6g+4] (0: the output's columns);
+// gtab[6g+5] (the rows holding data) is informational.
 // ld > 0 (a multiple of 64): every group writes into one matrix of ld-element
 // rows (codes at ld / 2 bytes per row, MMA-tiled atoms over ld / 64 column
 // groups), its offsets naming its first column. rows_max / pitch_max bound
@@ -223,8 +221,7 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
                                          uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
                                          uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
                                          int64_t ld, uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
-                                         double* partials, cudaStream_t s, const uint8_t* in_sf = nullptr,
-                                         const float* in_global = nullptr);
+                                         double* partials, cudaStream_t s);
 // Dense BF16 GEMM on the tensor cores (lmoe_api.cu): out[rows][cols] =
 // epi(x[rows][k] . w[cols][k]^T), token-major tiles, or weight-major ones for
 // rows <= 64 (split-K into `partial` when given). epi: EPI_* of gemm_tc.cuh

@@ -93,18 +93,9 @@ struct QxParams {
   int64_t gs_in, gs_codes, gs_sf;
   // ragged groups instead (gtab non-null): per group {first input row, input
   // rows, codes offset, scales offset (bytes), output pitch (0: out cols),
-  // rows holding data (the rest read as zero; NVFP4 input)}; group g draws
-  // its SR uniforms on stream + g * stream_step
+  // rows holding data}; group g draws its SR uniforms on stream + g * stream_step
   const int64_t* gtab;
   uint32_t stream_step;
-  // NVFP4 input: `in` holds E2M1 codes [*][cols/2] with MMA-tiled scales in_sf
-  // (over the absolute rows) and the global scale *in_global; an element is
-  // fp32(code * scale * global), formed exactly in fp64 and rounded once
-  int fp4in;
-  const uint8_t* in_sf;
-  const float* in_global;
-  float in_gs;
-  int64_t in_row0, real_rows;
   int vec;               // input 16-byte aligned: row segments read with 16-byte loads
   int64_t ld;            // elements per destination row (codes, and tiled scale atoms); 0: pitch
 };
@@ -116,12 +107,7 @@ __device__ __forceinline__ QxParams qx_group(const QxParams& p0) {
   const int64_t g = blockIdx.y;
   if (p0.gtab) {
     const int64_t* t = p0.gtab + g * 6;
-    if (p0.fp4in) {   // rows are addressed absolutely (the scales' tiling)
-      p.in_row0 = t[0];
-      p.real_rows = t[5];
-    } else {
-      p.in = static_cast<const uint8_t*>(p0.in) + t[0] * p0.cols * (p0.bf16 ? 2 : 4);
-    }
+    p.in = static_cast<const uint8_t*>(p0.in) + t[0] * p0.cols * (p0.bf16 ? 2 : 4);
     p.rows = t[1];
     p.codes += t[2];
     p.sf += t[3];
@@ -139,22 +125,7 @@ __device__ __forceinline__ QxParams qx_group(const QxParams& p0) {
   return p;
 }
 
-// E2M1 magnitude by code (0, 0.5, 1, 1.5, 2, 3, 4, 6), without a table.
-__device__ __forceinline__ double e2m1_mag_d(uint32_t c) {
-  return (c < 4) ? 0.5 * static_cast<double>(c) : (c < 6 ? static_cast<double>(c - 2) : (c == 6 ? 4.0 : 6.0));
-}
-
 __device__ __forceinline__ double load_in(const QxParams& p, int64_t r, int64_t c) {
-  if (p.fp4in) {
-    if (r >= p.real_rows) return 0.0;
-    const int64_t row = p.in_row0 + r;
-    const uint32_t byte = static_cast<const uint8_t*>(p.in)[row * (p.cols / 2) + (c >> 1)];
-    const uint32_t code = (c & 1) ? byte >> 4 : byte & 15u;
-    const int64_t j = c >> 4, g64 = p.cols / 64;
-    const uint32_t s = p.in_sf[((row >> 7) * g64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3)];
-    const double sc = e4m3_exact(s) * static_cast<double>(p.in_gs);
-    return static_cast<double>(__double2float_rn((code & 8u ? -1.0 : 1.0) * e2m1_mag_d(code & 7u) * sc));
-  }
   if (p.bf16) return static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(p.in)[r * p.cols + c]));
   return static_cast<double>(static_cast<const float*>(p.in)[r * p.cols + c]);
 }
@@ -233,8 +204,7 @@ __device__ __forceinline__ int64_t out_cols(const QxParams& p) { return p.transp
 // Pass 1: per-CTA maxima of |out| (fp64, exact).
 __global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, double* __restrict__ partials) {
   pdl_begin();
-  QxParams p = qx_group(p0);
-  if (p.fp4in) p.in_gs = __ldg(p.in_global);
+  const QxParams p = qx_group(p0);
   partials += static_cast<int64_t>(blockIdx.y) * gridDim.x;
   __shared__ double red[kXThreads / 32];
   const int64_t nb = out_cols(p) / 16, total = out_rows(p) * nb;
@@ -300,11 +270,12 @@ __device__ __forceinline__ int64_t tiled_off(int64_t row, int64_t j, int64_t gro
 // 16-row group sit in one half-warp (lane & 15 = row in the group), so a
 // 16 x 16 block's amax is a half-warp reduction. The item count is rounded up
 // to whole warps; items past the end take part in the reductions only.
+// Latency-bound: occupancy matters more than registers (bounded to 4 CTAs per
+// SM, 3 for the transform path, at no or negligible spilling).
 template <bool RHT>
-__global__ void __launch_bounds__(kXThreads) qx_encode_kernel(const QxParams p0) {
+__global__ void __launch_bounds__(kXThreads, RHT ? 3 : 4) qx_encode_kernel(const QxParams p0) {
   pdl_begin();
-  QxParams p = qx_group(p0);
-  if (p.fp4in) p.in_gs = __ldg(p.in_global);
+  const QxParams p = qx_group(p0);
   __shared__ double red[kXThreads / 32];
   __shared__ float s_gs;
   // global scale: s_g = fp32(amax / 2688) from the fp64 amax (1 when 0)
@@ -569,19 +540,12 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
                                          uint32_t flags, uint32_t rht_signs, uint64_t seed, uint32_t stream0,
                                          uint32_t stream_step, const int64_t* gtab, int groups, int64_t pitch_max,
                                          int64_t ld, uint8_t* codes, uint8_t* sf, float* global_out, int sf_layout,
-                                         double* partials, cudaStream_t s, const uint8_t* in_sf,
-                                         const float* in_global) {
+                                         double* partials, cudaStream_t s) {
   if (groups < 1 || groups > 65535 || !gtab || !global_out || rows_max < 0 || cols <= 0 || cols % 16)
-    return LMOE_ERR_INVALID_ARG;
-  // NVFP4 input: scales tiled over 64-column groups, read through the transform path
-  if (in_dtype == LMOE_NVFP4 && (!in_sf || !in_global || cols % 64 || !(flags & LMOE_QX_RHT)))
     return LMOE_ERR_INVALID_ARG;
   QxParams p = {};
   p.in = in;
   p.bf16 = in_dtype == LMOE_BF16;
-  p.fp4in = in_dtype == LMOE_NVFP4;
-  p.in_sf = in_sf;
-  p.in_global = in_global;
   p.rows = rows_max;
   p.cols = cols;
   p.transpose = (flags & LMOE_QX_TRANSPOSE) != 0;

@@ -18,10 +18,10 @@
 // with SR uniforms from Philox-4x32-10 on stream 4 e + 2 g + j (g: 0 first
 // GEMM, 1 second; j: 0 dgrad, 1 wgrad). Every step runs as one launch over
 // all experts: the quantiser with a group per expert (its own global scale
-// and SR stream; it reads aq and zq as NVFP4 codes), the grouped NVFP4 GEMM
-// for the forward recompute and both dgrads, its K-batched form for the
-// wgrads (each expert contracts over its own token count), and the two small
-// kernels below with a grid row per expert.
+// and SR stream), the grouped NVFP4 GEMM for the forward recompute and both
+// dgrads, its K-batched form for the wgrads (each expert contracts over its
+// own token count), and the three small kernels below with a grid row per
+// expert.
 #include <cuda_bf16.h>
 
 #include <vector>
@@ -116,6 +116,52 @@ __global__ void __launch_bounds__(kBwThreads) bw_dh_kernel(const float* __restri
   }
 }
 
+// Rows p0 .. p0 + R - 1 of NVFP4 codes [*, cols/2] with MMA-tiled scales
+// (groups64 = cols / 64) and a global scale, as fp32 [*][cols] at the same
+// rows; rows >= p0 + n are zero. A thread per 16-element block. Each value is
+// code * block scale * global rounded once to fp32: code * block scale has at
+// most 6 significant bits, so it is exact in fp32 and one fp32 multiplication
+// by the global scale rounds the exact product.
+__global__ void __launch_bounds__(kBwThreads) bw_dequant_kernel(const uint8_t* __restrict__ codes,
+                                                                 const uint8_t* __restrict__ sf,
+                                                                 const float* __restrict__ global,
+                                                                 const int64_t* __restrict__ etab, int cols,
+                                                                 float* __restrict__ out) {
+  pdl_begin();
+  const int64_t* t = etab + 4 * blockIdx.y;
+  const int64_t p0 = t[0], n = t[1], R = t[2];
+  const float s_g = __ldg(global);
+  const int nb = cols / 16, groups64 = cols / 64;
+  const int64_t total = R * nb;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / nb;
+    const int j = static_cast<int>(i % nb);
+    const int64_t row = p0 + r;
+    float4* dst = reinterpret_cast<float4*>(out + row * cols + j * 16);
+    if (r >= n) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    const uint2 b = __ldg(reinterpret_cast<const uint2*>(codes + row * (cols / 2) + j * 8));
+    const int64_t so = ((row >> 7) * groups64 + (j >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + (j & 3);
+    const uint32_t sc = __ldg(sf + so);
+    const int e = (sc >> 3) & 15, f = sc & 7;
+    const float dec = static_cast<float>(e == 0 ? f : 8 + f) * __int_as_float(((e == 0 ? -9 : e - 10) + 127) << 23);
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t c = ((k < 8 ? b.x : b.y) >> (4 * (k & 7))) & 15u;
+      const uint32_t m = c & 7u;   // E2M1 magnitude 0, 0.5, 1, 1.5, 2, 3, 4, 6
+      const float mag = m < 4 ? 0.5f * static_cast<float>(m) : (m < 6 ? static_cast<float>(m - 2) : (m == 6 ? 4.0f : 6.0f));
+      v[k] = __fmul_rn((c & 8u) ? -(mag * dec) : mag * dec, s_g);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+}
+
 // Grid for a per-expert loop over `items` (x), one row per expert (y): about
 // eight resident CTAs per SM over all experts.
 dim3 grid_per_expert(int64_t items, int N) {
@@ -128,7 +174,7 @@ dim3 grid_per_expert(int64_t items, int N) {
 
 // Workspace carve-up (all offsets 256-byte aligned).
 struct BwLayout {
-  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w2tc, w2ts, h, aqc, aqs, o, d_o, dh, qac,
+  size_t err, w1c, w1s, w1g, w2c, w2s, w2g, w1tc, w1ts, w2tc, w2ts, h, aqc, aqs, o, d_o, dh, deq, qac,
       qas, qag, dA, t1c, t1s, t1g, t2c, t2s, t2g, part, etab, gtab, ktab, total;
   int64_t P, Rmax, Ksum;
 };
@@ -166,6 +212,7 @@ BwLayout bw_layout_for(const lmoe_config* c, int64_t P, int64_t Rmax, int64_t Ks
   L.o = take(P * l * 4);
   L.d_o = take(P * l * 4);
   L.dh = take(P * m * 4);
+  L.deq = take(P * lm * 4);   // dequantised wgrad inputs aq, zq
   L.qac = take(P * lm / 2);
   L.qas = take(P * lm / 16);
   L.qag = take(N * 4);
@@ -413,15 +460,13 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
   const float* o = at<float>(ws, L.o);
   const int64_t K256max = ceil_to(L.Rmax, 256);
   const uint32_t T_RHT = LMOE_QX_TRANSPOSE | LMOE_QX_RHT;
-  // fp32 operands, or NVFP4 codes (in_sf, in_g: the wgrad inputs aq and zq,
-  // decoded exactly by the quantiser as it reads them)
-  auto quant = [&](int t, const void* in, int64_t cols, uint32_t flags, uint32_t stream0, uint8_t* c, uint8_t* sf,
-                   float* g, const uint8_t* in_sf = nullptr, const float* in_g = nullptr) {
+  auto quant = [&](int t, const float* in, int64_t cols, uint32_t flags, uint32_t stream0, uint8_t* c, uint8_t* sf,
+                   float* g) {
     const bool tr = (flags & LMOE_QX_TRANSPOSE) != 0;
-    return launch_nvfp4_quantize_groups(in, in_sf ? LMOE_NVFP4 : LMOE_F32, L.Rmax, cols, flags, rht_signs, seed,
-                                        stream0, 4, gt(t), N, tr ? K256max : cols, tr ? L.Ksum : 0, c, sf, g,
-                                        LMOE_SF_MMA_TILED, part, s, in_sf, in_g);
+    return launch_nvfp4_quantize_groups(in, LMOE_F32, L.Rmax, cols, flags, rht_signs, seed, stream0, 4, gt(t), N,
+                                        tr ? K256max : cols, tr ? L.Ksum : 0, c, sf, g, LMOE_SF_MMA_TILED, part, s);
   };
+  float* deq = at<float>(ws, L.deq);
   // every expert's wgrad in one K-batched launch: dW[e] [rows][cols] =
   // A[:, K_e] . B[:, K_e]^T over the expert's K256 columns (experts without
   // rows get a zero gradient)
@@ -465,9 +510,12 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
            static_cast<const int64_t*>(d_etab), static_cast<int>(m), dh);
   count_launch();
   // second GEMM, wgrad: dW2 = SR(RHT(do)^T) RN(RHT(aq)^T)^T  (contraction over the expert's K256 tokens)
+  launch_k(bw_dequant_kernel, grid_per_expert(L.Rmax * m / 16, N), dim3(kBwThreads), 0, s,
+           static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqc)), static_cast<const uint8_t*>(at<uint8_t>(ws, L.aqs)),
+           a_global, static_cast<const int64_t*>(d_etab), static_cast<int>(m), deq);
+  count_launch();
   if ((st = quant(1, d_o, l, T_RHT | LMOE_QX_SR, 3, t1c, t1s, t1g)) != LMOE_OK) return st;
-  if ((st = quant(2, at<uint8_t>(ws, L.aqc), m, T_RHT, 0, t2c, t2s, t2g, at<uint8_t>(ws, L.aqs), a_global)) != LMOE_OK)
-    return st;
+  if ((st = quant(2, deq, m, T_RHT, 0, t2c, t2s, t2g)) != LMOE_OK) return st;
   if ((st = wgrads(l, m, dw2)) != LMOE_OK) return st;
   // first GEMM, dgrad: dz = SR(dh) W1q  (W1^T [l][m] with 16 x 16 blocks), at the slot rows
   if ((st = quant(3, dh, m, LMOE_QX_SR, 0, qac, qas, qag)) != LMOE_OK) return st;
@@ -475,8 +523,11 @@ lmoe_status expert_backward_core(const lmoe_config* cfg, const int32_t* counts, 
                     dz, l, 0)) != LMOE_OK)
     return st;
   // first GEMM, wgrad: dW1 = SR(RHT(dh)^T) RN(RHT(zq)^T)^T
+  launch_k(bw_dequant_kernel, grid_per_expert(L.Rmax * l / 16, N), dim3(kBwThreads), 0, s, z_codes, z_sf, z_global,
+           static_cast<const int64_t*>(d_etab), static_cast<int>(l), deq);
+  count_launch();
   if ((st = quant(4, dh, m, T_RHT | LMOE_QX_SR, 1, t1c, t1s, t1g)) != LMOE_OK) return st;
-  if ((st = quant(5, z_codes, l, T_RHT, 0, t2c, t2s, t2g, z_sf, z_global)) != LMOE_OK) return st;
+  if ((st = quant(5, deq, l, T_RHT, 0, t2c, t2s, t2g)) != LMOE_OK) return st;
   if ((st = wgrads(m, l, dw1)) != LMOE_OK) return st;
   if (o_out && L.P > 0 &&
       cudaMemcpyAsync(o_out, o, static_cast<size_t>(L.P) * l * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
