@@ -202,7 +202,9 @@ __device__ __forceinline__ int64_t out_rows(const QxParams& p) { return p.transp
 __device__ __forceinline__ int64_t out_cols(const QxParams& p) { return p.transpose ? p.rows : p.cols; }
 
 // Pass 1: per-CTA maxima of |out| (fp64, exact).
-__global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, double* __restrict__ partials) {
+template <bool RHT>
+__global__ void __launch_bounds__(kXThreads, RHT ? 4 : 6) qx_amax_kernel(const QxParams p0,
+                                                                       double* __restrict__ partials) {
   pdl_begin();
   const QxParams p = qx_group(p0);
   partials += static_cast<int64_t>(blockIdx.y) * gridDim.x;
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kXThreads) qx_amax_kernel(const QxParams p0, d
     // (consecutive input columns) of one block column, so loads coalesce
     const int64_t ro = p.transpose ? b % out_rows(p) : b / nb;
     const int64_t j = p.transpose ? b / out_rows(p) : b % nb;
-    if (p.rht) {
+    if constexpr (RHT) {
       double v[16];
       load_block(p, ro, j, v);
 #pragma unroll
@@ -519,7 +521,7 @@ lmoe_status launch_nvfp4_quantize_ex(const void* in, int in_dtype, int64_t rows,
   const int sms = device_sm_count();
   const int np = nvfp4x_partials(R * (C / 16));
   if (!global_in) {
-    launch_k(qx_amax_kernel, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);
+    launch_k(p.rht ? qx_amax_kernel<true> : qx_amax_kernel<false>, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);
     count_launch();
   }
   p.partials = partials;
@@ -568,7 +570,7 @@ lmoe_status launch_nvfp4_quantize_groups(const void* in, int in_dtype, int64_t r
   p.ld = ld;
   const int sms = device_sm_count();
   const int np = nvfp4x_partials(R * (pitch / 16) > 0 ? R * (pitch / 16) : 1);
-  launch_k(qx_amax_kernel, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);
+  launch_k(p.rht ? qx_amax_kernel<true> : qx_amax_kernel<false>, dim3(np, groups), dim3(kXThreads), 0, s, p, partials);
   count_launch();
   p.partials = partials;
   p.np = np;
