@@ -13,6 +13,12 @@
 // order, each sorted by expert; the expert GEMMs want every local expert's
 // rows together (source rank ascending inside an expert) at padded offsets
 // (multiples of 128), so each (source, expert) block moves as a whole.
+// Peer-memory data plane: instead of an all-to-all and a reorder, each rank's
+// dispatch kernel stores its rows straight at their final rows in the owners'
+// buffers (the owner's padded row of this rank's first row for the expert,
+// plus the slot's rank within the expert here), and its combine kernel reads
+// the owners' expert outputs back from the same rows. Plain loads and stores
+// through the peers' pointers: no TMA and no multicast touch another GPU.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
