@@ -42,8 +42,8 @@ static bool make_map_fp4(CUtensorMap* map, const void* ptr, int64_t k, int64_t r
 }
 
 template <int EPI, bool BATCH = false>
-static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const Fp4Params& p, int grid,
-                              cudaStream_t s) {
+static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a32, const Fp4Params& p,
+                              int grid, cudaStream_t s) {
   auto kern = fp4_gemm_kernel<EPI, BATCH>;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -53,7 +53,7 @@ static lmoe_status launch_fp4(const CUtensorMap& a, const CUtensorMap& b, const 
       return LMOE_ERR_CUDA;
     mark_configured(configured, dev);
   }
-  launch_k(kern, dim3(grid), dim3(Fp4Smem::kThreads), Fp4Smem::kBytes, s, a, b, p);
+  launch_k(kern, dim3(grid), dim3(Fp4Smem::kThreads), Fp4Smem::kBytes, s, a, b, a32, p);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
@@ -63,7 +63,9 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   const bool batch = L.kgroups != nullptr;
   if (batch && (L.quant_out || L.f32_out || L.row_scale || L.a_rows % 128 || L.groups < 1)) return LMOE_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
+  CUtensorMap ma32;   // 32-row boxes for tiles with at most 32 real rows
   if (!make_map_fp4(&ma, L.a_codes, L.k, L.a_rows, 1, 128)) return LMOE_ERR_INVALID_ARG;
+  if (!make_map_fp4(&ma32, L.a_codes, L.k, L.a_rows, 1, 32)) return LMOE_ERR_INVALID_ARG;
   if (!make_map_fp4(&mb, L.b_codes, L.k, L.cols, batch ? 1 : L.groups, 256)) return LMOE_ERR_INVALID_ARG;
   Fp4Params p;
   p.rows = static_cast<int>(L.a_rows);
@@ -95,10 +97,10 @@ lmoe_status fp4_gemm(const Fp4Launch& L, uint32_t* err_word, cudaStream_t stream
   if (tiles > 0x7fffffff) return LMOE_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   if (grid <= 0) return LMOE_OK;
-  if (batch) return launch_fp4<FP4_EPI_GATE_BF16, true>(ma, mb, p, grid, stream);
-  if (L.quant_out) return launch_fp4<FP4_EPI_SQRELU_QUANT>(ma, mb, p, grid, stream);
-  if (L.f32_out) return launch_fp4<FP4_EPI_F32>(ma, mb, p, grid, stream);
-  return launch_fp4<FP4_EPI_GATE_BF16>(ma, mb, p, grid, stream);
+  if (batch) return launch_fp4<FP4_EPI_GATE_BF16, true>(ma, mb, ma32, p, grid, stream);
+  if (L.quant_out) return launch_fp4<FP4_EPI_SQRELU_QUANT>(ma, mb, ma32, p, grid, stream);
+  if (L.f32_out) return launch_fp4<FP4_EPI_F32>(ma, mb, ma32, p, grid, stream);
+  return launch_fp4<FP4_EPI_GATE_BF16>(ma, mb, ma32, p, grid, stream);
 }
 
 }  // namespace lmoe

@@ -156,7 +156,7 @@ __device__ __forceinline__ long long fp4_sf_offset(long long row, int j, int gro
 template <int EPI, bool BATCH = false>
 __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Fp4Params p) {
+                    const __grid_constant__ CUtensorMap tmA32, const Fp4Params p) {
   pdl_begin();
   using S = Fp4Smem;
   extern __shared__ uint8_t smem_raw[];
@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmA32);
     tma_prefetch_desc(&tmB);
   }
   int* s_pstart = reinterpret_cast<int*>(smem + S::kRowsOffset);   // [groups + 1] padded starts
@@ -271,8 +272,12 @@ __global__ void __launch_bounds__(Fp4Smem::kThreads, 1)
           uint8_t* sb = sa + S::kA;
           uint8_t* ssfa = sb + S::kB;
           uint8_t* ssfb = ssfa + S::kSFA;
-          mbar_arrive_expect_tx(&full[stage], S::kStage);
-          tma_load_3d(sa, &tmA, &full[stage], koff / 2 + kb * 128, act0, 0, pol_a);
+          // a tile of at most 32 real rows (decode) loads only those 32 rows of
+          // A: the MMA's other rows read stale codes, but an output row reads
+          // only its own A row and the epilogue stores real rows only
+          const bool thin = act_n <= 32;
+          mbar_arrive_expect_tx(&full[stage], thin ? S::kStage - S::kA + 32 * 128 : S::kStage);
+          tma_load_3d(sa, thin ? &tmA32 : &tmA, &full[stage], koff / 2 + kb * 128, act0, 0, pol_a);
           tma_load_3d(sb, &tmB, &full[stage], koff / 2 + kb * 128, w0, BATCH ? 0 : e, pol_w);
           bulk_load(ssfa, sfa_blk + kb * 4 * 512, S::kSFA, &full[stage]);
 #pragma unroll
