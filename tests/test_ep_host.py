@@ -186,3 +186,14 @@ def test_slot_bases_follow_the_ownership_and_padded_layout(G, N):
             f0, nl = plan["first_expert"], plan["local_experts"]
             for el in range(nl):
                 assert base[f0 + el] == plan["block_dst"][r * nl + el]
+
+
+def test_slot_bases_reject_bad_arguments():
+    sys.path.insert(0, ROOT)
+    import latentmoe_fwd_b200 as L
+    with pytest.raises(L.LmoeError):
+        L.ep_slot_bases(3, 0, np.zeros((3, 2), dtype=np.int32))          # more ranks than experts
+    with pytest.raises(L.LmoeError):
+        L.ep_slot_bases(2, 0, -np.ones((2, 4), dtype=np.int32))          # negative counts
+    with pytest.raises(L.LmoeError):
+        L.ep_slot_bases(2, 2, np.zeros((2, 4), dtype=np.int32))          # rank out of range
