@@ -203,3 +203,23 @@ def test_fp8_quantize_host_errors():
     with pytest.raises(L.LmoeError) as e:
         L.fp8_quantize(dummy, L.BF16, 4, 32, None, dummy, None, stream=0)   # amax scale needs a workspace
     assert e.value.status == L.ERR_WORKSPACE
+
+
+def test_transpose_and_ep_kernels_host_errors():
+    # argument checks that return before any device work
+    assert L.lib.lmoe_nvfp4_transpose_2d(16, 16, 1, 128, 128, None, 16, None) == L.ERR_INVALID_ARG
+    assert L.lib.lmoe_nvfp4_transpose_2d(16, 16, 1, 100, 128, 16, 16, None) == L.ERR_UNSUPPORTED   # rows % 128
+    assert L.lib.lmoe_nvfp4_transpose_2d(16, 16, 1, 128, 128, 24, 16, None) == L.ERR_INVALID_ARG   # unaligned
+    assert L.lib.lmoe_nvfp4_transpose_2d(None, None, 0, 128, 128, None, None, None) == L.OK        # nothing to do
+    assert L.lib.lmoe_ep_dispatch(4, 0, 8, 2, 16, 32, 16, 16, 16, 16, 16, 16, 64, None, None, None,
+                                  None) == L.ERR_INVALID_ARG                                        # K = 0
+    assert L.lib.lmoe_ep_dispatch(4, 2, 8, 2, 16, 24, 16, 16, 16, 16, 16, 16, 64, None, None, None,
+                                  None) == L.ERR_INVALID_ARG                                        # row bytes % 16
+    assert L.lib.lmoe_ep_dispatch(4, 2, 8, 2, 16, 32, 16, 16, 16, 16, 16, 16, 64, 16, None, None,
+                                  None) == L.ERR_INVALID_ARG                                        # gates, no buffers
+    assert L.lib.lmoe_ep_dispatch(0, 2, 8, 2, None, 0, None, None, None, None, None, None, 0, None, None, None,
+                                  None) == L.OK                                                     # no tokens
+    assert L.lib.lmoe_ep_combine(4, 2, 8, 2, 36, 16, 64, 16, 16, 16, 16, 16, 16, None,
+                                 None) == L.ERR_INVALID_ARG                                         # l % 8
+    assert L.lib.lmoe_ep_combine(4, 2, 8, 2, 64, 16, 64, 16, 16, 16, 16, 16, 24, None,
+                                 None) == L.ERR_INVALID_ARG                                         # unaligned c
