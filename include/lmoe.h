@@ -307,7 +307,13 @@ lmoe_status lmoe_combine(const lmoe_config* cfg, const void* y_perm, const int32
  * missing without it, missing shared-expert weights, missing NVFP4 scales,
  * NULL or unaligned x / out (not checked when T == 0, which launches
  * nothing), or a weight a TMA descriptor cannot address (not 16-byte
- * aligned); LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT. */
+ * aligned); LMOE_ERR_WORKSPACE; on the device, LMOE_ERR_DEVICE_TIMEOUT.
+ * Ordering: every launch is ordered after earlier work on `stream`, and
+ * later work on `stream` sees the result. With latent projections (BF16
+ * with T > 64, or NVFP4) the top-K and permutation run beside the
+ * down-projection on a library-owned stream of the same device, forked from
+ * and joined back to `stream` with events; the call can be captured in a
+ * CUDA graph. */
 lmoe_status lmoe_forward(const lmoe_config* cfg, const lmoe_weights* w, const void* x,
                          void* out, void* ws, size_t ws_bytes, void* stream);
 
