@@ -132,11 +132,15 @@ def status_string(s: int) -> str:
 
 
 def _p(t):
-    """Device (or host) pointer of a tensor, or None."""
+    """Device pointer of a tensor (or a raw address given as an int), or None.
+    A torch tensor in host memory is rejected here: its address would reach a
+    kernel as a device pointer."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if getattr(t, "is_cuda", True) is False:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
     return t.data_ptr()
 
 
@@ -316,7 +320,7 @@ def expert_backward_nvfp4(cfg: Config, counts, offsets, padded_offsets, z_codes,
 
 def grads(**kw) -> Grads:
     """lmoe_grads from device tensors (missing ones NULL)."""
-    return Grads(**{k: (None if v is None else v.data_ptr()) for k, v in kw.items()})
+    return Grads(**{k: _p(v) for k, v in kw.items()})
 
 
 def backward_nvfp4(cfg: Config, w: Weights, x, dout, a_global, seed, rht_signs, g: Grads, ws=None, stream=None):

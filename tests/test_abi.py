@@ -223,3 +223,17 @@ def test_transpose_and_ep_kernels_host_errors():
                                  None) == L.ERR_INVALID_ARG                                         # l % 8
     assert L.lib.lmoe_ep_combine(4, 2, 8, 2, 64, 16, 64, 16, 16, 16, 16, 16, 24, None,
                                  None) == L.ERR_INVALID_ARG                                         # unaligned c
+
+
+def test_binding_rejects_host_tensors():
+    # a torch tensor in host memory never reaches the library as a pointer
+    import torch
+    cfg = L.config(T=4, d=64, l=32, N=8, K=2, m=64)
+    x = torch.zeros((4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        L.forward(cfg, L.weights(w_router=16, w1=16, w2=16, w_down=16, w_up=16), x, 16, x, stream=0)
+    with pytest.raises(ValueError):
+        L.weights(w_router=x)
+    with pytest.raises(ValueError):
+        L.grads(dx=x)
+    assert L._p(None) is None and L._p(4096) == 4096
